@@ -1,0 +1,426 @@
+#!/usr/bin/env python
+"""Benchmark of the routed-expert MoE layer on B200: one step = one whole layer (gate, route,
+group, expert FFN, combine) over one batch of synthetic tokens.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--tokens T]
+    python bench.py --impl reference ...     # the CPU oracle, timed on the host cores
+
+Prints one JSON line (rank 0).  Timing: CUDA events on the launching stream, barrier +
+synchronize on both sides of exactly K steps, max over ranks.  L2: every step reads a layer
+other than the previous step's (rotation over resident layers whose weights total far more
+than L2) and fresh activations, so no weight byte is served from L2 by a previous step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+PROFILES = os.path.join(ROOT, "profiles")
+METRIC = "MoE-layer tokens/s and expert-weight HBM GB/s (fraction of roofline), 1 B200"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="coli", choices=["coli", "reference"])
+    ap.add_argument("--workload", default="glm_decode", choices=list(synth.WORKLOADS))
+    ap.add_argument("--tokens", type=int, default=0, help="tokens per step (default: workload's first)")
+    ap.add_argument("--layers", type=int, default=0, help="resident layers rotated (default 4)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained"), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def record_bytes(wl):
+    return synth.record_layout(wl.hidden, wl.inter, wl.fmt)["bytes"]
+
+
+def alg_bytes(wl, T, U):
+    """Algorithmic bytes of one layer: unique experts' records (+ shared), router weight and
+    bias, activations in, output out."""
+    rec = record_bytes(wl)
+    act = 4 if wl.act == "f32" else 2
+    return ((U + wl.n_shared) * rec + wl.n_experts * wl.hidden * 4 + wl.n_experts * 4
+            + T * wl.hidden * act + T * wl.hidden * 4)
+
+
+def alg_flops(wl, T):
+    return (T * wl.top_k + T * wl.n_shared) * 6 * wl.hidden * wl.inter + T * wl.n_experts * wl.hidden * 2
+
+
+def src_hash(paths):
+    h = hashlib.sha256()
+    for p in paths:
+        h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+class Clocks:
+    """nvidia-smi sampler around the loaded window."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={index}", f"--query-gpu={self.Q}",
+                                       "--format=csv,noheader,nounits", "-lms", "100"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(5)
+        except Exception:
+            self.p.kill()
+        self.f.flush()
+        rows = [r.split(",") for r in open(self.f.name).read().strip().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1])); mx = float(r[2])
+                for n, v in zip(names, r[5:9]):
+                    if v.strip().lower() == "active":
+                        reasons.add(n)
+            except Exception:
+                pass
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------- GPU arm ----------
+
+def gpu_arm(args, rank, world, dist):
+    import quantized_routed_expert_noaux_b200 as q
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    wl = synth.WORKLOADS[args.workload]
+    T = args.tokens or wl.tokens[0]
+    n_layers = args.layers or (4 if wl.hidden >= 2048 else 1)
+    cfg = q.config_for(wl)
+
+    layers = []
+    for l in range(n_layers):
+        ex = synth.make_expert_records(wl, device=dev, layer=l)
+        sh = synth.make_shared_record(wl, device=dev, layer=l)
+        Wr, b = synth.make_router(wl, device=dev, layer=l)
+        layers.append((ex, sh, Wr, b, q.weights_for(Wr, b, ex, sh)))
+    n_x = 64
+    xs = [synth.make_activations(wl, T, device=dev, step=1000 * rank + i) for i in range(n_x)]
+    K, W = args.steps, args.warmup
+    out = torch.empty(T, wl.hidden, dtype=torch.float32, device=dev)
+    ids_all = torch.empty(K, T, wl.top_k, dtype=torch.int32, device=dev)
+    ws = torch.empty(q.coli_moe_workspace_size(cfg, T), dtype=torch.uint8, device=dev)
+    st = torch.cuda.current_stream()
+
+    def step(i, ids=None):
+        ex, sh, Wr, b, wts = layers[i % n_layers]
+        q.coli_moe_layer(cfg, wts, xs[i % n_x], T, out, ids, None, ws, st.cuda_stream)
+
+    clocks = Clocks(dev.index if dev.index is not None else 0)
+    q.coli_moe_clear_error(ws)
+    t_soak = time.time()
+    i = 0
+    while i < W or time.time() - t_soak < 1.0:  # >= W warm-up steps and >= 1 s under load
+        step(i)
+        i += 1
+        if i % 256 == 0:
+            torch.cuda.synchronize()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for k in range(K):
+        step(k, ids_all[k])
+    e1.record(st)
+    torch.cuda.synchronize()
+    barrier()
+    ms = e0.elapsed_time(e1)
+    clk = clocks.stop()
+    err = q.coli_moe_error_word(ws)
+    if err:
+        raise RuntimeError(f"device error word {err:#x} after the timed region")
+    ms_max = ms
+    if dist is not None:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+
+    # algorithmic bytes of the timed steps (unique experts per step from the routing written)
+    ids_np = ids_all.cpu().numpy()
+    U = np.array([len(np.unique(ids_np[k])) for k in range(K)])
+    bytes_steps = sum(alg_bytes(wl, T, int(u)) for u in U)
+    expert_bytes = sum((int(u) + wl.n_shared) * record_bytes(wl) for u in U)
+
+    # live per-launch time of the expert FFN (gate/up + down GEMV kernels), same rotation
+    offs = torch.empty(wl.n_experts + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(T * wl.top_k, dtype=torch.int32, device=dev)
+    cnt = torch.empty(wl.n_experts, dtype=torch.int32, device=dev)
+    uq = torch.empty(wl.n_experts, dtype=torch.int32, device=dev)
+    nu = torch.empty(1, dtype=torch.int32, device=dev)
+    lg = torch.empty(T, wl.n_experts, dtype=torch.float32, device=dev)
+    tw = torch.empty(T, wl.top_k, dtype=torch.float32, device=dev)
+    tid = torch.empty(T, wl.top_k, dtype=torch.int32, device=dev)
+    n_ffn = min(K, 500)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n_ffn)]
+    for k in range(n_ffn):
+        ex, sh, Wr, b, wts = layers[k % n_layers]
+        x = xs[k % n_x]
+        q.coli_moe_gate(cfg, Wr, x, T, lg, st.cuda_stream)
+        q.coli_moe_route(cfg, lg, b, T, tid, tw, st.cuda_stream)
+        q.coli_moe_group(cfg, tid, T, cnt, offs, perm, uq, nu, ws, st.cuda_stream)
+        evs[k][0].record(st)
+        q.coli_moe_ffn(cfg, wts, x, T, tw, offs, perm, uq, nu, out, ws, st.cuda_stream)
+        evs[k][1].record(st)
+    torch.cuda.synchronize()
+    ffn_ms = sum(a.elapsed_time(b) for a, b in evs) / n_ffn
+    U_mean = float(U[:n_ffn].mean()) if len(U) else 0.0
+    ffn_bytes = (U_mean + wl.n_shared) * record_bytes(wl) + T * wl.hidden * (4 if wl.act == "f32" else 2) \
+        + T * wl.hidden * 4
+
+    # end to end through the C ABI with host buffers: pinned H2D of x, layer, D2H of out
+    x_host = [xs[i].cpu().pin_memory() for i in range(n_x)]
+    out_host = torch.empty(T, wl.hidden, dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(xs[0])
+    K2 = min(K, 1000)
+    barrier()
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(st)
+    for k in range(K2):
+        x_dev.copy_(x_host[k % n_x], non_blocking=True)
+        ex, sh, Wr, b, wts = layers[k % n_layers]
+        q.coli_moe_layer(cfg, wts, x_dev, T, out, None, None, ws, st.cuda_stream)
+        out_host.copy_(out, non_blocking=True)
+    f1.record(st)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = f0.elapsed_time(f1)
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    hbm, bf16, bf16s, peak_kind = peaks()
+    tok_s = world * K * T / (ms_max / 1e3)
+    achieved = ffn_bytes / (ffn_ms / 1e3) / 1e9
+    traffic = None
+    tf = os.path.join(PROFILES, f"{args.workload}_t{T}_traffic.json")
+    if os.path.exists(tf):
+        d = json.load(open(tf))
+        cur = src_hash([os.path.join(ROOT, "quantized_routed_expert_noaux_b200", "csrc", f)
+                        for f in d.get("sources", [])])
+        if d.get("source_hash") == cur:
+            traffic = d.get("traffic_bytes_per_launch")
+
+    res = {
+        "metric": METRIC,
+        "value": round(tok_s, 2),
+        "unit": "tokens/s",
+        "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": round(ms_max / K, 6),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic (seeded; weights N(0,0.02) quantised per row, activations N(0,1))",
+        "config": {
+            "workload": f"{wl.name} (GLM-5.2-shaped decode layer)" if wl.name == "glm_decode" else wl.name,
+            "tokens_per_step": T, "hidden": wl.hidden, "expert_inter": wl.inter,
+            "experts": wl.n_experts, "top_k": wl.top_k, "n_group": wl.n_group,
+            "topk_group": wl.topk_group, "shared_experts": wl.n_shared,
+            "weights": {4: "packed int4", 8: "int8", 2: "packed int2"}[wl.fmt] + " per-row f32 scales",
+            "activations": wl.act,
+            "l2": f"rotation over {n_layers} resident layers ({n_layers * wl.n_experts * record_bytes(wl) / 1e9:.1f} GB of expert records) + fresh activations every step; no flush",
+            "parallelism": f"replicas x{world}",
+        },
+        "expert_gbs": round(expert_bytes / (ms_max / 1e3) / 1e9, 1),
+        "layer_gbs": round(bytes_steps / (ms_max / 1e3) / 1e9, 1),
+        "layer_frac_of_hbm": round(bytes_steps / (ms_max / 1e3) / 1e9 / hbm, 4),
+        "unique_experts_mean": round(float(U.mean()), 2),
+        "roofline": {
+            "bound": "hbm",
+            "kernel": "expert FFN (gate/up GEMV + down GEMV with fused combine)",
+            "achieved": round(achieved, 1),
+            "peak": hbm,
+            "unit": "GB/s",
+            "frac": round(achieved / hbm, 4),
+            "traffic": traffic,
+            "peak_source": f"{peak_kind} hbm_gbs (copy bandwidth)",
+            "launch_us": round(ffn_ms * 1e3, 2),
+        },
+        "e2e": {"value": round(world * K2 * T / (e2e_ms / 1e3), 2), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(xs[0].numel() * xs[0].element_size()),
+                "d2h_bytes_per_step": int(out.numel() * 4)},
+        "gpu_launches": 5 * K,
+        "clocks": clk,
+    }
+    return res, (wl, T, layers, xs)
+
+
+# ------------------------------------------------------------------------- CPU oracle -------
+
+def _oracle_sample(wl, T_tokens, x_list, layers_dev, budget_s, device):
+    """Run the oracle on a bounded sample of the workload's tokens; returns (tokens, seconds,
+    threads)."""
+    import oracle
+    cfg = oracle.make_cfg(wl)
+    threads = os.cpu_count() or 1
+    ex, sh, Wr, b = layers_dev
+    Wr_h, b_h = Wr.cpu(), b.cpu()
+    cache = {}
+
+    def recs_for(xh, n):
+        lg = oracle.gate(cfg, Wr_h, xh, n)
+        ids, _ = oracle.route(cfg, lg, b_h, n)
+        for e in np.unique(ids):
+            if int(e) not in cache:
+                cache[int(e)] = ex[int(e)].cpu().numpy()
+        table = [cache.get(e) for e in range(wl.n_experts)]
+        return oracle.Records(table, None if sh is None else sh.cpu().numpy())
+
+    # calibrate on one token
+    x0 = x_list[0][:1].cpu()
+    R = recs_for(x0, 1)
+    t0 = time.time()
+    oracle.layer(cfg, Wr_h, b_h, R, x0, 1, n_threads=1)
+    per_tok = max(time.time() - t0, 1e-4)
+    n = int(max(1, min(budget_s * threads / per_tok, 4096)))
+    n = max(n, min(threads, 4096))
+    xs = torch.cat([x.cpu() for x in x_list], 0)
+    while xs.shape[0] < n:
+        xs = torch.cat([xs, xs], 0)
+    xs = xs[:n].contiguous()
+    R = recs_for(xs, n)
+    t0 = time.time()
+    oracle.layer(cfg, Wr_h, b_h, R, xs, n, n_threads=threads)
+    return n, time.time() - t0, threads
+
+
+def reference_arm(args):
+    """The CPU oracle as the reference implementation, on the host cores."""
+    wl = synth.WORKLOADS[args.workload]
+    T = args.tokens or wl.tokens[0]
+    device = "cuda" if torch.cuda.is_available() else "cpu"
+    import oracle
+    cfg = oracle.make_cfg(wl)
+    threads = os.cpu_count() or 1
+    K, W = args.steps, args.warmup
+    # the oracle is slow: a step is a bounded sample of T tokens, the same batch shape
+    ex = synth.make_expert_records(wl, device=device, experts=[])
+    sh = synth.make_shared_record(wl, device=device)
+    Wr, b = synth.make_router(wl, device=device)
+    Wr_h, b_h = Wr.cpu(), b.cpu()
+    per_step = []
+    made = set()
+    budget = 150.0
+    t_start = time.time()
+    steps_done = 0
+    for k in range(W + K):
+        x = synth.make_activations(wl, T, device=device, step=k).cpu()
+        lg = oracle.gate(cfg, Wr_h, x, T)
+        ids, _ = oracle.route(cfg, lg, b_h, T)
+        need = [int(e) for e in np.unique(ids) if int(e) not in made]
+        if need:
+            synth.make_expert_records(wl, device=device, experts=need, out=ex)
+            made.update(need)
+        table = [ex[e].cpu().numpy() if e in made else None for e in range(wl.n_experts)]
+        R = oracle.Records(table, None if sh is None else sh.cpu().numpy())
+        t0 = time.time()
+        oracle.layer(cfg, Wr_h, b_h, R, x, T, n_threads=threads)
+        dt = time.time() - t0
+        if k >= W:
+            per_step.append(dt)
+            steps_done += 1
+        if time.time() - t_start > budget and steps_done >= 1:
+            break
+    sec = sum(per_step)
+    val = steps_done * T / sec
+    return {
+        "metric": METRIC, "impl": "reference", "value": round(val, 4), "unit": "tokens/s",
+        "n_gpus": 1, "steps": steps_done, "warmup": W, "ms_per_step": round(1e3 * sec / steps_done, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)",
+        "config": {"workload": wl.name, "tokens_per_step": T},
+        "cpu_baseline": {"value": round(val, 4), "unit": "tokens/s", "cores": threads,
+                         "kind": "oracle",
+                         "sample": f"{steps_done} steps of {T} token(s) each (run stopped after {budget:.0f} s if K was larger)"},
+        "e2e": {"value": round(val, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        print(json.dumps(reference_arm(args)))
+        return
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist_mod
+        dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = dist_mod
+    res, ctx = gpu_arm(args, rank, world, dist)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        wl, T, layers, xs = ctx
+        n, sec, thr = _oracle_sample(wl, T, xs[:8], layers[0][:4], args.cpu_seconds, None)
+        res["cpu_baseline"] = {"value": round(n / sec, 4), "unit": "tokens/s", "cores": thr,
+                               "kind": "oracle",
+                               "sample": f"{n} tokens of the same workload (layer 0), {sec:.1f} s wall on {thr} threads"}
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res))
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,153 @@
+/*
+ * coli_moe.h -- C ABI of the routed-expert MoE layer on NVIDIA B200 (sm_100a).
+ *
+ * The layer (colibri-strix README, "What's implemented"): a DeepSeek-V3-style sigmoid router
+ * with the noaux_tc selection bias and routed_scaling_factor, batch-union grouping ("each unique
+ * expert of the batch is read once and applied to every position that routes to it"), SwiGLU
+ * experts stored as packed int4 (also int8 / packed int2) with per-row scales and dequantised on
+ * use, a shared expert, and the weighted combine.  The JustVugg/colibri README ("Never wait for
+ * the disk twice") adds that an expert's three matrices are stored adjacent.
+ *
+ * Conventions shared by every call
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The library allocates no
+ *     device memory; scratch comes from a caller-provided workspace (coli_moe_workspace_size).
+ *   - Every compute call is asynchronous on `stream` (a cudaStream_t passed as void*; NULL is
+ *     the legacy default stream).  Host-side validation happens before any launch; a non-OK
+ *     status means nothing was launched.
+ *   - Device-side anomalies (an expert id out of range, inconsistent grouping arrays) never
+ *     trap: the kernel skips the bad item and records a code in the workspace's error word,
+ *     which coli_moe_error_word() reads back.
+ *   - There is no CPU fallback: every step runs in this library's CUDA kernels.
+ *
+ * Record format (one per expert; the same for the shared expert with its own inter size)
+ *   Wg codes [I][H] | Wu codes [I][H] | Wd codes [H][I] | sg[I] f32 | su[I] f32 | sd[H] f32,
+ *   rows packed to whole bytes: int4 element 2j in the low nibble of byte j and 2j+1 in the
+ *   high nibble (two's complement, [-8,7]); int2 element 4j+k in bits [2k,2k+1] of byte j
+ *   ([-2,1]); int8 one signed byte.  The weight is code * scale of its output row.  Records sit
+ *   `expert_stride` bytes apart (a multiple of 256) and the record base must be 256-byte aligned.
+ *
+ * Tensor layouts (row-major):
+ *   x        [T][H]   float32 (act = COLI_ACT_F32) or bfloat16 bits (COLI_ACT_BF16), 16-B aligned
+ *   logits   [T][E]   float32
+ *   topk_ids [T][K]   int32, slot order = descending biased score (ties: lower expert id)
+ *   topk_w   [T][K]   float32
+ *   out      [T][H]   float32, 16-B aligned
+ */
+#ifndef COLI_MOE_H
+#define COLI_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    COLI_OK = 0,
+    COLI_ERR_INVALID_ARG = 1,  /* NULL pointer, negative size, bad enum value */
+    COLI_ERR_SHAPE = 2,        /* sizes inconsistent with each other or with the formats */
+    COLI_ERR_ALIGN = 3,        /* a pointer or stride misses its required alignment */
+    COLI_ERR_UNSUPPORTED = 4,  /* a valid configuration this build does not implement */
+    COLI_ERR_CUDA = 5,         /* a CUDA runtime call failed (launch, attribute, copy) */
+    COLI_ERR_DEVICE = 6,       /* the device error word was set by a kernel */
+    COLI_ERR_WORKSPACE = 7     /* workspace NULL, misaligned or smaller than required */
+} coli_status;
+
+typedef enum { COLI_W_INT2 = 2, COLI_W_INT4 = 4, COLI_W_INT8 = 8 } coli_wfmt;
+typedef enum { COLI_ACT_F32 = 0, COLI_ACT_BF16 = 1 } coli_act;
+
+/* Device error word codes (bit flags, OR-ed together by the kernels). */
+#define COLI_DEVERR_EXPERT_ID 0x1   /* an expert id or unique-list entry outside [0, E) */
+#define COLI_DEVERR_GROUPING 0x2    /* offsets/perm inconsistent (slot outside [0, T*K)) */
+
+typedef struct {
+    int hidden;             /* H */
+    int inter;              /* I, routed expert intermediate size */
+    int n_experts;          /* E (<= 1024) */
+    int top_k;              /* K (<= 32) */
+    int n_group;            /* G; E % G == 0 */
+    int topk_group;         /* TG, 1 <= TG <= G */
+    int n_shared;           /* 0 or 1 */
+    int shared_inter;       /* I_s; must equal inter when n_shared == 1 */
+    double routed_scaling;  /* rsf */
+    int wfmt;               /* coli_wfmt */
+    int act;                /* coli_act */
+} coli_moe_config;
+
+typedef struct {
+    const float *router_w;     /* [E][H] float32 */
+    const float *router_bias;  /* [E] float32, the noaux_tc selection bias */
+    const uint8_t *experts;    /* E records, expert_stride bytes apart, 256-B aligned */
+    size_t expert_stride;      /* bytes; multiple of 256 and >= the record size */
+    const uint8_t *shared;     /* the shared expert's record (NULL when n_shared == 0) */
+} coli_moe_weights;
+
+/* Text for a status code (static storage). */
+const char *coli_moe_status_str(coli_status s);
+
+/* Bytes of one record for (hidden, inter, wfmt), before padding to 256.  Host only. */
+coli_status coli_moe_record_bytes(int hidden, int inter, int wfmt, size_t *bytes);
+
+/* Validates a configuration (the same checks every call makes).  Host only. */
+coli_status coli_moe_check_config(const coli_moe_config *cfg);
+
+/* Workspace bytes that coli_moe_layer / coli_moe_ffn / coli_moe_group need for up to
+ * max_tokens tokens.  The workspace must be 256-byte aligned and is owned by the caller; calls
+ * that share one workspace must be ordered on the GPU (same stream or events).  Host only. */
+coli_status coli_moe_workspace_size(const coli_moe_config *cfg, int max_tokens, size_t *bytes);
+
+/* Clears the workspace's device error word (asynchronous on stream). */
+coli_status coli_moe_clear_error(void *ws, void *stream);
+
+/* Synchronises `stream` and returns the workspace's device error word in *code (0 = clean). */
+coli_status coli_moe_error_word(void *ws, void *stream, int *code);
+
+/* a1, router gate projection (colibri-strix README, "What's implemented": sigmoid router).
+ * logits[t][e] = float32( sum_h x[t][h] * router_w[e][h] ), the products and the sum taken in
+ * double precision, rounded once to float32.  T = 0 is a no-op. */
+coli_status coli_moe_gate(const coli_moe_config *cfg, const float *router_w, const void *x,
+                          int T, float *logits, void *stream);
+
+/* a2, noaux_tc routing (colibri-strix README, "What's implemented": DeepSeek-V3-style sigmoid
+ * router (noaux_tc, routed_scaling_factor)).  Per token, in double: s = 1/(1+exp(-logit)),
+ * c = s + bias; if G > 1 each group scores the sum of its two largest c and the TG best groups
+ * are kept (ties: lower group); the K largest c among kept experts are selected (ties: lower
+ * id), written in descending c order; topk_w[k] = float32(s_k / sum_k s_k * routed_scaling).
+ * The bias steers selection only.  T = 0 is a no-op. */
+coli_status coli_moe_route(const coli_moe_config *cfg, const float *logits, const float *bias,
+                           int T, int32_t *topk_ids, float *topk_w, void *stream);
+
+/* a3, batch-union grouping (colibri-strix README, "What's implemented": batch-union MoE).
+ * A stable counting sort of the T*K slots s = t*K + k by expert id: counts[E], offsets[E+1]
+ * (exclusive scan, offsets[E] = T*K), perm[T*K] (slot indices grouped by expert, ascending
+ * slot index inside each expert), unique_ids[E] (ids with counts > 0, ascending, the rest -1),
+ * n_unique[1].  Ids outside [0,E) are skipped and flagged in the error word of `ws`. */
+coli_status coli_moe_group(const coli_moe_config *cfg, const int32_t *topk_ids, int T,
+                           int32_t *counts, int32_t *offsets, int32_t *perm,
+                           int32_t *unique_ids, int32_t *n_unique, void *ws, size_t ws_bytes,
+                           void *stream);
+
+/* a4..a7 for a given routing (JustVugg/colibri README, "Never wait for the disk twice":
+ * batched positions read each unique expert once; colibri-strix README, "What's implemented":
+ * dequant-on-use, shared expert).  For every unique expert e and every slot routed to it:
+ * y = sd .* (Qd (SiLU(sg .* (Qg x)) .* (su .* (Qu x)))) with the codes Q dequantised in
+ * registers; out[t] = sum over t's experts of topk_w * y + y_shared (weight 1).  The grouping
+ * arrays are those coli_moe_group writes.  `out` is fully overwritten.  Each expert's weights
+ * are streamed from HBM once per call. */
+coli_status coli_moe_ffn(const coli_moe_config *cfg, const coli_moe_weights *w, const void *x,
+                         int T, const float *topk_w, const int32_t *offsets,
+                         const int32_t *perm, const int32_t *unique_ids,
+                         const int32_t *n_unique, float *out, void *ws, size_t ws_bytes,
+                         void *stream);
+
+/* The whole layer: gate, route, group, ffn (all of the above, in that order, on `stream`).
+ * topk_ids_out / topk_w_out may be NULL; when given they receive the routing. */
+coli_status coli_moe_layer(const coli_moe_config *cfg, const coli_moe_weights *w,
+                           const void *x, int T, float *out, int32_t *topk_ids_out,
+                           float *topk_w_out, void *ws, size_t ws_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* COLI_MOE_H */

@@ -1,0 +1,270 @@
+// coli_moe.cu -- the C ABI of libcoli_moe.so: argument validation, workspace carve-up, and the
+// launch sequence of the layer.  No device memory is allocated here; no CPU fallback exists.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "coli_moe.h"
+#include "internal.h"
+
+namespace coli {
+
+namespace {
+
+inline size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+inline bool aligned(const void *p, size_t a) {
+    return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+
+coli_status from_cuda(cudaError_t e) { return e == cudaSuccess ? COLI_OK : COLI_ERR_CUDA; }
+
+int row_bytes(int n, int fmt) { return n * fmt / 8; }
+
+}  // namespace
+
+int device_sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+WsLayout ws_layout(const coli_moe_config &c, int T) {
+    WsLayout L;
+    const size_t n = static_cast<size_t>(T) * c.top_k;
+    const size_t E = static_cast<size_t>(c.n_experts);
+    size_t o = 0;
+    L.err = o;      o = align256(o + 256);
+    L.logits = o;   o = align256(o + static_cast<size_t>(T) * E * 4);
+    L.ids = o;      o = align256(o + n * 4);
+    L.w = o;        o = align256(o + n * 4);
+    L.counts = o;   o = align256(o + E * 4);
+    L.offsets = o;  o = align256(o + (E + 1) * 4);
+    L.perm = o;     o = align256(o + n * 4);
+    L.unique = o;   o = align256(o + E * 4);
+    L.nuniq = o;    o = align256(o + 4);
+    L.h = o;        o = align256(o + (n + static_cast<size_t>(T) * c.n_shared) * c.inter * 4);
+    L.total = o;
+    return L;
+}
+
+}  // namespace coli
+
+using namespace coli;
+
+extern "C" {
+
+const char *coli_moe_status_str(coli_status s) {
+    switch (s) {
+        case COLI_OK: return "ok";
+        case COLI_ERR_INVALID_ARG: return "invalid argument";
+        case COLI_ERR_SHAPE: return "inconsistent shape";
+        case COLI_ERR_ALIGN: return "misaligned pointer or stride";
+        case COLI_ERR_UNSUPPORTED: return "unsupported configuration";
+        case COLI_ERR_CUDA: return "CUDA runtime error";
+        case COLI_ERR_DEVICE: return "device error word set";
+        case COLI_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    }
+    return "unknown status";
+}
+
+coli_status coli_moe_record_bytes(int hidden, int inter, int wfmt, size_t *bytes) {
+    if (!bytes) return COLI_ERR_INVALID_ARG;
+    if (wfmt != COLI_W_INT4 && wfmt != COLI_W_INT8 && wfmt != COLI_W_INT2) return COLI_ERR_INVALID_ARG;
+    if (hidden <= 0 || inter <= 0) return COLI_ERR_SHAPE;
+    if ((static_cast<long>(hidden) * wfmt) % 8 || (static_cast<long>(inter) * wfmt) % 8) return COLI_ERR_SHAPE;
+    const size_t rh = static_cast<size_t>(hidden) * wfmt / 8, ri = static_cast<size_t>(inter) * wfmt / 8;
+    *bytes = 2 * static_cast<size_t>(inter) * rh + static_cast<size_t>(hidden) * ri +
+             (2 * static_cast<size_t>(inter) + hidden) * sizeof(float);
+    return COLI_OK;
+}
+
+coli_status coli_moe_check_config(const coli_moe_config *c) {
+    if (!c) return COLI_ERR_INVALID_ARG;
+    if (c->wfmt != COLI_W_INT4 && c->wfmt != COLI_W_INT8 && c->wfmt != COLI_W_INT2) return COLI_ERR_INVALID_ARG;
+    if (c->act != COLI_ACT_F32 && c->act != COLI_ACT_BF16) return COLI_ERR_INVALID_ARG;
+    if (c->hidden <= 0 || c->inter <= 0 || c->n_experts <= 0 || c->top_k <= 0 || c->n_group <= 0 ||
+        c->topk_group <= 0 || c->n_shared < 0)
+        return COLI_ERR_SHAPE;
+    if (!(c->routed_scaling > 0.0)) return COLI_ERR_INVALID_ARG;
+    if (c->n_experts % c->n_group) return COLI_ERR_SHAPE;
+    if (c->topk_group > c->n_group) return COLI_ERR_SHAPE;
+    const int gs = c->n_experts / c->n_group;
+    if (c->n_group > 1 && c->topk_group < c->n_group && gs < 2) return COLI_ERR_SHAPE;
+    if (c->top_k > c->topk_group * gs) return COLI_ERR_SHAPE;
+    if (c->n_experts > 1024 || c->top_k > 32 || c->n_group > 32) return COLI_ERR_UNSUPPORTED;
+    if (c->n_shared > 1) return COLI_ERR_UNSUPPORTED;
+    if (c->n_shared == 1 && c->shared_inter != c->inter) return COLI_ERR_UNSUPPORTED;
+    if (c->hidden % 64 || c->inter % 64) return COLI_ERR_SHAPE;
+    if (!gemv_shape_ok(row_bytes(c->hidden, c->wfmt)) || !gemv_shape_ok(row_bytes(c->inter, c->wfmt)))
+        return COLI_ERR_UNSUPPORTED;
+    return COLI_OK;
+}
+
+coli_status coli_moe_workspace_size(const coli_moe_config *c, int max_tokens, size_t *bytes) {
+    if (!bytes) return COLI_ERR_INVALID_ARG;
+    coli_status s = coli_moe_check_config(c);
+    if (s != COLI_OK) return s;
+    if (max_tokens < 0) return COLI_ERR_SHAPE;
+    *bytes = ws_layout(*c, max_tokens > 0 ? max_tokens : 1).total;
+    return COLI_OK;
+}
+
+coli_status coli_moe_clear_error(void *ws, void *stream) {
+    if (!ws || !aligned(ws, 256)) return COLI_ERR_WORKSPACE;
+    return from_cuda(cudaMemsetAsync(ws, 0, sizeof(int), static_cast<cudaStream_t>(stream)));
+}
+
+coli_status coli_moe_error_word(void *ws, void *stream, int *code) {
+    if (!ws || !code || !aligned(ws, 256)) return COLI_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int v = 0;
+    cudaError_t e = cudaMemcpyAsync(&v, ws, sizeof(int), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return COLI_ERR_CUDA;
+    *code = v;
+    return COLI_OK;
+}
+
+coli_status coli_moe_gate(const coli_moe_config *c, const float *router_w, const void *x, int T,
+                          float *logits, void *stream) {
+    coli_status s = coli_moe_check_config(c);
+    if (s != COLI_OK) return s;
+    if (T < 0) return COLI_ERR_SHAPE;
+    if (T == 0) return COLI_OK;
+    if (!router_w || !x || !logits) return COLI_ERR_INVALID_ARG;
+    if (!aligned(router_w, 16) || !aligned(x, 16) || !aligned(logits, 4)) return COLI_ERR_ALIGN;
+    return from_cuda(launch_gate(*c, router_w, x, T, logits, static_cast<cudaStream_t>(stream)));
+}
+
+coli_status coli_moe_route(const coli_moe_config *c, const float *logits, const float *bias, int T,
+                           int32_t *topk_ids, float *topk_w, void *stream) {
+    coli_status s = coli_moe_check_config(c);
+    if (s != COLI_OK) return s;
+    if (T < 0) return COLI_ERR_SHAPE;
+    if (T == 0) return COLI_OK;
+    if (!logits || !bias || !topk_ids || !topk_w) return COLI_ERR_INVALID_ARG;
+    if (!aligned(logits, 4) || !aligned(bias, 4) || !aligned(topk_ids, 4) || !aligned(topk_w, 4))
+        return COLI_ERR_ALIGN;
+    return from_cuda(launch_route(*c, logits, bias, T, topk_ids, topk_w, static_cast<cudaStream_t>(stream)));
+}
+
+coli_status coli_moe_group(const coli_moe_config *c, const int32_t *topk_ids, int T, int32_t *counts,
+                           int32_t *offsets, int32_t *perm, int32_t *unique_ids, int32_t *n_unique,
+                           void *ws, size_t ws_bytes, void *stream) {
+    coli_status s = coli_moe_check_config(c);
+    if (s != COLI_OK) return s;
+    if (T < 0) return COLI_ERR_SHAPE;
+    if (!ws || !aligned(ws, 256) || ws_bytes < 256) return COLI_ERR_WORKSPACE;
+    if (!counts || !offsets || !unique_ids || !n_unique) return COLI_ERR_INVALID_ARG;
+    if (T > 0 && (!topk_ids || !perm)) return COLI_ERR_INVALID_ARG;
+    if (static_cast<long>(T) * c->top_k > (1L << 30)) return COLI_ERR_SHAPE;
+    return from_cuda(launch_group(*c, topk_ids, T, counts, offsets, perm, unique_ids, n_unique,
+                                  static_cast<int *>(ws), static_cast<cudaStream_t>(stream)));
+}
+
+static coli_status check_weights(const coli_moe_config *c, const coli_moe_weights *w, bool need_router) {
+    if (!w) return COLI_ERR_INVALID_ARG;
+    if (!w->experts) return COLI_ERR_INVALID_ARG;
+    if (need_router && (!w->router_w || !w->router_bias)) return COLI_ERR_INVALID_ARG;
+    if (c->n_shared == 1 && !w->shared) return COLI_ERR_INVALID_ARG;
+    size_t rb = 0;
+    coli_status s = coli_moe_record_bytes(c->hidden, c->inter, c->wfmt, &rb);
+    if (s != COLI_OK) return s;
+    if (w->expert_stride < rb) return COLI_ERR_SHAPE;
+    if (w->expert_stride % 256 || !aligned(w->experts, 256)) return COLI_ERR_ALIGN;
+    if (w->shared && !aligned(w->shared, 256)) return COLI_ERR_ALIGN;
+    if (need_router && (!aligned(w->router_w, 16) || !aligned(w->router_bias, 4))) return COLI_ERR_ALIGN;
+    return COLI_OK;
+}
+
+static FfnParams make_params(const coli_moe_config *c, const coli_moe_weights *w, const void *x, int T,
+                             const float *topk_w, const int32_t *offsets, const int32_t *perm,
+                             const int32_t *unique, const int32_t *n_unique, float *out, float *h,
+                             int *err) {
+    FfnParams p;
+    p.H = c->hidden; p.I = c->inter; p.E = c->n_experts; p.K = c->top_k; p.T = T; p.S = c->n_shared;
+    p.fmt = c->wfmt; p.act = c->act;
+    p.experts = w->experts; p.stride = w->expert_stride; p.shared = w->shared;
+    p.rb_h = static_cast<size_t>(c->hidden) * c->wfmt / 8;
+    p.rb_i = static_cast<size_t>(c->inter) * c->wfmt / 8;
+    p.off_wu = static_cast<size_t>(c->inter) * p.rb_h;
+    p.off_wd = 2 * p.off_wu;
+    p.off_sg = p.off_wd + static_cast<size_t>(c->hidden) * p.rb_i;
+    p.off_su = p.off_sg + static_cast<size_t>(c->inter) * 4;
+    p.off_sd = p.off_su + static_cast<size_t>(c->inter) * 4;
+    p.x = x; p.topk_w = topk_w; p.offsets = offsets; p.perm = perm; p.unique = unique;
+    p.n_unique = n_unique; p.h = h; p.out = out; p.err = err;
+    return p;
+}
+
+static coli_status run_ffn(const FfnParams &p, cudaStream_t st) {
+    return from_cuda(launch_ffn_gemv(p, st));
+}
+
+coli_status coli_moe_ffn(const coli_moe_config *c, const coli_moe_weights *w, const void *x, int T,
+                         const float *topk_w, const int32_t *offsets, const int32_t *perm,
+                         const int32_t *unique_ids, const int32_t *n_unique, float *out, void *ws,
+                         size_t ws_bytes, void *stream) {
+    coli_status s = coli_moe_check_config(c);
+    if (s != COLI_OK) return s;
+    if (T < 0) return COLI_ERR_SHAPE;
+    if (T == 0) return COLI_OK;
+    s = check_weights(c, w, false);
+    if (s != COLI_OK) return s;
+    if (!x || !topk_w || !offsets || !perm || !unique_ids || !n_unique || !out) return COLI_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(out, 16)) return COLI_ERR_ALIGN;
+    if (T > gemv_max_tokens(*c)) return COLI_ERR_UNSUPPORTED;
+    const WsLayout L = ws_layout(*c, T);
+    if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return COLI_ERR_WORKSPACE;
+    char *base = static_cast<char *>(ws);
+    FfnParams p = make_params(c, w, x, T, topk_w, offsets, perm, unique_ids, n_unique, out,
+                              reinterpret_cast<float *>(base + L.h), reinterpret_cast<int *>(base + L.err));
+    return run_ffn(p, static_cast<cudaStream_t>(stream));
+}
+
+coli_status coli_moe_layer(const coli_moe_config *c, const coli_moe_weights *w, const void *x, int T,
+                           float *out, int32_t *topk_ids_out, float *topk_w_out, void *ws,
+                           size_t ws_bytes, void *stream) {
+    coli_status s = coli_moe_check_config(c);
+    if (s != COLI_OK) return s;
+    if (T < 0) return COLI_ERR_SHAPE;
+    if (T == 0) return COLI_OK;
+    s = check_weights(c, w, true);
+    if (s != COLI_OK) return s;
+    if (!x || !out) return COLI_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(out, 16)) return COLI_ERR_ALIGN;
+    if ((topk_ids_out && !aligned(topk_ids_out, 4)) || (topk_w_out && !aligned(topk_w_out, 4)))
+        return COLI_ERR_ALIGN;
+    if (T > gemv_max_tokens(*c)) return COLI_ERR_UNSUPPORTED;
+    const WsLayout L = ws_layout(*c, T);
+    if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return COLI_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char *base = static_cast<char *>(ws);
+    float *logits = reinterpret_cast<float *>(base + L.logits);
+    int32_t *ids = topk_ids_out ? topk_ids_out : reinterpret_cast<int32_t *>(base + L.ids);
+    float *wts = topk_w_out ? topk_w_out : reinterpret_cast<float *>(base + L.w);
+    int32_t *counts = reinterpret_cast<int32_t *>(base + L.counts);
+    int32_t *offsets = reinterpret_cast<int32_t *>(base + L.offsets);
+    int32_t *perm = reinterpret_cast<int32_t *>(base + L.perm);
+    int32_t *uniq = reinterpret_cast<int32_t *>(base + L.unique);
+    int32_t *nu = reinterpret_cast<int32_t *>(base + L.nuniq);
+    int *err = reinterpret_cast<int *>(base + L.err);
+
+    cudaError_t e = launch_gate(*c, w->router_w, x, T, logits, st);
+    if (e == cudaSuccess) e = launch_route(*c, logits, w->router_bias, T, ids, wts, st);
+    if (e == cudaSuccess) e = launch_group(*c, ids, T, counts, offsets, perm, uniq, nu, err, st);
+    if (e != cudaSuccess) return COLI_ERR_CUDA;
+    FfnParams p = make_params(c, w, x, T, wts, offsets, perm, uniq, nu, out,
+                              reinterpret_cast<float *>(base + L.h), err);
+    return run_ffn(p, st);
+}
+
+}  // extern "C"

@@ -1,0 +1,66 @@
+// internal.h -- declarations shared by the translation units of libcoli_moe.so (not installed).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "coli_moe.h"
+
+namespace coli {
+
+// Parameters of the expert half of the layer (a4..a7), shared by the GEMV and MMA kernels.
+struct FfnParams {
+    int H, I, E, K, T, S;              // S = n_shared (0 or 1); shared inter == I
+    int fmt;                           // 4, 8, 2
+    int act;                           // coli_act of x
+    const uint8_t *experts;            // E records
+    size_t stride;                     // record stride, bytes
+    const uint8_t *shared;             // shared record or nullptr
+    size_t off_wu, off_wd, off_sg, off_su, off_sd;  // byte offsets inside a record
+    size_t rb_h, rb_i;                 // bytes of a row of length H / of length I
+    const void *x;                     // [T][H] f32 or bf16
+    const float *topk_w;               // [T*K]
+    const int32_t *offsets;            // [E+1]
+    const int32_t *perm;               // [T*K]
+    const int32_t *unique;             // [E]
+    const int32_t *n_unique;           // [1]
+    float *h;                          // [(T*K + T*S)][I] f32 intermediate (GEMV path)
+    float *out;                        // [T][H]
+    int *err;                          // device error word
+};
+
+// Workspace carve-up (all offsets 256-B aligned).
+struct WsLayout {
+    size_t err;      // int error word (+ pad)
+    size_t logits;   // [T][E] f32
+    size_t ids;      // [T*K] i32
+    size_t w;        // [T*K] f32
+    size_t counts;   // [E] i32
+    size_t offsets;  // [E+1] i32
+    size_t perm;     // [T*K] i32
+    size_t unique;   // [E] i32
+    size_t nuniq;    // [1] i32
+    size_t h;        // [(T*K+T*S)][I] f32
+    size_t total;
+};
+
+WsLayout ws_layout(const coli_moe_config &c, int T);
+
+// Launchers (return cudaGetLastError()).
+cudaError_t launch_gate(const coli_moe_config &c, const float *Wr, const void *x, int T,
+                        float *logits, cudaStream_t st);
+cudaError_t launch_route(const coli_moe_config &c, const float *logits, const float *bias,
+                         int T, int32_t *ids, float *w, cudaStream_t st);
+cudaError_t launch_group(const coli_moe_config &c, const int32_t *ids, int T, int32_t *counts,
+                         int32_t *offsets, int32_t *perm, int32_t *unique, int32_t *n_unique,
+                         int *err, cudaStream_t st);
+cudaError_t launch_ffn_gemv(const FfnParams &p, cudaStream_t st);
+
+// Shape rules of the GEMV path (checked on the host before launch).
+bool gemv_shape_ok(int row_bytes);
+int gemv_max_tokens(const coli_moe_config &c);
+
+int device_sm_count();
+
+}  // namespace coli

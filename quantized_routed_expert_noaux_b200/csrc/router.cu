@@ -1,0 +1,381 @@
+// router.cu -- a1 gate, a2 noaux_tc routing and a3 batch-union grouping on sm_100a.
+//
+// The router of the colibri-strix README ("What's implemented": DeepSeek-V3-style sigmoid router
+// with noaux_tc and routed_scaling_factor) and the batch-union step of the same section.  The
+// gate sums exact double products in double and rounds once to float32; selection compares in
+// double, so the float32 logits and the chosen experts do not depend on summation order beyond
+// double rounding.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "internal.h"
+
+namespace coli {
+
+namespace {
+
+constexpr unsigned FULL = 0xffffffffu;
+
+__device__ __forceinline__ float bf16_to_f32(uint16_t b) {
+    return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+template <int ACT>
+__device__ __forceinline__ void load_x4(const void *x, size_t idx, float v[4]) {
+    if (ACT == COLI_ACT_F32) {
+        float4 f = __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(x) + idx));
+        v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+    } else {
+        uint2 u = __ldg(reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(x) + idx));
+        v[0] = __uint_as_float(u.x << 16);
+        v[1] = __uint_as_float(u.x & 0xffff0000u);
+        v[2] = __uint_as_float(u.y << 16);
+        v[3] = __uint_as_float(u.y & 0xffff0000u);
+    }
+}
+
+// ---------------------------------------------------------------- a1 gate, few tokens ------
+// One warp per expert row; every lane walks the row with float4 loads and keeps one double
+// accumulator per token of the current token block.
+template <int ACT, int TT>
+__global__ void __launch_bounds__(128) gate_rows_kernel(const float *__restrict__ Wr,
+                                                        const void *__restrict__ x, int T,
+                                                        int H, int E,
+                                                        float *__restrict__ logits) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int e = blockIdx.x * 4 + warp;
+    if (e >= E) return;
+    const float *wrow = Wr + static_cast<size_t>(e) * H;
+    for (int t0 = 0; t0 < T; t0 += TT) {
+        double acc[TT];
+#pragma unroll
+        for (int i = 0; i < TT; ++i) acc[i] = 0.0;
+        for (int h = lane * 4; h < H; h += 128) {
+            const float4 wv = __ldg(reinterpret_cast<const float4 *>(wrow + h));
+#pragma unroll
+            for (int i = 0; i < TT; ++i) {
+                if (t0 + i < T) {
+                    float xv[4];
+                    load_x4<ACT>(x, static_cast<size_t>(t0 + i) * H + h, xv);
+                    acc[i] = fma(static_cast<double>(wv.x), static_cast<double>(xv[0]), acc[i]);
+                    acc[i] = fma(static_cast<double>(wv.y), static_cast<double>(xv[1]), acc[i]);
+                    acc[i] = fma(static_cast<double>(wv.z), static_cast<double>(xv[2]), acc[i]);
+                    acc[i] = fma(static_cast<double>(wv.w), static_cast<double>(xv[3]), acc[i]);
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < TT; ++i) {
+            double v = acc[i];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
+            if (lane == 0 && t0 + i < T)
+                logits[static_cast<size_t>(t0 + i) * E + e] = static_cast<float>(v);
+        }
+    }
+}
+
+// ---------------------------------------------------------------- a1 gate, many tokens -----
+// Tiled double-precision product logits[T,E] = X[T,H] * Wr[E,H]^T.  CTA tile 64 tokens x 64
+// experts, K step 16, 256 threads holding 4x4 double accumulators each.
+constexpr int GT_M = 64, GT_N = 64, GT_K = 16;
+
+template <int ACT>
+__global__ void __launch_bounds__(256) gate_tiled_kernel(const float *__restrict__ Wr,
+                                                         const void *__restrict__ x, int T,
+                                                         int H, int E,
+                                                         float *__restrict__ logits) {
+    __shared__ double xs[GT_K][GT_M + 2];
+    __shared__ double ws[GT_K][GT_N + 2];
+    const int tid = threadIdx.x;
+    const int t0 = blockIdx.y * GT_M, e0 = blockIdx.x * GT_N;
+    const int tx = tid % 16, ty = tid / 16;  // 16 x 16 threads, 4 x 4 outputs each
+    double acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+
+    for (int k0 = 0; k0 < H; k0 += GT_K) {
+        // 64 rows x 16 columns of each operand: 1024 elements, 4 per thread
+        for (int idx = tid; idx < GT_M * GT_K; idx += 256) {
+            const int r = idx / GT_K, k = idx % GT_K;
+            const int t = t0 + r, e = e0 + r;
+            double xv = 0.0, wv = 0.0;
+            if (t < T) {
+                if (ACT == COLI_ACT_F32)
+                    xv = static_cast<double>(static_cast<const float *>(x)[static_cast<size_t>(t) * H + k0 + k]);
+                else
+                    xv = static_cast<double>(bf16_to_f32(static_cast<const uint16_t *>(x)[static_cast<size_t>(t) * H + k0 + k]));
+            }
+            if (e < E) wv = static_cast<double>(Wr[static_cast<size_t>(e) * H + k0 + k]);
+            xs[k][r] = xv;
+            ws[k][r] = wv;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < GT_K; ++k) {
+            double a[4], b[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[i] = xs[k][ty * 4 + i];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) b[j] = ws[k][tx * 4 + j];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fma(a[i], b[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int t = t0 + ty * 4 + i, e = e0 + tx * 4 + j;
+            if (t < T && e < E) logits[static_cast<size_t>(t) * E + e] = static_cast<float>(acc[i][j]);
+        }
+}
+
+// ---------------------------------------------------------------- a2 route -----------------
+__device__ __forceinline__ bool beats(double va, int ia, double vb, int ib) {
+    return va > vb || (va == vb && ia < ib);
+}
+
+// Warp-wide arg-max of (value desc, index asc); every lane ends with the winner.
+__device__ __forceinline__ void warp_argmax(double &v, int &i) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const double ov = __shfl_xor_sync(FULL, v, o);
+        const int oi = __shfl_xor_sync(FULL, i, o);
+        if (beats(ov, oi, v, i)) { v = ov; i = oi; }
+    }
+}
+
+// One warp per token.  Lane l holds experts e = l + 32 v, v < VPL.
+template <int VPL>
+__global__ void __launch_bounds__(128) route_kernel(const float *__restrict__ logits,
+                                                    const float *__restrict__ bias, int T,
+                                                    int E, int K, int G, int TG, double rsf,
+                                                    int32_t *__restrict__ ids,
+                                                    float *__restrict__ wout) {
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (t >= T) return;
+    const int gs = E / G;
+    double s[VPL], c[VPL];
+    bool taken[VPL];
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+        const int e = lane + 32 * v;
+        taken[v] = false;
+        if (e < E) {
+            const double l = static_cast<double>(logits[static_cast<size_t>(t) * E + e]);
+            s[v] = 1.0 / (1.0 + exp(-l));
+            c[v] = s[v] + static_cast<double>(bias[e]);
+        } else {
+            s[v] = 0.0;
+            c[v] = -INFINITY;
+        }
+    }
+    // group stage: kept-group bit mask (G <= 32)
+    uint32_t kept = (G >= 32) ? FULL : ((1u << G) - 1u);
+    if (G > 1 && TG < G) {
+        double my_score = -INFINITY;
+        for (int g = 0; g < G; ++g) {
+            double a1 = -INFINITY, a2 = -INFINITY;  // two largest values of this lane
+#pragma unroll
+            for (int v = 0; v < VPL; ++v) {
+                const int e = lane + 32 * v;
+                if (e < E && e / gs == g) {
+                    if (c[v] > a1) { a2 = a1; a1 = c[v]; }
+                    else if (c[v] > a2) { a2 = c[v]; }
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {  // merge pairs of sorted top-2 lists
+                const double b1 = __shfl_xor_sync(FULL, a1, o);
+                const double b2 = __shfl_xor_sync(FULL, a2, o);
+                const double n1 = fmax(a1, b1);
+                const double n2 = fmax(fmin(a1, b1), fmax(a2, b2));
+                a1 = n1; a2 = n2;
+            }
+            if (lane == g) my_score = a1 + a2;
+        }
+        kept = 0u;
+        for (int r = 0; r < TG; ++r) {
+            double v = (lane < G && !((kept >> lane) & 1u)) ? my_score : -INFINITY;
+            int i = (lane < G && !((kept >> lane) & 1u)) ? lane : 0x7fffffff;
+            warp_argmax(v, i);
+            kept |= 1u << i;
+        }
+    }
+    // expert stage: K arg-max picks; lane k keeps the unbiased score of slot k
+    double my_s = 0.0;
+    int my_id = -1;
+    for (int k = 0; k < K; ++k) {
+        double bv = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int v = 0; v < VPL; ++v) {
+            const int e = lane + 32 * v;
+            if (e < E && !taken[v] && ((kept >> (e / gs)) & 1u) && beats(c[v], e, bv, bi)) {
+                bv = c[v];
+                bi = e;
+            }
+        }
+        warp_argmax(bv, bi);
+        double sv = 0.0;
+#pragma unroll
+        for (int v = 0; v < VPL; ++v)
+            if (lane + 32 * v == bi) { taken[v] = true; sv = s[v]; }
+        const int owner = bi & 31;
+        sv = __shfl_sync(FULL, sv, owner);
+        if (lane == k) { my_s = sv; my_id = bi; }
+    }
+    double denom = 0.0;
+    for (int k = 0; k < K; ++k) denom += __shfl_sync(FULL, my_s, k);
+    if (lane < K) {
+        ids[static_cast<size_t>(t) * K + lane] = my_id;
+        wout[static_cast<size_t>(t) * K + lane] = static_cast<float>((my_s / denom) * rsf);
+    }
+}
+
+// ---------------------------------------------------------------- a3 group -----------------
+// One CTA.  Histogram with shared-memory integer atomics, exclusive scan, then a stable
+// placement pass over chunks of blockDim slots: warp peers by __match_any_sync give the rank
+// inside a warp, per-warp per-expert counts give the rank across warps.
+__global__ void __launch_bounds__(1024) group_kernel(const int32_t *__restrict__ ids, int n,
+                                                     int E, int32_t *__restrict__ counts,
+                                                     int32_t *__restrict__ offsets,
+                                                     int32_t *__restrict__ perm,
+                                                     int32_t *__restrict__ unique,
+                                                     int32_t *__restrict__ n_unique,
+                                                     int *__restrict__ err) {
+    extern __shared__ int sm[];
+    const int nw = blockDim.x >> 5;
+    int *cnt = sm;             // [E]
+    int *cursor = sm + E;      // [E]
+    int *wc = sm + 2 * E;      // [nw][E]
+    __shared__ int bad;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (tid == 0) bad = 0;
+    for (int e = tid; e < E; e += blockDim.x) cnt[e] = 0;
+    for (int i = tid; i < nw * E; i += blockDim.x) wc[i] = 0;
+    __syncthreads();
+    for (int s = tid; s < n; s += blockDim.x) {
+        const int id = ids[s];
+        if (id >= 0 && id < E) atomicAdd(&cnt[id], 1);
+        else bad = 1;
+    }
+    __syncthreads();
+    // exclusive scans of counts and of the non-empty flags, by warp 0 (E <= 1024)
+    if (warp == 0) {
+        const int per = (E + 31) / 32;
+        const int b = lane * per;
+        int sc = 0, su = 0;
+        for (int e = b; e < b + per && e < E; ++e) { sc += cnt[e]; su += cnt[e] > 0; }
+        int ic = sc, iu = su;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int a = __shfl_up_sync(FULL, ic, o), bb = __shfl_up_sync(FULL, iu, o);
+            if (lane >= o) { ic += a; iu += bb; }
+        }
+        int rc = ic - sc, ru = iu - su;
+        for (int e = b; e < b + per && e < E; ++e) {
+            offsets[e] = rc;
+            cursor[e] = rc;
+            counts[e] = cnt[e];
+            if (cnt[e] > 0) unique[ru++] = e;
+            rc += cnt[e];
+        }
+        if (lane == 31) {
+            offsets[E] = ic;
+            *n_unique = iu;
+            for (int e = iu; e < E; ++e) unique[e] = -1;
+        }
+    }
+    __syncthreads();
+    const unsigned lt = (1u << lane) - 1u;
+    for (int base = 0; base < n; base += blockDim.x) {
+        const int s = base + tid;
+        const int id = (s < n) ? ids[s] : -1;
+        const bool ok = id >= 0 && id < E;
+        const int key = ok ? id : -1 - lane;
+        const unsigned peers = __match_any_sync(FULL, key);
+        const int rank = __popc(peers & lt);
+        if (ok && rank == 0) wc[warp * E + id] = __popc(peers);
+        __syncthreads();
+        if (ok) {
+            int pos = cursor[id] + rank;
+            for (int w = 0; w < warp; ++w) pos += wc[w * E + id];
+            perm[pos] = s;
+        }
+        __syncthreads();
+        for (int e = tid; e < E; e += blockDim.x) {
+            int add = 0;
+            for (int w = 0; w < nw; ++w) { add += wc[w * E + e]; wc[w * E + e] = 0; }
+            cursor[e] += add;
+        }
+        __syncthreads();
+    }
+    // slots with a bad id are not placed; the tail of perm is marked
+    if (tid == 0 && bad) {
+        atomicOr(err, COLI_DEVERR_EXPERT_ID);
+        for (int p = offsets[E]; p < n; ++p) perm[p] = -1;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_gate(const coli_moe_config &c, const float *Wr, const void *x, int T,
+                        float *logits, cudaStream_t st) {
+    const int H = c.hidden, E = c.n_experts;
+    if (T <= 16) {
+        dim3 grid((E + 3) / 4);
+        if (c.act == COLI_ACT_F32)
+            gate_rows_kernel<COLI_ACT_F32, 8><<<grid, 128, 0, st>>>(Wr, x, T, H, E, logits);
+        else
+            gate_rows_kernel<COLI_ACT_BF16, 8><<<grid, 128, 0, st>>>(Wr, x, T, H, E, logits);
+    } else {
+        dim3 grid((E + GT_N - 1) / GT_N, (T + GT_M - 1) / GT_M);
+        if (c.act == COLI_ACT_F32)
+            gate_tiled_kernel<COLI_ACT_F32><<<grid, 256, 0, st>>>(Wr, x, T, H, E, logits);
+        else
+            gate_tiled_kernel<COLI_ACT_BF16><<<grid, 256, 0, st>>>(Wr, x, T, H, E, logits);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_route(const coli_moe_config &c, const float *logits, const float *bias,
+                         int T, int32_t *ids, float *w, cudaStream_t st) {
+    const int E = c.n_experts;
+    dim3 grid((T + 3) / 4);
+    const int vpl = (E + 31) / 32;
+#define COLI_ROUTE(V)                                                                        \
+    route_kernel<V><<<grid, 128, 0, st>>>(logits, bias, T, E, c.top_k, c.n_group,            \
+                                          c.topk_group, c.routed_scaling, ids, w)
+    if (vpl <= 1) COLI_ROUTE(1);
+    else if (vpl <= 2) COLI_ROUTE(2);
+    else if (vpl <= 4) COLI_ROUTE(4);
+    else if (vpl <= 8) COLI_ROUTE(8);
+    else if (vpl <= 16) COLI_ROUTE(16);
+    else COLI_ROUTE(32);
+#undef COLI_ROUTE
+    return cudaGetLastError();
+}
+
+cudaError_t launch_group(const coli_moe_config &c, const int32_t *ids, int T, int32_t *counts,
+                         int32_t *offsets, int32_t *perm, int32_t *unique, int32_t *n_unique,
+                         int *err, cudaStream_t st) {
+    const int n = T * c.top_k, E = c.n_experts;
+    const int threads = n <= 256 ? 256 : 1024;
+    const size_t smem = static_cast<size_t>(2 + threads / 32) * E * sizeof(int);
+    cudaError_t e = cudaFuncSetAttribute(group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    group_kernel<<<1, threads, smem, st>>>(ids, n, E, counts, offsets, perm, unique, n_unique, err);
+    return cudaGetLastError();
+}
+
+}  // namespace coli

@@ -1,0 +1,93 @@
+"""The C-ABI library loads, exports every entry point include/coli_moe.h declares, and
+validates arguments on the host before touching the GPU (CPU only: no compute calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "coli_moe.h")
+
+q = pytest.importorskip("quantized_routed_expert_noaux_b200")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(coli_moe_\w+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported():
+    syms = declared_symbols()
+    assert len(syms) >= 10
+    lib = ctypes.CDLL(q.LIB_PATH)
+    missing = [s for s in syms if not hasattr(lib, s)]
+    assert not missing, missing
+
+
+def test_binding_names_match_header():
+    for s in declared_symbols():
+        assert hasattr(q, s), f"binding lacks {s}"
+
+
+def test_status_strings():
+    assert q.coli_moe_status_str(0) == "ok"
+    assert "workspace" in q.coli_moe_status_str(7)
+    assert q.coli_moe_status_str(99) == "unknown status"
+
+
+@pytest.mark.parametrize("name", list(synth.WORKLOADS))
+def test_workload_configs_are_accepted(name):
+    wl = synth.WORKLOADS[name]
+    cfg = q.config_for(wl)
+    q.coli_moe_check_config(cfg)
+    assert q.coli_moe_record_bytes(wl.hidden, wl.inter, wl.fmt) == \
+        synth.record_layout(wl.hidden, wl.inter, wl.fmt)["bytes"]
+    assert q.coli_moe_workspace_size(cfg, 64) % 256 == 0
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("wfmt", 3, 1), ("act", 5, 1), ("n_group", 3, 2), ("topk_group", 9, 2),
+    ("top_k", 33, 4), ("top_k", 200, 2), ("hidden", 100, 2), ("n_shared", 2, 4), ("n_experts", 2048, 4), ("n_experts", 250, 2),
+    ("shared_inter", 1024, 4), ("routed_scaling", 0.0, 1),
+])
+def test_bad_config_rejected(field, value, status):
+    cfg = q.config_for(synth.WORKLOADS["glm_decode"])
+    setattr(cfg, field, value)
+    with pytest.raises(q.ColiError) as ei:
+        q.coli_moe_check_config(cfg)
+    assert ei.value.status == status
+
+
+def test_host_validation_before_launch():
+    cfg = q.config_for(synth.WORKLOADS["tiny"])
+    # T = 0 is a no-op and negative T a shape error: both decided without a device
+    q.coli_moe_gate(cfg, None, None, 0, None, stream=0)
+    with pytest.raises(q.ColiError) as ei:
+        q.coli_moe_gate(cfg, None, None, -1, None, stream=0)
+    assert ei.value.status == 2
+    with pytest.raises(q.ColiError) as ei:
+        q.coli_moe_gate(cfg, None, None, 3, None, stream=0)
+    assert ei.value.status == 1
+    # misaligned activation pointer
+    with pytest.raises(q.ColiError) as ei:
+        q.coli_moe_gate(cfg, 256, 258, 3, 512, stream=0)
+    assert ei.value.status == 3
+    # layer without a workspace
+    w = q.MoEWeights(256, 512, 1024, 51200, 2048)
+    rc = q.lib.coli_moe_layer(ctypes.byref(cfg), ctypes.byref(w), 4096, 2, 8192, None, None,
+                              None, 0, None)
+    assert rc == 7
+    # misaligned record stride
+    w.expert_stride = 51200 + 16
+    rc = q.lib.coli_moe_layer(ctypes.byref(cfg), ctypes.byref(w), 4096, 2, 8192, None, None,
+                              None, 0, None)
+    assert rc == 3
+    # stride smaller than a record
+    w.expert_stride = 256
+    rc = q.lib.coli_moe_layer(ctypes.byref(cfg), ctypes.byref(w), 4096, 2, 8192, None, None,
+                              None, 0, None)
+    assert rc == 2
