@@ -147,6 +147,29 @@ coli_status coli_moe_layer(const coli_moe_config *cfg, const coli_moe_weights *w
                            const void *x, int T, float *out, int32_t *topk_ids_out,
                            float *topk_w_out, void *ws, size_t ws_bytes, void *stream);
 
+/* Size of the static scratch array behind coli_moe_layer_noalloc (8 MiB per GPU). */
+#define COLI_MOE_STATIC_SCRATCH_BYTES (8u << 20)
+
+/* The whole layer, like coli_moe_layer, for callers that cannot allocate device memory: a
+ * plugin inside a serving engine whose GPU memory pool is fixed when the engine starts, or a
+ * real-time loop that must never pay for cudaMalloc's device-wide synchronisation.  The pages
+ * have no counterpart of this call; it exists for such callers only.
+ *   - Allocates nothing.  The caller passes x, out and the optional routing outputs as for
+ *     coli_moe_layer; every other byte the layer needs lives in one static device array of
+ *     COLI_MOE_STATIC_SCRATCH_BYTES that every GPU loading this library holds until exit.
+ *   - The first call on each device looks up that array's device address (cudaGetSymbolAddress
+ *     with the device current) and caches it; make that first call before any stream capture.
+ *   - Returns COLI_ERR_WORKSPACE when the call needs more scratch than the array holds
+ *     (coli_moe_workspace_size(cfg, T) > COLI_MOE_STATIC_SCRATCH_BYTES), before any launch.
+ *   - All calls on a device share the one array and it keeps the last call's contents; each call
+ *     clears the part that must start at zero.  Calls that overlap on the GPU (different streams
+ *     without ordering between them) race on the array and give wrong results: order them.
+ *   - The device error word lives inside the array and is not readable by the caller; device
+ *     anomalies still never trap. */
+coli_status coli_moe_layer_noalloc(const coli_moe_config *cfg, const coli_moe_weights *w,
+                                   const void *x, int T, float *out, int32_t *topk_ids_out,
+                                   float *topk_w_out, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -17,6 +17,7 @@ __all__ = [
     "coli_moe_status_str", "coli_moe_record_bytes", "coli_moe_check_config",
     "coli_moe_workspace_size", "coli_moe_clear_error", "coli_moe_error_word",
     "coli_moe_gate", "coli_moe_route", "coli_moe_group", "coli_moe_ffn", "coli_moe_layer",
+    "coli_moe_layer_noalloc", "STATIC_SCRATCH_BYTES",
     "config_for", "weights_for",
     "COLI_W_INT2", "COLI_W_INT4", "COLI_W_INT8", "COLI_ACT_F32", "COLI_ACT_BF16",
 ]
@@ -71,6 +72,8 @@ def _load():
     L.coli_moe_group.argtypes = [cfgp, P, I, P, P, P, P, P, P, S, P]
     L.coli_moe_ffn.argtypes = [cfgp, wp, P, I, P, P, P, P, P, P, P, S, P]
     L.coli_moe_layer.argtypes = [cfgp, wp, P, I, P, P, P, P, S, P]
+    L.coli_moe_layer_noalloc.argtypes = [cfgp, wp, P, I, P, P, P, P]
+    L.coli_moe_layer_noalloc.restype = I
     for name in ("coli_moe_record_bytes", "coli_moe_check_config", "coli_moe_workspace_size",
                  "coli_moe_clear_error", "coli_moe_error_word", "coli_moe_gate",
                  "coli_moe_route", "coli_moe_group", "coli_moe_ffn", "coli_moe_layer"):
@@ -165,6 +168,21 @@ def coli_moe_layer(cfg, weights: MoEWeights, x, T, out, topk_ids_out, topk_w_out
     _check("coli_moe_layer", lib.coli_moe_layer(
         C.byref(cfg), C.byref(weights), _p(x), T, _p(out), _p(topk_ids_out), _p(topk_w_out),
         _p(ws), _nbytes(ws), _stream(stream)))
+
+
+# Size of the static scratch array behind coli_moe_layer_noalloc (COLI_MOE_STATIC_SCRATCH_BYTES).
+STATIC_SCRATCH_BYTES = 8 << 20
+
+
+def coli_moe_layer_noalloc(cfg, weights: MoEWeights, x, T, out, topk_ids_out=None,
+                           topk_w_out=None, stream=None) -> None:
+    """The whole layer for callers that cannot allocate device memory (a plugin whose GPU memory
+    pool is fixed at start-up, a real-time loop that cannot afford cudaMalloc's synchronisation):
+    no workspace argument; the library's static per-GPU scratch array is used instead.  Calls on
+    one device share that array, so calls that overlap on the GPU must be ordered."""
+    _check("coli_moe_layer_noalloc", lib.coli_moe_layer_noalloc(
+        C.byref(cfg), C.byref(weights), _p(x), T, _p(out), _p(topk_ids_out), _p(topk_w_out),
+        _stream(stream)))
 
 
 def config_for(wl) -> MoEConfig:
