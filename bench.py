@@ -295,7 +295,7 @@ def gpu_arm(args, rank, world, dist):
         "e2e": {"value": round(world * K2 * T / (e2e_ms / 1e3), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(xs[0].numel() * xs[0].element_size()),
                 "d2h_bytes_per_step": int(out.numel() * 4)},
-        "gpu_launches": 5 * K,
+        "gpu_launches": q.coli_moe_layer_kernels(cfg, T) * K,
         "clocks": clk,
     }
     return res, (wl, T, layers, xs)

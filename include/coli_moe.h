@@ -60,6 +60,7 @@ typedef enum { COLI_ACT_F32 = 0, COLI_ACT_BF16 = 1 } coli_act;
 /* Device error word codes (bit flags, OR-ed together by the kernels). */
 #define COLI_DEVERR_EXPERT_ID 0x1   /* an expert id or unique-list entry outside [0, E) */
 #define COLI_DEVERR_GROUPING 0x2    /* offsets/perm inconsistent (slot outside [0, T*K)) */
+#define COLI_DEVERR_TIMEOUT 0x4     /* a bounded device-side wait ran out (the call's output is invalid) */
 
 typedef struct {
     int hidden;             /* H */
@@ -94,10 +95,17 @@ coli_status coli_moe_check_config(const coli_moe_config *cfg);
 
 /* Workspace bytes that coli_moe_layer / coli_moe_ffn / coli_moe_group need for up to
  * max_tokens tokens.  The workspace must be 256-byte aligned and is owned by the caller; calls
- * that share one workspace must be ordered on the GPU (same stream or events).  Host only. */
+ * that share one workspace must be ordered on the GPU (same stream or events).  Its first 256
+ * bytes (error word and the counters of the fused decode path) must be zero before its first
+ * use: call coli_moe_clear_error once after allocating it (and after a call that reported
+ * COLI_DEVERR_TIMEOUT).  Complete calls leave the counters zero.  Host only. */
 coli_status coli_moe_workspace_size(const coli_moe_config *cfg, int max_tokens, size_t *bytes);
 
-/* Clears the workspace's device error word (asynchronous on stream). */
+/* Number of kernels coli_moe_layer launches for T tokens with this configuration (2 on the fused
+ * decode path: router kernel + persistent FFN kernel; 5 otherwise).  Host only. */
+coli_status coli_moe_layer_kernels(const coli_moe_config *cfg, int T, int *n_kernels);
+
+/* Zeroes the workspace header: the device error word and the counters (asynchronous). */
 coli_status coli_moe_clear_error(void *ws, void *stream);
 
 /* Synchronises `stream` and returns the workspace's device error word in *code (0 = clean). */

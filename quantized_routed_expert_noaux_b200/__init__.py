@@ -17,7 +17,7 @@ __all__ = [
     "coli_moe_status_str", "coli_moe_record_bytes", "coli_moe_check_config",
     "coli_moe_workspace_size", "coli_moe_clear_error", "coli_moe_error_word",
     "coli_moe_gate", "coli_moe_route", "coli_moe_group", "coli_moe_ffn", "coli_moe_layer",
-    "coli_moe_layer_noalloc", "STATIC_SCRATCH_BYTES",
+    "coli_moe_layer_noalloc", "STATIC_SCRATCH_BYTES", "coli_moe_layer_kernels",
     "config_for", "weights_for",
     "COLI_W_INT2", "COLI_W_INT4", "COLI_W_INT8", "COLI_ACT_F32", "COLI_ACT_BF16",
 ]
@@ -30,7 +30,7 @@ DEVERR_EXPERT_ID, DEVERR_GROUPING = 0x1, 0x2
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m quantized_routed_expert_noaux_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python quantized_routed_expert_noaux_b200/build.py` "
         "(there is no CPU fallback for this layer)")
 
 
@@ -73,6 +73,8 @@ def _load():
     L.coli_moe_ffn.argtypes = [cfgp, wp, P, I, P, P, P, P, P, P, P, S, P]
     L.coli_moe_layer.argtypes = [cfgp, wp, P, I, P, P, P, P, S, P]
     L.coli_moe_layer_noalloc.argtypes = [cfgp, wp, P, I, P, P, P, P]
+    L.coli_moe_layer_kernels.argtypes = [cfgp, I, C.POINTER(I)]
+    L.coli_moe_layer_kernels.restype = I
     L.coli_moe_layer_noalloc.restype = I
     for name in ("coli_moe_record_bytes", "coli_moe_check_config", "coli_moe_workspace_size",
                  "coli_moe_clear_error", "coli_moe_error_word", "coli_moe_gate",
@@ -137,6 +139,12 @@ def coli_moe_error_word(ws, stream=None) -> int:
     v = C.c_int()
     _check("coli_moe_error_word", lib.coli_moe_error_word(_p(ws), _stream(stream), C.byref(v)))
     return v.value
+
+
+def coli_moe_layer_kernels(cfg, T) -> int:
+    n = C.c_int()
+    _check("coli_moe_layer_kernels", lib.coli_moe_layer_kernels(C.byref(cfg), T, C.byref(n)))
+    return n.value
 
 
 def coli_moe_gate(cfg, router_w, x, T, logits, stream=None) -> None:

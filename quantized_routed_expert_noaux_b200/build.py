@@ -1,6 +1,8 @@
 """Build libcoli_moe.so in-tree with nvcc for sm_100a (B200).
 
-    python -m quantized_routed_expert_noaux_b200.build [--force] [--verbose]
+    python quantized_routed_expert_noaux_b200/build.py [--force] [--verbose]
+
+(run it by path: importing the package loads the library this script builds)
 
 Each .cu under csrc/ is compiled to an object with
 `-gencode arch=compute_100a,code=sm_100a -O3 -lineinfo`, then linked into one shared library

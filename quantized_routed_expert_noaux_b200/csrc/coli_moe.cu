@@ -41,7 +41,7 @@ WsLayout ws_layout(const coli_moe_config &c, int T) {
     const size_t n = static_cast<size_t>(T) * c.top_k;
     const size_t E = static_cast<size_t>(c.n_experts);
     size_t o = 0;
-    L.err = o;      o = align256(o + 256);
+    L.err = o;      o = align256(o + WS_HEADER);
     L.logits = o;   o = align256(o + static_cast<size_t>(T) * E * 4);
     L.ids = o;      o = align256(o + n * 4);
     L.w = o;        o = align256(o + n * 4);
@@ -119,7 +119,7 @@ coli_status coli_moe_workspace_size(const coli_moe_config *c, int max_tokens, si
 
 coli_status coli_moe_clear_error(void *ws, void *stream) {
     if (!ws || !aligned(ws, 256)) return COLI_ERR_WORKSPACE;
-    return from_cuda(cudaMemsetAsync(ws, 0, sizeof(int), static_cast<cudaStream_t>(stream)));
+    return from_cuda(cudaMemsetAsync(ws, 0, WS_HEADER, static_cast<cudaStream_t>(stream)));
 }
 
 coli_status coli_moe_error_word(void *ws, void *stream, int *code) {
@@ -130,6 +130,16 @@ coli_status coli_moe_error_word(void *ws, void *stream, int *code) {
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return COLI_ERR_CUDA;
     *code = v;
+    return COLI_OK;
+}
+
+coli_status coli_moe_layer_kernels(const coli_moe_config *c, int T, int *n_kernels) {
+    if (!n_kernels) return COLI_ERR_INVALID_ARG;
+    coli_status s = coli_moe_check_config(c);
+    if (s != COLI_OK) return s;
+    if (T < 0) return COLI_ERR_SHAPE;
+    DecodePlan pl;
+    *n_kernels = T == 0 ? 0 : (decode_plan(*c, T, &pl) ? 2 : 5);
     return COLI_OK;
 }
 
@@ -205,7 +215,24 @@ static FfnParams make_params(const coli_moe_config *c, const coli_moe_weights *w
     return p;
 }
 
-static coli_status run_ffn(const FfnParams &p, cudaStream_t st) {
+static DecodeParams make_decode(const coli_moe_config *c, const FfnParams &f, char *base) {
+    DecodeParams d = {};
+    d.f = f;
+    d.rsf = c->routed_scaling;
+    d.G = c->n_group;
+    d.TG = c->topk_group;
+    d.gbar = reinterpret_cast<unsigned *>(base + WS_GBAR);
+    d.gdep = reinterpret_cast<unsigned *>(base + WS_GDEP);
+    d.route_cnt = reinterpret_cast<unsigned *>(base + WS_ROUTE_CNT);
+    d.tok_cnt = reinterpret_cast<unsigned *>(base + WS_TOK_CNT);
+    return d;
+}
+
+// The expert half for a given routing: the fused decode kernel when the shape allows it, else
+// the general GEMV kernels.
+static coli_status run_ffn(const coli_moe_config *c, const FfnParams &p, char *base, cudaStream_t st) {
+    DecodePlan pl;
+    if (decode_plan(*c, p.T, &pl)) return from_cuda(launch_ffn_decode(make_decode(c, p, base), pl, st, false));
     return from_cuda(launch_ffn_gemv(p, st));
 }
 
@@ -227,7 +254,7 @@ coli_status coli_moe_ffn(const coli_moe_config *c, const coli_moe_weights *w, co
     char *base = static_cast<char *>(ws);
     FfnParams p = make_params(c, w, x, T, topk_w, offsets, perm, unique_ids, n_unique, out,
                               reinterpret_cast<float *>(base + L.h), reinterpret_cast<int *>(base + L.err));
-    return run_ffn(p, static_cast<cudaStream_t>(stream));
+    return run_ffn(c, p, base, static_cast<cudaStream_t>(stream));
 }
 
 coli_status coli_moe_layer(const coli_moe_config *c, const coli_moe_weights *w, const void *x, int T,
@@ -258,13 +285,31 @@ coli_status coli_moe_layer(const coli_moe_config *c, const coli_moe_weights *w, 
     int32_t *nu = reinterpret_cast<int32_t *>(base + L.nuniq);
     int *err = reinterpret_cast<int *>(base + L.err);
 
+    FfnParams p = make_params(c, w, x, T, wts, offsets, perm, uniq, nu, out,
+                              reinterpret_cast<float *>(base + L.h), err);
+    DecodePlan pl;
+    if (decode_plan(*c, T, &pl)) {
+        // fused decode path: router kernel, then the FFN kernel as its programmatic dependent
+        DecodeParams d = make_decode(c, p, base);
+        d.Wr = w->router_w;
+        d.bias = w->router_bias;
+        d.logits = logits;
+        d.ids = ids;
+        d.wts = wts;
+        d.f_counts = counts;
+        d.f_offsets = offsets;
+        d.f_perm = perm;
+        d.f_unique = uniq;
+        d.f_nuniq = nu;
+        cudaError_t e = launch_router_decode(d, st);
+        if (e == cudaSuccess) e = launch_ffn_decode(d, pl, st, true);
+        return from_cuda(e);
+    }
     cudaError_t e = launch_gate(*c, w->router_w, x, T, logits, st);
     if (e == cudaSuccess) e = launch_route(*c, logits, w->router_bias, T, ids, wts, st);
     if (e == cudaSuccess) e = launch_group(*c, ids, T, counts, offsets, perm, uniq, nu, err, st);
     if (e != cudaSuccess) return COLI_ERR_CUDA;
-    FfnParams p = make_params(c, w, x, T, wts, offsets, perm, uniq, nu, out,
-                              reinterpret_cast<float *>(base + L.h), err);
-    return run_ffn(p, st);
+    return run_ffn(c, p, base, st);
 }
 
 }  // extern "C"

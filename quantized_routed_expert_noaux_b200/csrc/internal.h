@@ -30,6 +30,43 @@ struct FfnParams {
     int *err;                          // device error word
 };
 
+// Workspace header (first 256 bytes): error word, then counters of the fused decode path.
+// All must be zero before the first call on a workspace (coli_moe_clear_error zeroes them);
+// the kernels leave them zero after every complete call.
+constexpr int WS_ERR = 0, WS_GBAR = 64, WS_GDEP = 96, WS_ROUTE_CNT = 128, WS_TOK_CNT = 160;  // 8 token words
+constexpr int WS_HEADER = 256;
+
+// Shared-memory plan of the fused decode FFN kernel (decode.cu).
+struct DecodePlan {
+    int grid, Lh, Li, P1, P2, R1, S, SB;
+    int st_up, st_sg, st_su, st_sd;       // byte offsets inside a ring stage
+    size_t off_route, off_x, off_xs, off_xc, off_red, off_ring, smem;
+    int red1_len;
+};
+
+// Parameters of the fused decode path (router kernel K1 and FFN kernel K2).
+struct DecodeParams {
+    FfnParams f;
+    // K1: gate + route + group
+    const float *Wr, *bias;
+    float *logits;
+    int32_t *ids;
+    float *wts;
+    int32_t *f_counts, *f_offsets, *f_perm, *f_unique, *f_nuniq;
+    double rsf;
+    int G, TG;
+    unsigned *tok_cnt, *route_cnt, *gbar, *gdep;
+    // K2 plan (copied from DecodePlan)
+    int grid, Lh, Li, P1, P2, R1, S, SB;
+    int st_up, st_sg, st_su, st_sd;
+    size_t off_route, off_x, off_xs, off_xc, off_red, off_ring;
+    int red1_len;
+};
+
+bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan);
+cudaError_t launch_router_decode(DecodeParams p, cudaStream_t st);
+cudaError_t launch_ffn_decode(DecodeParams p, const DecodePlan &pl, cudaStream_t st, bool pdl);
+
 // Workspace carve-up (all offsets 256-B aligned).
 struct WsLayout {
     size_t err;      // int error word (+ pad)

@@ -174,6 +174,8 @@ def _gpu_group(cfg, ids_dev, T, E, ws):
 
 @pytest.mark.parametrize("name,T,routing", [("tiny", 8, "oracle"), ("tiny", 5, "one_expert"),
                                             ("olmoe", 32, "oracle"), ("glm_decode", 4, "oracle"),
+                                            ("glm_decode", 4, "one_expert"),
+                                            ("glm_decode", 1, "oracle"),
                                             ("glm_decode", 16, "one_expert")])
 def test_ffn_matches_oracle(name, T, routing):
     L = layer_for(name)
@@ -227,7 +229,9 @@ def test_ffn_flags_bad_unique_list():
 # --------------------------------------------------------------------------- whole layer --
 
 @pytest.mark.parametrize("name,T", [("tiny", 8), ("tiny", 1), ("tiny", 37), ("olmoe", 1),
-                                    ("olmoe", 32), ("glm_decode", 1), ("glm_decode", 4)])
+                                    ("olmoe", 32), ("olmoe", 3), ("glm_decode", 1),
+                                    ("glm_decode", 2), ("glm_decode", 3), ("glm_decode", 4),
+                                    ("glm_decode", 5)])
 def test_layer_matches_oracle(name, T):
     L = layer_for(name)
     x = synth.make_activations(L.wl, T, device="cuda", step=T)
@@ -266,12 +270,25 @@ def test_batch_union_equals_per_token_bitwise(name, T):
         np.testing.assert_array_equal(o1[0], out[t])
 
 
-def test_layer_deterministic():
+@pytest.mark.parametrize("T", [1, 4])
+def test_layer_deterministic_and_repeatable(T):
+    """Repeated calls on one workspace give identical bits (the fused path's counters return to
+    zero after every call) and leave the error word clean."""
     L = layer_for("glm_decode")
-    x = synth.make_activations(L.wl, 4, device="cuda", step=5)
-    a = run_layer(L, x, 4)[0]
-    b = run_layer(L, x, 4)[0]
-    np.testing.assert_array_equal(a, b)
+    cfg = q.config_for(L.wl)
+    ws = workspace(cfg, T)
+    q.coli_moe_clear_error(ws)
+    outs = []
+    for rep in range(3):
+        x = synth.make_activations(L.wl, T, device="cuda", step=5)
+        out = torch.empty(T, L.wl.hidden, dtype=torch.float32, device="cuda")
+        q.coli_moe_layer(cfg, L.weights(), x, T, out, None, None, ws)
+        outs.append(out.cpu().numpy())
+    assert q.coli_moe_error_word(ws) == 0
+    hdr = ws[:256].view(torch.int32).cpu().numpy()
+    assert (hdr == 0).all(), hdr
+    np.testing.assert_array_equal(outs[0], outs[1])
+    np.testing.assert_array_equal(outs[0], outs[2])
 
 
 def test_layer_zero_tokens_is_noop():
