@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--layers", type=int, default=0, help="resident layers rotated (default 4)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--profile", action="store_true",
+                    help="only run warmup+steps layer calls (for ncu captures); prints no JSON")
     return ap.parse_args()
 
 
@@ -152,6 +154,15 @@ def gpu_arm(args, rank, world, dist):
     def step(i, ids=None):
         ex, sh, Wr, b, wts = layers[i % n_layers]
         q.coli_moe_layer(cfg, wts, xs[i % n_x], T, out, ids, None, ws, st.cuda_stream)
+
+    if args.profile:
+        q.coli_moe_clear_error(ws)
+        for i in range(W + K):
+            step(i)
+        torch.cuda.synchronize()
+        if q.coli_moe_error_word(ws):
+            raise RuntimeError("device error word set")
+        return None, None
 
     clocks = Clocks(dev.index if dev.index is not None else 0)
     q.coli_moe_clear_error(ws)
@@ -409,6 +420,8 @@ def main():
         dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
         dist = dist_mod
     res, ctx = gpu_arm(args, rank, world, dist)
+    if res is None:
+        return
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         wl, T, layers, xs = ctx
         n, sec, thr = _oracle_sample(wl, T, xs[:8], layers[0][:4], args.cpu_seconds, None)

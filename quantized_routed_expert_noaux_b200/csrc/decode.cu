@@ -33,10 +33,10 @@ namespace coli {
 namespace {
 
 constexpr unsigned FULL = 0xffffffffu;
-constexpr int NCW = 12;              // consumer warps
+constexpr int NCW = 16;              // consumer warps
 constexpr int NC = NCW * 32;         // consumer threads
 constexpr int NT = NC + 32;          // + producer warp
-constexpr int RPT1 = 3;              // phase-1 rows per thread per stage
+constexpr int PS1 = 8;               // (gate, up) row pairs per phase-1 stage
 constexpr int RPT2MAX = 8;           // phase-2 rows per thread over the whole CTA row range
 constexpr int CONS_BAR = 1;          // named barrier id of the consumer warps
 constexpr long long WAIT_CYCLES = 4000000000LL;  // ~2 s at 1.9 GHz: bound of every spin-wait
@@ -307,25 +307,40 @@ __global__ void __launch_bounds__(256) router_decode_kernel(DecodeParams p) {
     const int half = threadIdx.x >> 7, l = threadIdx.x & 127;
     const int e = blockIdx.x * 2 + half;
     __shared__ double red[8];
-    // a1: one Wr row per 128 threads, products and sums in double
+    // a1: one Wr row per 128 threads, products and sums in double.  Loads are issued in groups
+    // of GB so that a thread's whole slice of the row is in flight at once (H <= GB * 512 * 2).
+    constexpr int GB = 6;
     double acc = 0.0;
     if (e < E) {
         const float *wrow = p.Wr + static_cast<size_t>(e) * H;
-        for (int h0 = l * 4; h0 < H; h0 += 512) {
-            const float4 wv = __ldg(reinterpret_cast<const float4 *>(wrow + h0));
-            float xv[4];
-            if (p.f.act == COLI_ACT_F32) {
-                const float4 f = __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(p.f.x) + static_cast<size_t>(t) * H + h0));
-                xv[0] = f.x; xv[1] = f.y; xv[2] = f.z; xv[3] = f.w;
-            } else {
-                const uint2 u = __ldg(reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(p.f.x) + static_cast<size_t>(t) * H + h0));
-                xv[0] = __uint_as_float(u.x << 16); xv[1] = __uint_as_float(u.x & 0xffff0000u);
-                xv[2] = __uint_as_float(u.y << 16); xv[3] = __uint_as_float(u.y & 0xffff0000u);
+        for (int base = l * 4; base < H; base += GB * 512) {
+            float4 wv[GB];
+            float xv[GB][4];
+#pragma unroll
+            for (int g = 0; g < GB; ++g) {
+                const int h0 = base + g * 512;
+                if (h0 < H) {
+                    wv[g] = __ldg(reinterpret_cast<const float4 *>(wrow + h0));
+                    if (p.f.act == COLI_ACT_F32) {
+                        const float4 f4 = __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(p.f.x) + static_cast<size_t>(t) * H + h0));
+                        xv[g][0] = f4.x; xv[g][1] = f4.y; xv[g][2] = f4.z; xv[g][3] = f4.w;
+                    } else {
+                        const uint2 u = __ldg(reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(p.f.x) + static_cast<size_t>(t) * H + h0));
+                        xv[g][0] = __uint_as_float(u.x << 16); xv[g][1] = __uint_as_float(u.x & 0xffff0000u);
+                        xv[g][2] = __uint_as_float(u.y << 16); xv[g][3] = __uint_as_float(u.y & 0xffff0000u);
+                    }
+                } else {
+                    wv[g] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    xv[g][0] = xv[g][1] = xv[g][2] = xv[g][3] = 0.f;
+                }
             }
-            acc = fma(static_cast<double>(wv.x), static_cast<double>(xv[0]), acc);
-            acc = fma(static_cast<double>(wv.y), static_cast<double>(xv[1]), acc);
-            acc = fma(static_cast<double>(wv.z), static_cast<double>(xv[2]), acc);
-            acc = fma(static_cast<double>(wv.w), static_cast<double>(xv[3]), acc);
+#pragma unroll
+            for (int g = 0; g < GB; ++g) {
+                acc = fma(static_cast<double>(wv[g].x), static_cast<double>(xv[g][0]), acc);
+                acc = fma(static_cast<double>(wv[g].y), static_cast<double>(xv[g][1]), acc);
+                acc = fma(static_cast<double>(wv[g].z), static_cast<double>(xv[g][2]), acc);
+                acc = fma(static_cast<double>(wv[g].w), static_cast<double>(xv[g][3]), acc);
+            }
         }
     }
 #pragma unroll
@@ -378,12 +393,18 @@ __global__ void __launch_bounds__(256) router_decode_kernel(DecodeParams p) {
 }
 
 // ------------------------------------------------------------------------- K2 FFN ----------
-struct Stage1 { int we, r0, n; };
-
+// Phase 1: a stage holds PS (gate row, up row) pairs of one expert; consumer warp w works on pair
+// w % PS of the stages whose sequence number is w / PS modulo NCW / PS, reduces its rows with
+// shuffles and writes h itself.  Every consumer warp waits on every stage's full barrier and
+// arrives on its empty barrier (count NCW), so a stage is refilled only after all its readers
+// are done.  Phase 2: a stage holds the CTA's whole block of down rows of one expert; consumer
+// thread (p2, c2) owns chunk c2 of rows p2 + P2*m and keeps per-(row, token) partial sums in
+// registers across experts; one cross-lane reduction at the end.
 template <int FMT, int TMAX>
-__global__ void __maxnreg__(128) ffn_decode_kernel(DecodeParams p) {
+__global__ void __maxnreg__(112) ffn_decode_kernel(DecodeParams p) {
     constexpr int CPC = Fmt<FMT>::CPC;       // codes per 16-byte chunk
     constexpr int XW = CPC / 2;              // int32 words of 16-bit activations per chunk
+    constexpr int XV = XW / 4;               // int4 vectors per chunk
     extern __shared__ __align__(1024) unsigned char sm[];
     const FfnParams &f = p.f;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -391,21 +412,21 @@ __global__ void __maxnreg__(128) ffn_decode_kernel(DecodeParams p) {
     const int S = p.S;
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm);          // full[S], empty[S]
     int *rt = reinterpret_cast<int *>(sm + p.off_route);         // routing cache
-    int *xq = reinterpret_cast<int *>(sm + p.off_x);              // [T][Lh][XW]
+    int4 *xq = reinterpret_cast<int4 *>(sm + p.off_x);            // [T][XV][Lh] (transposed)
     float *xs = reinterpret_cast<float *>(sm + p.off_xs);         // [T][Lh] scale
     int *xc = reinterpret_cast<int *>(sm + p.off_xc);             // [T][Lh] correction
-    float *red1 = reinterpret_cast<float *>(sm + p.off_red);      // phase-1 partials (2 buffers)
-    float *hb = reinterpret_cast<float *>(sm + p.off_x);          // phase-2 h buffer (aliases x)
+    float *red2 = reinterpret_cast<float *>(sm + p.off_red);      // phase-2 partials
+    float4 *hb = reinterpret_cast<float4 *>(sm + p.off_x);        // phase-2 h (aliases x)
     unsigned char *ring = sm + p.off_ring;
     const uint32_t bar0 = smem_u32(bars);
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
+    const int Lh = p.Lh, Li = p.Li;
+    const int PS = p.R1;                     // pairs per phase-1 stage
 
-    // row ranges of this CTA
     const int i_lo = static_cast<int>(static_cast<long>(f.I) * b / G), i_hi = static_cast<int>(static_cast<long>(f.I) * (b + 1) / G);
     const int j_lo = static_cast<int>(static_cast<long>(f.H) * b / G), j_hi = static_cast<int>(static_cast<long>(f.H) * (b + 1) / G);
-    const int R1 = p.R1;
-    const int n1 = (i_hi - i_lo + R1 - 1) / R1;  // phase-1 stages per expert
+    const int n1 = (i_hi - i_lo + PS - 1) / PS;  // phase-1 stages per expert
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -416,45 +437,35 @@ __global__ void __maxnreg__(128) ffn_decode_kernel(DecodeParams p) {
     }
     __syncthreads();
 
-    // record of work-expert we: shared first (needs no routing), then unique[we - S]
-    auto record = [&](int we, int U, const int *uniq) -> const uint8_t * {
-        if (we < f.S) return f.shared;
-        const int e = uniq[we - f.S];
-        return (e >= 0 && e < f.E) ? f.experts + static_cast<size_t>(e) * f.stride : nullptr;
-    };
-
     if (warp == 0) {
         // ---------------------------------------------------------------- producer --------
         if (lane != 0) return;
         const uint64_t pol = evict_first_policy();
-        int seq = 0;
-        int U = 0;
+        int seq = 0, U = 0;
         int uniq[32];
-        bool have_routing = false;
-        bool ok = true;
-        auto get_routing = [&]() {
-            if (have_routing) return;
-            grid_dep_wait();
-            U = __ldcg(f.n_unique);
-            U = U < 0 ? 0 : (U > 32 ? 32 : U);
-            for (int u = 0; u < U; ++u) uniq[u] = __ldcg(f.unique + u);
-            have_routing = true;
+        bool have_routing = false, ok = true;
+        auto record = [&](int we) -> const uint8_t * {
+            if (we < f.S) return f.shared;
+            const int e = uniq[we - f.S];
+            return (e >= 0 && e < f.E) ? f.experts + static_cast<size_t>(e) * f.stride : nullptr;
         };
-        // phase 1
         for (int we = 0; ok; ++we) {
-            if (we >= f.S) get_routing();
-            if (we >= f.S + U && have_routing) break;
-            const uint8_t *rec = record(we, U, uniq);
+            if (we >= f.S && !have_routing) {
+                grid_dep_wait();
+                U = __ldcg(f.n_unique);
+                U = U < 0 ? 0 : (U > 32 ? 32 : U);
+                for (int u = 0; u < U; ++u) uniq[u] = __ldcg(f.unique + u);
+                have_routing = true;
+            }
+            if (have_routing && we >= f.S + U) break;
+            const uint8_t *rec = record(we);
             for (int k = 0; k < n1 && ok; ++k, ++seq) {
                 const int s = seq % S;
                 const uint32_t par = (seq / S) & 1;
                 if (!mbar_wait(empty_bar(s), par ^ 1)) { ok = false; break; }
-                const int r0 = i_lo + k * R1, n = min(R1, i_hi - r0);
+                const int r0 = i_lo + k * PS, n = min(PS, i_hi - r0);
                 const uint32_t dst = smem_u32(ring + static_cast<size_t>(s) * p.SB);
-                if (rec == nullptr) {  // bad unique entry: complete the phase without data
-                    mbar_arrive(full_bar(s));
-                    continue;
-                }
+                if (rec == nullptr) { mbar_arrive(full_bar(s)); continue; }
                 const int a0 = r0 & ~3, a1 = (r0 + n + 3) & ~3;
                 const uint32_t bytes = 2u * n * static_cast<uint32_t>(f.rb_h) + 2u * 4u * (a1 - a0);
                 mbar_expect_tx(full_bar(s), bytes);
@@ -464,12 +475,10 @@ __global__ void __maxnreg__(128) ffn_decode_kernel(DecodeParams p) {
                 bulk_g2s(dst + p.st_su, rec + f.off_su + 4 * a0, 4 * (a1 - a0), full_bar(s), pol);
             }
         }
-        // phase 2: one stage per expert (the CTA's whole row block)
-        for (int we = 0; ok && we < f.S + U; ++we) {
-            const uint8_t *rec = record(we, U, uniq);
+        for (int we = 0; ok && we < f.S + U; ++we, ++seq) {
+            const uint8_t *rec = record(we);
             const int s = seq % S;
             const uint32_t par = (seq / S) & 1;
-            ++seq;
             if (!mbar_wait(empty_bar(s), par ^ 1)) { ok = false; break; }
             const uint32_t dst = smem_u32(ring + static_cast<size_t>(s) * p.SB);
             if (rec == nullptr) { mbar_arrive(full_bar(s)); continue; }
@@ -486,70 +495,81 @@ __global__ void __maxnreg__(128) ffn_decode_kernel(DecodeParams p) {
 
     // -------------------------------------------------------------------- consumers --------
     const int ct = threadIdx.x - 32;
-    const int cw = ct >> 5;  // consumer warp
+    const int cw = ct >> 5;
     const int T = f.T;
-    const int Lh = p.Lh, Li = p.Li;
     bool ok = true;
 
-    // activations -> 16-bit block fixed point per (token, chunk) (see file comment)
+    // activations -> 16-bit block fixed point per (token, chunk), transposed for conflict-free
+    // reads: int4 vector v of chunk c of token t at xq[(t * XV + v) * Lh + c]
     for (int idx = ct; idx < T * Lh; idx += NC) {
         const int t = idx / Lh, c = idx % Lh;
-        const size_t base = static_cast<size_t>(t) * f.H + static_cast<size_t>(c) * CPC;
+        const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(f.x) +
+                                                          static_cast<size_t>(t) * f.H + static_cast<size_t>(c) * CPC);
+        uint32_t raw[CPC / 2];  // bf16 pairs
+#pragma unroll
+        for (int i = 0; i < CPC / 8; ++i) {
+            const uint4 v = __ldg(src + i);
+            raw[4 * i] = v.x; raw[4 * i + 1] = v.y; raw[4 * i + 2] = v.z; raw[4 * i + 3] = v.w;
+        }
         auto xval = [&](int j) -> float {
-            if (f.act == COLI_ACT_F32) return __ldg(static_cast<const float *>(f.x) + base + j);
-            return bf16f(__ldg(static_cast<const uint16_t *>(f.x) + base + j));
+            const uint32_t w2 = raw[j >> 1];
+            return __uint_as_float((j & 1) ? (w2 & 0xffff0000u) : (w2 << 16));
         };
         float mx = 0.f;
+#pragma unroll
         for (int j = 0; j < CPC; ++j) mx = fmaxf(mx, fabsf(xval(j)));
         int ex = 0;
         if (mx > 0.f) frexpf(mx, &ex);            // mx < 2^ex
         const float up = ldexpf(1.0f, 15 - ex);    // |x * up| < 2^15
         auto mq = [&](int j) -> int { return max(-32767, min(32767, __float2int_rn(xval(j) * up))); };
         auto pk = [](int a, int bb) { return static_cast<int>((static_cast<uint32_t>(a) & 0xffffu) | (static_cast<uint32_t>(bb) << 16)); };
-        int *dst = xq + static_cast<size_t>(idx) * XW;
+        int w[XW];
         int sum = 0;
         if (FMT == 4) {
+#pragma unroll
             for (int i = 0; i < 4; ++i) {
                 int m[8];
 #pragma unroll
                 for (int j = 0; j < 8; ++j) { m[j] = mq(8 * i + j); sum += m[j]; }
-                dst[4 * i + 0] = pk(m[0], m[2]);
-                dst[4 * i + 1] = pk(m[4], m[6]);
-                dst[4 * i + 2] = pk(m[1], m[3]);
-                dst[4 * i + 3] = pk(m[5], m[7]);
+                w[4 * i + 0] = pk(m[0], m[2]);
+                w[4 * i + 1] = pk(m[4], m[6]);
+                w[4 * i + 2] = pk(m[1], m[3]);
+                w[4 * i + 3] = pk(m[5], m[7]);
             }
             xc[idx] = 8 * sum;
         } else if (FMT == 8) {
-            for (int i = 0; i < 8; ++i) dst[i] = pk(mq(2 * i), mq(2 * i + 1));
+#pragma unroll
+            for (int i = 0; i < 8; ++i) w[i] = pk(mq(2 * i), mq(2 * i + 1));
             xc[idx] = 0;
         } else {
+#pragma unroll
             for (int i = 0; i < 4; ++i) {
                 int m[16];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) { m[j] = mq(16 * i + j); sum += m[j]; }
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    dst[8 * i + 2 * k + 0] = pk(m[k], m[4 + k]);
-                    dst[8 * i + 2 * k + 1] = pk(m[8 + k], m[12 + k]);
+                    w[8 * i + 2 * k + 0] = pk(m[k], m[4 + k]);
+                    w[8 * i + 2 * k + 1] = pk(m[8 + k], m[12 + k]);
                 }
             }
             xc[idx] = 2 * sum;
         }
+#pragma unroll
+        for (int v = 0; v < XV; ++v)
+            xq[(static_cast<size_t>(t) * XV + v) * Lh + c] = make_int4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
         xs[idx] = 1.0f / up;
     }
-    cons_sync();
 
-    // routing cache (filled after the dependency wait): [0] U, then per work expert:
-    // slot begin, count; then per slot position: token, weight bits, h row
+    // routing cache: [0] U; rBeg/rCnt per work expert; per slot: token, weight, h row
     int *rU = rt;
-    int *rBeg = rt + 1;                    // [32 + 1]
-    int *rCnt = rBeg + 33;                 // [33]
-    int *rTok = rCnt + 33;                 // [T*K + T]
+    int *rBeg = rt + 1;
+    int *rCnt = rBeg + 33;
+    int *rTok = rCnt + 33;
     float *rW = reinterpret_cast<float *>(rTok + 8 * 33);
     int *rH = reinterpret_cast<int *>(rW + 8 * 33);
     bool have_routing = false;
     auto get_routing = [&]() {
-        if (have_routing) return;
         grid_dep_wait();
         if (ct == 0) {
             int U = __ldcg(f.n_unique);
@@ -582,23 +602,17 @@ __global__ void __maxnreg__(128) ffn_decode_kernel(DecodeParams p) {
         cons_sync();
         have_routing = true;
     };
-    // the shared expert's slots need no routing
-    if (ct == 0 && f.S) {
-        rBeg[0] = 0x40000000;  // marker: shared slots are computed, not cached
-        rCnt[0] = T;
-    }
-    cons_sync();
+    cons_sync();  // activations ready
 
     // ------------------------------------------------ phase 1: gate/up, h = SiLU(g)*u -----
-    const int p1 = ct / Lh, c1 = ct % Lh;      // row slot, chunk
-    const int P1 = p.P1;
-    const int nwr1 = Lh / 32;                  // warps per row
-    int seq = 0;
-    int U = 0;
     // After a timed-out wait a thread keeps walking the same loops and barriers (skipping later
     // waits), so that no consumer is ever left alone at a named barrier.
+    const int NJ = Lh / 32;                  // chunks per lane in a row
+    const int NGRP = NCW / PS;               // stage groups
+    const int my_pair = cw % PS, my_grp = cw / PS;
+    int seq = 0, U = 0;
     for (int we = 0;; ++we) {
-        if (we >= f.S) { get_routing(); U = *rU; }
+        if (we >= f.S && !have_routing) { get_routing(); U = *rU; }
         if (have_routing && we >= f.S + U) break;
         const bool shared = we < f.S;
         const int cnt = shared ? T : rCnt[we];
@@ -607,89 +621,57 @@ __global__ void __maxnreg__(128) ffn_decode_kernel(DecodeParams p) {
             const int s = seq % S;
             const uint32_t par = (seq / S) & 1;
             if (ok && !mbar_wait(full_bar(s), par)) ok = false;
-            const int r0 = i_lo + k * R1, n = min(R1, i_hi - r0);
-            const unsigned char *st = ring + static_cast<size_t>(s) * p.SB;
-            uint4 qg[RPT1], qu[RPT1];
+            const int r0 = i_lo + k * PS, n = min(PS, i_hi - r0);
+            const bool mine = ok && (seq % NGRP) == my_grp && my_pair < n && my_grp < NGRP;
+            if (mine) {
+                const unsigned char *st = ring + static_cast<size_t>(s) * p.SB;
+                const unsigned char *rg = st + static_cast<size_t>(my_pair) * f.rb_h;
+                const unsigned char *ru = st + p.st_up + static_cast<size_t>(my_pair) * f.rb_h;
+                float g[TMAX], u[TMAX];
 #pragma unroll
-            for (int m = 0; m < RPT1; ++m) {
-                const int row = p1 + P1 * m;
-                if (row < n) {
-                    qg[m] = lds128(st + static_cast<size_t>(row) * f.rb_h + c1 * 16);
-                    qu[m] = lds128(st + p.st_up + static_cast<size_t>(row) * f.rb_h + c1 * 16);
-                } else {
-                    qg[m] = make_uint4(0, 0, 0, 0);
-                    qu[m] = qg[m];
+                for (int q = 0; q < TMAX; ++q) { g[q] = 0.f; u[q] = 0.f; }
+                for (int j = 0; j < NJ; ++j) {
+                    const int c = lane + 32 * j;
+                    const uint4 qg = lds128(rg + c * 16);
+                    const uint4 qu = lds128(ru + c * 16);
+#pragma unroll
+                    for (int q = 0; q < TMAX; ++q) {
+                        if (q < cnt) {
+                            const int tok = shared ? q : rTok[beg + q];
+                            int xr[XW];
+#pragma unroll
+                            for (int v = 0; v < XV; ++v) {
+                                const int4 t4 = xq[(static_cast<size_t>(tok) * XV + v) * Lh + c];
+                                xr[4 * v] = t4.x; xr[4 * v + 1] = t4.y; xr[4 * v + 2] = t4.z; xr[4 * v + 3] = t4.w;
+                            }
+                            const float sc = xs[tok * Lh + c];
+                            const int corr = xc[tok * Lh + c];
+                            g[q] = __fmaf_rn(static_cast<float>(idot_chunk<FMT>(qg, xr, corr)), sc, g[q]);
+                            u[q] = __fmaf_rn(static_cast<float>(idot_chunk<FMT>(qu, xr, corr)), sc, u[q]);
+                        }
+                    }
                 }
-            }
-            const int a0 = r0 & ~3;
-            float sgv[RPT1], suv[RPT1];
+                const int a0 = r0 & ~3;
+                const float sgv = reinterpret_cast<const float *>(st + p.st_sg)[r0 + my_pair - a0];
+                const float suv = reinterpret_cast<const float *>(st + p.st_su)[r0 + my_pair - a0];
 #pragma unroll
-            for (int m = 0; m < RPT1; ++m) {
-                const int row = p1 + P1 * m;
-                const int rr = row < n ? r0 + row - a0 : 0;
-                sgv[m] = reinterpret_cast<const float *>(st + p.st_sg)[rr];
-                suv[m] = reinterpret_cast<const float *>(st + p.st_su)[rr];
+                for (int q = 0; q < TMAX; ++q) {
+                    if (q < cnt) {
+                        const float gq = __fmul_rn(warp_allsum(g[q]), sgv);
+                        const float uq = __fmul_rn(warp_allsum(u[q]), suv);
+                        if (lane == q) {
+                            const int hrow = shared ? T * f.K + q : rH[beg + q];
+                            f.h[static_cast<size_t>(hrow) * f.I + r0 + my_pair] =
+                                __fmul_rn(__fdiv_rn(gq, __fadd_rn(1.0f, expf(-gq))), uq);
+                        }
+                    }
+                }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(empty_bar(s));
-            float *rb = red1 + (seq & 1) * p.red1_len;
-            for (int q0 = 0; q0 < cnt; q0 += TMAX) {
-                float vg[RPT1][TMAX], vu[RPT1][TMAX];
-#pragma unroll
-                for (int q = 0; q < TMAX; ++q) {
-                    const bool valid = q0 + q < cnt;
-                    const int tok = valid ? (shared ? q0 + q : rTok[beg + q0 + q]) : 0;
-                    const int *xp = xq + (static_cast<size_t>(tok) * Lh + c1) * XW;
-                    const float sc = xs[tok * Lh + c1];
-                    const int corr = xc[tok * Lh + c1];
-                    int xr[XW];
-#pragma unroll
-                    for (int i = 0; i < XW / 4; ++i) {
-                        const int4 v = reinterpret_cast<const int4 *>(xp)[i];
-                        xr[4 * i] = v.x; xr[4 * i + 1] = v.y; xr[4 * i + 2] = v.z; xr[4 * i + 3] = v.w;
-                    }
-#pragma unroll
-                    for (int m = 0; m < RPT1; ++m) {
-                        vg[m][q] = valid ? static_cast<float>(idot_chunk<FMT>(qg[m], xr, corr)) * sc : 0.f;
-                        vu[m][q] = valid ? static_cast<float>(idot_chunk<FMT>(qu[m], xr, corr)) * sc : 0.f;
-                    }
-                }
-#pragma unroll
-                for (int m = 0; m < RPT1; ++m)
-#pragma unroll
-                    for (int q = 0; q < TMAX; ++q) {
-                        const float g = warp_allsum(vg[m][q]);
-                        const float u = warp_allsum(vu[m][q]);
-                        if (lane == 0) {
-                            const int base = ((p1 * RPT1 + m) * TMAX + q) * 2 * nwr1 + (c1 >> 5);
-                            rb[base] = g;
-                            rb[base + nwr1] = u;
-                        }
-                    }
-                cons_sync();
-                // finalize by the first warp of each row slot: lane = (m, q); the scales were read
-                // from the stage before it was released
-                if (c1 < RPT1 * TMAX) {
-                    const int m = c1 / TMAX, q = c1 % TMAX;
-                    const int row = p1 + P1 * m;
-                    if (ok && row < n && q0 + q < cnt) {
-                        float sg = 0.f, su = 0.f;
-#pragma unroll
-                        for (int mm = 0; mm < RPT1; ++mm)
-                            if (mm == m) { sg = sgv[mm]; su = suv[mm]; }
-                        const int base = ((p1 * RPT1 + m) * TMAX + q) * 2 * nwr1;
-                        float g = 0.f, u = 0.f;
-                        for (int w = 0; w < nwr1; ++w) { g += rb[base + w]; u += rb[base + nwr1 + w]; }
-                        g *= sg;
-                        u *= su;
-                        const int hrow = shared ? T * f.K + q0 + q : rH[beg + q0 + q];
-                        f.h[static_cast<size_t>(hrow) * f.I + r0 + row] = (g / (1.0f + expf(-g))) * u;
-                    }
-                }
-                if (q0 + TMAX < cnt) cons_sync();
-            }
         }
     }
+
     // ------------------------------------------------ grid barrier ------------------------
     cons_sync();
     if (ct == 0) {
@@ -713,6 +695,7 @@ __global__ void __maxnreg__(128) ffn_decode_kernel(DecodeParams p) {
     const int p2 = ct / Li, c2 = ct % Li;
     const int P2 = p.P2;
     const int nwr2 = Li / 32;
+    constexpr int HV = CPC / 4;              // float4 vectors of h per chunk
     float acc[RPT2MAX][TMAX];
 #pragma unroll
     for (int m = 0; m < RPT2MAX; ++m)
@@ -721,20 +704,22 @@ __global__ void __maxnreg__(128) ffn_decode_kernel(DecodeParams p) {
     const int nrows = j_hi - j_lo;
     const int a0d = j_lo & ~3;
     const int nwe = f.S + U;
-    const int I4 = f.I / 4;
-    const size_t hbuf = static_cast<size_t>(TMAX) * f.I;  // floats per h buffer
-    // h rows of one expert's slots -> shared memory with cp.async (one buffer per expert parity)
+    // h of an expert's slots -> shared memory with cp.async, transposed: float4 vector v of
+    // chunk c of slot q at hb[buf][(q * HV + v) * Li + c]
+    const size_t hbuf = static_cast<size_t>(TMAX) * HV * Li;  // float4 per buffer
     auto stage_h = [&](int we) {
         const bool shd = we < f.S;
         const int cnt = shd ? T : rCnt[we];
         const int beg = shd ? 0 : rBeg[we];
-        float *dstb = hb + (we & 1) * hbuf;
-        for (int idx = ct; idx < cnt * I4; idx += NC) {
-            const int q = idx / I4, c4 = idx % I4;
+        float4 *dstb = hb + (we & 1) * hbuf;
+        const int per = HV * Li;             // float4 per slot
+        for (int idx = ct; idx < cnt * per; idx += NC) {
+            const int q = idx / per, r = idx % per;
+            const int c = r / HV, v = r % HV;  // source order: chunk-major
             const int hrow = shd ? T * f.K + q : rH[beg + q];
-            const uint32_t d = smem_u32(dstb + static_cast<size_t>(q) * f.I + 4 * c4);
+            const uint32_t d = smem_u32(dstb + (static_cast<size_t>(q) * HV + v) * Li + c);
             asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d),
-                         "l"(f.h + static_cast<size_t>(hrow) * f.I + 4 * c4) : "memory");
+                         "l"(f.h + static_cast<size_t>(hrow) * f.I + static_cast<size_t>(c) * CPC + 4 * v) : "memory");
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
@@ -751,32 +736,34 @@ __global__ void __maxnreg__(128) ffn_decode_kernel(DecodeParams p) {
             asm volatile("cp.async.wait_group 0;" ::: "memory");
         }
         cons_sync();                               // buffer we&1 is complete
-        const float *hcur = hb + (we & 1) * hbuf;
+        const float4 *hcur = hb + (we & 1) * hbuf;
         const int s = seq % S;
         const uint32_t par = (seq / S) & 1;
         ++seq;
         if (ok && !mbar_wait(full_bar(s), par)) ok = false;
-        const unsigned char *st = ring + static_cast<size_t>(s) * p.SB;
-        const float *sdp = reinterpret_cast<const float *>(st + p.st_sd) + (j_lo - a0d);
-        for (int q = 0; q < cnt; ++q) {
-            const int tok = shared ? q : rTok[beg + q];
-            const float wq = shared ? 1.0f : rW[beg + q];
-            float hr[CPC];
-            const float4 *hp = reinterpret_cast<const float4 *>(hcur + static_cast<size_t>(q) * f.I + c2 * CPC);
+        if (ok) {
+            const unsigned char *st = ring + static_cast<size_t>(s) * p.SB;
+            const float *sdp = reinterpret_cast<const float *>(st + p.st_sd) + (j_lo - a0d);
+            for (int q = 0; q < cnt; ++q) {
+                const int tok = shared ? q : rTok[beg + q];
+                const float wq = shared ? 1.0f : rW[beg + q];
+                float hr[CPC];
 #pragma unroll
-            for (int i = 0; i < CPC / 4; ++i) {
-                const float4 v = hp[i];
-                hr[4 * i] = v.x; hr[4 * i + 1] = v.y; hr[4 * i + 2] = v.z; hr[4 * i + 3] = v.w;
-            }
+                for (int v = 0; v < HV; ++v) {
+                    const float4 t4 = hcur[(static_cast<size_t>(q) * HV + v) * Li + c2];
+                    hr[4 * v] = t4.x; hr[4 * v + 1] = t4.y; hr[4 * v + 2] = t4.z; hr[4 * v + 3] = t4.w;
+                }
 #pragma unroll
-            for (int m = 0; m < RPT2MAX; ++m) {
-                const int row = p2 + P2 * m;
-                if (row < nrows) {
-                    const uint4 qd = lds128(st + static_cast<size_t>(row) * f.rb_i + c2 * 16);
-                    const float d = fdot_chunk<FMT>(qd, hr) * (wq * sdp[row]);
+                for (int m = 0; m < RPT2MAX; ++m) {
+                    const int row = p2 + P2 * m;
+                    if (row < nrows) {
+                        const uint4 qd = lds128(st + static_cast<size_t>(row) * f.rb_i + c2 * 16);
+                        const float wsd = __fmul_rn(wq, sdp[row]);
+                        const float d = fdot_chunk<FMT>(qd, hr);
 #pragma unroll
-                    for (int t2 = 0; t2 < TMAX; ++t2)
-                        if (t2 == tok) acc[m][t2] += d;
+                        for (int t2 = 0; t2 < TMAX; ++t2)
+                            if (t2 == tok) acc[m][t2] = __fmaf_rn(d, wsd, acc[m][t2]);
+                    }
                 }
             }
         }
@@ -785,13 +772,14 @@ __global__ void __maxnreg__(128) ffn_decode_kernel(DecodeParams p) {
     }
     if (!ok) atomicOr(f.err, COLI_DEVERR_TIMEOUT);
     // cross-lane reduction of the accumulators, then one store per (token, row)
-    float *red2 = red1;
 #pragma unroll
     for (int m = 0; m < RPT2MAX; ++m)
 #pragma unroll
         for (int q = 0; q < TMAX; ++q) {
-            const float v = warp_allsum(acc[m][q]);
-            if (lane == 0) red2[((p2 * RPT2MAX + m) * TMAX + q) * nwr2 + (c2 >> 5)] = v;
+            if (q < T) {
+                const float v = warp_allsum(acc[m][q]);
+                if (lane == 0) red2[((p2 * RPT2MAX + m) * TMAX + q) * nwr2 + (c2 >> 5)] = v;
+            }
         }
     cons_sync();
     for (int fi = ct; fi < P2 * RPT2MAX * T; fi += NC) {
@@ -799,10 +787,9 @@ __global__ void __maxnreg__(128) ffn_decode_kernel(DecodeParams p) {
         const int row = ps + P2 * m;
         if (row >= nrows) continue;
         float v = 0.f;
-        for (int w = 0; w < nwr2; ++w) v += red2[((ps * RPT2MAX + m) * TMAX + q) * nwr2 + w];
+        for (int w = 0; w < nwr2; ++w) v = __fadd_rn(v, red2[((ps * RPT2MAX + m) * TMAX + q) * nwr2 + w]);
         f.out[static_cast<size_t>(q) * f.H + j_lo + row] = v;
     }
-    (void)cw;
 }
 
 template <int FMT, int TMAX>
@@ -845,42 +832,40 @@ bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan) {
     const int sms = device_sm_count();
     const int rb_h = c.hidden * c.wfmt / 8, rb_i = c.inter * c.wfmt / 8;
     const int Lh = rb_h / 16, Li = rb_i / 16;
-    if (rb_h % 16 || rb_i % 16 || Lh % 32 || Li % 32 || NC % Lh || NC % Li) return false;
-    const int P1 = NC / Lh, P2 = NC / Li;
-    const int rows1 = (c.inter + sms - 1) / sms, rows2 = (c.hidden + sms - 1) / sms;
+    if (rb_h % 16 || rb_i % 16 || Lh % 32 || Li % 32 || NC % Li) return false;
+    if (NCW % PS1) return false;
+    const int P2 = NC / Li;
+    const int rows2 = (c.hidden + sms - 1) / sms;
     if (c.inter < sms || c.hidden < sms) return false;
     if (rows2 > P2 * RPT2MAX) return false;
-    const int R1 = P1 * RPT1;
-    (void)rows1;
-    const int CPC = 128 / c.wfmt;
+    const int tmax = T <= 1 ? 1 : (T <= 2 ? 2 : 4);
     DecodePlan pl;
     pl.grid = sms;
-    pl.Lh = Lh; pl.Li = Li; pl.P1 = P1; pl.P2 = P2; pl.R1 = R1;
+    pl.Lh = Lh; pl.Li = Li; pl.P1 = 0; pl.P2 = P2; pl.R1 = PS1;
     // stage layout (phase 1: gate rows | up rows | sg | su; phase 2: down rows | sd)
-    const int scal1 = ((R1 + 8 + 3) / 4) * 16;
+    const int scal1 = ((PS1 + 8 + 3) / 4) * 16;
     const int scal2 = ((rows2 + 8 + 3) / 4) * 16;
-    pl.st_up = R1 * rb_h;
-    pl.st_sg = 2 * R1 * rb_h;
+    pl.st_up = PS1 * rb_h;
+    pl.st_sg = 2 * PS1 * rb_h;
     pl.st_su = pl.st_sg + scal1;
     const int sb1 = pl.st_su + scal1;
     pl.st_sd = rows2 * rb_i;
     const int sb2 = pl.st_sd + scal2;
     pl.SB = ((sb1 > sb2 ? sb1 : sb2) + 127) / 128 * 128;
-    // shared memory: barriers | routing cache | x (or h buffer) | x scales | corrections | partials | ring
+    // shared memory: barriers | routing cache | x (phase 1) or h (phase 2) | x scales |
+    // corrections | phase-2 partials | ring
     size_t o = 1024;  // barriers (up to 64 stages)
     pl.off_route = o; o += 4096;
     pl.off_x = o;
     const size_t xbytes = static_cast<size_t>(T) * c.hidden * 2;
-    const int tmax = T <= 1 ? 1 : (T <= 2 ? 2 : 4);
     const size_t hbytes = static_cast<size_t>(2) * tmax * c.inter * 4;  // two buffers of TMAX h rows
     o += ((xbytes > hbytes ? xbytes : hbytes) + 127) / 128 * 128;
     pl.off_xs = o; o += static_cast<size_t>(T) * Lh * 4;
     pl.off_xc = o; o += static_cast<size_t>(T) * Lh * 4;
     o = (o + 127) / 128 * 128;
-    pl.red1_len = P1 * RPT1 * tmax * 2 * (Lh / 32);
+    pl.red1_len = 0;
     const int red2_len = P2 * RPT2MAX * tmax * (Li / 32);
-    const int redl = 2 * pl.red1_len > red2_len ? 2 * pl.red1_len : red2_len;
-    pl.off_red = o; o += static_cast<size_t>(redl) * 4;
+    pl.off_red = o; o += static_cast<size_t>(red2_len) * 4;
     o = (o + 1023) / 1024 * 1024;
     pl.off_ring = o;
     const size_t budget = 227 * 1024;
@@ -888,7 +873,6 @@ bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan) {
     pl.S = static_cast<int>((budget - o) / pl.SB);
     if (pl.S > 8) pl.S = 8;
     pl.smem = o + static_cast<size_t>(pl.S) * pl.SB;
-    (void)CPC;
     *plan = pl;
     return true;
 }
