@@ -87,6 +87,9 @@ typedef struct {
 /* Text for a status code (static storage). */
 const char *coli_moe_status_str(coli_status s);
 
+/* Name and text of the CUDA error behind the calling thread's last COLI_ERR_CUDA ("" if none). */
+const char *coli_moe_last_cuda_error(void);
+
 /* Bytes of one record for (hidden, inter, wfmt), before padding to 256.  Host only. */
 coli_status coli_moe_record_bytes(int hidden, int inter, int wfmt, size_t *bytes);
 

@@ -14,7 +14,7 @@ from typing import Optional
 
 __all__ = [
     "ColiError", "MoEConfig", "MoEWeights", "lib", "LIB_PATH",
-    "coli_moe_status_str", "coli_moe_record_bytes", "coli_moe_check_config",
+    "coli_moe_status_str", "coli_moe_last_cuda_error", "coli_moe_record_bytes", "coli_moe_check_config",
     "coli_moe_workspace_size", "coli_moe_clear_error", "coli_moe_error_word",
     "coli_moe_gate", "coli_moe_route", "coli_moe_group", "coli_moe_ffn", "coli_moe_layer",
     "coli_moe_layer_noalloc", "STATIC_SCRATCH_BYTES", "coli_moe_layer_kernels",
@@ -53,7 +53,10 @@ class MoEWeights(C.Structure):
 class ColiError(RuntimeError):
     def __init__(self, fn: str, status: int):
         self.status = status
-        super().__init__(f"{fn}: {coli_moe_status_str(status)} (status {status})")
+        extra = ""
+        if status == 5:
+            extra = " [" + lib.coli_moe_last_cuda_error().decode() + "]"
+        super().__init__(f"{fn}: {coli_moe_status_str(status)} (status {status}){extra}")
 
 
 def _load():
@@ -62,6 +65,8 @@ def _load():
     cfgp, wp = C.POINTER(MoEConfig), C.POINTER(MoEWeights)
     L.coli_moe_status_str.argtypes = [I]
     L.coli_moe_status_str.restype = C.c_char_p
+    L.coli_moe_last_cuda_error.argtypes = []
+    L.coli_moe_last_cuda_error.restype = C.c_char_p
     L.coli_moe_record_bytes.argtypes = [I, I, I, C.POINTER(S)]
     L.coli_moe_check_config.argtypes = [cfgp]
     L.coli_moe_workspace_size.argtypes = [cfgp, I, C.POINTER(S)]
@@ -112,6 +117,10 @@ def _check(fn: str, status: int) -> None:
 
 def coli_moe_status_str(status: int) -> str:
     return lib.coli_moe_status_str(status).decode()
+
+
+def coli_moe_last_cuda_error() -> str:
+    return lib.coli_moe_last_cuda_error().decode()
 
 
 def coli_moe_record_bytes(hidden: int, inter: int, wfmt: int) -> int:

@@ -2,6 +2,7 @@
 // launch sequence of the layer.  No device memory is allocated here; no CPU fallback exists.
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdio.h>
 #include <string.h>
 
 #include "coli_moe.h"
@@ -17,7 +18,13 @@ inline bool aligned(const void *p, size_t a) {
     return (reinterpret_cast<uintptr_t>(p) % a) == 0;
 }
 
-coli_status from_cuda(cudaError_t e) { return e == cudaSuccess ? COLI_OK : COLI_ERR_CUDA; }
+thread_local char g_last_cuda_error[256] = "";
+
+coli_status from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return COLI_OK;
+    record_cuda_error(e);
+    return COLI_ERR_CUDA;
+}
 
 int row_bytes(int n, int fmt) { return n * fmt / 8; }
 
@@ -34,6 +41,23 @@ int device_sm_count() {
         cached[dev] = n;
     }
     return cached[dev];
+}
+
+size_t device_smem_optin() {
+    static size_t cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 227 * 1024;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess || n <= 0)
+            n = 227 * 1024;
+        cached[dev] = static_cast<size_t>(n);
+    }
+    return cached[dev];
+}
+
+void record_cuda_error(cudaError_t e) {
+    snprintf(g_last_cuda_error, sizeof g_last_cuda_error, "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
 }
 
 WsLayout ws_layout(const coli_moe_config &c, int T) {
@@ -74,6 +98,8 @@ const char *coli_moe_status_str(coli_status s) {
     }
     return "unknown status";
 }
+
+const char *coli_moe_last_cuda_error(void) { return g_last_cuda_error; }
 
 coli_status coli_moe_record_bytes(int hidden, int inter, int wfmt, size_t *bytes) {
     if (!bytes) return COLI_ERR_INVALID_ARG;
@@ -308,7 +334,7 @@ coli_status coli_moe_layer(const coli_moe_config *c, const coli_moe_weights *w, 
     cudaError_t e = launch_gate(*c, w->router_w, x, T, logits, st);
     if (e == cudaSuccess) e = launch_route(*c, logits, w->router_bias, T, ids, wts, st);
     if (e == cudaSuccess) e = launch_group(*c, ids, T, counts, offsets, perm, uniq, nu, err, st);
-    if (e != cudaSuccess) return COLI_ERR_CUDA;
+    if (e != cudaSuccess) return from_cuda(e);
     return run_ffn(c, p, base, st);
 }
 

@@ -54,10 +54,12 @@ __device__ __forceinline__ void mbar_arrive(uint32_t a) {
 __device__ __forceinline__ void mbar_expect_tx(uint32_t a, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(a), "r"(bytes) : "memory");
 }
+// try_wait with a suspend-time hint (ns): a waiting warp sleeps instead of spinning, leaving
+// issue slots to the warps that compute; it is woken when the phase completes.
 __device__ __forceinline__ bool mbar_try(uint32_t a, uint32_t parity) {
     uint32_t ok;
-    asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
-                 : "=r"(ok) : "r"(a), "r"(parity) : "memory");
+    asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
+                 : "=r"(ok) : "r"(a), "r"(parity), "r"(20000u) : "memory");
     return ok != 0;
 }
 // Bounded wait: false when the bound ran out (the caller records the error and gives up).
@@ -171,26 +173,51 @@ template <> struct Fpos<2> {  // element k: bits 2k
     static constexpr uint32_t FLIP = 0xAAAAAAAAu, MASK = 0x3u;
 };
 
+__device__ __forceinline__ uint64_t pack_b64(uint32_t lo, uint32_t hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+    return r;
+}
+__device__ __forceinline__ uint64_t sub_f32x2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
+// hr holds the chunk's activations as float pairs (element 2i in the low half).  Element k of a
+// word accumulates into the low lane for even k and the high lane for odd k.
 template <int FMT>
-__device__ __forceinline__ float fdot_chunk(const uint4 q, const float *hr) {
+__device__ __forceinline__ float fdot_chunk(const uint4 q, const uint64_t *hr) {
     using F = Fpos<FMT>;
     const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-    float a0 = 0.f, a1 = 0.f;
+    uint64_t acc = 0ull;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const uint32_t f0 = w[i] ^ F::FLIP;
         const uint32_t f1 = f0 >> F::SHIFT;
 #pragma unroll
-        for (int k = 0; k < F::CPW; ++k) {
-            const int pos = k < F::CUT ? k : k - F::SHIFT / F::BITS;
-            const uint32_t src = k < F::CUT ? f0 : f1;
-            const uint32_t bits = (src & (F::MASK << (F::BITS * pos))) | (static_cast<uint32_t>(150 - F::BITS * pos) << 23);
-            const float v = __uint_as_float(bits) - (static_cast<float>(1u << (23 - F::BITS * pos)) + static_cast<float>(F::BIAS));
-            if (k & 1) a1 = fmaf(v, hr[i * F::CPW + k], a1);
-            else a0 = fmaf(v, hr[i * F::CPW + k], a0);
+        for (int k = 0; k < F::CPW; k += 2) {
+            uint32_t bits[2];
+            float off[2];
+#pragma unroll
+            for (int d = 0; d < 2; ++d) {
+                const int kk = k + d;
+                const int pos = kk < F::CUT ? kk : kk - F::SHIFT / F::BITS;
+                const uint32_t src = kk < F::CUT ? f0 : f1;
+                bits[d] = (src & (F::MASK << (F::BITS * pos))) | (static_cast<uint32_t>(150 - F::BITS * pos) << 23);
+                off[d] = static_cast<float>(1u << (23 - F::BITS * pos)) + static_cast<float>(F::BIAS);
+            }
+            const uint64_t v = sub_f32x2(pack_b64(bits[0], bits[1]),
+                                         pack_b64(__float_as_uint(off[0]), __float_as_uint(off[1])));
+            acc = fma_f32x2(v, hr[(i * F::CPW + k) >> 1], acc);
         }
     }
-    return a0 + a1;
+    return __fadd_rn(__uint_as_float(static_cast<uint32_t>(acc)), __uint_as_float(static_cast<uint32_t>(acc >> 32)));
 }
 
 __device__ __forceinline__ float warp_allsum(float v) {
@@ -628,24 +655,33 @@ __global__ void __maxnreg__(112) ffn_decode_kernel(DecodeParams p) {
                 const unsigned char *rg = st + static_cast<size_t>(my_pair) * f.rb_h;
                 const unsigned char *ru = st + p.st_up + static_cast<size_t>(my_pair) * f.rb_h;
                 float g[TMAX], u[TMAX];
+                const int4 *xb[TMAX];
+                const float *xsb[TMAX];
+                const int *xcb[TMAX];
 #pragma unroll
-                for (int q = 0; q < TMAX; ++q) { g[q] = 0.f; u[q] = 0.f; }
+                for (int q = 0; q < TMAX; ++q) {
+                    g[q] = 0.f; u[q] = 0.f;
+                    const int tok = q < cnt ? (shared ? q : rTok[beg + q]) : 0;
+                    xb[q] = xq + static_cast<size_t>(tok) * XV * Lh + lane;
+                    xsb[q] = xs + tok * Lh + lane;
+                    xcb[q] = xc + tok * Lh + lane;
+                }
+                const unsigned char *rgl = rg + lane * 16, *rul = ru + lane * 16;
+#pragma unroll 2
                 for (int j = 0; j < NJ; ++j) {
-                    const int c = lane + 32 * j;
-                    const uint4 qg = lds128(rg + c * 16);
-                    const uint4 qu = lds128(ru + c * 16);
+                    const uint4 qg = lds128(rgl + j * 512);
+                    const uint4 qu = lds128(rul + j * 512);
 #pragma unroll
                     for (int q = 0; q < TMAX; ++q) {
                         if (q < cnt) {
-                            const int tok = shared ? q : rTok[beg + q];
                             int xr[XW];
 #pragma unroll
                             for (int v = 0; v < XV; ++v) {
-                                const int4 t4 = xq[(static_cast<size_t>(tok) * XV + v) * Lh + c];
+                                const int4 t4 = xb[q][v * Lh + 32 * j];
                                 xr[4 * v] = t4.x; xr[4 * v + 1] = t4.y; xr[4 * v + 2] = t4.z; xr[4 * v + 3] = t4.w;
                             }
-                            const float sc = xs[tok * Lh + c];
-                            const int corr = xc[tok * Lh + c];
+                            const float sc = xsb[q][32 * j];
+                            const int corr = xcb[q][32 * j];
                             g[q] = __fmaf_rn(static_cast<float>(idot_chunk<FMT>(qg, xr, corr)), sc, g[q]);
                             u[q] = __fmaf_rn(static_cast<float>(idot_chunk<FMT>(qu, xr, corr)), sc, u[q]);
                         }
@@ -747,11 +783,11 @@ __global__ void __maxnreg__(112) ffn_decode_kernel(DecodeParams p) {
             for (int q = 0; q < cnt; ++q) {
                 const int tok = shared ? q : rTok[beg + q];
                 const float wq = shared ? 1.0f : rW[beg + q];
-                float hr[CPC];
+                uint64_t hr[CPC / 2];
 #pragma unroll
                 for (int v = 0; v < HV; ++v) {
-                    const float4 t4 = hcur[(static_cast<size_t>(q) * HV + v) * Li + c2];
-                    hr[4 * v] = t4.x; hr[4 * v + 1] = t4.y; hr[4 * v + 2] = t4.z; hr[4 * v + 3] = t4.w;
+                    const ulonglong2 t2 = *reinterpret_cast<const ulonglong2 *>(hcur + (static_cast<size_t>(q) * HV + v) * Li + c2);
+                    hr[2 * v] = t2.x; hr[2 * v + 1] = t2.y;
                 }
 #pragma unroll
                 for (int m = 0; m < RPT2MAX; ++m) {
@@ -868,7 +904,7 @@ bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan) {
     pl.off_red = o; o += static_cast<size_t>(red2_len) * 4;
     o = (o + 1023) / 1024 * 1024;
     pl.off_ring = o;
-    const size_t budget = 227 * 1024;
+    const size_t budget = device_smem_optin() - 1024;
     if (o + 2 * static_cast<size_t>(pl.SB) > budget) return false;
     pl.S = static_cast<int>((budget - o) / pl.SB);
     if (pl.S > 8) pl.S = 8;

@@ -99,5 +99,7 @@ bool gemv_shape_ok(int row_bytes);
 int gemv_max_tokens(const coli_moe_config &c);
 
 int device_sm_count();
+size_t device_smem_optin();  // max dynamic shared memory per block (opt-in)
+void record_cuda_error(cudaError_t e);
 
 }  // namespace coli
