@@ -110,48 +110,48 @@ __device__ __forceinline__ int idot_chunk<4>(const uint4 q, const int *xp, int c
     // u = q + 8 per nibble (flip of the sign bit); bytes of lo hold elements 0,2,4,6 of a word,
     // bytes of hi hold 1,3,5,7.  xp holds per word: (m0,m2) (m4,m6) (m1,m3) (m5,m7).
     const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-    int acc = -corr;  // corr = 8 * sum(m)
+    int a0 = -corr, a1 = 0, a2 = 0, a3 = 0;  // corr = 8 * sum(m); four independent chains
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const uint32_t f = w[i] ^ 0x88888888u;
         const uint32_t lo = f & 0x0F0F0F0Fu;
         const uint32_t hi = (f >> 4) & 0x0F0F0F0Fu;
-        acc = __dp2a_lo(xp[4 * i + 0], static_cast<int>(lo), acc);
-        acc = __dp2a_hi(xp[4 * i + 1], static_cast<int>(lo), acc);
-        acc = __dp2a_lo(xp[4 * i + 2], static_cast<int>(hi), acc);
-        acc = __dp2a_hi(xp[4 * i + 3], static_cast<int>(hi), acc);
+        a0 = __dp2a_lo(xp[4 * i + 0], static_cast<int>(lo), a0);
+        a1 = __dp2a_hi(xp[4 * i + 1], static_cast<int>(lo), a1);
+        a2 = __dp2a_lo(xp[4 * i + 2], static_cast<int>(hi), a2);
+        a3 = __dp2a_hi(xp[4 * i + 3], static_cast<int>(hi), a3);
     }
-    return acc;
+    return (a0 + a1) + (a2 + a3);
 }
 template <>
 __device__ __forceinline__ int idot_chunk<8>(const uint4 q, const int *xp, int) {
     // signed bytes in natural order; xp holds (m0,m1) (m2,m3) per word
     const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-    int acc = 0;
+    int a0 = 0, a1 = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        acc = __dp2a_lo(xp[2 * i + 0], static_cast<int>(w[i]), acc);
-        acc = __dp2a_hi(xp[2 * i + 1], static_cast<int>(w[i]), acc);
+        a0 = __dp2a_lo(xp[2 * i + 0], static_cast<int>(w[i]), a0);
+        a1 = __dp2a_hi(xp[2 * i + 1], static_cast<int>(w[i]), a1);
     }
-    return acc;
+    return a0 + a1;
 }
 template <>
 __device__ __forceinline__ int idot_chunk<2>(const uint4 q, const int *xp, int corr) {
     // u = q + 2 per 2-bit field; extraction k gives bytes with elements 4j+k (j = byte);
     // xp holds per word and k: (m_k, m_{4+k}) (m_{8+k}, m_{12+k}).
     const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-    int acc = -corr;  // corr = 2 * sum(m)
+    int a[4] = {-corr, 0, 0, 0};  // corr = 2 * sum(m)
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const uint32_t f = w[i] ^ 0xAAAAAAAAu;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const uint32_t b = (f >> (2 * k)) & 0x03030303u;
-            acc = __dp2a_lo(xp[8 * i + 2 * k + 0], static_cast<int>(b), acc);
-            acc = __dp2a_hi(xp[8 * i + 2 * k + 1], static_cast<int>(b), acc);
+            a[k] = __dp2a_lo(xp[8 * i + 2 * k + 0], static_cast<int>(b), a[k]);
+            a[k] = __dp2a_hi(xp[8 * i + 2 * k + 1], static_cast<int>(b), a[k]);
         }
     }
-    return acc;
+    return (a[0] + a[1]) + (a[2] + a[3]);
 }
 
 // Float decode of codes at their bit position.  A code field u sitting at mantissa bits
@@ -189,35 +189,53 @@ __device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c
     return r;
 }
 
-// hr holds the chunk's activations as float pairs (element 2i in the low half).  Element k of a
-// word accumulates into the low lane for even k and the high lane for odd k.
+// One word of codes against its four activation pairs: acc += decoded codes * h (packed pairs).
 template <int FMT>
-__device__ __forceinline__ float fdot_chunk(const uint4 q, const uint64_t *hr) {
+__device__ __forceinline__ uint64_t fdot_word(uint32_t w, const uint64_t *hw, uint64_t acc) {
     using F = Fpos<FMT>;
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-    uint64_t acc = 0ull;
+    const uint32_t f0 = w ^ F::FLIP;
+    const uint32_t f1 = f0 >> F::SHIFT;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t f0 = w[i] ^ F::FLIP;
-        const uint32_t f1 = f0 >> F::SHIFT;
+    for (int k = 0; k < F::CPW; k += 2) {
+        uint32_t bits[2];
+        float off[2];
 #pragma unroll
-        for (int k = 0; k < F::CPW; k += 2) {
-            uint32_t bits[2];
-            float off[2];
-#pragma unroll
-            for (int d = 0; d < 2; ++d) {
-                const int kk = k + d;
-                const int pos = kk < F::CUT ? kk : kk - F::SHIFT / F::BITS;
-                const uint32_t src = kk < F::CUT ? f0 : f1;
-                bits[d] = (src & (F::MASK << (F::BITS * pos))) | (static_cast<uint32_t>(150 - F::BITS * pos) << 23);
-                off[d] = static_cast<float>(1u << (23 - F::BITS * pos)) + static_cast<float>(F::BIAS);
-            }
-            const uint64_t v = sub_f32x2(pack_b64(bits[0], bits[1]),
-                                         pack_b64(__float_as_uint(off[0]), __float_as_uint(off[1])));
-            acc = fma_f32x2(v, hr[(i * F::CPW + k) >> 1], acc);
+        for (int d = 0; d < 2; ++d) {
+            const int kk = k + d;
+            const int pos = kk < F::CUT ? kk : kk - F::SHIFT / F::BITS;
+            const uint32_t src = kk < F::CUT ? f0 : f1;
+            bits[d] = (src & (F::MASK << (F::BITS * pos))) | (static_cast<uint32_t>(150 - F::BITS * pos) << 23);
+            off[d] = static_cast<float>(1u << (23 - F::BITS * pos)) + static_cast<float>(F::BIAS);
         }
+        const uint64_t v = sub_f32x2(pack_b64(bits[0], bits[1]),
+                                     pack_b64(__float_as_uint(off[0]), __float_as_uint(off[1])));
+        acc = fma_f32x2(v, hw[k >> 1], acc);
     }
-    return __fadd_rn(__uint_as_float(static_cast<uint32_t>(acc)), __uint_as_float(static_cast<uint32_t>(acc >> 32)));
+    return acc;
+}
+
+__device__ __forceinline__ float sum_pair(uint64_t v) {
+    return __fadd_rn(__uint_as_float(static_cast<uint32_t>(v)), __uint_as_float(static_cast<uint32_t>(v >> 32)));
+}
+
+// Dots of two chunks of codes (two rows) with the same activations, four independent chains.
+// hr holds the chunk's activations as float pairs (element 2i in the low half); element k of a
+// word accumulates into the low lane for even k and the high lane for odd k; words 0-1 and 2-3
+// go to separate pairs, summed at the end.
+template <int FMT>
+__device__ __forceinline__ void fdot2_chunk(const uint4 q0, const uint4 q1, const uint64_t *hr, float &d0, float &d1) {
+    constexpr int HP = Fpos<FMT>::CPW / 2;  // activation pairs per word
+    uint64_t a0 = 0ull, b0 = 0ull, a1 = 0ull, b1 = 0ull;
+    a0 = fdot_word<FMT>(q0.x, hr + 0 * HP, a0);
+    a1 = fdot_word<FMT>(q1.x, hr + 0 * HP, a1);
+    b0 = fdot_word<FMT>(q0.z, hr + 2 * HP, b0);
+    b1 = fdot_word<FMT>(q1.z, hr + 2 * HP, b1);
+    a0 = fdot_word<FMT>(q0.y, hr + 1 * HP, a0);
+    a1 = fdot_word<FMT>(q1.y, hr + 1 * HP, a1);
+    b0 = fdot_word<FMT>(q0.w, hr + 3 * HP, b0);
+    b1 = fdot_word<FMT>(q1.w, hr + 3 * HP, b1);
+    d0 = __fadd_rn(sum_pair(a0), sum_pair(b0));
+    d1 = __fadd_rn(sum_pair(a1), sum_pair(b1));
 }
 
 __device__ __forceinline__ float warp_allsum(float v) {
@@ -283,48 +301,52 @@ __device__ void route_token_cta(const DecodeParams &p, int t, double *cs, double
     }
 }
 
-// Group the T*K slots of the batch with one CTA (T*K <= 64).
-__device__ void group_batch_cta(const DecodeParams &p, int *sid, int *scnt, int *soff, int *sflag) {
+// Group the n = T*K <= 32 slots of the batch: warp 0 ranks the slots by (expert id, slot) with
+// shuffles (a stable sort), the unique list follows from the sorted order; every thread fills the
+// per-expert counts and offsets by scanning the n slots.
+__device__ void group_batch_cta(const DecodeParams &p, int *sid, int *ssorted) {
     const int E = p.f.E, n = p.f.T * p.f.K;
     const int tid = threadIdx.x;
-    for (int s = tid; s < n; s += blockDim.x) sid[s] = __ldcg(p.ids + s);
-    __syncthreads();
-    for (int e = tid; e < E; e += blockDim.x) {
-        int c = 0;
-        for (int s = 0; s < n; ++s) c += sid[s] == e;
-        scnt[e] = c;
-        sflag[e] = c > 0;
-    }
-    __syncthreads();
-    if (tid == 0) {  // E <= 1024 sequential scans: a few microseconds at most, E ~ 256 here
-        int o = 0, u = 0;
-        for (int e = 0; e < E; ++e) {
-            soff[e] = o;
-            o += scnt[e];
-            const int f = sflag[e];
-            sflag[e] = f ? u : -1;
-            u += f;
+    if (tid < 32) {
+        const int lane = tid;
+        const int id = lane < n ? __ldcg(p.ids + lane) : 0x7fffffff;
+        sid[lane] = id;
+        int r = 0;
+        for (int s2 = 0; s2 < 32; ++s2) {
+            const int o = __shfl_sync(FULL, id, s2);
+            r += (o < id) || (o == id && s2 < lane);
         }
-        soff[E] = o;
-        p.f_offsets[E] = o;
-        *p.f_nuniq = u;
-    }
-    __syncthreads();
-    for (int e = tid; e < E; e += blockDim.x) {
-        p.f_counts[e] = scnt[e];
-        p.f_offsets[e] = soff[e];
-        if (scnt[e] > 0) {
-            int k = soff[e];
-            for (int s = 0; s < n; ++s)
-                if (sid[s] == e) p.f_perm[k++] = s;
-            p.f_unique[sflag[e]] = e;
+        if (lane < n) {
+            p.f_perm[r] = lane;
+            ssorted[r] = id;
+        }
+        __syncwarp();
+        const int idr = lane < n ? ssorted[lane] : 0x7fffffff;
+        const bool first = lane < n && (lane == 0 || ssorted[lane - 1] != idr);
+        const unsigned m = __ballot_sync(FULL, first);
+        const int up = __popc(m & ((1u << lane) - 1u));
+        if (first) p.f_unique[up] = idr;
+        if (lane == 0) {
+            *p.f_nuniq = __popc(m);
+            p.f_offsets[E] = n;
         }
     }
     __syncthreads();
-    if (tid == 0) {
-        const int u = *p.f_nuniq;
-        for (int e = u; e < E; ++e) p.f_unique[e] = -1;
+    for (int e = tid; e < E; e += blockDim.x) {
+        int c = 0, lt = 0;
+        for (int s2 = 0; s2 < n; ++s2) {
+            const int v = sid[s2];
+            c += v == e;
+            lt += v < e;
+        }
+        p.f_counts[e] = c;
+        p.f_offsets[e] = lt;
     }
+    // unique entries past the last are -1: the number of distinct ids is known to every thread
+    int distinct = 0;
+    for (int s2 = 0; s2 < n; ++s2) distinct += (s2 == 0 || ssorted[s2 - 1] != ssorted[s2]);
+    for (int e = tid; e < E; e += blockDim.x)
+        if (e >= distinct) p.f_unique[e] = -1;
 }
 
 __global__ void __launch_bounds__(256) router_decode_kernel(DecodeParams p) {
@@ -408,10 +430,8 @@ __global__ void __launch_bounds__(256) router_decode_kernel(DecodeParams p) {
     if (!last) return;
     __threadfence();
     int *sid = sel_id + 32;
-    int *scnt = sid + 64;
-    int *soff = scnt + E;
-    int *sflag = soff + E + 1;
-    group_batch_cta(p, sid, scnt, soff, sflag);
+    int *ssorted = sid + 64;
+    group_batch_cta(p, sid, ssorted);
     __syncthreads();
     if (threadIdx.x == 0) {
         *p.route_cnt = 0u;
@@ -428,7 +448,7 @@ __global__ void __launch_bounds__(256) router_decode_kernel(DecodeParams p) {
 // thread (p2, c2) owns chunk c2 of rows p2 + P2*m and keeps per-(row, token) partial sums in
 // registers across experts; one cross-lane reduction at the end.
 template <int FMT, int TMAX>
-__global__ void __maxnreg__(112) ffn_decode_kernel(DecodeParams p) {
+__global__ void __maxnreg__(96) ffn_decode_kernel(DecodeParams p) {
     constexpr int CPC = Fmt<FMT>::CPC;       // codes per 16-byte chunk
     constexpr int XW = CPC / 2;              // int32 words of 16-bit activations per chunk
     constexpr int XV = XW / 4;               // int4 vectors per chunk
@@ -598,14 +618,12 @@ __global__ void __maxnreg__(112) ffn_decode_kernel(DecodeParams p) {
     bool have_routing = false;
     auto get_routing = [&]() {
         grid_dep_wait();
-        if (ct == 0) {
+        if (cw == 0) {  // lane u handles unique expert u (U <= 32)
             int U = __ldcg(f.n_unique);
             U = U < 0 ? 0 : (U > 32 ? 32 : U);
-            *rU = U;
-            int pos = 0;
-            for (int u = 0; u < U; ++u) {
-                const int e = __ldcg(f.unique + u);
-                int b0 = 0, c0 = 0;
+            int e = -1, b0 = 0, c0 = 0;
+            if (lane < U) {
+                e = __ldcg(f.unique + lane);
                 if (e >= 0 && e < f.E) {
                     b0 = __ldcg(f.offsets + e);
                     c0 = __ldcg(f.offsets + e + 1) - b0;
@@ -613,16 +631,25 @@ __global__ void __maxnreg__(112) ffn_decode_kernel(DecodeParams p) {
                 } else {
                     atomicOr(f.err, COLI_DEVERR_EXPERT_ID);
                 }
-                rBeg[f.S + u] = pos;
-                rCnt[f.S + u] = c0;
+            }
+            int pos = c0;  // exclusive scan of the slot counts
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(FULL, pos, o);
+                if (lane >= o) pos += v;
+            }
+            pos -= c0;
+            if (lane == 0) *rU = U;
+            if (lane < U) {
+                rBeg[f.S + lane] = pos;
+                rCnt[f.S + lane] = c0;
                 for (int q = 0; q < c0; ++q) {
                     const int sl = __ldcg(f.perm + b0 + q);
                     const bool good = sl >= 0 && sl < T * f.K;
                     if (!good) atomicOr(f.err, COLI_DEVERR_GROUPING);
-                    rTok[pos] = good ? sl / f.K : 0;
-                    rW[pos] = good ? __ldcg(f.topk_w + sl) : 0.f;
-                    rH[pos] = good ? b0 + q : 0;
-                    ++pos;
+                    rTok[pos + q] = good ? sl / f.K : 0;
+                    rW[pos + q] = good ? __ldcg(f.topk_w + sl) : 0.f;
+                    rH[pos + q] = good ? b0 + q : 0;
                 }
             }
         }
@@ -790,15 +817,22 @@ __global__ void __maxnreg__(112) ffn_decode_kernel(DecodeParams p) {
                     hr[2 * v] = t2.x; hr[2 * v + 1] = t2.y;
                 }
 #pragma unroll
-                for (int m = 0; m < RPT2MAX; ++m) {
-                    const int row = p2 + P2 * m;
-                    if (row < nrows) {
-                        const uint4 qd = lds128(st + static_cast<size_t>(row) * f.rb_i + c2 * 16);
-                        const float wsd = __fmul_rn(wq, sdp[row]);
-                        const float d = fdot_chunk<FMT>(qd, hr);
+                for (int m = 0; m < RPT2MAX; m += 2) {
+                    const int row0 = p2 + P2 * m, row1 = row0 + P2;
+                    if (row0 < nrows) {
+                        const bool has1 = row1 < nrows;
+                        const uint4 qd0 = lds128(st + static_cast<size_t>(row0) * f.rb_i + c2 * 16);
+                        const uint4 qd1 = has1 ? lds128(st + static_cast<size_t>(row1) * f.rb_i + c2 * 16) : make_uint4(0, 0, 0, 0);
+                        const float wsd0 = __fmul_rn(wq, sdp[row0]);
+                        const float wsd1 = has1 ? __fmul_rn(wq, sdp[row1]) : 0.f;
+                        float d0, d1;
+                        fdot2_chunk<FMT>(qd0, qd1, hr, d0, d1);
 #pragma unroll
                         for (int t2 = 0; t2 < TMAX; ++t2)
-                            if (t2 == tok) acc[m][t2] = __fmaf_rn(d, wsd, acc[m][t2]);
+                            if (t2 == tok) {
+                                acc[m][t2] = __fmaf_rn(d0, wsd0, acc[m][t2]);
+                                acc[m + 1][t2] = __fmaf_rn(d1, wsd1, acc[m + 1][t2]);
+                            }
                     }
                 }
             }
@@ -859,6 +893,22 @@ cudaError_t launch_k2_t(const DecodeParams &p, size_t smem, cudaStream_t st, boo
 
 }  // namespace
 
+// The register allocation of a kernel instantiation bounds its block size: check it fits NT.
+template <int FMT, int TMAX>
+static bool fits_block() {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, ffn_decode_kernel<FMT, TMAX>) != cudaSuccess) return false;
+    return fa.maxThreadsPerBlock >= NT;
+}
+static bool kernel_fits(int fmt, int T) {
+    const int tm = T <= 1 ? 1 : (T <= 2 ? 2 : 4);
+#define COLI_FITS(F)                                                        \
+    if (fmt == F) return tm == 1 ? fits_block<F, 1>() : (tm == 2 ? fits_block<F, 2>() : fits_block<F, 4>());
+    COLI_FITS(4) COLI_FITS(8) COLI_FITS(2)
+#undef COLI_FITS
+    return false;
+}
+
 // Shape rules and the shared-memory plan of the fused decode path.
 bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan) {
     if (T < 1 || T > 4) return false;
@@ -875,6 +925,7 @@ bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan) {
     if (c.inter < sms || c.hidden < sms) return false;
     if (rows2 > P2 * RPT2MAX) return false;
     const int tmax = T <= 1 ? 1 : (T <= 2 ? 2 : 4);
+    if (!kernel_fits(c.wfmt, T)) return false;
     DecodePlan pl;
     pl.grid = sms;
     pl.Lh = Lh; pl.Li = Li; pl.P1 = 0; pl.P2 = P2; pl.R1 = PS1;
