@@ -327,6 +327,7 @@ coli_status coli_moe_layer(const coli_moe_config *c, const coli_moe_weights *w, 
         d.f_perm = perm;
         d.f_unique = uniq;
         d.f_nuniq = nu;
+        d.route_here = 1;
         cudaError_t e = launch_router_decode(d, st);
         if (e == cudaSuccess) e = launch_ffn_decode(d, pl, st, true);
         return from_cuda(e);

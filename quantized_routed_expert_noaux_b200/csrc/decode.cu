@@ -2,11 +2,13 @@
 //
 // Two launches, the second one programmatically dependent on the first:
 //
-//  K1 router_decode_kernel  a1 gate on grid (E/2, T): two Wr rows per CTA, products and sums in
-//                           double.  The last CTA to finish a token routes it (a2, noaux_tc,
-//                           colibri-strix README "What's implemented"), the last token router
-//                           groups the batch (a3, batch-union).  No CTA ever waits on another:
-//                           "last arrival" is decided by an atomic ticket.
+//  K1 gate_decode_kernel    a1 gate on grid (E, T): one Wr row per CTA, products and sums in
+//                           double.  Light enough to share every SM with the FFN kernel.
+//                           Every FFN CTA then routes the batch itself from the logits (a2,
+//                           noaux_tc, colibri-strix README "What's implemented") and groups it
+//                           (a3, batch-union): the same code on the same inputs, so all CTAs agree
+//                           bit for bit and no CTA waits on another; CTA 0 writes the routing
+//                           outputs of the call.
 //  K2 ffn_decode_kernel     a4..a7, persistent, one CTA per SM.  Warp 0 streams weight rows
 //                           into a shared-memory ring with bulk asynchronous copies (TMA engine,
 //                           mbarrier completion); the other warps dequantise from the ring.
@@ -38,7 +40,9 @@ constexpr int NC = NCW * 32;         // consumer threads
 constexpr int NT = NC + 32;          // + producer warp
 constexpr int PS1 = 8;               // (gate, up) row pairs per phase-1 stage
 constexpr int RPT2MAX = 8;           // phase-2 rows per thread over the whole CTA row range
-constexpr int CONS_BAR = 1;          // named barrier id of the consumer warps
+constexpr int CONS_BAR = 1;          // named barrier id of the consumer warps (2..5: per-token routing)
+// routing cache in shared memory (int offsets): U | unique[32] | beg[33] | cnt[33] | tok[32] | w[32] | hrow[32] | sorted slots[32]
+constexpr int RT_UNIQ = 1, RT_BEG = 33, RT_CNT = 66, RT_TOK = 99, RT_W = 131, RT_H = 163, RT_SORT = 195;
 constexpr long long WAIT_CYCLES = 4000000000LL;  // ~2 s at 1.9 GHz: bound of every spin-wait
 
 // ------------------------------------------------------------------------- PTX helpers -----
@@ -84,6 +88,7 @@ __device__ __forceinline__ uint64_t evict_first_policy() {
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void cons_sync() { asm volatile("bar.sync %0, %1;" ::"n"(CONS_BAR), "n"(NC) : "memory"); }
+__device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 __device__ __forceinline__ uint4 lds128(const unsigned char *p) { return *reinterpret_cast<const uint4 *>(p); }
 __device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
     unsigned v;
@@ -94,7 +99,6 @@ __device__ __forceinline__ float4 ldcg4(const float *p) {
     return __ldcg(reinterpret_cast<const float4 *>(p));
 }
 
-__device__ __forceinline__ float bf16f(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
 
 // ------------------------------------------------------------------------- code formats ----
 // Codes per 16-byte chunk: int4 32, int8 16, int2 64.
@@ -154,88 +158,93 @@ __device__ __forceinline__ int idot_chunk<2>(const uint4 q, const int *xp, int c
     return (a[0] + a[1]) + (a[2] + a[3]);
 }
 
-// Float decode of codes at their bit position.  A code field u sitting at mantissa bits
-// [B*pos, B*pos + B) of a float whose exponent makes bit B*pos weigh exactly 1 (biased exponent
-// 150 - B*pos) reads as 2^(23 - B*pos) + u; subtracting 2^(23 - B*pos) + BIAS gives the
-// two's-complement code q = u - BIAS exactly (u is the code with its sign bit flipped).  Fields
-// above bit 19 are first shifted down by SHIFT so that every field stays inside the mantissa.
-template <int FMT> struct Fpos;
-template <> struct Fpos<4> {  // element k of a word: nibble k at bits 4k
-    static constexpr int SHIFT = 12, CUT = 5, BITS = 4, CPW = 8, BIAS = 8;
-    static constexpr uint32_t FLIP = 0x88888888u, MASK = 0xFu;
-};
-template <> struct Fpos<8> {  // element k: byte k at bits 8k
-    static constexpr int SHIFT = 16, CUT = 2, BITS = 8, CPW = 4, BIAS = 128;
-    static constexpr uint32_t FLIP = 0x80808080u, MASK = 0xFFu;
-};
-template <> struct Fpos<2> {  // element k: bits 2k
-    static constexpr int SHIFT = 10, CUT = 11, BITS = 2, CPW = 16, BIAS = 2;
-    static constexpr uint32_t FLIP = 0xAAAAAAAAu, MASK = 0x3u;
-};
-
-__device__ __forceinline__ uint64_t pack_b64(uint32_t lo, uint32_t hi) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
-    return r;
-}
-__device__ __forceinline__ uint64_t sub_f32x2(uint64_t a, uint64_t b) {
-    uint64_t r;
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-    return r;
-}
-__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t r;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-    return r;
-}
-
-// One word of codes against its four activation pairs: acc += decoded codes * h (packed pairs).
+// Phase 2 activations (h) as 30-bit fixed point split into two signed 16-bit halves,
+// m = hi * 2^15 + lo, with one power-of-two scale per chunk; both halves use the same code
+// extraction and the layout of idot_chunk.  Returns the two exact integer sums.
 template <int FMT>
-__device__ __forceinline__ uint64_t fdot_word(uint32_t w, const uint64_t *hw, uint64_t acc) {
-    using F = Fpos<FMT>;
-    const uint32_t f0 = w ^ F::FLIP;
-    const uint32_t f1 = f0 >> F::SHIFT;
+__device__ __forceinline__ void idot2_chunk(const uint4 q, const int *xh, const int *xl, int ch, int cl,
+                                            int &sh, int &sl);
+
+template <>
+__device__ __forceinline__ void idot2_chunk<4>(const uint4 q, const int *xh, const int *xl, int ch, int cl,
+                                               int &sh, int &sl) {
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    int h0 = -ch, h1 = 0, l0 = -cl, l1 = 0;
 #pragma unroll
-    for (int k = 0; k < F::CPW; k += 2) {
-        uint32_t bits[2];
-        float off[2];
-#pragma unroll
-        for (int d = 0; d < 2; ++d) {
-            const int kk = k + d;
-            const int pos = kk < F::CUT ? kk : kk - F::SHIFT / F::BITS;
-            const uint32_t src = kk < F::CUT ? f0 : f1;
-            bits[d] = (src & (F::MASK << (F::BITS * pos))) | (static_cast<uint32_t>(150 - F::BITS * pos) << 23);
-            off[d] = static_cast<float>(1u << (23 - F::BITS * pos)) + static_cast<float>(F::BIAS);
-        }
-        const uint64_t v = sub_f32x2(pack_b64(bits[0], bits[1]),
-                                     pack_b64(__float_as_uint(off[0]), __float_as_uint(off[1])));
-        acc = fma_f32x2(v, hw[k >> 1], acc);
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t f = w[i] ^ 0x88888888u;
+        const int lo = static_cast<int>(f & 0x0F0F0F0Fu);
+        const int hi = static_cast<int>((f >> 4) & 0x0F0F0F0Fu);
+        h0 = __dp2a_lo(xh[4 * i + 0], lo, h0);
+        l0 = __dp2a_lo(xl[4 * i + 0], lo, l0);
+        h1 = __dp2a_hi(xh[4 * i + 1], lo, h1);
+        l1 = __dp2a_hi(xl[4 * i + 1], lo, l1);
+        h0 = __dp2a_lo(xh[4 * i + 2], hi, h0);
+        l0 = __dp2a_lo(xl[4 * i + 2], hi, l0);
+        h1 = __dp2a_hi(xh[4 * i + 3], hi, h1);
+        l1 = __dp2a_hi(xl[4 * i + 3], hi, l1);
     }
-    return acc;
+    sh = h0 + h1;
+    sl = l0 + l1;
+}
+template <>
+__device__ __forceinline__ void idot2_chunk<8>(const uint4 q, const int *xh, const int *xl, int, int,
+                                               int &sh, int &sl) {
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    int h0 = 0, h1 = 0, l0 = 0, l1 = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        h0 = __dp2a_lo(xh[2 * i + 0], static_cast<int>(w[i]), h0);
+        l0 = __dp2a_lo(xl[2 * i + 0], static_cast<int>(w[i]), l0);
+        h1 = __dp2a_hi(xh[2 * i + 1], static_cast<int>(w[i]), h1);
+        l1 = __dp2a_hi(xl[2 * i + 1], static_cast<int>(w[i]), l1);
+    }
+    sh = h0 + h1;
+    sl = l0 + l1;
+}
+template <>
+__device__ __forceinline__ void idot2_chunk<2>(const uint4 q, const int *xh, const int *xl, int ch, int cl,
+                                               int &sh, int &sl) {
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    int h[2] = {-ch, 0}, l[2] = {-cl, 0};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t f = w[i] ^ 0xAAAAAAAAu;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int bb = static_cast<int>((f >> (2 * k)) & 0x03030303u);
+            h[k & 1] = __dp2a_lo(xh[8 * i + 2 * k + 0], bb, h[k & 1]);
+            l[k & 1] = __dp2a_lo(xl[8 * i + 2 * k + 0], bb, l[k & 1]);
+            h[k & 1] = __dp2a_hi(xh[8 * i + 2 * k + 1], bb, h[k & 1]);
+            l[k & 1] = __dp2a_hi(xl[8 * i + 2 * k + 1], bb, l[k & 1]);
+        }
+    }
+    sh = h[0] + h[1];
+    sl = l[0] + l[1];
 }
 
-__device__ __forceinline__ float sum_pair(uint64_t v) {
-    return __fadd_rn(__uint_as_float(static_cast<uint32_t>(v)), __uint_as_float(static_cast<uint32_t>(v >> 32)));
-}
-
-// Dots of two chunks of codes (two rows) with the same activations, four independent chains.
-// hr holds the chunk's activations as float pairs (element 2i in the low half); element k of a
-// word accumulates into the low lane for even k and the high lane for odd k; words 0-1 and 2-3
-// go to separate pairs, summed at the end.
+// Position in a chunk's packed 16-bit layout (word index and half) of chunk element j, matching
+// idot_chunk / idot2_chunk.
 template <int FMT>
-__device__ __forceinline__ void fdot2_chunk(const uint4 q0, const uint4 q1, const uint64_t *hr, float &d0, float &d1) {
-    constexpr int HP = Fpos<FMT>::CPW / 2;  // activation pairs per word
-    uint64_t a0 = 0ull, b0 = 0ull, a1 = 0ull, b1 = 0ull;
-    a0 = fdot_word<FMT>(q0.x, hr + 0 * HP, a0);
-    a1 = fdot_word<FMT>(q1.x, hr + 0 * HP, a1);
-    b0 = fdot_word<FMT>(q0.z, hr + 2 * HP, b0);
-    b1 = fdot_word<FMT>(q1.z, hr + 2 * HP, b1);
-    a0 = fdot_word<FMT>(q0.y, hr + 1 * HP, a0);
-    a1 = fdot_word<FMT>(q1.y, hr + 1 * HP, a1);
-    b0 = fdot_word<FMT>(q0.w, hr + 3 * HP, b0);
-    b1 = fdot_word<FMT>(q1.w, hr + 3 * HP, b1);
-    d0 = __fadd_rn(sum_pair(a0), sum_pair(b0));
-    d1 = __fadd_rn(sum_pair(a1), sum_pair(b1));
+__device__ __forceinline__ void pack_slot(int j, int &word, int &half);
+template <>
+__device__ __forceinline__ void pack_slot<4>(int j, int &word, int &half) {
+    const int i = j >> 3, k = j & 7;  // word i of codes, element k
+    // (m0,m2) (m4,m6) (m1,m3) (m5,m7)
+    const int sub = (k & 1) ? ((k >> 2) ? 3 : 2) : ((k >> 2) ? 1 : 0);
+    word = 4 * i + sub;
+    half = (k >> 1) & 1;
+}
+template <>
+__device__ __forceinline__ void pack_slot<8>(int j, int &word, int &half) {
+    word = j >> 1;
+    half = j & 1;
+}
+template <>
+__device__ __forceinline__ void pack_slot<2>(int j, int &word, int &half) {
+    const int i = j >> 4, r = j & 15, k = r & 3, jb = r >> 2;  // element 16i + 4jb + k
+    word = 8 * i + 2 * k + (jb >> 1);
+    half = jb & 1;
 }
 
 __device__ __forceinline__ float warp_allsum(float v) {
@@ -249,194 +258,143 @@ __device__ __forceinline__ bool beats(double va, int ia, double vb, int ib) {
     return va > vb || (va == vb && ia < ib);
 }
 
-// Route token t with the whole CTA (256 threads) and write ids/weights; smem scratch given.
-__device__ void route_token_cta(const DecodeParams &p, int t, double *cs, double *ss, double *gsc,
-                                int *kept, int *sel_id, double *sel_s) {
+constexpr int RMAX_BLOCKS = 8;  // E <= 256 on the fused path
+struct RouteSmem {
+    double btop1[RMAX_BLOCKS], btop2[RMAX_BLOCKS], gsc[32];
+    double cval[RMAX_BLOCKS * 8], cs[RMAX_BLOCKS * 8];  // per block: its K <= 8 best
+    int cid[RMAX_BLOCKS * 8], kept[32];
+    double sel_s[32];
+    int sel_id[32];
+    int out_id[8];
+    float out_w[8];
+};
+
+// Route token t with four consumer warps (w4 = warp index within the four, barrier id bar).
+// Experts are taken in blocks of 32 (one per lane); a group is a whole number of blocks (or
+// G = 1).  Per block: the two largest biased scores (group score) and the block's K best experts
+// by rank among its 32 lanes; the union of the kept blocks' K best (at most 32 candidates) is
+// ranked by one warp.  Selections, ties and weights are those of the per-token definition
+// (largest biased score, lower id on ties, weights from the unbiased scores renormalised in slot
+// order, times routed_scaling).  Writes the token's ids and weights into rs.
+__device__ void route_token(const DecodeParams &p, int t, int w4, int lane, int bar, RouteSmem &r) {
     const int E = p.f.E, K = p.f.K, G = p.G, TG = p.TG;
-    const int gs = E / G;
-    const int tid = threadIdx.x;
-    for (int e = tid; e < E; e += blockDim.x) {
+    const int gs = E / G, nb = E / 32, bpg = gs / 32;
+    const bool grouped = G > 1 && TG < G;
+    for (int bk = w4; bk < nb; bk += 4) {
+        const int e = bk * 32 + lane;
         const double l = static_cast<double>(__ldcg(p.logits + static_cast<size_t>(t) * E + e));
         const double s = 1.0 / (1.0 + exp(-l));
-        ss[e] = s;
-        cs[e] = s + static_cast<double>(p.bias[e]);
-    }
-    __syncthreads();
-    if (G > 1 && TG < G) {
-        for (int g = tid; g < G; g += blockDim.x) {
-            double a1 = -INFINITY, a2 = -INFINITY;
-            for (int e = g * gs; e < (g + 1) * gs; ++e) {
-                const double v = cs[e];
-                if (v > a1) { a2 = a1; a1 = v; }
-                else if (v > a2) { a2 = v; }
-            }
-            gsc[g] = a1 + a2;
-        }
-        __syncthreads();
-        for (int g = tid; g < G; g += blockDim.x) {
-            int r = 0;
-            for (int h = 0; h < G; ++h) r += beats(gsc[h], h, gsc[g], g);
-            kept[g] = r < TG;
-        }
-    } else {
-        for (int g = tid; g < G; g += blockDim.x) kept[g] = 1;
-    }
-    __syncthreads();
-    for (int e = tid; e < E; e += blockDim.x) {
-        if (!kept[e / gs]) continue;
-        const double v = cs[e];
-        int r = 0;
-        for (int g = 0; g < G; ++g) {
-            if (!kept[g]) continue;
-            for (int f = g * gs; f < (g + 1) * gs; ++f) r += beats(cs[f], f, v, e);
-        }
-        if (r < K) { sel_id[r] = e; sel_s[r] = ss[e]; }
-    }
-    __syncthreads();
-    if (tid < K) {
-        double denom = 0.0;
-        for (int k = 0; k < K; ++k) denom += sel_s[k];
-        p.ids[static_cast<size_t>(t) * K + tid] = sel_id[tid];
-        p.wts[static_cast<size_t>(t) * K + tid] = static_cast<float>((sel_s[tid] / denom) * p.rsf);
-    }
-}
-
-// Group the n = T*K <= 32 slots of the batch: warp 0 ranks the slots by (expert id, slot) with
-// shuffles (a stable sort), the unique list follows from the sorted order; every thread fills the
-// per-expert counts and offsets by scanning the n slots.
-__device__ void group_batch_cta(const DecodeParams &p, int *sid, int *ssorted) {
-    const int E = p.f.E, n = p.f.T * p.f.K;
-    const int tid = threadIdx.x;
-    if (tid < 32) {
-        const int lane = tid;
-        const int id = lane < n ? __ldcg(p.ids + lane) : 0x7fffffff;
-        sid[lane] = id;
-        int r = 0;
-        for (int s2 = 0; s2 < 32; ++s2) {
-            const int o = __shfl_sync(FULL, id, s2);
-            r += (o < id) || (o == id && s2 < lane);
-        }
-        if (lane < n) {
-            p.f_perm[r] = lane;
-            ssorted[r] = id;
-        }
-        __syncwarp();
-        const int idr = lane < n ? ssorted[lane] : 0x7fffffff;
-        const bool first = lane < n && (lane == 0 || ssorted[lane - 1] != idr);
-        const unsigned m = __ballot_sync(FULL, first);
-        const int up = __popc(m & ((1u << lane) - 1u));
-        if (first) p.f_unique[up] = idr;
-        if (lane == 0) {
-            *p.f_nuniq = __popc(m);
-            p.f_offsets[E] = n;
-        }
-    }
-    __syncthreads();
-    for (int e = tid; e < E; e += blockDim.x) {
-        int c = 0, lt = 0;
-        for (int s2 = 0; s2 < n; ++s2) {
-            const int v = sid[s2];
-            c += v == e;
-            lt += v < e;
-        }
-        p.f_counts[e] = c;
-        p.f_offsets[e] = lt;
-    }
-    // unique entries past the last are -1: the number of distinct ids is known to every thread
-    int distinct = 0;
-    for (int s2 = 0; s2 < n; ++s2) distinct += (s2 == 0 || ssorted[s2 - 1] != ssorted[s2]);
-    for (int e = tid; e < E; e += blockDim.x)
-        if (e >= distinct) p.f_unique[e] = -1;
-}
-
-__global__ void __launch_bounds__(256) router_decode_kernel(DecodeParams p) {
-    grid_dep_launch();  // let the FFN kernel start streaming the shared expert
-    const int H = p.f.H, E = p.f.E;
-    const int t = blockIdx.y;
-    const int half = threadIdx.x >> 7, l = threadIdx.x & 127;
-    const int e = blockIdx.x * 2 + half;
-    __shared__ double red[8];
-    // a1: one Wr row per 128 threads, products and sums in double.  Loads are issued in groups
-    // of GB so that a thread's whole slice of the row is in flight at once (H <= GB * 512 * 2).
-    constexpr int GB = 6;
-    double acc = 0.0;
-    if (e < E) {
-        const float *wrow = p.Wr + static_cast<size_t>(e) * H;
-        for (int base = l * 4; base < H; base += GB * 512) {
-            float4 wv[GB];
-            float xv[GB][4];
+        const double c = s + static_cast<double>(p.bias[e]);
+        if (grouped) {
+            double a1 = c, a2 = -INFINITY;
 #pragma unroll
-            for (int g = 0; g < GB; ++g) {
-                const int h0 = base + g * 512;
-                if (h0 < H) {
-                    wv[g] = __ldg(reinterpret_cast<const float4 *>(wrow + h0));
-                    if (p.f.act == COLI_ACT_F32) {
-                        const float4 f4 = __ldg(reinterpret_cast<const float4 *>(static_cast<const float *>(p.f.x) + static_cast<size_t>(t) * H + h0));
-                        xv[g][0] = f4.x; xv[g][1] = f4.y; xv[g][2] = f4.z; xv[g][3] = f4.w;
-                    } else {
-                        const uint2 u = __ldg(reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(p.f.x) + static_cast<size_t>(t) * H + h0));
-                        xv[g][0] = __uint_as_float(u.x << 16); xv[g][1] = __uint_as_float(u.x & 0xffff0000u);
-                        xv[g][2] = __uint_as_float(u.y << 16); xv[g][3] = __uint_as_float(u.y & 0xffff0000u);
-                    }
-                } else {
-                    wv[g] = make_float4(0.f, 0.f, 0.f, 0.f);
-                    xv[g][0] = xv[g][1] = xv[g][2] = xv[g][3] = 0.f;
+            for (int o = 16; o > 0; o >>= 1) {
+                const double b1 = __shfl_xor_sync(FULL, a1, o);
+                const double b2 = __shfl_xor_sync(FULL, a2, o);
+                const double n1 = fmax(a1, b1);
+                const double n2 = fmax(fmin(a1, b1), fmax(a2, b2));
+                a1 = n1; a2 = n2;
+            }
+            if (lane == 0) { r.btop1[bk] = a1; r.btop2[bk] = a2; }
+        }
+        int rank = 0;
+        for (int o = 0; o < 32; ++o) {
+            const double oc = __shfl_sync(FULL, c, o);
+            rank += beats(oc, bk * 32 + o, c, e);
+        }
+        if (rank < K) {
+            r.cval[bk * K + rank] = c;
+            r.cs[bk * K + rank] = s;
+            r.cid[bk * K + rank] = e;
+        }
+    }
+    named_sync(bar, 128);
+    if (grouped) {
+        const int tid = w4 * 32 + lane;
+        for (int g = tid; g < G; g += 128) {
+            double a1 = -INFINITY, a2 = -INFINITY;
+            for (int bk = g * bpg; bk < (g + 1) * bpg; ++bk) {
+                const double v[2] = {r.btop1[bk], r.btop2[bk]};
+                for (int k = 0; k < 2; ++k) {
+                    if (v[k] > a1) { a2 = a1; a1 = v[k]; }
+                    else if (v[k] > a2) { a2 = v[k]; }
                 }
             }
+            r.gsc[g] = a1 + a2;
+        }
+        named_sync(bar, 128);
+        for (int g = tid; g < G; g += 128) {
+            int rk = 0;
+            for (int h = 0; h < G; ++h) rk += beats(r.gsc[h], h, r.gsc[g], g);
+            r.kept[g] = rk < TG;
+        }
+        named_sync(bar, 128);
+    }
+    if (w4 == 0) {
+        double c = -INFINITY, s = 0.0;
+        int id = 0x7fffffff;
+        int n = 0;
+        for (int bk = 0; bk < nb; ++bk) {
+            const bool keep = !grouped || r.kept[(bk * 32) / gs];
+            if (!keep) continue;
+            for (int k = 0; k < K; ++k, ++n)
+                if (n == lane) { c = r.cval[bk * K + k]; s = r.cs[bk * K + k]; id = r.cid[bk * K + k]; }
+        }
+        int rank = 0;
+        for (int o = 0; o < 32; ++o) {
+            const double oc = __shfl_sync(FULL, c, o);
+            const int oi = __shfl_sync(FULL, id, o);
+            rank += beats(oc, oi, c, id);
+        }
+        if (rank < K) { r.sel_s[rank] = s; r.sel_id[rank] = id; }
+        __syncwarp();
+        if (lane < K) {
+            double denom = 0.0;
+            for (int k = 0; k < K; ++k) denom += r.sel_s[k];
+            r.out_id[lane] = r.sel_id[lane];
+            r.out_w[lane] = static_cast<float>((r.sel_s[lane] / denom) * p.rsf);
+        }
+    }
+}
+
+// a1 only: grid (E, T), 128 threads; logit (t, e) summed in double from exact double products.
+__global__ void __launch_bounds__(128) gate_decode_kernel(DecodeParams p) {
+    grid_dep_launch();  // the FFN kernel starts streaming the shared expert right away
+    constexpr int GB = 6;
+    const int H = p.f.H, E = p.f.E;
+    const int e = blockIdx.x, t = blockIdx.y;
+    const int l = threadIdx.x;
+    __shared__ double red[4];
+    const float *wrow = p.Wr + static_cast<size_t>(e) * H;
+    const uint16_t *xrow = static_cast<const uint16_t *>(p.f.x) + static_cast<size_t>(t) * H;
+    double acc = 0.0;
+    for (int base = l * 4; base < H; base += GB * 512) {
+        float4 wv[GB];
+        uint2 xv[GB];
 #pragma unroll
-            for (int g = 0; g < GB; ++g) {
-                acc = fma(static_cast<double>(wv[g].x), static_cast<double>(xv[g][0]), acc);
-                acc = fma(static_cast<double>(wv[g].y), static_cast<double>(xv[g][1]), acc);
-                acc = fma(static_cast<double>(wv[g].z), static_cast<double>(xv[g][2]), acc);
-                acc = fma(static_cast<double>(wv[g].w), static_cast<double>(xv[g][3]), acc);
+        for (int g = 0; g < GB; ++g) {
+            const int h0 = base + g * 512;
+            if (h0 < H) {
+                wv[g] = __ldg(reinterpret_cast<const float4 *>(wrow + h0));
+                xv[g] = __ldg(reinterpret_cast<const uint2 *>(xrow + h0));
+            } else {
+                wv[g] = make_float4(0.f, 0.f, 0.f, 0.f);
+                xv[g] = make_uint2(0u, 0u);
             }
+        }
+#pragma unroll
+        for (int g = 0; g < GB; ++g) {
+            acc = fma(static_cast<double>(wv[g].x), static_cast<double>(__uint_as_float(xv[g].x << 16)), acc);
+            acc = fma(static_cast<double>(wv[g].y), static_cast<double>(__uint_as_float(xv[g].x & 0xffff0000u)), acc);
+            acc = fma(static_cast<double>(wv[g].z), static_cast<double>(__uint_as_float(xv[g].y << 16)), acc);
+            acc = fma(static_cast<double>(wv[g].w), static_cast<double>(__uint_as_float(xv[g].y & 0xffff0000u)), acc);
         }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(FULL, acc, o);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+    if ((l & 31) == 0) red[l >> 5] = acc;
     __syncthreads();
-    if (l == 0 && e < E) {
-        const double s = red[half * 4 + 0] + red[half * 4 + 1] + red[half * 4 + 2] + red[half * 4 + 3];
-        p.logits[static_cast<size_t>(t) * E + e] = static_cast<float>(s);
-    }
-    // last CTA of token t routes it; last token router groups the batch
-    __shared__ int last;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        const unsigned ticket = atomicAdd(p.tok_cnt + t, 1u);
-        last = ticket == gridDim.x - 1;
-    }
-    __syncthreads();
-    if (!last) return;
-    __threadfence();
-    extern __shared__ unsigned char dyn[];
-    double *cs = reinterpret_cast<double *>(dyn);
-    double *ss = cs + E;
-    double *gsc = ss + E;
-    double *sel_s = gsc + 32;
-    int *kept = reinterpret_cast<int *>(sel_s + 32);
-    int *sel_id = kept + 32;
-    route_token_cta(p, t, cs, ss, gsc, kept, sel_id, sel_s);
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        p.tok_cnt[t] = 0u;
-        __threadfence();
-        const unsigned ticket = atomicAdd(p.route_cnt, 1u);
-        last = ticket == gridDim.y - 1;
-    }
-    __syncthreads();
-    if (!last) return;
-    __threadfence();
-    int *sid = sel_id + 32;
-    int *ssorted = sid + 64;
-    group_batch_cta(p, sid, ssorted);
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        *p.route_cnt = 0u;
-        __threadfence();
-    }
+    if (l == 0) p.logits[static_cast<size_t>(t) * E + e] = static_cast<float>((red[0] + red[1]) + (red[2] + red[3]));
 }
 
 // ------------------------------------------------------------------------- K2 FFN ----------
@@ -463,11 +421,11 @@ __global__ void __maxnreg__(96) ffn_decode_kernel(DecodeParams p) {
     float *xs = reinterpret_cast<float *>(sm + p.off_xs);         // [T][Lh] scale
     int *xc = reinterpret_cast<int *>(sm + p.off_xc);             // [T][Lh] correction
     float *red2 = reinterpret_cast<float *>(sm + p.off_red);      // phase-2 partials
-    float4 *hb = reinterpret_cast<float4 *>(sm + p.off_x);        // phase-2 h (aliases x)
     unsigned char *ring = sm + p.off_ring;
     const uint32_t bar0 = smem_u32(bars);
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
+    const uint32_t route_bar = bar0 + 8u * (2 * S);  // consumers -> producer: routing cache ready
     const int Lh = p.Lh, Li = p.Li;
     const int PS = p.R1;                     // pairs per phase-1 stage
 
@@ -480,6 +438,7 @@ __global__ void __maxnreg__(96) ffn_decode_kernel(DecodeParams p) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), NCW);
         }
+        mbar_init(route_bar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
@@ -489,7 +448,7 @@ __global__ void __maxnreg__(96) ffn_decode_kernel(DecodeParams p) {
         if (lane != 0) return;
         const uint64_t pol = evict_first_policy();
         int seq = 0, U = 0;
-        int uniq[32];
+        int uniq[32] = {0};
         bool have_routing = false, ok = true;
         auto record = [&](int we) -> const uint8_t * {
             if (we < f.S) return f.shared;
@@ -498,10 +457,10 @@ __global__ void __maxnreg__(96) ffn_decode_kernel(DecodeParams p) {
         };
         for (int we = 0; ok; ++we) {
             if (we >= f.S && !have_routing) {
-                grid_dep_wait();
-                U = __ldcg(f.n_unique);
-                U = U < 0 ? 0 : (U > 32 ? 32 : U);
-                for (int u = 0; u < U; ++u) uniq[u] = __ldcg(f.unique + u);
+                if (!mbar_wait(route_bar, 0)) { ok = false; break; }
+                const int *rtc = reinterpret_cast<const int *>(sm + p.off_route);
+                U = rtc[0];
+                for (int u = 0; u < U; ++u) uniq[u] = rtc[RT_UNIQ + u];
                 have_routing = true;
             }
             if (have_routing && we >= f.S + U) break;
@@ -610,15 +569,78 @@ __global__ void __maxnreg__(96) ffn_decode_kernel(DecodeParams p) {
 
     // routing cache: [0] U; rBeg/rCnt per work expert; per slot: token, weight, h row
     int *rU = rt;
-    int *rBeg = rt + 1;
-    int *rCnt = rBeg + 33;
-    int *rTok = rCnt + 33;
-    float *rW = reinterpret_cast<float *>(rTok + 8 * 33);
-    int *rH = reinterpret_cast<int *>(rW + 8 * 33);
+    int *rBeg = rt + RT_BEG;
+    int *rCnt = rt + RT_CNT;
+    int *rTok = rt + RT_TOK;
+    float *rW = reinterpret_cast<float *>(rt + RT_W);
+    int *rH = rt + RT_H;
     bool have_routing = false;
+    int *rUniq = rt + RT_UNIQ;             // unique expert ids (for the producer)
+    RouteSmem *rsm = reinterpret_cast<RouteSmem *>(sm + p.off_x + static_cast<size_t>(T) * f.H * 2);
+    int *sorted_slot = rt + RT_SORT;
     auto get_routing = [&]() {
         grid_dep_wait();
-        if (cw == 0) {  // lane u handles unique expert u (U <= 32)
+        const int n = T * f.K;
+        if (p.route_here) {
+            // every CTA routes the batch from the logits (same code, same inputs, same result)
+            if (cw < 4 * T) route_token(p, cw >> 2, cw & 3, lane, 2 + (cw >> 2), rsm[cw >> 2]);
+            cons_sync();
+            if (cw == 0) {
+                const int s0 = lane;
+                const int id = s0 < n ? rsm[s0 / f.K].out_id[s0 % f.K] : 0x7fffffff;
+                int rk = 0;
+                for (int o = 0; o < 32; ++o) {
+                    const int oid = __shfl_sync(FULL, id, o);
+                    rk += (oid < id) || (oid == id && o < lane);
+                }
+                if (s0 < n) sorted_slot[rk] = s0;
+                __syncwarp();
+                const int sl = lane < n ? sorted_slot[lane] : 0;
+                const int idr = lane < n ? rsm[sl / f.K].out_id[sl % f.K] : 0x7fffffff;
+                const int idp = __shfl_up_sync(FULL, idr, 1);
+                const bool first = lane < n && (lane == 0 || idp != idr);
+                const unsigned m = __ballot_sync(FULL, first);
+                const int U = __popc(m);
+                const int up = __popc(m & ((1u << lane) - 1u));
+                if (first) {
+                    const unsigned rest = lane < 31 ? (m >> (lane + 1)) : 0u;
+                    const int nxt = rest ? lane + __ffs(rest) : n;
+                    rBeg[f.S + up] = lane;
+                    rCnt[f.S + up] = nxt - lane;
+                    rUniq[up] = idr;
+                }
+                if (lane < n) {
+                    rTok[lane] = sl / f.K;
+                    rW[lane] = rsm[sl / f.K].out_w[sl % f.K];
+                    rH[lane] = lane;
+                }
+                if (lane == 0) *rU = U;
+                if (blockIdx.x == 0) {  // the routing outputs of the call
+                    if (s0 < n) {
+                        p.ids[s0] = id;
+                        p.wts[s0] = rsm[s0 / f.K].out_w[s0 % f.K];
+                    }
+                    if (lane < n) p.f_perm[lane] = sl;
+                    if (first) p.f_unique[up] = idr;
+                    if (lane == 0) { *p.f_nuniq = U; p.f_offsets[f.E] = n; }
+                }
+            }
+            cons_sync();
+            if (blockIdx.x == 0) {
+                const int U = *rU;
+                for (int e = ct; e < f.E; e += NC) {
+                    int c = 0, lt = 0;
+                    for (int s2 = 0; s2 < n; ++s2) {
+                        const int v = rsm[s2 / f.K].out_id[s2 % f.K];
+                        c += v == e;
+                        lt += v < e;
+                    }
+                    p.f_counts[e] = c;
+                    p.f_offsets[e] = lt;
+                    if (e >= U) p.f_unique[e] = -1;
+                }
+            }
+        } else if (cw == 0) {  // routing given: lane u handles unique expert u (U <= 32)
             int U = __ldcg(f.n_unique);
             U = U < 0 ? 0 : (U > 32 ? 32 : U);
             int e = -1, b0 = 0, c0 = 0;
@@ -643,6 +665,7 @@ __global__ void __maxnreg__(96) ffn_decode_kernel(DecodeParams p) {
             if (lane < U) {
                 rBeg[f.S + lane] = pos;
                 rCnt[f.S + lane] = c0;
+                rUniq[lane] = e;
                 for (int q = 0; q < c0; ++q) {
                     const int sl = __ldcg(f.perm + b0 + q);
                     const bool good = sl >= 0 && sl < T * f.K;
@@ -654,6 +677,7 @@ __global__ void __maxnreg__(96) ffn_decode_kernel(DecodeParams p) {
             }
         }
         cons_sync();
+        if (ct == 0) mbar_arrive(route_bar);
         have_routing = true;
     };
     cons_sync();  // activations ready
@@ -755,10 +779,12 @@ __global__ void __maxnreg__(96) ffn_decode_kernel(DecodeParams p) {
     cons_sync();
 
     // ------------------------------------------------ phase 2: down + combine -------------
+    // h of one expert's slots is converted once per CTA into 29-bit fixed point split in two
+    // 16-bit halves per chunk (4 elements per thread, chunk maximum over 8 lanes), double
+    // buffered; the next expert's h is prefetched into registers while the current one is used.
     const int p2 = ct / Li, c2 = ct % Li;
     const int P2 = p.P2;
     const int nwr2 = Li / 32;
-    constexpr int HV = CPC / 4;              // float4 vectors of h per chunk
     float acc[RPT2MAX][TMAX];
 #pragma unroll
     for (int m = 0; m < RPT2MAX; ++m)
@@ -767,39 +793,91 @@ __global__ void __maxnreg__(96) ffn_decode_kernel(DecodeParams p) {
     const int nrows = j_hi - j_lo;
     const int a0d = j_lo & ~3;
     const int nwe = f.S + U;
-    // h of an expert's slots -> shared memory with cp.async, transposed: float4 vector v of
-    // chunk c of slot q at hb[buf][(q * HV + v) * Li + c]
-    const size_t hbuf = static_cast<size_t>(TMAX) * HV * Li;  // float4 per buffer
-    auto stage_h = [&](int we) {
+    // buffer layout (int4 vectors): [buf][slot][part hi/lo][XV][Li]; per (buf, slot, chunk):
+    // scale (float) and the two corrections
+    int4 *hq = reinterpret_cast<int4 *>(sm + p.off_x);
+    const size_t hq_buf = static_cast<size_t>(TMAX) * 2 * XV * Li;       // int4 per buffer
+    float *hsc = reinterpret_cast<float *>(sm + p.off_xs);                // [buf][slot][Li]
+    int *hcr = reinterpret_cast<int *>(sm + p.off_xc);                    // [buf][slot][2][Li]
+    const int ngrp = f.I / 4;                                              // 4-element groups per slot
+    float4 pre[TMAX];
+    auto fetch_h = [&](int we) {
         const bool shd = we < f.S;
         const int cnt = shd ? T : rCnt[we];
         const int beg = shd ? 0 : rBeg[we];
-        float4 *dstb = hb + (we & 1) * hbuf;
-        const int per = HV * Li;             // float4 per slot
-        for (int idx = ct; idx < cnt * per; idx += NC) {
-            const int q = idx / per, r = idx % per;
-            const int c = r / HV, v = r % HV;  // source order: chunk-major
-            const int hrow = shd ? T * f.K + q : rH[beg + q];
-            const uint32_t d = smem_u32(dstb + (static_cast<size_t>(q) * HV + v) * Li + c);
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d),
-                         "l"(f.h + static_cast<size_t>(hrow) * f.I + static_cast<size_t>(c) * CPC + 4 * v) : "memory");
+#pragma unroll
+        for (int q = 0; q < TMAX; ++q) {
+            if (q < cnt && ct < ngrp) {
+                const int hrow = shd ? T * f.K + q : rH[beg + q];
+                pre[q] = ldcg4(f.h + static_cast<size_t>(hrow) * f.I + 4 * ct);
+            }
         }
-        asm volatile("cp.async.commit_group;" ::: "memory");
     };
-    if (nwe > 0) stage_h(0);
+    auto convert_h = [&](int we, int buf) {
+        const bool shd = we < f.S;
+        const int cnt = shd ? T : rCnt[we];
+        const int c = ct >> 3, sub = ct & 7;  // 8 lanes per chunk of 32 elements (int4 codes)
+        constexpr int GPC = CPC / 4;          // 4-element groups per chunk
+#pragma unroll
+        for (int q = 0; q < TMAX; ++q) {
+            if (q < cnt) {
+                const bool act = ct < ngrp;
+                const float v[4] = {pre[q].x, pre[q].y, pre[q].z, pre[q].w};
+                float mx = act ? fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3]))) : 0.f;
+#pragma unroll
+                for (int o = GPC / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
+                int ex = mx > 0.f ? static_cast<int>((__float_as_uint(mx) >> 23) & 0xFF) - 126 : 0;
+                ex = max(ex, -96);                                          // mx < 2^ex
+                const float up = __uint_as_float(static_cast<uint32_t>(127 + 29 - ex) << 23);  // 2^(29-ex)
+                int sum_h = 0, sum_l = 0;
+                if (act) {
+                    const int cc = (4 * ct) / CPC;                          // chunk of these elements
+#pragma unroll
+                    for (int e2 = 0; e2 < 4; ++e2) {
+                        const int j = (4 * ct + e2) % CPC;
+                        const float sc = __fmul_rn(v[e2], up);               // |sc| < 2^29
+                        const float th = __fmaf_rn(sc, 1.0f / 32768.0f, 12582912.0f);
+                        const int hi = static_cast<int>(__float_as_uint(th)) - 0x4B400000;
+                        const float r = __fmaf_rn(-__fsub_rn(th, 12582912.0f), 32768.0f, sc);  // exact
+                        const float tl = __fadd_rn(r, 12582912.0f);
+                        const int lo = static_cast<int>(__float_as_uint(tl)) - 0x4B400000;
+                        sum_h += hi;
+                        sum_l += lo;
+                        int word, half;
+                        pack_slot<FMT>(j, word, half);
+                        int16_t *ph = reinterpret_cast<int16_t *>(hq + buf * hq_buf + ((static_cast<size_t>(q) * 2 + 0) * XV + (word >> 2)) * Li + cc);
+                        int16_t *pl = reinterpret_cast<int16_t *>(hq + buf * hq_buf + ((static_cast<size_t>(q) * 2 + 1) * XV + (word >> 2)) * Li + cc);
+                        ph[2 * (word & 3) + half] = static_cast<int16_t>(hi);
+                        pl[2 * (word & 3) + half] = static_cast<int16_t>(lo);
+                    }
+                }
+#pragma unroll
+                for (int o = GPC / 2; o > 0; o >>= 1) {
+                    sum_h += __shfl_xor_sync(FULL, sum_h, o);
+                    sum_l += __shfl_xor_sync(FULL, sum_l, o);
+                }
+                if (act && (ct % GPC) == 0) {
+                    const int cc = (4 * ct) / CPC;
+                    const int bias = FMT == 4 ? 8 : (FMT == 2 ? 2 : 0);
+                    hsc[(buf * TMAX + q) * Li + cc] = __uint_as_float(static_cast<uint32_t>(127 - 29 + ex) << 23);
+                    hcr[((buf * TMAX + q) * 2 + 0) * Li + cc] = bias * sum_h;
+                    hcr[((buf * TMAX + q) * 2 + 1) * Li + cc] = bias * sum_l;
+                }
+                (void)c; (void)sub;
+            }
+        }
+    };
+    if (nwe > 0) {
+        fetch_h(0);
+        convert_h(0, 0);
+    }
+    cons_sync();
     for (int we = 0; we < nwe; ++we) {
         const bool shared = we < f.S;
         const int cnt = shared ? T : rCnt[we];
         const int beg = shared ? 0 : rBeg[we];
-        cons_sync();                               // everyone is done with buffer (we+1)&1
-        if (we + 1 < nwe) {
-            stage_h(we + 1);
-            asm volatile("cp.async.wait_group 1;" ::: "memory");
-        } else {
-            asm volatile("cp.async.wait_group 0;" ::: "memory");
-        }
-        cons_sync();                               // buffer we&1 is complete
-        const float4 *hcur = hb + (we & 1) * hbuf;
+        const int buf = we & 1;
+        if (we + 1 < nwe) fetch_h(we + 1);
         const int s = seq % S;
         const uint32_t par = (seq / S) & 1;
         ++seq;
@@ -810,35 +888,37 @@ __global__ void __maxnreg__(96) ffn_decode_kernel(DecodeParams p) {
             for (int q = 0; q < cnt; ++q) {
                 const int tok = shared ? q : rTok[beg + q];
                 const float wq = shared ? 1.0f : rW[beg + q];
-                uint64_t hr[CPC / 2];
+                int xh[XW], xl[XW];
 #pragma unroll
-                for (int v = 0; v < HV; ++v) {
-                    const ulonglong2 t2 = *reinterpret_cast<const ulonglong2 *>(hcur + (static_cast<size_t>(q) * HV + v) * Li + c2);
-                    hr[2 * v] = t2.x; hr[2 * v + 1] = t2.y;
+                for (int v = 0; v < XV; ++v) {
+                    const int4 a4 = hq[buf * hq_buf + ((static_cast<size_t>(q) * 2 + 0) * XV + v) * Li + c2];
+                    const int4 b4 = hq[buf * hq_buf + ((static_cast<size_t>(q) * 2 + 1) * XV + v) * Li + c2];
+                    xh[4 * v] = a4.x; xh[4 * v + 1] = a4.y; xh[4 * v + 2] = a4.z; xh[4 * v + 3] = a4.w;
+                    xl[4 * v] = b4.x; xl[4 * v + 1] = b4.y; xl[4 * v + 2] = b4.z; xl[4 * v + 3] = b4.w;
                 }
+                const float hs = hsc[(buf * TMAX + q) * Li + c2];
+                const int ch = hcr[((buf * TMAX + q) * 2 + 0) * Li + c2];
+                const int cl = hcr[((buf * TMAX + q) * 2 + 1) * Li + c2];
 #pragma unroll
-                for (int m = 0; m < RPT2MAX; m += 2) {
-                    const int row0 = p2 + P2 * m, row1 = row0 + P2;
-                    if (row0 < nrows) {
-                        const bool has1 = row1 < nrows;
-                        const uint4 qd0 = lds128(st + static_cast<size_t>(row0) * f.rb_i + c2 * 16);
-                        const uint4 qd1 = has1 ? lds128(st + static_cast<size_t>(row1) * f.rb_i + c2 * 16) : make_uint4(0, 0, 0, 0);
-                        const float wsd0 = __fmul_rn(wq, sdp[row0]);
-                        const float wsd1 = has1 ? __fmul_rn(wq, sdp[row1]) : 0.f;
-                        float d0, d1;
-                        fdot2_chunk<FMT>(qd0, qd1, hr, d0, d1);
+                for (int m = 0; m < RPT2MAX; ++m) {
+                    const int row = p2 + P2 * m;
+                    if (row < nrows) {
+                        const uint4 qd = lds128(st + static_cast<size_t>(row) * f.rb_i + c2 * 16);
+                        int sh, sl;
+                        idot2_chunk<FMT>(qd, xh, xl, ch, cl, sh, sl);
+                        const float d = __fmul_rn(__fmaf_rn(static_cast<float>(sh), 32768.0f, static_cast<float>(sl)), hs);
+                        const float wsd = __fmul_rn(wq, sdp[row]);
 #pragma unroll
                         for (int t2 = 0; t2 < TMAX; ++t2)
-                            if (t2 == tok) {
-                                acc[m][t2] = __fmaf_rn(d0, wsd0, acc[m][t2]);
-                                acc[m + 1][t2] = __fmaf_rn(d1, wsd1, acc[m + 1][t2]);
-                            }
+                            if (t2 == tok) acc[m][t2] = __fmaf_rn(d, wsd, acc[m][t2]);
                     }
                 }
             }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(empty_bar(s));
+        if (we + 1 < nwe) convert_h(we + 1, buf ^ 1);
+        cons_sync();
     }
     if (!ok) atomicOr(f.err, COLI_DEVERR_TIMEOUT);
     // cross-lane reduction of the accumulators, then one store per (token, row)
@@ -914,7 +994,17 @@ bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan) {
     if (T < 1 || T > 4) return false;
     if (c.act != COLI_ACT_BF16) return false;  // 16-bit block fixed point is exact for bf16 only
     if (c.n_experts > 1024 || c.top_k * T > 32 || c.n_group > 32) return false;
-    if (c.hidden % 512) return false;
+    if (c.hidden % 512 || c.hidden > 12 * 512) return false;
+    // router blocks of 32 experts: groups are whole blocks, at most 32 candidates, K <= 8
+    if (c.n_experts % 32 || c.n_experts > 32 * RMAX_BLOCKS || c.top_k > 8) return false;
+    {
+        const int gs = c.n_experts / c.n_group;
+        const bool grouped = c.n_group > 1 && c.topk_group < c.n_group;
+        if (grouped && gs % 32) return false;
+        const int kept_blocks = grouped ? c.topk_group * gs / 32 : c.n_experts / 32;
+        if (kept_blocks * c.top_k > 32) return false;
+    }
+    if (c.inter > 4 * NC) return false;  // phase-2 conversion: 4 elements per consumer thread
     const int sms = device_sm_count();
     const int rb_h = c.hidden * c.wfmt / 8, rb_i = c.inter * c.wfmt / 8;
     const int Lh = rb_h / 16, Li = rb_i / 16;
@@ -944,11 +1034,13 @@ bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan) {
     size_t o = 1024;  // barriers (up to 64 stages)
     pl.off_route = o; o += 4096;
     pl.off_x = o;
-    const size_t xbytes = static_cast<size_t>(T) * c.hidden * 2;
+    const size_t xbytes = static_cast<size_t>(T) * c.hidden * 2 + static_cast<size_t>(T) * sizeof(RouteSmem);
     const size_t hbytes = static_cast<size_t>(2) * tmax * c.inter * 4;  // two buffers of TMAX h rows
     o += ((xbytes > hbytes ? xbytes : hbytes) + 127) / 128 * 128;
-    pl.off_xs = o; o += static_cast<size_t>(T) * Lh * 4;
-    pl.off_xc = o; o += static_cast<size_t>(T) * Lh * 4;
+    // x scales / corrections (phase 1) or h scales / corrections (phase 2)
+    const size_t xsb = static_cast<size_t>(T) * Lh * 4, hsb = static_cast<size_t>(2) * tmax * Li * 4;
+    pl.off_xs = o; o += (xsb > hsb ? xsb : hsb);
+    pl.off_xc = o; o += (xsb > 2 * hsb ? xsb : 2 * hsb);
     o = (o + 127) / 128 * 128;
     pl.red1_len = 0;
     const int red2_len = P2 * RPT2MAX * tmax * (Li / 32);
@@ -980,12 +1072,8 @@ cudaError_t launch_ffn_decode(DecodeParams p, const DecodePlan &pl, cudaStream_t
 }
 
 cudaError_t launch_router_decode(DecodeParams p, cudaStream_t st) {
-    const int E = p.f.E;
-    const size_t smem = static_cast<size_t>(E) * 16 + 64 * 8 + (32 + 32 + 64) * 4 + static_cast<size_t>(3 * E + 1) * 4 + 64;
-    cudaError_t e = cudaFuncSetAttribute(router_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    dim3 grid((E + 1) / 2, p.f.T);
-    router_decode_kernel<<<grid, 256, smem, st>>>(p);
+    dim3 grid(p.f.E, p.f.T);
+    gate_decode_kernel<<<grid, 128, 0, st>>>(p);
     return cudaGetLastError();
 }
 

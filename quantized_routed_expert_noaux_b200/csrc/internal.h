@@ -56,6 +56,7 @@ struct DecodeParams {
     double rsf;
     int G, TG;
     unsigned *tok_cnt, *route_cnt, *gbar, *gdep;
+    int route_here;  // 1: the FFN kernel routes from logits; 0: routing arrays are inputs
     // K2 plan (copied from DecodePlan)
     int grid, Lh, Li, P1, P2, R1, S, SB;
     int st_up, st_sg, st_su, st_sd;

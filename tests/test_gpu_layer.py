@@ -261,13 +261,20 @@ def test_layer_alternate_containers_sampled(name):
 @pytest.mark.parametrize("name,T", [("tiny", 8), ("glm_decode", 4), ("olmoe", 32)])
 def test_batch_union_equals_per_token_bitwise(name, T):
     """The batch reads each unique expert once, yet every token's output is bit-identical to
-    the token run alone."""
+    the token run alone whenever both calls take the same kernels (the fused decode path and the
+    general path differ in their exact rounding; across them the outputs agree within the
+    float32-accumulate tolerance)."""
     L = layer_for(name)
+    cfg = q.config_for(L.wl)
+    same_path = q.coli_moe_layer_kernels(cfg, T) == q.coli_moe_layer_kernels(cfg, 1)
     x = synth.make_activations(L.wl, T, device="cuda", step=11)
     out, _, _ = run_layer(L, x, T)
     for t in range(T):
         o1, _, _ = run_layer(L, x[t:t + 1].contiguous(), 1)
-        np.testing.assert_array_equal(o1[0], out[t])
+        if same_path:
+            np.testing.assert_array_equal(o1[0], out[t])
+        else:
+            assert normwise_err(o1, out[t:t + 1]) <= TOL_GEMV
 
 
 @pytest.mark.parametrize("T", [1, 4])
