@@ -165,7 +165,7 @@ coli_status coli_moe_layer_kernels(const coli_moe_config *c, int T, int *n_kerne
     if (s != COLI_OK) return s;
     if (T < 0) return COLI_ERR_SHAPE;
     DecodePlan pl;
-    *n_kernels = T == 0 ? 0 : (decode_plan(*c, T, &pl) ? 2 : 5);
+    *n_kernels = T == 0 ? 0 : (decode_plan(*c, T, &pl) ? 1 : 5);
     return COLI_OK;
 }
 
@@ -258,7 +258,7 @@ static DecodeParams make_decode(const coli_moe_config *c, const FfnParams &f, ch
 // the general GEMV kernels.
 static coli_status run_ffn(const coli_moe_config *c, const FfnParams &p, char *base, cudaStream_t st) {
     DecodePlan pl;
-    if (decode_plan(*c, p.T, &pl)) return from_cuda(launch_ffn_decode(make_decode(c, p, base), pl, st, false));
+    if (decode_plan(*c, p.T, &pl)) return from_cuda(launch_ffn_decode(make_decode(c, p, base), pl, st));
     return from_cuda(launch_ffn_gemv(p, st));
 }
 
@@ -315,7 +315,7 @@ coli_status coli_moe_layer(const coli_moe_config *c, const coli_moe_weights *w, 
                               reinterpret_cast<float *>(base + L.h), err);
     DecodePlan pl;
     if (decode_plan(*c, T, &pl)) {
-        // fused decode path: router kernel, then the FFN kernel as its programmatic dependent
+        // fused decode path: one persistent kernel (gate, route, group, FFN, combine)
         DecodeParams d = make_decode(c, p, base);
         d.Wr = w->router_w;
         d.bias = w->router_bias;
@@ -328,9 +328,7 @@ coli_status coli_moe_layer(const coli_moe_config *c, const coli_moe_weights *w, 
         d.f_unique = uniq;
         d.f_nuniq = nu;
         d.route_here = 1;
-        cudaError_t e = launch_router_decode(d, st);
-        if (e == cudaSuccess) e = launch_ffn_decode(d, pl, st, true);
-        return from_cuda(e);
+        return from_cuda(launch_ffn_decode(d, pl, st));
     }
     cudaError_t e = launch_gate(*c, w->router_w, x, T, logits, st);
     if (e == cudaSuccess) e = launch_route(*c, logits, w->router_bias, T, ids, wts, st);

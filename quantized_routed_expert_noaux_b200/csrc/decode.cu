@@ -1,15 +1,14 @@
 // decode.cu -- the fused decode path of the layer for a few tokens (decode and MTP verify).
 //
-// Two launches, the second one programmatically dependent on the first:
+// One persistent launch, one CTA per SM (ffn_decode_kernel):
 //
-//  K1 gate_decode_kernel    a1 gate on grid (E, T): one Wr row per CTA, products and sums in
-//                           double.  Light enough to share every SM with the FFN kernel.
-//                           Every FFN CTA then routes the batch itself from the logits (a2,
-//                           noaux_tc, colibri-strix README "What's implemented") and groups it
-//                           (a3, batch-union): the same code on the same inputs, so all CTAs agree
-//                           bit for bit and no CTA waits on another; CTA 0 writes the routing
-//                           outputs of the call.
-//  K2 ffn_decode_kernel     a4..a7, persistent, one CTA per SM.  Warp 0 streams weight rows
+//  phase 0  a1 gate: CTA b computes the logits of experts [b*E/G, (b+1)*E/G) in double from
+//           exact double products and arrives on a grid counter.  After the shared expert's
+//           gate/up rows, every CTA waits for all logits and routes the batch itself (a2,
+//           noaux_tc, colibri-strix README "What's implemented") and groups it (a3, batch-union):
+//           the same code on the same inputs, so all CTAs agree bit for bit; CTA 0 writes the
+//           routing outputs of the call.  (For coli_moe_ffn the routing arrays are inputs.)
+//  phases 1-2 (a4..a7).  Warp 0 streams weight rows
 //                           into a shared-memory ring with bulk asynchronous copies (TMA engine,
 //                           mbarrier completion); the other warps dequantise from the ring.
 //                           Phase 1 (gate/up) splits every expert's I rows evenly over the CTAs
@@ -86,7 +85,6 @@ __device__ __forceinline__ uint64_t evict_first_policy() {
     return p;
 }
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void cons_sync() { asm volatile("bar.sync %0, %1;" ::"n"(CONS_BAR), "n"(NC) : "memory"); }
 __device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 __device__ __forceinline__ uint4 lds128(const unsigned char *p) { return *reinterpret_cast<const uint4 *>(p); }
@@ -357,46 +355,6 @@ __device__ void route_token(const DecodeParams &p, int t, int w4, int lane, int 
     }
 }
 
-// a1 only: grid (E, T), 128 threads; logit (t, e) summed in double from exact double products.
-__global__ void __launch_bounds__(128) gate_decode_kernel(DecodeParams p) {
-    grid_dep_launch();  // the FFN kernel starts streaming the shared expert right away
-    constexpr int GB = 6;
-    const int H = p.f.H, E = p.f.E;
-    const int e = blockIdx.x, t = blockIdx.y;
-    const int l = threadIdx.x;
-    __shared__ double red[4];
-    const float *wrow = p.Wr + static_cast<size_t>(e) * H;
-    const uint16_t *xrow = static_cast<const uint16_t *>(p.f.x) + static_cast<size_t>(t) * H;
-    double acc = 0.0;
-    for (int base = l * 4; base < H; base += GB * 512) {
-        float4 wv[GB];
-        uint2 xv[GB];
-#pragma unroll
-        for (int g = 0; g < GB; ++g) {
-            const int h0 = base + g * 512;
-            if (h0 < H) {
-                wv[g] = __ldg(reinterpret_cast<const float4 *>(wrow + h0));
-                xv[g] = __ldg(reinterpret_cast<const uint2 *>(xrow + h0));
-            } else {
-                wv[g] = make_float4(0.f, 0.f, 0.f, 0.f);
-                xv[g] = make_uint2(0u, 0u);
-            }
-        }
-#pragma unroll
-        for (int g = 0; g < GB; ++g) {
-            acc = fma(static_cast<double>(wv[g].x), static_cast<double>(__uint_as_float(xv[g].x << 16)), acc);
-            acc = fma(static_cast<double>(wv[g].y), static_cast<double>(__uint_as_float(xv[g].x & 0xffff0000u)), acc);
-            acc = fma(static_cast<double>(wv[g].z), static_cast<double>(__uint_as_float(xv[g].y << 16)), acc);
-            acc = fma(static_cast<double>(wv[g].w), static_cast<double>(__uint_as_float(xv[g].y & 0xffff0000u)), acc);
-        }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(FULL, acc, o);
-    if ((l & 31) == 0) red[l >> 5] = acc;
-    __syncthreads();
-    if (l == 0) p.logits[static_cast<size_t>(t) * E + e] = static_cast<float>((red[0] + red[1]) + (red[2] + red[3]));
-}
-
 // ------------------------------------------------------------------------- K2 FFN ----------
 // Phase 1: a stage holds PS (gate row, up row) pairs of one expert; consumer warp w works on pair
 // w % PS of the stages whose sequence number is w / PS modulo NCW / PS, reduces its rows with
@@ -405,7 +363,7 @@ __global__ void __launch_bounds__(128) gate_decode_kernel(DecodeParams p) {
 // are done.  Phase 2: a stage holds the CTA's whole block of down rows of one expert; consumer
 // thread (p2, c2) owns chunk c2 of rows p2 + P2*m and keeps per-(row, token) partial sums in
 // registers across experts; one cross-lane reduction at the end.
-template <int FMT, int TMAX>
+template <int FMT, int TMAX, int NJ>
 __global__ void __maxnreg__(96) ffn_decode_kernel(DecodeParams p) {
     constexpr int CPC = Fmt<FMT>::CPC;       // codes per 16-byte chunk
     constexpr int XW = CPC / 2;              // int32 words of 16-bit activations per chunk
@@ -579,9 +537,15 @@ __global__ void __maxnreg__(96) ffn_decode_kernel(DecodeParams p) {
     RouteSmem *rsm = reinterpret_cast<RouteSmem *>(sm + p.off_x + static_cast<size_t>(T) * f.H * 2);
     int *sorted_slot = rt + RT_SORT;
     auto get_routing = [&]() {
-        grid_dep_wait();
         const int n = T * f.K;
         if (p.route_here) {
+            if (ct == 0) {  // every CTA's logits are written
+                const long long t0 = clock64();
+                while (ld_acquire(p.gbar) < static_cast<unsigned>(G)) {
+                    if (clock64() - t0 > WAIT_CYCLES) { atomicOr(f.err, COLI_DEVERR_TIMEOUT); break; }
+                }
+            }
+            cons_sync();
             // every CTA routes the batch from the logits (same code, same inputs, same result)
             if (cw < 4 * T) route_token(p, cw >> 2, cw & 3, lane, 2 + (cw >> 2), rsm[cw >> 2]);
             cons_sync();
@@ -640,7 +604,7 @@ __global__ void __maxnreg__(96) ffn_decode_kernel(DecodeParams p) {
                     if (e >= U) p.f_unique[e] = -1;
                 }
             }
-        } else if (cw == 0) {  // routing given: lane u handles unique expert u (U <= 32)
+        } else if (grid_dep_wait(), cw == 0) {  // routing given: lane u handles unique expert u
             int U = __ldcg(f.n_unique);
             U = U < 0 ? 0 : (U > 32 ? 32 : U);
             int e = -1, b0 = 0, c0 = 0;
@@ -682,10 +646,45 @@ __global__ void __maxnreg__(96) ffn_decode_kernel(DecodeParams p) {
     };
     cons_sync();  // activations ready
 
+    // phase 0 (layer calls): this CTA's share of the router gate, logits[t][e] in double from
+    // exact double products, then an arrival on the grid counter (the wait comes later, after
+    // the shared expert's rows, in get_routing)
+    if (p.route_here) {
+        const int e0 = static_cast<int>(static_cast<long>(f.E) * b / G), e1 = static_cast<int>(static_cast<long>(f.E) * (b + 1) / G);
+        double *gred = reinterpret_cast<double *>(sm + p.off_red);
+        for (int job = e0 * T; job < e1 * T; ++job) {
+            const int e = job / T, t = job % T;
+            const float *wrow = p.Wr + static_cast<size_t>(e) * f.H;
+            const uint16_t *xrow = static_cast<const uint16_t *>(f.x) + static_cast<size_t>(t) * f.H;
+            double acc = 0.0;
+            for (int h0 = ct * 4; h0 < f.H; h0 += NC * 4) {
+                const float4 wv = __ldg(reinterpret_cast<const float4 *>(wrow + h0));
+                const uint2 xv = __ldg(reinterpret_cast<const uint2 *>(xrow + h0));
+                acc = fma(static_cast<double>(wv.x), static_cast<double>(__uint_as_float(xv.x << 16)), acc);
+                acc = fma(static_cast<double>(wv.y), static_cast<double>(__uint_as_float(xv.x & 0xffff0000u)), acc);
+                acc = fma(static_cast<double>(wv.z), static_cast<double>(__uint_as_float(xv.y << 16)), acc);
+                acc = fma(static_cast<double>(wv.w), static_cast<double>(__uint_as_float(xv.y & 0xffff0000u)), acc);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(FULL, acc, o);
+            if (lane == 0) gred[cw] = acc;
+            cons_sync();
+            if (ct == 0) {
+                double sum = 0.0;
+                for (int w2 = 0; w2 < NCW; ++w2) sum += gred[w2];
+                p.logits[static_cast<size_t>(t) * f.E + e] = static_cast<float>(sum);
+            }
+            cons_sync();
+        }
+        if (ct == 0) {
+            __threadfence();
+            atomicAdd(p.gbar, 1u);
+        }
+    }
+
     // ------------------------------------------------ phase 1: gate/up, h = SiLU(g)*u -----
     // After a timed-out wait a thread keeps walking the same loops and barriers (skipping later
     // waits), so that no consumer is ever left alone at a named barrier.
-    const int NJ = Lh / 32;                  // chunks per lane in a row
     const int NGRP = NCW / PS;               // stage groups
     const int my_pair = cw % PS, my_grp = cw / PS;
     int seq = 0, U = 0;
@@ -718,7 +717,7 @@ __global__ void __maxnreg__(96) ffn_decode_kernel(DecodeParams p) {
                     xcb[q] = xc + tok * Lh + lane;
                 }
                 const unsigned char *rgl = rg + lane * 16, *rul = ru + lane * 16;
-#pragma unroll 2
+#pragma unroll
                 for (int j = 0; j < NJ; ++j) {
                     const uint4 qg = lds128(rgl + j * 512);
                     const uint4 qu = lds128(rul + j * 512);
@@ -764,10 +763,10 @@ __global__ void __maxnreg__(96) ffn_decode_kernel(DecodeParams p) {
     if (ct == 0) {
         __threadfence();
         atomicAdd(p.gbar, 1u);
+        const unsigned target = static_cast<unsigned>(G) * (p.route_here ? 2u : 1u);
         const long long t0 = clock64();
-        while (ld_acquire(p.gbar) < static_cast<unsigned>(G)) {
+        while (ld_acquire(p.gbar) < target) {
             if (clock64() - t0 > WAIT_CYCLES) { atomicOr(f.err, COLI_DEVERR_TIMEOUT); break; }
-            __nanosleep(64);
         }
         // the last CTA to leave the barrier zeroes both counters for the next call
         if (atomicAdd(p.gdep, 1u) == static_cast<unsigned>(G) - 1u) {
@@ -942,52 +941,52 @@ __global__ void __maxnreg__(96) ffn_decode_kernel(DecodeParams p) {
     }
 }
 
-template <int FMT, int TMAX>
-cudaError_t launch_k2(const DecodeParams &p, size_t smem, cudaStream_t st, bool pdl) {
-    auto kern = ffn_decode_kernel<FMT, TMAX>;
+template <int FMT, int TMAX, int NJ>
+cudaError_t launch_k2(const DecodeParams &p, size_t smem, cudaStream_t st) {
+    auto kern = ffn_decode_kernel<FMT, TMAX, NJ>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.grid);
-    cfg.blockDim = dim3(NT);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    int na = 0;
-    if (pdl) {
-        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[na].val.programmaticStreamSerializationAllowed = 1;
-        ++na;
-    }
-    cfg.attrs = attr;
-    cfg.numAttrs = na;
-    return cudaLaunchKernelEx(&cfg, kern, p);
+    kern<<<p.grid, NT, smem, st>>>(p);
+    return cudaGetLastError();
 }
 
-template <int FMT>
-cudaError_t launch_k2_t(const DecodeParams &p, size_t smem, cudaStream_t st, bool pdl) {
-    if (p.f.T <= 1) return launch_k2<FMT, 1>(p, smem, st, pdl);
-    if (p.f.T <= 2) return launch_k2<FMT, 2>(p, smem, st, pdl);
-    return launch_k2<FMT, 4>(p, smem, st, pdl);
+template <int FMT, int NJ>
+cudaError_t launch_k2_t(const DecodeParams &p, size_t smem, cudaStream_t st) {
+    if (p.f.T <= 1) return launch_k2<FMT, 1, NJ>(p, smem, st);
+    if (p.f.T <= 2) return launch_k2<FMT, 2, NJ>(p, smem, st);
+    return launch_k2<FMT, 4, NJ>(p, smem, st);
+}
+
+// The instantiated (format, chunks per lane) pairs: GLM-5.2 shapes (hidden 6144) in the three
+// containers and the OLMoE shape (hidden 2048) in int4.
+template <int FMT, int NJ>
+static bool fits_block_t(int T) {
+    cudaFuncAttributes fa;
+    cudaError_t e;
+    if (T <= 1) e = cudaFuncGetAttributes(&fa, ffn_decode_kernel<FMT, 1, NJ>);
+    else if (T <= 2) e = cudaFuncGetAttributes(&fa, ffn_decode_kernel<FMT, 2, NJ>);
+    else e = cudaFuncGetAttributes(&fa, ffn_decode_kernel<FMT, 4, NJ>);
+    return e == cudaSuccess && fa.maxThreadsPerBlock >= NT;
+}
+
+static bool kernel_fits(int fmt, int nj, int T) {
+    if (fmt == 4 && nj == 6) return fits_block_t<4, 6>(T);
+    if (fmt == 4 && nj == 2) return fits_block_t<4, 2>(T);
+    if (fmt == 8 && nj == 12) return fits_block_t<8, 12>(T);
+    if (fmt == 2 && nj == 3) return fits_block_t<2, 3>(T);
+    return false;
+}
+
+static cudaError_t launch_k2_any(const DecodeParams &p, size_t smem, cudaStream_t st) {
+    const int nj = p.Lh / 32;
+    if (p.f.fmt == 4 && nj == 6) return launch_k2_t<4, 6>(p, smem, st);
+    if (p.f.fmt == 4 && nj == 2) return launch_k2_t<4, 2>(p, smem, st);
+    if (p.f.fmt == 8 && nj == 12) return launch_k2_t<8, 12>(p, smem, st);
+    if (p.f.fmt == 2 && nj == 3) return launch_k2_t<2, 3>(p, smem, st);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace
-
-// The register allocation of a kernel instantiation bounds its block size: check it fits NT.
-template <int FMT, int TMAX>
-static bool fits_block() {
-    cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, ffn_decode_kernel<FMT, TMAX>) != cudaSuccess) return false;
-    return fa.maxThreadsPerBlock >= NT;
-}
-static bool kernel_fits(int fmt, int T) {
-    const int tm = T <= 1 ? 1 : (T <= 2 ? 2 : 4);
-#define COLI_FITS(F)                                                        \
-    if (fmt == F) return tm == 1 ? fits_block<F, 1>() : (tm == 2 ? fits_block<F, 2>() : fits_block<F, 4>());
-    COLI_FITS(4) COLI_FITS(8) COLI_FITS(2)
-#undef COLI_FITS
-    return false;
-}
 
 // Shape rules and the shared-memory plan of the fused decode path.
 bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan) {
@@ -1015,7 +1014,7 @@ bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan) {
     if (c.inter < sms || c.hidden < sms) return false;
     if (rows2 > P2 * RPT2MAX) return false;
     const int tmax = T <= 1 ? 1 : (T <= 2 ? 2 : 4);
-    if (!kernel_fits(c.wfmt, T)) return false;
+    if (!kernel_fits(c.wfmt, Lh / 32, T)) return false;
     DecodePlan pl;
     pl.grid = sms;
     pl.Lh = Lh; pl.Li = Li; pl.P1 = 0; pl.P2 = P2; pl.R1 = PS1;
@@ -1044,7 +1043,7 @@ bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan) {
     o = (o + 127) / 128 * 128;
     pl.red1_len = 0;
     const int red2_len = P2 * RPT2MAX * tmax * (Li / 32);
-    pl.off_red = o; o += static_cast<size_t>(red2_len) * 4;
+    pl.off_red = o; o += (static_cast<size_t>(red2_len) * 4 > NCW * 8 ? static_cast<size_t>(red2_len) * 4 : NCW * 8);
     o = (o + 1023) / 1024 * 1024;
     pl.off_ring = o;
     const size_t budget = device_smem_optin() - 1024;
@@ -1063,18 +1062,9 @@ static void fill_plan(DecodeParams &p, const DecodePlan &pl) {
     p.off_red = pl.off_red; p.off_ring = pl.off_ring; p.red1_len = pl.red1_len;
 }
 
-cudaError_t launch_ffn_decode(DecodeParams p, const DecodePlan &pl, cudaStream_t st, bool pdl) {
+cudaError_t launch_ffn_decode(DecodeParams p, const DecodePlan &pl, cudaStream_t st) {
     fill_plan(p, pl);
-    if (p.f.fmt == 4) return launch_k2_t<4>(p, pl.smem, st, pdl);
-    if (p.f.fmt == 8) return launch_k2_t<8>(p, pl.smem, st, pdl);
-    if (p.f.fmt == 2) return launch_k2_t<2>(p, pl.smem, st, pdl);
-    return cudaErrorInvalidValue;
-}
-
-cudaError_t launch_router_decode(DecodeParams p, cudaStream_t st) {
-    dim3 grid(p.f.E, p.f.T);
-    gate_decode_kernel<<<grid, 128, 0, st>>>(p);
-    return cudaGetLastError();
+    return launch_k2_any(p, pl.smem, st);
 }
 
 }  // namespace coli

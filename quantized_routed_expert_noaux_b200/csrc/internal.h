@@ -65,8 +65,7 @@ struct DecodeParams {
 };
 
 bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan);
-cudaError_t launch_router_decode(DecodeParams p, cudaStream_t st);
-cudaError_t launch_ffn_decode(DecodeParams p, const DecodePlan &pl, cudaStream_t st, bool pdl);
+cudaError_t launch_ffn_decode(DecodeParams p, const DecodePlan &pl, cudaStream_t st);
 
 // Workspace carve-up (all offsets 256-B aligned).
 struct WsLayout {
