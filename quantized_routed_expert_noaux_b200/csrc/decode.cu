@@ -657,13 +657,22 @@ __global__ void __maxnreg__(96) ffn_decode_kernel(DecodeParams p) {
             const float *wrow = p.Wr + static_cast<size_t>(e) * f.H;
             const uint16_t *xrow = static_cast<const uint16_t *>(f.x) + static_cast<size_t>(t) * f.H;
             double acc = 0.0;
-            for (int h0 = ct * 4; h0 < f.H; h0 += NC * 4) {
-                const float4 wv = __ldg(reinterpret_cast<const float4 *>(wrow + h0));
-                const uint2 xv = __ldg(reinterpret_cast<const uint2 *>(xrow + h0));
-                acc = fma(static_cast<double>(wv.x), static_cast<double>(__uint_as_float(xv.x << 16)), acc);
-                acc = fma(static_cast<double>(wv.y), static_cast<double>(__uint_as_float(xv.x & 0xffff0000u)), acc);
-                acc = fma(static_cast<double>(wv.z), static_cast<double>(__uint_as_float(xv.y << 16)), acc);
-                acc = fma(static_cast<double>(wv.w), static_cast<double>(__uint_as_float(xv.y & 0xffff0000u)), acc);
+            constexpr int GLD = 3;  // all of a thread's loads in flight together (H <= 3 * 2048)
+            float4 wv[GLD];
+            uint2 xv[GLD];
+#pragma unroll
+            for (int g = 0; g < GLD; ++g) {
+                const int h0 = ct * 4 + g * NC * 4;
+                const bool in = h0 < f.H;
+                wv[g] = in ? __ldg(reinterpret_cast<const float4 *>(wrow + h0)) : make_float4(0.f, 0.f, 0.f, 0.f);
+                xv[g] = in ? __ldg(reinterpret_cast<const uint2 *>(xrow + h0)) : make_uint2(0u, 0u);
+            }
+#pragma unroll
+            for (int g = 0; g < GLD; ++g) {
+                acc = fma(static_cast<double>(wv[g].x), static_cast<double>(__uint_as_float(xv[g].x << 16)), acc);
+                acc = fma(static_cast<double>(wv[g].y), static_cast<double>(__uint_as_float(xv[g].x & 0xffff0000u)), acc);
+                acc = fma(static_cast<double>(wv[g].z), static_cast<double>(__uint_as_float(xv[g].y << 16)), acc);
+                acc = fma(static_cast<double>(wv[g].w), static_cast<double>(__uint_as_float(xv[g].y & 0xffff0000u)), acc);
             }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(FULL, acc, o);
@@ -993,7 +1002,7 @@ bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan) {
     if (T < 1 || T > 4) return false;
     if (c.act != COLI_ACT_BF16) return false;  // 16-bit block fixed point is exact for bf16 only
     if (c.n_experts > 1024 || c.top_k * T > 32 || c.n_group > 32) return false;
-    if (c.hidden % 512 || c.hidden > 12 * 512) return false;
+    if (c.hidden % 512 || c.hidden > 3 * NC * 4) return false;
     // router blocks of 32 experts: groups are whole blocks, at most 32 candidates, K <= 8
     if (c.n_experts % 32 || c.n_experts > 32 * RMAX_BLOCKS || c.top_k > 8) return false;
     {
