@@ -30,6 +30,9 @@ int row_bytes(int n, int fmt) { return n * fmt / 8; }
 
 }  // namespace
 
+// Batches with many tokens per expert take the tensor-core grouped GEMM when its shape rules hold.
+static bool use_mma(const coli_moe_config *c, int T) { return T > MMA_MIN_TOKENS && mma_shape_ok(*c); }
+
 int device_sm_count() {
     static int cached[64] = {0};
     int dev = 0;
@@ -75,6 +78,7 @@ WsLayout ws_layout(const coli_moe_config &c, int T) {
     L.unique = o;   o = align256(o + E * 4);
     L.nuniq = o;    o = align256(o + 4);
     L.h = o;        o = align256(o + (n + static_cast<size_t>(T) * c.n_shared) * c.inter * 4);
+    L.tiles = o;    o = align256(o + (3 * static_cast<size_t>(mma_tiles_max(c, T)) + 1) * 4);
     L.total = o;
     return L;
 }
@@ -165,7 +169,7 @@ coli_status coli_moe_layer_kernels(const coli_moe_config *c, int T, int *n_kerne
     if (s != COLI_OK) return s;
     if (T < 0) return COLI_ERR_SHAPE;
     DecodePlan pl;
-    *n_kernels = T == 0 ? 0 : (decode_plan(*c, T, &pl) ? 1 : 5);
+    *n_kernels = T == 0 ? 0 : (decode_plan(*c, T, &pl) ? 1 : (use_mma(c, T) ? 6 : 5));
     return COLI_OK;
 }
 
@@ -257,6 +261,20 @@ static DecodeParams make_decode(const coli_moe_config *c, const FfnParams &f, ch
 // The expert half for a given routing: the fused decode kernel when the shape allows it, else
 // the general GEMV kernels.
 static coli_status run_ffn(const coli_moe_config *c, const FfnParams &p, char *base, cudaStream_t st) {
+    if (use_mma(c, p.T)) {
+        const WsLayout L = ws_layout(*c, p.T);
+        MmaParams m;
+        m.f = p;
+        m.hb = reinterpret_cast<__nv_bfloat16 *>(base + L.h);
+        m.ntiles_max = mma_tiles_max(*c, p.T);
+        int *tl = reinterpret_cast<int *>(base + L.tiles);
+        m.tile_u = tl;
+        m.tile_n0 = tl + m.ntiles_max;
+        m.tile_cnt = tl + 2 * m.ntiles_max;
+        m.ntiles = tl + 3 * m.ntiles_max;
+        m.n_routed_slots = c->n_experts;
+        return from_cuda(launch_ffn_mma(m, st));
+    }
     DecodePlan pl;
     if (decode_plan(*c, p.T, &pl)) return from_cuda(launch_ffn_decode(make_decode(c, p, base), pl, st));
     return from_cuda(launch_ffn_gemv(p, st));
@@ -274,7 +292,7 @@ coli_status coli_moe_ffn(const coli_moe_config *c, const coli_moe_weights *w, co
     if (s != COLI_OK) return s;
     if (!x || !topk_w || !offsets || !perm || !unique_ids || !n_unique || !out) return COLI_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(out, 16)) return COLI_ERR_ALIGN;
-    if (T > gemv_max_tokens(*c)) return COLI_ERR_UNSUPPORTED;
+    if (T > gemv_max_tokens(*c) && !use_mma(c, T)) return COLI_ERR_UNSUPPORTED;
     const WsLayout L = ws_layout(*c, T);
     if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return COLI_ERR_WORKSPACE;
     char *base = static_cast<char *>(ws);
@@ -296,7 +314,7 @@ coli_status coli_moe_layer(const coli_moe_config *c, const coli_moe_weights *w, 
     if (!aligned(x, 16) || !aligned(out, 16)) return COLI_ERR_ALIGN;
     if ((topk_ids_out && !aligned(topk_ids_out, 4)) || (topk_w_out && !aligned(topk_w_out, 4)))
         return COLI_ERR_ALIGN;
-    if (T > gemv_max_tokens(*c)) return COLI_ERR_UNSUPPORTED;
+    if (T > gemv_max_tokens(*c) && !use_mma(c, T)) return COLI_ERR_UNSUPPORTED;
     const WsLayout L = ws_layout(*c, T);
     if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return COLI_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -1,6 +1,7 @@
 // internal.h -- declarations shared by the translation units of libcoli_moe.so (not installed).
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -67,6 +68,22 @@ struct DecodeParams {
 bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan);
 cudaError_t launch_ffn_decode(DecodeParams p, const DecodePlan &pl, cudaStream_t st);
 
+// Parameters of the tensor-core grouped-GEMM path (ffn_mma.cu).
+struct MmaParams {
+    FfnParams f;
+    __nv_bfloat16 *hb;          // h in bf16, [(T*K + T*S)][I]
+    int *tile_u, *tile_n0, *tile_cnt, *ntiles;  // device-built tile table
+    int ntiles_max;
+    int n_routed_slots;         // work-expert index of the shared expert
+};
+
+int mma_tiles_max(const coli_moe_config &c, int T);
+bool mma_shape_ok(const coli_moe_config &c);
+cudaError_t launch_ffn_mma(MmaParams p, cudaStream_t st);
+
+// Batches above this many tokens take the tensor-core path when its shape rules hold.
+constexpr int MMA_MIN_TOKENS = 64;
+
 // Workspace carve-up (all offsets 256-B aligned).
 struct WsLayout {
     size_t err;      // int error word (+ pad)
@@ -78,7 +95,8 @@ struct WsLayout {
     size_t perm;     // [T*K] i32
     size_t unique;   // [E] i32
     size_t nuniq;    // [1] i32
-    size_t h;        // [(T*K+T*S)][I] f32
+    size_t h;        // [(T*K+T*S)][I] f32 (GEMV paths) or bf16 (tensor-core path)
+    size_t tiles;    // tensor-core tile table: 3 * ntiles_max + 1 ints
     size_t total;
 };
 

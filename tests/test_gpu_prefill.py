@@ -1,0 +1,98 @@
+"""GPU parity of the tensor-core grouped-GEMM path (batches above 64 tokens, int4 weights).
+
+h is rounded to bf16 before the down projection, so outputs are compared with the bf16-MMA
+tolerance (2e-3 normwise per token); routing and grouping stay bit-exact.  The oracle computes
+sampled tokens one by one (the layer is per-token).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests._common import TOL_MMA, Layer, normwise_err, oracle_gate
+
+pytestmark = pytest.mark.gpu
+
+q = pytest.importorskip("quantized_routed_expert_noaux_b200")
+
+_L = {}
+
+
+def layer(name):
+    if name not in _L:
+        _L.clear()
+        torch.cuda.empty_cache()
+        _L[name] = Layer(synth.WORKLOADS[name], "cuda", 0)
+    return _L[name]
+
+
+def _group_gpu(cfg, ids_dev, T, E, ws):
+    dev = lambda n: torch.empty(n, dtype=torch.int32, device="cuda")
+    counts, offsets, perm, uniq, nu = dev(E), dev(E + 1), dev(T * cfg.top_k), dev(E), dev(1)
+    q.coli_moe_group(cfg, ids_dev, T, counts, offsets, perm, uniq, nu, ws)
+    return offsets, perm, uniq, nu
+
+
+@pytest.mark.parametrize("T,routing", [(96, "oracle"), (300, "oracle"), (160, "one_expert"),
+                                       (65, "oracle")])
+def test_mma_ffn_matches_oracle(T, routing):
+    L = layer("glm_decode")
+    wl = L.wl
+    cfg = q.config_for(wl)
+    assert q.coli_moe_layer_kernels(cfg, T) == 6  # tensor-core path
+    ocfg = oracle.make_cfg(wl)
+    x = synth.make_activations(wl, T, device="cuda", step=30 + T)
+    if routing == "oracle":
+        lg = oracle_gate(ocfg, L.Wr.cpu(), x.cpu(), T)
+        ids_np, w_np = oracle.route(ocfg, lg, L.bias.cpu(), T)
+    else:
+        rng = np.random.default_rng(T)
+        ids_np = np.zeros((T, wl.top_k), np.int32)
+        for t in range(T):
+            others = rng.choice([e for e in range(wl.n_experts) if e != 3], wl.top_k - 1,
+                                replace=False)
+            ids_np[t] = [3] + list(others)
+        w_np = rng.uniform(0.1, 1.0, size=(T, wl.top_k)).astype(np.float32)
+    ws = torch.empty(q.coli_moe_workspace_size(cfg, T), dtype=torch.uint8, device="cuda")
+    q.coli_moe_clear_error(ws)
+    offsets, perm, uniq, nu = _group_gpu(cfg, torch.from_numpy(ids_np).cuda(), T, wl.n_experts, ws)
+    out = torch.full((T, wl.hidden), float("nan"), device="cuda")
+    q.coli_moe_ffn(cfg, L.weights(), x, T, torch.from_numpy(w_np).cuda(), offsets, perm, uniq,
+                   nu, out, ws)
+    assert q.coli_moe_error_word(ws) == 0
+    got = out.cpu().numpy()
+    assert np.isfinite(got).all()
+    toks = sorted(set([0, 1, T // 3, T // 2, T - 2, T - 1]))
+    ref = oracle.ffn(ocfg, L.host_records(ids_np[toks]), x.cpu()[toks], len(toks), ids_np[toks],
+                     w_np[toks])
+    err = normwise_err(got[toks], ref)
+    assert err <= TOL_MMA, err
+
+
+def test_prefill_layer_zipf_2048():
+    """The GLM-5.2-shaped prefill layer: 2048 tokens, Zipf(1.1) expert popularity."""
+    L = layer("glm_prefill")
+    wl = L.wl
+    T = 2048
+    cfg = q.config_for(wl)
+    x = synth.make_activations(wl, T, device="cuda", step=0)
+    out = torch.empty(T, wl.hidden, dtype=torch.float32, device="cuda")
+    ids = torch.empty(T, wl.top_k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, wl.top_k, dtype=torch.float32, device="cuda")
+    ws = torch.empty(q.coli_moe_workspace_size(cfg, T), dtype=torch.uint8, device="cuda")
+    q.coli_moe_clear_error(ws)
+    q.coli_moe_layer(cfg, L.weights(), x, T, out, ids, w, ws)
+    assert q.coli_moe_error_word(ws) == 0
+    ocfg = oracle.make_cfg(wl)
+    lg = oracle_gate(ocfg, L.Wr.cpu(), x.cpu(), T)
+    ids_ref, w_ref = oracle.route(ocfg, lg, L.bias.cpu(), T)
+    np.testing.assert_array_equal(ids.cpu().numpy(), ids_ref)
+    np.testing.assert_array_equal(w.cpu().numpy(), w_ref)
+    counts = np.bincount(ids_ref.reshape(-1), minlength=wl.n_experts)
+    assert counts.max() > 200  # Zipf head: several hundred tokens on the most popular expert
+    toks = [0, 7, 511, 1024, 1500, 2047]
+    recs = L.host_records(ids_ref[toks])
+    ref = oracle.ffn(ocfg, recs, x.cpu()[toks], len(toks), ids_ref[toks], w_ref[toks])
+    err = normwise_err(out.cpu().numpy()[toks], ref)
+    assert err <= TOL_MMA, err
