@@ -267,6 +267,40 @@ def gpu_arm(args, rank, world, dist):
         if d.get("source_hash") == cur:
             traffic = d.get("traffic_bytes_per_launch")
 
+    n_kern = q.coli_moe_layer_kernels(cfg, T)
+    if n_kern == 7:
+        # tensor-core path: int8 MMAs on two 8-bit activation slices, i.e. two int8 operations per
+        # algorithmic multiply-add -- the bf16 tensor rate; ~1 ms launches back to back -> sustained
+        ffn_flops = (T * wl.top_k + T * wl.n_shared) * 6.0 * wl.hidden * wl.inter
+        tf_s = ffn_flops / (ffn_ms / 1e3) / 1e12
+        peak_t = bf16s if bf16s else bf16
+        roofline = {
+            "bound": "tensor",
+            "kernel": "expert FFN (x quantisation, gate/up int8 GEMM, h quantisation, down int8 GEMM + combine)",
+            "achieved": round(tf_s, 1),
+            "peak": peak_t,
+            "unit": "TFLOP/s",
+            "frac": round(tf_s / peak_t, 4),
+            "traffic": traffic,
+            "peak_source": f"{peak_kind} bf16_tflops{'_sustained' if bf16s else ''} (int8 with two activation "
+                           "slices runs algorithmic flops at the bf16 rate)",
+            "launch_us": round(ffn_ms * 1e3, 2),
+            "hbm_gbs_of_weights": round(ffn_bytes / (ffn_ms / 1e3) / 1e9, 1),
+        }
+    else:
+        roofline = {
+            "bound": "hbm",
+            "kernel": ("fused decode layer kernel (FFN part)" if n_kern == 1
+                       else "expert FFN (gate/up GEMV + down GEMV with fused combine)"),
+            "achieved": round(achieved, 1),
+            "peak": hbm,
+            "unit": "GB/s",
+            "frac": round(achieved / hbm, 4),
+            "traffic": traffic,
+            "peak_source": f"{peak_kind} hbm_gbs (copy bandwidth)",
+            "launch_us": round(ffn_ms * 1e3, 2),
+        }
+
     res = {
         "metric": METRIC,
         "value": round(tok_s, 2),
@@ -292,21 +326,11 @@ def gpu_arm(args, rank, world, dist):
         "layer_gbs": round(bytes_steps / (ms_max / 1e3) / 1e9, 1),
         "layer_frac_of_hbm": round(bytes_steps / (ms_max / 1e3) / 1e9 / hbm, 4),
         "unique_experts_mean": round(float(U.mean()), 2),
-        "roofline": {
-            "bound": "hbm",
-            "kernel": "expert FFN (gate/up GEMV + down GEMV with fused combine)",
-            "achieved": round(achieved, 1),
-            "peak": hbm,
-            "unit": "GB/s",
-            "frac": round(achieved / hbm, 4),
-            "traffic": traffic,
-            "peak_source": f"{peak_kind} hbm_gbs (copy bandwidth)",
-            "launch_us": round(ffn_ms * 1e3, 2),
-        },
+        "roofline": roofline,
         "e2e": {"value": round(world * K2 * T / (e2e_ms / 1e3), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(xs[0].numel() * xs[0].element_size()),
                 "d2h_bytes_per_step": int(out.numel() * 4)},
-        "gpu_launches": q.coli_moe_layer_kernels(cfg, T) * K,
+        "gpu_launches": n_kern * K,
         "clocks": clk,
     }
     return res, (wl, T, layers, xs)

@@ -31,7 +31,7 @@ int row_bytes(int n, int fmt) { return n * fmt / 8; }
 }  // namespace
 
 // Batches with many tokens per expert take the tensor-core grouped GEMM when its shape rules hold.
-static bool use_mma(const coli_moe_config *c, int T) { return T > MMA_MIN_TOKENS && mma_shape_ok(*c); }
+static bool use_tc(const coli_moe_config *c, int T) { return T > TC_MIN_TOKENS && tc_shape_ok(*c); }
 
 int device_sm_count() {
     static int cached[64] = {0};
@@ -77,8 +77,18 @@ WsLayout ws_layout(const coli_moe_config &c, int T) {
     L.perm = o;     o = align256(o + n * 4);
     L.unique = o;   o = align256(o + E * 4);
     L.nuniq = o;    o = align256(o + 4);
-    L.h = o;        o = align256(o + (n + static_cast<size_t>(T) * c.n_shared) * c.inter * 4);
-    L.tiles = o;    o = align256(o + (3 * static_cast<size_t>(mma_tiles_max(c, T)) + 1) * 4);
+    const size_t slots = n + static_cast<size_t>(T) * c.n_shared;
+    L.h = o;        o = align256(o + slots * c.inter * 4);
+    const bool tc = use_tc(&c, T);
+    const size_t H = static_cast<size_t>(c.hidden), I = static_cast<size_t>(c.inter);
+    L.xq = o;       o = align256(o + (tc ? 2 * slots * H : 0));
+    L.hq = o;       o = align256(o + (tc ? 2 * slots * I : 0));
+    L.sx = o;       o = align256(o + (tc ? slots * 4 : 0));
+    L.sh = o;       o = align256(o + (tc ? slots * 4 : 0));
+    L.tok_of = o;   o = align256(o + (tc ? slots * 4 : 0));
+    L.w_of = o;     o = align256(o + (tc ? slots * 4 : 0));
+    L.chunks = o;   o = align256(o + (tc ? static_cast<size_t>(tc_max_chunks(c, T)) * 16 : 0));
+    L.n_chunks = o; o = align256(o + (tc ? 4 : 0));
     L.total = o;
     return L;
 }
@@ -169,7 +179,7 @@ coli_status coli_moe_layer_kernels(const coli_moe_config *c, int T, int *n_kerne
     if (s != COLI_OK) return s;
     if (T < 0) return COLI_ERR_SHAPE;
     DecodePlan pl;
-    *n_kernels = T == 0 ? 0 : (decode_plan(*c, T, &pl) ? 1 : (use_mma(c, T) ? 6 : 5));
+    *n_kernels = T == 0 ? 0 : (decode_plan(*c, T, &pl) ? 1 : (use_tc(c, T) ? 7 : 5));
     return COLI_OK;
 }
 
@@ -261,19 +271,20 @@ static DecodeParams make_decode(const coli_moe_config *c, const FfnParams &f, ch
 // The expert half for a given routing: the fused decode kernel when the shape allows it, else
 // the general GEMV kernels.
 static coli_status run_ffn(const coli_moe_config *c, const FfnParams &p, char *base, cudaStream_t st) {
-    if (use_mma(c, p.T)) {
+    if (use_tc(c, p.T)) {
         const WsLayout L = ws_layout(*c, p.T);
-        MmaParams m;
-        m.f = p;
-        m.hb = reinterpret_cast<__nv_bfloat16 *>(base + L.h);
-        m.ntiles_max = mma_tiles_max(*c, p.T);
-        int *tl = reinterpret_cast<int *>(base + L.tiles);
-        m.tile_u = tl;
-        m.tile_n0 = tl + m.ntiles_max;
-        m.tile_cnt = tl + 2 * m.ntiles_max;
-        m.ntiles = tl + 3 * m.ntiles_max;
-        m.n_routed_slots = c->n_experts;
-        return from_cuda(launch_ffn_mma(m, st));
+        TcBuffers b;
+        b.xq = reinterpret_cast<int8_t *>(base + L.xq);
+        b.hq = reinterpret_cast<int8_t *>(base + L.hq);
+        b.sx = reinterpret_cast<float *>(base + L.sx);
+        b.sh = reinterpret_cast<float *>(base + L.sh);
+        b.tok_of = reinterpret_cast<int *>(base + L.tok_of);
+        b.w_of = reinterpret_cast<float *>(base + L.w_of);
+        b.hbuf = reinterpret_cast<float *>(base + L.h);
+        b.chunks = reinterpret_cast<int4 *>(base + L.chunks);
+        b.n_chunks = reinterpret_cast<int *>(base + L.n_chunks);
+        b.max_chunks = tc_max_chunks(*c, p.T);
+        return from_cuda(launch_ffn_tc(p, b, st));
     }
     DecodePlan pl;
     if (decode_plan(*c, p.T, &pl)) return from_cuda(launch_ffn_decode(make_decode(c, p, base), pl, st));
@@ -292,7 +303,7 @@ coli_status coli_moe_ffn(const coli_moe_config *c, const coli_moe_weights *w, co
     if (s != COLI_OK) return s;
     if (!x || !topk_w || !offsets || !perm || !unique_ids || !n_unique || !out) return COLI_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(out, 16)) return COLI_ERR_ALIGN;
-    if (T > gemv_max_tokens(*c) && !use_mma(c, T)) return COLI_ERR_UNSUPPORTED;
+    if (T > gemv_max_tokens(*c) && !use_tc(c, T)) return COLI_ERR_UNSUPPORTED;
     const WsLayout L = ws_layout(*c, T);
     if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return COLI_ERR_WORKSPACE;
     char *base = static_cast<char *>(ws);
@@ -314,7 +325,7 @@ coli_status coli_moe_layer(const coli_moe_config *c, const coli_moe_weights *w, 
     if (!aligned(x, 16) || !aligned(out, 16)) return COLI_ERR_ALIGN;
     if ((topk_ids_out && !aligned(topk_ids_out, 4)) || (topk_w_out && !aligned(topk_w_out, 4)))
         return COLI_ERR_ALIGN;
-    if (T > gemv_max_tokens(*c) && !use_mma(c, T)) return COLI_ERR_UNSUPPORTED;
+    if (T > gemv_max_tokens(*c) && !use_tc(c, T)) return COLI_ERR_UNSUPPORTED;
     const WsLayout L = ws_layout(*c, T);
     if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return COLI_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);

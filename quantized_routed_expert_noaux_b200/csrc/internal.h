@@ -68,21 +68,25 @@ struct DecodeParams {
 bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan);
 cudaError_t launch_ffn_decode(DecodeParams p, const DecodePlan &pl, cudaStream_t st);
 
-// Parameters of the tensor-core grouped-GEMM path (ffn_mma.cu).
-struct MmaParams {
-    FfnParams f;
-    __nv_bfloat16 *hb;          // h in bf16, [(T*K + T*S)][I]
-    int *tile_u, *tile_n0, *tile_cnt, *ntiles;  // device-built tile table
-    int ntiles_max;
-    int n_routed_slots;         // work-expert index of the shared expert
+// Buffers of the tensor-core grouped-GEMM path (ffn_tc.cu), carved from the workspace.
+struct TcBuffers {
+    int8_t *xq;          // [2*slots][H]: x of each slot's token as 16-bit fixed point, hi/lo rows
+    int8_t *hq;          // [2*slots][I]: h of each slot, same encoding
+    float *sx, *sh;      // [slots]: row scales of xq, hq
+    int *tok_of;         // [slots]: token of the slot
+    float *w_of;         // [slots]: combine weight of the slot
+    float *hbuf;         // [slots][I]: h in float32
+    int4 *chunks;        // chunk table
+    int *n_chunks;
+    int max_chunks;
 };
 
-int mma_tiles_max(const coli_moe_config &c, int T);
-bool mma_shape_ok(const coli_moe_config &c);
-cudaError_t launch_ffn_mma(MmaParams p, cudaStream_t st);
+int tc_max_chunks(const coli_moe_config &c, int T);
+bool tc_shape_ok(const coli_moe_config &c);
+cudaError_t launch_ffn_tc(const FfnParams &f, const TcBuffers &b, cudaStream_t st);
 
 // Batches above this many tokens take the tensor-core path when its shape rules hold.
-constexpr int MMA_MIN_TOKENS = 64;
+constexpr int TC_MIN_TOKENS = 64;
 
 // Workspace carve-up (all offsets 256-B aligned).
 struct WsLayout {
@@ -95,8 +99,9 @@ struct WsLayout {
     size_t perm;     // [T*K] i32
     size_t unique;   // [E] i32
     size_t nuniq;    // [1] i32
-    size_t h;        // [(T*K+T*S)][I] f32 (GEMV paths) or bf16 (tensor-core path)
-    size_t tiles;    // tensor-core tile table: 3 * ntiles_max + 1 ints
+    size_t h;        // [(T*K+T*S)][I] f32 intermediate
+    // tensor-core path only (zero size otherwise)
+    size_t xq, hq, sx, sh, tok_of, w_of, chunks, n_chunks;
     size_t total;
 };
 

@@ -77,64 +77,115 @@ __global__ void __launch_bounds__(128) gate_rows_kernel(const float *__restrict_
 }
 
 // ---------------------------------------------------------------- a1 gate, many tokens -----
-// Tiled double-precision product logits[T,E] = X[T,H] * Wr[E,H]^T.  CTA tile 64 tokens x 64
-// experts, K step 16, 256 threads holding 4x4 double accumulators each.
-constexpr int GT_M = 64, GT_N = 64, GT_K = 16;
+// logits[T,E] = X[T,H] * Wr[E,H]^T on the fp64 tensor cores (mma.sync m8n8k4, double operands
+// and accumulators): every product of a bf16 or float32 activation and a float32 weight is exact
+// in double and sums are double, as in the per-row kernel above; only the summation order
+// differs.  CTA tile 64 tokens x 32 experts (4 warps of 32 x 16), K chunks of 32 staged in
+// shared memory as double, the next chunk's global loads in flight during the current chunk.
+constexpr int GM = 64, GN = 32, GK = 32;
+constexpr int GKP = GK + 4;  // row pitch (doubles): the 8 x 4 fragment reads hit each bank twice
+
+__device__ __forceinline__ void dmma(double &d0, double &d1, double a, double b) {
+    asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+                 : "+d"(d0), "+d"(d1) : "d"(a), "d"(b));
+}
 
 template <int ACT>
-__global__ void __launch_bounds__(256) gate_tiled_kernel(const float *__restrict__ Wr,
-                                                         const void *__restrict__ x, int T,
-                                                         int H, int E,
-                                                         float *__restrict__ logits) {
-    __shared__ double xs[GT_K][GT_M + 2];
-    __shared__ double ws[GT_K][GT_N + 2];
-    const int tid = threadIdx.x;
-    const int t0 = blockIdx.y * GT_M, e0 = blockIdx.x * GT_N;
-    const int tx = tid % 16, ty = tid / 16;  // 16 x 16 threads, 4 x 4 outputs each
-    double acc[4][4];
+__global__ void __launch_bounds__(128) gate_dmma_kernel(const float *__restrict__ Wr,
+                                                        const void *__restrict__ x, int T, int H,
+                                                        int E, float *__restrict__ logits) {
+    __shared__ double xs[GM][GKP];
+    __shared__ double ws[GN][GKP];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int t0 = blockIdx.y * GM, e0 = blockIdx.x * GN;
+    // staging: x row tid/2, k [16*(tid%2), +16); Wr row tid/4, k [8*(tid%4), +8)
+    const int xr = tid >> 1, xk = 16 * (tid & 1);
+    const int wr = tid >> 2, wk = 8 * (tid & 3);
+    const bool xok = t0 + xr < T, wok = e0 + wr < E;
+    float xv[16], wv[8];
+    auto load = [&](int k0) {
+        if (xok) {
+            if (ACT == COLI_ACT_F32) {
+                const float4 *p = reinterpret_cast<const float4 *>(static_cast<const float *>(x) +
+                                                                   static_cast<size_t>(t0 + xr) * H + k0 + xk);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float4 f = __ldg(p + i);
+                    xv[4 * i] = f.x; xv[4 * i + 1] = f.y; xv[4 * i + 2] = f.z; xv[4 * i + 3] = f.w;
+                }
+            } else {
+                const uint4 *p = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(x) +
+                                                                 static_cast<size_t>(t0 + xr) * H + k0 + xk);
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const uint4 u = __ldg(p + i);
+                    const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        xv[8 * i + 2 * j] = __uint_as_float(w4[j] << 16);
+                        xv[8 * i + 2 * j + 1] = __uint_as_float(w4[j] & 0xffff0000u);
+                    }
+                }
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) xv[i] = 0.f;
+        }
+        if (wok) {
+            const float4 *p = reinterpret_cast<const float4 *>(Wr + static_cast<size_t>(e0 + wr) * H + k0 + wk);
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const float4 f = __ldg(p + i);
+                wv[4 * i] = f.x; wv[4 * i + 1] = f.y; wv[4 * i + 2] = f.z; wv[4 * i + 3] = f.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) wv[i] = 0.f;
+        }
+    };
+    const int wm = warp & 1, wn = warp >> 1;  // warp tile: tokens [32*wm, +32), experts [16*wn, +16)
+    const int fr = lane >> 2, fk = lane & 3;  // fragment row (token / expert) and k of this lane
+    double acc[4][2][2];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = 0.0;
+        for (int j = 0; j < 2; ++j) acc[i][j][0] = acc[i][j][1] = 0.0;
 
-    for (int k0 = 0; k0 < H; k0 += GT_K) {
-        // 64 rows x 16 columns of each operand: 1024 elements, 4 per thread
-        for (int idx = tid; idx < GT_M * GT_K; idx += 256) {
-            const int r = idx / GT_K, k = idx % GT_K;
-            const int t = t0 + r, e = e0 + r;
-            double xv = 0.0, wv = 0.0;
-            if (t < T) {
-                if (ACT == COLI_ACT_F32)
-                    xv = static_cast<double>(static_cast<const float *>(x)[static_cast<size_t>(t) * H + k0 + k]);
-                else
-                    xv = static_cast<double>(bf16_to_f32(static_cast<const uint16_t *>(x)[static_cast<size_t>(t) * H + k0 + k]));
-            }
-            if (e < E) wv = static_cast<double>(Wr[static_cast<size_t>(e) * H + k0 + k]);
-            xs[k][r] = xv;
-            ws[k][r] = wv;
-        }
+    load(0);
+    for (int k0 = 0; k0 < H; k0 += GK) {
+        __syncthreads();  // the previous chunk's fragments have been read
+#pragma unroll
+        for (int i = 0; i < 16; ++i) xs[xr][xk + i] = static_cast<double>(xv[i]);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ws[wr][wk + i] = static_cast<double>(wv[i]);
         __syncthreads();
+        if (k0 + GK < H) load(k0 + GK);
 #pragma unroll
-        for (int k = 0; k < GT_K; ++k) {
-            double a[4], b[4];
+        for (int k4 = 0; k4 < GK; k4 += 4) {
+            double a[4], b[2];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) a[i] = xs[k][ty * 4 + i];
+            for (int i = 0; i < 4; ++i) a[i] = xs[32 * wm + 8 * i + fr][k4 + fk];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) b[j] = ws[k][tx * 4 + j];
+            for (int j = 0; j < 2; ++j) b[j] = ws[16 * wn + 8 * j + fr][k4 + fk];
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = fma(a[i], b[j], acc[i][j]);
+                for (int j = 0; j < 2; ++j) dmma(acc[i][j][0], acc[i][j][1], a[i], b[j]);
         }
-        __syncthreads();
     }
+    // accumulator (i, j): token 32*wm + 8*i + fr, experts 16*wn + 8*j + 2*fk + {0, 1}
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 4; ++i) {
+        const int t = t0 + 32 * wm + 8 * i + fr;
+        if (t >= T) continue;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int t = t0 + ty * 4 + i, e = e0 + tx * 4 + j;
-            if (t < T && e < E) logits[static_cast<size_t>(t) * E + e] = static_cast<float>(acc[i][j]);
-        }
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int e = e0 + 16 * wn + 8 * j + 2 * fk + h;
+                if (e < E) logits[static_cast<size_t>(t) * E + e] = static_cast<float>(acc[i][j][h]);
+            }
+    }
 }
 
 // ---------------------------------------------------------------- a2 route -----------------
@@ -338,11 +389,11 @@ cudaError_t launch_gate(const coli_moe_config &c, const float *Wr, const void *x
         else
             gate_rows_kernel<COLI_ACT_BF16, 8><<<grid, 128, 0, st>>>(Wr, x, T, H, E, logits);
     } else {
-        dim3 grid((E + GT_N - 1) / GT_N, (T + GT_M - 1) / GT_M);
+        dim3 grid((E + GN - 1) / GN, (T + GM - 1) / GM);
         if (c.act == COLI_ACT_F32)
-            gate_tiled_kernel<COLI_ACT_F32><<<grid, 256, 0, st>>>(Wr, x, T, H, E, logits);
+            gate_dmma_kernel<COLI_ACT_F32><<<grid, 128, 0, st>>>(Wr, x, T, H, E, logits);
         else
-            gate_tiled_kernel<COLI_ACT_BF16><<<grid, 256, 0, st>>>(Wr, x, T, H, E, logits);
+            gate_dmma_kernel<COLI_ACT_BF16><<<grid, 128, 0, st>>>(Wr, x, T, H, E, logits);
     }
     return cudaGetLastError();
 }

@@ -13,8 +13,10 @@ import synth
 # FFN tolerance of the float32-accumulate (CUDA-core) path: normwise per token,
 # max_j |y - y_ref| / max_j |y_ref|.
 TOL_GEMV = 1e-4
-# bf16 tensor-core path (h rounded to bf16 before the down projection).
-TOL_MMA = 2e-3
+# Tensor-core path (int8 MMA): x and h are rounded to 16-bit fixed point per row (half a unit of
+# 2^-15 of the row maximum); with max/rms ~4.5 for x and ~10 for h the per-element errors are
+# ~4e-5 and ~9e-5 of the row rms, and the normwise output error is of that order.
+TOL_TC = 3e-4
 
 
 def normwise_err(got, ref) -> float:
