@@ -17,15 +17,21 @@
 // The approximations are the two 16-bit roundings (x, h; 2^-16 of the row maximum) and float32
 // epilogue arithmetic.
 //
-// One persistent CTA per SM, warp-specialised, tiles (chunk of <= 128 tokens of one expert x one
+// One persistent CTA per SM, warp-specialised, tiles (chunk of <= 96 tokens of one expert x one
 // block of weight rows) taken round-robin:
 //   warp 12     TMA producer: per k-block of 128, the packed A tile (128 rows x 64 B, 64-byte
-//               swizzle) and the B rows (16-row boxes of 128 B, 128-byte swizzle) into a ring stage.
+//               swizzle; one 4-D box holds the gate and the up rows) and the B rows (boxes of
+//               128/64/32/16 rows of 128 B, 128-byte swizzle) into a ring stage; one lane per copy.
 //   warps 0-3   converters: one thread per weight row unpacks its 64 bytes into 128 signed bytes
 //               and stores them with tcgen05.st into a TMEM A stage; the MMA reads A from tensor
 //               memory, so unpacked weights never pass through shared memory.
-//   warp 13     MMA issuer: 4 x tcgen05.mma (K = 32) per k-block into one TMEM accumulator.
-//   warps 4-11  epilogue: tcgen05.ld of the accumulator and the output arithmetic.
+//   warp 13     MMA issuer (one elected lane, operands computed warp-uniformly): 4 x tcgen05.mma
+//               (K = 32, N <= 192) per k-block into one of two TMEM accumulators, so a tile's
+//               epilogue overlaps the next tile's main loop.
+//   warps 4-11  epilogue: tcgen05.ld of the accumulator and the output arithmetic; the tile's
+//               per-token scales, tokens and weights are staged in shared memory first.
+// TMEM (512 columns): accumulator b at columns [256b, 256b + 192); the four 32-column A stages
+// fill the gaps [192, 256) and [448, 512).
 // Inside every group of 8 k the order is permuted to (0,2,4,6,1,3,5,7) on both operands: the
 // unpacking yields the even and the odd codes of a word as separate words, and the activation
 // bytes are written in the same order, so every dot product is unchanged.
@@ -42,20 +48,22 @@ namespace coli {
 namespace {
 
 constexpr int KB = 128;                       // k per ring stage
-constexpr int MAXTOK = 128;                   // tokens per chunk
-constexpr int NSTAGE = 5;                     // shared-memory ring stages
-constexpr int NTS = 8;                        // TMEM A stages (KB / 4 = 32 columns each)
+constexpr int MAXTOK = 96;                    // tokens per chunk: N = 192 (hi and lo row per token)
+constexpr int NSTAGE = 6;                     // shared-memory ring stages
+constexpr int NTS = 4;                        // TMEM A stages (KB / 4 = 32 columns each)
 constexpr int A_RAW = 128 * (KB / 2);         // packed int4 A tile: 8 KB
-constexpr int B_MAX = 2 * MAXTOK * KB;        // B rows of one stage: 32 KB
-constexpr int STAGE_BYTES = A_RAW + B_MAX;
-constexpr int BOX_ROWS = 16;                  // B rows per TMA box
+constexpr int B_MAX = 2 * MAXTOK * KB;        // B rows of one stage: 24 KB
+constexpr int STAGE_BYTES = A_RAW + B_MAX;    // 32 KB, a multiple of 1024
+constexpr int NBOX = 4;                       // B box heights 16 << i rows
 constexpr int W_CONV = 4, W_EPI0 = 4, N_EPI = 8, W_PROD = 12, W_MMA = 13;
 constexpr int TC_THREADS = 14 * 32;
-constexpr uint32_t A_COL0 = 2 * MAXTOK;       // TMEM columns [0, 256): accumulator; then A stages
+constexpr uint32_t D_STRIDE = 256;            // accumulator b at TMEM column 256 * b
+constexpr uint32_t A_COL0 = 2 * MAXTOK;       // TMEM column of A stage 0
 constexpr uint32_t TMEM_COLS = 512;
 constexpr long long WAIT_CYCLES = 4000000000LL;  // ~2 s at 1.9 GHz: bound of every wait
 constexpr float QMAX = 32512.0f;              // |X| <= 32512 keeps Xh = (X + 128) >> 8 in [-127, 127]
 constexpr size_t TC_SMEM = static_cast<size_t>(NSTAGE) * STAGE_BYTES + 1024;
+constexpr int EPI_BAR = 1;                    // named barrier of the epilogue warps
 
 // kind::i8 instruction descriptor: D s32 (bits 4-5 = 2), A and B signed 8-bit (bits 7-9, 10-12
 // = 1), both K-major, M = 128 (bits 24-28 = M >> 4); N >> 3 goes to bits 17-22.
@@ -80,8 +88,17 @@ __device__ __forceinline__ bool mbar_try(uint32_t a, uint32_t parity) {
                  : "=r"(ok) : "r"(a), "r"(parity), "r"(20000u) : "memory");
     return ok != 0;
 }
-// Bounded wait; false when the bound ran out or another role has already given up.
+// Non-blocking test of a phase.
+__device__ __forceinline__ bool mbar_test(uint32_t a, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{ .reg .pred p; mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+                 : "=r"(ok) : "r"(a), "r"(parity) : "memory");
+    return ok != 0;
+}
+// Bounded wait; false when the bound ran out or another role has already given up.  A phase
+// that has already completed is taken with the non-blocking test.
 __device__ __forceinline__ bool mbar_wait(uint32_t a, uint32_t parity, volatile int *abort, int *err) {
+    if (mbar_test(a, parity)) return true;
     if (*abort) return false;
     if (mbar_try(a, parity)) return true;
     const long long t0 = clock64();
@@ -101,9 +118,10 @@ __device__ __forceinline__ void mbar_drain(uint32_t a, uint32_t parity) {
     while (!mbar_try(a, parity))
         if (clock64() - t0 > WAIT_CYCLES) return;
 }
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *m, int c0, int c1, int c2, uint32_t bar) {
-    asm volatile("cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
-                 ::"r"(dst), "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(c2), "r"(bar) : "memory");
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *m, int c0, int c1, int c2, int c3,
+                                            uint32_t bar) {
+    asm volatile("cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];"
+                 ::"r"(dst), "l"(reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar) : "memory");
 }
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *m, int c0, int c1, uint32_t bar) {
     asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
@@ -151,19 +169,39 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r) {
         : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-// 16 consecutive 32-bit columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, int *v) {
-    uint32_t r[16];
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+// 32 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, int *v) {
+    uint32_t r[32];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+                 "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-                   "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+                   "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+                   "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+                   "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
                  : "r"(taddr));
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = static_cast<int>(r[i]);
+    for (int i = 0; i < 32; ++i) v[i] = static_cast<int>(r[i]);
+}
+// Barrier of the epilogue warps that also ORs a predicate over them: every warp takes the same
+// decision (used to give up together, so no warp is left waiting at the barrier).
+__device__ __forceinline__ bool epi_sync_or(bool pred) {
+    uint32_t r;
+    asm volatile("{ .reg .pred p, q; setp.ne.u32 p, %1, 0; bar.red.or.pred q, %2, %3, p; selp.u32 %0, 1, 0, q; }"
+                 : "=r"(r) : "r"(static_cast<uint32_t>(pred)), "n"(EPI_BAR), "n"(N_EPI * 32) : "memory");
+    return r != 0;
 }
 
 __device__ __forceinline__ int round16(int v) { return (v + 15) & ~15; }
+// TMEM column of A stage j: 192, 224, 448, 480.
+__device__ __forceinline__ uint32_t a_col(int j) {
+    return static_cast<uint32_t>(j >> 1) * D_STRIDE + A_COL0 + 32u * static_cast<uint32_t>(j & 1);
+}
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile("{ .reg .pred P; elect.sync _|P, 0xffffffff; selp.b32 %0, 1, 0, P; }" : "=r"(pred));
+    return pred != 0;
+}
 
 // ------------------------------------------------------------------ activation quantisation --
 // 8 consecutive values -> 8 hi bytes and 8 lo bytes of X = rint(v * inv), in the (0,2,4,6,1,3,5,7)
@@ -361,22 +399,30 @@ struct GemmArgs {
     float *hbuf;             // [slots][I]
 };
 
+// Tensor maps of one GEMM: packed weight rows (routed records, shared record) as 4-D byte
+// tensors {row bytes, rows, matrices, records}, and the quantised B rows with four box heights.
+struct TcMaps {
+    CUtensorMap a, as;
+    CUtensorMap b[NBOX];
+};
+
 // PHASE 1: gate/up.  A = 64 gate rows + the same 64 up rows of one expert (TMEM lanes 32q..32q+15
 //          gate rows 16q.., lanes 32q+16.. the matching up rows), B = quantised x; epilogue
 //          h = SiLU(g) * u into hbuf (float32).
 // PHASE 2: down.  A = 128 rows of Wd, B = quantised h; epilogue out[token] += w * y.
 template <int PHASE>
 __global__ void __launch_bounds__(TC_THREADS, 1)
-tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmAs,
-               const __grid_constant__ CUtensorMap tmB, const GemmArgs p) {
+tc_gemm_kernel(const __grid_constant__ TcMaps maps, const GemmArgs p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    __shared__ __align__(8) uint64_t bars[2 * NSTAGE + 2 * NTS + 3];
+    __shared__ __align__(8) uint64_t bars[2 * NSTAGE + 2 * NTS + 5];
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
+    __shared__ float s_bs[2][MAXTOK], s_w[2][MAXTOK];
+    __shared__ int s_tk[2][MAXTOK];
     uint64_t *full = bars, *empty = bars + NSTAGE, *tfull = bars + 2 * NSTAGE, *tempty = tfull + NTS;
-    uint64_t *dfull = tempty + NTS, *dempty = dfull + 1, *drain = dempty + 1;
+    uint64_t *dfull = tempty + NTS, *dempty = dfull + 2, *drain = dempty + 2;
     volatile int *abort = &s_abort;
 
     const FfnParams &f = p.f;
@@ -398,8 +444,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             mbar_init(smem_u32(&tfull[i]), W_CONV * 32);
             mbar_init(smem_u32(&tempty[i]), 1);
         }
-        mbar_init(smem_u32(dfull), 1);
-        mbar_init(smem_u32(dempty), N_EPI * 32);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(smem_u32(&dfull[i]), 1);
+            mbar_init(smem_u32(&dempty[i]), N_EPI * 32);
+        }
         mbar_init(smem_u32(drain), 1);
         s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -411,73 +459,87 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 
     if (warp == W_PROD) {
         // ------------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            uint32_t it = 0;
-            for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
-                const int4 c = p.chunks[t / MB];
-                const int m = t % MB;
-                const int nrows = round16(2 * c.z);
-                const CUtensorMap *ta = c.x >= 0 ? &tmA : &tmAs;
-                const int ez = c.x >= 0 ? c.x : 0;
-                for (int kb = 0; kb < KT; ++kb, ++it) {
-                    const int s = it % NSTAGE;
-                    if (!mbar_wait(smem_u32(&empty[s]), ((it / NSTAGE) & 1) ^ 1, abort, f.err)) goto prod_done;
-                    const uint32_t st = smem_u32(sm + s * STAGE_BYTES);
-                    const uint32_t fb = smem_u32(&full[s]);
-                    mbar_expect_tx(fb, A_RAW + nrows * KB);
-                    if (PHASE == 1) {
-                        tma_load_3d(st, ta, kb * (KB / 2), m * 64, ez, fb);
-                        tma_load_3d(st + A_RAW / 2, ta, kb * (KB / 2), f.I + m * 64, ez, fb);
-                    } else {
-                        tma_load_3d(st, ta, kb * (KB / 2), m * 128, ez, fb);
+        // lane 0: the A box; lane 1 + i: the B box of 128 >> i rows when bit 3 - i of nrows/16 is set
+        uint32_t it = 0;
+        for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+            const int4 c = p.chunks[t / MB];
+            const int m = t % MB;
+            const int n16 = round16(2 * c.z) / 16;
+            const CUtensorMap *ta = c.x >= 0 ? &maps.a : &maps.as;
+            const int ez = c.x >= 0 ? c.x : 0;
+            for (int kb = 0; kb < KT; ++kb, ++it) {
+                const int s = it % NSTAGE;
+                if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&empty[s]), ((it / NSTAGE) & 1) ^ 1, abort, f.err)))
+                    goto prod_done;
+                const uint32_t st = smem_u32(sm + s * STAGE_BYTES);
+                const uint32_t fb = smem_u32(&full[s]);
+                if (lane == 0) mbar_expect_tx(fb, A_RAW + n16 * 16 * KB);
+                __syncwarp();
+                if (lane == 0) {
+                    tma_load_4d(st, ta, kb * (KB / 2), m * MROWS, 0, ez, fb);
+                } else if (lane <= NBOX) {
+                    const int bit = NBOX - lane;
+                    if ((n16 >> bit) & 1) {
+                        const int row0 = 16 * ((n16 >> (bit + 1)) << (bit + 1));  // rows of the larger boxes
+                        tma_load_2d(st + A_RAW + row0 * KB, &maps.b[bit], kb * KB, 2 * c.y + row0, fb);
                     }
-                    for (int j = 0; j < nrows / BOX_ROWS; ++j)
-                        tma_load_2d(st + A_RAW + j * BOX_ROWS * KB, &tmB, kb * KB, 2 * c.y + BOX_ROWS * j, fb);
                 }
             }
-        prod_done:
-            if (*abort) {
-                // let the copies already issued land before the CTA's shared memory is released
-                for (uint32_t k = it > NSTAGE ? it - NSTAGE : 0; k < it; ++k)
-                    mbar_drain(smem_u32(&full[k % NSTAGE]), (k / NSTAGE) & 1);
-            }
+        }
+    prod_done:
+        if (*abort && lane == 0) {
+            // let the copies already issued land before the CTA's shared memory is released
+            for (uint32_t k = it > NSTAGE ? it - NSTAGE : 0; k < it; ++k)
+                mbar_drain(smem_u32(&full[k % NSTAGE]), (k / NSTAGE) & 1);
         }
     } else if (warp == W_MMA) {
         // ------------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            uint32_t it = 0, tl = 0;
-            for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tl) {
-                const int4 c = p.chunks[t / MB];
-                const int nrows = round16(2 * c.z);
-                const uint32_t idesc = IDESC_I8 | (static_cast<uint32_t>(nrows >> 3) << 17);
-                if (!mbar_wait(smem_u32(dempty), (tl & 1) ^ 1, abort, f.err)) goto mma_done;
+        // the whole warp runs the loop (uniform operands); one elected lane issues
+        uint32_t it = 0, tl = 0;
+        // B descriptor of stage s, k-step kk: the start-address field (bits 0-13, address >> 4)
+        // advances by STAGE_BYTES >> 4 per stage and by 2 per 32-byte k-step
+        const uint64_t bdesc0 = smem_desc_sw128(smem_u32(sm + A_RAW));
+        for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tl) {
+            const int4 c = p.chunks[t / MB];
+            const int nrows = round16(2 * c.z);
+            const uint32_t idesc = IDESC_I8 | (static_cast<uint32_t>(nrows >> 3) << 17);
+            const int db = tl & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&dempty[db]), ((tl >> 1) & 1) ^ 1, abort, f.err)))
+                goto mma_done;
+            tc_fence_after();
+            const uint32_t dt = tbase + db * D_STRIDE;
+            for (int kb = 0; kb < KT; ++kb, ++it) {
+                const int s = it % NSTAGE, ts = it % NTS;
+                if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&full[s]), (it / NSTAGE) & 1, abort, f.err)))
+                    goto mma_done;
+                if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&tfull[ts]), (it / NTS) & 1, abort, f.err)))
+                    goto mma_done;
                 tc_fence_after();
-                for (int kb = 0; kb < KT; ++kb, ++it) {
-                    const int s = it % NSTAGE, ts = it % NTS;
-                    if (!mbar_wait(smem_u32(&full[s]), (it / NSTAGE) & 1, abort, f.err)) goto mma_done;
-                    if (!mbar_wait(smem_u32(&tfull[ts]), (it / NTS) & 1, abort, f.err)) goto mma_done;
-                    tc_fence_after();
-                    const uint32_t b0 = smem_u32(sm + s * STAGE_BYTES + A_RAW);
-                    const uint32_t a0 = tbase + A_COL0 + ts * (KB / 4);
+                const uint64_t bd = bdesc0 + static_cast<uint64_t>(s * (STAGE_BYTES >> 4));
+                const uint32_t a0 = tbase + a_col(ts);
+                if (elect_one()) {
 #pragma unroll
                     for (int kk = 0; kk < KB / 32; ++kk)
-                        mma_i8(tbase, a0 + kk * 8, smem_desc_sw128(b0 + kk * 32), idesc, (kb | kk) != 0);
+                        mma_i8(dt, a0 + kk * 8, bd + 2 * kk, idesc, (kb | kk) != 0);
                     mma_commit(smem_u32(&empty[s]));
                     mma_commit(smem_u32(&tempty[ts]));
                 }
-                mma_commit(smem_u32(dfull));
+                __syncwarp();
             }
-        mma_done:
-            // every MMA issued so far has completed once this commit arrives
-            mma_commit(smem_u32(drain));
-            mbar_drain(smem_u32(drain), 0);
+            if (elect_one()) mma_commit(smem_u32(&dfull[db]));
+            __syncwarp();
         }
+    mma_done:
+        // every MMA issued so far has completed once this commit arrives
+        if (elect_one()) mma_commit(smem_u32(drain));
+        __syncwarp();
+        mbar_drain(smem_u32(drain), 0);
     } else if (warp < W_CONV) {
         // ------------------------------------------------------------------ converters
         const int q = warp;
         const int rho = PHASE == 1 ? (lane < 16 ? 16 * q + lane : 64 + 16 * q + (lane - 16)) : 32 * q + lane;
         const int swz = (rho >> 1) & 3;  // 64-byte swizzle: 16-byte chunk c of row r sits at c ^ ((r >> 1) & 3)
-        const uint32_t ta = tbase + (static_cast<uint32_t>(32 * q) << 16) + A_COL0;
+        const uint32_t ta = tbase + (static_cast<uint32_t>(32 * q) << 16);
         uint32_t it = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
             for (int kb = 0; kb < KT; ++kb, ++it) {
@@ -489,9 +551,6 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 #pragma unroll
                 for (int cch = 0; cch < 4; ++cch) v[cch] = *reinterpret_cast<const uint4 *>(row + ((cch ^ swz) << 4));
                 mbar_arrive(smem_u32(&empty[s]));
-                if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&tempty[ts]), ((it / NTS) & 1) ^ 1, abort, f.err)))
-                    goto conv_done;
-                tc_fence_after();
                 uint32_t o[32];
 #pragma unroll
                 for (int cch = 0; cch < 4; ++cch) {
@@ -502,7 +561,10 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                         o[8 * cch + 2 * i + 1] = w4[i] & 0xF0F0F0F0u;     // codes 1,3,5,7
                     }
                 }
-                tmem_st32(ta + ts * (KB / 4), o);
+                if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&tempty[ts]), ((it / NTS) & 1) ^ 1, abort, f.err)))
+                    goto conv_done;
+                tc_fence_after();
+                tmem_st32(ta + a_col(ts), o);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(smem_u32(&tfull[ts]));
@@ -512,63 +574,74 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     } else {
         // ------------------------------------------------------------------ epilogue
         const int q = (warp - W_EPI0) & 3, half = (warp - W_EPI0) >> 2;
-        const uint32_t tl_addr = tbase + (static_cast<uint32_t>(32 * q) << 16);
+        const int et = threadIdx.x - W_EPI0 * 32;  // 0 .. 255
         uint32_t tl = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tl) {
             const int4 c = p.chunks[t / MB];
             const int m = t % MB;
             const int n = c.z, pos0 = c.y;
-            const int nrows = round16(2 * n);
+            const int ngrp = (round16(2 * n) + 31) / 32;  // groups of 32 columns = 16 tokens
             const uint8_t *rec = c.x >= 0 ? f.experts + static_cast<size_t>(c.x) * f.stride : f.shared;
+            const int pb = tl & 1, db = tl & 1;
+            // per-token data of the tile (double-buffered by tile parity; the barrier below also
+            // orders every warp's reads of tile tl - 2 before these writes)
+            if (et < n) {
+                s_bs[pb][et] = p.bscale[pos0 + et];
+                if (PHASE == 2) {
+                    s_w[pb][et] = p.w_of[pos0 + et];
+                    s_tk[pb][et] = p.tok_of[pos0 + et];
+                }
+            }
+            if (epi_sync_or(*abort != 0)) break;
             // warp-uniform: tcgen05.ld below is a warp-collective instruction
-            if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(dfull), tl & 1, abort, f.err))) break;
+            if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&dfull[db]), (tl >> 1) & 1, abort, f.err)))
+                continue;  // given up: every epilogue warp leaves at the next barrier
             tc_fence_after();
+            const uint32_t dt = tbase + (static_cast<uint32_t>(32 * q) << 16) + db * D_STRIDE;
             if (PHASE == 1) {
                 const bool gate = lane < 16;
                 const int irow = m * 64 + 16 * q + (lane & 15);
                 const float sc = reinterpret_cast<const float *>(rec + (gate ? f.off_sg : f.off_su))[irow];
-                for (int cc = half; cc < nrows / 16; cc += 2) {
-                    int v[16];
-                    tmem_ld16(tl_addr + 16 * cc, v);
-                    float d[8];
+                for (int g = half; g < ngrp; g += 2) {
+                    int v[32];
+                    tmem_ld32(dt + 32 * g, v);
+                    float d[16];
 #pragma unroll
-                    for (int j = 0; j < 8; ++j)
+                    for (int j = 0; j < 16; ++j)
                         d[j] = sc * fmaf(256.0f, static_cast<float>(v[2 * j]), static_cast<float>(v[2 * j + 1]));
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        // gate lanes keep tokens 0-3 of the group of 8, up lanes tokens 4-7
-                        const float keep = gate ? d[i] : d[4 + i];
-                        const float other = __shfl_xor_sync(0xffffffffu, gate ? d[4 + i] : d[i], 16);
-                        const int j = 8 * cc + (gate ? i : 4 + i);
+                    for (int i = 0; i < 8; ++i) {
+                        // gate lanes keep tokens 0-7 of the group, up lanes tokens 8-15
+                        const float keep = gate ? d[i] : d[8 + i];
+                        const float other = __shfl_xor_sync(0xffffffffu, gate ? d[8 + i] : d[i], 16);
+                        const int j = 16 * g + (gate ? i : 8 + i);
                         if (j < n) {
-                            const int pos = pos0 + j;
-                            const float bs = p.bscale[pos];
-                            const float g = (gate ? keep : other) * bs;
-                            const float u = (gate ? other : keep) * bs;
-                            p.hbuf[static_cast<size_t>(pos) * f.I + irow] = g / (1.0f + expf(-g)) * u;
+                            const float bs = s_bs[pb][j];
+                            const float gv = (gate ? keep : other) * bs;
+                            const float uv = (gate ? other : keep) * bs;
+                            p.hbuf[static_cast<size_t>(pos0 + j) * f.I + irow] = gv / (1.0f + expf(-gv)) * uv;
                         }
                     }
                 }
             } else {
                 const int r = m * 128 + 32 * q + lane;
                 const float sd = reinterpret_cast<const float *>(rec + f.off_sd)[r];
-                for (int cc = half; cc < nrows / 16; cc += 2) {
-                    int v[16];
-                    tmem_ld16(tl_addr + 16 * cc, v);
+                for (int g = half; g < ngrp; g += 2) {
+                    int v[32];
+                    tmem_ld32(dt + 32 * g, v);
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const int jj = 8 * cc + j;
+                    for (int j = 0; j < 16; ++j) {
+                        const int jj = 16 * g + j;
                         if (jj < n) {
-                            const int pos = pos0 + jj;
                             const float y = fmaf(256.0f, static_cast<float>(v[2 * j]), static_cast<float>(v[2 * j + 1])) *
-                                            (sd * p.bscale[pos]);
-                            atomicAdd(f.out + static_cast<size_t>(p.tok_of[pos]) * f.H + r, p.w_of[pos] * y);
+                                            (sd * s_bs[pb][jj]);
+                            atomicAdd(f.out + static_cast<size_t>(s_tk[pb][jj]) * f.H + r, s_w[pb][jj] * y);
                         }
                     }
                 }
             }
             tc_fence_before();
-            mbar_arrive(smem_u32(dempty));
+            mbar_arrive(smem_u32(&dempty[db]));
         }
     }
 
@@ -599,27 +672,34 @@ bool encode_u8(CUtensorMap *m, const void *base, cuuint32_t rank, const cuuint64
                const cuuint64_t *strides, const cuuint32_t *box, CUtensorMapSwizzle sw) {
     const PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
     if (!enc) return false;
-    const cuuint32_t es[3] = {1, 1, 1};
+    const cuuint32_t es[5] = {1, 1, 1, 1, 1};  // rank <= 5
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, const_cast<void *>(base), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Packed weight rows of a set of records as a 3-D byte tensor {row bytes, rows, records}.
-bool weight_map(CUtensorMap *m, const uint8_t *base, size_t row_bytes, size_t rows, size_t nrec,
-                size_t rec_stride, cuuint32_t box_rows) {
-    const cuuint64_t dims[3] = {row_bytes, rows, nrec};
-    const cuuint64_t strides[2] = {row_bytes, rec_stride};
-    const cuuint32_t box[3] = {KB / 2, box_rows, 1};
-    return encode_u8(m, base, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B);
+// Packed weight rows of a set of records as a 4-D byte tensor {row bytes, rows, matrices,
+// records}; the box takes `box_rows` rows of `box_mats` consecutive matrices.
+bool weight_map(CUtensorMap *m, const uint8_t *base, size_t row_bytes, size_t rows, size_t mats, size_t nrec,
+                size_t rec_stride, cuuint32_t box_rows, cuuint32_t box_mats) {
+    const cuuint64_t dims[4] = {row_bytes, rows, mats, nrec};
+    const cuuint64_t strides[3] = {row_bytes, rows * row_bytes, rec_stride};
+    const cuuint32_t box[4] = {KB / 2, box_rows, box_mats, 1};
+    return encode_u8(m, base, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
-// Quantised B rows {len bytes, 2 * slots rows}.
-bool act_map(CUtensorMap *m, const int8_t *base, size_t len, size_t rows) {
+// Quantised B rows {len bytes, 2 * slots rows}, boxes of `box_rows` rows.
+bool act_map(CUtensorMap *m, const int8_t *base, size_t len, size_t rows, cuuint32_t box_rows) {
     const cuuint64_t dims[2] = {len, rows};
     const cuuint64_t strides[1] = {len};
-    const cuuint32_t box[2] = {KB, BOX_ROWS};
+    const cuuint32_t box[2] = {KB, box_rows};
     return encode_u8(m, base, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+bool act_maps(TcMaps *m, const int8_t *base, size_t len, size_t rows) {
+    for (int i = 0; i < NBOX; ++i)
+        if (!act_map(&m->b[i], base, len, rows, 16u << i)) return false;
+    return true;
 }
 
 }  // namespace
@@ -670,20 +750,20 @@ cudaError_t launch_ffn_tc(const FfnParams &f, const TcBuffers &b, cudaStream_t s
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     // tensor maps (host-side encodings of the operands' shapes; no device work)
-    CUtensorMap mA1, mA1s, mA2, mA2s, mB1, mB2;
-    const size_t rbh = f.rb_h, rbi = f.rb_i;
-    const size_t rec_bytes = f.off_sd + static_cast<size_t>(f.H) * 4;
+    TcMaps m1, m2;
+    const size_t rbh = f.rb_h, rbi = f.rb_i, I = f.I, H = f.H;
+    const size_t rec_bytes = f.off_sd + H * 4;
     const size_t rec_pad = (rec_bytes + 255) & ~static_cast<size_t>(255);
-    bool ok = weight_map(&mA1, f.experts, rbh, 2 * static_cast<size_t>(f.I), f.E, f.stride, 64) &&
-              weight_map(&mA2, f.experts + f.off_wd, rbi, f.H, f.E, f.stride, 128) &&
-              act_map(&mB1, b.xq, f.H, 2 * static_cast<size_t>(slots)) &&
-              act_map(&mB2, b.hq, f.I, 2 * static_cast<size_t>(slots));
+    bool ok = weight_map(&m1.a, f.experts, rbh, I, 2, f.E, f.stride, 64, 2) &&
+              weight_map(&m2.a, f.experts + f.off_wd, rbi, H, 1, f.E, f.stride, 128, 1) &&
+              act_maps(&m1, b.xq, H, 2 * static_cast<size_t>(slots)) &&
+              act_maps(&m2, b.hq, I, 2 * static_cast<size_t>(slots));
     if (ok && f.S) {
-        ok = weight_map(&mA1s, f.shared, rbh, 2 * static_cast<size_t>(f.I), 1, rec_pad, 64) &&
-             weight_map(&mA2s, f.shared + f.off_wd, rbi, f.H, 1, rec_pad, 128);
+        ok = weight_map(&m1.as, f.shared, rbh, I, 2, 1, rec_pad, 64, 2) &&
+             weight_map(&m2.as, f.shared + f.off_wd, rbi, H, 1, 1, rec_pad, 128, 1);
     } else {
-        mA1s = mA1;
-        mA2s = mA2;
+        m1.as = m1.a;
+        m2.as = m2.a;
     }
     if (!ok) return cudaErrorInvalidValue;
 
@@ -704,7 +784,7 @@ cudaError_t launch_ffn_tc(const FfnParams &f, const TcBuffers &b, cudaStream_t s
 
     // 2. gate/up GEMM -> h (float32)
     g.bscale = b.sx;
-    tc_gemm_kernel<1><<<grid, TC_THREADS, TC_SMEM, st>>>(mA1, mA1s, mB1, g);
+    tc_gemm_kernel<1><<<grid, TC_THREADS, TC_SMEM, st>>>(m1, g);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     // 3. h quantisation
@@ -718,7 +798,7 @@ cudaError_t launch_ffn_tc(const FfnParams &f, const TcBuffers &b, cudaStream_t s
 
     // 4. down GEMM + weighted combine into out
     g.bscale = b.sh;
-    tc_gemm_kernel<2><<<grid, TC_THREADS, TC_SMEM, st>>>(mA2, mA2s, mB2, g);
+    tc_gemm_kernel<2><<<grid, TC_THREADS, TC_SMEM, st>>>(m2, g);
     return cudaGetLastError();
 }
 
