@@ -19,9 +19,11 @@
 //
 // One persistent CTA per SM, warp-specialised, tiles (chunk of <= 96 tokens of one expert x one
 // block of weight rows) taken round-robin:
-//   warp 12     TMA producer: per k-block of 128, the packed A tile (128 rows x 64 B, 64-byte
-//               swizzle; one 4-D box holds the gate and the up rows) and the B rows (boxes of
-//               128/64/32/16 rows of 128 B, 128-byte swizzle) into a ring stage; one lane per copy.
+//   warp 12     A producer: per k-block of 128, the packed A tile (128 rows x 64 B, 64-byte
+//               swizzle; one 4-D box holds the gate and the up rows) into the A ring, whose stages
+//               the converters release as soon as they have read them.
+//   warp 14     B producer: the k-block's B rows (boxes of 128/64/32/16 rows of 128 B, 128-byte
+//               swizzle) into the B ring, released by the MMAs' completion; one lane per box.
 //   warps 0-3   converters: one thread per weight row unpacks its 64 bytes into 128 signed bytes
 //               and stores them with tcgen05.st into a TMEM A stage; the MMA reads A from tensor
 //               memory, so unpacked weights never pass through shared memory.
@@ -49,20 +51,22 @@ namespace {
 
 constexpr int KB = 128;                       // k per ring stage
 constexpr int MAXTOK = 96;                    // tokens per chunk: N = 192 (hi and lo row per token)
-constexpr int NSTAGE = 6;                     // shared-memory ring stages
-constexpr int NTS = 4;                        // TMEM A stages (KB / 4 = 32 columns each)
+constexpr int NA = 8;                         // A ring stages (packed int4 tiles)
+constexpr int NB = 6;                         // B ring stages
 constexpr int A_RAW = 128 * (KB / 2);         // packed int4 A tile: 8 KB
 constexpr int B_MAX = 2 * MAXTOK * KB;        // B rows of one stage: 24 KB
-constexpr int STAGE_BYTES = A_RAW + B_MAX;    // 32 KB, a multiple of 1024
 constexpr int NBOX = 4;                       // B box heights 16 << i rows
-constexpr int W_CONV = 4, W_EPI0 = 4, N_EPI = 8, W_PROD = 12, W_MMA = 13;
-constexpr int TC_THREADS = 14 * 32;
+constexpr int W_CONV = 4, W_EPI0 = 4, N_EPI = 8, W_PRODA = 12, W_MMA = 13, W_PRODB = 14;
+constexpr int TC_THREADS = 15 * 32;
 constexpr uint32_t D_STRIDE = 256;            // accumulator b at TMEM column 256 * b
 constexpr uint32_t A_COL0 = 2 * MAXTOK;       // TMEM column of A stage 0
+constexpr int SPG = (256 - 2 * MAXTOK) / 32;  // 32-column A stages in the gap after each accumulator
+constexpr int NTS = 2 * SPG;                  // TMEM A stages
+static_assert(SPG >= 1, "no room for TMEM A stages");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr long long WAIT_CYCLES = 4000000000LL;  // ~2 s at 1.9 GHz: bound of every wait
 constexpr float QMAX = 32512.0f;              // |X| <= 32512 keeps Xh = (X + 128) >> 8 in [-127, 127]
-constexpr size_t TC_SMEM = static_cast<size_t>(NSTAGE) * STAGE_BYTES + 1024;
+constexpr size_t TC_SMEM = static_cast<size_t>(NA) * A_RAW + static_cast<size_t>(NB) * B_MAX + 1024;
 constexpr int EPI_BAR = 1;                    // named barrier of the epilogue warps
 
 // kind::i8 instruction descriptor: D s32 (bits 4-5 = 2), A and B signed 8-bit (bits 7-9, 10-12
@@ -193,9 +197,9 @@ __device__ __forceinline__ bool epi_sync_or(bool pred) {
 }
 
 __device__ __forceinline__ int round16(int v) { return (v + 15) & ~15; }
-// TMEM column of A stage j: 192, 224, 448, 480.
+// TMEM column of A stage j: the gaps [2 * MAXTOK, 256) and [256 + 2 * MAXTOK, 512).
 __device__ __forceinline__ uint32_t a_col(int j) {
-    return static_cast<uint32_t>(j >> 1) * D_STRIDE + A_COL0 + 32u * static_cast<uint32_t>(j & 1);
+    return static_cast<uint32_t>(j / SPG) * D_STRIDE + A_COL0 + 32u * static_cast<uint32_t>(j % SPG);
 }
 __device__ __forceinline__ bool elect_one() {
     uint32_t pred = 0;
@@ -416,12 +420,13 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const GemmArgs p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    __shared__ __align__(8) uint64_t bars[2 * NSTAGE + 2 * NTS + 5];
+    __shared__ __align__(8) uint64_t bars[2 * NA + 2 * NB + 2 * NTS + 5];
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
     __shared__ float s_bs[2][MAXTOK], s_w[2][MAXTOK];
     __shared__ int s_tk[2][MAXTOK];
-    uint64_t *full = bars, *empty = bars + NSTAGE, *tfull = bars + 2 * NSTAGE, *tempty = tfull + NTS;
+    uint64_t *afull = bars, *aempty = afull + NA, *bfull = aempty + NA, *bempty = bfull + NB;
+    uint64_t *tfull = bempty + NB, *tempty = tfull + NTS;
     uint64_t *dfull = tempty + NTS, *dempty = dfull + 2, *drain = dempty + 2;
     volatile int *abort = &s_abort;
 
@@ -436,9 +441,13 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const GemmArgs p) {
 
     if (warp == 0) tmem_alloc(smem_u32(&s_tmem), TMEM_COLS);
     if (threadIdx.x == 32) {
-        for (int i = 0; i < NSTAGE; ++i) {
-            mbar_init(smem_u32(&full[i]), 1);
-            mbar_init(smem_u32(&empty[i]), W_CONV * 32 + 1);
+        for (int i = 0; i < NA; ++i) {
+            mbar_init(smem_u32(&afull[i]), 1);
+            mbar_init(smem_u32(&aempty[i]), W_CONV * 32);
+        }
+        for (int i = 0; i < NB; ++i) {
+            mbar_init(smem_u32(&bfull[i]), 1);
+            mbar_init(smem_u32(&bempty[i]), 1);
         }
         for (int i = 0; i < NTS; ++i) {
             mbar_init(smem_u32(&tfull[i]), W_CONV * 32);
@@ -457,9 +466,15 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const GemmArgs p) {
     tc_fence_after();
     const uint32_t tbase = s_tmem;
 
-    if (warp == W_PROD) {
-        // ------------------------------------------------------------------ TMA producer
-        // lane 0: the A box; lane 1 + i: the B box of 128 >> i rows when bit 3 - i of nrows/16 is set
+    unsigned char *sa = sm;                                        // A ring
+    unsigned char *sb = sm + static_cast<size_t>(NA) * A_RAW;      // B ring
+    if (warp == W_PRODA || warp == W_PRODB) {
+        // ------------------------------------------------------------------ TMA producers
+        // A warp, lane 0: the A box.  B warp, lane i < 4: the box of 128 >> i rows when bit 3 - i
+        // of nrows/16 is set.
+        const bool is_a = warp == W_PRODA;
+        const int nst = is_a ? NA : NB;
+        uint64_t *fullb = is_a ? afull : bfull, *emptyb = is_a ? aempty : bempty;
         uint32_t it = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
             const int4 c = p.chunks[t / MB];
@@ -468,20 +483,19 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const GemmArgs p) {
             const CUtensorMap *ta = c.x >= 0 ? &maps.a : &maps.as;
             const int ez = c.x >= 0 ? c.x : 0;
             for (int kb = 0; kb < KT; ++kb, ++it) {
-                const int s = it % NSTAGE;
-                if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&empty[s]), ((it / NSTAGE) & 1) ^ 1, abort, f.err)))
+                const int s = it % nst;
+                if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&emptyb[s]), ((it / nst) & 1) ^ 1, abort, f.err)))
                     goto prod_done;
-                const uint32_t st = smem_u32(sm + s * STAGE_BYTES);
-                const uint32_t fb = smem_u32(&full[s]);
-                if (lane == 0) mbar_expect_tx(fb, A_RAW + n16 * 16 * KB);
+                const uint32_t fb = smem_u32(&fullb[s]);
+                if (lane == 0) mbar_expect_tx(fb, is_a ? A_RAW : n16 * 16 * KB);
                 __syncwarp();
-                if (lane == 0) {
-                    tma_load_4d(st, ta, kb * (KB / 2), m * MROWS, 0, ez, fb);
-                } else if (lane <= NBOX) {
-                    const int bit = NBOX - lane;
+                if (is_a) {
+                    if (lane == 0) tma_load_4d(smem_u32(sa + s * A_RAW), ta, kb * (KB / 2), m * MROWS, 0, ez, fb);
+                } else if (lane < NBOX) {
+                    const int bit = NBOX - 1 - lane;
                     if ((n16 >> bit) & 1) {
                         const int row0 = 16 * ((n16 >> (bit + 1)) << (bit + 1));  // rows of the larger boxes
-                        tma_load_2d(st + A_RAW + row0 * KB, &maps.b[bit], kb * KB, 2 * c.y + row0, fb);
+                        tma_load_2d(smem_u32(sb + s * B_MAX + row0 * KB), &maps.b[bit], kb * KB, 2 * c.y + row0, fb);
                     }
                 }
             }
@@ -489,16 +503,16 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const GemmArgs p) {
     prod_done:
         if (*abort && lane == 0) {
             // let the copies already issued land before the CTA's shared memory is released
-            for (uint32_t k = it > NSTAGE ? it - NSTAGE : 0; k < it; ++k)
-                mbar_drain(smem_u32(&full[k % NSTAGE]), (k / NSTAGE) & 1);
+            for (uint32_t k = it > static_cast<uint32_t>(nst) ? it - nst : 0; k < it; ++k)
+                mbar_drain(smem_u32(&fullb[k % nst]), (k / nst) & 1);
         }
     } else if (warp == W_MMA) {
         // ------------------------------------------------------------------ MMA issuer
         // the whole warp runs the loop (uniform operands); one elected lane issues
         uint32_t it = 0, tl = 0;
         // B descriptor of stage s, k-step kk: the start-address field (bits 0-13, address >> 4)
-        // advances by STAGE_BYTES >> 4 per stage and by 2 per 32-byte k-step
-        const uint64_t bdesc0 = smem_desc_sw128(smem_u32(sm + A_RAW));
+        // advances by B_MAX >> 4 per stage and by 2 per 32-byte k-step
+        const uint64_t bdesc0 = smem_desc_sw128(smem_u32(sb));
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tl) {
             const int4 c = p.chunks[t / MB];
             const int nrows = round16(2 * c.z);
@@ -509,19 +523,19 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const GemmArgs p) {
             tc_fence_after();
             const uint32_t dt = tbase + db * D_STRIDE;
             for (int kb = 0; kb < KT; ++kb, ++it) {
-                const int s = it % NSTAGE, ts = it % NTS;
-                if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&full[s]), (it / NSTAGE) & 1, abort, f.err)))
+                const int s = it % NB, ts = it % NTS;
+                if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&bfull[s]), (it / NB) & 1, abort, f.err)))
                     goto mma_done;
                 if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&tfull[ts]), (it / NTS) & 1, abort, f.err)))
                     goto mma_done;
                 tc_fence_after();
-                const uint64_t bd = bdesc0 + static_cast<uint64_t>(s * (STAGE_BYTES >> 4));
+                const uint64_t bd = bdesc0 + static_cast<uint64_t>(s * (B_MAX >> 4));
                 const uint32_t a0 = tbase + a_col(ts);
                 if (elect_one()) {
 #pragma unroll
                     for (int kk = 0; kk < KB / 32; ++kk)
                         mma_i8(dt, a0 + kk * 8, bd + 2 * kk, idesc, (kb | kk) != 0);
-                    mma_commit(smem_u32(&empty[s]));
+                    mma_commit(smem_u32(&bempty[s]));
                     mma_commit(smem_u32(&tempty[ts]));
                 }
                 __syncwarp();
@@ -543,14 +557,14 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const GemmArgs p) {
         uint32_t it = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
             for (int kb = 0; kb < KT; ++kb, ++it) {
-                const int s = it % NSTAGE, ts = it % NTS;
-                if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&full[s]), (it / NSTAGE) & 1, abort, f.err)))
+                const int s = it % NA, ts = it % NTS;
+                if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&afull[s]), (it / NA) & 1, abort, f.err)))
                     goto conv_done;
-                const unsigned char *row = sm + s * STAGE_BYTES + rho * (KB / 2);
+                const unsigned char *row = sa + s * A_RAW + rho * (KB / 2);
                 uint4 v[4];
 #pragma unroll
                 for (int cch = 0; cch < 4; ++cch) v[cch] = *reinterpret_cast<const uint4 *>(row + ((cch ^ swz) << 4));
-                mbar_arrive(smem_u32(&empty[s]));
+                mbar_arrive(smem_u32(&aempty[s]));
                 uint32_t o[32];
 #pragma unroll
                 for (int cch = 0; cch < 4; ++cch) {
