@@ -21,8 +21,9 @@
 // held as 16-bit block fixed point (per 16-byte chunk of codes, one power-of-two scale) with
 // dp2a integer dot products, exact in int32; the activation is exact for every element within a
 // factor 2^7 of its chunk's largest magnitude (bf16 has 8 significant bits), smaller elements are
-// rounded to 2^-15 of that maximum.  Phase 2 uses float32 with a positional magic-exponent
-// decode (codes at their bit position, the activation pre-scaled by the matching power of two).
+// rounded to 2^-15 of that maximum.  Phase 2 takes h as 16-bit fixed point per chunk split in two
+// signed bytes and the codes as signed bytes (16q for int4, 64q for int2), so dp4a integer dot
+// products are exact; h is rounded to 2^-16 of its chunk's largest magnitude.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -156,93 +157,85 @@ __device__ __forceinline__ int idot_chunk<2>(const uint4 q, const int *xp, int c
     return (a[0] + a[1]) + (a[2] + a[3]);
 }
 
-// Phase 2 activations (h) as 30-bit fixed point split into two signed 16-bit halves,
-// m = hi * 2^15 + lo, with one power-of-two scale per chunk; both halves use the same code
-// extraction and the layout of idot_chunk.  Returns the two exact integer sums.
+// Phase 2 activations (h) as 16-bit fixed point per chunk, X = rint(h * 32512 / max|h|), split
+// X = 256 * Xh + Xl into two signed bytes; the codes become signed bytes scaled by a power of
+// two (the int4 nibble in the high half of a byte is 16q, an int2 field in the top two bits is
+// 64q), so one dp4a takes four products of each part exactly.  Slice word order follows the
+// byte extraction below (h_slot).  Returns the two exact integer sums.
+template <int FMT> struct Ph2 {
+    static constexpr int MUL = FMT == 4 ? 16 : (FMT == 2 ? 64 : 1);  // code byte = MUL * q
+    static constexpr int XW8 = Fmt<FMT>::CPC / 4;                    // int8x4 words per chunk and part
+    static constexpr int XV8 = XW8 / 4;                              // int4 vectors per chunk and part
+};
 template <int FMT>
-__device__ __forceinline__ void idot2_chunk(const uint4 q, const int *xh, const int *xl, int ch, int cl,
-                                            int &sh, int &sl);
+__device__ __forceinline__ void idot4_chunk(const uint4 q, const int *xh, const int *xl, int &sh, int &sl);
 
 template <>
-__device__ __forceinline__ void idot2_chunk<4>(const uint4 q, const int *xh, const int *xl, int ch, int cl,
-                                               int &sh, int &sl) {
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-    int h0 = -ch, h1 = 0, l0 = -cl, l1 = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t f = w[i] ^ 0x88888888u;
-        const int lo = static_cast<int>(f & 0x0F0F0F0Fu);
-        const int hi = static_cast<int>((f >> 4) & 0x0F0F0F0Fu);
-        h0 = __dp2a_lo(xh[4 * i + 0], lo, h0);
-        l0 = __dp2a_lo(xl[4 * i + 0], lo, l0);
-        h1 = __dp2a_hi(xh[4 * i + 1], lo, h1);
-        l1 = __dp2a_hi(xl[4 * i + 1], lo, l1);
-        h0 = __dp2a_lo(xh[4 * i + 2], hi, h0);
-        l0 = __dp2a_lo(xl[4 * i + 2], hi, l0);
-        h1 = __dp2a_hi(xh[4 * i + 3], hi, h1);
-        l1 = __dp2a_hi(xl[4 * i + 3], hi, l1);
-    }
-    sh = h0 + h1;
-    sl = l0 + l1;
-}
-template <>
-__device__ __forceinline__ void idot2_chunk<8>(const uint4 q, const int *xh, const int *xl, int, int,
-                                               int &sh, int &sl) {
+__device__ __forceinline__ void idot4_chunk<4>(const uint4 q, const int *xh, const int *xl, int &sh, int &sl) {
+    // word i (codes 8i..8i+7): (w << 4) & 0xF0F0F0F0 holds codes 0,2,4,6, w & 0xF0F0F0F0 codes 1,3,5,7
     const uint32_t w[4] = {q.x, q.y, q.z, q.w};
     int h0 = 0, h1 = 0, l0 = 0, l1 = 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        h0 = __dp2a_lo(xh[2 * i + 0], static_cast<int>(w[i]), h0);
-        l0 = __dp2a_lo(xl[2 * i + 0], static_cast<int>(w[i]), l0);
-        h1 = __dp2a_hi(xh[2 * i + 1], static_cast<int>(w[i]), h1);
-        l1 = __dp2a_hi(xl[2 * i + 1], static_cast<int>(w[i]), l1);
+        const int ev = static_cast<int>((w[i] << 4) & 0xF0F0F0F0u);
+        const int od = static_cast<int>(w[i] & 0xF0F0F0F0u);
+        h0 = __dp4a(ev, xh[2 * i], h0);
+        l0 = __dp4a(ev, xl[2 * i], l0);
+        h1 = __dp4a(od, xh[2 * i + 1], h1);
+        l1 = __dp4a(od, xl[2 * i + 1], l1);
     }
     sh = h0 + h1;
     sl = l0 + l1;
 }
 template <>
-__device__ __forceinline__ void idot2_chunk<2>(const uint4 q, const int *xh, const int *xl, int ch, int cl,
-                                               int &sh, int &sl) {
+__device__ __forceinline__ void idot4_chunk<8>(const uint4 q, const int *xh, const int *xl, int &sh, int &sl) {
+    // signed bytes in natural order
     const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-    int h[2] = {-ch, 0}, l[2] = {-cl, 0};
+    int h0 = 0, h1 = 0, l0 = 0, l1 = 0;
+#pragma unroll
+    for (int i = 0; i < 4; i += 2) {
+        h0 = __dp4a(static_cast<int>(w[i]), xh[i], h0);
+        l0 = __dp4a(static_cast<int>(w[i]), xl[i], l0);
+        h1 = __dp4a(static_cast<int>(w[i + 1]), xh[i + 1], h1);
+        l1 = __dp4a(static_cast<int>(w[i + 1]), xl[i + 1], l1);
+    }
+    sh = h0 + h1;
+    sl = l0 + l1;
+}
+template <>
+__device__ __forceinline__ void idot4_chunk<2>(const uint4 q, const int *xh, const int *xl, int &sh, int &sl) {
+    // word i (codes 16i..16i+15): (w << (6 - 2k)) & 0xC0C0C0C0 holds codes k, 4+k, 8+k, 12+k
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    int h[2] = {0, 0}, l[2] = {0, 0};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const uint32_t f = w[i] ^ 0xAAAAAAAAu;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-            const int bb = static_cast<int>((f >> (2 * k)) & 0x03030303u);
-            h[k & 1] = __dp2a_lo(xh[8 * i + 2 * k + 0], bb, h[k & 1]);
-            l[k & 1] = __dp2a_lo(xl[8 * i + 2 * k + 0], bb, l[k & 1]);
-            h[k & 1] = __dp2a_hi(xh[8 * i + 2 * k + 1], bb, h[k & 1]);
-            l[k & 1] = __dp2a_hi(xl[8 * i + 2 * k + 1], bb, l[k & 1]);
+            const int bb = static_cast<int>((w[i] << (6 - 2 * k)) & 0xC0C0C0C0u);
+            h[k & 1] = __dp4a(bb, xh[4 * i + k], h[k & 1]);
+            l[k & 1] = __dp4a(bb, xl[4 * i + k], l[k & 1]);
         }
     }
     sh = h[0] + h[1];
     sl = l[0] + l[1];
 }
 
-// Position in a chunk's packed 16-bit layout (word index and half) of chunk element j, matching
-// idot_chunk / idot2_chunk.
+// Position of chunk element j in the chunk's int8x4 slice layout (word, byte), matching
+// idot4_chunk.
 template <int FMT>
-__device__ __forceinline__ void pack_slot(int j, int &word, int &half);
-template <>
-__device__ __forceinline__ void pack_slot<4>(int j, int &word, int &half) {
-    const int i = j >> 3, k = j & 7;  // word i of codes, element k
-    // (m0,m2) (m4,m6) (m1,m3) (m5,m7)
-    const int sub = (k & 1) ? ((k >> 2) ? 3 : 2) : ((k >> 2) ? 1 : 0);
-    word = 4 * i + sub;
-    half = (k >> 1) & 1;
-}
-template <>
-__device__ __forceinline__ void pack_slot<8>(int j, int &word, int &half) {
-    word = j >> 1;
-    half = j & 1;
-}
-template <>
-__device__ __forceinline__ void pack_slot<2>(int j, int &word, int &half) {
-    const int i = j >> 4, r = j & 15, k = r & 3, jb = r >> 2;  // element 16i + 4jb + k
-    word = 8 * i + 2 * k + (jb >> 1);
-    half = jb & 1;
+__device__ __forceinline__ void h_slot(int j, int &word, int &byte) {
+    if (FMT == 4) {
+        const int i = j >> 3, k = j & 7;
+        word = 2 * i + (k & 1);
+        byte = k >> 1;
+    } else if (FMT == 8) {
+        word = j >> 2;
+        byte = j & 3;
+    } else {
+        const int i = j >> 4, k = j & 15;
+        word = 4 * i + (k & 3);
+        byte = k >> 2;
+    }
 }
 
 __device__ __forceinline__ float warp_allsum(float v) {
@@ -787,8 +780,8 @@ __global__ void __maxnreg__(96) ffn_decode_kernel(DecodeParams p) {
     cons_sync();
 
     // ------------------------------------------------ phase 2: down + combine -------------
-    // h of one expert's slots is converted once per CTA into 29-bit fixed point split in two
-    // 16-bit halves per chunk (4 elements per thread, chunk maximum over 8 lanes), double
+    // h of one expert's slots is converted once per CTA into 16-bit fixed point per chunk split
+    // in two signed bytes (4 elements per thread, chunk maximum over the chunk's lanes), double
     // buffered; the next expert's h is prefetched into registers while the current one is used.
     const int p2 = ct / Li, c2 = ct % Li;
     const int P2 = p.P2;
@@ -801,12 +794,12 @@ __global__ void __maxnreg__(96) ffn_decode_kernel(DecodeParams p) {
     const int nrows = j_hi - j_lo;
     const int a0d = j_lo & ~3;
     const int nwe = f.S + U;
-    // buffer layout (int4 vectors): [buf][slot][part hi/lo][XV][Li]; per (buf, slot, chunk):
-    // scale (float) and the two corrections
+    // buffer layout (int4 vectors): [buf][slot][part hi/lo][XV8][Li]; per (buf, slot, chunk):
+    // one float scale
+    constexpr int XW8 = Ph2<FMT>::XW8, XV8 = Ph2<FMT>::XV8;
     int4 *hq = reinterpret_cast<int4 *>(sm + p.off_x);
-    const size_t hq_buf = static_cast<size_t>(TMAX) * 2 * XV * Li;       // int4 per buffer
+    const size_t hq_buf = static_cast<size_t>(TMAX) * 2 * XV8 * Li;      // int4 per buffer
     float *hsc = reinterpret_cast<float *>(sm + p.off_xs);                // [buf][slot][Li]
-    int *hcr = reinterpret_cast<int *>(sm + p.off_xc);                    // [buf][slot][2][Li]
     const int ngrp = f.I / 4;                                              // 4-element groups per slot
     float4 pre[TMAX];
     auto fetch_h = [&](int we) {
@@ -824,8 +817,7 @@ __global__ void __maxnreg__(96) ffn_decode_kernel(DecodeParams p) {
     auto convert_h = [&](int we, int buf) {
         const bool shd = we < f.S;
         const int cnt = shd ? T : rCnt[we];
-        const int c = ct >> 3, sub = ct & 7;  // 8 lanes per chunk of 32 elements (int4 codes)
-        constexpr int GPC = CPC / 4;          // 4-element groups per chunk
+        constexpr int GPC = CPC / 4;          // threads (4 elements each) per chunk
 #pragma unroll
         for (int q = 0; q < TMAX; ++q) {
             if (q < cnt) {
@@ -834,44 +826,25 @@ __global__ void __maxnreg__(96) ffn_decode_kernel(DecodeParams p) {
                 float mx = act ? fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3]))) : 0.f;
 #pragma unroll
                 for (int o = GPC / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
-                int ex = mx > 0.f ? static_cast<int>((__float_as_uint(mx) >> 23) & 0xFF) - 126 : 0;
-                ex = max(ex, -96);                                          // mx < 2^ex
-                const float up = __uint_as_float(static_cast<uint32_t>(127 + 29 - ex) << 23);  // 2^(29-ex)
-                int sum_h = 0, sum_l = 0;
+                const float inv = mx > 0.f ? __fdiv_rn(32512.0f, mx) : 0.f;
                 if (act) {
                     const int cc = (4 * ct) / CPC;                          // chunk of these elements
 #pragma unroll
                     for (int e2 = 0; e2 < 4; ++e2) {
                         const int j = (4 * ct + e2) % CPC;
-                        const float sc = __fmul_rn(v[e2], up);               // |sc| < 2^29
-                        const float th = __fmaf_rn(sc, 1.0f / 32768.0f, 12582912.0f);
-                        const int hi = static_cast<int>(__float_as_uint(th)) - 0x4B400000;
-                        const float r = __fmaf_rn(-__fsub_rn(th, 12582912.0f), 32768.0f, sc);  // exact
-                        const float tl = __fadd_rn(r, 12582912.0f);
-                        const int lo = static_cast<int>(__float_as_uint(tl)) - 0x4B400000;
-                        sum_h += hi;
-                        sum_l += lo;
-                        int word, half;
-                        pack_slot<FMT>(j, word, half);
-                        int16_t *ph = reinterpret_cast<int16_t *>(hq + buf * hq_buf + ((static_cast<size_t>(q) * 2 + 0) * XV + (word >> 2)) * Li + cc);
-                        int16_t *pl = reinterpret_cast<int16_t *>(hq + buf * hq_buf + ((static_cast<size_t>(q) * 2 + 1) * XV + (word >> 2)) * Li + cc);
-                        ph[2 * (word & 3) + half] = static_cast<int16_t>(hi);
-                        pl[2 * (word & 3) + half] = static_cast<int16_t>(lo);
+                        const int X = max(-32512, min(32512, __float2int_rn(__fmul_rn(v[e2], inv))));
+                        const int xh = (X + 128) >> 8;                      // in [-127, 127]
+                        const int xl = X - 256 * xh;                        // in [-128, 127]
+                        int word, byte;
+                        h_slot<FMT>(j, word, byte);
+                        int8_t *ph = reinterpret_cast<int8_t *>(hq + buf * hq_buf + ((static_cast<size_t>(q) * 2 + 0) * XV8 + (word >> 2)) * Li + cc);
+                        int8_t *pl = reinterpret_cast<int8_t *>(hq + buf * hq_buf + ((static_cast<size_t>(q) * 2 + 1) * XV8 + (word >> 2)) * Li + cc);
+                        ph[4 * (word & 3) + byte] = static_cast<int8_t>(xh);
+                        pl[4 * (word & 3) + byte] = static_cast<int8_t>(xl);
                     }
+                    if ((ct % GPC) == 0)
+                        hsc[(buf * TMAX + q) * Li + cc] = __fdiv_rn(mx, 32512.0f * Ph2<FMT>::MUL);
                 }
-#pragma unroll
-                for (int o = GPC / 2; o > 0; o >>= 1) {
-                    sum_h += __shfl_xor_sync(FULL, sum_h, o);
-                    sum_l += __shfl_xor_sync(FULL, sum_l, o);
-                }
-                if (act && (ct % GPC) == 0) {
-                    const int cc = (4 * ct) / CPC;
-                    const int bias = FMT == 4 ? 8 : (FMT == 2 ? 2 : 0);
-                    hsc[(buf * TMAX + q) * Li + cc] = __uint_as_float(static_cast<uint32_t>(127 - 29 + ex) << 23);
-                    hcr[((buf * TMAX + q) * 2 + 0) * Li + cc] = bias * sum_h;
-                    hcr[((buf * TMAX + q) * 2 + 1) * Li + cc] = bias * sum_l;
-                }
-                (void)c; (void)sub;
             }
         }
     };
@@ -896,25 +869,23 @@ __global__ void __maxnreg__(96) ffn_decode_kernel(DecodeParams p) {
             for (int q = 0; q < cnt; ++q) {
                 const int tok = shared ? q : rTok[beg + q];
                 const float wq = shared ? 1.0f : rW[beg + q];
-                int xh[XW], xl[XW];
+                int xh[XW8], xl[XW8];
 #pragma unroll
-                for (int v = 0; v < XV; ++v) {
-                    const int4 a4 = hq[buf * hq_buf + ((static_cast<size_t>(q) * 2 + 0) * XV + v) * Li + c2];
-                    const int4 b4 = hq[buf * hq_buf + ((static_cast<size_t>(q) * 2 + 1) * XV + v) * Li + c2];
+                for (int v = 0; v < XV8; ++v) {
+                    const int4 a4 = hq[buf * hq_buf + ((static_cast<size_t>(q) * 2 + 0) * XV8 + v) * Li + c2];
+                    const int4 b4 = hq[buf * hq_buf + ((static_cast<size_t>(q) * 2 + 1) * XV8 + v) * Li + c2];
                     xh[4 * v] = a4.x; xh[4 * v + 1] = a4.y; xh[4 * v + 2] = a4.z; xh[4 * v + 3] = a4.w;
                     xl[4 * v] = b4.x; xl[4 * v + 1] = b4.y; xl[4 * v + 2] = b4.z; xl[4 * v + 3] = b4.w;
                 }
                 const float hs = hsc[(buf * TMAX + q) * Li + c2];
-                const int ch = hcr[((buf * TMAX + q) * 2 + 0) * Li + c2];
-                const int cl = hcr[((buf * TMAX + q) * 2 + 1) * Li + c2];
 #pragma unroll
                 for (int m = 0; m < RPT2MAX; ++m) {
                     const int row = p2 + P2 * m;
                     if (row < nrows) {
                         const uint4 qd = lds128(st + static_cast<size_t>(row) * f.rb_i + c2 * 16);
                         int sh, sl;
-                        idot2_chunk<FMT>(qd, xh, xl, ch, cl, sh, sl);
-                        const float d = __fmul_rn(__fmaf_rn(static_cast<float>(sh), 32768.0f, static_cast<float>(sl)), hs);
+                        idot4_chunk<FMT>(qd, xh, xl, sh, sl);
+                        const float d = __fmul_rn(__fmaf_rn(static_cast<float>(sh), 256.0f, static_cast<float>(sl)), hs);
                         const float wsd = __fmul_rn(wq, sdp[row]);
 #pragma unroll
                         for (int t2 = 0; t2 < TMAX; ++t2)
