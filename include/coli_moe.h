@@ -105,7 +105,8 @@ coli_status coli_moe_check_config(const coli_moe_config *cfg);
 coli_status coli_moe_workspace_size(const coli_moe_config *cfg, int max_tokens, size_t *bytes);
 
 /* Number of kernels coli_moe_layer launches for T tokens with this configuration (1 on the fused
- * decode path: one persistent kernel for the whole layer; 5 otherwise).  Host only. */
+ * decode path: one persistent kernel for the whole layer; 7 on the tensor-core path; 5
+ * otherwise).  Host only. */
 coli_status coli_moe_layer_kernels(const coli_moe_config *cfg, int T, int *n_kernels);
 
 /* Zeroes the workspace header: the device error word and the counters (asynchronous). */

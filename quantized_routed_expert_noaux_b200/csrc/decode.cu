@@ -251,9 +251,9 @@ __device__ __forceinline__ bool beats(double va, int ia, double vb, int ib) {
 
 constexpr int RMAX_BLOCKS = 8;  // E <= 256 on the fused path
 struct RouteSmem {
-    double btop1[RMAX_BLOCKS], btop2[RMAX_BLOCKS], gsc[32];
+    double btop1[RMAX_BLOCKS], btop2[RMAX_BLOCKS];
     double cval[RMAX_BLOCKS * 8], cs[RMAX_BLOCKS * 8];  // per block: its K <= 8 best
-    int cid[RMAX_BLOCKS * 8], kept[32];
+    int cid[RMAX_BLOCKS * 8];
     double sel_s[32];
     int sel_id[32];
     int out_id[8];
@@ -263,88 +263,127 @@ struct RouteSmem {
 // Route token t with four consumer warps (w4 = warp index within the four, barrier id bar).
 // Experts are taken in blocks of 32 (one per lane); a group is a whole number of blocks (or
 // G = 1).  Per block: the two largest biased scores (group score) and the block's K best experts
-// by rank among its 32 lanes; the union of the kept blocks' K best (at most 32 candidates) is
-// ranked by one warp.  Selections, ties and weights are those of the per-token definition
-// (largest biased score, lower id on ties, weights from the unbiased scores renormalised in slot
-// order, times routed_scaling).  Writes the token's ids and weights into rs.
+// by rank among its 32 lanes; warp w4 handles blocks w4, w4 + 4 together so that their loads,
+// sigmoids and shuffles overlap.  Warp 0 then ranks the groups, takes the kept blocks' K best
+// (at most 32 candidates, one per lane) and ranks them.  Selections, ties and weights are those
+// of the per-token definition (largest biased score, lower id on ties, weights from the
+// unbiased scores renormalised in slot order, times routed_scaling).  Writes the token's ids and
+// weights into r.
 __device__ void route_token(const DecodeParams &p, int t, int w4, int lane, int bar, RouteSmem &r) {
     const int E = p.f.E, K = p.f.K, G = p.G, TG = p.TG;
     const int gs = E / G, nb = E / 32, bpg = gs / 32;
     const bool grouped = G > 1 && TG < G;
-    for (int bk = w4; bk < nb; bk += 4) {
-        const int e = bk * 32 + lane;
-        const double l = static_cast<double>(__ldcg(p.logits + static_cast<size_t>(t) * E + e));
-        const double s = 1.0 / (1.0 + exp(-l));
-        const double c = s + static_cast<double>(p.bias[e]);
-        if (grouped) {
-            double a1 = c, a2 = -INFINITY;
+    constexpr int BPW = RMAX_BLOCKS / 4;  // blocks per warp
+    double c[BPW], s[BPW];
+    float lf[BPW], bf[BPW];
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const double b1 = __shfl_xor_sync(FULL, a1, o);
-                const double b2 = __shfl_xor_sync(FULL, a2, o);
-                const double n1 = fmax(a1, b1);
-                const double n2 = fmax(fmin(a1, b1), fmax(a2, b2));
-                a1 = n1; a2 = n2;
+    for (int j = 0; j < BPW; ++j) {
+        const int e = (w4 + 4 * j) * 32 + lane;
+        const bool on = w4 + 4 * j < nb;
+        lf[j] = on ? __ldcg(p.logits + static_cast<size_t>(t) * E + e) : 0.f;
+        bf[j] = on ? __ldg(p.bias + e) : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < BPW; ++j) {
+        s[j] = 1.0 / (1.0 + exp(-static_cast<double>(lf[j])));
+        c[j] = s[j] + static_cast<double>(bf[j]);
+    }
+    if (grouped) {
+        double a1[BPW], a2[BPW];
+#pragma unroll
+        for (int j = 0; j < BPW; ++j) { a1[j] = c[j]; a2[j] = -INFINITY; }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+            for (int j = 0; j < BPW; ++j) {
+                const double b1 = __shfl_xor_sync(FULL, a1[j], o);
+                const double b2 = __shfl_xor_sync(FULL, a2[j], o);
+                const double n1 = fmax(a1[j], b1);
+                const double n2 = fmax(fmin(a1[j], b1), fmax(a2[j], b2));
+                a1[j] = n1; a2[j] = n2;
             }
-            if (lane == 0) { r.btop1[bk] = a1; r.btop2[bk] = a2; }
         }
-        int rank = 0;
-        for (int o = 0; o < 32; ++o) {
-            const double oc = __shfl_sync(FULL, c, o);
-            rank += beats(oc, bk * 32 + o, c, e);
+        if (lane == 0) {
+#pragma unroll
+            for (int j = 0; j < BPW; ++j)
+                if (w4 + 4 * j < nb) { r.btop1[w4 + 4 * j] = a1[j]; r.btop2[w4 + 4 * j] = a2[j]; }
         }
-        if (rank < K) {
-            r.cval[bk * K + rank] = c;
-            r.cs[bk * K + rank] = s;
-            r.cid[bk * K + rank] = e;
+    }
+    int rank[BPW];
+#pragma unroll
+    for (int j = 0; j < BPW; ++j) rank[j] = 0;
+#pragma unroll
+    for (int o = 0; o < 32; ++o) {
+#pragma unroll
+        for (int j = 0; j < BPW; ++j) {
+            const double oc = __shfl_sync(FULL, c[j], o);
+            rank[j] += (oc > c[j] || (oc == c[j] && o < lane)) ? 1 : 0;  // same block: id order = lane order
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < BPW; ++j) {
+        const int bk = w4 + 4 * j;
+        if (bk < nb && rank[j] < K) {
+            r.cval[bk * K + rank[j]] = c[j];
+            r.cs[bk * K + rank[j]] = s[j];
+            r.cid[bk * K + rank[j]] = bk * 32 + lane;
         }
     }
     named_sync(bar, 128);
+    if (w4 != 0) return;
+    // kept blocks: all, or those of the TG best groups (group g = lane)
+    unsigned kmask;
     if (grouped) {
-        const int tid = w4 * 32 + lane;
-        for (int g = tid; g < G; g += 128) {
+        double gsc = -INFINITY;
+        if (lane < G) {
             double a1 = -INFINITY, a2 = -INFINITY;
-            for (int bk = g * bpg; bk < (g + 1) * bpg; ++bk) {
+            for (int bk = lane * bpg; bk < (lane + 1) * bpg; ++bk) {
                 const double v[2] = {r.btop1[bk], r.btop2[bk]};
+#pragma unroll
                 for (int k = 0; k < 2; ++k) {
                     if (v[k] > a1) { a2 = a1; a1 = v[k]; }
                     else if (v[k] > a2) { a2 = v[k]; }
                 }
             }
-            r.gsc[g] = a1 + a2;
+            gsc = a1 + a2;
         }
-        named_sync(bar, 128);
-        for (int g = tid; g < G; g += 128) {
-            int rk = 0;
-            for (int h = 0; h < G; ++h) rk += beats(r.gsc[h], h, r.gsc[g], g);
-            r.kept[g] = rk < TG;
-        }
-        named_sync(bar, 128);
-    }
-    if (w4 == 0) {
-        double c = -INFINITY, s = 0.0;
-        int id = 0x7fffffff;
-        int n = 0;
-        for (int bk = 0; bk < nb; ++bk) {
-            const bool keep = !grouped || r.kept[(bk * 32) / gs];
-            if (!keep) continue;
-            for (int k = 0; k < K; ++k, ++n)
-                if (n == lane) { c = r.cval[bk * K + k]; s = r.cs[bk * K + k]; id = r.cid[bk * K + k]; }
-        }
-        int rank = 0;
+        int rk = 0;
+#pragma unroll
         for (int o = 0; o < 32; ++o) {
-            const double oc = __shfl_sync(FULL, c, o);
-            const int oi = __shfl_sync(FULL, id, o);
-            rank += beats(oc, oi, c, id);
+            const double og = __shfl_sync(FULL, gsc, o);
+            rk += (o < G && (og > gsc || (og == gsc && o < lane))) ? 1 : 0;
         }
-        if (rank < K) { r.sel_s[rank] = s; r.sel_id[rank] = id; }
-        __syncwarp();
-        if (lane < K) {
-            double denom = 0.0;
-            for (int k = 0; k < K; ++k) denom += r.sel_s[k];
-            r.out_id[lane] = r.sel_id[lane];
-            r.out_w[lane] = static_cast<float>((r.sel_s[lane] / denom) * p.rsf);
-        }
+        const unsigned gmask = __ballot_sync(FULL, lane < G && rk < TG);
+        kmask = __ballot_sync(FULL, lane < nb && ((gmask >> ((lane * 32) / gs)) & 1u));
+    } else {
+        kmask = __ballot_sync(FULL, lane < nb);
+    }
+    // candidate of this lane: rank k of the kb-th kept block
+    double c2 = -INFINITY, s2 = 0.0;
+    int id = 0x7fffffff;
+    if (lane < __popc(kmask) * K) {
+        const int kb = lane / K, k = lane - kb * K;
+        unsigned m = kmask;
+        for (int i = 0; i < kb; ++i) m &= m - 1u;  // drop the kb lowest kept blocks
+        const int bk = __ffs(m) - 1;
+        c2 = r.cval[bk * K + k];
+        s2 = r.cs[bk * K + k];
+        id = r.cid[bk * K + k];
+    }
+    int rank2 = 0;
+#pragma unroll
+    for (int o = 0; o < 32; ++o) {
+        const double oc = __shfl_sync(FULL, c2, o);
+        const int oi = __shfl_sync(FULL, id, o);
+        rank2 += beats(oc, oi, c2, id) ? 1 : 0;
+    }
+    if (rank2 < K) { r.sel_s[rank2] = s2; r.sel_id[rank2] = id; }
+    __syncwarp();
+    if (lane < K) {
+        double denom = 0.0;
+        for (int k = 0; k < K; ++k) denom += r.sel_s[k];
+        r.out_id[lane] = r.sel_id[lane];
+        r.out_w[lane] = static_cast<float>((r.sel_s[lane] / denom) * p.rsf);
     }
 }
 
@@ -543,17 +582,24 @@ __global__ void __maxnreg__(96) ffn_decode_kernel(DecodeParams p) {
             if (cw < 4 * T) route_token(p, cw >> 2, cw & 3, lane, 2 + (cw >> 2), rsm[cw >> 2]);
             cons_sync();
             if (cw == 0) {
+                // slot s0 = lane: token s0 / K, rank s0 % K; stable sort of the slots by expert id
                 const int s0 = lane;
-                const int id = s0 < n ? rsm[s0 / f.K].out_id[s0 % f.K] : 0x7fffffff;
+                const int t0 = s0 < n ? s0 / f.K : 0;
+                const int id = s0 < n ? rsm[t0].out_id[s0 - t0 * f.K] : 0x7fffffff;
+                const float w0 = s0 < n ? rsm[t0].out_w[s0 - t0 * f.K] : 0.f;
                 int rk = 0;
+#pragma unroll
                 for (int o = 0; o < 32; ++o) {
                     const int oid = __shfl_sync(FULL, id, o);
-                    rk += (oid < id) || (oid == id && o < lane);
+                    rk += ((oid < id) || (oid == id && o < lane)) ? 1 : 0;
                 }
                 if (s0 < n) sorted_slot[rk] = s0;
                 __syncwarp();
+                // position `lane` of the grouped order holds slot sl
                 const int sl = lane < n ? sorted_slot[lane] : 0;
-                const int idr = lane < n ? rsm[sl / f.K].out_id[sl % f.K] : 0x7fffffff;
+                const int idr = __shfl_sync(FULL, id, sl);
+                const int tr = __shfl_sync(FULL, t0, sl);
+                const float wr = __shfl_sync(FULL, w0, sl);
                 const int idp = __shfl_up_sync(FULL, idr, 1);
                 const bool first = lane < n && (lane == 0 || idp != idr);
                 const unsigned m = __ballot_sync(FULL, first);
@@ -567,15 +613,15 @@ __global__ void __maxnreg__(96) ffn_decode_kernel(DecodeParams p) {
                     rUniq[up] = idr;
                 }
                 if (lane < n) {
-                    rTok[lane] = sl / f.K;
-                    rW[lane] = rsm[sl / f.K].out_w[sl % f.K];
+                    rTok[lane] = tr;
+                    rW[lane] = wr;
                     rH[lane] = lane;
                 }
                 if (lane == 0) *rU = U;
                 if (blockIdx.x == 0) {  // the routing outputs of the call
                     if (s0 < n) {
                         p.ids[s0] = id;
-                        p.wts[s0] = rsm[s0 / f.K].out_w[s0 % f.K];
+                        p.wts[s0] = w0;
                     }
                     if (lane < n) p.f_perm[lane] = sl;
                     if (first) p.f_unique[up] = idr;
