@@ -20,11 +20,18 @@ _L = {}
 TC_KERNELS = 7  # gate, route, group, x quantisation, gate/up GEMM, h quantisation, down GEMM
 
 
+# f32 activations and four 64-row gate/up m-blocks: the tiny layer's router and expert counts at
+# the smallest shape the tensor-core path takes (hidden and inter multiples of 256)
+_EXTRA = {"tiny_wide": synth.WORKLOADS["tiny"].replace(name="tiny_wide", hidden=512, inter=256,
+                                                      shared_inter=256)}
+
+
 def layer(name):
     if name not in _L:
         _L.clear()
         torch.cuda.empty_cache()
-        _L[name] = Layer(synth.WORKLOADS[name], "cuda", 0)
+        wl = _EXTRA[name] if name in _EXTRA else synth.WORKLOADS[name]
+        _L[name] = Layer(wl, "cuda", 0)
     return _L[name]
 
 
@@ -49,12 +56,12 @@ def _routing(L, ocfg, x, T, routing):
     return ids_np, w_np
 
 
-# (workload, tokens, routing): chunks of 1..128 tokens with ragged tails; one expert with exactly
-# 128 and with 160 tokens (two chunks); just above the 64-token threshold; f32 activations and
-# two m-blocks (tiny); no shared expert (olmoe).
+# (workload, tokens, routing): chunks of 1..96 tokens with ragged tails; one expert with 128 and
+# with 160 tokens (two chunks each); just above the 64-token threshold; f32 activations and
+# four gate/up m-blocks (tiny_wide); no shared expert (olmoe).
 CASES = [("glm_decode", 96, "oracle"), ("glm_decode", 300, "oracle"), ("glm_decode", 160, "one_expert"),
          ("glm_decode", 128, "one_expert"), ("glm_decode", 65, "oracle"), ("olmoe", 200, "oracle"),
-         ("olmoe", 97, "one_expert"), ("tiny", 100, "oracle")]
+         ("olmoe", 97, "one_expert"), ("tiny_wide", 100, "oracle")]
 
 
 @pytest.mark.parametrize("name,T,routing", CASES)
