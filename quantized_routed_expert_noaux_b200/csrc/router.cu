@@ -5,6 +5,7 @@
 // gate sums exact double products in double and rounds once to float32; selection compares in
 // double, so the float32 logits and the chosen experts do not depend on summation order beyond
 // double rounding.
+#include <cooperative_groups.h>
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -80,8 +81,10 @@ __global__ void __launch_bounds__(128) gate_rows_kernel(const float *__restrict_
 // logits[T,E] = X[T,H] * Wr[E,H]^T on the fp64 tensor cores (mma.sync m8n8k4, double operands
 // and accumulators): every product of a bf16 or float32 activation and a float32 weight is exact
 // in double and sums are double, as in the per-row kernel above; only the summation order
-// differs.  CTA tile 64 tokens x 32 experts (4 warps of 32 x 16), K chunks of 32 staged in
-// shared memory as double, the next chunk's global loads in flight during the current chunk.
+// differs.  A cluster of two CTAs computes one 64-token x 32-expert tile, each CTA one half of
+// H (4 warps of 32 x 16, K chunks of 32 staged in shared memory as double, the next chunk's
+// global loads in flight during the current chunk); the second CTA's partial sums go into the
+// first CTA's shared memory and are added in a fixed order (first half + second half).
 constexpr int GM = 64, GN = 32, GK = 32;
 constexpr int GKP = GK + 4;  // row pitch (doubles): the 8 x 4 fragment reads hit each bank twice
 
@@ -91,13 +94,17 @@ __device__ __forceinline__ void dmma(double &d0, double &d1, double a, double b)
 }
 
 template <int ACT>
-__global__ void __launch_bounds__(128) gate_dmma_kernel(const float *__restrict__ Wr,
-                                                        const void *__restrict__ x, int T, int H,
-                                                        int E, float *__restrict__ logits) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128)
+gate_dmma_kernel(const float *__restrict__ Wr, const void *__restrict__ x, int T, int H, int E,
+                 float *__restrict__ logits) {
     __shared__ double xs[GM][GKP];
     __shared__ double ws[GN][GKP];
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    const unsigned kh = cluster.block_rank();  // 0: first half of H, 1: second half
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int t0 = blockIdx.y * GM, e0 = blockIdx.x * GN;
+    const int t0 = blockIdx.y * GM, e0 = (blockIdx.x >> 1) * GN;
+    const int kbeg = static_cast<int>(kh) * (H / 2), kend = kbeg + H / 2;
     // staging: x row tid/2, k [16*(tid%2), +16); Wr row tid/4, k [8*(tid%4), +8)
     const int xr = tid >> 1, xk = 16 * (tid & 1);
     const int wr = tid >> 2, wk = 8 * (tid & 3);
@@ -151,15 +158,15 @@ __global__ void __launch_bounds__(128) gate_dmma_kernel(const float *__restrict_
 #pragma unroll
         for (int j = 0; j < 2; ++j) acc[i][j][0] = acc[i][j][1] = 0.0;
 
-    load(0);
-    for (int k0 = 0; k0 < H; k0 += GK) {
+    load(kbeg);
+    for (int k0 = kbeg; k0 < kend; k0 += GK) {
         __syncthreads();  // the previous chunk's fragments have been read
 #pragma unroll
         for (int i = 0; i < 16; ++i) xs[xr][xk + i] = static_cast<double>(xv[i]);
 #pragma unroll
         for (int i = 0; i < 8; ++i) ws[wr][wk + i] = static_cast<double>(wv[i]);
         __syncthreads();
-        if (k0 + GK < H) load(k0 + GK);
+        if (k0 + GK < kend) load(k0 + GK);
 #pragma unroll
         for (int k4 = 0; k4 < GK; k4 += 4) {
             double a[4], b[2];
@@ -173,6 +180,27 @@ __global__ void __launch_bounds__(128) gate_dmma_kernel(const float *__restrict_
                 for (int j = 0; j < 2; ++j) dmma(acc[i][j][0], acc[i][j][1], a[i], b[j]);
         }
     }
+    // second half's partial sums into the first CTA's shared memory (its staging buffer, free
+    // once both CTAs are past the first cluster barrier), then first + second in that order
+    double *xch = &xs[0][0];  // 16 doubles per thread, element i of thread tid at [i * 128 + tid]
+    cluster.sync();
+    if (kh == 1) {
+        double *dst = cluster.map_shared_rank(xch, 0);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) dst[((i * 2 + j) * 2 + h) * 128 + tid] = acc[i][j][h];
+    }
+    cluster.sync();
+    if (kh == 1) return;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) acc[i][j][h] = acc[i][j][h] + xch[((i * 2 + j) * 2 + h) * 128 + tid];
     // accumulator (i, j): token 32*wm + 8*i + fr, experts 16*wn + 8*j + 2*fk + {0, 1}
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -389,7 +417,7 @@ cudaError_t launch_gate(const coli_moe_config &c, const float *Wr, const void *x
         else
             gate_rows_kernel<COLI_ACT_BF16, 8><<<grid, 128, 0, st>>>(Wr, x, T, H, E, logits);
     } else {
-        dim3 grid((E + GN - 1) / GN, (T + GM - 1) / GM);
+        dim3 grid(2 * ((E + GN - 1) / GN), (T + GM - 1) / GM);  // clusters of two CTAs along x
         if (c.act == COLI_ACT_F32)
             gate_dmma_kernel<COLI_ACT_F32><<<grid, 128, 0, st>>>(Wr, x, T, H, E, logits);
         else
