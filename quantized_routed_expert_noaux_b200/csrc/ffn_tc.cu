@@ -19,21 +19,20 @@
 //
 // One persistent CTA per SM, warp-specialised, tiles (chunk of <= 96 tokens of one expert x one
 // block of weight rows) taken round-robin:
-//   warp 12     A producer: per k-block of 256, the packed A tile (128 rows x 128 B, 128-byte
+//   warp 12     A producer: per k-block of 128, the packed A tile (128 rows x 64 B, 64-byte
 //               swizzle; one 4-D box holds the gate and the up rows) into the A ring, whose stages
 //               the converters release as soon as they have read them.
-//   warp 14     B producer: the k-block's B rows as two 128-byte-wide halves (boxes of
-//               128/64/32/16 rows, 128-byte swizzle) into the B ring, released by the MMAs'
-//               completion; one lane per box.
+//   warp 14     B producer: the k-block's B rows (boxes of 128/64/32/16 rows of 128 B, 128-byte
+//               swizzle) into the B ring, released by the MMAs' completion; one lane per box.
 //   warps 0-3   converters: one thread per weight row unpacks its 64 bytes into 128 signed bytes
 //               and stores them with tcgen05.st into a TMEM A stage; the MMA reads A from tensor
 //               memory, so unpacked weights never pass through shared memory.
-//   warp 13     MMA issuer (one elected lane, operands computed warp-uniformly): 8 x tcgen05.mma
+//   warp 13     MMA issuer (one elected lane, operands computed warp-uniformly): 4 x tcgen05.mma
 //               (K = 32, N <= 192) per k-block into one of two TMEM accumulators, so a tile's
 //               epilogue overlaps the next tile's main loop.
 //   warps 4-11  epilogue: tcgen05.ld of the accumulator and the output arithmetic; the tile's
 //               per-token scales, tokens and weights are staged in shared memory first.
-// TMEM (512 columns): accumulator b at columns [256b, 256b + 192); the two 64-column A stages
+// TMEM (512 columns): accumulator b at columns [256b, 256b + 192); the four 32-column A stages
 // fill the gaps [192, 256) and [448, 512).
 // Inside every group of 8 k the order is permuted to (0,2,4,6,1,3,5,7) on both operands: the
 // unpacking yields the even and the odd codes of a word as separate words, and the activation
@@ -50,20 +49,18 @@ namespace coli {
 
 namespace {
 
-constexpr int KB = 256;                       // k per ring stage (two 128-byte B halves)
+constexpr int KB = 128;                       // k per ring stage
 constexpr int MAXTOK = 96;                    // tokens per chunk: N = 192 (hi and lo row per token)
-constexpr int NA = 4;                         // A ring stages (packed int4 tiles)
-constexpr int NB = 3;                         // B ring stages
-constexpr int A_RAW = 128 * (KB / 2);         // packed int4 A tile: 16 KB
-constexpr int B_HALF = 2 * MAXTOK * 128;      // B rows of one 128-byte half: 24 KB
-constexpr int B_MAX = 2 * B_HALF;             // B rows of one stage: 48 KB
+constexpr int NA = 8;                         // A ring stages (packed int4 tiles)
+constexpr int NB = 6;                         // B ring stages
+constexpr int A_RAW = 128 * (KB / 2);         // packed int4 A tile: 8 KB
+constexpr int B_MAX = 2 * MAXTOK * KB;        // B rows of one stage: 24 KB
 constexpr int NBOX = 4;                       // B box heights 16 << i rows
 constexpr int W_CONV = 4, W_EPI0 = 4, N_EPI = 8, W_PRODA = 12, W_MMA = 13, W_PRODB = 14;
 constexpr int TC_THREADS = 15 * 32;
 constexpr uint32_t D_STRIDE = 256;            // accumulator b at TMEM column 256 * b
 constexpr uint32_t A_COL0 = 2 * MAXTOK;       // TMEM column of A stage 0
-constexpr int ACOLS = KB / 4;                 // TMEM columns of one A stage (4 signed bytes each)
-constexpr int SPG = (256 - 2 * MAXTOK) / ACOLS;  // A stages in the gap after each accumulator
+constexpr int SPG = (256 - 2 * MAXTOK) / 32;  // 32-column A stages in the gap after each accumulator
 constexpr int NTS = 2 * SPG;                  // TMEM A stages
 static_assert(SPG >= 1, "no room for TMEM A stages");
 constexpr uint32_t TMEM_COLS = 512;
@@ -202,7 +199,7 @@ __device__ __forceinline__ bool epi_sync_or(bool pred) {
 __device__ __forceinline__ int round16(int v) { return (v + 15) & ~15; }
 // TMEM column of A stage j: the gaps [2 * MAXTOK, 256) and [256 + 2 * MAXTOK, 512).
 __device__ __forceinline__ uint32_t a_col(int j) {
-    return static_cast<uint32_t>(j / SPG) * D_STRIDE + A_COL0 + static_cast<uint32_t>(ACOLS) * static_cast<uint32_t>(j % SPG);
+    return static_cast<uint32_t>(j / SPG) * D_STRIDE + A_COL0 + 32u * static_cast<uint32_t>(j % SPG);
 }
 __device__ __forceinline__ bool elect_one() {
     uint32_t pred = 0;
@@ -473,8 +470,8 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const GemmArgs p) {
     unsigned char *sb = sm + static_cast<size_t>(NA) * A_RAW;      // B ring
     if (warp == W_PRODA || warp == W_PRODB) {
         // ------------------------------------------------------------------ TMA producers
-        // A warp, lane 0: the A box.  B warp, lane 4h + i (h: 128-byte half of the k-block): the
-        // box of 128 >> i rows when bit 3 - i of nrows/16 is set.
+        // A warp, lane 0: the A box.  B warp, lane i < 4: the box of 128 >> i rows when bit 3 - i
+        // of nrows/16 is set.
         const bool is_a = warp == W_PRODA;
         const int nst = is_a ? NA : NB;
         uint64_t *fullb = is_a ? afull : bfull, *emptyb = is_a ? aempty : bempty;
@@ -494,12 +491,11 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const GemmArgs p) {
                 __syncwarp();
                 if (is_a) {
                     if (lane == 0) tma_load_4d(smem_u32(sa + s * A_RAW), ta, kb * (KB / 2), m * MROWS, 0, ez, fb);
-                } else if (lane < 2 * NBOX) {
-                    const int h = lane / NBOX, bit = NBOX - 1 - lane % NBOX;
+                } else if (lane < NBOX) {
+                    const int bit = NBOX - 1 - lane;
                     if ((n16 >> bit) & 1) {
                         const int row0 = 16 * ((n16 >> (bit + 1)) << (bit + 1));  // rows of the larger boxes
-                        tma_load_2d(smem_u32(sb + s * B_MAX + h * B_HALF + row0 * 128), &maps.b[bit],
-                                    kb * KB + 128 * h, 2 * c.y + row0, fb);
+                        tma_load_2d(smem_u32(sb + s * B_MAX + row0 * KB), &maps.b[bit], kb * KB, 2 * c.y + row0, fb);
                     }
                 }
             }
@@ -515,7 +511,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const GemmArgs p) {
         // the whole warp runs the loop (uniform operands); one elected lane issues
         uint32_t it = 0, tl = 0;
         // B descriptor of stage s, k-step kk: the start-address field (bits 0-13, address >> 4)
-        // advances by B_MAX >> 4 per stage, B_HALF >> 4 per 128-byte half and 2 per 32-byte step
+        // advances by B_MAX >> 4 per stage and by 2 per 32-byte k-step
         const uint64_t bdesc0 = smem_desc_sw128(smem_u32(sb));
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tl) {
             const int4 c = p.chunks[t / MB];
@@ -538,7 +534,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const GemmArgs p) {
                 if (elect_one()) {
 #pragma unroll
                     for (int kk = 0; kk < KB / 32; ++kk)
-                        mma_i8(dt, a0 + kk * 8, bd + (kk >> 2) * (B_HALF >> 4) + 2 * (kk & 3), idesc, (kb | kk) != 0);
+                        mma_i8(dt, a0 + kk * 8, bd + 2 * kk, idesc, (kb | kk) != 0);
                     mma_commit(smem_u32(&bempty[s]));
                     mma_commit(smem_u32(&tempty[ts]));
                 }
@@ -556,7 +552,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const GemmArgs p) {
         // ------------------------------------------------------------------ converters
         const int q = warp;
         const int rho = PHASE == 1 ? (lane < 16 ? 16 * q + lane : 64 + 16 * q + (lane - 16)) : 32 * q + lane;
-        const int swz = rho & 7;  // 128-byte swizzle: 16-byte chunk c of row r sits at c ^ (r & 7)
+        const int swz = (rho >> 1) & 3;  // 64-byte swizzle: 16-byte chunk c of row r sits at c ^ ((r >> 1) & 3)
         const uint32_t ta = tbase + (static_cast<uint32_t>(32 * q) << 16);
         uint32_t it = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
@@ -565,28 +561,24 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const GemmArgs p) {
                 if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&afull[s]), (it / NA) & 1, abort, f.err)))
                     goto conv_done;
                 const unsigned char *row = sa + s * A_RAW + rho * (KB / 2);
-                uint4 v[8];
+                uint4 v[4];
 #pragma unroll
-                for (int cch = 0; cch < 8; ++cch) v[cch] = *reinterpret_cast<const uint4 *>(row + ((cch ^ swz) << 4));
+                for (int cch = 0; cch < 4; ++cch) v[cch] = *reinterpret_cast<const uint4 *>(row + ((cch ^ swz) << 4));
                 mbar_arrive(smem_u32(&aempty[s]));
+                uint32_t o[32];
+#pragma unroll
+                for (int cch = 0; cch < 4; ++cch) {
+                    const uint32_t w4[4] = {v[cch].x, v[cch].y, v[cch].z, v[cch].w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        o[8 * cch + 2 * i] = (w4[i] << 4) & 0xF0F0F0F0u;  // codes 0,2,4,6 of the word
+                        o[8 * cch + 2 * i + 1] = w4[i] & 0xF0F0F0F0u;     // codes 1,3,5,7
+                    }
+                }
                 if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&tempty[ts]), ((it / NTS) & 1) ^ 1, abort, f.err)))
                     goto conv_done;
                 tc_fence_after();
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {  // two halves of 128 codes = 32 TMEM columns each
-                    uint32_t o[32];
-#pragma unroll
-                    for (int cch = 0; cch < 4; ++cch) {
-                        const uint4 vv = v[4 * hh + cch];
-                        const uint32_t w4[4] = {vv.x, vv.y, vv.z, vv.w};
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            o[8 * cch + 2 * i] = (w4[i] << 4) & 0xF0F0F0F0u;  // codes 0,2,4,6 of the word
-                            o[8 * cch + 2 * i + 1] = w4[i] & 0xF0F0F0F0u;     // codes 1,3,5,7
-                        }
-                    }
-                    tmem_st32(ta + a_col(ts) + 32 * hh, o);
-                }
+                tmem_st32(ta + a_col(ts), o);
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(smem_u32(&tfull[ts]));
@@ -707,14 +699,14 @@ bool weight_map(CUtensorMap *m, const uint8_t *base, size_t row_bytes, size_t ro
     const cuuint64_t dims[4] = {row_bytes, rows, mats, nrec};
     const cuuint64_t strides[3] = {row_bytes, rows * row_bytes, rec_stride};
     const cuuint32_t box[4] = {KB / 2, box_rows, box_mats, 1};
-    return encode_u8(m, base, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+    return encode_u8(m, base, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 // Quantised B rows {len bytes, 2 * slots rows}, boxes of `box_rows` rows.
 bool act_map(CUtensorMap *m, const int8_t *base, size_t len, size_t rows, cuuint32_t box_rows) {
     const cuuint64_t dims[2] = {len, rows};
     const cuuint64_t strides[1] = {len};
-    const cuuint32_t box[2] = {128, box_rows};
+    const cuuint32_t box[2] = {KB, box_rows};
     return encode_u8(m, base, 2, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
@@ -734,9 +726,9 @@ int tc_max_chunks(const coli_moe_config &c, int T) {
 }
 
 bool tc_shape_ok(const coli_moe_config &c) {
-    // m-blocks of 64 (gate/up) and 128 (down) rows, k-blocks of 256, int32 accumulators exact
+    // m-blocks of 64 (gate/up) and 128 (down) rows, k-blocks of 128, int32 accumulators exact
     // for K <= 65536 (|16q * X| <= 2^14 per product)
-    return c.wfmt == COLI_W_INT4 && c.hidden % KB == 0 && c.inter % KB == 0 && c.hidden <= 65536 &&
+    return c.wfmt == COLI_W_INT4 && c.hidden % 128 == 0 && c.inter % 128 == 0 && c.hidden <= 65536 &&
            c.inter <= 65536;
 }
 

@@ -81,10 +81,11 @@ __global__ void __launch_bounds__(128) gate_rows_kernel(const float *__restrict_
 // logits[T,E] = X[T,H] * Wr[E,H]^T on the fp64 tensor cores (mma.sync m8n8k4, double operands
 // and accumulators): every product of a bf16 or float32 activation and a float32 weight is exact
 // in double and sums are double, as in the per-row kernel above; only the summation order
-// differs.  A cluster of two CTAs computes one 64-token x 32-expert tile, each CTA one half of
-// H (4 warps of 32 x 16, K chunks of 32 staged in shared memory as double, the next chunk's
-// global loads in flight during the current chunk); the second CTA's partial sums go into the
-// first CTA's shared memory and are added in a fixed order (first half + second half).
+// differs.  A cluster of CL CTAs (2 or 4) computes one 64-token x 32-expert tile, each CTA one
+// CL-th of H (4 warps of 32 x 16, K chunks of 32 staged in shared memory as double, the next
+// chunk's global loads in flight during the current chunk); partial sums travel through
+// distributed shared memory and are added pairwise in a fixed order: p0 + p1 (and p2 + p3,
+// then (p0 + p1) + (p2 + p3)).
 constexpr int GM = 64, GN = 32, GK = 32;
 constexpr int GKP = GK + 4;  // row pitch (doubles): the 8 x 4 fragment reads hit each bank twice
 
@@ -93,18 +94,18 @@ __device__ __forceinline__ void dmma(double &d0, double &d1, double a, double b)
                  : "+d"(d0), "+d"(d1) : "d"(a), "d"(b));
 }
 
-template <int ACT>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128)
+template <int ACT, int CL>
+__global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(128)
 gate_dmma_kernel(const float *__restrict__ Wr, const void *__restrict__ x, int T, int H, int E,
                  float *__restrict__ logits) {
     __shared__ double xs[GM][GKP];
     __shared__ double ws[GN][GKP];
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
-    const unsigned kh = cluster.block_rank();  // 0: first half of H, 1: second half
+    const int kr = static_cast<int>(cluster.block_rank());  // part kr of H
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int t0 = blockIdx.y * GM, e0 = (blockIdx.x >> 1) * GN;
-    const int kbeg = static_cast<int>(kh) * (H / 2), kend = kbeg + H / 2;
+    const int t0 = blockIdx.y * GM, e0 = (blockIdx.x / CL) * GN;
+    const int kbeg = kr * (H / CL), kend = kbeg + H / CL;
     // staging: x row tid/2, k [16*(tid%2), +16); Wr row tid/4, k [8*(tid%4), +8)
     const int xr = tid >> 1, xk = 16 * (tid & 1);
     const int wr = tid >> 2, wk = 8 * (tid & 3);
@@ -180,27 +181,37 @@ gate_dmma_kernel(const float *__restrict__ Wr, const void *__restrict__ x, int T
                 for (int j = 0; j < 2; ++j) dmma(acc[i][j][0], acc[i][j][1], a[i], b[j]);
         }
     }
-    // second half's partial sums into the first CTA's shared memory (its staging buffer, free
-    // once both CTAs are past the first cluster barrier), then first + second in that order
+    // partial sums through the partner's shared memory (its staging buffer, free once every CTA
+    // of the cluster is past the barrier before the copy); every CTA takes every barrier
     double *xch = &xs[0][0];  // 16 doubles per thread, element i of thread tid at [i * 128 + tid]
-    cluster.sync();
-    if (kh == 1) {
-        double *dst = cluster.map_shared_rank(xch, 0);
+    auto send = [&](int to) {
+        double *dst = cluster.map_shared_rank(xch, to);
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
             for (int j = 0; j < 2; ++j)
 #pragma unroll
                 for (int h = 0; h < 2; ++h) dst[((i * 2 + j) * 2 + h) * 128 + tid] = acc[i][j][h];
-    }
+    };
+    auto take = [&]() {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) acc[i][j][h] = acc[i][j][h] + xch[((i * 2 + j) * 2 + h) * 128 + tid];
+    };
     cluster.sync();
-    if (kh == 1) return;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) acc[i][j][h] = acc[i][j][h] + xch[((i * 2 + j) * 2 + h) * 128 + tid];
+    if (kr & 1) send(kr - 1);  // p1 -> rank 0, p3 -> rank 2
+    cluster.sync();
+    if (!(kr & 1)) take();     // rank 0: p0 + p1; rank 2: p2 + p3
+    if (CL == 4) {
+        cluster.sync();        // rank 0 has read its buffer
+        if (kr == 2) send(0);
+        cluster.sync();
+        if (kr == 0) take();   // (p0 + p1) + (p2 + p3)
+    }
+    if (kr != 0) return;
     // accumulator (i, j): token 32*wm + 8*i + fr, experts 16*wn + 8*j + 2*fk + {0, 1}
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -417,11 +428,20 @@ cudaError_t launch_gate(const coli_moe_config &c, const float *Wr, const void *x
         else
             gate_rows_kernel<COLI_ACT_BF16, 8><<<grid, 128, 0, st>>>(Wr, x, T, H, E, logits);
     } else {
-        dim3 grid(2 * ((E + GN - 1) / GN), (T + GM - 1) / GM);  // clusters of two CTAs along x
-        if (c.act == COLI_ACT_F32)
-            gate_dmma_kernel<COLI_ACT_F32><<<grid, 128, 0, st>>>(Wr, x, T, H, E, logits);
-        else
-            gate_dmma_kernel<COLI_ACT_BF16><<<grid, 128, 0, st>>>(Wr, x, T, H, E, logits);
+        // clusters of CL CTAs along x, each CTA a CL-th of H (a whole number of 32-wide chunks)
+        const int cl = H % (4 * GK) == 0 ? 4 : 2;
+        dim3 grid(cl * ((E + GN - 1) / GN), (T + GM - 1) / GM);
+        if (cl == 4) {
+            if (c.act == COLI_ACT_F32)
+                gate_dmma_kernel<COLI_ACT_F32, 4><<<grid, 128, 0, st>>>(Wr, x, T, H, E, logits);
+            else
+                gate_dmma_kernel<COLI_ACT_BF16, 4><<<grid, 128, 0, st>>>(Wr, x, T, H, E, logits);
+        } else {
+            if (c.act == COLI_ACT_F32)
+                gate_dmma_kernel<COLI_ACT_F32, 2><<<grid, 128, 0, st>>>(Wr, x, T, H, E, logits);
+            else
+                gate_dmma_kernel<COLI_ACT_BF16, 2><<<grid, 128, 0, st>>>(Wr, x, T, H, E, logits);
+        }
     }
     return cudaGetLastError();
 }

@@ -142,3 +142,29 @@ def test_prefill_layer_zipf_2048():
     err = normwise_err(out.cpu().numpy()[toks], ref)
     print(f"glm prefill T=2048: normwise error {err:.2e}")
     assert err <= TOL_TC, err
+
+
+def test_prefill_layer_repeatable_all_tokens():
+    """Every token of the 2048-token layer agrees across repeated calls on the same input.
+
+    The down projection combines with float atomics, so runs may differ in the last bits of a
+    sum (~1e-7 relative); a pipeline race would change whole rows of a tile by orders more."""
+    L = layer("glm_prefill")
+    wl = L.wl
+    T = 2048
+    cfg = q.config_for(wl)
+    x = synth.make_activations(wl, T, device="cuda", step=1)
+    ws = torch.empty(q.coli_moe_workspace_size(cfg, T), dtype=torch.uint8, device="cuda")
+    q.coli_moe_clear_error(ws)
+    outs, idss = [], []
+    for _ in range(3):
+        out = torch.empty(T, wl.hidden, dtype=torch.float32, device="cuda")
+        ids = torch.empty(T, wl.top_k, dtype=torch.int32, device="cuda")
+        w = torch.empty(T, wl.top_k, dtype=torch.float32, device="cuda")
+        q.coli_moe_layer(cfg, L.weights(), x, T, out, ids, w, ws)
+        assert q.coli_moe_error_word(ws) == 0
+        outs.append(out.cpu().numpy())
+        idss.append(ids.cpu().numpy())
+    for r in (1, 2):
+        np.testing.assert_array_equal(idss[r], idss[0])
+        assert normwise_err(outs[r], outs[0]) <= 1e-5
