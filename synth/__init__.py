@@ -80,6 +80,9 @@ WORKLOADS: Dict[str, Workload] = {
                       act="bf16", tokens=(1, 32), bias_std=0.0, seed=1),
     "glm_decode": Workload("glm_decode", fmt=4, tokens=(1, 4), seed=2, **_GLM),
     "glm_prefill": Workload("glm_prefill", fmt=4, tokens=(2048,), seed=2, zipf_s=1.1, **_GLM),
+    # GLM-5.2 expert shapes with 32 experts and uniform routing: a 0.6 GB layer on which the
+    # tensor-core kernels run with mostly full token chunks (small enough for ncu captures)
+    "glm_e32": Workload("glm_e32", fmt=4, tokens=(1024,), seed=2, **dict(_GLM, n_experts=32)),
     "glm_int8": Workload("glm_int8", fmt=8, tokens=(64,), seed=4, n_layers=4, **_GLM),
     "glm_int2": Workload("glm_int2", fmt=2, tokens=(64,), seed=4, n_layers=4, **_GLM),
 }
