@@ -258,6 +258,31 @@ def test_layer_alternate_containers_sampled(name):
     assert err <= TOL_GEMV, err
 
 
+def test_decode_shapes_take_fused_kernel():
+    """Decode shapes run as one fused launch (a fall back to the five-kernel path would give the
+    same outputs, only slower, so the launch count is checked here)."""
+    for name, Ts in (("glm_decode", (1, 2, 3, 4)), ("olmoe", (1, 2, 4)), ("glm_int2", (1, 4))):
+        cfg = q.config_for(synth.WORKLOADS[name])
+        for T in Ts:
+            assert q.coli_moe_layer_kernels(cfg, T) == 1, (name, T)
+
+
+@pytest.mark.parametrize("name", ["glm_int8", "glm_int2"])
+@pytest.mark.parametrize("T", [1, 2])
+def test_layer_alternate_containers_decode(name, T):
+    """One and two tokens on int8 and int2 codes, every token (int2 takes the fused decode
+    kernel; int8's down rows per CTA exceed its phase-2 row split, so it takes the GEMV path)."""
+    L = layer_for(name)
+    assert q.coli_moe_layer_kernels(q.config_for(L.wl), T) == (1 if name == "glm_int2" else 5)
+    x = synth.make_activations(L.wl, T, device="cuda", step=20 + T)
+    out, ids, w = run_layer(L, x, T)
+    ref, ids_ref, w_ref, _ = oracle_layer_tokens(L, x.cpu(), range(T))
+    np.testing.assert_array_equal(ids, ids_ref)
+    np.testing.assert_array_equal(w, w_ref)
+    err = normwise_err(out, ref)
+    assert err <= TOL_GEMV, err
+
+
 @pytest.mark.parametrize("name,T", [("tiny", 8), ("glm_decode", 4), ("olmoe", 32)])
 def test_batch_union_equals_per_token_bitwise(name, T):
     """The batch reads each unique expert once, yet every token's output is bit-identical to
