@@ -159,6 +159,19 @@ coli_status coli_moe_layer(const coli_moe_config *cfg, const coli_moe_weights *w
                            const void *x, int T, float *out, int32_t *topk_ids_out,
                            float *topk_w_out, void *ws, size_t ws_bytes, void *stream);
 
+/* Residual update between chained layers (JustVugg/colibri README, "Never wait for the disk
+ * twice": the GPU-resident pipeline keeps the residual stream on the device across layers).
+ * x_next[t][h] = x[t][h] + out[t][h] for t < T, h < hidden: one float32 addition (round to
+ * nearest even); with bf16 activations (cfg->act) x and x_next are bf16 and the sum is rounded
+ * to bf16 (round to nearest even, NaN kept), with float32 activations they are float32.
+ *   x, x_next  [T][hidden] device, row-major, the activation type of cfg; x_next may be x (in
+ *              place) but must not overlap out.
+ *   out        [T][hidden] float32 device, a layer's output.
+ * Pointers 16-byte aligned (COLI_ERR_ALIGN otherwise); T < 0 is COLI_ERR_SHAPE, T = 0 a no-op.
+ * Asynchronous on `stream`; allocates nothing. */
+coli_status coli_moe_residual(const coli_moe_config *cfg, const void *x, const float *out, int T,
+                              void *x_next, void *stream);
+
 /* Size of the static scratch array behind coli_moe_layer_noalloc (8 MiB per GPU). */
 #define COLI_MOE_STATIC_SCRATCH_BYTES (8u << 20)
 

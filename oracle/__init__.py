@@ -44,6 +44,8 @@ def _load():
     lib.oracle_ffn_union.argtypes = [C.POINTER(OracleCfg), P, P, P, C.c_int, P, P, P]
     lib.oracle_layer.argtypes = [C.POINTER(OracleCfg), P, P, P, P, P, C.c_int, P, P, P, P,
                                  C.c_int]
+    lib.oracle_residual.argtypes = [C.POINTER(OracleCfg), P, P, C.c_size_t, P]
+    lib.oracle_residual.restype = None
     return lib
 
 
@@ -202,3 +204,15 @@ def layer(cfg: OracleCfg, Wr, bias, recs: Records, x, T: int, n_threads: int = 1
                           n_threads) != 0:
         raise ValueError("oracle layer failed")
     return out, ids, w, lg
+
+
+def residual(cfg: OracleCfg, x, out) -> np.ndarray:
+    """x + out as the next layer's input: float32 sum, rounded to bf16 for bf16 activations.
+    Returns bf16 bit patterns (uint16) for bf16 activations, float32 otherwise."""
+    x = _x(cfg, x)
+    out = _np(out, np.float32)
+    if out.shape != x.shape:
+        raise ValueError("x and out shapes differ")
+    nxt = np.empty_like(x)
+    lib().oracle_residual(C.byref(cfg), _ptr(x), _ptr(out), x.size, _ptr(nxt))
+    return nxt

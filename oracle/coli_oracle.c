@@ -371,6 +371,36 @@ int oracle_ffn_union(const oracle_cfg *cfg, const uint8_t *const *experts,
     return rc;
 }
 
+/* ---------------------------------------------------------------- residual ---------------- */
+
+/* float -> bf16 bits, round to nearest even on the dropped low half. */
+static uint16_t bf16_round_even(float v) {
+    uint32_t u;
+    memcpy(&u, &v, sizeof u);
+    if ((u & 0x7fffffffu) > 0x7f800000u) return (uint16_t)((u >> 16) | 0x40u); /* NaN */
+    uint32_t keep = u >> 16, dropped = u & 0xffffu;
+    if (dropped > 0x8000u || (dropped == 0x8000u && (keep & 1u))) keep += 1u;
+    return (uint16_t)keep;
+}
+
+void oracle_residual(const oracle_cfg *cfg, const void *x, const float *out, size_t n, void *x_next) {
+    if (cfg->act == 1) {
+        const uint16_t *xb = (const uint16_t *)x;
+        uint16_t *nb = (uint16_t *)x_next;
+        for (size_t i = 0; i < n; i++) {
+            uint32_t u = (uint32_t)xb[i] << 16;
+            float xv;
+            memcpy(&xv, &u, sizeof xv);
+            float s = xv + out[i];
+            nb[i] = bf16_round_even(s);
+        }
+    } else {
+        const float *xf = (const float *)x;
+        float *nf = (float *)x_next;
+        for (size_t i = 0; i < n; i++) nf[i] = xf[i] + out[i];
+    }
+}
+
 /* ---------------------------------------------------------------- whole layer ------------- */
 
 int oracle_layer(const oracle_cfg *cfg, const float *Wr, const float *bias,

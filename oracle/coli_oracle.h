@@ -106,6 +106,13 @@ int oracle_layer(const oracle_cfg *cfg, const float *Wr, const float *bias,
                  const uint8_t *const *experts, const uint8_t *shared, const void *x, int T,
                  double *out, int32_t *ids, float *w, float *logits, int n_threads);
 
+/* Residual update between chained layers (JustVugg/colibri README, "Never wait for the disk
+ * twice": the residual stream stays on the device from layer to layer).  For n elements,
+ * x_next = x + out as one IEEE single addition; with bf16 activations (cfg->act = 1) x and
+ * x_next are bf16 bit patterns and the sum is rounded to bf16, round to nearest even (a NaN
+ * stays a quiet NaN); with float32 activations both are float32. */
+void oracle_residual(const oracle_cfg *cfg, const void *x, const float *out, size_t n, void *x_next);
+
 #ifdef __cplusplus
 }
 #endif

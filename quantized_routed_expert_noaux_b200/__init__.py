@@ -79,11 +79,13 @@ def _load():
     L.coli_moe_layer.argtypes = [cfgp, wp, P, I, P, P, P, P, S, P]
     L.coli_moe_layer_noalloc.argtypes = [cfgp, wp, P, I, P, P, P, P]
     L.coli_moe_layer_kernels.argtypes = [cfgp, I, C.POINTER(I)]
+    L.coli_moe_residual.argtypes = [cfgp, P, P, I, P, P]
     L.coli_moe_layer_kernels.restype = I
     L.coli_moe_layer_noalloc.restype = I
     for name in ("coli_moe_record_bytes", "coli_moe_check_config", "coli_moe_workspace_size",
                  "coli_moe_clear_error", "coli_moe_error_word", "coli_moe_gate",
-                 "coli_moe_route", "coli_moe_group", "coli_moe_ffn", "coli_moe_layer"):
+                 "coli_moe_route", "coli_moe_group", "coli_moe_ffn", "coli_moe_layer",
+                 "coli_moe_residual"):
         getattr(L, name).restype = I
     return L
 
@@ -185,6 +187,12 @@ def coli_moe_layer(cfg, weights: MoEWeights, x, T, out, topk_ids_out, topk_w_out
     _check("coli_moe_layer", lib.coli_moe_layer(
         C.byref(cfg), C.byref(weights), _p(x), T, _p(out), _p(topk_ids_out), _p(topk_w_out),
         _p(ws), _nbytes(ws), _stream(stream)))
+
+
+def coli_moe_residual(cfg, x, out, T, x_next, stream=None) -> None:
+    """x_next = x + out between chained layers (float32 sum; bf16 activations rounded to bf16)."""
+    _check("coli_moe_residual", lib.coli_moe_residual(
+        C.byref(cfg), _p(x), _p(out), T, _p(x_next), _stream(stream)))
 
 
 # Size of the static scratch array behind coli_moe_layer_noalloc (COLI_MOE_STATIC_SCRATCH_BYTES).

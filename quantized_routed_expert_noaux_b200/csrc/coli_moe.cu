@@ -7,6 +7,7 @@
 
 #include "coli_moe.h"
 #include "internal.h"
+#include "residual.h"
 
 namespace coli {
 
@@ -192,6 +193,17 @@ coli_status coli_moe_gate(const coli_moe_config *c, const float *router_w, const
     if (!router_w || !x || !logits) return COLI_ERR_INVALID_ARG;
     if (!aligned(router_w, 16) || !aligned(x, 16) || !aligned(logits, 4)) return COLI_ERR_ALIGN;
     return from_cuda(launch_gate(*c, router_w, x, T, logits, static_cast<cudaStream_t>(stream)));
+}
+
+coli_status coli_moe_residual(const coli_moe_config *c, const void *x, const float *out, int T,
+                              void *x_next, void *stream) {
+    coli_status s = coli_moe_check_config(c);
+    if (s != COLI_OK) return s;
+    if (T < 0) return COLI_ERR_SHAPE;
+    if (T == 0) return COLI_OK;
+    if (!x || !out || !x_next) return COLI_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(out, 16) || !aligned(x_next, 16)) return COLI_ERR_ALIGN;
+    return from_cuda(launch_residual(*c, x, out, T, x_next, static_cast<cudaStream_t>(stream)));
 }
 
 coli_status coli_moe_route(const coli_moe_config *c, const float *logits, const float *bias, int T,

@@ -91,3 +91,18 @@ def test_host_validation_before_launch():
     rc = q.lib.coli_moe_layer(ctypes.byref(cfg), ctypes.byref(w), 4096, 2, 8192, None, None,
                               None, 0, None)
     assert rc == 2
+
+
+def test_residual_host_validation():
+    cfg = q.config_for(synth.WORKLOADS["olmoe"])
+    q.coli_moe_residual(cfg, None, None, 0, None, stream=0)  # T = 0: no-op
+    with pytest.raises(q.ColiError) as ei:
+        q.coli_moe_residual(cfg, None, None, -1, None, stream=0)
+    assert ei.value.status == 2
+    with pytest.raises(q.ColiError) as ei:
+        q.coli_moe_residual(cfg, None, 256, 2, 512, stream=0)
+    assert ei.value.status == 1
+    with pytest.raises(q.ColiError) as ei:
+        q.coli_moe_residual(cfg, 264, 256, 2, 512, stream=0)  # x not 16-byte aligned
+    assert ei.value.status == 3
+

@@ -10,7 +10,9 @@
   float64 matmuls over the generator's codes x scales;
 * gate: numpy float64 matmul rounded to float32;
 * layer: batch-union equals per-token bit for bit, and the layer equals the sum of its parts
-  computed by numpy.
+  computed by numpy;
+* residual update: hand-worked ties of the bf16 rounding, and numpy's float32 sum rounded by
+  torch's float32-to-bf16 conversion (round to nearest even).
 """
 import itertools
 import json
@@ -358,3 +360,51 @@ def test_layer_threads_do_not_change_result():
     a = oracle.layer(cfg, Wr, bias, R, x, T, n_threads=1)[0]
     b = oracle.layer(cfg, Wr, bias, R, x, T, n_threads=4)[0]
     np.testing.assert_array_equal(a, b)
+
+
+# ------------------------------------------------------------------------ residual update --
+
+def _bf16_bits(vals):
+    return torch.tensor(vals, dtype=torch.float32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def test_residual_hand_worked_ties():
+    """bf16 keeps 8 significant bits: at 1.0 its spacing is 2^-7, so 1 + 2^-8 is a tie that
+    rounds to the even 1.0 (0x3f80) and 1 + 3*2^-8 one that rounds to 1 + 2^-6 (0x3f82);
+    1 + 2^-8 + 2^-20 lies above the tie and rounds up to 0x3f81."""
+    cfg = oracle.make_cfg(synth.WORKLOADS["olmoe"])
+    x = _bf16_bits([1.0, 1.0, 1.0, -1.0, 0.0])
+    out = np.array([2.0 ** -8, 3 * 2.0 ** -8, 2.0 ** -8 + 2.0 ** -20, -(2.0 ** -8), -0.0], np.float32)
+    got = oracle.residual(cfg, x, out)
+    assert [int(v) for v in got] == [0x3F80, 0x3F82, 0x3F81, 0xBF80, 0x0000]
+
+
+def test_residual_against_torch_rounding():
+    """numpy's IEEE float32 sum, rounded by torch's float32 -> bf16 conversion, on random values,
+    exact ties, the overflow edge and NaN."""
+    cfg = oracle.make_cfg(synth.WORKLOADS["olmoe"])
+    rng = np.random.default_rng(5)
+    n = 50000
+    x = _bf16_bits(rng.normal(0, 1, n).astype(np.float32))
+    out = (rng.normal(0, 1, n) * 10.0 ** rng.integers(-6, 3, n)).astype(np.float32)
+    # exact ties: x = 0 and out with its low 16 bits 0x8000 (odd and even kept halves)
+    ties = (rng.integers(0x3000, 0x4800, 2000).astype(np.uint32) << 16) | 0x8000
+    x = np.concatenate([x, np.zeros(2000, np.uint16), _bf16_bits([3.3895313892515355e38, 1.0])])
+    out = np.concatenate([out, ties.view(np.float32), np.array([1.0e36, np.nan], np.float32)])
+    got = oracle.residual(cfg, x, out)
+    xs = (x.astype(np.uint32) << 16).view(np.float32)
+    s = (xs + out).astype(np.float32)
+    want = torch.from_numpy(s).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    nan = np.isnan(s)
+    np.testing.assert_array_equal(got[~nan], want[~nan])
+    assert ((got[nan] & 0x7F80) == 0x7F80).all() and ((got[nan] & 0x7F) != 0).all()
+    assert got[-2] == 0x7F80  # the largest bf16 plus 1e36 (past half a bf16 step there) rounds to +inf
+
+
+def test_residual_f32_is_ieee_sum():
+    cfg = oracle.make_cfg(synth.WORKLOADS["tiny"])
+    rng = np.random.default_rng(6)
+    x = rng.normal(0, 1, 4096).astype(np.float32)
+    out = rng.normal(0, 1e-3, 4096).astype(np.float32)
+    np.testing.assert_array_equal(oracle.residual(cfg, x, out), x + out)
+
