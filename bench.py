@@ -268,15 +268,18 @@ def gpu_arm(args, rank, world, dist):
             traffic = d.get("traffic_bytes_per_launch")
 
     n_kern = q.coli_moe_layer_kernels(cfg, T)
-    if n_kern == 7:
-        # tensor-core path: int8 MMAs on two 8-bit activation slices, i.e. two int8 operations per
-        # algorithmic multiply-add -- the bf16 tensor rate; ~1 ms launches back to back -> sustained
-        ffn_flops = (T * wl.top_k + T * wl.n_shared) * 6.0 * wl.hidden * wl.inter
+    # tensor-core path: int8 MMAs on two 8-bit activation slices, i.e. two int8 operations per
+    # algorithmic multiply-add -- the bf16 tensor rate; ~1 ms launches back to back -> sustained.
+    # Its bound is whichever of the flops and the bytes takes longer at the measured peaks (small
+    # batches on that path are bound by HBM like decode).
+    ffn_flops = (T * wl.top_k + T * wl.n_shared) * 6.0 * wl.hidden * wl.inter
+    peak_t = bf16s if bf16s else bf16
+    tc_kernel = "expert FFN (x quantisation, gate/up int8 GEMM, h quantisation, down int8 GEMM + combine)"
+    if n_kern == 7 and ffn_flops / (peak_t * 1e12) > ffn_bytes / (hbm * 1e9):
         tf_s = ffn_flops / (ffn_ms / 1e3) / 1e12
-        peak_t = bf16s if bf16s else bf16
         roofline = {
             "bound": "tensor",
-            "kernel": "expert FFN (x quantisation, gate/up int8 GEMM, h quantisation, down int8 GEMM + combine)",
+            "kernel": tc_kernel,
             "achieved": round(tf_s, 1),
             "peak": peak_t,
             "unit": "TFLOP/s",
@@ -290,8 +293,8 @@ def gpu_arm(args, rank, world, dist):
     else:
         roofline = {
             "bound": "hbm",
-            "kernel": ("fused decode layer kernel (FFN part)" if n_kern == 1
-                       else "expert FFN (gate/up GEMV + down GEMV with fused combine)"),
+            "kernel": ("fused decode layer kernel (FFN part)" if n_kern == 1 else
+                       tc_kernel if n_kern == 7 else "expert FFN (gate/up GEMV + down GEMV with fused combine)"),
             "achieved": round(achieved, 1),
             "peak": hbm,
             "unit": "GB/s",

@@ -31,7 +31,7 @@ int row_bytes(int n, int fmt) { return n * fmt / 8; }
 
 }  // namespace
 
-// Batches with many tokens per expert take the tensor-core grouped GEMM when its shape rules hold.
+// Batches beyond decode size take the tensor-core grouped GEMM when its shape rules hold.
 static bool use_tc(const coli_moe_config *c, int T) { return T > TC_MIN_TOKENS && tc_shape_ok(*c); }
 
 int device_sm_count() {

@@ -8,7 +8,7 @@
 //     chunk of a weight row, so the matching slice of the activation vector is converted once
 //     per (expert, token) and reused across R rows held in flight;
 //   * gate/up kernel: passes of P*R rows of one expert (routed experts in unique-id order, then
-//     the shared expert), split contiguously over a fixed grid; it writes h = SiLU(g) * u;
+//     the shared expert), dealt round-robin over a fixed grid; it writes h = SiLU(g) * u;
 //   * down kernel: each CTA owns a contiguous block of output rows and walks every unique
 //     expert (then the shared one) for them, so out[t, j] is summed in one place, in a fixed
 //     order, with no atomics.  The combine weight and the row scale are applied there.
@@ -199,10 +199,9 @@ __global__ void __launch_bounds__(GU_THREADS) gateup_kernel(FfnParams p, int L, 
     const int rpp = P * R;
     const int ppe = (p.I + rpp - 1) / rpp;
     const long total = static_cast<long>(nwe) * ppe;
-    const long beg = total * blockIdx.x / gridDim.x;
-    const long end = total * (blockIdx.x + 1) / gridDim.x;
-
-    for (long pi = beg; pi < end; ++pi) {
+    // passes dealt round-robin over the grid: a pass costs in proportion to its expert's token
+    // count, and the shared expert (all T tokens) would otherwise load a few CTAs only
+    for (long pi = blockIdx.x; pi < total; pi += gridDim.x) {
         const int we = static_cast<int>(pi / ppe);
         const int i0 = static_cast<int>(pi % ppe) * rpp;
         const ExpertRef ex = expert_ref(p, we, U);

@@ -19,6 +19,11 @@ TOL_GEMV = 1e-4
 TOL_TC = 3e-4
 
 
+def tol_for(q, cfg, T) -> float:
+    """FFN tolerance of the path coli_moe_layer / coli_moe_ffn take for T tokens."""
+    return TOL_TC if q.coli_moe_layer_kernels(cfg, T) == 7 else TOL_GEMV
+
+
 def normwise_err(got, ref) -> float:
     got = np.asarray(got, np.float64)
     ref = np.asarray(ref, np.float64)

@@ -3,7 +3,7 @@ layers): x_{l+1} = bf16(x_l + out_l) on the device between the layers.
 
 The residual update is compared bit for bit with the oracle.  Each layer is compared with the
 oracle fed the device's own input (teacher forcing): routing bit-exact on sampled tokens, the
-output within the float32-accumulate tolerance.  The oracle also runs the chain on its own from
+output within the tolerance of the path it takes.  The oracle also runs the chain on its own from
 the first input for two tokens; that end-to-end difference is printed, not gated.
 """
 import numpy as np
@@ -12,7 +12,7 @@ import torch
 
 import oracle
 import synth
-from tests._common import TOL_GEMV, Layer, normwise_err, oracle_layer_tokens
+from tests._common import Layer, normwise_err, oracle_layer_tokens, tol_for
 
 pytestmark = pytest.mark.gpu
 
@@ -89,7 +89,7 @@ def test_chained_layers_teacher_forced(name):
         np.testing.assert_array_equal(ids.cpu().numpy()[toks], ids_ref)
         np.testing.assert_array_equal(w.cpu().numpy()[toks], w_ref)
         err = normwise_err(out.cpu().numpy()[toks], ref)
-        assert err <= TOL_GEMV, (layer, err)
+        assert err <= tol_for(q, cfg, T), (layer, err)
         x_next = torch.empty_like(x)
         q.coli_moe_residual(cfg, x, out, T, x_next)
         torch.cuda.synchronize()

@@ -1,4 +1,4 @@
-"""GPU parity of the tensor-core grouped-GEMM path (batches above 64 tokens, int4 weights).
+"""GPU parity of the tensor-core grouped-GEMM path (batches above 4 tokens, int4 weights).
 
 x and h enter the int8 MMAs as 16-bit fixed point per row, so outputs are compared with the
 tensor-core tolerance (TOL_TC, normwise per token); routing and grouping stay bit-exact.  The
@@ -57,11 +57,12 @@ def _routing(L, ocfg, x, T, routing):
 
 
 # (workload, tokens, routing): chunks of 1..96 tokens with ragged tails; one expert with 128 and
-# with 160 tokens (two chunks each); just above the 64-token threshold; f32 activations and
-# four gate/up m-blocks (tiny_wide); no shared expert (olmoe).
+# with 160 tokens (two chunks each); one token above the fused decode limit (5: chunks of one
+# token); f32 activations and four gate/up m-blocks (tiny_wide); no shared expert (olmoe).
 CASES = [("glm_decode", 96, "oracle"), ("glm_decode", 300, "oracle"), ("glm_decode", 160, "one_expert"),
-         ("glm_decode", 128, "one_expert"), ("glm_decode", 65, "oracle"), ("olmoe", 200, "oracle"),
-         ("olmoe", 97, "one_expert"), ("tiny_wide", 100, "oracle")]
+         ("glm_decode", 128, "one_expert"), ("glm_decode", 65, "oracle"), ("glm_decode", 5, "oracle"),
+         ("olmoe", 200, "oracle"), ("olmoe", 97, "one_expert"), ("olmoe", 8, "oracle"),
+         ("tiny_wide", 100, "oracle")]
 
 
 @pytest.mark.parametrize("name,T,routing", CASES)
