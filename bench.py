@@ -75,6 +75,22 @@ def alg_flops(wl, T):
     return (T * wl.top_k + T * wl.n_shared) * 6 * wl.hidden * wl.inter + T * wl.n_experts * wl.hidden * 2
 
 
+def max_over_ranks(value, dist, device):
+    """The largest per-rank value (a timed region's device time) over all ranks; the value
+    itself on one rank."""
+    if dist is None:
+        return value
+    t = torch.tensor([value], device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world, steps, tokens, ms_max):
+    """Tokens of all ranks (each runs `steps` steps of `tokens` tokens) per second of the
+    slowest rank's time."""
+    return world * steps * tokens / (ms_max / 1e3)
+
+
 def src_hash(paths):
     h = hashlib.sha256()
     for p in paths:
@@ -193,11 +209,7 @@ def gpu_arm(args, rank, world, dist):
     err = q.coli_moe_error_word(ws)
     if err:
         raise RuntimeError(f"device error word {err:#x} after the timed region")
-    ms_max = ms
-    if dist is not None:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, dist, dev)
 
     # algorithmic bytes of the timed steps (unique experts per step from the routing written)
     ids_np = ids_all.cpu().numpy()
@@ -249,14 +261,10 @@ def gpu_arm(args, rank, world, dist):
     f1.record(st)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = f0.elapsed_time(f1)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1), dist, dev)
 
     hbm, bf16, bf16s, peak_kind = peaks()
-    tok_s = world * K * T / (ms_max / 1e3)
+    tok_s = whole_job_rate(world, K, T, ms_max)
     achieved = ffn_bytes / (ffn_ms / 1e3) / 1e9
     traffic = None
     tf = os.path.join(PROFILES, f"{args.workload}_t{T}_traffic.json")
@@ -330,7 +338,7 @@ def gpu_arm(args, rank, world, dist):
         "layer_frac_of_hbm": round(bytes_steps / (ms_max / 1e3) / 1e9 / hbm, 4),
         "unique_experts_mean": round(float(U.mean()), 2),
         "roofline": roofline,
-        "e2e": {"value": round(world * K2 * T / (e2e_ms / 1e3), 2), "unit": "tokens/s",
+        "e2e": {"value": round(whole_job_rate(world, K2, T, e2e_ms), 2), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(xs[0].numel() * xs[0].element_size()),
                 "d2h_bytes_per_step": int(out.numel() * 4)},
         "gpu_launches": n_kern * K,
