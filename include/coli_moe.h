@@ -48,7 +48,7 @@ typedef enum {
     COLI_ERR_INVALID_ARG = 1,  /* NULL pointer, negative size, bad enum value */
     COLI_ERR_SHAPE = 2,        /* sizes inconsistent with each other or with the formats */
     COLI_ERR_ALIGN = 3,        /* a pointer or stride misses its required alignment */
-    COLI_ERR_UNSUPPORTED = 4,  /* a valid configuration this build does not implement */
+    COLI_ERR_UNSUPPORTED = 4,  /* a valid configuration that this library does not implement */
     COLI_ERR_CUDA = 5,         /* a CUDA runtime call failed (launch, attribute, copy) */
     COLI_ERR_DEVICE = 6,       /* the device error word was set by a kernel */
     COLI_ERR_WORKSPACE = 7     /* workspace NULL, misaligned or smaller than required */
