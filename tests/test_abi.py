@@ -106,3 +106,21 @@ def test_residual_host_validation():
         q.coli_moe_residual(cfg, 264, 256, 2, 512, stream=0)  # x not 16-byte aligned
     assert ei.value.status == 3
 
+
+
+def test_dispatch_rule_on_the_host():
+    """Batches above 4 tokens take the tensor-core path (7 launches) for int4 records whose
+    hidden and inter sizes are multiples of 128; int8 / int2 records take the GEMV path (5);
+    an empty batch launches nothing.  (Up to 4 tokens the fused decode kernel needs the device's
+    shared-memory size, so that choice is checked by the GPU tests.)"""
+    for name in ("tiny", "olmoe", "glm_decode", "glm_prefill"):
+        cfg = q.config_for(synth.WORKLOADS[name])
+        assert q.coli_moe_layer_kernels(cfg, 0) == 0
+        for T in (5, 8, 64, 65, 2048):
+            assert q.coli_moe_layer_kernels(cfg, T) == 7, (name, T)
+    for name in ("glm_int8", "glm_int2"):
+        cfg = q.config_for(synth.WORKLOADS[name])
+        for T in (5, 64, 256):
+            assert q.coli_moe_layer_kernels(cfg, T) == 5, (name, T)
+    odd = q.config_for(synth.WORKLOADS["tiny"].replace(inter=64, shared_inter=64))
+    assert q.coli_moe_layer_kernels(odd, 32) == 5  # inter not a multiple of 128
