@@ -1,12 +1,13 @@
 /*
  * coli_moe.h -- C ABI of the routed-expert MoE layer on NVIDIA B200 (sm_100a).
  *
- * The layer (colibri-strix README, "What's implemented"): a DeepSeek-V3-style sigmoid router
- * with the noaux_tc selection bias and routed_scaling_factor, batch-union grouping ("each unique
- * expert of the batch is read once and applied to every position that routes to it"), SwiGLU
- * experts stored as packed int4 (also int8 / packed int2) with per-row scales and dequantised on
- * use, a shared expert, and the weighted combine.  The JustVugg/colibri README ("Never wait for
- * the disk twice") adds that an expert's three matrices are stored adjacent.
+ * The layer (colibri-strix README, "What's implemented"): a sigmoid router in the DeepSeek-V3
+ * manner, whose noaux_tc bias steers the selection and whose weights are renormalised and scaled
+ * by routed_scaling_factor; batch-union grouping, in which every expert that some token of the
+ * batch selects is fetched one time and serves all of those tokens; SwiGLU experts stored as
+ * packed int4 (also int8 / packed int2) with per-row scales, dequantised on use; a shared
+ * expert; and the weighted combine.  The JustVugg/colibri README ("Never wait for the disk
+ * twice") keeps an expert's gate, up and down matrices together in one record.
  *
  * Conventions shared by every call
  *   - All tensor pointers are DEVICE pointers owned by the caller.  The library allocates no
@@ -121,8 +122,8 @@ coli_status coli_moe_error_word(void *ws, void *stream, int *code);
 coli_status coli_moe_gate(const coli_moe_config *cfg, const float *router_w, const void *x,
                           int T, float *logits, void *stream);
 
-/* a2, noaux_tc routing (colibri-strix README, "What's implemented": DeepSeek-V3-style sigmoid
- * router (noaux_tc, routed_scaling_factor)).  Per token, in double: s = 1/(1+exp(-logit)),
+/* a2, noaux_tc routing (colibri-strix README, "What's implemented": the DeepSeek-V3 sigmoid
+ * router, its noaux_tc bias and routed_scaling_factor).  Per token, in double: s = 1/(1+exp(-logit)),
  * c = s + bias; if G > 1 each group scores the sum of its two largest c and the TG best groups
  * are kept (ties: lower group); the K largest c among kept experts are selected (ties: lower
  * id), written in descending c order; topk_w[k] = float32(s_k / sum_k s_k * routed_scaling).
@@ -141,7 +142,8 @@ coli_status coli_moe_group(const coli_moe_config *cfg, const int32_t *topk_ids, 
                            void *stream);
 
 /* a4..a7 for a given routing (JustVugg/colibri README, "Never wait for the disk twice":
- * batched positions read each unique expert once; colibri-strix README, "What's implemented":
+ * the experts a batch needs are fetched once for all of its positions; colibri-strix README,
+ * "What's implemented":
  * dequant-on-use, shared expert).  For every unique expert e and every slot routed to it:
  * y = sd .* (Qd (SiLU(sg .* (Qg x)) .* (su .* (Qu x)))) with the codes Q dequantised in
  * registers; out[t] = sum over t's experts of topk_w * y + y_shared (weight 1).  The grouping

@@ -35,8 +35,8 @@ int oracle_record_bytes(int hidden, int inter, int fmt, size_t *bytes)
     return 0;
 }
 
-/* Decode a packed row (colibri-strix README, "What's implemented": packed int4 / packed int2
- * containers, bit-identical to the int8 container).  Two's complement in 4 or 2 bits. */
+/* Decode a packed row (colibri-strix README, "What's implemented": packed int4 and int2 rows
+ * decode to exactly the codes of the int8 container).  Two's complement in 4 or 2 bits. */
 int oracle_unpack_row(const uint8_t *row, int n, int fmt, int8_t *q)
 {
     size_t nb;
@@ -137,7 +137,7 @@ static int beats(double va, int ia, double vb, int ib)
     return va > vb || (va == vb && ia < ib);
 }
 
-/* DeepSeek-V3-style sigmoid router with the noaux_tc selection bias and routed_scaling_factor
+/* The sigmoid router of DeepSeek-V3 with its noaux_tc selection bias and routed_scaling_factor
  * (colibri-strix README, "What's implemented").  Readings where the pages are silent: the
  * bias steers selection only; a group scores the sum of its two largest biased scores; only
  * experts of the kept groups can be chosen; ties go to the lower index; slots are ordered by
@@ -223,9 +223,9 @@ int oracle_route(const oracle_cfg *cfg, const float *logits, const float *bias, 
 
 /* ---------------------------------------------------------------- a3 group ---------------- */
 
-/* Batch-union grouping (colibri-strix README, "What's implemented": each unique expert of the
- * batch is read once and applied to every position routed to it): a stable counting sort of
- * the slots by expert id. */
+/* Batch-union grouping (colibri-strix README, "What's implemented": an expert chosen anywhere
+ * in the batch is fetched once and used for all the positions that chose it): a stable
+ * counting sort of the slots by expert id. */
 int oracle_group(int T, int K, int E, const int32_t *ids, int32_t *counts, int32_t *offsets,
                  int32_t *perm, int32_t *unique, int32_t *n_unique)
 {

@@ -11,8 +11,8 @@
  * rule of the JustVugg/colibri README, section "File: c/tools/README.md" (the reference output
  * is computed from the dequantised weights so that an engine reproduces it exactly).
  *
- * What the layer computes (colibri-strix README, "What's implemented": DeepSeek-V3-style
- * sigmoid router with noaux_tc and routed_scaling_factor, a shared expert, batch-union MoE,
+ * What the layer computes (colibri-strix README, "What's implemented": a DeepSeek-V3 sigmoid
+ * router (noaux_tc bias, routed_scaling_factor), a shared expert, batch-union MoE,
  * int8 / packed int4 / packed int2 containers with per-row scales and dequant-on-use):
  *
  *   a1 gate     logits[t,e] = (float) sum_h x[t,h] * Wr[e,h]            (double sum, h order)

@@ -1,7 +1,7 @@
 // router.cu -- a1 gate, a2 noaux_tc routing and a3 batch-union grouping on sm_100a.
 //
-// The router of the colibri-strix README ("What's implemented": DeepSeek-V3-style sigmoid router
-// with noaux_tc and routed_scaling_factor) and the batch-union step of the same section.  The
+// The router of the colibri-strix README ("What's implemented": a DeepSeek-V3 sigmoid router,
+// noaux_tc bias, routed_scaling_factor) and the batch-union step of the same section.  The
 // gate sums exact double products in double and rounds once to float32; selection compares in
 // double, so the float32 logits and the chosen experts do not depend on summation order beyond
 // double rounding.
