@@ -17,7 +17,7 @@ __all__ = [
     "coli_moe_status_str", "coli_moe_last_cuda_error", "coli_moe_record_bytes", "coli_moe_check_config",
     "coli_moe_workspace_size", "coli_moe_clear_error", "coli_moe_error_word",
     "coli_moe_gate", "coli_moe_route", "coli_moe_group", "coli_moe_ffn", "coli_moe_layer",
-    "coli_moe_layer_noalloc", "STATIC_SCRATCH_BYTES", "coli_moe_layer_kernels",
+    "coli_moe_layer_noalloc", "STATIC_SCRATCH_BYTES", "coli_moe_layer_kernels", "coli_moe_residual",
     "config_for", "weights_for",
     "COLI_W_INT2", "COLI_W_INT4", "COLI_W_INT8", "COLI_ACT_F32", "COLI_ACT_BF16",
 ]

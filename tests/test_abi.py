@@ -31,6 +31,7 @@ def test_every_declared_symbol_is_exported():
 def test_binding_names_match_header():
     for s in declared_symbols():
         assert hasattr(q, s), f"binding lacks {s}"
+        assert s in q.__all__, f"{s} missing from __all__"
 
 
 def test_status_strings():
