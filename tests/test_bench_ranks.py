@@ -2,6 +2,7 @@
 device time is the max over ranks, the rate counts every rank's tokens, and under a multi-rank
 launch the reference arm runs on rank 0 alone (the other ranks exit at once, printing nothing)."""
 import os
+import socket
 import subprocess
 import sys
 
@@ -29,7 +30,9 @@ def _rank_main(rank, world, port, times, out_q):
 
 def test_max_over_ranks_and_rate_gloo():
     world, times = 2, [12.5, 20.0]
-    port = 29600 + os.getpid() % 1000
+    with socket.socket() as sk:  # a free local port for the rendezvous
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     procs = [ctx.Process(target=_rank_main, args=(r, world, port, times, q)) for r in range(world)]
