@@ -44,6 +44,8 @@ def parse():
     ap.add_argument("--tokens", type=int, default=0, help="tokens per step (default: workload's first)")
     ap.add_argument("--layers", type=int, default=0, help="resident layers rotated (default 4)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="default workload only: skip the 2048-token prefill measurement")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--profile", action="store_true",
                     help="only run warmup+steps layer calls (for ncu captures); prints no JSON")
@@ -143,25 +145,45 @@ class Clocks:
 
 # ------------------------------------------------------------------------- GPU arm ----------
 
-def gpu_arm(args, rank, world, dist):
+# arithmetic of each execution path (coli_moe_layer_kernels -> path), for the `dtype` key
+PATH_DTYPE = {
+    1: "int8 x int8 tensor-core MMA (int32 accumulate) on 24-bit fixed-point activations, f32 epilogue",
+    5: "f32 CUDA-core GEMV on dequantised codes",
+    7: "int8 x int8 tensor-core MMA (int32 accumulate) on 16-bit fixed-point activations, f32 epilogue",
+}
+PATH_NAME = {1: "fused decode kernel", 5: "gate/route/group + GEMV expert kernels",
+             7: "gate/route/group + tensor-core grouped GEMM"}
+
+
+def workload_config(wl, T):
+    """The `config` keys that name the workload (shared by both arms)."""
+    return {
+        "workload": {"glm_decode": "glm_decode (GLM-5.2-shaped decode layer)",
+                     "glm_prefill": "glm_prefill (GLM-5.2-shaped 2048-token prefill layer, Zipf(1.1) popularity)"
+                     }.get(wl.name, wl.name),
+        "tokens_per_step": T, "hidden": wl.hidden, "expert_inter": wl.inter,
+        "experts": wl.n_experts, "top_k": wl.top_k, "n_group": wl.n_group,
+        "topk_group": wl.topk_group, "shared_experts": wl.n_shared,
+        "weights": {4: "packed int4", 8: "int8", 2: "packed int2"}[wl.fmt] + " per-row f32 scales",
+        "activations": wl.act,
+    }
+
+
+def measure(args, wl, T, n_layers, K, W, rank, world, dist, dev, label):
+    """Time K whole-layer steps of workload `wl` at T tokens (after >= W warm-up steps), the
+    expert FFN launches alone, and the end-to-end rate with host buffers.  Returns the result
+    dict and the context the CPU baseline needs."""
     import quantized_routed_expert_noaux_b200 as q
 
-    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
-    torch.cuda.set_device(dev)
-    wl = synth.WORKLOADS[args.workload]
-    T = args.tokens or wl.tokens[0]
-    n_layers = args.layers or (4 if wl.hidden >= 2048 else 1)
     cfg = q.config_for(wl)
-
     layers = []
     for l in range(n_layers):
         ex = synth.make_expert_records(wl, device=dev, layer=l)
         sh = synth.make_shared_record(wl, device=dev, layer=l)
         Wr, b = synth.make_router(wl, device=dev, layer=l)
         layers.append((ex, sh, Wr, b, q.weights_for(Wr, b, ex, sh)))
-    n_x = 64
+    n_x = 64 if T <= 64 else 4
     xs = [synth.make_activations(wl, T, device=dev, step=1000 * rank + i) for i in range(n_x)]
-    K, W = args.steps, args.warmup
     out = torch.empty(T, wl.hidden, dtype=torch.float32, device=dev)
     ids_all = torch.empty(K, T, wl.top_k, dtype=torch.int32, device=dev)
     ws = torch.empty(q.coli_moe_workspace_size(cfg, T), dtype=torch.uint8, device=dev)
@@ -180,6 +202,10 @@ def gpu_arm(args, rank, world, dist):
             raise RuntimeError("device error word set")
         return None, None
 
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
     clocks = Clocks(dev.index if dev.index is not None else 0)
     q.coli_moe_clear_error(ws)
     t_soak = time.time()
@@ -190,11 +216,6 @@ def gpu_arm(args, rank, world, dist):
         if i % 256 == 0:
             torch.cuda.synchronize()
     torch.cuda.synchronize()
-
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -208,7 +229,7 @@ def gpu_arm(args, rank, world, dist):
     clk = clocks.stop()
     err = q.coli_moe_error_word(ws)
     if err:
-        raise RuntimeError(f"device error word {err:#x} after the timed region")
+        raise RuntimeError(f"device error word {err:#x} after the timed region ({label})")
     ms_max = max_over_ranks(ms, dist, dev)
 
     # algorithmic bytes of the timed steps (unique experts per step from the routing written)
@@ -217,7 +238,8 @@ def gpu_arm(args, rank, world, dist):
     bytes_steps = sum(alg_bytes(wl, T, int(u)) for u in U)
     expert_bytes = sum((int(u) + wl.n_shared) * record_bytes(wl) for u in U)
 
-    # live per-launch time of the expert FFN (gate/up + down GEMV kernels), same rotation
+    # live per-launch time of the expert FFN part (coli_moe_ffn on the same rotation), on the
+    # launching stream
     offs = torch.empty(wl.n_experts + 1, dtype=torch.int32, device=dev)
     perm = torch.empty(T * wl.top_k, dtype=torch.int32, device=dev)
     cnt = torch.empty(wl.n_experts, dtype=torch.int32, device=dev)
@@ -241,8 +263,8 @@ def gpu_arm(args, rank, world, dist):
     torch.cuda.synchronize()
     ffn_ms = sum(a.elapsed_time(b) for a, b in evs) / n_ffn
     U_mean = float(U[:n_ffn].mean()) if len(U) else 0.0
-    ffn_bytes = (U_mean + wl.n_shared) * record_bytes(wl) + T * wl.hidden * (4 if wl.act == "f32" else 2) \
-        + T * wl.hidden * 4
+    act = 4 if wl.act == "f32" else 2
+    ffn_bytes = (U_mean + wl.n_shared) * record_bytes(wl) + T * wl.hidden * act + T * wl.hidden * 4
 
     # end to end through the C ABI with host buffers: pinned H2D of x, layer, D2H of out
     x_host = [xs[i].cpu().pin_memory() for i in range(n_x)]
@@ -265,9 +287,8 @@ def gpu_arm(args, rank, world, dist):
 
     hbm, bf16, bf16s, peak_kind = peaks()
     tok_s = whole_job_rate(world, K, T, ms_max)
-    achieved = ffn_bytes / (ffn_ms / 1e3) / 1e9
     traffic = None
-    tf = os.path.join(PROFILES, f"{args.workload}_t{T}_traffic.json")
+    tf = os.path.join(PROFILES, f"{wl.name}_t{T}_traffic.json")
     if os.path.exists(tf):
         d = json.load(open(tf))
         cur = src_hash([os.path.join(ROOT, "quantized_routed_expert_noaux_b200", "csrc", f)
@@ -276,66 +297,51 @@ def gpu_arm(args, rank, world, dist):
             traffic = d.get("traffic_bytes_per_launch")
 
     n_kern = q.coli_moe_layer_kernels(cfg, T)
-    # tensor-core path: int8 MMAs on two 8-bit activation slices, i.e. two int8 operations per
-    # algorithmic multiply-add -- the bf16 tensor rate; ~1 ms launches back to back -> sustained.
-    # Its bound is whichever of the flops and the bytes takes longer at the measured peaks (small
-    # batches on that path are bound by HBM like decode).
+    # Tensor-core path: int8 MMAs on two 8-bit activation slices, i.e. two int8 operations per
+    # algorithmic multiply-add -- the bf16 tensor rate; ~1 ms launches back to back -> sustained
+    # peak.  The bound is whichever of the flops and the bytes takes longer at the measured
+    # peaks (small batches on that path are bound by HBM like decode).
     ffn_flops = (T * wl.top_k + T * wl.n_shared) * 6.0 * wl.hidden * wl.inter
     peak_t = bf16s if bf16s else bf16
     tc_kernel = "expert FFN (x quantisation, gate/up int8 GEMM, h quantisation, down int8 GEMM + combine)"
     if n_kern == 7 and ffn_flops / (peak_t * 1e12) > ffn_bytes / (hbm * 1e9):
         tf_s = ffn_flops / (ffn_ms / 1e3) / 1e12
         roofline = {
-            "bound": "tensor",
-            "kernel": tc_kernel,
-            "achieved": round(tf_s, 1),
-            "peak": peak_t,
-            "unit": "TFLOP/s",
-            "frac": round(tf_s / peak_t, 4),
-            "traffic": traffic,
-            "peak_source": f"{peak_kind} bf16_tflops{'_sustained' if bf16s else ''} (int8 with two activation "
-                           "slices runs algorithmic flops at the bf16 rate)",
+            "bound": "tensor", "kernel": tc_kernel, "achieved": round(tf_s, 1), "peak": peak_t,
+            "unit": "TFLOP/s", "frac": round(tf_s / peak_t, 4), "traffic": traffic,
+            "peak_source": f"{peak_kind} bf16_tflops{'_sustained' if bf16s else ''} (int8 with two "
+                           "activation slices runs algorithmic flops at the bf16 rate); frac of measured",
             "launch_us": round(ffn_ms * 1e3, 2),
             "hbm_gbs_of_weights": round(ffn_bytes / (ffn_ms / 1e3) / 1e9, 1),
         }
     else:
+        achieved = ffn_bytes / (ffn_ms / 1e3) / 1e9
         roofline = {
             "bound": "hbm",
             "kernel": ("fused decode layer kernel (FFN part)" if n_kern == 1 else
                        tc_kernel if n_kern == 7 else "expert FFN (gate/up GEMV + down GEMV with fused combine)"),
-            "achieved": round(achieved, 1),
-            "peak": hbm,
-            "unit": "GB/s",
-            "frac": round(achieved / hbm, 4),
-            "traffic": traffic,
-            "peak_source": f"{peak_kind} hbm_gbs (copy bandwidth)",
+            "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+            "frac": round(achieved / hbm, 4), "traffic": traffic,
+            "peak_source": f"{peak_kind} hbm_gbs (copy bandwidth); frac of measured",
             "launch_us": round(ffn_ms * 1e3, 2),
         }
-
+    # whole-layer roofline: max(bytes / HBM, flops / tensor peak) over the measured step time
+    layer_flops = alg_flops(wl, T)
+    t_roof = max(bytes_steps / K / (hbm * 1e9), layer_flops / (peak_t * 1e12))
     res = {
-        "metric": METRIC,
         "value": round(tok_s, 2),
         "unit": "tokens/s",
-        "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": round(ms_max / K, 6),
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
-        "dtype": "f32",
-        "data": "synthetic (seeded; weights N(0,0.02) quantised per row, activations N(0,1))",
-        "config": {
-            "workload": f"{wl.name} (GLM-5.2-shaped decode layer)" if wl.name == "glm_decode" else wl.name,
-            "tokens_per_step": T, "hidden": wl.hidden, "expert_inter": wl.inter,
-            "experts": wl.n_experts, "top_k": wl.top_k, "n_group": wl.n_group,
-            "topk_group": wl.topk_group, "shared_experts": wl.n_shared,
-            "weights": {4: "packed int4", 8: "int8", 2: "packed int2"}[wl.fmt] + " per-row f32 scales",
-            "activations": wl.act,
-            "l2": f"rotation over {n_layers} resident layers ({n_layers * wl.n_experts * record_bytes(wl) / 1e9:.1f} GB of expert records) + fresh activations every step; no flush",
-            "parallelism": f"replicas x{world}",
-        },
+        "dtype": PATH_DTYPE[n_kern],
+        "path": PATH_NAME[n_kern],
+        "config": dict(workload_config(wl, T),
+                       l2=f"rotation over {n_layers} resident layers ({n_layers * wl.n_experts * record_bytes(wl) / 1e9:.1f} GB of expert records) + fresh activations every step; no flush",
+                       parallelism=f"replicas x{world}"),
         "expert_gbs": round(expert_bytes / (ms_max / 1e3) / 1e9, 1),
         "layer_gbs": round(bytes_steps / (ms_max / 1e3) / 1e9, 1),
         "layer_frac_of_hbm": round(bytes_steps / (ms_max / 1e3) / 1e9 / hbm, 4),
+        "layer_roofline_us": round(t_roof * 1e6, 2),
+        "layer_frac_of_roofline": round(t_roof / (ms_max / K / 1e3), 4),
         "unique_experts_mean": round(float(U.mean()), 2),
         "roofline": roofline,
         "e2e": {"value": round(whole_job_rate(world, K2, T, e2e_ms), 2), "unit": "tokens/s",
@@ -345,6 +351,33 @@ def gpu_arm(args, rank, world, dist):
         "clocks": clk,
     }
     return res, (wl, T, layers, xs)
+
+
+def gpu_arm(args, rank, world, dist):
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    wl = synth.WORKLOADS[args.workload]
+    T = args.tokens or wl.tokens[0]
+    n_layers = args.layers or (4 if wl.hidden >= 2048 else 1)
+    K, W = args.steps, args.warmup
+    res, ctx = measure(args, wl, T, n_layers, K, W, rank, world, dist, dev, wl.name)
+    if res is None:
+        return None, None
+    line = {"metric": METRIC, "value": res.pop("value"), "unit": res.pop("unit"), "n_gpus": world,
+            "steps": K, "warmup": W, "ms_per_step": res.pop("ms_per_step"),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": res.pop("dtype"),
+            "data": "synthetic (seeded; weights N(0,0.02) quantised per row, activations N(0,1))"}
+    line.update(res)
+    if args.workload == "glm_decode" and not args.no_prefill:
+        # the second headline workload: the 2048-token prefill layer, its own timed region
+        pwl = synth.WORKLOADS["glm_prefill"]
+        pres, pctx = measure(args, pwl, pwl.tokens[0], 2, min(K, 20), max(W, 3), rank, world, dist,
+                             dev, pwl.name)
+        pres["steps"] = min(K, 20)
+        line["prefill"] = pres
+        ctx = ctx + (pctx,)
+    return line, ctx
 
 
 # ------------------------------------------------------------------------- CPU oracle -------
@@ -384,6 +417,12 @@ def _oracle_sample(wl, T_tokens, x_list, layers_dev, budget_s, device):
     t0 = time.time()
     oracle.layer(cfg, Wr_h, b_h, R, xs, n, n_threads=threads)
     return n, time.time() - t0, threads
+
+
+def cpu_baseline(wl, T, xs, layers, seconds):
+    n, sec, thr = _oracle_sample(wl, T, xs[:8], layers[0][:4], seconds, None)
+    return {"value": round(n / sec, 4), "unit": "tokens/s", "cores": thr, "kind": "oracle",
+            "sample": f"{n} tokens of the same workload (layer 0), {sec:.1f} s wall on {thr} threads"}
 
 
 def reference_arm(args):
@@ -430,8 +469,9 @@ def reference_arm(args):
         "n_gpus": 1, "steps": steps_done, "warmup": W, "ms_per_step": round(1e3 * sec / steps_done, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded)",
-        "config": {"workload": wl.name, "tokens_per_step": T},
-        "cpu_baseline": {"value": round(val, 4), "unit": "tokens/s", "cores": threads,
+        "config": dict(workload_config(wl, T), parallelism="host cores (oracle)"),
+        # the oracle parallelises over tokens: a step of T tokens keeps min(T, threads) busy
+        "cpu_baseline": {"value": round(val, 4), "unit": "tokens/s", "cores": min(threads, T),
                          "kind": "oracle",
                          "sample": f"{steps_done} steps of {T} token(s) each (run stopped after {budget:.0f} s if K was larger)"},
         "e2e": {"value": round(val, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -458,11 +498,11 @@ def main():
     if res is None:
         return
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        wl, T, layers, xs = ctx
-        n, sec, thr = _oracle_sample(wl, T, xs[:8], layers[0][:4], args.cpu_seconds, None)
-        res["cpu_baseline"] = {"value": round(n / sec, 4), "unit": "tokens/s", "cores": thr,
-                               "kind": "oracle",
-                               "sample": f"{n} tokens of the same workload (layer 0), {sec:.1f} s wall on {thr} threads"}
+        wl, T, layers, xs = ctx[:4]
+        res["cpu_baseline"] = cpu_baseline(wl, T, xs, layers, args.cpu_seconds)
+        if len(ctx) > 4:
+            pwl, pT, players, pxs = ctx[4]
+            res["prefill"]["cpu_baseline"] = cpu_baseline(pwl, pT, pxs, players, args.cpu_seconds)
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()

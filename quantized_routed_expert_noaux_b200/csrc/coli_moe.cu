@@ -324,6 +324,24 @@ coli_status coli_moe_ffn(const coli_moe_config *c, const coli_moe_weights *w, co
     return run_ffn(c, p, base, static_cast<cudaStream_t>(stream));
 }
 
+}  // extern "C"
+
+// Every host-side check of coli_moe_layer except the workspace's (T >= 1).
+coli_status coli::layer_args_status(const coli_moe_config *c, const coli_moe_weights *w, const void *x,
+                                    int T, const float *out, const int32_t *topk_ids_out,
+                                    const float *topk_w_out) {
+    coli_status s = check_weights(c, w, true);
+    if (s != COLI_OK) return s;
+    if (!x || !out) return COLI_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(out, 16)) return COLI_ERR_ALIGN;
+    if ((topk_ids_out && !aligned(topk_ids_out, 4)) || (topk_w_out && !aligned(topk_w_out, 4)))
+        return COLI_ERR_ALIGN;
+    if (T > gemv_max_tokens(*c) && !use_tc(c, T)) return COLI_ERR_UNSUPPORTED;
+    return COLI_OK;
+}
+
+extern "C" {
+
 coli_status coli_moe_layer(const coli_moe_config *c, const coli_moe_weights *w, const void *x, int T,
                            float *out, int32_t *topk_ids_out, float *topk_w_out, void *ws,
                            size_t ws_bytes, void *stream) {
@@ -331,13 +349,8 @@ coli_status coli_moe_layer(const coli_moe_config *c, const coli_moe_weights *w, 
     if (s != COLI_OK) return s;
     if (T < 0) return COLI_ERR_SHAPE;
     if (T == 0) return COLI_OK;
-    s = check_weights(c, w, true);
+    s = layer_args_status(c, w, x, T, out, topk_ids_out, topk_w_out);
     if (s != COLI_OK) return s;
-    if (!x || !out) return COLI_ERR_INVALID_ARG;
-    if (!aligned(x, 16) || !aligned(out, 16)) return COLI_ERR_ALIGN;
-    if ((topk_ids_out && !aligned(topk_ids_out, 4)) || (topk_w_out && !aligned(topk_w_out, 4)))
-        return COLI_ERR_ALIGN;
-    if (T > gemv_max_tokens(*c) && !use_tc(c, T)) return COLI_ERR_UNSUPPORTED;
     const WsLayout L = ws_layout(*c, T);
     if (!ws || !aligned(ws, 256) || ws_bytes < L.total) return COLI_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -123,6 +123,12 @@ cudaError_t launch_ffn_gemv(const FfnParams &p, cudaStream_t st);
 bool gemv_shape_ok(int row_bytes);
 int gemv_max_tokens(const coli_moe_config &c);
 
+// Host-side checks of a whole-layer call other than the workspace's (weights, pointers,
+// alignment, token count); T >= 1.  No launch.
+coli_status layer_args_status(const coli_moe_config *c, const coli_moe_weights *w, const void *x,
+                              int T, const float *out, const int32_t *topk_ids_out,
+                              const float *topk_w_out);
+
 int device_sm_count();
 size_t device_smem_optin();  // max dynamic shared memory per block (opt-in)
 void record_cuda_error(cudaError_t e);

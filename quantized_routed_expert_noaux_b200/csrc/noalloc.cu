@@ -54,12 +54,16 @@ extern "C" coli_status coli_moe_layer_noalloc(const coli_moe_config *cfg, const 
     s = coli_moe_workspace_size(cfg, T, &need);
     if (s != COLI_OK) return s;
     if (need > static_cast<size_t>(COLI_MOE_STATIC_SCRATCH_BYTES)) return COLI_ERR_WORKSPACE;
+    // every argument check before the first GPU operation: a rejected call launches nothing
+    s = coli::layer_args_status(cfg, w, x, T, out, topk_ids_out, topk_w_out);
+    if (s != COLI_OK) return s;
     void *ws = nullptr;
     s = static_scratch(&ws);
     if (s != COLI_OK) return s;
     // The array keeps the previous call's contents: the header (error word and counters) must
     // start at zero for every call.
-    if (cudaMemsetAsync(ws, 0, 256, static_cast<cudaStream_t>(stream)) != cudaSuccess) return COLI_ERR_CUDA;
+    if (cudaMemsetAsync(ws, 0, coli::WS_HEADER, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return COLI_ERR_CUDA;
     return coli_moe_layer(cfg, w, x, T, out, topk_ids_out, topk_w_out, ws,
                           static_cast<size_t>(COLI_MOE_STATIC_SCRATCH_BYTES), stream);
 }

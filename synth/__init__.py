@@ -83,6 +83,11 @@ WORKLOADS: Dict[str, Workload] = {
     # GLM-5.2 expert shapes with 32 experts and uniform routing: a 0.6 GB layer on which the
     # tensor-core kernels run with mostly full token chunks (small enough for ncu captures)
     "glm_e32": Workload("glm_e32", fmt=4, tokens=(1024,), seed=2, **dict(_GLM, n_experts=32)),
+    # GLM-5.2 expert shapes with 64 experts (8 groups, 4 kept) and the prefill layer's Zipf(1.1)
+    # popularity at 512 tokens: ~64 tokens per expert on average with a long tail of small
+    # ones, as on the 2048-token layer, in a 1.2 GB layer (small enough for ncu captures)
+    "glm_zipf_e64": Workload("glm_zipf_e64", fmt=4, tokens=(512,), seed=2, zipf_s=1.1,
+                             **dict(_GLM, n_experts=64)),
     "glm_int8": Workload("glm_int8", fmt=8, tokens=(64,), seed=4, n_layers=4, **_GLM),
     "glm_int2": Workload("glm_int2", fmt=2, tokens=(64,), seed=4, n_layers=4, **_GLM),
 }
