@@ -61,7 +61,7 @@ def peaks():
 
 
 def record_bytes(wl):
-    return synth.record_layout(wl.hidden, wl.inter, wl.fmt)["bytes"]
+    return synth.record_layout(wl.hidden, wl.inter, wl.fmt, wl.group)["bytes"]
 
 
 def alg_bytes(wl, T, U):

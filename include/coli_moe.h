@@ -21,11 +21,15 @@
  *   - There is no CPU fallback: every step runs in this library's CUDA kernels.
  *
  * Record format (one per expert; the same for the shared expert with its own inter size)
- *   Wg codes [I][H] | Wu codes [I][H] | Wd codes [H][I] | sg[I] f32 | su[I] f32 | sd[H] f32,
+ *   Wg codes [I][H] | Wu codes [I][H] | Wd codes [H][I] | sg | su | sd (float32 scales),
  *   rows packed to whole bytes: int4 element 2j in the low nibble of byte j and 2j+1 in the
  *   high nibble (two's complement, [-8,7]); int2 element 4j+k in bits [2k,2k+1] of byte j
- *   ([-2,1]); int8 one signed byte.  The weight is code * scale of its output row.  Records sit
- *   `expert_stride` bytes apart (a multiple of 256) and the record base must be 256-byte aligned.
+ *   ([-2,1]); int8 one signed byte.  Per-row container (group_size 0): sg[I], su[I], sd[H], the
+ *   weight is code * scale of its output row.  Group-scaled container (group_size 64, int4 only;
+ *   the JustVugg/colibri README, "Get started -> 2. Get the model", recommends this GLM-5.2
+ *   build): sg[I][H/64], su[I][H/64], sd[H][I/64], the weight is code * scale of its group of 64
+ *   consecutive columns of the row.  Records sit `expert_stride` bytes apart (a multiple of
+ *   256) and the record base must be 256-byte aligned.
  *
  * Tensor layouts (row-major):
  *   x        [T][H]   float32 (act = COLI_ACT_F32) or bfloat16 bits (COLI_ACT_BF16), 16-B aligned
@@ -75,6 +79,7 @@ typedef struct {
     double routed_scaling;  /* rsf */
     int wfmt;               /* coli_wfmt */
     int act;                /* coli_act */
+    int group_size;         /* 0: one scale per weight row; 64: one per 64 columns (int4 only) */
 } coli_moe_config;
 
 typedef struct {
@@ -91,8 +96,8 @@ const char *coli_moe_status_str(coli_status s);
 /* Name and text of the CUDA error behind the calling thread's last COLI_ERR_CUDA ("" if none). */
 const char *coli_moe_last_cuda_error(void);
 
-/* Bytes of one record for (hidden, inter, wfmt), before padding to 256.  Host only. */
-coli_status coli_moe_record_bytes(int hidden, int inter, int wfmt, size_t *bytes);
+/* Bytes of one record for (hidden, inter, wfmt, group_size), before padding to 256.  Host only. */
+coli_status coli_moe_record_bytes(int hidden, int inter, int wfmt, int group_size, size_t *bytes);
 
 /* Validates a configuration (the same checks every call makes).  Host only. */
 coli_status coli_moe_check_config(const coli_moe_config *cfg);
@@ -173,6 +178,15 @@ coli_status coli_moe_layer(const coli_moe_config *cfg, const coli_moe_weights *w
  * Asynchronous on `stream`; allocates nothing. */
 coli_status coli_moe_residual(const coli_moe_config *cfg, const void *x, const float *out, int T,
                               void *x_next, void *stream);
+
+/* Testing aid for the bounded device-side waits of the fused decode kernel (the one-launch
+ * path that coli_moe_layer_kernels reports as 1 kernel).  wait_cycles > 0 replaces the default
+ * bound (about 2 s of SM clock) of every wait in that kernel's later launches made by the
+ * calling thread; unreachable != 0 raises its grid-barrier targets beyond reach, so that every
+ * such wait runs out: the call still completes, each wait ends within its bound, nothing traps,
+ * the workspace's error word gets COLI_DEVERR_TIMEOUT and the outputs are invalid.  (0, 0)
+ * restores the defaults.  Host only; COLI_ERR_INVALID_ARG for a negative bound. */
+coli_status coli_moe_debug_set_wait(long long wait_cycles, int unreachable);
 
 /* Size of the static scratch array behind coli_moe_layer_noalloc (8 MiB per GPU). */
 #define COLI_MOE_STATIC_SCRATCH_BYTES (8u << 20)

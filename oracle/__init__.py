@@ -24,14 +24,14 @@ class OracleCfg(C.Structure):
         ("hidden", C.c_int), ("inter", C.c_int), ("n_experts", C.c_int), ("top_k", C.c_int),
         ("n_group", C.c_int), ("topk_group", C.c_int), ("n_shared", C.c_int),
         ("shared_inter", C.c_int), ("routed_scaling", C.c_double), ("fmt", C.c_int),
-        ("act", C.c_int),
+        ("act", C.c_int), ("group", C.c_int),
     ]
 
 
 def _load():
     lib = C.CDLL(_build.build())
     P = C.c_void_p
-    lib.oracle_record_bytes.argtypes = [C.c_int, C.c_int, C.c_int, C.POINTER(C.c_size_t)]
+    lib.oracle_record_bytes.argtypes = [C.c_int, C.c_int, C.c_int, C.c_int, C.POINTER(C.c_size_t)]
     lib.oracle_unpack_row.argtypes = [P, C.c_int, C.c_int, P]
     lib.oracle_pack_row.argtypes = [P, C.c_int, C.c_int, P]
     lib.oracle_gate.argtypes = [C.POINTER(OracleCfg), P, P, C.c_int, P]
@@ -86,16 +86,16 @@ def make_cfg(wl) -> OracleCfg:
     """OracleCfg from a synth.Workload (or anything with the same attributes)."""
     return OracleCfg(wl.hidden, wl.inter, wl.n_experts, wl.top_k, wl.n_group, wl.topk_group,
                      wl.n_shared, wl.shared_inter, float(wl.routed_scaling), wl.fmt,
-                     0 if wl.act == "f32" else 1)
+                     0 if wl.act == "f32" else 1, getattr(wl, "group", 0))
 
 
 def _x(cfg: OracleCfg, x):
     return _np(x, np.float32 if cfg.act == 0 else np.uint16)
 
 
-def record_bytes(hidden: int, inter: int, fmt: int) -> int:
+def record_bytes(hidden: int, inter: int, fmt: int, group: int = 0) -> int:
     n = C.c_size_t()
-    if lib().oracle_record_bytes(hidden, inter, fmt, C.byref(n)) != 0:
+    if lib().oracle_record_bytes(hidden, inter, fmt, group, C.byref(n)) != 0:
         raise ValueError("bad record shape")
     return n.value
 

@@ -24,14 +24,26 @@ static int row_bytes(int n, int fmt, size_t *out)
     return -1;
 }
 
-/* Record = three code matrices stored adjacent, then their per-row scales (JustVugg/colibri
- * README, "Never wait for the disk twice": an expert's three matrices sit next to each other). */
-int oracle_record_bytes(int hidden, int inter, int fmt, size_t *bytes)
+/* Scales per row of a matrix with `cols` columns: one (per-row container) or cols / group
+ * (group-scaled container, JustVugg/colibri README, "Get started -> 2. Get the model": the
+ * recommended GLM-5.2 build is group-scaled, gs64).  -1 when group does not divide cols. */
+static long scales_per_row(int cols, int group)
+{
+    if (group == 0) return 1;
+    if (group < 0 || cols % group) return -1;
+    return cols / group;
+}
+
+/* Record = three code matrices stored adjacent, then their scales (JustVugg/colibri README,
+ * "Never wait for the disk twice": an expert's three matrices sit next to each other). */
+int oracle_record_bytes(int hidden, int inter, int fmt, int group, size_t *bytes)
 {
     size_t rh, ri;
     if (row_bytes(hidden, fmt, &rh) || row_bytes(inter, fmt, &ri)) return -1;
+    const long nh = scales_per_row(hidden, group), ni = scales_per_row(inter, group);
+    if (nh < 0 || ni < 0) return -1;
     *bytes = 2 * (size_t)inter * rh + (size_t)hidden * ri
-           + (2 * (size_t)inter + (size_t)hidden) * sizeof(float);
+           + (2 * (size_t)inter * (size_t)nh + (size_t)hidden * (size_t)ni) * sizeof(float);
     return 0;
 }
 
@@ -81,9 +93,11 @@ int oracle_pack_row(const int8_t *q, int n, int fmt, uint8_t *row)
     return 0;
 }
 
-/* Dequantise one element: weight = code * row scale, exact in double (dequant-on-use,
- * colibri-strix README, "What's implemented"). */
-static double dequant(const uint8_t *mat, size_t rb, int fmt, const float *scales, int r, int c)
+/* Dequantise one element: weight = code * its scale, exact in double (dequant-on-use,
+ * colibri-strix README, "What's implemented").  The scale is the row's (group == 0) or that of
+ * the element's group of `group` consecutive columns of the row. */
+static double dequant(const uint8_t *mat, size_t rb, int fmt, const float *scales, int r, int c,
+                      int cols, int group)
 {
     const uint8_t *row = mat + (size_t)r * rb;
     int v;
@@ -98,7 +112,8 @@ static double dequant(const uint8_t *mat, size_t rb, int fmt, const float *scale
         int code = (byte >> (2 * (c % 4))) & 0x03;
         v = (code >= 2) ? code - 4 : code;
     }
-    return (double)v * (double)scales[r];
+    const size_t si = group == 0 ? (size_t)r : (size_t)r * (size_t)(cols / group) + (size_t)(c / group);
+    return (double)v * (double)scales[si];
 }
 
 /* ---------------------------------------------------------------- activations ------------- */
@@ -262,25 +277,31 @@ void oracle_expert(const oracle_cfg *cfg, const uint8_t *record, int inter, cons
         for (int j = 0; j < H; j++) y[j] = NAN;
         return;
     }
+    const int grp = cfg->group;
+    const long nh = scales_per_row(H, grp), ni = scales_per_row(I, grp);
+    if (nh < 0 || ni < 0) {
+        for (int j = 0; j < H; j++) y[j] = NAN;
+        return;
+    }
     const uint8_t *Wg = record;
     const uint8_t *Wu = Wg + (size_t)I * rh;
     const uint8_t *Wd = Wu + (size_t)I * rh;
     const float *sg = (const float *)(Wd + (size_t)H * ri);
-    const float *su = sg + I;
-    const float *sd = su + I;
+    const float *su = sg + (size_t)I * nh;
+    const float *sd = su + (size_t)I * nh;
 
     double *a = (double *)malloc(sizeof(double) * (size_t)I);
     for (int i = 0; i < I; i++) {
         double g = 0.0, u = 0.0;
         for (int h = 0; h < H; h++) {
-            g += dequant(Wg, rh, fmt, sg, i, h) * x[h];
-            u += dequant(Wu, rh, fmt, su, i, h) * x[h];
+            g += dequant(Wg, rh, fmt, sg, i, h, H, grp) * x[h];
+            u += dequant(Wu, rh, fmt, su, i, h, H, grp) * x[h];
         }
         a[i] = (g / (1.0 + exp(-g))) * u;
     }
     for (int j = 0; j < H; j++) {
         double acc = 0.0;
-        for (int i = 0; i < I; i++) acc += dequant(Wd, ri, fmt, sd, j, i) * a[i];
+        for (int i = 0; i < I; i++) acc += dequant(Wd, ri, fmt, sd, j, i, I, grp) * a[i];
         y[j] = acc;
     }
     free(a);

@@ -51,12 +51,15 @@ typedef struct {
     double routed_scaling;
     int fmt;           /* 4, 8 or 2 */
     int act;           /* 0 f32, 1 bf16 */
+    int group;         /* 0: one scale per row; g > 0: one scale per g consecutive columns */
 } oracle_cfg;
 
 /* Bytes of one expert record with intermediate size `inter` (unpadded; callers pad to 256).
  * Record layout: Wg codes [I][H], Wu codes [I][H], Wd codes [H][I] (row-major, each row packed
- * to whole bytes), then float32 scales sg[I], su[I], sd[H].  Returns 0 on success. */
-int oracle_record_bytes(int hidden, int inter, int fmt, size_t *bytes);
+ * to whole bytes), then float32 scales sg, su, sd: per row (sg[I], su[I], sd[H]) when group is
+ * 0, else per group of `group` consecutive columns (sg[I][H/group], su[I][H/group],
+ * sd[H][I/group]).  Returns 0 on success, -1 when a size does not fit the format. */
+int oracle_record_bytes(int hidden, int inter, int fmt, int group, size_t *bytes);
 
 /* Container decode: n codes of one packed row -> two's-complement integers.
  * int4: element 2j in the low nibble of byte j, 2j+1 in the high nibble, range [-8, 7].

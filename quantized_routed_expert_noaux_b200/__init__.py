@@ -18,6 +18,7 @@ __all__ = [
     "coli_moe_workspace_size", "coli_moe_clear_error", "coli_moe_error_word",
     "coli_moe_gate", "coli_moe_route", "coli_moe_group", "coli_moe_ffn", "coli_moe_layer",
     "coli_moe_layer_noalloc", "STATIC_SCRATCH_BYTES", "coli_moe_layer_kernels", "coli_moe_residual",
+    "coli_moe_debug_set_wait",
     "config_for", "weights_for",
     "COLI_W_INT2", "COLI_W_INT4", "COLI_W_INT8", "COLI_ACT_F32", "COLI_ACT_BF16",
 ]
@@ -26,7 +27,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libcoli_moe
 
 COLI_W_INT2, COLI_W_INT4, COLI_W_INT8 = 2, 4, 8
 COLI_ACT_F32, COLI_ACT_BF16 = 0, 1
-DEVERR_EXPERT_ID, DEVERR_GROUPING = 0x1, 0x2
+DEVERR_EXPERT_ID, DEVERR_GROUPING, DEVERR_TIMEOUT = 0x1, 0x2, 0x4
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -39,7 +40,7 @@ class MoEConfig(C.Structure):
         ("hidden", C.c_int), ("inter", C.c_int), ("n_experts", C.c_int), ("top_k", C.c_int),
         ("n_group", C.c_int), ("topk_group", C.c_int), ("n_shared", C.c_int),
         ("shared_inter", C.c_int), ("routed_scaling", C.c_double), ("wfmt", C.c_int),
-        ("act", C.c_int),
+        ("act", C.c_int), ("group_size", C.c_int),
     ]
 
 
@@ -67,7 +68,7 @@ def _load():
     L.coli_moe_status_str.restype = C.c_char_p
     L.coli_moe_last_cuda_error.argtypes = []
     L.coli_moe_last_cuda_error.restype = C.c_char_p
-    L.coli_moe_record_bytes.argtypes = [I, I, I, C.POINTER(S)]
+    L.coli_moe_record_bytes.argtypes = [I, I, I, I, C.POINTER(S)]
     L.coli_moe_check_config.argtypes = [cfgp]
     L.coli_moe_workspace_size.argtypes = [cfgp, I, C.POINTER(S)]
     L.coli_moe_clear_error.argtypes = [P, P]
@@ -80,12 +81,13 @@ def _load():
     L.coli_moe_layer_noalloc.argtypes = [cfgp, wp, P, I, P, P, P, P]
     L.coli_moe_layer_kernels.argtypes = [cfgp, I, C.POINTER(I)]
     L.coli_moe_residual.argtypes = [cfgp, P, P, I, P, P]
+    L.coli_moe_debug_set_wait.argtypes = [C.c_longlong, I]
     L.coli_moe_layer_kernels.restype = I
     L.coli_moe_layer_noalloc.restype = I
     for name in ("coli_moe_record_bytes", "coli_moe_check_config", "coli_moe_workspace_size",
                  "coli_moe_clear_error", "coli_moe_error_word", "coli_moe_gate",
                  "coli_moe_route", "coli_moe_group", "coli_moe_ffn", "coli_moe_layer",
-                 "coli_moe_residual"):
+                 "coli_moe_residual", "coli_moe_debug_set_wait"):
         getattr(L, name).restype = I
     return L
 
@@ -125,9 +127,9 @@ def coli_moe_last_cuda_error() -> str:
     return lib.coli_moe_last_cuda_error().decode()
 
 
-def coli_moe_record_bytes(hidden: int, inter: int, wfmt: int) -> int:
+def coli_moe_record_bytes(hidden: int, inter: int, wfmt: int, group_size: int = 0) -> int:
     n = C.c_size_t()
-    _check("coli_moe_record_bytes", lib.coli_moe_record_bytes(hidden, inter, wfmt, C.byref(n)))
+    _check("coli_moe_record_bytes", lib.coli_moe_record_bytes(hidden, inter, wfmt, group_size, C.byref(n)))
     return n.value
 
 
@@ -210,13 +212,19 @@ def coli_moe_layer_noalloc(cfg, weights: MoEWeights, x, T, out, topk_ids_out=Non
         _stream(stream)))
 
 
+def coli_moe_debug_set_wait(wait_cycles: int, unreachable: bool) -> None:
+    """Testing aid: the fused decode kernel's wait bound (cycles, 0 = default) and whether its
+    grid-barrier targets are out of reach (every wait then runs out and reports a timeout)."""
+    _check("coli_moe_debug_set_wait", lib.coli_moe_debug_set_wait(wait_cycles, int(bool(unreachable))))
+
+
 def config_for(wl) -> MoEConfig:
     """MoEConfig with the shape fields of a workload description (any object with the
     attributes hidden, inter, n_experts, top_k, n_group, topk_group, n_shared, shared_inter,
     routed_scaling, fmt and act = "f32" | "bf16")."""
     return MoEConfig(wl.hidden, wl.inter, wl.n_experts, wl.top_k, wl.n_group, wl.topk_group,
                      wl.n_shared, wl.shared_inter, float(wl.routed_scaling), wl.fmt,
-                     COLI_ACT_F32 if wl.act == "f32" else COLI_ACT_BF16)
+                     COLI_ACT_F32 if wl.act == "f32" else COLI_ACT_BF16, getattr(wl, "group", 0))
 
 
 def weights_for(router_w, router_bias, experts, shared=None) -> MoEWeights:

@@ -20,6 +20,10 @@ inline bool aligned(const void *p, size_t a) {
 }
 
 thread_local char g_last_cuda_error[256] = "";
+// testing aid (coli_moe_debug_set_wait): the fused decode kernel's wait bound and a flag that
+// makes its grid-barrier targets unreachable
+thread_local long long g_wait_cycles = 0;
+thread_local int g_unreachable = 0;
 
 coli_status from_cuda(cudaError_t e) {
     if (e == cudaSuccess) return COLI_OK;
@@ -116,14 +120,25 @@ const char *coli_moe_status_str(coli_status s) {
 
 const char *coli_moe_last_cuda_error(void) { return g_last_cuda_error; }
 
-coli_status coli_moe_record_bytes(int hidden, int inter, int wfmt, size_t *bytes) {
+coli_status coli_moe_debug_set_wait(long long wait_cycles, int unreachable) {
+    if (wait_cycles < 0) return COLI_ERR_INVALID_ARG;
+    g_wait_cycles = wait_cycles;
+    g_unreachable = unreachable != 0;
+    return COLI_OK;
+}
+
+coli_status coli_moe_record_bytes(int hidden, int inter, int wfmt, int group_size, size_t *bytes) {
     if (!bytes) return COLI_ERR_INVALID_ARG;
     if (wfmt != COLI_W_INT4 && wfmt != COLI_W_INT8 && wfmt != COLI_W_INT2) return COLI_ERR_INVALID_ARG;
+    if (group_size != 0 && group_size != 64) return COLI_ERR_INVALID_ARG;
+    if (group_size && wfmt != COLI_W_INT4) return COLI_ERR_UNSUPPORTED;
     if (hidden <= 0 || inter <= 0) return COLI_ERR_SHAPE;
     if ((static_cast<long>(hidden) * wfmt) % 8 || (static_cast<long>(inter) * wfmt) % 8) return COLI_ERR_SHAPE;
+    if (group_size && (hidden % group_size || inter % group_size)) return COLI_ERR_SHAPE;
     const size_t rh = static_cast<size_t>(hidden) * wfmt / 8, ri = static_cast<size_t>(inter) * wfmt / 8;
+    const size_t nh = group_size ? hidden / group_size : 1, ni = group_size ? inter / group_size : 1;
     *bytes = 2 * static_cast<size_t>(inter) * rh + static_cast<size_t>(hidden) * ri +
-             (2 * static_cast<size_t>(inter) + hidden) * sizeof(float);
+             (2 * static_cast<size_t>(inter) * nh + static_cast<size_t>(hidden) * ni) * sizeof(float);
     return COLI_OK;
 }
 
@@ -131,6 +146,8 @@ coli_status coli_moe_check_config(const coli_moe_config *c) {
     if (!c) return COLI_ERR_INVALID_ARG;
     if (c->wfmt != COLI_W_INT4 && c->wfmt != COLI_W_INT8 && c->wfmt != COLI_W_INT2) return COLI_ERR_INVALID_ARG;
     if (c->act != COLI_ACT_F32 && c->act != COLI_ACT_BF16) return COLI_ERR_INVALID_ARG;
+    if (c->group_size != 0 && c->group_size != 64) return COLI_ERR_INVALID_ARG;
+    if (c->group_size && c->wfmt != COLI_W_INT4) return COLI_ERR_UNSUPPORTED;
     if (c->hidden <= 0 || c->inter <= 0 || c->n_experts <= 0 || c->top_k <= 0 || c->n_group <= 0 ||
         c->topk_group <= 0 || c->n_shared < 0)
         return COLI_ERR_SHAPE;
@@ -238,7 +255,7 @@ static coli_status check_weights(const coli_moe_config *c, const coli_moe_weight
     if (need_router && (!w->router_w || !w->router_bias)) return COLI_ERR_INVALID_ARG;
     if (c->n_shared == 1 && !w->shared) return COLI_ERR_INVALID_ARG;
     size_t rb = 0;
-    coli_status s = coli_moe_record_bytes(c->hidden, c->inter, c->wfmt, &rb);
+    coli_status s = coli_moe_record_bytes(c->hidden, c->inter, c->wfmt, c->group_size, &rb);
     if (s != COLI_OK) return s;
     if (w->expert_stride < rb) return COLI_ERR_SHAPE;
     if (w->expert_stride % 256 || !aligned(w->experts, 256)) return COLI_ERR_ALIGN;
@@ -259,9 +276,12 @@ static FfnParams make_params(const coli_moe_config *c, const coli_moe_weights *w
     p.rb_i = static_cast<size_t>(c->inter) * c->wfmt / 8;
     p.off_wu = static_cast<size_t>(c->inter) * p.rb_h;
     p.off_wd = 2 * p.off_wu;
+    p.group = c->group_size;
+    p.nsh = c->group_size ? c->hidden / c->group_size : 1;  // scales per Wg / Wu row
+    p.nsi = c->group_size ? c->inter / c->group_size : 1;   // scales per Wd row
     p.off_sg = p.off_wd + static_cast<size_t>(c->hidden) * p.rb_i;
-    p.off_su = p.off_sg + static_cast<size_t>(c->inter) * 4;
-    p.off_sd = p.off_su + static_cast<size_t>(c->inter) * 4;
+    p.off_su = p.off_sg + static_cast<size_t>(c->inter) * p.nsh * 4;
+    p.off_sd = p.off_su + static_cast<size_t>(c->inter) * p.nsh * 4;
     p.x = x; p.topk_w = topk_w; p.offsets = offsets; p.perm = perm; p.unique = unique;
     p.n_unique = n_unique; p.h = h; p.out = out; p.err = err;
     return p;
@@ -275,8 +295,8 @@ static DecodeParams make_decode(const coli_moe_config *c, const FfnParams &f, ch
     d.TG = c->topk_group;
     d.gbar = reinterpret_cast<unsigned *>(base + WS_GBAR);
     d.gdep = reinterpret_cast<unsigned *>(base + WS_GDEP);
-    d.route_cnt = reinterpret_cast<unsigned *>(base + WS_ROUTE_CNT);
-    d.tok_cnt = reinterpret_cast<unsigned *>(base + WS_TOK_CNT);
+    d.wait_cycles = g_wait_cycles;
+    d.gate_extra = g_unreachable ? 1000000u : 0u;
     return d;
 }
 

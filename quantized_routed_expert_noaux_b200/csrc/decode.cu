@@ -1,29 +1,39 @@
 // decode.cu -- the fused decode path of the layer for a few tokens (decode and MTP verify).
 //
-// One persistent launch, one CTA per SM (ffn_decode_kernel):
+// One persistent cooperative launch, one CTA per SM, one producer warp and 16 consumer warps
+// (ffn_decode_kernel):
 //
-//  phase 0  a1 gate: CTA b computes the logits of experts [b*E/G, (b+1)*E/G) in double from
-//           exact double products and arrives on a grid counter.  After the shared expert's
-//           gate/up rows, every CTA waits for all logits and routes the batch itself (a2,
-//           noaux_tc, colibri-strix README "What's implemented") and groups it (a3, batch-union):
-//           the same code on the same inputs, so all CTAs agree bit for bit; CTA 0 writes the
-//           routing outputs of the call.  (For coli_moe_ffn the routing arrays are inputs.)
-//  phases 1-2 (a4..a7).  Warp 0 streams weight rows
-//                           into a shared-memory ring with bulk asynchronous copies (TMA engine,
-//                           mbarrier completion); the other warps dequantise from the ring.
-//                           Phase 1 (gate/up) splits every expert's I rows evenly over the CTAs
-//                           and writes h = SiLU(g)*u; a grid barrier; phase 2 (down + combine)
-//                           gives every CTA a block of output rows over all experts and sums
-//                           them in registers in a fixed order: no atomics, deterministic.  The
-//                           shared expert comes first, so its rows stream while K1 routes.
+//  start    every consumer thread loads its slice of the activations and of this CTA's router
+//           rows at once.  a1 gate: the CTA's logits (experts [b*E/G, (b+1)*E/G)) are summed in
+//           double from exact double products and published with an arrival on a grid counter.
+//           The activations become 24-bit fixed point per token row (scale 2^(e-22) with
+//           max|x| < 2^e), exact for every bf16 element within 2^15 of the row's maximum, held
+//           as three signed byte slices in the layout of the tensor-core B operand.
+//  phase 1  (a4, and a6 for the shared expert) gate/up rows stream through a shared-memory ring
+//           (bulk asynchronous copies by the producer warp, mbarrier completion).  A tile is 8
+//           gate rows and the same 8 up rows of one expert; two groups of 8 warps take tiles in
+//           turn, each warp a slice of K, with int8 tensor-core MMAs (mma.sync m16n8k32,
+//           int32 accumulation over all of K: exact) of the unpacked codes against every
+//           token's three slices.  A group's partial sums meet in shared memory; one warp
+//           forms g and u per (row, token) and writes h = SiLU(g) * u in float32.  The shared
+//           expert's tiles run first; then every CTA waits for all logits and routes the batch
+//           itself (a2, noaux_tc, colibri-strix README "What's implemented") and groups it (a3,
+//           batch-union): the same code on the same inputs, so all CTAs agree bit for bit; CTA
+//           0 writes the routing outputs of the call.  (For coli_moe_ffn the routing arrays
+//           are inputs.)  Routed tiles are dealt over the CTAs as one flat list.
+//  barrier  bounded grid barrier (every h row complete).
+//  phase 2  (a5, a7) each CTA owns H/G output rows of every expert.  Warp w owns one 64-byte
+//           column chunk of the down rows: it turns its chunk of each slot's h into 24-bit
+//           fixed point per chunk (three byte slices, scale 2^(e-22)), multiplies with the
+//           tensor cores and accumulates w * sd * dot per (row, token) in float registers over
+//           the experts in a fixed order (shared expert first, then the unique ids ascending).
+//           One cross-warp reduction at the end, no atomics: deterministic, and batch-union
+//           output equals per-token output bit for bit.
 //
-// Dequantisation (dequant-on-use, same README section): phase 1 multiplies codes by activations
-// held as 16-bit block fixed point (per 16-byte chunk of codes, one power-of-two scale) with
-// dp2a integer dot products, exact in int32; the activation is exact for every element within a
-// factor 2^7 of its chunk's largest magnitude (bf16 has 8 significant bits), smaller elements are
-// rounded to 2^-15 of that maximum.  Phase 2 takes h as 16-bit fixed point per chunk split in two
-// signed bytes and the codes as signed bytes (16q for int4, 64q for int2), so dp4a integer dot
-// products are exact; h is rounded to 2^-16 of its chunk's largest magnitude.
+// Dequantisation (dequant-on-use, same README section): the codes enter the MMA as signed
+// bytes scaled by a power of two (the int4 nibble in the high half of a byte is 16q, an int2
+// field in the top two bits 64q); the row scale and the activation scale are applied once per
+// dot product in the epilogue.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -38,11 +48,13 @@ constexpr unsigned FULL = 0xffffffffu;
 constexpr int NCW = 16;              // consumer warps
 constexpr int NC = NCW * 32;         // consumer threads
 constexpr int NT = NC + 32;          // + producer warp
-constexpr int PS1 = 8;               // (gate, up) row pairs per phase-1 stage
-constexpr int RPT2MAX = 8;           // phase-2 rows per thread over the whole CTA row range
-constexpr int CONS_BAR = 1;          // named barrier id of the consumer warps (2..5: per-token routing)
-// routing cache in shared memory (int offsets): U | unique[32] | beg[33] | cnt[33] | tok[32] | w[32] | hrow[32] | sorted slots[32]
-constexpr int RT_UNIQ = 1, RT_BEG = 33, RT_CNT = 66, RT_TOK = 99, RT_W = 131, RT_H = 163, RT_SORT = 195;
+constexpr int GW = 8;                // warps of a phase-1 group
+constexpr int NGRP = NCW / GW;       // phase-1 groups
+constexpr int MAXTOK = 4;            // tokens of the fused path
+constexpr int MAXWE = 33;            // work experts: the shared one + up to 32 unique routed
+constexpr int ROWPAD = 64;           // bytes added to each staged row (conflict-free 16-byte loads)
+// named barriers: 0 __syncthreads, 1 all consumers, 2.. group full, 4.. group reduction free
+constexpr int BAR_CONS = 1, BAR_GFULL = 2, BAR_GFREE = 4;
 constexpr long long WAIT_CYCLES = 4000000000LL;  // ~2 s at 1.9 GHz: bound of every spin-wait
 
 // ------------------------------------------------------------------------- PTX helpers -----
@@ -58,8 +70,7 @@ __device__ __forceinline__ void mbar_arrive(uint32_t a) {
 __device__ __forceinline__ void mbar_expect_tx(uint32_t a, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(a), "r"(bytes) : "memory");
 }
-// try_wait with a suspend-time hint (ns): a waiting warp sleeps instead of spinning, leaving
-// issue slots to the warps that compute; it is woken when the phase completes.
+// try_wait with a suspend-time hint (ns): a waiting warp sleeps instead of spinning.
 __device__ __forceinline__ bool mbar_try(uint32_t a, uint32_t parity) {
     uint32_t ok;
     asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
@@ -67,11 +78,11 @@ __device__ __forceinline__ bool mbar_try(uint32_t a, uint32_t parity) {
     return ok != 0;
 }
 // Bounded wait: false when the bound ran out (the caller records the error and gives up).
-__device__ __forceinline__ bool mbar_wait(uint32_t a, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait(uint32_t a, uint32_t parity, long long bound) {
     if (mbar_try(a, parity)) return true;
     const long long t0 = clock64();
     while (!mbar_try(a, parity)) {
-        if (clock64() - t0 > WAIT_CYCLES) return false;
+        if (clock64() - t0 > bound) return false;
     }
     return true;
 }
@@ -80,283 +91,213 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
                  ::"r"(dst), "l"(src), "r"(bytes), "r"(mbar), "l"(policy) : "memory");
 }
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ uint64_t evict_first_policy() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
     return p;
 }
-__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void cons_sync() { asm volatile("bar.sync %0, %1;" ::"n"(CONS_BAR), "n"(NC) : "memory"); }
+__device__ __forceinline__ uint64_t evict_last_policy() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
 __device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
-__device__ __forceinline__ uint4 lds128(const unsigned char *p) { return *reinterpret_cast<const uint4 *>(p); }
+__device__ __forceinline__ void named_arrive(int id, int n) { asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+__device__ __forceinline__ void cons_sync() { named_sync(BAR_CONS, NC); }
 __device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
     unsigned v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
-__device__ __forceinline__ float4 ldcg4(const float *p) {
-    return __ldcg(reinterpret_cast<const float4 *>(p));
-}
 
+// D (16x8 int32) += A (16x32 int8) * B (32x8 int8).  Fragments (thread = 4 * group + tig):
+// a0 / a2 row `group`, a1 / a3 row `group + 8`; a0, a1 hold k = 4 tig + j, a2, a3 hold
+// k = 16 + 4 tig + j (byte j); b0 / b1 hold the same k of column `group`; d0, d1 row `group`
+// columns 2 tig, 2 tig + 1; d2, d3 row `group + 8`.
+__device__ __forceinline__ void mma_s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                       uint32_t b0, uint32_t b1) {
+    asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                 : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
 
 // ------------------------------------------------------------------------- code formats ----
-// Codes per 16-byte chunk: int4 32, int8 16, int2 64.
-template <int FMT> struct Fmt { static constexpr int CPC = 128 / FMT; };
-
-// Integer dot of one 16-byte chunk of codes with its activation chunk (16-bit pairs laid out by
-// prepare_x below).  Returns sum_j q_j * m_j exactly.
-template <int FMT>
-__device__ __forceinline__ int idot_chunk(const uint4 q, const int *xp, int corr);
-
-template <>
-__device__ __forceinline__ int idot_chunk<4>(const uint4 q, const int *xp, int corr) {
-    // u = q + 8 per nibble (flip of the sign bit); bytes of lo hold elements 0,2,4,6 of a word,
-    // bytes of hi hold 1,3,5,7.  xp holds per word: (m0,m2) (m4,m6) (m1,m3) (m5,m7).
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-    int a0 = -corr, a1 = 0, a2 = 0, a3 = 0;  // corr = 8 * sum(m); four independent chains
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t f = w[i] ^ 0x88888888u;
-        const uint32_t lo = f & 0x0F0F0F0Fu;
-        const uint32_t hi = (f >> 4) & 0x0F0F0F0Fu;
-        a0 = __dp2a_lo(xp[4 * i + 0], static_cast<int>(lo), a0);
-        a1 = __dp2a_hi(xp[4 * i + 1], static_cast<int>(lo), a1);
-        a2 = __dp2a_lo(xp[4 * i + 2], static_cast<int>(hi), a2);
-        a3 = __dp2a_hi(xp[4 * i + 3], static_cast<int>(hi), a3);
+// A 64-byte chunk of a row holds CPC codes; each of the 4 threads of a quad loads 16 bytes of
+// it and feeds MPC MMAs (k = 32 each).  The codes become signed bytes MUL * q.  Inside a chunk,
+// MMA m, thread tig, A register a0 byte j holds code pos0(tig, m, j) and a2 byte j code
+// pos0 + OFS2 (the B slices follow the same positions, so the dot products are unchanged).
+template <int FMT> struct Fmt;
+template <> struct Fmt<4> {
+    static constexpr int CPC = 128, MPC = 4, MUL = 16;
+    // word m of a thread's 16 bytes holds codes 32 tig + 8 m + (0..7); even codes -> a0, odd -> a2
+    __device__ static __forceinline__ void unpack(const uint4 q, int m, uint32_t &lo, uint32_t &hi) {
+        const uint32_t w = m == 0 ? q.x : (m == 1 ? q.y : (m == 2 ? q.z : q.w));
+        lo = (w << 4) & 0xF0F0F0F0u;
+        hi = w & 0xF0F0F0F0u;
     }
-    return (a0 + a1) + (a2 + a3);
-}
-template <>
-__device__ __forceinline__ int idot_chunk<8>(const uint4 q, const int *xp, int) {
-    // signed bytes in natural order; xp holds (m0,m1) (m2,m3) per word
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-    int a0 = 0, a1 = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        a0 = __dp2a_lo(xp[2 * i + 0], static_cast<int>(w[i]), a0);
-        a1 = __dp2a_hi(xp[2 * i + 1], static_cast<int>(w[i]), a1);
+    // element p of a chunk -> (tig, m, half, byte)
+    __device__ static __forceinline__ void place(int p, int &tig, int &m, int &half, int &byte) {
+        tig = p >> 5;
+        m = (p >> 3) & 3;
+        byte = (p >> 1) & 3;
+        half = p & 1;
     }
-    return a0 + a1;
-}
-template <>
-__device__ __forceinline__ int idot_chunk<2>(const uint4 q, const int *xp, int corr) {
-    // u = q + 2 per 2-bit field; extraction k gives bytes with elements 4j+k (j = byte);
-    // xp holds per word and k: (m_k, m_{4+k}) (m_{8+k}, m_{12+k}).
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-    int a[4] = {-corr, 0, 0, 0};  // corr = 2 * sum(m)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint32_t f = w[i] ^ 0xAAAAAAAAu;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const uint32_t b = (f >> (2 * k)) & 0x03030303u;
-            a[k] = __dp2a_lo(xp[8 * i + 2 * k + 0], static_cast<int>(b), a[k]);
-            a[k] = __dp2a_hi(xp[8 * i + 2 * k + 1], static_cast<int>(b), a[k]);
-        }
-    }
-    return (a[0] + a[1]) + (a[2] + a[3]);
-}
-
-// Phase 2 activations (h) as 16-bit fixed point per chunk, X = rint(h * 32512 / max|h|), split
-// X = 256 * Xh + Xl into two signed bytes; the codes become signed bytes scaled by a power of
-// two (the int4 nibble in the high half of a byte is 16q, an int2 field in the top two bits is
-// 64q), so one dp4a takes four products of each part exactly.  Slice word order follows the
-// byte extraction below (h_slot).  Returns the two exact integer sums.
-template <int FMT> struct Ph2 {
-    static constexpr int MUL = FMT == 4 ? 16 : (FMT == 2 ? 64 : 1);  // code byte = MUL * q
-    static constexpr int XW8 = Fmt<FMT>::CPC / 4;                    // int8x4 words per chunk and part
-    static constexpr int XV8 = XW8 / 4;                              // int4 vectors per chunk and part
 };
+template <> struct Fmt<2> {
+    static constexpr int CPC = 256, MPC = 8, MUL = 64;
+    // word i of a thread's 16 bytes holds codes 64 tig + 16 i + 4 j + k (byte j, field k); MMA
+    // 2i takes fields 0 (a0) and 1 (a2), MMA 2i + 1 fields 2 and 3
+    __device__ static __forceinline__ void unpack(const uint4 q, int m, uint32_t &lo, uint32_t &hi) {
+        const int i = m >> 1;
+        const uint32_t w = i == 0 ? q.x : (i == 1 ? q.y : (i == 2 ? q.z : q.w));
+        const int k0 = 2 * (m & 1);
+        lo = (w << (6 - 2 * k0)) & 0xC0C0C0C0u;
+        hi = (w << (4 - 2 * k0)) & 0xC0C0C0C0u;
+    }
+    __device__ static __forceinline__ void place(int p, int &tig, int &m, int &half, int &byte) {
+        tig = p >> 6;
+        const int i = (p >> 4) & 3, k = p & 3;
+        m = 2 * i + (k >> 1);
+        half = k & 1;
+        byte = (p >> 2) & 3;
+    }
+};
+
+// The group-scaled container (scales per 64 consecutive codes, int4) keeps every MMA inside one
+// group: MMA m of a chunk takes codes [32 m, 32 m + 32), thread tig the 8 codes 32 m + 8 tig +
+// (0..7) (word m of its A registers, read from byte 16 m + 4 tig); MMAs 2u and 2u + 1 are group
+// u of the chunk.  With per-row scales a thread reads one 16-byte run instead (Fmt::place).
+template <int FMT, int GS> struct Place {
+    __device__ static __forceinline__ void at(int p, int &tig, int &m, int &half, int &byte) {
+        Fmt<FMT>::place(p, tig, m, half, byte);
+    }
+    // the thread's 16 bytes of A for a 64-byte chunk starting at `chunk`
+    __device__ static __forceinline__ uint4 load_a(const unsigned char *chunk, int tig) {
+        return *reinterpret_cast<const uint4 *>(chunk + 16 * tig);
+    }
+};
+template <> struct Place<4, 64> {
+    __device__ static __forceinline__ void at(int p, int &tig, int &m, int &half, int &byte) {
+        m = p >> 5;
+        tig = (p >> 3) & 3;
+        byte = (p >> 1) & 3;
+        half = p & 1;
+    }
+    __device__ static __forceinline__ uint4 load_a(const unsigned char *chunk, int tig) {
+        const uint32_t *w = reinterpret_cast<const uint32_t *>(chunk + 4 * tig);
+        return make_uint4(w[0], w[4], w[8], w[12]);
+    }
+};
+
+// Byte offset, inside one column's block of a chunk (4 tig x 8 MPC bytes), of B byte `byte` of
+// register `half` of MMA m for thread tig.  16-byte units are permuted per column so that the
+// 8 threads of a quarter warp (two columns x four tig) read 8 distinct bank groups.
 template <int FMT>
-__device__ __forceinline__ void idot4_chunk(const uint4 q, const int *xh, const int *xl, int &sh, int &sl);
-
-template <>
-__device__ __forceinline__ void idot4_chunk<4>(const uint4 q, const int *xh, const int *xl, int &sh, int &sl) {
-    // word i (codes 8i..8i+7): (w << 4) & 0xF0F0F0F0 holds codes 0,2,4,6, w & 0xF0F0F0F0 codes 1,3,5,7
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-    int h0 = 0, h1 = 0, l0 = 0, l1 = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int ev = static_cast<int>((w[i] << 4) & 0xF0F0F0F0u);
-        const int od = static_cast<int>(w[i] & 0xF0F0F0F0u);
-        h0 = __dp4a(ev, xh[2 * i], h0);
-        l0 = __dp4a(ev, xl[2 * i], l0);
-        h1 = __dp4a(od, xh[2 * i + 1], h1);
-        l1 = __dp4a(od, xl[2 * i + 1], l1);
-    }
-    sh = h0 + h1;
-    sl = l0 + l1;
+__device__ __forceinline__ int b_off(int col, int tig, int m, int half, int byte) {
+    constexpr int MPC = Fmt<FMT>::MPC;
+    const int u = m >> 1;  // 16-byte unit of the thread's 8 MPC bytes
+    int su;
+    if (MPC == 4) su = u ^ (col & 1);
+    else su = u ^ (tig >> 1) ^ ((col & 1) << 1);
+    return tig * 8 * MPC + su * 16 + (m & 1) * 8 + half * 4 + byte;
 }
-template <>
-__device__ __forceinline__ void idot4_chunk<8>(const uint4 q, const int *xh, const int *xl, int &sh, int &sl) {
-    // signed bytes in natural order
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-    int h0 = 0, h1 = 0, l0 = 0, l1 = 0;
-#pragma unroll
-    for (int i = 0; i < 4; i += 2) {
-        h0 = __dp4a(static_cast<int>(w[i]), xh[i], h0);
-        l0 = __dp4a(static_cast<int>(w[i]), xl[i], l0);
-        h1 = __dp4a(static_cast<int>(w[i + 1]), xh[i + 1], h1);
-        l1 = __dp4a(static_cast<int>(w[i + 1]), xl[i + 1], l1);
-    }
-    sh = h0 + h1;
-    sl = l0 + l1;
-}
-template <>
-__device__ __forceinline__ void idot4_chunk<2>(const uint4 q, const int *xh, const int *xl, int &sh, int &sl) {
-    // word i (codes 16i..16i+15): (w << (6 - 2k)) & 0xC0C0C0C0 holds codes k, 4+k, 8+k, 12+k
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-    int h[2] = {0, 0}, l[2] = {0, 0};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int bb = static_cast<int>((w[i] << (6 - 2 * k)) & 0xC0C0C0C0u);
-            h[k & 1] = __dp4a(bb, xh[4 * i + k], h[k & 1]);
-            l[k & 1] = __dp4a(bb, xl[4 * i + k], l[k & 1]);
-        }
-    }
-    sh = h[0] + h[1];
-    sl = l[0] + l[1];
-}
-
-// Position of chunk element j in the chunk's int8x4 slice layout (word, byte), matching
-// idot4_chunk.
+// The thread's B registers of one chunk for MMAs 2u and 2u + 1 (one 16-byte unit): b0, b1 of
+// MMA 2u, then b0, b1 of MMA 2u + 1.
 template <int FMT>
-__device__ __forceinline__ void h_slot(int j, int &word, int &byte) {
-    if (FMT == 4) {
-        const int i = j >> 3, k = j & 7;
-        word = 2 * i + (k & 1);
-        byte = k >> 1;
-    } else if (FMT == 8) {
-        word = j >> 2;
-        byte = j & 3;
-    } else {
-        const int i = j >> 4, k = j & 15;
-        word = 4 * i + (k & 3);
-        byte = k >> 2;
-    }
+__device__ __forceinline__ uint4 load_b2(const unsigned char *colblk, int col, int tig, int u) {
+    return *reinterpret_cast<const uint4 *>(colblk + b_off<FMT>(col, tig, 2 * u, 0, 0));
 }
 
-__device__ __forceinline__ float warp_allsum(float v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
-    return v;
+// Three signed byte slices of a 24-bit fixed-point value: X = 65536 s2 + 256 s1 + s0.
+__device__ __forceinline__ void slices3(int X, int &s0, int &s1, int &s2) {
+    s0 = static_cast<int>(static_cast<int8_t>(X & 0xff));
+    const int r = (X - s0) >> 8;
+    s1 = static_cast<int>(static_cast<int8_t>(r & 0xff));
+    s2 = (r - s1) >> 8;
 }
 
-// ------------------------------------------------------------------------- K1 router -------
+// ------------------------------------------------------------------------- routing ---------
 __device__ __forceinline__ bool beats(double va, int ia, double vb, int ib) {
     return va > vb || (va == vb && ia < ib);
 }
 
-constexpr int RMAX_BLOCKS = 8;  // E <= 256 on the fused path
-struct RouteSmem {
-    double btop1[RMAX_BLOCKS], btop2[RMAX_BLOCKS];
-    double cval[RMAX_BLOCKS * 8], cs[RMAX_BLOCKS * 8];  // per block: its K <= 8 best
-    int cid[RMAX_BLOCKS * 8];
-    double sel_s[32];
-    int sel_id[32];
-    int out_id[8];
-    float out_w[8];
+constexpr int RMAX_BLOCKS = 8;  // E <= 256 on the fused path: blocks of 32 experts
+struct RouteToken {             // per token, shared memory
+    double cval[RMAX_BLOCKS][8], cs[RMAX_BLOCKS][8];  // per block: its best max(K, 2) experts
+    int cid[RMAX_BLOCKS][8];
+    double sel_s[8];
+    int sel_id[8];
+};
+struct RouteCache {             // the routing of the call, shared memory
+    int U;                      // unique routed experts
+    int uniq[32];               // their ids, ascending
+    int slot[MAXWE][MAXTOK];    // h row of (work expert, token), -1 when not routed
+    float wgt[MAXWE][MAXTOK];   // combine weight of (work expert, token), 0 when not routed
+    int ids[MAXTOK][8];         // per token: selected ids, slot order
+    float w[MAXTOK][8];         //            and weights
+    int sorted[32];             // grouped order of the slots
+    float xscale[MAXTOK];       // activation scale of each token row, 2^(e - 22)
+    int err;
 };
 
-// Route token t with four consumer warps (w4 = warp index within the four, barrier id bar).
-// Experts are taken in blocks of 32 (one per lane); a group is a whole number of blocks (or
-// G = 1).  Per block: the two largest biased scores (group score) and the block's K best experts
-// by rank among its 32 lanes; warp w4 handles blocks w4, w4 + 4 together so that their loads,
-// sigmoids and shuffles overlap.  Warp 0 then ranks the groups, takes the kept blocks' K best
-// (at most 32 candidates, one per lane) and ranks them.  Selections, ties and weights are those
-// of the per-token definition (largest biased score, lower id on ties, weights from the
-// unbiased scores renormalised in slot order, times routed_scaling).  Writes the token's ids and
-// weights into r.
-__device__ void route_token(const DecodeParams &p, int t, int w4, int lane, int bar, RouteSmem &r) {
-    const int E = p.f.E, K = p.f.K, G = p.G, TG = p.TG;
-    const int gs = E / G, nb = E / 32, bpg = gs / 32;
-    const bool grouped = G > 1 && TG < G;
-    constexpr int BPW = RMAX_BLOCKS / 4;  // blocks per warp
-    double c[BPW], s[BPW];
-    float lf[BPW], bf[BPW];
-#pragma unroll
-    for (int j = 0; j < BPW; ++j) {
-        const int e = (w4 + 4 * j) * 32 + lane;
-        const bool on = w4 + 4 * j < nb;
-        lf[j] = on ? __ldcg(p.logits + static_cast<size_t>(t) * E + e) : 0.f;
-        bf[j] = on ? __ldg(p.bias + e) : 0.f;
-    }
-#pragma unroll
-    for (int j = 0; j < BPW; ++j) {
-        s[j] = 1.0 / (1.0 + exp(-static_cast<double>(lf[j])));
-        c[j] = s[j] + static_cast<double>(bf[j]);
-    }
-    if (grouped) {
-        double a1[BPW], a2[BPW];
-#pragma unroll
-        for (int j = 0; j < BPW; ++j) { a1[j] = c[j]; a2[j] = -INFINITY; }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-#pragma unroll
-            for (int j = 0; j < BPW; ++j) {
-                const double b1 = __shfl_xor_sync(FULL, a1[j], o);
-                const double b2 = __shfl_xor_sync(FULL, a2[j], o);
-                const double n1 = fmax(a1[j], b1);
-                const double n2 = fmax(fmin(a1[j], b1), fmax(a2[j], b2));
-                a1[j] = n1; a2[j] = n2;
-            }
-        }
-        if (lane == 0) {
-#pragma unroll
-            for (int j = 0; j < BPW; ++j)
-                if (w4 + 4 * j < nb) { r.btop1[w4 + 4 * j] = a1[j]; r.btop2[w4 + 4 * j] = a2[j]; }
-        }
-    }
-    int rank[BPW];
-#pragma unroll
-    for (int j = 0; j < BPW; ++j) rank[j] = 0;
+// Step A: the best max(K, 2) of one 32-expert block of token t (lane = expert in the block).
+__device__ void route_block(const DecodeParams &p, int t, int blk, int lane, RouteToken &r) {
+    const int E = p.f.E, K = p.f.K;
+    const int e = blk * 32 + lane;
+    const float lf = __ldcg(p.logits + static_cast<size_t>(t) * E + e);
+    const float bf = __ldg(p.bias + e);
+    const double s = 1.0 / (1.0 + exp(-static_cast<double>(lf)));
+    const double c = s + static_cast<double>(bf);
+    int rank = 0;
 #pragma unroll
     for (int o = 0; o < 32; ++o) {
-#pragma unroll
-        for (int j = 0; j < BPW; ++j) {
-            const double oc = __shfl_sync(FULL, c[j], o);
-            rank[j] += (oc > c[j] || (oc == c[j] && o < lane)) ? 1 : 0;  // same block: id order = lane order
-        }
+        const double oc = __shfl_sync(FULL, c, o);
+        rank += (oc > c || (oc == c && o < lane)) ? 1 : 0;  // same block: id order = lane order
     }
-#pragma unroll
-    for (int j = 0; j < BPW; ++j) {
-        const int bk = w4 + 4 * j;
-        if (bk < nb && rank[j] < K) {
-            r.cval[bk * K + rank[j]] = c[j];
-            r.cs[bk * K + rank[j]] = s[j];
-            r.cid[bk * K + rank[j]] = bk * 32 + lane;
-        }
+    const int keep = K > 2 ? K : 2;
+    if (rank < keep) {
+        r.cval[blk][rank] = c;
+        r.cs[blk][rank] = s;
+        r.cid[blk][rank] = e;
     }
-    named_sync(bar, 128);
-    if (w4 != 0) return;
-    // kept blocks: all, or those of the TG best groups (group g = lane)
+}
+
+// Step B: group stage, selection and weights of token t (one warp).  Selections, ties and
+// weights are those of the per-token definition: largest biased score first, lower id on
+// ties; groups score the sum of their two largest biased scores, lower group on ties; weights
+// from the unbiased scores renormalised in slot order, times routed_scaling.
+__device__ void route_select(const DecodeParams &p, int t, int lane, RouteToken &r, RouteCache &rc) {
+    const int E = p.f.E, K = p.f.K, G = p.G, TG = p.TG;
+    const int nb = E / 32;
+    const bool grouped = G > 1 && TG < G;
     unsigned kmask;
     if (grouped) {
+        const int bpg = (E / G) / 32;
         double gsc = -INFINITY;
         if (lane < G) {
             double a1 = -INFINITY, a2 = -INFINITY;
             for (int bk = lane * bpg; bk < (lane + 1) * bpg; ++bk) {
-                const double v[2] = {r.btop1[bk], r.btop2[bk]};
 #pragma unroll
                 for (int k = 0; k < 2; ++k) {
-                    if (v[k] > a1) { a2 = a1; a1 = v[k]; }
-                    else if (v[k] > a2) { a2 = v[k]; }
+                    const double v = r.cval[bk][k];
+                    if (v > a1) { a2 = a1; a1 = v; }
+                    else if (v > a2) { a2 = v; }
                 }
             }
             gsc = a1 + a2;
         }
         int rk = 0;
-#pragma unroll
-        for (int o = 0; o < 32; ++o) {
+        for (int o = 0; o < G; ++o) {
             const double og = __shfl_sync(FULL, gsc, o);
-            rk += (o < G && (og > gsc || (og == gsc && o < lane))) ? 1 : 0;
+            rk += (og > gsc || (og == gsc && o < lane)) ? 1 : 0;
         }
         const unsigned gmask = __ballot_sync(FULL, lane < G && rk < TG);
-        kmask = __ballot_sync(FULL, lane < nb && ((gmask >> ((lane * 32) / gs)) & 1u));
+        kmask = __ballot_sync(FULL, lane < nb && ((gmask >> (lane / bpg)) & 1u));
     } else {
-        kmask = __ballot_sync(FULL, lane < nb);
+        kmask = nb >= 32 ? FULL : ((1u << nb) - 1u);
     }
     // candidate of this lane: rank k of the kb-th kept block
     double c2 = -INFINITY, s2 = 0.0;
@@ -366,9 +307,9 @@ __device__ void route_token(const DecodeParams &p, int t, int w4, int lane, int 
         unsigned m = kmask;
         for (int i = 0; i < kb; ++i) m &= m - 1u;  // drop the kb lowest kept blocks
         const int bk = __ffs(m) - 1;
-        c2 = r.cval[bk * K + k];
-        s2 = r.cs[bk * K + k];
-        id = r.cid[bk * K + k];
+        c2 = r.cval[bk][k];
+        s2 = r.cs[bk][k];
+        id = r.cid[bk][k];
     }
     int rank2 = 0;
 #pragma unroll
@@ -382,51 +323,61 @@ __device__ void route_token(const DecodeParams &p, int t, int w4, int lane, int 
     if (lane < K) {
         double denom = 0.0;
         for (int k = 0; k < K; ++k) denom += r.sel_s[k];
-        r.out_id[lane] = r.sel_id[lane];
-        r.out_w[lane] = static_cast<float>((r.sel_s[lane] / denom) * p.rsf);
+        rc.ids[t][lane] = r.sel_id[lane];
+        rc.w[t][lane] = static_cast<float>((r.sel_s[lane] / denom) * p.rsf);
     }
 }
 
-// ------------------------------------------------------------------------- K2 FFN ----------
-// Phase 1: a stage holds PS (gate row, up row) pairs of one expert; consumer warp w works on pair
-// w % PS of the stages whose sequence number is w / PS modulo NCW / PS, reduces its rows with
-// shuffles and writes h itself.  Every consumer warp waits on every stage's full barrier and
-// arrives on its empty barrier (count NCW), so a stage is refilled only after all its readers
-// are done.  Phase 2: a stage holds the CTA's whole block of down rows of one expert; consumer
-// thread (p2, c2) owns chunk c2 of rows p2 + P2*m and keeps per-(row, token) partial sums in
-// registers across experts; one cross-lane reduction at the end.
-template <int FMT, int TMAX, int NJ>
-__global__ void __maxnreg__(96) ffn_decode_kernel(DecodeParams p) {
-    constexpr int CPC = Fmt<FMT>::CPC;       // codes per 16-byte chunk
-    constexpr int XW = CPC / 2;              // int32 words of 16-bit activations per chunk
-    constexpr int XV = XW / 4;               // int4 vectors per chunk
+// ------------------------------------------------------------------------- the kernel ------
+// Shared-memory regions (byte offsets from the plan): barriers | routing cache | per-token
+// routing scratch | activation slices (phase 1) aliased with h slices and the final reduction
+// (phase 2) | group reduction buffers | gate partials | ring.
+template <int FMT, int TT, int GI, int GS>
+__global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
+    using F = Fmt<FMT>;
+    using PL = Place<FMT, GS>;
+    constexpr int CPC = F::CPC, MPC = F::MPC;
+    constexpr int MAXT = TT;                          // tokens of this instantiation (T <= TT)
+    constexpr int NB = (3 * TT + 7) / 8;              // 8-column MMA blocks (3 slices per token)
     extern __shared__ __align__(1024) unsigned char sm[];
     const FfnParams &f = p.f;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = gridDim.x, b = blockIdx.x;
-    const int S = p.S;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm);          // full[S], empty[S]
-    int *rt = reinterpret_cast<int *>(sm + p.off_route);         // routing cache
-    int4 *xq = reinterpret_cast<int4 *>(sm + p.off_x);            // [T][XV][Lh] (transposed)
-    float *xs = reinterpret_cast<float *>(sm + p.off_xs);         // [T][Lh] scale
-    int *xc = reinterpret_cast<int *>(sm + p.off_xc);             // [T][Lh] correction
-    float *red2 = reinterpret_cast<float *>(sm + p.off_red);      // phase-2 partials
+    const int T = f.T, S = p.S;
+    const long long bound = p.wait_cycles;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm);
+    RouteCache &rc = *reinterpret_cast<RouteCache *>(sm + p.off_route);
+    RouteToken *rtok = reinterpret_cast<RouteToken *>(sm + p.off_rtok);
+    unsigned char *xb = sm + p.off_x;                  // activation slices, B layout
+    int4 *red1 = reinterpret_cast<int4 *>(sm + p.off_red1);
+    double *gpart = reinterpret_cast<double *>(sm + p.off_gate);
     unsigned char *ring = sm + p.off_ring;
     const uint32_t bar0 = smem_u32(bars);
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
     const uint32_t route_bar = bar0 + 8u * (2 * S);  // consumers -> producer: routing cache ready
-    const int Lh = p.Lh, Li = p.Li;
-    const int PS = p.R1;                     // pairs per phase-1 stage
 
-    const int i_lo = static_cast<int>(static_cast<long>(f.I) * b / G), i_hi = static_cast<int>(static_cast<long>(f.I) * (b + 1) / G);
+    // geometry
+    const int rb_h = static_cast<int>(f.rb_h), rb_i = static_cast<int>(f.rb_i);
+    const int SK1 = p.SK1, nks1 = rb_h / SK1;          // phase-1 stage: 16 rows x SK1 bytes
+    const int SK2 = p.SK2, nks2 = rb_i / SK2;          // phase-2 stage: nrows x SK2 bytes
+    // staged row strides: 64 bytes of padding for 16-byte A loads, 16 for 4-byte ones
+    constexpr int PAD = GS ? 16 : ROWPAD;
+    const int st1 = SK1 + PAD, st2 = SK2 + PAD;
+    const int gps1 = GS ? SK1 * 8 / FMT / GS : 0;     // scale groups per row of a phase-1 stage
+    const int gps2 = GS ? SK2 * 8 / FMT / GS : 0;     // and of a phase-2 stage
+    const int NRB = f.I / 8;                           // tiles (8 row pairs) per expert
     const int j_lo = static_cast<int>(static_cast<long>(f.H) * b / G), j_hi = static_cast<int>(static_cast<long>(f.H) * (b + 1) / G);
-    const int n1 = (i_hi - i_lo + PS - 1) / PS;  // phase-1 stages per expert
+    const int nrows = j_hi - j_lo;
+    const int a0d = j_lo & ~3;
+    const int sh_lo = f.S ? static_cast<int>(static_cast<long>(NRB) * b / G) : 0;
+    const int sh_hi = f.S ? static_cast<int>(static_cast<long>(NRB) * (b + 1) / G) : 0;
+    const int nsh = sh_hi - sh_lo;                     // shared-expert tiles of this CTA
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(full_bar(s), 1);
-            mbar_init(empty_bar(s), NCW);
+            mbar_init(empty_bar(s), GW);               // every stage is read by 8 warps
         }
         mbar_init(route_bar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -437,384 +388,474 @@ __global__ void __maxnreg__(96) ffn_decode_kernel(DecodeParams p) {
         // ---------------------------------------------------------------- producer --------
         if (lane != 0) return;
         const uint64_t pol = evict_first_policy();
+        const uint64_t keep = evict_last_policy();
         int seq = 0, U = 0;
-        int uniq[32] = {0};
-        bool have_routing = false, ok = true;
+        bool ok = true;
         auto record = [&](int we) -> const uint8_t * {
             if (we < f.S) return f.shared;
-            const int e = uniq[we - f.S];
+            const int e = rc.uniq[we - f.S];
             return (e >= 0 && e < f.E) ? f.experts + static_cast<size_t>(e) * f.stride : nullptr;
         };
-        for (int we = 0; ok; ++we) {
-            if (we >= f.S && !have_routing) {
-                if (!mbar_wait(route_bar, 0)) { ok = false; break; }
-                const int *rtc = reinterpret_cast<const int *>(sm + p.off_route);
-                U = rtc[0];
-                for (int u = 0; u < U; ++u) uniq[u] = rtc[RT_UNIQ + u];
-                have_routing = true;
-            }
-            if (have_routing && we >= f.S + U) break;
-            const uint8_t *rec = record(we);
-            for (int k = 0; k < n1 && ok; ++k, ++seq) {
+        auto stage1 = [&](const uint8_t *rec, int rb) {
+            const int r0 = rb * 8;
+            for (int part = 0; part < nks1 && ok; ++part, ++seq) {
                 const int s = seq % S;
                 const uint32_t par = (seq / S) & 1;
-                if (!mbar_wait(empty_bar(s), par ^ 1)) { ok = false; break; }
-                const int r0 = i_lo + k * PS, n = min(PS, i_hi - r0);
-                const uint32_t dst = smem_u32(ring + static_cast<size_t>(s) * p.SB);
+                if (!mbar_wait(empty_bar(s), par ^ 1, bound)) { ok = false; break; }
                 if (rec == nullptr) { mbar_arrive(full_bar(s)); continue; }
-                const int a0 = r0 & ~3, a1 = (r0 + n + 3) & ~3;
-                const uint32_t bytes = 2u * n * static_cast<uint32_t>(f.rb_h) + 2u * 4u * (a1 - a0);
+                const uint32_t dst = smem_u32(ring + static_cast<size_t>(s) * p.SB);
+                const uint32_t bytes = 16u * SK1 + (GS ? 16u * 4u * gps1 : (part == 0 ? 64u : 0u));
                 mbar_expect_tx(full_bar(s), bytes);
-                bulk_g2s(dst, rec + static_cast<size_t>(r0) * f.rb_h, n * f.rb_h, full_bar(s), pol);
-                bulk_g2s(dst + p.st_up, rec + f.off_wu + static_cast<size_t>(r0) * f.rb_h, n * f.rb_h, full_bar(s), pol);
-                bulk_g2s(dst + p.st_sg, rec + f.off_sg + 4 * a0, 4 * (a1 - a0), full_bar(s), pol);
-                bulk_g2s(dst + p.st_su, rec + f.off_su + 4 * a0, 4 * (a1 - a0), full_bar(s), pol);
+                for (int r = 0; r < 8; ++r) {
+                    const size_t src = static_cast<size_t>(r0 + r) * rb_h + static_cast<size_t>(part) * SK1;
+                    bulk_g2s(dst + r * st1, rec + src, SK1, full_bar(s), pol);
+                    bulk_g2s(dst + (8 + r) * st1, rec + f.off_wu + src, SK1, full_bar(s), pol);
+                }
+                if (GS) {  // this part's group scales: gate rows, then up rows, gps1 each
+                    for (int r = 0; r < 8; ++r) {
+                        const size_t g0 = (static_cast<size_t>(r0 + r) * f.nsh + static_cast<size_t>(part) * gps1) * 4;
+                        bulk_g2s(dst + 16 * st1 + r * 4 * gps1, rec + f.off_sg + g0, 4 * gps1, full_bar(s), pol);
+                        bulk_g2s(dst + 16 * st1 + (8 + r) * 4 * gps1, rec + f.off_su + g0, 4 * gps1, full_bar(s), pol);
+                    }
+                } else if (part == 0) {
+                    bulk_g2s(dst + 16 * st1, rec + f.off_sg + 4 * r0, 32, full_bar(s), pol);
+                    bulk_g2s(dst + 16 * st1 + 32, rec + f.off_su + 4 * r0, 32, full_bar(s), pol);
+                }
+            }
+        };
+        // phase 1: the shared expert's tiles, then (once routed) the flat list of routed tiles
+        for (int l = 0; l < nsh && ok; ++l) stage1(f.shared, sh_lo + l);
+        if (f.S && ok) {  // the shared expert's down rows go to L2 while the batch is routed
+            for (int part = 0; part < nks2; ++part)
+                for (int r = 0; r < nrows; ++r)
+                    bulk_prefetch_l2(f.shared + f.off_wd + static_cast<size_t>(j_lo + r) * rb_i + static_cast<size_t>(part) * SK2, SK2);
+        }
+        if (ok && !mbar_wait(route_bar, 0, bound)) ok = false;
+        if (ok) U = rc.U;
+        const long nr = static_cast<long>(U) * NRB;
+        const int r_lo = static_cast<int>(nr * b / G), r_hi = static_cast<int>(nr * (b + 1) / G);
+        for (int tau = r_lo; tau < r_hi && ok; ++tau) stage1(record(f.S + tau / NRB), tau % NRB);
+        // phase 2: every work expert's block of down rows, in K parts
+        for (int we = 0; we < f.S + U && ok; ++we) {
+            const uint8_t *rec = record(we);
+            for (int part = 0; part < nks2 && ok; ++part, ++seq) {
+                const int s = seq % S;
+                const uint32_t par = (seq / S) & 1;
+                if (!mbar_wait(empty_bar(s), par ^ 1, bound)) { ok = false; break; }
+                if (rec == nullptr) { mbar_arrive(full_bar(s)); continue; }
+                const uint32_t dst = smem_u32(ring + static_cast<size_t>(s) * p.SB);
+                const int a1 = (j_hi + 3) & ~3;
+                const uint32_t bytes = static_cast<uint32_t>(nrows) * SK2 +
+                                       (GS ? static_cast<uint32_t>(nrows) * 4u * gps2 : 4u * (a1 - a0d));
+                mbar_expect_tx(full_bar(s), bytes);
+                const uint64_t pl = we < f.S ? keep : pol;
+                for (int r = 0; r < nrows; ++r)
+                    bulk_g2s(dst + r * st2, rec + f.off_wd + static_cast<size_t>(j_lo + r) * rb_i + static_cast<size_t>(part) * SK2,
+                             SK2, full_bar(s), pl);
+                if (GS) {  // this part's group scales of the CTA's rows, gps2 per row
+                    for (int r = 0; r < nrows; ++r)
+                        bulk_g2s(dst + p.st_sd + r * 4 * gps2,
+                                 rec + f.off_sd + (static_cast<size_t>(j_lo + r) * f.nsi + static_cast<size_t>(part) * gps2) * 4,
+                                 4 * gps2, full_bar(s), pl);
+                } else {
+                    bulk_g2s(dst + p.st_sd, rec + f.off_sd + 4 * a0d, 4 * (a1 - a0d), full_bar(s), pl);  // every part
+                }
             }
         }
-        for (int we = 0; ok && we < f.S + U; ++we, ++seq) {
-            const uint8_t *rec = record(we);
-            const int s = seq % S;
-            const uint32_t par = (seq / S) & 1;
-            if (!mbar_wait(empty_bar(s), par ^ 1)) { ok = false; break; }
-            const uint32_t dst = smem_u32(ring + static_cast<size_t>(s) * p.SB);
-            if (rec == nullptr) { mbar_arrive(full_bar(s)); continue; }
-            const int n = j_hi - j_lo;
-            const int a0 = j_lo & ~3, a1 = (j_hi + 3) & ~3;
-            const uint32_t bytes = n * static_cast<uint32_t>(f.rb_i) + 4u * (a1 - a0);
-            mbar_expect_tx(full_bar(s), bytes);
-            bulk_g2s(dst, rec + f.off_wd + static_cast<size_t>(j_lo) * f.rb_i, n * f.rb_i, full_bar(s), pol);
-            bulk_g2s(dst + p.st_sd, rec + f.off_sd + 4 * a0, 4 * (a1 - a0), full_bar(s), pol);
-        }
         if (!ok) atomicOr(f.err, COLI_DEVERR_TIMEOUT);
+        // Drain: the last fill of every ring slot has landed before this thread (and with it the
+        // CTA) exits, also when a wait ran out and the consumers gave up on the stage.
+        for (int s = 0; s < S && s < seq; ++s) {
+            const int q = s + S * ((seq - 1 - s) / S);  // last sequence number held by slot s
+            if (!mbar_wait(full_bar(s), (q / S) & 1, bound)) atomicOr(f.err, COLI_DEVERR_TIMEOUT);
+        }
         return;
     }
 
     // -------------------------------------------------------------------- consumers --------
     const int ct = threadIdx.x - 32;
     const int cw = ct >> 5;
-    const int T = f.T;
+    const int g8 = lane >> 2, tig = lane & 3;
     bool ok = true;
 
-    // activations -> 16-bit block fixed point per (token, chunk), transposed for conflict-free
-    // reads: int4 vector v of chunk c of token t at xq[(t * XV + v) * Lh + c]
-    for (int idx = ct; idx < T * Lh; idx += NC) {
-        const int t = idx / Lh, c = idx % Lh;
-        const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(f.x) +
-                                                          static_cast<size_t>(t) * f.H + static_cast<size_t>(c) * CPC);
-        uint32_t raw[CPC / 2];  // bf16 pairs
-#pragma unroll
-        for (int i = 0; i < CPC / 8; ++i) {
-            const uint4 v = __ldg(src + i);
-            raw[4 * i] = v.x; raw[4 * i + 1] = v.y; raw[4 * i + 2] = v.z; raw[4 * i + 3] = v.w;
-        }
-        auto xval = [&](int j) -> float {
-            const uint32_t w2 = raw[j >> 1];
-            return __uint_as_float((j & 1) ? (w2 & 0xffff0000u) : (w2 << 16));
-        };
-        float mx = 0.f;
-#pragma unroll
-        for (int j = 0; j < CPC; ++j) mx = fmaxf(mx, fabsf(xval(j)));
-        int ex = 0;
-        if (mx > 0.f) frexpf(mx, &ex);            // mx < 2^ex
-        const float up = ldexpf(1.0f, 15 - ex);    // |x * up| < 2^15
-        auto mq = [&](int j) -> int { return max(-32767, min(32767, __float2int_rn(xval(j) * up))); };
-        auto pk = [](int a, int bb) { return static_cast<int>((static_cast<uint32_t>(a) & 0xffffu) | (static_cast<uint32_t>(bb) << 16)); };
-        int w[XW];
-        int sum = 0;
-        if (FMT == 4) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                int m[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) { m[j] = mq(8 * i + j); sum += m[j]; }
-                w[4 * i + 0] = pk(m[0], m[2]);
-                w[4 * i + 1] = pk(m[4], m[6]);
-                w[4 * i + 2] = pk(m[1], m[3]);
-                w[4 * i + 3] = pk(m[5], m[7]);
-            }
-            xc[idx] = 8 * sum;
-        } else if (FMT == 8) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) w[i] = pk(mq(2 * i), mq(2 * i + 1));
-            xc[idx] = 0;
-        } else {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                int m[16];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) { m[j] = mq(16 * i + j); sum += m[j]; }
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    w[8 * i + 2 * k + 0] = pk(m[k], m[4 + k]);
-                    w[8 * i + 2 * k + 1] = pk(m[8 + k], m[12 + k]);
-                }
-            }
-            xc[idx] = 2 * sum;
-        }
-#pragma unroll
-        for (int v = 0; v < XV; ++v)
-            xq[(static_cast<size_t>(t) * XV + v) * Lh + c] = make_int4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
-        xs[idx] = 1.0f / up;
+    for (int i = ct; i < MAXWE * MAXTOK; i += NC) {
+        (&rc.slot[0][0])[i] = -1;
+        (&rc.wgt[0][0])[i] = 0.f;
     }
+    if (ct == 0) rc.err = 0;
 
-    // routing cache: [0] U; rBeg/rCnt per work expert; per slot: token, weight, h row
-    int *rU = rt;
-    int *rBeg = rt + RT_BEG;
-    int *rCnt = rt + RT_CNT;
-    int *rTok = rt + RT_TOK;
-    float *rW = reinterpret_cast<float *>(rt + RT_W);
-    int *rH = rt + RT_H;
-    bool have_routing = false;
-    int *rUniq = rt + RT_UNIQ;             // unique expert ids (for the producer)
-    RouteSmem *rsm = reinterpret_cast<RouteSmem *>(sm + p.off_x + static_cast<size_t>(T) * f.H * 2);
-    int *sorted_slot = rt + RT_SORT;
-    auto get_routing = [&]() {
-        const int n = T * f.K;
-        if (p.route_here) {
-            if (ct == 0) {  // every CTA's logits are written
-                const long long t0 = clock64();
-                while (ld_acquire(p.gbar) < static_cast<unsigned>(G)) {
-                    if (clock64() - t0 > WAIT_CYCLES) { atomicOr(f.err, COLI_DEVERR_TIMEOUT); break; }
-                }
-            }
-            cons_sync();
-            // every CTA routes the batch from the logits (same code, same inputs, same result)
-            if (cw < 4 * T) route_token(p, cw >> 2, cw & 3, lane, 2 + (cw >> 2), rsm[cw >> 2]);
-            cons_sync();
-            if (cw == 0) {
-                // slot s0 = lane: token s0 / K, rank s0 % K; stable sort of the slots by expert id
-                const int s0 = lane;
-                const int t0 = s0 < n ? s0 / f.K : 0;
-                const int id = s0 < n ? rsm[t0].out_id[s0 - t0 * f.K] : 0x7fffffff;
-                const float w0 = s0 < n ? rsm[t0].out_w[s0 - t0 * f.K] : 0.f;
-                int rk = 0;
+    // ---- start: activations (and the gate) ----
+    // thread ct owns elements h = 4 ct + 2048 gi (gi < GI) of every token
+    const int e0 = static_cast<int>(static_cast<long>(f.E) * b / G), e1 = static_cast<int>(static_cast<long>(f.E) * (b + 1) / G);
+    const int ne = p.route_here ? e1 - e0 : 0;        // router rows of this CTA (<= 2)
+    {
+        uint2 xv[MAXT][GI];
+        float4 wv[2][GI];
 #pragma unroll
-                for (int o = 0; o < 32; ++o) {
-                    const int oid = __shfl_sync(FULL, id, o);
-                    rk += ((oid < id) || (oid == id && o < lane)) ? 1 : 0;
-                }
-                if (s0 < n) sorted_slot[rk] = s0;
-                __syncwarp();
-                // position `lane` of the grouped order holds slot sl
-                const int sl = lane < n ? sorted_slot[lane] : 0;
-                const int idr = __shfl_sync(FULL, id, sl);
-                const int tr = __shfl_sync(FULL, t0, sl);
-                const float wr = __shfl_sync(FULL, w0, sl);
-                const int idp = __shfl_up_sync(FULL, idr, 1);
-                const bool first = lane < n && (lane == 0 || idp != idr);
-                const unsigned m = __ballot_sync(FULL, first);
-                const int U = __popc(m);
-                const int up = __popc(m & ((1u << lane) - 1u));
-                if (first) {
-                    const unsigned rest = lane < 31 ? (m >> (lane + 1)) : 0u;
-                    const int nxt = rest ? lane + __ffs(rest) : n;
-                    rBeg[f.S + up] = lane;
-                    rCnt[f.S + up] = nxt - lane;
-                    rUniq[up] = idr;
-                }
-                if (lane < n) {
-                    rTok[lane] = tr;
-                    rW[lane] = wr;
-                    rH[lane] = lane;
-                }
-                if (lane == 0) *rU = U;
-                if (blockIdx.x == 0) {  // the routing outputs of the call
-                    if (s0 < n) {
-                        p.ids[s0] = id;
-                        p.wts[s0] = w0;
+        for (int t = 0; t < MAXT; ++t)
+#pragma unroll
+            for (int gi = 0; gi < GI; ++gi)
+                xv[t][gi] = t < T ? __ldg(reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(f.x) + static_cast<size_t>(t) * f.H + 4 * ct + 2048 * gi))
+                                  : make_uint2(0u, 0u);
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int gi = 0; gi < GI; ++gi)
+                wv[j][gi] = j < ne ? __ldg(reinterpret_cast<const float4 *>(p.Wr + static_cast<size_t>(e0 + j) * f.H + 4 * ct + 2048 * gi))
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+        auto xval = [&](int t, int gi, int k) -> float {
+            const uint32_t w2 = (k < 2) ? xv[t][gi].x : xv[t][gi].y;
+            return __uint_as_float((k & 1) ? (w2 & 0xffff0000u) : (w2 << 16));
+        };
+        // per-token row maximum
+        float *xmax = reinterpret_cast<float *>(gpart + NCW * 2 * MAXTOK);  // [NCW][MAXTOK]
+#pragma unroll
+        for (int t = 0; t < MAXT; ++t) {
+            float m = 0.f;
+#pragma unroll
+            for (int gi = 0; gi < GI; ++gi)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) m = fmaxf(m, fabsf(xval(t, gi, k)));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
+            if (lane == 0) xmax[cw * MAXTOK + t] = m;
+        }
+        // gate partial dot products (exact double products, double sums)
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int t = 0; t < MAXT; ++t) {
+                if (j < ne && t < T) {
+                    double acc = 0.0;
+#pragma unroll
+                    for (int gi = 0; gi < GI; ++gi) {
+                        const float4 w4 = wv[j][gi];
+                        acc = fma(static_cast<double>(w4.x), static_cast<double>(xval(t, gi, 0)), acc);
+                        acc = fma(static_cast<double>(w4.y), static_cast<double>(xval(t, gi, 1)), acc);
+                        acc = fma(static_cast<double>(w4.z), static_cast<double>(xval(t, gi, 2)), acc);
+                        acc = fma(static_cast<double>(w4.w), static_cast<double>(xval(t, gi, 3)), acc);
                     }
-                    if (lane < n) p.f_perm[lane] = sl;
-                    if (first) p.f_unique[up] = idr;
-                    if (lane == 0) { *p.f_nuniq = U; p.f_offsets[f.E] = n; }
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(FULL, acc, o);
+                    if (lane == 0) gpart[cw * 2 * MAXTOK + j * MAXTOK + t] = acc;
                 }
             }
-            cons_sync();
-            if (blockIdx.x == 0) {
-                const int U = *rU;
-                for (int e = ct; e < f.E; e += NC) {
-                    int c = 0, lt = 0;
-                    for (int s2 = 0; s2 < n; ++s2) {
-                        const int v = rsm[s2 / f.K].out_id[s2 % f.K];
-                        c += v == e;
-                        lt += v < e;
+        cons_sync();
+        if (ct < ne * T) {  // one logit per thread of warp 0: the 16 warps' partials in order
+            const int j = ct / T, t = ct % T;
+            double sum = 0.0;
+            for (int w2 = 0; w2 < NCW; ++w2) sum += gpart[w2 * 2 * MAXTOK + j * MAXTOK + t];
+            p.logits[static_cast<size_t>(t) * f.E + e0 + j] = static_cast<float>(sum);
+            __threadfence();
+        }
+        if (cw == 0 && p.route_here) {
+            __syncwarp();
+            if (lane == 0) atomicAdd(p.gbar, 1u);
+        }
+        // activation slices: X = rint(x * 2^(22 - e)), max|x| < 2^e
+        const int NCOL = 3 * T;
+        const size_t colblk = 4 * 8 * MPC;             // bytes of one column's block of a chunk
+#pragma unroll
+        for (int t = 0; t < MAXT; ++t) {
+            if (t < T) {
+                float m = 0.f;
+                for (int w2 = 0; w2 < NCW; ++w2) m = fmaxf(m, xmax[w2 * MAXTOK + t]);
+                int ex = 0;
+                if (m > 0.f) frexpf(m, &ex);
+                const float up = ldexpf(1.0f, 22 - ex);
+                if (ct == 0) rc.xscale[t] = ldexpf(1.0f, ex - 22);
+#pragma unroll
+                for (int gi = 0; gi < GI; ++gi) {
+                    const int h0 = 4 * ct + 2048 * gi;
+                    const int kc = h0 / CPC, p0 = h0 % CPC;
+                    int sl[4][3];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int X = __float2int_rn(xval(t, gi, k) * up);
+                        slices3(X, sl[k][0], sl[k][1], sl[k][2]);
                     }
-                    p.f_counts[e] = c;
-                    p.f_offsets[e] = lt;
-                    if (e >= U) p.f_unique[e] = -1;
+#pragma unroll
+                    for (int s = 0; s < 3; ++s) {
+                        const int col = 3 * t + s;
+                        unsigned char *blk = xb + (static_cast<size_t>(kc) * NCOL + col) * colblk;
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            int tg, m2, hf, by;
+                            PL::at(p0 + k, tg, m2, hf, by);
+                            blk[b_off<FMT>(col, tg, m2, hf, by)] = static_cast<unsigned char>(sl[k][s] & 0xff);
+                        }
+                    }
                 }
             }
-        } else if (grid_dep_wait(), cw == 0) {  // routing given: lane u handles unique expert u
+        }
+    }
+    if (!p.route_here) {
+        // routing given (coli_moe_ffn): warp 0, lane u handles unique expert u
+        if (cw == 0) {
             int U = __ldcg(f.n_unique);
             U = U < 0 ? 0 : (U > 32 ? 32 : U);
-            int e = -1, b0 = 0, c0 = 0;
             if (lane < U) {
-                e = __ldcg(f.unique + lane);
+                const int e = __ldcg(f.unique + lane);
+                rc.uniq[lane] = e;
                 if (e >= 0 && e < f.E) {
-                    b0 = __ldcg(f.offsets + e);
-                    c0 = __ldcg(f.offsets + e + 1) - b0;
-                    if (b0 < 0 || c0 < 0 || b0 + c0 > T * f.K || c0 > TMAX) { c0 = 0; atomicOr(f.err, COLI_DEVERR_GROUPING); }
+                    const int b0 = __ldcg(f.offsets + e);
+                    int c0 = __ldcg(f.offsets + e + 1) - b0;
+                    if (b0 < 0 || c0 < 0 || b0 + c0 > T * f.K || c0 > T) { c0 = 0; atomicOr(f.err, COLI_DEVERR_GROUPING); }
+                    for (int qq = 0; qq < c0; ++qq) {
+                        const int sl = __ldcg(f.perm + b0 + qq);
+                        if (sl < 0 || sl >= T * f.K) { atomicOr(f.err, COLI_DEVERR_GROUPING); continue; }
+                        const int tok = sl / f.K;
+                        rc.slot[f.S + lane][tok] = b0 + qq;
+                        rc.wgt[f.S + lane][tok] = __ldcg(f.topk_w + sl);
+                    }
                 } else {
                     atomicOr(f.err, COLI_DEVERR_EXPERT_ID);
                 }
             }
-            int pos = c0;  // exclusive scan of the slot counts
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int v = __shfl_up_sync(FULL, pos, o);
-                if (lane >= o) pos += v;
-            }
-            pos -= c0;
-            if (lane == 0) *rU = U;
-            if (lane < U) {
-                rBeg[f.S + lane] = pos;
-                rCnt[f.S + lane] = c0;
-                rUniq[lane] = e;
-                for (int q = 0; q < c0; ++q) {
-                    const int sl = __ldcg(f.perm + b0 + q);
-                    const bool good = sl >= 0 && sl < T * f.K;
-                    if (!good) atomicOr(f.err, COLI_DEVERR_GROUPING);
-                    rTok[pos + q] = good ? sl / f.K : 0;
-                    rW[pos + q] = good ? __ldcg(f.topk_w + sl) : 0.f;
-                    rH[pos + q] = good ? b0 + q : 0;
-                }
+            if (lane == 0) rc.U = U;
+        }
+    }
+    if (f.S && ct < T) {
+        rc.slot[0][ct] = T * f.K + ct;
+        rc.wgt[0][ct] = 1.0f;
+    }
+    cons_sync();  // activation slices and (given routing) the routing cache ready
+
+    // ---- routing of the batch by every CTA (layer calls) ----
+    auto route_batch = [&]() {
+        if (ct == 0) {  // every CTA's logits are written
+            const long long t0 = clock64();
+            const unsigned target = static_cast<unsigned>(G) + p.gate_extra;
+            while (ld_acquire(p.gbar) < target) {
+                if (clock64() - t0 > bound) { atomicOr(f.err, COLI_DEVERR_TIMEOUT); break; }
             }
         }
         cons_sync();
-        if (ct == 0) mbar_arrive(route_bar);
-        have_routing = true;
+        const int nb = f.E / 32;
+        for (int job = cw; job < T * nb; job += NCW) route_block(p, job / nb, job % nb, lane, rtok[job / nb]);
+        cons_sync();
+        if (cw < T) route_select(p, cw, lane, rtok[cw], rc);
+        cons_sync();
+        if (cw == 0) {
+            // slot s = t K + k; stable sort of the slots by expert id
+            const int n = T * f.K;
+            const int t0 = lane < n ? lane / f.K : 0;
+            const int id = lane < n ? rc.ids[t0][lane - t0 * f.K] : 0x7fffffff;
+            const float w0 = lane < n ? rc.w[t0][lane - t0 * f.K] : 0.f;
+            int rk = 0;
+#pragma unroll
+            for (int o = 0; o < 32; ++o) {
+                const int oid = __shfl_sync(FULL, id, o);
+                rk += ((oid < id) || (oid == id && o < lane)) ? 1 : 0;
+            }
+            if (lane < n) rc.sorted[rk] = lane;
+            __syncwarp();
+            const int sl = lane < n ? rc.sorted[lane] : 0;  // position `lane` holds slot sl
+            const int idr = __shfl_sync(FULL, id, sl);
+            const int tr = __shfl_sync(FULL, t0, sl);
+            const float wr = __shfl_sync(FULL, w0, sl);
+            const int idp = __shfl_up_sync(FULL, idr, 1);
+            const bool first = lane < n && (lane == 0 || idp != idr);
+            const unsigned m = __ballot_sync(FULL, first);
+            const int U = __popc(m);
+            const int u = __popc(m & ((2u << lane) - 1u)) - 1;  // unique index of position lane
+            if (first) rc.uniq[u] = idr;
+            if (lane < n) {
+                if (idr < 0 || idr >= f.E) atomicOr(f.err, COLI_DEVERR_EXPERT_ID);
+                rc.slot[f.S + u][tr] = lane;
+                rc.wgt[f.S + u][tr] = wr;
+            }
+            if (lane == 0) rc.U = U;
+            if (blockIdx.x == 0) {  // the routing outputs of the call
+                if (lane < n) {
+                    p.ids[lane] = id;
+                    p.wts[lane] = w0;
+                    p.f_perm[lane] = sl;
+                }
+                if (first) p.f_unique[u] = idr;
+                if (lane == 0) { *p.f_nuniq = U; p.f_offsets[f.E] = n; }
+            }
+        }
+        cons_sync();
+        if (blockIdx.x == 0) {
+            const int n = T * f.K, U = rc.U;
+            for (int e = ct; e < f.E; e += NC) {
+                int c = 0, lt = 0;
+                for (int s2 = 0; s2 < n; ++s2) {
+                    const int v = rc.ids[s2 / f.K][s2 % f.K];
+                    c += v == e;
+                    lt += v < e;
+                }
+                p.f_counts[e] = c;
+                p.f_offsets[e] = lt;
+                if (e >= U) p.f_unique[e] = -1;
+            }
+        }
     };
-    cons_sync();  // activations ready
-
-    // phase 0 (layer calls): this CTA's share of the router gate, logits[t][e] in double from
-    // exact double products, then an arrival on the grid counter (the wait comes later, after
-    // the shared expert's rows, in get_routing)
-    if (p.route_here) {
-        const int e0 = static_cast<int>(static_cast<long>(f.E) * b / G), e1 = static_cast<int>(static_cast<long>(f.E) * (b + 1) / G);
-        double *gred = reinterpret_cast<double *>(sm + p.off_red);
-        for (int job = e0 * T; job < e1 * T; ++job) {
-            const int e = job / T, t = job % T;
-            const float *wrow = p.Wr + static_cast<size_t>(e) * f.H;
-            const uint16_t *xrow = static_cast<const uint16_t *>(f.x) + static_cast<size_t>(t) * f.H;
-            double acc = 0.0;
-            constexpr int GLD = 3;  // all of a thread's loads in flight together (H <= 3 * 2048)
-            float4 wv[GLD];
-            uint2 xv[GLD];
-#pragma unroll
-            for (int g = 0; g < GLD; ++g) {
-                const int h0 = ct * 4 + g * NC * 4;
-                const bool in = h0 < f.H;
-                wv[g] = in ? __ldg(reinterpret_cast<const float4 *>(wrow + h0)) : make_float4(0.f, 0.f, 0.f, 0.f);
-                xv[g] = in ? __ldg(reinterpret_cast<const uint2 *>(xrow + h0)) : make_uint2(0u, 0u);
-            }
-#pragma unroll
-            for (int g = 0; g < GLD; ++g) {
-                acc = fma(static_cast<double>(wv[g].x), static_cast<double>(__uint_as_float(xv[g].x << 16)), acc);
-                acc = fma(static_cast<double>(wv[g].y), static_cast<double>(__uint_as_float(xv[g].x & 0xffff0000u)), acc);
-                acc = fma(static_cast<double>(wv[g].z), static_cast<double>(__uint_as_float(xv[g].y << 16)), acc);
-                acc = fma(static_cast<double>(wv[g].w), static_cast<double>(__uint_as_float(xv[g].y & 0xffff0000u)), acc);
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(FULL, acc, o);
-            if (lane == 0) gred[cw] = acc;
-            cons_sync();
-            if (ct == 0) {
-                double sum = 0.0;
-                for (int w2 = 0; w2 < NCW; ++w2) sum += gred[w2];
-                p.logits[static_cast<size_t>(t) * f.E + e] = static_cast<float>(sum);
-            }
-            cons_sync();
-        }
-        if (ct == 0) {
-            __threadfence();
-            atomicAdd(p.gbar, 1u);
-        }
-    }
 
     // ------------------------------------------------ phase 1: gate/up, h = SiLU(g)*u -----
-    // After a timed-out wait a thread keeps walking the same loops and barriers (skipping later
-    // waits), so that no consumer is ever left alone at a named barrier.
-    const int NGRP = NCW / PS;               // stage groups
-    const int my_pair = cw % PS, my_grp = cw / PS;
-    int seq = 0, U = 0;
-    for (int we = 0;; ++we) {
-        if (we >= f.S && !have_routing) { get_routing(); U = *rU; }
-        if (have_routing && we >= f.S + U) break;
-        const bool shared = we < f.S;
-        const int cnt = shared ? T : rCnt[we];
-        const int beg = shared ? 0 : rBeg[we];
-        for (int k = 0; k < n1; ++k, ++seq) {
+    // After a timed-out wait a warp keeps walking the same loops and barriers (skipping later
+    // waits and MMAs), so that no consumer is ever left alone at a named barrier, and releases no
+    // more ring stages: the producer then runs out of its own bounded waits, and its drain makes
+    // sure no copy is still landing in shared memory when the CTA exits.
+    const int grp = cw / GW, wg = cw % GW;
+    const int cpw1 = SK1 / 64 / GW;                   // chunks of a stage per warp
+    const size_t colblk = 4 * 8 * MPC;
+    int seq = 0, U = 0, my_tiles = 0;
+    long r_lo = 0, r_hi = 0;
+    const int NCOL = 3 * T;
+    for (int lam = 0;; ++lam) {
+        if (lam == nsh) {
+            if (p.route_here) route_batch();
+            if (ct == 0) mbar_arrive(route_bar);
+            U = rc.U;
+            const long nr = static_cast<long>(U) * NRB;
+            r_lo = nr * b / G;
+            r_hi = nr * (b + 1) / G;
+        }
+        if (lam >= nsh && lam - nsh >= r_hi - r_lo) break;
+        int we, rb;
+        if (lam < nsh) { we = 0; rb = sh_lo + lam; }
+        else { const long tau = r_lo + (lam - nsh); we = f.S + static_cast<int>(tau / NRB); rb = static_cast<int>(tau % NRB); }
+        if ((lam % NGRP) != grp) { seq += nks1; continue; }
+        int D[NB][4];       // per-row scales: exact int32 sums over all of K
+        float Dg[NB][4];    // group scales: float sums of (group sum x group scale)
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) { D[nb][i] = 0; Dg[nb][i] = 0.f; }
+        const unsigned char *scal = nullptr;
+        for (int part = 0; part < nks1; ++part, ++seq) {
             const int s = seq % S;
             const uint32_t par = (seq / S) & 1;
-            if (ok && !mbar_wait(full_bar(s), par)) ok = false;
-            const int r0 = i_lo + k * PS, n = min(PS, i_hi - r0);
-            const bool mine = ok && (seq % NGRP) == my_grp && my_pair < n && my_grp < NGRP;
-            if (mine) {
-                const unsigned char *st = ring + static_cast<size_t>(s) * p.SB;
-                const unsigned char *rg = st + static_cast<size_t>(my_pair) * f.rb_h;
-                const unsigned char *ru = st + p.st_up + static_cast<size_t>(my_pair) * f.rb_h;
-                float g[TMAX], u[TMAX];
-                const int4 *xb[TMAX];
-                const float *xsb[TMAX];
-                const int *xcb[TMAX];
+            if (ok && !mbar_wait(full_bar(s), par, bound)) ok = false;
+            ok = __all_sync(FULL, ok);  // warp-uniform: the MMAs below need every lane
+            const unsigned char *st = ring + static_cast<size_t>(s) * p.SB;
+            if (part == 0) scal = st + 16 * st1;
+            if (ok) {
+                for (int cc = 0; cc < cpw1; ++cc) {
+                    const int c = wg * cpw1 + cc;                    // chunk inside the stage
+                    const int kc = part * (SK1 / 64) + c;            // chunk inside the row
+                    const uint4 qa = PL::load_a(st + g8 * st1 + 64 * c, tig);
+                    const uint4 qb = PL::load_a(st + (g8 + 8) * st1 + 64 * c, tig);
+                    const unsigned char *xk = xb + static_cast<size_t>(kc) * NCOL * colblk;
 #pragma unroll
-                for (int q = 0; q < TMAX; ++q) {
-                    g[q] = 0.f; u[q] = 0.f;
-                    const int tok = q < cnt ? (shared ? q : rTok[beg + q]) : 0;
-                    xb[q] = xq + static_cast<size_t>(tok) * XV * Lh + lane;
-                    xsb[q] = xs + tok * Lh + lane;
-                    xcb[q] = xc + tok * Lh + lane;
-                }
-                const unsigned char *rgl = rg + lane * 16, *rul = ru + lane * 16;
+                    for (int u = 0; u < MPC / 2; ++u) {
+                        uint4 bv[NB];
 #pragma unroll
-                for (int j = 0; j < NJ; ++j) {
-                    const uint4 qg = lds128(rgl + j * 512);
-                    const uint4 qu = lds128(rul + j * 512);
-#pragma unroll
-                    for (int q = 0; q < TMAX; ++q) {
-                        if (q < cnt) {
-                            int xr[XW];
-#pragma unroll
-                            for (int v = 0; v < XV; ++v) {
-                                const int4 t4 = xb[q][v * Lh + 32 * j];
-                                xr[4 * v] = t4.x; xr[4 * v + 1] = t4.y; xr[4 * v + 2] = t4.z; xr[4 * v + 3] = t4.w;
-                            }
-                            const float sc = xsb[q][32 * j];
-                            const int corr = xcb[q][32 * j];
-                            g[q] = __fmaf_rn(static_cast<float>(idot_chunk<FMT>(qg, xr, corr)), sc, g[q]);
-                            u[q] = __fmaf_rn(static_cast<float>(idot_chunk<FMT>(qu, xr, corr)), sc, u[q]);
+                        for (int nb = 0; nb < NB; ++nb) {
+                            const int col = nb * 8 + g8;
+                            bv[nb] = col < NCOL ? load_b2<FMT>(xk + col * colblk, col, tig, u) : make_uint4(0u, 0u, 0u, 0u);
                         }
-                    }
-                }
-                const int a0 = r0 & ~3;
-                const float sgv = reinterpret_cast<const float *>(st + p.st_sg)[r0 + my_pair - a0];
-                const float suv = reinterpret_cast<const float *>(st + p.st_su)[r0 + my_pair - a0];
+                        int Du[NB][4];  // group-scaled container: this group's sums
 #pragma unroll
-                for (int q = 0; q < TMAX; ++q) {
-                    if (q < cnt) {
-                        const float gq = __fmul_rn(warp_allsum(g[q]), sgv);
-                        const float uq = __fmul_rn(warp_allsum(u[q]), suv);
-                        if (lane == q) {
-                            const int hrow = shared ? T * f.K + q : rH[beg + q];
-                            f.h[static_cast<size_t>(hrow) * f.I + r0 + my_pair] =
-                                __fmul_rn(__fdiv_rn(gq, __fadd_rn(1.0f, expf(-gq))), uq);
+                        for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) Du[nb][i] = 0;
+#pragma unroll
+                        for (int mm = 0; mm < 2; ++mm) {
+                            uint32_t a0, a2, a1, a3;
+                            F::unpack(qa, 2 * u + mm, a0, a2);
+                            F::unpack(qb, 2 * u + mm, a1, a3);
+#pragma unroll
+                            for (int nb = 0; nb < NB; ++nb)
+                                mma_s8(GS ? Du[nb] : D[nb], a0, a1, a2, a3, mm ? bv[nb].z : bv[nb].x, mm ? bv[nb].w : bv[nb].y);
+                        }
+                        if (GS) {  // group u of the chunk: rows g8 (gate) and g8 + 8 (up)
+                            const float *gsc = reinterpret_cast<const float *>(st + 16 * st1);
+                            const float sa = gsc[g8 * gps1 + 2 * c + u];
+                            const float sb = gsc[(g8 + 8) * gps1 + 2 * c + u];
+#pragma unroll
+                            for (int nb = 0; nb < NB; ++nb) {
+                                Dg[nb][0] = __fmaf_rn(static_cast<float>(Du[nb][0]), sa, Dg[nb][0]);
+                                Dg[nb][1] = __fmaf_rn(static_cast<float>(Du[nb][1]), sa, Dg[nb][1]);
+                                Dg[nb][2] = __fmaf_rn(static_cast<float>(Du[nb][2]), sb, Dg[nb][2]);
+                                Dg[nb][3] = __fmaf_rn(static_cast<float>(Du[nb][3]), sb, Dg[nb][3]);
+                            }
                         }
                     }
                 }
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(empty_bar(s));
+            // stage 0 of the tile holds the row scales until the epilogue has read them: it is
+            // released after the reduction (below), the other parts now
+            if (ok && part > 0 && lane == 0) mbar_arrive(empty_bar(s));
         }
+        // group reduction of the partial sums, then one warp forms h
+        const int tile_seq0 = seq - nks1;
+        if (my_tiles > 0 && wg != 0) named_sync(BAR_GFREE + grp, GW * 32);
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb)
+            red1[((grp * GW + wg) * NB + nb) * 32 + lane] =
+                GS ? make_int4(__float_as_int(Dg[nb][0]), __float_as_int(Dg[nb][1]), __float_as_int(Dg[nb][2]), __float_as_int(Dg[nb][3]))
+                   : make_int4(D[nb][0], D[nb][1], D[nb][2], D[nb][3]);
+        named_sync(BAR_GFULL + grp, GW * 32);
+        if (wg == 0) {
+            const int pr = lane & 7, t = lane >> 3;  // row pair, token
+            const int slot = t < T ? rc.slot[we][t] : -1;
+            if (ok && slot >= 0 && GS) {
+                // group-scaled: the partials already carry the weights' scales
+                double gsum = 0.0, usum = 0.0;
+#pragma unroll
+                for (int sidx = 0; sidx < 3; ++sidx) {
+                    const int col = 3 * t + sidx, nb = col >> 3, c8 = col & 7;
+                    const int ln = pr * 4 + (c8 >> 1), ix = c8 & 1;
+                    float gs = 0.f, us = 0.f;
+                    for (int w2 = 0; w2 < GW; ++w2) {
+                        const float *v = reinterpret_cast<const float *>(&red1[((grp * GW + w2) * NB + nb) * 32 + ln]);
+                        gs = __fadd_rn(gs, v[ix]);
+                        us = __fadd_rn(us, v[2 + ix]);
+                    }
+                    const double wsl = sidx == 0 ? 1.0 : (sidx == 1 ? 256.0 : 65536.0);
+                    gsum += wsl * gs;
+                    usum += wsl * us;
+                }
+                const double xs = static_cast<double>(rc.xscale[t]) / F::MUL;
+                const float gq = static_cast<float>(gsum * xs);
+                const float uq = static_cast<float>(usum * xs);
+                f.h[static_cast<size_t>(slot) * f.I + rb * 8 + pr] = __fmul_rn(__fdiv_rn(gq, __fadd_rn(1.0f, expf(-gq))), uq);
+            } else if (ok && slot >= 0) {
+                long long gsum = 0, usum = 0;
+#pragma unroll
+                for (int sidx = 0; sidx < 3; ++sidx) {
+                    const int col = 3 * t + sidx, nb = col >> 3, c8 = col & 7;
+                    const int ln = pr * 4 + (c8 >> 1), ix = c8 & 1;
+                    int gs = 0, us = 0;
+                    for (int w2 = 0; w2 < GW; ++w2) {
+                        const int *v = reinterpret_cast<const int *>(&red1[((grp * GW + w2) * NB + nb) * 32 + ln]);
+                        gs += v[ix];
+                        us += v[2 + ix];
+                    }
+                    const long long wsl = sidx == 0 ? 1LL : (sidx == 1 ? 256LL : 65536LL);
+                    gsum += wsl * gs;
+                    usum += wsl * us;
+                }
+                const float sgv = reinterpret_cast<const float *>(scal)[pr];
+                const float suv = reinterpret_cast<const float *>(scal + 32)[pr];
+                const double xs = static_cast<double>(rc.xscale[t]) / F::MUL;
+                const float gq = static_cast<float>(static_cast<double>(gsum) * xs * static_cast<double>(sgv));
+                const float uq = static_cast<float>(static_cast<double>(usum) * xs * static_cast<double>(suv));
+                f.h[static_cast<size_t>(slot) * f.I + rb * 8 + pr] = __fmul_rn(__fdiv_rn(gq, __fadd_rn(1.0f, expf(-gq))), uq);
+            }
+            __syncwarp();
+            named_arrive(BAR_GFREE + grp, GW * 32);
+        }
+        // stage 0 of the tile (it held the row scales) is released now
+        __syncwarp();
+        if (ok && lane == 0) mbar_arrive(empty_bar(tile_seq0 % S));
+        ++my_tiles;
     }
+    if (my_tiles > 0 && wg != 0) named_sync(BAR_GFREE + grp, GW * 32);  // the last arrival
 
     // ------------------------------------------------ grid barrier ------------------------
     cons_sync();
     if (ct == 0) {
         __threadfence();
         atomicAdd(p.gbar, 1u);
-        const unsigned target = static_cast<unsigned>(G) * (p.route_here ? 2u : 1u);
+        const unsigned target = static_cast<unsigned>(G) * (p.route_here ? 2u : 1u) + p.gate_extra;
         const long long t0 = clock64();
         while (ld_acquire(p.gbar) < target) {
-            if (clock64() - t0 > WAIT_CYCLES) { atomicOr(f.err, COLI_DEVERR_TIMEOUT); break; }
+            if (clock64() - t0 > bound) { atomicOr(f.err, COLI_DEVERR_TIMEOUT); break; }
         }
         // the last CTA to leave the barrier zeroes both counters for the next call
         if (atomicAdd(p.gdep, 1u) == static_cast<unsigned>(G) - 1u) {
@@ -826,189 +867,211 @@ __global__ void __maxnreg__(96) ffn_decode_kernel(DecodeParams p) {
     cons_sync();
 
     // ------------------------------------------------ phase 2: down + combine -------------
-    // h of one expert's slots is converted once per CTA into 16-bit fixed point per chunk split
-    // in two signed bytes (4 elements per thread, chunk maximum over the chunk's lanes), double
-    // buffered; the next expert's h is prefetched into registers while the current one is used.
-    const int p2 = ct / Li, c2 = ct % Li;
-    const int P2 = p.P2;
-    const int nwr2 = Li / 32;
-    float acc[RPT2MAX][TMAX];
-#pragma unroll
-    for (int m = 0; m < RPT2MAX; ++m)
-#pragma unroll
-        for (int q = 0; q < TMAX; ++q) acc[m][q] = 0.f;
-    const int nrows = j_hi - j_lo;
-    const int a0d = j_lo & ~3;
+    // warp cw owns chunk cw of the down rows (when the rows have that many 64-byte chunks)
+    constexpr int CPL = CPC / 32;                     // h elements per lane of a chunk
+    constexpr int RT2 = 3;                            // 16-row tiles of the CTA's output rows
+    const int nch2 = rb_i / 64;
+    const int cpp2 = SK2 / 64;                        // chunks per phase-2 stage
+    const bool active2 = cw < nch2;
+    const int part2 = cw / cpp2, cl2 = cw % cpp2;
     const int nwe = f.S + U;
-    // buffer layout (int4 vectors): [buf][slot][part hi/lo][XV8][Li]; per (buf, slot, chunk):
-    // one float scale
-    constexpr int XW8 = Ph2<FMT>::XW8, XV8 = Ph2<FMT>::XV8;
-    int4 *hq = reinterpret_cast<int4 *>(sm + p.off_x);
-    const size_t hq_buf = static_cast<size_t>(TMAX) * 2 * XV8 * Li;      // int4 per buffer
-    float *hsc = reinterpret_cast<float *>(sm + p.off_xs);                // [buf][slot][Li]
-    const int ngrp = f.I / 4;                                              // 4-element groups per slot
-    float4 pre[TMAX];
-    auto fetch_h = [&](int we) {
-        const bool shd = we < f.S;
-        const int cnt = shd ? T : rCnt[we];
-        const int beg = shd ? 0 : rBeg[we];
+    unsigned char *hb = sm + p.off_x + static_cast<size_t>(cw) * NCOL * colblk;  // this warp's h slices
+    float acc[RT2][NB][4];
 #pragma unroll
-        for (int q = 0; q < TMAX; ++q) {
-            if (q < cnt && ct < ngrp) {
-                const int hrow = shd ? T * f.K + q : rH[beg + q];
-                pre[q] = ldcg4(f.h + static_cast<size_t>(hrow) * f.I + 4 * ct);
+    for (int rt = 0; rt < RT2; ++rt)
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[rt][nb][i] = 0.f;
+    float hv[MAXT][CPL];
+    auto fetch_h = [&](int we) {
+#pragma unroll
+        for (int t = 0; t < MAXT; ++t) {
+            const int slot = t < T ? rc.slot[we][t] : -1;
+#pragma unroll
+            for (int k = 0; k < CPL; k += 4) {
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (slot >= 0 && active2)
+                    v = __ldcg(reinterpret_cast<const float4 *>(f.h + static_cast<size_t>(slot) * f.I + cw * CPC + lane * CPL + k));
+                hv[t][k] = v.x; hv[t][k + 1] = v.y; hv[t][k + 2] = v.z; hv[t][k + 3] = v.w;
             }
         }
     };
-    auto convert_h = [&](int we, int buf) {
-        const bool shd = we < f.S;
-        const int cnt = shd ? T : rCnt[we];
-        constexpr int GPC = CPC / 4;          // threads (4 elements each) per chunk
+    if (nwe > 0) fetch_h(0);
+    for (int we = 0; we < nwe; ++we) {
+        const int s = (seq + we * nks2 + part2) % S;
+        const uint32_t par = ((seq + we * nks2 + part2) / S) & 1;
+        // h of this expert's slots -> 24-bit fixed point per chunk, three byte slices
+        float fcol[NB][2];
+        if (active2) {
 #pragma unroll
-        for (int q = 0; q < TMAX; ++q) {
-            if (q < cnt) {
-                const bool act = ct < ngrp;
-                const float v[4] = {pre[q].x, pre[q].y, pre[q].z, pre[q].w};
-                float mx = act ? fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3]))) : 0.f;
+            for (int t = 0; t < MAXT; ++t) {
+                if (t < T) {
+                    float m = 0.f;
 #pragma unroll
-                for (int o = GPC / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
-                const float inv = mx > 0.f ? __fdiv_rn(32512.0f, mx) : 0.f;
-                if (act) {
-                    const int cc = (4 * ct) / CPC;                          // chunk of these elements
+                    for (int k = 0; k < CPL; ++k) m = fmaxf(m, fabsf(hv[t][k]));
 #pragma unroll
-                    for (int e2 = 0; e2 < 4; ++e2) {
-                        const int j = (4 * ct + e2) % CPC;
-                        const int X = max(-32512, min(32512, __float2int_rn(__fmul_rn(v[e2], inv))));
-                        const int xh = (X + 128) >> 8;                      // in [-127, 127]
-                        const int xl = X - 256 * xh;                        // in [-128, 127]
-                        int word, byte;
-                        h_slot<FMT>(j, word, byte);
-                        int8_t *ph = reinterpret_cast<int8_t *>(hq + buf * hq_buf + ((static_cast<size_t>(q) * 2 + 0) * XV8 + (word >> 2)) * Li + cc);
-                        int8_t *pl = reinterpret_cast<int8_t *>(hq + buf * hq_buf + ((static_cast<size_t>(q) * 2 + 1) * XV8 + (word >> 2)) * Li + cc);
-                        ph[4 * (word & 3) + byte] = static_cast<int8_t>(xh);
-                        pl[4 * (word & 3) + byte] = static_cast<int8_t>(xl);
+                    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
+                    int ex = 0;
+                    if (m > 0.f) frexpf(m, &ex);
+                    const float up = ldexpf(1.0f, 22 - ex);
+                    // column factors of this token: combine weight x scale x slice weight
+                    const float base = rc.wgt[we][t] * ldexpf(1.0f, ex - 22) / F::MUL;
+#pragma unroll
+                    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                        for (int i = 0; i < 2; ++i) {
+                            const int col = nb * 8 + 2 * tig + i;
+                            if (col / 3 == t) fcol[nb][i] = base * (col % 3 == 0 ? 1.0f : (col % 3 == 1 ? 256.0f : 65536.0f));
+                        }
+#pragma unroll
+                    for (int k = 0; k < CPL; ++k) {
+                        int s0, s1, s2;
+                        slices3(__float2int_rn(hv[t][k] * up), s0, s1, s2);
+                        int tg, m2, hf, by;
+                        PL::at(lane * CPL + k, tg, m2, hf, by);
+                        hb[(3 * t + 0) * colblk + b_off<FMT>(3 * t + 0, tg, m2, hf, by)] = static_cast<unsigned char>(s0 & 0xff);
+                        hb[(3 * t + 1) * colblk + b_off<FMT>(3 * t + 1, tg, m2, hf, by)] = static_cast<unsigned char>(s1 & 0xff);
+                        hb[(3 * t + 2) * colblk + b_off<FMT>(3 * t + 2, tg, m2, hf, by)] = static_cast<unsigned char>(s2 & 0xff);
                     }
-                    if ((ct % GPC) == 0)
-                        hsc[(buf * TMAX + q) * Li + cc] = __fdiv_rn(mx, 32512.0f * Ph2<FMT>::MUL);
                 }
             }
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                for (int i = 0; i < 2; ++i)
+                    if (nb * 8 + 2 * tig + i >= NCOL) fcol[nb][i] = 0.f;
         }
-    };
-    if (nwe > 0) {
-        fetch_h(0);
-        convert_h(0, 0);
-    }
-    cons_sync();
-    for (int we = 0; we < nwe; ++we) {
-        const bool shared = we < f.S;
-        const int cnt = shared ? T : rCnt[we];
-        const int beg = shared ? 0 : rBeg[we];
-        const int buf = we & 1;
+        __syncwarp();
         if (we + 1 < nwe) fetch_h(we + 1);
-        const int s = seq % S;
-        const uint32_t par = (seq / S) & 1;
-        ++seq;
-        if (ok && !mbar_wait(full_bar(s), par)) ok = false;
-        if (ok) {
+        if (ok && active2 && !mbar_wait(full_bar(s), par, bound)) ok = false;
+        ok = __all_sync(FULL, ok);
+        if (ok && active2) {
             const unsigned char *st = ring + static_cast<size_t>(s) * p.SB;
             const float *sdp = reinterpret_cast<const float *>(st + p.st_sd) + (j_lo - a0d);
-            for (int q = 0; q < cnt; ++q) {
-                const int tok = shared ? q : rTok[beg + q];
-                const float wq = shared ? 1.0f : rW[beg + q];
-                int xh[XW8], xl[XW8];
+            const float *sdg = reinterpret_cast<const float *>(st + p.st_sd);  // [nrows][gps2]
+            uint32_t bf[MPC][NB][2];
 #pragma unroll
-                for (int v = 0; v < XV8; ++v) {
-                    const int4 a4 = hq[buf * hq_buf + ((static_cast<size_t>(q) * 2 + 0) * XV8 + v) * Li + c2];
-                    const int4 b4 = hq[buf * hq_buf + ((static_cast<size_t>(q) * 2 + 1) * XV8 + v) * Li + c2];
-                    xh[4 * v] = a4.x; xh[4 * v + 1] = a4.y; xh[4 * v + 2] = a4.z; xh[4 * v + 3] = a4.w;
-                    xl[4 * v] = b4.x; xl[4 * v + 1] = b4.y; xl[4 * v + 2] = b4.z; xl[4 * v + 3] = b4.w;
+            for (int u = 0; u < MPC / 2; ++u)
+#pragma unroll
+                for (int nb = 0; nb < NB; ++nb) {
+                    const int col = nb * 8 + g8;
+                    const uint4 v = col < NCOL ? load_b2<FMT>(hb + col * colblk, col, tig, u) : make_uint4(0u, 0u, 0u, 0u);
+                    bf[2 * u][nb][0] = v.x;
+                    bf[2 * u][nb][1] = v.y;
+                    bf[2 * u + 1][nb][0] = v.z;
+                    bf[2 * u + 1][nb][1] = v.w;
                 }
-                const float hs = hsc[(buf * TMAX + q) * Li + c2];
 #pragma unroll
-                for (int m = 0; m < RPT2MAX; ++m) {
-                    const int row = p2 + P2 * m;
-                    if (row < nrows) {
-                        const uint4 qd = lds128(st + static_cast<size_t>(row) * f.rb_i + c2 * 16);
-                        int sh, sl;
-                        idot4_chunk<FMT>(qd, xh, xl, sh, sl);
-                        const float d = __fmul_rn(__fmaf_rn(static_cast<float>(sh), 256.0f, static_cast<float>(sl)), hs);
-                        const float wsd = __fmul_rn(wq, sdp[row]);
+            for (int rt = 0; rt < RT2; ++rt) {
+                const int ra = rt * 16 + g8, rbw = ra + 8;
+                if (rt * 16 < nrows) {
+                    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+                    const uint4 qa = ra < nrows ? PL::load_a(st + ra * st2 + 64 * cl2, tig) : z;
+                    const uint4 qb = rbw < nrows ? PL::load_a(st + rbw * st2 + 64 * cl2, tig) : z;
+                    // per-row scales: one sum over the chunk; group scales: one per group u
+                    constexpr int NU = GS ? MPC / 2 : 1;
 #pragma unroll
-                        for (int t2 = 0; t2 < TMAX; ++t2)
-                            if (t2 == tok) acc[m][t2] = __fmaf_rn(d, wsd, acc[m][t2]);
+                    for (int ug = 0; ug < NU; ++ug) {
+                        int D[NB][4];
+#pragma unroll
+                        for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) D[nb][i] = 0;
+#pragma unroll
+                        for (int m = ug * (MPC / NU); m < (ug + 1) * (MPC / NU); ++m) {
+                            uint32_t a0, a2, a1, a3;
+                            F::unpack(qa, m, a0, a2);
+                            F::unpack(qb, m, a1, a3);
+#pragma unroll
+                            for (int nb = 0; nb < NB; ++nb) mma_s8(D[nb], a0, a1, a2, a3, bf[m][nb][0], bf[m][nb][1]);
+                        }
+                        float sda, sdb;
+                        if (GS) {  // group ug of this warp's chunk, rows ra and rbw
+                            sda = ra < nrows ? sdg[ra * gps2 + 2 * cl2 + ug] : 0.f;
+                            sdb = rbw < nrows ? sdg[rbw * gps2 + 2 * cl2 + ug] : 0.f;
+                        } else {
+                            sda = ra < nrows ? sdp[ra] : 0.f;
+                            sdb = rbw < nrows ? sdp[rbw] : 0.f;
+                        }
+#pragma unroll
+                        for (int nb = 0; nb < NB; ++nb) {
+                            acc[rt][nb][0] = __fmaf_rn(static_cast<float>(D[nb][0]), sda * fcol[nb][0], acc[rt][nb][0]);
+                            acc[rt][nb][1] = __fmaf_rn(static_cast<float>(D[nb][1]), sda * fcol[nb][1], acc[rt][nb][1]);
+                            acc[rt][nb][2] = __fmaf_rn(static_cast<float>(D[nb][2]), sdb * fcol[nb][0], acc[rt][nb][2]);
+                            acc[rt][nb][3] = __fmaf_rn(static_cast<float>(D[nb][3]), sdb * fcol[nb][1], acc[rt][nb][3]);
+                        }
                     }
                 }
             }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(empty_bar(s));
-        if (we + 1 < nwe) convert_h(we + 1, buf ^ 1);
-        cons_sync();
+        if (ok && active2 && lane == 0) mbar_arrive(empty_bar(s));
     }
     if (!ok) atomicOr(f.err, COLI_DEVERR_TIMEOUT);
-    // cross-lane reduction of the accumulators, then one store per (token, row)
+    // cross-warp reduction (the h slices are no longer needed: the region is reused)
+    cons_sync();
+    float *red2 = reinterpret_cast<float *>(sm + p.off_x);  // [warp][rt][nb][lane][4]
+    if (active2) {
 #pragma unroll
-    for (int m = 0; m < RPT2MAX; ++m)
+        for (int rt = 0; rt < RT2; ++rt)
 #pragma unroll
-        for (int q = 0; q < TMAX; ++q) {
-            if (q < T) {
-                const float v = warp_allsum(acc[m][q]);
-                if (lane == 0) red2[((p2 * RPT2MAX + m) * TMAX + q) * nwr2 + (c2 >> 5)] = v;
+            for (int nb = 0; nb < NB; ++nb)
+                reinterpret_cast<float4 *>(red2)[((cw * RT2 + rt) * NB + nb) * 32 + lane] =
+                    make_float4(acc[rt][nb][0], acc[rt][nb][1], acc[rt][nb][2], acc[rt][nb][3]);
+    }
+    cons_sync();
+    const int nact = nch2 < NCW ? nch2 : NCW;
+    for (int fi = ct; fi < nrows * T; fi += NC) {
+        const int r = fi / T, t = fi % T;
+        const int rt = r >> 4, rr = r & 15, gg = rr & 7, hi = rr >> 3;
+        float v = 0.f;
+        for (int w2 = 0; w2 < nact; ++w2) {
+#pragma unroll
+            for (int sidx = 0; sidx < 3; ++sidx) {
+                const int col = 3 * t + sidx, nb = col >> 3, c8 = col & 7;
+                const int ln = gg * 4 + (c8 >> 1), ix = 2 * hi + (c8 & 1);
+                v = __fadd_rn(v, red2[(((w2 * RT2 + rt) * NB + nb) * 32 + ln) * 4 + ix]);
             }
         }
-    cons_sync();
-    for (int fi = ct; fi < P2 * RPT2MAX * T; fi += NC) {
-        const int q = fi % T, m = (fi / T) % RPT2MAX, ps = fi / (T * RPT2MAX);
-        const int row = ps + P2 * m;
-        if (row >= nrows) continue;
-        float v = 0.f;
-        for (int w = 0; w < nwr2; ++w) v = __fadd_rn(v, red2[((ps * RPT2MAX + m) * TMAX + q) * nwr2 + w]);
-        f.out[static_cast<size_t>(q) * f.H + j_lo + row] = v;
+        f.out[static_cast<size_t>(t) * f.H + j_lo + r] = v;
     }
 }
 
-template <int FMT, int TMAX, int NJ>
-cudaError_t launch_k2(const DecodeParams &p, size_t smem, cudaStream_t st) {
-    auto kern = ffn_decode_kernel<FMT, TMAX, NJ>;
+template <int FMT, int TT, int GI, int GS>
+cudaError_t launch_k(const DecodeParams &p, size_t smem, cudaStream_t st) {
+    auto kern = ffn_decode_kernel<FMT, TT, GI, GS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    kern<<<p.grid, NT, smem, st>>>(p);
-    return cudaGetLastError();
+    // cooperative: the grid barriers need every CTA resident at once; the launch waits for the
+    // whole grid to fit (or fails) instead of leaving CTAs spinning for SMs held elsewhere
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.grid);
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
-template <int FMT, int NJ>
-cudaError_t launch_k2_t(const DecodeParams &p, size_t smem, cudaStream_t st) {
-    if (p.f.T <= 1) return launch_k2<FMT, 1, NJ>(p, smem, st);
-    if (p.f.T <= 2) return launch_k2<FMT, 2, NJ>(p, smem, st);
-    return launch_k2<FMT, 4, NJ>(p, smem, st);
+template <int FMT, int GI, int GS>
+cudaError_t launch_nb(const DecodeParams &p, size_t smem, cudaStream_t st) {
+    if (p.f.T <= 1) return launch_k<FMT, 1, GI, GS>(p, smem, st);
+    if (p.f.T <= 2) return launch_k<FMT, 2, GI, GS>(p, smem, st);
+    return launch_k<FMT, 4, GI, GS>(p, smem, st);
 }
 
-// The instantiated (format, chunks per lane) pairs: GLM-5.2 shapes (hidden 6144) in the three
-// containers and the OLMoE shape (hidden 2048) in int4.
-template <int FMT, int NJ>
-static bool fits_block_t(int T) {
-    cudaFuncAttributes fa;
-    cudaError_t e;
-    if (T <= 1) e = cudaFuncGetAttributes(&fa, ffn_decode_kernel<FMT, 1, NJ>);
-    else if (T <= 2) e = cudaFuncGetAttributes(&fa, ffn_decode_kernel<FMT, 2, NJ>);
-    else e = cudaFuncGetAttributes(&fa, ffn_decode_kernel<FMT, 4, NJ>);
-    return e == cudaSuccess && fa.maxThreadsPerBlock >= NT;
-}
-
-static bool kernel_fits(int fmt, int nj, int T) {
-    if (fmt == 4 && nj == 6) return fits_block_t<4, 6>(T);
-    if (fmt == 4 && nj == 2) return fits_block_t<4, 2>(T);
-    if (fmt == 8 && nj == 12) return fits_block_t<8, 12>(T);
-    if (fmt == 2 && nj == 3) return fits_block_t<2, 3>(T);
-    return false;
-}
-
-static cudaError_t launch_k2_any(const DecodeParams &p, size_t smem, cudaStream_t st) {
-    const int nj = p.Lh / 32;
-    if (p.f.fmt == 4 && nj == 6) return launch_k2_t<4, 6>(p, smem, st);
-    if (p.f.fmt == 4 && nj == 2) return launch_k2_t<4, 2>(p, smem, st);
-    if (p.f.fmt == 8 && nj == 12) return launch_k2_t<8, 12>(p, smem, st);
-    if (p.f.fmt == 2 && nj == 3) return launch_k2_t<2, 3>(p, smem, st);
+static cudaError_t launch_any(const DecodeParams &p, size_t smem, cudaStream_t st) {
+    const int gi = p.f.H / 2048;
+    if (p.f.fmt == 4 && gi == 3 && p.f.group == 64) return launch_nb<4, 3, 64>(p, smem, st);
+    if (p.f.group) return cudaErrorInvalidValue;
+    if (p.f.fmt == 4 && gi == 3) return launch_nb<4, 3, 0>(p, smem, st);
+    if (p.f.fmt == 4 && gi == 1) return launch_nb<4, 1, 0>(p, smem, st);
+    if (p.f.fmt == 2 && gi == 3) return launch_nb<2, 3, 0>(p, smem, st);
     return cudaErrorInvalidValue;
 }
 
@@ -1016,81 +1079,90 @@ static cudaError_t launch_k2_any(const DecodeParams &p, size_t smem, cudaStream_
 
 // Shape rules and the shared-memory plan of the fused decode path.
 bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan) {
-    if (T < 1 || T > 4) return false;
-    if (c.act != COLI_ACT_BF16) return false;  // 16-bit block fixed point is exact for bf16 only
-    if (c.n_experts > 1024 || c.top_k * T > 32 || c.n_group > 32) return false;
-    if (c.hidden % 512 || c.hidden > 3 * NC * 4) return false;
-    // router blocks of 32 experts: groups are whole blocks, at most 32 candidates, K <= 8
-    if (c.n_experts % 32 || c.n_experts > 32 * RMAX_BLOCKS || c.top_k > 8) return false;
+    if (T < 1 || T > MAXTOK) return false;
+    if (c.act != COLI_ACT_BF16) return false;
+    if (c.wfmt != COLI_W_INT4 && c.wfmt != COLI_W_INT2) return false;
+    const int gs = c.group_size;                      // 0 or 64 (int4 only)
+    if (gs && (c.wfmt != COLI_W_INT4 || gs != 64 || c.hidden != 6144)) return false;
+    // router: blocks of 32 experts; groups are whole blocks; at most 32 candidates, K <= 8
+    if (c.n_experts % 32 || c.n_experts > 32 * RMAX_BLOCKS || c.top_k > 8 || c.n_group > 32) return false;
     {
-        const int gs = c.n_experts / c.n_group;
+        const int gsz = c.n_experts / c.n_group;
         const bool grouped = c.n_group > 1 && c.topk_group < c.n_group;
-        if (grouped && gs % 32) return false;
-        const int kept_blocks = grouped ? c.topk_group * gs / 32 : c.n_experts / 32;
+        if (grouped && gsz % 32) return false;
+        const int kept_blocks = grouped ? c.topk_group * gsz / 32 : c.n_experts / 32;
         if (kept_blocks * c.top_k > 32) return false;
     }
-    if (c.inter > 4 * NC) return false;  // phase-2 conversion: 4 elements per consumer thread
+    if (c.top_k * T > 32) return false;
+    // activations: 4 elements per consumer thread per 2048 (hidden 2048 or 6144)
+    if (c.hidden != 2048 && c.hidden != 6144) return false;
+    const int bits = c.wfmt;
+    const int rb_h = c.hidden * bits / 8, rb_i = c.inter * bits / 8;
+    const int cpc = bits == 4 ? 128 : 256;
+    if (c.hidden % cpc || c.inter % 8) return false;
+    // phase-1 stage: 16 rows x SK1 bytes, SK1 a multiple of 8 warps x 64 bytes, at most 1536
+    int nks1 = 1;
+    while (rb_h / nks1 > 1536 || rb_h % nks1) ++nks1;
+    const int SK1 = rb_h / nks1;
+    if (SK1 % (GW * 64)) return false;
+    // phase-2 stage: the CTA's rows x 512 bytes (8 chunks, one per warp of a half)
+    if (rb_i % 512) return false;
+    const int nch2 = rb_i / 64;
+    if (nch2 != 8 && nch2 != 16) return false;
+    const int SK2 = 512;
     const int sms = device_sm_count();
-    const int rb_h = c.hidden * c.wfmt / 8, rb_i = c.inter * c.wfmt / 8;
-    const int Lh = rb_h / 16, Li = rb_i / 16;
-    if (rb_h % 16 || rb_i % 16 || Lh % 32 || Li % 32 || NC % Li) return false;
-    if (NCW % PS1) return false;
-    const int P2 = NC / Li;
     const int rows2 = (c.hidden + sms - 1) / sms;
-    if (c.inter < sms || c.hidden < sms) return false;
-    if (rows2 > P2 * RPT2MAX) return false;
-    const int tmax = T <= 1 ? 1 : (T <= 2 ? 2 : 4);
-    if (!kernel_fits(c.wfmt, Lh / 32, T)) return false;
-    DecodePlan pl;
+    if (rows2 > 48 || c.inter / 8 < 1) return false;
+    if ((c.n_experts + sms - 1) / sms > 2) return false;  // at most two router rows per CTA
+    const int NB = 3 * T <= 8 ? 1 : 2;
+    const int mpc = bits == 4 ? 4 : 8;
+    const size_t colblk = 4 * 8 * mpc;
+    DecodePlan pl = {};
     pl.grid = sms;
-    pl.Lh = Lh; pl.Li = Li; pl.P1 = 0; pl.P2 = P2; pl.R1 = PS1;
-    // stage layout (phase 1: gate rows | up rows | sg | su; phase 2: down rows | sd)
-    const int scal1 = ((PS1 + 8 + 3) / 4) * 16;
-    const int scal2 = ((rows2 + 8 + 3) / 4) * 16;
-    pl.st_up = PS1 * rb_h;
-    pl.st_sg = 2 * PS1 * rb_h;
-    pl.st_su = pl.st_sg + scal1;
-    const int sb1 = pl.st_su + scal1;
-    pl.st_sd = rows2 * rb_i;
-    const int sb2 = pl.st_sd + scal2;
+    pl.SK1 = SK1;
+    pl.SK2 = SK2;
+    const int pad = gs ? 16 : ROWPAD;
+    const int st1 = SK1 + pad, st2 = SK2 + pad;
+    const int gps1 = gs ? SK1 * 8 / bits / gs : 0, gps2 = gs ? SK2 * 8 / bits / gs : 0;
+    const int sb1 = 16 * st1 + (gs ? 16 * 4 * gps1 : 64);  // 16 rows + their scales
+    pl.st_sd = rows2 * st2;
+    const int sb2 = pl.st_sd + (gs ? rows2 * 4 * gps2 : ((rows2 + 8 + 3) / 4) * 16);
     pl.SB = ((sb1 > sb2 ? sb1 : sb2) + 127) / 128 * 128;
-    // shared memory: barriers | routing cache | x (phase 1) or h (phase 2) | x scales |
-    // corrections | phase-2 partials | ring
-    size_t o = 1024;  // barriers (up to 64 stages)
-    pl.off_route = o; o += 4096;
-    pl.off_x = o;
-    const size_t xbytes = static_cast<size_t>(T) * c.hidden * 2 + static_cast<size_t>(T) * sizeof(RouteSmem);
-    const size_t hbytes = static_cast<size_t>(2) * tmax * c.inter * 4;  // two buffers of TMAX h rows
-    o += ((xbytes > hbytes ? xbytes : hbytes) + 127) / 128 * 128;
-    // x scales / corrections (phase 1) or h scales / corrections (phase 2)
-    const size_t xsb = static_cast<size_t>(T) * Lh * 4, hsb = static_cast<size_t>(2) * tmax * Li * 4;
-    pl.off_xs = o; o += (xsb > hsb ? xsb : hsb);
-    pl.off_xc = o; o += (xsb > 2 * hsb ? xsb : 2 * hsb);
+    size_t o = 1024;                                  // mbarriers (up to 60 stages)
+    pl.off_route = o; o += (sizeof(RouteCache) + 127) / 128 * 128;
+    pl.off_rtok = o; o += (static_cast<size_t>(T) * sizeof(RouteToken) + 127) / 128 * 128;
+    pl.off_gate = o; o += NCW * 2 * MAXTOK * 8 + NCW * MAXTOK * 4;
     o = (o + 127) / 128 * 128;
-    pl.red1_len = 0;
-    const int red2_len = P2 * RPT2MAX * tmax * (Li / 32);
-    pl.off_red = o; o += (static_cast<size_t>(red2_len) * 4 > NCW * 8 ? static_cast<size_t>(red2_len) * 4 : NCW * 8);
+    pl.off_red1 = o; o += static_cast<size_t>(NGRP) * GW * NB * 32 * 16;
+    o = (o + 127) / 128 * 128;
+    // activation slices (phase 1) | per-warp h slices, then the final reduction (phase 2)
+    const size_t xbytes = static_cast<size_t>(c.hidden / cpc) * 3 * T * colblk;
+    const size_t hbytes = static_cast<size_t>(NCW) * 3 * T * colblk;
+    const size_t rbytes = static_cast<size_t>(NCW) * 3 * NB * 32 * 16;
+    size_t abytes = xbytes > hbytes ? xbytes : hbytes;
+    abytes = abytes > rbytes ? abytes : rbytes;
+    pl.off_x = o; o += (abytes + 127) / 128 * 128;
     o = (o + 1023) / 1024 * 1024;
     pl.off_ring = o;
     const size_t budget = device_smem_optin() - 1024;
-    if (o + 2 * static_cast<size_t>(pl.SB) > budget) return false;
+    if (o + 3 * static_cast<size_t>(pl.SB) > budget) return false;
     pl.S = static_cast<int>((budget - o) / pl.SB);
-    if (pl.S > 8) pl.S = 8;
+    if (pl.S > 60) pl.S = 60;
     pl.smem = o + static_cast<size_t>(pl.S) * pl.SB;
     *plan = pl;
     return true;
 }
 
 static void fill_plan(DecodeParams &p, const DecodePlan &pl) {
-    p.grid = pl.grid; p.Lh = pl.Lh; p.Li = pl.Li; p.P1 = pl.P1; p.P2 = pl.P2; p.R1 = pl.R1;
-    p.S = pl.S; p.SB = pl.SB; p.st_up = pl.st_up; p.st_sg = pl.st_sg; p.st_su = pl.st_su; p.st_sd = pl.st_sd;
-    p.off_route = pl.off_route; p.off_x = pl.off_x; p.off_xs = pl.off_xs; p.off_xc = pl.off_xc;
-    p.off_red = pl.off_red; p.off_ring = pl.off_ring; p.red1_len = pl.red1_len;
+    p.grid = pl.grid; p.SK1 = pl.SK1; p.SK2 = pl.SK2; p.S = pl.S; p.SB = pl.SB; p.st_sd = pl.st_sd;
+    p.off_route = pl.off_route; p.off_rtok = pl.off_rtok; p.off_gate = pl.off_gate;
+    p.off_red1 = pl.off_red1; p.off_x = pl.off_x; p.off_ring = pl.off_ring;
 }
 
 cudaError_t launch_ffn_decode(DecodeParams p, const DecodePlan &pl, cudaStream_t st) {
     fill_plan(p, pl);
-    return launch_k2_any(p, pl.smem, st);
+    if (p.wait_cycles <= 0) p.wait_cycles = WAIT_CYCLES;
+    return launch_any(p, pl.smem, st);
 }
 
 }  // namespace coli

@@ -215,12 +215,20 @@ __global__ void __launch_bounds__(GU_THREADS) gateup_kernel(FfnParams p, int L, 
         const float *sg = reinterpret_cast<const float *>(ex.rec + p.off_sg);
         const float *su = reinterpret_cast<const float *>(ex.rec + p.off_su);
         uint4 qg[R], qu[R];
+        // group-scaled container: the scale of this lane's chunk (its group of 64 columns)
+        float lg[R], lu[R];
 #pragma unroll
         for (int r = 0; r < R; ++r) {
             const int i = i0 + slot * R + r;
+            lg[r] = lu[r] = 1.0f;
             if (active && i < p.I) {
                 qg[r] = ld_stream(wg + static_cast<size_t>(i) * p.rb_h + c * 16);
                 qu[r] = ld_stream(wu + static_cast<size_t>(i) * p.rb_h + c * 16);
+                if (p.group) {
+                    const size_t gi = static_cast<size_t>(i) * p.nsh + (c * NC) / p.group;
+                    lg[r] = __ldg(sg + gi);
+                    lu[r] = __ldg(su + gi);
+                }
             } else {
                 qg[r] = make_uint4(0, 0, 0, 0);
                 qu[r] = make_uint4(0, 0, 0, 0);
@@ -239,8 +247,8 @@ __global__ void __launch_bounds__(GU_THREADS) gateup_kernel(FfnParams p, int L, 
             float ag[R], au[R];
 #pragma unroll
             for (int r = 0; r < R; ++r) {
-                ag[r] = active ? dot_chunk<FMT>(opaque(qg[r]), xr) : 0.f;
-                au[r] = active ? dot_chunk<FMT>(opaque(qu[r]), xr) : 0.f;
+                ag[r] = active ? lg[r] * dot_chunk<FMT>(opaque(qg[r]), xr) : 0.f;
+                au[r] = active ? lu[r] * dot_chunk<FMT>(opaque(qu[r]), xr) : 0.f;
                 ag[r] = warp_sum(ag[r], L);
                 au[r] = warp_sum(au[r], L);
             }
@@ -271,8 +279,8 @@ __global__ void __launch_bounds__(GU_THREADS) gateup_kernel(FfnParams p, int L, 
                 for (int r = 0; r < R; ++r) {
                     const int i = i0 + slot * R + r;
                     if (i < p.I) {
-                        const float g = sg[i] * ag[r];
-                        const float u = su[i] * au[r];
+                        const float g = (p.group ? 1.0f : sg[i]) * ag[r];
+                        const float u = (p.group ? 1.0f : su[i]) * au[r];
                         p.h[static_cast<size_t>(hrow) * p.I + i] = (g / (1.0f + expf(-g))) * u;
                     }
                 }
@@ -309,11 +317,14 @@ __global__ void __launch_bounds__(DN_THREADS) down_kernel(FfnParams p, int L, in
             const uint8_t *wd = ex.rec + p.off_wd;
             const float *sd = reinterpret_cast<const float *>(ex.rec + p.off_sd);
             uint4 qd[R];
+            float ld[R];  // group-scaled container: the scale of this lane's chunk
 #pragma unroll
             for (int r = 0; r < R; ++r) {
                 const int j = j0 + slot * R + r;
                 qd[r] = (active && j < p.H) ? ld_stream(wd + static_cast<size_t>(j) * p.rb_i + c * 16)
                                             : make_uint4(0, 0, 0, 0);
+                ld[r] = (p.group && active && j < p.H) ? __ldg(sd + static_cast<size_t>(j) * p.nsi + (c * NC) / p.group)
+                                                       : 1.0f;
             }
             for (int q = 0; q < ex.count; ++q) {
                 int tok, hrow;
@@ -324,7 +335,7 @@ __global__ void __launch_bounds__(DN_THREADS) down_kernel(FfnParams p, int L, in
                 float a[R];
 #pragma unroll
                 for (int r = 0; r < R; ++r) {
-                    a[r] = active ? dot_chunk<FMT>(opaque(qd[r]), hr) : 0.f;
+                    a[r] = active ? ld[r] * dot_chunk<FMT>(opaque(qd[r]), hr) : 0.f;
                     a[r] = warp_sum(a[r], L);
                 }
                 if (nwarp_row > 1) {
@@ -347,7 +358,7 @@ __global__ void __launch_bounds__(DN_THREADS) down_kernel(FfnParams p, int L, in
 #pragma unroll
                     for (int r = 0; r < R; ++r) {
                         const int j = j0 + slot * R + r;
-                        if (j < p.H) acc[tok * rpp + slot * R + r] += wt * (sd[j] * a[r]);
+                        if (j < p.H) acc[tok * rpp + slot * R + r] += wt * ((p.group ? 1.0f : sd[j]) * a[r]);
                     }
                 }
             }

@@ -15,6 +15,8 @@ struct FfnParams {
     int H, I, E, K, T, S;              // S = n_shared (0 or 1); shared inter == I
     int fmt;                           // 4, 8, 2
     int act;                           // coli_act of x
+    int group;                         // 0: per-row scales; 64: per 64 columns of a row
+    int nsh, nsi;                      // scales per gate/up row and per down row
     const uint8_t *experts;            // E records
     size_t stride;                     // record stride, bytes
     const uint8_t *shared;             // shared record or nullptr
@@ -34,21 +36,19 @@ struct FfnParams {
 // Workspace header (first 256 bytes): error word, then counters of the fused decode path.
 // All must be zero before the first call on a workspace (coli_moe_clear_error zeroes them);
 // the kernels leave them zero after every complete call.
-constexpr int WS_ERR = 0, WS_GBAR = 64, WS_GDEP = 96, WS_ROUTE_CNT = 128, WS_TOK_CNT = 160;  // 8 token words
+constexpr int WS_ERR = 0, WS_GBAR = 64, WS_GDEP = 96;
 constexpr int WS_HEADER = 256;
 
-// Shared-memory plan of the fused decode FFN kernel (decode.cu).
+// Shared-memory plan of the fused decode kernel (decode.cu).
 struct DecodePlan {
-    int grid, Lh, Li, P1, P2, R1, S, SB;
-    int st_up, st_sg, st_su, st_sd;       // byte offsets inside a ring stage
-    size_t off_route, off_x, off_xs, off_xc, off_red, off_ring, smem;
-    int red1_len;
+    int grid, S, SB, SK1, SK2, st_sd;                 // ring: S stages of SB bytes
+    size_t off_route, off_rtok, off_gate, off_red1, off_x, off_ring, smem;
 };
 
-// Parameters of the fused decode path (router kernel K1 and FFN kernel K2).
+// Parameters of the fused decode kernel.
 struct DecodeParams {
     FfnParams f;
-    // K1: gate + route + group
+    // gate + route + group
     const float *Wr, *bias;
     float *logits;
     int32_t *ids;
@@ -56,13 +56,13 @@ struct DecodeParams {
     int32_t *f_counts, *f_offsets, *f_perm, *f_unique, *f_nuniq;
     double rsf;
     int G, TG;
-    unsigned *tok_cnt, *route_cnt, *gbar, *gdep;
-    int route_here;  // 1: the FFN kernel routes from logits; 0: routing arrays are inputs
-    // K2 plan (copied from DecodePlan)
-    int grid, Lh, Li, P1, P2, R1, S, SB;
-    int st_up, st_sg, st_su, st_sd;
-    size_t off_route, off_x, off_xs, off_xc, off_red, off_ring;
-    int red1_len;
+    unsigned *gbar, *gdep;
+    int route_here;         // 1: the kernel routes from its own logits; 0: routing arrays are inputs
+    long long wait_cycles;  // bound of every device-side wait (0: the default, ~2 s)
+    unsigned gate_extra;    // added to the grid-barrier targets (nonzero only to test the bound)
+    // plan (copied from DecodePlan)
+    int grid, S, SB, SK1, SK2, st_sd;
+    size_t off_route, off_rtok, off_gate, off_red1, off_x, off_ring;
 };
 
 bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan);

@@ -332,39 +332,60 @@ __global__ void __launch_bounds__(128) route_kernel(const float *__restrict__ lo
 }
 
 // ---------------------------------------------------------------- a3 group -----------------
-// One CTA.  Histogram with shared-memory integer atomics, exclusive scan, then a stable
-// placement pass over chunks of blockDim slots: warp peers by __match_any_sync give the rank
-// inside a warp, per-warp per-expert counts give the rank across warps.
-__global__ void __launch_bounds__(1024) group_kernel(const int32_t *__restrict__ ids, int n,
-                                                     int E, int32_t *__restrict__ counts,
-                                                     int32_t *__restrict__ offsets,
-                                                     int32_t *__restrict__ perm,
-                                                     int32_t *__restrict__ unique,
-                                                     int32_t *__restrict__ n_unique,
-                                                     int *__restrict__ err) {
+// One CTA of 32 warps; warp w owns the contiguous slot range [w n / 32, (w + 1) n / 32).
+// Pass 1: each warp counts its range per expert (32 slots at a time, peers by __match_any_sync;
+// the leader of each id adds the peer count).  Pass 2: per expert, an exclusive scan over the
+// warps and an exclusive scan of the expert totals give every (warp, expert) its first position.
+// Pass 3: each warp places its slots in order (rank among the batch's peers plus its running
+// cursor).  Stable: a warp's slots keep their order, and warp w's slots of an expert follow those
+// of warps < w.  Only warp-level synchronisation inside the passes.
+constexpr int GROUP_WARPS = 32;
+
+__global__ void __launch_bounds__(GROUP_WARPS * 32) group_kernel(const int32_t *__restrict__ ids, int n,
+                                                                 int E, int32_t *__restrict__ counts,
+                                                                 int32_t *__restrict__ offsets,
+                                                                 int32_t *__restrict__ perm,
+                                                                 int32_t *__restrict__ unique,
+                                                                 int32_t *__restrict__ n_unique,
+                                                                 int *__restrict__ err) {
     extern __shared__ int sm[];
-    const int nw = blockDim.x >> 5;
-    int *cnt = sm;             // [E]
-    int *cursor = sm + E;      // [E]
-    int *wc = sm + 2 * E;      // [nw][E]
+    int *wc = sm;                // [GROUP_WARPS][E]: counts, then first positions, then cursors
+    int *tot = sm + GROUP_WARPS * E;  // [E]
     __shared__ int bad;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int s_lo = static_cast<int>(static_cast<long>(n) * warp / GROUP_WARPS);
+    const int s_hi = static_cast<int>(static_cast<long>(n) * (warp + 1) / GROUP_WARPS);
     if (tid == 0) bad = 0;
-    for (int e = tid; e < E; e += blockDim.x) cnt[e] = 0;
-    for (int i = tid; i < nw * E; i += blockDim.x) wc[i] = 0;
+    for (int i = tid; i < GROUP_WARPS * E; i += blockDim.x) wc[i] = 0;
     __syncthreads();
-    for (int s = tid; s < n; s += blockDim.x) {
-        const int id = ids[s];
-        if (id >= 0 && id < E) atomicAdd(&cnt[id], 1);
-        else bad = 1;
+    const unsigned lt = (1u << lane) - 1u;
+    int *mine = wc + warp * E;
+    for (int base = s_lo; base < s_hi; base += 32) {
+        const int s = base + lane;
+        const int id = s < s_hi ? ids[s] : -1;
+        const bool ok = id >= 0 && id < E;
+        if (s < s_hi && !ok) bad = 1;
+        const unsigned peers = __match_any_sync(FULL, ok ? id : -1 - lane);
+        if (ok && (peers & lt) == 0) mine[id] += __popc(peers);
+        __syncwarp();
     }
     __syncthreads();
-    // exclusive scans of counts and of the non-empty flags, by warp 0 (E <= 1024)
+    for (int e = tid; e < E; e += blockDim.x) {  // exclusive scan over the warps, per expert
+        int run = 0;
+        for (int w = 0; w < GROUP_WARPS; ++w) {
+            const int c = wc[w * E + e];
+            wc[w * E + e] = run;
+            run += c;
+        }
+        tot[e] = run;
+    }
+    __syncthreads();
+    // exclusive scans of the totals and of the non-empty flags, by warp 0 (E <= 1024)
     if (warp == 0) {
         const int per = (E + 31) / 32;
         const int b = lane * per;
         int sc = 0, su = 0;
-        for (int e = b; e < b + per && e < E; ++e) { sc += cnt[e]; su += cnt[e] > 0; }
+        for (int e = b; e < b + per && e < E; ++e) { sc += tot[e]; su += tot[e] > 0; }
         int ic = sc, iu = su;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
@@ -374,10 +395,11 @@ __global__ void __launch_bounds__(1024) group_kernel(const int32_t *__restrict__
         int rc = ic - sc, ru = iu - su;
         for (int e = b; e < b + per && e < E; ++e) {
             offsets[e] = rc;
-            cursor[e] = rc;
-            counts[e] = cnt[e];
-            if (cnt[e] > 0) unique[ru++] = e;
-            rc += cnt[e];
+            counts[e] = tot[e];
+            if (tot[e] > 0) unique[ru++] = e;
+            const int c = tot[e];
+            tot[e] = rc;  // first position of expert e
+            rc += c;
         }
         if (lane == 31) {
             offsets[E] = ic;
@@ -386,29 +408,19 @@ __global__ void __launch_bounds__(1024) group_kernel(const int32_t *__restrict__
         }
     }
     __syncthreads();
-    const unsigned lt = (1u << lane) - 1u;
-    for (int base = 0; base < n; base += blockDim.x) {
-        const int s = base + tid;
-        const int id = (s < n) ? ids[s] : -1;
+    for (int i = tid; i < GROUP_WARPS * E; i += blockDim.x) wc[i] += tot[i % E];
+    __syncthreads();
+    for (int base = s_lo; base < s_hi; base += 32) {
+        const int s = base + lane;
+        const int id = s < s_hi ? ids[s] : -1;
         const bool ok = id >= 0 && id < E;
-        const int key = ok ? id : -1 - lane;
-        const unsigned peers = __match_any_sync(FULL, key);
-        const int rank = __popc(peers & lt);
-        if (ok && rank == 0) wc[warp * E + id] = __popc(peers);
-        __syncthreads();
-        if (ok) {
-            int pos = cursor[id] + rank;
-            for (int w = 0; w < warp; ++w) pos += wc[w * E + id];
-            perm[pos] = s;
-        }
-        __syncthreads();
-        for (int e = tid; e < E; e += blockDim.x) {
-            int add = 0;
-            for (int w = 0; w < nw; ++w) { add += wc[w * E + e]; wc[w * E + e] = 0; }
-            cursor[e] += add;
-        }
-        __syncthreads();
+        const unsigned peers = __match_any_sync(FULL, ok ? id : -1 - lane);
+        if (ok) perm[mine[id] + __popc(peers & lt)] = s;
+        __syncwarp();
+        if (ok && (peers & lt) == 0) mine[id] += __popc(peers);
+        __syncwarp();
     }
+    __syncthreads();
     // slots with a bad id are not placed; the tail of perm is marked
     if (tid == 0 && bad) {
         atomicOr(err, COLI_DEVERR_EXPERT_ID);
@@ -468,12 +480,11 @@ cudaError_t launch_group(const coli_moe_config &c, const int32_t *ids, int T, in
                          int32_t *offsets, int32_t *perm, int32_t *unique, int32_t *n_unique,
                          int *err, cudaStream_t st) {
     const int n = T * c.top_k, E = c.n_experts;
-    const int threads = n <= 256 ? 256 : 1024;
-    const size_t smem = static_cast<size_t>(2 + threads / 32) * E * sizeof(int);
+    const size_t smem = static_cast<size_t>(GROUP_WARPS + 1) * E * sizeof(int);
     cudaError_t e = cudaFuncSetAttribute(group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    group_kernel<<<1, threads, smem, st>>>(ids, n, E, counts, offsets, perm, unique, n_unique, err);
+    group_kernel<<<1, GROUP_WARPS * 32, smem, st>>>(ids, n, E, counts, offsets, perm, unique, n_unique, err);
     return cudaGetLastError();
 }
 

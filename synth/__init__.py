@@ -63,6 +63,7 @@ class Workload:
     seed: int
     zipf_s: float = 0.0      # > 0: Zipf popularity offsets in the selection bias
     n_layers: int = 1        # consecutive layers resident at once (chained workloads)
+    group: int = 0           # 0: one scale per weight row; g: one per g consecutive columns
 
     def replace(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
@@ -88,6 +89,9 @@ WORKLOADS: Dict[str, Workload] = {
     # ones, as on the 2048-token layer, in a 1.2 GB layer (small enough for ncu captures)
     "glm_zipf_e64": Workload("glm_zipf_e64", fmt=4, tokens=(512,), seed=2, zipf_s=1.1,
                              **dict(_GLM, n_experts=64)),
+    # the group-scaled int4 container (one scale per 64 consecutive weights of a row) at the
+    # GLM-5.2 decode shape: the pages' recommended GLM-5.2 build
+    "glm_gs64": Workload("glm_gs64", fmt=4, tokens=(1, 4), seed=5, group=64, **_GLM),
     "glm_int8": Workload("glm_int8", fmt=8, tokens=(64,), seed=4, n_layers=4, **_GLM),
     "glm_int2": Workload("glm_int2", fmt=2, tokens=(64,), seed=4, n_layers=4, **_GLM),
 }
@@ -97,17 +101,20 @@ def _row_bytes(n: int, fmt: int) -> int:
     return n * fmt // 8
 
 
-def record_layout(hidden: int, inter: int, fmt: int) -> dict:
-    """Byte offsets of the six parts of one record and the padded record size."""
+def record_layout(hidden: int, inter: int, fmt: int, group: int = 0) -> dict:
+    """Byte offsets of the six parts of one record and the padded record size.  Scales are one
+    float32 per row, or with `group` one per `group` consecutive columns of a row."""
     rh, ri = _row_bytes(hidden, fmt), _row_bytes(inter, fmt)
+    nh = hidden // group if group else 1
+    ni = inter // group if group else 1
     o = {}
     o["wg"] = 0
     o["wu"] = inter * rh
     o["wd"] = 2 * inter * rh
     o["sg"] = o["wd"] + hidden * ri
-    o["su"] = o["sg"] + 4 * inter
-    o["sd"] = o["su"] + 4 * inter
-    o["bytes"] = o["sd"] + 4 * hidden
+    o["su"] = o["sg"] + 4 * inter * nh
+    o["sd"] = o["su"] + 4 * inter * nh
+    o["bytes"] = o["sd"] + 4 * hidden * ni
     o["stride"] = (o["bytes"] + 255) // 256 * 256
     o["row_bytes_h"], o["row_bytes_i"] = rh, ri
     return o
@@ -123,15 +130,18 @@ def _gen(device, *key: int) -> torch.Generator:
     return g
 
 
-def quantize_rows(w: torch.Tensor, fmt: int):
-    """Per-row symmetric quantisation: returns (codes int8 [R,C], scales float32 [R])."""
+def quantize_rows(w: torch.Tensor, fmt: int, group: int = 0):
+    """Symmetric quantisation per row (group 0: codes int8 [R,C], scales float32 [R]) or per
+    group of `group` consecutive columns of a row (scales float32 [R, C/group])."""
     qmax, qmin = QMAX[fmt], QMIN[fmt]
-    absmax = w.abs().amax(dim=1)
+    R, Cn = w.shape
+    wg = w.reshape(R, Cn // group, group) if group else w.reshape(R, 1, Cn)
+    absmax = wg.abs().amax(dim=2)
     scale = (absmax / qmax).to(torch.float32)
     safe = torch.where(scale > 0, scale, torch.ones_like(scale))
-    q = torch.round(w / safe[:, None]).clamp_(qmin, qmax)
-    q = torch.where(scale[:, None] > 0, q, torch.zeros_like(q))
-    return q.to(torch.int8), scale
+    q = torch.round(wg / safe[:, :, None]).clamp_(qmin, qmax)
+    q = torch.where(scale[:, :, None] > 0, q, torch.zeros_like(q))
+    return q.reshape(R, Cn).to(torch.int8), (scale if group else scale[:, 0])
 
 
 def pack_codes(q: torch.Tensor, fmt: int) -> torch.Tensor:
@@ -152,20 +162,20 @@ def pack_codes(q: torch.Tensor, fmt: int) -> torch.Tensor:
 
 
 def _one_record(hidden: int, inter: int, fmt: int, g: torch.Generator, device,
-                keep_codes: bool = False):
-    lay = record_layout(hidden, inter, fmt)
+                keep_codes: bool = False, group: int = 0):
+    lay = record_layout(hidden, inter, fmt, group)
     rec = torch.zeros(lay["stride"], dtype=torch.uint8, device=device)
     parts = {}
     for name, (r, c) in (("g", (inter, hidden)), ("u", (inter, hidden)), ("d", (hidden, inter))):
         w = torch.randn(r, c, generator=g, device=device, dtype=torch.float32) * WEIGHT_STD
-        q, s = quantize_rows(w, fmt)
+        q, s = quantize_rows(w, fmt, group)
         parts[name] = (q, s)
     rec[lay["wg"]:lay["wu"]] = pack_codes(parts["g"][0], fmt).reshape(-1)
     rec[lay["wu"]:lay["wd"]] = pack_codes(parts["u"][0], fmt).reshape(-1)
     rec[lay["wd"]:lay["sg"]] = pack_codes(parts["d"][0], fmt).reshape(-1)
-    rec[lay["sg"]:lay["su"]] = parts["g"][1].view(torch.uint8)
-    rec[lay["su"]:lay["sd"]] = parts["u"][1].view(torch.uint8)
-    rec[lay["sd"]:lay["bytes"]] = parts["d"][1].view(torch.uint8)
+    rec[lay["sg"]:lay["su"]] = parts["g"][1].contiguous().view(torch.uint8).reshape(-1)
+    rec[lay["su"]:lay["sd"]] = parts["u"][1].contiguous().view(torch.uint8).reshape(-1)
+    rec[lay["sd"]:lay["bytes"]] = parts["d"][1].contiguous().view(torch.uint8).reshape(-1)
     return (rec, parts) if keep_codes else (rec, None)
 
 
@@ -176,14 +186,14 @@ def make_expert_records(wl: Workload, device="cpu", layer: int = 0,
 
     With keep_codes, also returns {e: {"g"|"u"|"d": (codes int8, scales f32)}} -- the int8
     container view of the same weights, used by the container pins."""
-    lay = record_layout(wl.hidden, wl.inter, wl.fmt)
+    lay = record_layout(wl.hidden, wl.inter, wl.fmt, wl.group)
     E = wl.n_experts
     recs = out if out is not None else torch.zeros(E, lay["stride"], dtype=torch.uint8,
                                                     device=device)
     codes = {}
     for e in (range(E) if experts is None else experts):
         g = _gen(device, wl.seed, layer, 1, e)
-        rec, parts = _one_record(wl.hidden, wl.inter, wl.fmt, g, device, keep_codes)
+        rec, parts = _one_record(wl.hidden, wl.inter, wl.fmt, g, device, keep_codes, wl.group)
         recs[e].copy_(rec)
         if keep_codes:
             codes[e] = parts
@@ -195,7 +205,7 @@ def make_shared_record(wl: Workload, device="cpu", layer: int = 0, keep_codes: b
     if wl.n_shared == 0:
         return (None, None) if keep_codes else None
     g = _gen(device, wl.seed, layer, 2)
-    rec, parts = _one_record(wl.hidden, wl.shared_inter, wl.fmt, g, device, keep_codes)
+    rec, parts = _one_record(wl.hidden, wl.shared_inter, wl.fmt, g, device, keep_codes, wl.group)
     return (rec, parts) if keep_codes else rec
 
 

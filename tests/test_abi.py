@@ -45,13 +45,13 @@ def test_workload_configs_are_accepted(name):
     wl = synth.WORKLOADS[name]
     cfg = q.config_for(wl)
     q.coli_moe_check_config(cfg)
-    assert q.coli_moe_record_bytes(wl.hidden, wl.inter, wl.fmt) == \
-        synth.record_layout(wl.hidden, wl.inter, wl.fmt)["bytes"]
+    assert q.coli_moe_record_bytes(wl.hidden, wl.inter, wl.fmt, wl.group) == \
+        synth.record_layout(wl.hidden, wl.inter, wl.fmt, wl.group)["bytes"]
     assert q.coli_moe_workspace_size(cfg, 64) % 256 == 0
 
 
 @pytest.mark.parametrize("field,value,status", [
-    ("wfmt", 3, 1), ("act", 5, 1), ("n_group", 3, 2), ("topk_group", 9, 2),
+    ("wfmt", 3, 1), ("act", 5, 1), ("group_size", 32, 1), ("group_size", -64, 1), ("n_group", 3, 2), ("topk_group", 9, 2),
     ("top_k", 33, 4), ("top_k", 200, 2), ("hidden", 100, 2), ("n_shared", 2, 4), ("n_experts", 2048, 4), ("n_experts", 250, 2),
     ("shared_inter", 1024, 4), ("routed_scaling", 0.0, 1),
 ])
@@ -125,3 +125,13 @@ def test_dispatch_rule_on_the_host():
             assert q.coli_moe_layer_kernels(cfg, T) == 5, (name, T)
     odd = q.config_for(synth.WORKLOADS["tiny"].replace(inter=64, shared_inter=64))
     assert q.coli_moe_layer_kernels(odd, 32) == 5  # inter not a multiple of 128
+
+
+def test_group_scaled_container_is_int4_only():
+    wl = synth.WORKLOADS["glm_int8"].replace(group=64)
+    with pytest.raises(q.ColiError) as ei:
+        q.coli_moe_check_config(q.config_for(wl))
+    assert ei.value.status == 4
+    with pytest.raises(q.ColiError):
+        q.coli_moe_record_bytes(6144, 2048, 8, 64)
+    assert q.coli_moe_record_bytes(6144, 2048, 4, 64) == 21_233_664

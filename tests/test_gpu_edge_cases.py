@@ -150,3 +150,36 @@ def test_layer_activation_outliers(T, factor):
     err = normwise_err(out.cpu().numpy()[toks], ref)
     print(f"T={T} outlier x{factor:g}: normwise error {err:.2e}")
     assert err <= (TOL_GEMV if fused else TOL_TC_OUTLIER), err
+
+
+def test_fused_kernel_waits_run_out_and_the_workspace_recovers():
+    """Every device-side wait of the fused decode kernel is bounded.  With its grid-barrier
+    targets made unreachable and a short bound, the call still completes (no trap, no hang),
+    reports COLI_DEVERR_TIMEOUT, and after coli_moe_clear_error the same workspace serves a
+    normal call whose output matches the oracle."""
+    import time
+    L = layer_for("olmoe")
+    wl = L.wl
+    cfg = q.config_for(wl)
+    T = 1
+    assert q.coli_moe_layer_kernels(cfg, T) == 1
+    x = synth.make_activations(wl, T, device="cuda", step=77)
+    ws = torch.empty(q.coli_moe_workspace_size(cfg, T), dtype=torch.uint8, device="cuda")
+    out = torch.empty(T, wl.hidden, device="cuda")
+    q.coli_moe_clear_error(ws)
+    q.coli_moe_debug_set_wait(1_000_000, True)  # ~0.5 ms per wait at the B200's clock
+    try:
+        t0 = time.time()
+        q.coli_moe_layer(cfg, L.weights(), x, T, out, None, None, ws)
+        err = q.coli_moe_error_word(ws)
+        elapsed = time.time() - t0
+    finally:
+        q.coli_moe_debug_set_wait(0, False)
+    assert err & q.DEVERR_TIMEOUT, err
+    assert elapsed < 5.0, elapsed
+    q.coli_moe_clear_error(ws)
+    assert (ws[:256] == 0).all()
+    q.coli_moe_layer(cfg, L.weights(), x, T, out, None, None, ws)
+    assert q.coli_moe_error_word(ws) == 0
+    ref, _, _, _ = oracle_layer_tokens(L, x.cpu(), range(T))
+    assert normwise_err(out.cpu().numpy(), ref) <= TOL_GEMV

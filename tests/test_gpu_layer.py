@@ -176,7 +176,9 @@ def _gpu_group(cfg, ids_dev, T, E, ws):
                                             ("olmoe", 32, "oracle"), ("glm_decode", 4, "oracle"),
                                             ("glm_decode", 4, "one_expert"),
                                             ("glm_decode", 1, "oracle"),
-                                            ("glm_decode", 16, "one_expert")])
+                                            ("glm_decode", 16, "one_expert"),
+                                            ("glm_gs64", 4, "one_expert"),
+                                            ("glm_gs64", 3, "oracle")])
 def test_ffn_matches_oracle(name, T, routing):
     L = layer_for(name)
     wl = L.wl
@@ -231,7 +233,8 @@ def test_ffn_flags_bad_unique_list():
 @pytest.mark.parametrize("name,T", [("tiny", 8), ("tiny", 1), ("tiny", 37), ("olmoe", 1),
                                     ("olmoe", 32), ("olmoe", 3), ("glm_decode", 1),
                                     ("glm_decode", 2), ("glm_decode", 3), ("glm_decode", 4),
-                                    ("glm_decode", 5)])
+                                    ("glm_decode", 5), ("glm_gs64", 1), ("glm_gs64", 2),
+                                    ("glm_gs64", 4), ("glm_gs64", 5), ("glm_gs64", 24)])
 def test_layer_matches_oracle(name, T):
     L = layer_for(name)
     x = synth.make_activations(L.wl, T, device="cuda", step=T)
@@ -261,7 +264,8 @@ def test_layer_alternate_containers_sampled(name):
 def test_decode_shapes_take_fused_kernel():
     """Decode shapes run as one fused launch (a fall back to the five-kernel path would give the
     same outputs, only slower, so the launch count is checked here)."""
-    for name, Ts in (("glm_decode", (1, 2, 3, 4)), ("olmoe", (1, 2, 4)), ("glm_int2", (1, 4))):
+    for name, Ts in (("glm_decode", (1, 2, 3, 4)), ("olmoe", (1, 2, 4)), ("glm_int2", (1, 4)),
+                     ("glm_gs64", (1, 2, 3, 4))):
         cfg = q.config_for(synth.WORKLOADS[name])
         for T in Ts:
             assert q.coli_moe_layer_kernels(cfg, T) == 1, (name, T)

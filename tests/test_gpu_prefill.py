@@ -58,7 +58,7 @@ def _routing(L, ocfg, x, T, routing):
 
 
 # (workload, tokens, routing): chunks of 1..96 tokens with ragged tails; one expert with 128 and
-# with 160 tokens (two chunks each); one token above the fused decode limit (5: chunks of one
+# with 160 tokens (two chunks each, the second ragged); one token above the fused decode limit (5: chunks of one
 # token); f32 activations and four gate/up m-blocks (tiny_wide); no shared expert (olmoe).
 CASES = [("glm_decode", 96, "oracle"), ("glm_decode", 300, "oracle"), ("glm_decode", 160, "one_expert"),
          ("glm_decode", 128, "one_expert"), ("glm_decode", 65, "oracle"), ("glm_decode", 5, "oracle"),

@@ -408,3 +408,80 @@ def test_residual_f32_is_ieee_sum():
     out = rng.normal(0, 1e-3, 4096).astype(np.float32)
     np.testing.assert_array_equal(oracle.residual(cfg, x, out), x + out)
 
+
+
+# ------------------------------------------------------------------ group-scaled int4 -------
+# The group-scaled container (one scale per 64 consecutive weights of a row; JustVugg/colibri
+# README, "Get started -> 2. Get the model" recommends the gs64 GLM-5.2 build).
+
+def test_record_bytes_gs64_glm():
+    # codes as in the per-row container (18,874,368 B) + float32 scales: Wg and Wu 2048 rows x
+    # 96 groups each, Wd 6144 rows x 32 groups -> 4 * (2 * 196,608 + 196,608) = 2,359,296 B
+    assert oracle.record_bytes(6144, 2048, 4, 64) == 18_874_368 + 2_359_296 == 21_233_664
+    assert synth.record_layout(6144, 2048, 4, 64)["bytes"] == 21_233_664
+    with pytest.raises(ValueError):
+        oracle.record_bytes(6144 + 32, 2048, 4, 64)  # a group must not straddle a row end
+
+
+def _np_expert_grouped(parts, x, group):
+    """numpy float64 reference over the generator's codes x group scales (each scale repeated
+    over its `group` columns)."""
+    def w(name):
+        q, s = parts[name]
+        return q.numpy().astype(np.float64) * np.repeat(s.numpy().astype(np.float64), group, axis=1)
+    gg = w("g") @ x
+    a = gg / (1.0 + np.exp(-gg)) * (w("u") @ x)
+    return w("d") @ a
+
+
+def test_expert_gs64_against_numpy():
+    wl = synth.WORKLOADS["tiny"].replace(group=64)
+    recs, codes = synth.make_expert_records(wl, experts=[3], keep_codes=True)
+    assert codes[3]["g"][1].shape == (wl.inter, wl.hidden // 64)
+    cfg = oracle.make_cfg(wl)
+    x = np.random.default_rng(4).standard_normal(wl.hidden)
+    y = oracle.expert(cfg, recs[3], wl.inter, x)
+    ref = _np_expert_grouped(codes[3], x, 64)
+    np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-15 * np.abs(ref).max())
+
+
+def test_expert_gs64_with_equal_group_scales_is_the_per_row_expert():
+    """A group-scaled record whose group scales all equal their row's scale dequantises to the
+    same weights as the per-row record: the outputs agree bit for bit."""
+    wl = synth.WORKLOADS["tiny"]
+    H, I = wl.hidden, wl.inter
+    recs, codes = synth.make_expert_records(wl, experts=[1], keep_codes=True)
+    lay_r = synth.record_layout(H, I, 4)
+    lay_g = synth.record_layout(H, I, 4, 64)
+    rec_g = np.zeros(lay_g["stride"], np.uint8)
+    rec_r = recs[1].numpy()
+    rec_g[:lay_g["sg"]] = rec_r[:lay_r["sg"]]  # the codes are the same bytes
+    for name, key, cols in (("g", "sg", H), ("u", "su", H), ("d", "sd", I)):
+        s = np.repeat(codes[1][name][1].numpy()[:, None], cols // 64, axis=1).astype(np.float32)
+        b = s.reshape(-1).view(np.uint8)
+        rec_g[lay_g[key]:lay_g[key] + b.size] = b
+    x = np.random.default_rng(5).standard_normal(H)
+    y_r = oracle.expert(oracle.make_cfg(wl), rec_r, I, x)
+    y_g = oracle.expert(oracle.make_cfg(wl.replace(group=64)), rec_g, I, x)
+    np.testing.assert_array_equal(y_g, y_r)
+
+
+def test_expert_gs64_group_scales_act_on_their_group_only():
+    """Doubling one group's down-projection scale in every row changes y by exactly the part of
+    the dot product that the group's 64 columns carry: y' - y equals y restricted to that group
+    (computed with the other group's scales set to zero)."""
+    wl = synth.WORKLOADS["tiny"].replace(group=64)   # inter 128: two groups per down row
+    cfg = oracle.make_cfg(wl)
+    recs = synth.make_expert_records(wl, experts=[2])
+    rec = recs[2].numpy().copy()
+    lay = synth.record_layout(wl.hidden, wl.inter, 4, 64)
+    x = np.random.default_rng(6).standard_normal(wl.hidden)
+    y = oracle.expert(cfg, rec, wl.inter, x)
+    sd = rec[lay["sd"]:lay["bytes"]].view(np.float32).reshape(wl.hidden, 2)
+    r_dbl = rec.copy()
+    r_dbl[lay["sd"]:lay["bytes"]] = (sd * np.array([1.0, 2.0], np.float32)).reshape(-1).view(np.uint8)
+    r_only = rec.copy()
+    r_only[lay["sd"]:lay["bytes"]] = (sd * np.array([0.0, 1.0], np.float32)).reshape(-1).view(np.uint8)
+    d = oracle.expert(cfg, r_dbl, wl.inter, x) - y
+    np.testing.assert_allclose(d, oracle.expert(cfg, r_only, wl.inter, x), rtol=1e-12,
+                               atol=1e-14 * np.abs(y).max())
