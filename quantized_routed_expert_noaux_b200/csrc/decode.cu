@@ -52,7 +52,6 @@ constexpr int GW = 8;                // warps of a phase-1 group
 constexpr int NGRP = NCW / GW;       // phase-1 groups
 constexpr int MAXTOK = 4;            // tokens of the fused path
 constexpr int MAXWE = 33;            // work experts: the shared one + up to 32 unique routed
-constexpr int ROWPAD = 64;           // bytes added to each staged row (conflict-free 16-byte loads)
 // named barriers: 0 __syncthreads, 1 all consumers, 2.. group full, 4.. group reduction free
 constexpr int BAR_CONS = 1, BAR_GFULL = 2, BAR_GFREE = 4;
 constexpr long long WAIT_CYCLES = 4000000000LL;  // ~2 s at 1.9 GHz: bound of every spin-wait
@@ -66,6 +65,9 @@ __device__ __forceinline__ void mbar_init(uint32_t a, uint32_t count) {
 }
 __device__ __forceinline__ void mbar_arrive(uint32_t a) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(a) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cnt(uint32_t a, uint32_t count) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(a), "r"(count) : "memory");
 }
 __device__ __forceinline__ void mbar_expect_tx(uint32_t a, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(a), "r"(bytes) : "memory");
@@ -163,32 +165,6 @@ template <> struct Fmt<2> {
         m = 2 * i + (k >> 1);
         half = k & 1;
         byte = (p >> 2) & 3;
-    }
-};
-
-// The group-scaled container (scales per 64 consecutive codes, int4) keeps every MMA inside one
-// group: MMA m of a chunk takes codes [32 m, 32 m + 32), thread tig the 8 codes 32 m + 8 tig +
-// (0..7) (word m of its A registers, read from byte 16 m + 4 tig); MMAs 2u and 2u + 1 are group
-// u of the chunk.  With per-row scales a thread reads one 16-byte run instead (Fmt::place).
-template <int FMT, int GS> struct Place {
-    __device__ static __forceinline__ void at(int p, int &tig, int &m, int &half, int &byte) {
-        Fmt<FMT>::place(p, tig, m, half, byte);
-    }
-    // the thread's 16 bytes of A for a 64-byte chunk starting at `chunk`
-    __device__ static __forceinline__ uint4 load_a(const unsigned char *chunk, int tig) {
-        return *reinterpret_cast<const uint4 *>(chunk + 16 * tig);
-    }
-};
-template <> struct Place<4, 64> {
-    __device__ static __forceinline__ void at(int p, int &tig, int &m, int &half, int &byte) {
-        m = p >> 5;
-        tig = (p >> 3) & 3;
-        byte = (p >> 1) & 3;
-        half = p & 1;
-    }
-    __device__ static __forceinline__ uint4 load_a(const unsigned char *chunk, int tig) {
-        const uint32_t *w = reinterpret_cast<const uint32_t *>(chunk + 4 * tig);
-        return make_uint4(w[0], w[4], w[8], w[12]);
     }
 };
 
@@ -330,15 +306,19 @@ __device__ void route_select(const DecodeParams &p, int t, int lane, RouteToken 
 
 // ------------------------------------------------------------------------- the kernel ------
 // Shared-memory regions (byte offsets from the plan): barriers | routing cache | per-token
-// routing scratch | activation slices (phase 1) aliased with h slices and the final reduction
-// (phase 2) | group reduction buffers | gate partials | ring.
-template <int FMT, int TT, int GI, int GS>
+// routing scratch | gate partials | group reduction buffers | activation slices (phase 1)
+// aliased with the h slices and the final reduction (phase 2) | ring.
+// Ring stages: phase 1 holds one tile (8 gate rows | the same 8 up rows | their scales), each
+// matrix's rows one contiguous copy; phase 2 holds the CTA's block of down rows of one expert
+// (one contiguous copy) and their scales.  Few large copies: a single producer thread issues
+// them at a rate far below that of the TMA engine's data path.
+template <int FMT, int TT, int GS>
 __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
     using F = Fmt<FMT>;
-    using PL = Place<FMT, GS>;
     constexpr int CPC = F::CPC, MPC = F::MPC;
     constexpr int MAXT = TT;                          // tokens of this instantiation (T <= TT)
     constexpr int NB = (3 * TT + 7) / 8;              // 8-column MMA blocks (3 slices per token)
+    constexpr int EG = FMT == 4 ? 8 : 16;             // activations converted together (whole B words)
     extern __shared__ __align__(1024) unsigned char sm[];
     const FfnParams &f = p.f;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -351,6 +331,7 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
     unsigned char *xb = sm + p.off_x;                  // activation slices, B layout
     int4 *red1 = reinterpret_cast<int4 *>(sm + p.off_red1);
     double *gpart = reinterpret_cast<double *>(sm + p.off_gate);
+    float *xmax = reinterpret_cast<float *>(gpart + NCW * 2 * MAXTOK);  // [NCW][MAXTOK]
     unsigned char *ring = sm + p.off_ring;
     const uint32_t bar0 = smem_u32(bars);
     auto full_bar = [&](int s) { return bar0 + 8u * s; };
@@ -359,13 +340,6 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
 
     // geometry
     const int rb_h = static_cast<int>(f.rb_h), rb_i = static_cast<int>(f.rb_i);
-    const int SK1 = p.SK1, nks1 = rb_h / SK1;          // phase-1 stage: 16 rows x SK1 bytes
-    const int SK2 = p.SK2, nks2 = rb_i / SK2;          // phase-2 stage: nrows x SK2 bytes
-    // staged row strides: 64 bytes of padding for 16-byte A loads, 16 for 4-byte ones
-    constexpr int PAD = GS ? 16 : ROWPAD;
-    const int st1 = SK1 + PAD, st2 = SK2 + PAD;
-    const int gps1 = GS ? SK1 * 8 / FMT / GS : 0;     // scale groups per row of a phase-1 stage
-    const int gps2 = GS ? SK2 * 8 / FMT / GS : 0;     // and of a phase-2 stage
     const int NRB = f.I / 8;                           // tiles (8 row pairs) per expert
     const int j_lo = static_cast<int>(static_cast<long>(f.H) * b / G), j_hi = static_cast<int>(static_cast<long>(f.H) * (b + 1) / G);
     const int nrows = j_hi - j_lo;
@@ -373,11 +347,12 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
     const int sh_lo = f.S ? static_cast<int>(static_cast<long>(NRB) * b / G) : 0;
     const int sh_hi = f.S ? static_cast<int>(static_cast<long>(NRB) * (b + 1) / G) : 0;
     const int nsh = sh_hi - sh_lo;                     // shared-expert tiles of this CTA
+    const int sc1 = GS ? 8 * f.nsh * 4 : 32;           // bytes of one matrix's scales in a tile stage
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
             mbar_init(full_bar(s), 1);
-            mbar_init(empty_bar(s), GW);               // every stage is read by 8 warps
+            mbar_init(empty_bar(s), NCW);  // phase 1: 8 warps x 2; phase 2: the active warps
         }
         mbar_init(route_bar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -398,69 +373,44 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
         };
         auto stage1 = [&](const uint8_t *rec, int rb) {
             const int r0 = rb * 8;
-            for (int part = 0; part < nks1 && ok; ++part, ++seq) {
-                const int s = seq % S;
-                const uint32_t par = (seq / S) & 1;
-                if (!mbar_wait(empty_bar(s), par ^ 1, bound)) { ok = false; break; }
-                if (rec == nullptr) { mbar_arrive(full_bar(s)); continue; }
-                const uint32_t dst = smem_u32(ring + static_cast<size_t>(s) * p.SB);
-                const uint32_t bytes = 16u * SK1 + (GS ? 16u * 4u * gps1 : (part == 0 ? 64u : 0u));
-                mbar_expect_tx(full_bar(s), bytes);
-                for (int r = 0; r < 8; ++r) {
-                    const size_t src = static_cast<size_t>(r0 + r) * rb_h + static_cast<size_t>(part) * SK1;
-                    bulk_g2s(dst + r * st1, rec + src, SK1, full_bar(s), pol);
-                    bulk_g2s(dst + (8 + r) * st1, rec + f.off_wu + src, SK1, full_bar(s), pol);
-                }
-                if (GS) {  // this part's group scales: gate rows, then up rows, gps1 each
-                    for (int r = 0; r < 8; ++r) {
-                        const size_t g0 = (static_cast<size_t>(r0 + r) * f.nsh + static_cast<size_t>(part) * gps1) * 4;
-                        bulk_g2s(dst + 16 * st1 + r * 4 * gps1, rec + f.off_sg + g0, 4 * gps1, full_bar(s), pol);
-                        bulk_g2s(dst + 16 * st1 + (8 + r) * 4 * gps1, rec + f.off_su + g0, 4 * gps1, full_bar(s), pol);
-                    }
-                } else if (part == 0) {
-                    bulk_g2s(dst + 16 * st1, rec + f.off_sg + 4 * r0, 32, full_bar(s), pol);
-                    bulk_g2s(dst + 16 * st1 + 32, rec + f.off_su + 4 * r0, 32, full_bar(s), pol);
-                }
-            }
+            const int s = seq % S;
+            const uint32_t par = (seq / S) & 1;
+            if (!mbar_wait(empty_bar(s), par ^ 1, bound)) { ok = false; return; }
+            ++seq;  // counts filled stages only (the drain waits for the last fill of each slot)
+            if (rec == nullptr) { mbar_arrive(full_bar(s)); return; }
+            const uint32_t dst = smem_u32(ring + static_cast<size_t>(s) * p.SB);
+            mbar_expect_tx(full_bar(s), 16u * rb_h + 2u * sc1);
+            const size_t so = GS ? static_cast<size_t>(r0) * f.nsh * 4 : static_cast<size_t>(4 * r0);
+            bulk_g2s(dst, rec + static_cast<size_t>(r0) * rb_h, 8 * rb_h, full_bar(s), pol);
+            bulk_g2s(dst + 8 * rb_h, rec + f.off_wu + static_cast<size_t>(r0) * rb_h, 8 * rb_h, full_bar(s), pol);
+            bulk_g2s(dst + 16 * rb_h, rec + f.off_sg + so, sc1, full_bar(s), pol);
+            bulk_g2s(dst + 16 * rb_h + sc1, rec + f.off_su + so, sc1, full_bar(s), pol);
         };
         // phase 1: the shared expert's tiles, then (once routed) the flat list of routed tiles
         for (int l = 0; l < nsh && ok; ++l) stage1(f.shared, sh_lo + l);
-        if (f.S && ok) {  // the shared expert's down rows go to L2 while the batch is routed
-            for (int part = 0; part < nks2; ++part)
-                for (int r = 0; r < nrows; ++r)
-                    bulk_prefetch_l2(f.shared + f.off_wd + static_cast<size_t>(j_lo + r) * rb_i + static_cast<size_t>(part) * SK2, SK2);
-        }
+        if (f.S && ok)  // the shared expert's down rows go to L2 while the batch is routed
+            bulk_prefetch_l2(f.shared + f.off_wd + static_cast<size_t>(j_lo) * rb_i, static_cast<uint32_t>(nrows) * rb_i);
         if (ok && !mbar_wait(route_bar, 0, bound)) ok = false;
         if (ok) U = rc.U;
         const long nr = static_cast<long>(U) * NRB;
         const int r_lo = static_cast<int>(nr * b / G), r_hi = static_cast<int>(nr * (b + 1) / G);
         for (int tau = r_lo; tau < r_hi && ok; ++tau) stage1(record(f.S + tau / NRB), tau % NRB);
-        // phase 2: every work expert's block of down rows, in K parts
+        // phase 2: every work expert's block of down rows and their scales
+        const int a1 = (j_hi + 3) & ~3;
+        const uint32_t sdb = GS ? static_cast<uint32_t>(nrows) * f.nsi * 4 : 4u * (a1 - a0d);
         for (int we = 0; we < f.S + U && ok; ++we) {
             const uint8_t *rec = record(we);
-            for (int part = 0; part < nks2 && ok; ++part, ++seq) {
-                const int s = seq % S;
-                const uint32_t par = (seq / S) & 1;
-                if (!mbar_wait(empty_bar(s), par ^ 1, bound)) { ok = false; break; }
-                if (rec == nullptr) { mbar_arrive(full_bar(s)); continue; }
-                const uint32_t dst = smem_u32(ring + static_cast<size_t>(s) * p.SB);
-                const int a1 = (j_hi + 3) & ~3;
-                const uint32_t bytes = static_cast<uint32_t>(nrows) * SK2 +
-                                       (GS ? static_cast<uint32_t>(nrows) * 4u * gps2 : 4u * (a1 - a0d));
-                mbar_expect_tx(full_bar(s), bytes);
-                const uint64_t pl = we < f.S ? keep : pol;
-                for (int r = 0; r < nrows; ++r)
-                    bulk_g2s(dst + r * st2, rec + f.off_wd + static_cast<size_t>(j_lo + r) * rb_i + static_cast<size_t>(part) * SK2,
-                             SK2, full_bar(s), pl);
-                if (GS) {  // this part's group scales of the CTA's rows, gps2 per row
-                    for (int r = 0; r < nrows; ++r)
-                        bulk_g2s(dst + p.st_sd + r * 4 * gps2,
-                                 rec + f.off_sd + (static_cast<size_t>(j_lo + r) * f.nsi + static_cast<size_t>(part) * gps2) * 4,
-                                 4 * gps2, full_bar(s), pl);
-                } else {
-                    bulk_g2s(dst + p.st_sd, rec + f.off_sd + 4 * a0d, 4 * (a1 - a0d), full_bar(s), pl);  // every part
-                }
-            }
+            const int s = seq % S;
+            const uint32_t par = (seq / S) & 1;
+            if (!mbar_wait(empty_bar(s), par ^ 1, bound)) { ok = false; break; }
+            ++seq;
+            if (rec == nullptr) { mbar_arrive(full_bar(s)); continue; }
+            const uint32_t dst = smem_u32(ring + static_cast<size_t>(s) * p.SB);
+            mbar_expect_tx(full_bar(s), static_cast<uint32_t>(nrows) * rb_i + sdb);
+            const uint64_t pl = we < f.S ? keep : pol;
+            bulk_g2s(dst, rec + f.off_wd + static_cast<size_t>(j_lo) * rb_i, static_cast<uint32_t>(nrows) * rb_i, full_bar(s), pl);
+            bulk_g2s(dst + p.st_sd, rec + f.off_sd + (GS ? static_cast<size_t>(j_lo) * f.nsi * 4 : static_cast<size_t>(4 * a0d)),
+                     sdb, full_bar(s), pl);
         }
         if (!ok) atomicOr(f.err, COLI_DEVERR_TIMEOUT);
         // Drain: the last fill of every ring slot has landed before this thread (and with it the
@@ -476,113 +426,128 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
     const int ct = threadIdx.x - 32;
     const int cw = ct >> 5;
     const int g8 = lane >> 2, tig = lane & 3;
+    const int NCOL = 3 * T;
+    const int colblk = 4 * 8 * MPC;                   // bytes of one column's block of a chunk
     bool ok = true;
 
     for (int i = ct; i < MAXWE * MAXTOK; i += NC) {
         (&rc.slot[0][0])[i] = -1;
         (&rc.wgt[0][0])[i] = 0.f;
     }
-    if (ct == 0) rc.err = 0;
 
-    // ---- start: activations (and the gate) ----
-    // thread ct owns elements h = 4 ct + 2048 gi (gi < GI) of every token
+    // ---- start: activations and the gate ----
+    // thread ct owns the groups of EG activations q = ct + NC r of every token
     const int e0 = static_cast<int>(static_cast<long>(f.E) * b / G), e1 = static_cast<int>(static_cast<long>(f.E) * (b + 1) / G);
     const int ne = p.route_here ? e1 - e0 : 0;        // router rows of this CTA (<= 2)
-    {
-        uint2 xv[MAXT][GI];
-        float4 wv[2][GI];
+    const int NQ = f.H / EG;
+    auto load_x = [&](int t, int q, uint32_t (&w)[EG / 2]) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(f.x) + static_cast<size_t>(t) * f.H + q * EG);
 #pragma unroll
-        for (int t = 0; t < MAXT; ++t)
-#pragma unroll
-            for (int gi = 0; gi < GI; ++gi)
-                xv[t][gi] = t < T ? __ldg(reinterpret_cast<const uint2 *>(static_cast<const uint16_t *>(f.x) + static_cast<size_t>(t) * f.H + 4 * ct + 2048 * gi))
-                                  : make_uint2(0u, 0u);
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-#pragma unroll
-            for (int gi = 0; gi < GI; ++gi)
-                wv[j][gi] = j < ne ? __ldg(reinterpret_cast<const float4 *>(p.Wr + static_cast<size_t>(e0 + j) * f.H + 4 * ct + 2048 * gi))
-                                   : make_float4(0.f, 0.f, 0.f, 0.f);
-        auto xval = [&](int t, int gi, int k) -> float {
-            const uint32_t w2 = (k < 2) ? xv[t][gi].x : xv[t][gi].y;
-            return __uint_as_float((k & 1) ? (w2 & 0xffff0000u) : (w2 << 16));
-        };
-        // per-token row maximum
-        float *xmax = reinterpret_cast<float *>(gpart + NCW * 2 * MAXTOK);  // [NCW][MAXTOK]
-#pragma unroll
-        for (int t = 0; t < MAXT; ++t) {
-            float m = 0.f;
-#pragma unroll
-            for (int gi = 0; gi < GI; ++gi)
-#pragma unroll
-                for (int k = 0; k < 4; ++k) m = fmaxf(m, fabsf(xval(t, gi, k)));
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
-            if (lane == 0) xmax[cw * MAXTOK + t] = m;
+        for (int i = 0; i < EG / 8; ++i) {
+            const uint4 v = __ldg(src + i);
+            w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
         }
-        // gate partial dot products (exact double products, double sums)
+    };
+    auto bf = [](const uint32_t (&w)[EG / 2], int k) -> float {
+        return __uint_as_float((k & 1) ? (w[k >> 1] & 0xffff0000u) : (w[k >> 1] << 16));
+    };
+    {
+        double acc[2][MAXT];
+        float mx[MAXT];
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
+        for (int t = 0; t < MAXT; ++t) { acc[0][t] = acc[1][t] = 0.0; mx[t] = 0.f; }
+        for (int q = ct; q < NQ; q += NC) {
+            float wv[2][EG];
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int i = 0; i < EG / 4; ++i) {
+                    const float4 v = j < ne ? __ldg(reinterpret_cast<const float4 *>(p.Wr + static_cast<size_t>(e0 + j) * f.H + q * EG) + i)
+                                            : make_float4(0.f, 0.f, 0.f, 0.f);
+                    wv[j][4 * i] = v.x; wv[j][4 * i + 1] = v.y; wv[j][4 * i + 2] = v.z; wv[j][4 * i + 3] = v.w;
+                }
 #pragma unroll
             for (int t = 0; t < MAXT; ++t) {
-                if (j < ne && t < T) {
-                    double acc = 0.0;
+                if (t < T) {
+                    uint32_t w[EG / 2];
+                    load_x(t, q, w);
 #pragma unroll
-                    for (int gi = 0; gi < GI; ++gi) {
-                        const float4 w4 = wv[j][gi];
-                        acc = fma(static_cast<double>(w4.x), static_cast<double>(xval(t, gi, 0)), acc);
-                        acc = fma(static_cast<double>(w4.y), static_cast<double>(xval(t, gi, 1)), acc);
-                        acc = fma(static_cast<double>(w4.z), static_cast<double>(xval(t, gi, 2)), acc);
-                        acc = fma(static_cast<double>(w4.w), static_cast<double>(xval(t, gi, 3)), acc);
+                    for (int k = 0; k < EG; ++k) {
+                        const float xv = bf(w, k);
+                        mx[t] = fmaxf(mx[t], fabsf(xv));
+                        acc[0][t] = fma(static_cast<double>(wv[0][k]), static_cast<double>(xv), acc[0][t]);
+                        acc[1][t] = fma(static_cast<double>(wv[1][k]), static_cast<double>(xv), acc[1][t]);
                     }
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(FULL, acc, o);
-                    if (lane == 0) gpart[cw * 2 * MAXTOK + j * MAXTOK + t] = acc;
                 }
             }
-        cons_sync();
-        if (ct < ne * T) {  // one logit per thread of warp 0: the 16 warps' partials in order
-            const int j = ct / T, t = ct % T;
-            double sum = 0.0;
-            for (int w2 = 0; w2 < NCW; ++w2) sum += gpart[w2 * 2 * MAXTOK + j * MAXTOK + t];
-            p.logits[static_cast<size_t>(t) * f.E + e0 + j] = static_cast<float>(sum);
-            __threadfence();
         }
-        if (cw == 0 && p.route_here) {
-            __syncwarp();
-            if (lane == 0) atomicAdd(p.gbar, 1u);
-        }
-        // activation slices: X = rint(x * 2^(22 - e)), max|x| < 2^e
-        const int NCOL = 3 * T;
-        const size_t colblk = 4 * 8 * MPC;             // bytes of one column's block of a chunk
 #pragma unroll
         for (int t = 0; t < MAXT; ++t) {
-            if (t < T) {
-                float m = 0.f;
-                for (int w2 = 0; w2 < NCW; ++w2) m = fmaxf(m, xmax[w2 * MAXTOK + t]);
-                int ex = 0;
-                if (m > 0.f) frexpf(m, &ex);
-                const float up = ldexpf(1.0f, 22 - ex);
-                if (ct == 0) rc.xscale[t] = ldexpf(1.0f, ex - 22);
 #pragma unroll
-                for (int gi = 0; gi < GI; ++gi) {
-                    const int h0 = 4 * ct + 2048 * gi;
-                    const int kc = h0 / CPC, p0 = h0 % CPC;
-                    int sl[4][3];
+            for (int o = 16; o > 0; o >>= 1) {
+                mx[t] = fmaxf(mx[t], __shfl_xor_sync(FULL, mx[t], o));
+                acc[0][t] += __shfl_xor_sync(FULL, acc[0][t], o);
+                acc[1][t] += __shfl_xor_sync(FULL, acc[1][t], o);
+            }
+            if (lane == 0) {
+                xmax[cw * MAXTOK + t] = mx[t];
+                gpart[cw * 2 * MAXTOK + t] = acc[0][t];
+                gpart[cw * 2 * MAXTOK + MAXTOK + t] = acc[1][t];
+            }
+        }
+    }
+    cons_sync();
+    if (ct < ne * T) {  // one logit per thread of warp 0: the 16 warps' partials in order
+        const int j = ct / T, t = ct % T;
+        double sum = 0.0;
+        for (int w2 = 0; w2 < NCW; ++w2) sum += gpart[w2 * 2 * MAXTOK + j * MAXTOK + t];
+        p.logits[static_cast<size_t>(t) * f.E + e0 + j] = static_cast<float>(sum);
+        __threadfence();
+    }
+    if (cw == 0 && p.route_here) {
+        __syncwarp();
+        if (lane == 0) atomicAdd(p.gbar, 1u);
+    }
+    // activation slices: X = rint(x * 2^(22 - e)), max|x| < 2^e, written as whole B words
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const int X = __float2int_rn(xval(t, gi, k) * up);
-                        slices3(X, sl[k][0], sl[k][1], sl[k][2]);
-                    }
+    for (int t = 0; t < MAXT; ++t) {
+        if (t < T) {
+            float m = 0.f;
+            for (int w2 = 0; w2 < NCW; ++w2) m = fmaxf(m, xmax[w2 * MAXTOK + t]);
+            int ex = 0;
+            if (m > 0.f) frexpf(m, &ex);
+            const float up = ldexpf(1.0f, 22 - ex);
+            if (ct == 0) rc.xscale[t] = ldexpf(1.0f, ex - 22);
+            for (int q = ct; q < NQ; q += NC) {
+                uint32_t w[EG / 2];
+                load_x(t, q, w);
+                uint32_t sl[3][EG];  // slice bytes of the EG elements
 #pragma unroll
-                    for (int s = 0; s < 3; ++s) {
-                        const int col = 3 * t + s;
-                        unsigned char *blk = xb + (static_cast<size_t>(kc) * NCOL + col) * colblk;
+                for (int k = 0; k < EG; ++k) {
+                    int s0, s1, s2;
+                    slices3(__float2int_rn(bf(w, k) * up), s0, s1, s2);
+                    sl[0][k] = static_cast<uint32_t>(s0) & 0xffu;
+                    sl[1][k] = static_cast<uint32_t>(s1) & 0xffu;
+                    sl[2][k] = static_cast<uint32_t>(s2) & 0xffu;
+                }
+                const int h0 = q * EG, kc = h0 / CPC, p0 = h0 % CPC;
+#pragma unroll
+                for (int s = 0; s < 3; ++s) {
+                    const int col = 3 * t + s;
+                    unsigned char *blk = xb + (static_cast<size_t>(kc) * NCOL + col) * colblk;
+                    if (FMT == 4) {  // elements p0 + 2j (+1) -> byte j of register half 0 (1)
+                        const int tg = p0 >> 5, m = (p0 >> 3) & 3;
+#pragma unroll
+                        for (int hf = 0; hf < 2; ++hf) {
+                            const uint32_t word = sl[s][hf] | (sl[s][2 + hf] << 8) | (sl[s][4 + hf] << 16) | (sl[s][6 + hf] << 24);
+                            *reinterpret_cast<uint32_t *>(blk + b_off<FMT>(col, tg, m, hf, 0)) = word;
+                        }
+                    } else {         // elements p0 + 4j + k -> byte j of field k's register
+                        const int tg = p0 >> 6, i4 = (p0 >> 4) & 3;
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
-                            int tg, m2, hf, by;
-                            PL::at(p0 + k, tg, m2, hf, by);
-                            blk[b_off<FMT>(col, tg, m2, hf, by)] = static_cast<unsigned char>(sl[k][s] & 0xff);
+                            const uint32_t word = sl[s][k] | (sl[s][4 + k] << 8) | (sl[s][8 + k] << 16) | (sl[s][12 + k] << 24);
+                            *reinterpret_cast<uint32_t *>(blk + b_off<FMT>(col, tg, 2 * i4 + (k >> 1), k & 1, 0)) = word;
                         }
                     }
                 }
@@ -693,17 +658,29 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
         }
     };
 
+    // One MMA of the chunk's codes against B, into the per-row sum D or, for the group-scaled
+    // container, split by group: a thread's codes lie in group tig >> 1 of the 64-byte chunk, so
+    // group g's MMA takes the A registers of lanes with tig >> 1 == g and zeros elsewhere.
+    auto mma_chunk = [&](int (&D)[4], int (&D1)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                         uint32_t b0, uint32_t b1) {
+        if (GS) {
+            const bool g1 = (tig >> 1) != 0;
+            mma_s8(D, g1 ? 0u : a0, g1 ? 0u : a1, g1 ? 0u : a2, g1 ? 0u : a3, b0, b1);
+            mma_s8(D1, g1 ? a0 : 0u, g1 ? a1 : 0u, g1 ? a2 : 0u, g1 ? a3 : 0u, b0, b1);
+        } else {
+            mma_s8(D, a0, a1, a2, a3, b0, b1);
+        }
+    };
+
     // ------------------------------------------------ phase 1: gate/up, h = SiLU(g)*u -----
     // After a timed-out wait a warp keeps walking the same loops and barriers (skipping later
     // waits and MMAs), so that no consumer is ever left alone at a named barrier, and releases no
     // more ring stages: the producer then runs out of its own bounded waits, and its drain makes
     // sure no copy is still landing in shared memory when the CTA exits.
     const int grp = cw / GW, wg = cw % GW;
-    const int cpw1 = SK1 / 64 / GW;                   // chunks of a stage per warp
-    const size_t colblk = 4 * 8 * MPC;
+    const int cpw1 = rb_h / 64 / GW;                  // chunks of a row per warp
     int seq = 0, U = 0, my_tiles = 0;
     long r_lo = 0, r_hi = 0;
-    const int NCOL = 3 * T;
     for (int lam = 0;; ++lam) {
         if (lam == nsh) {
             if (p.route_here) route_batch();
@@ -717,72 +694,65 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
         int we, rb;
         if (lam < nsh) { we = 0; rb = sh_lo + lam; }
         else { const long tau = r_lo + (lam - nsh); we = f.S + static_cast<int>(tau / NRB); rb = static_cast<int>(tau % NRB); }
-        if ((lam % NGRP) != grp) { seq += nks1; continue; }
+        const int s = seq % S;
+        const uint32_t par = (seq / S) & 1;
+        ++seq;
+        if ((lam % NGRP) != grp) continue;
         int D[NB][4];       // per-row scales: exact int32 sums over all of K
         float Dg[NB][4];    // group scales: float sums of (group sum x group scale)
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
             for (int i = 0; i < 4; ++i) { D[nb][i] = 0; Dg[nb][i] = 0.f; }
-        const unsigned char *scal = nullptr;
-        for (int part = 0; part < nks1; ++part, ++seq) {
-            const int s = seq % S;
-            const uint32_t par = (seq / S) & 1;
-            if (ok && !mbar_wait(full_bar(s), par, bound)) ok = false;
-            ok = __all_sync(FULL, ok);  // warp-uniform: the MMAs below need every lane
-            const unsigned char *st = ring + static_cast<size_t>(s) * p.SB;
-            if (part == 0) scal = st + 16 * st1;
-            if (ok) {
-                for (int cc = 0; cc < cpw1; ++cc) {
-                    const int c = wg * cpw1 + cc;                    // chunk inside the stage
-                    const int kc = part * (SK1 / 64) + c;            // chunk inside the row
-                    const uint4 qa = PL::load_a(st + g8 * st1 + 64 * c, tig);
-                    const uint4 qb = PL::load_a(st + (g8 + 8) * st1 + 64 * c, tig);
-                    const unsigned char *xk = xb + static_cast<size_t>(kc) * NCOL * colblk;
+        if (ok && !mbar_wait(full_bar(s), par, bound)) ok = false;
+        ok = __all_sync(FULL, ok);  // warp-uniform: the MMAs below need every lane
+        const unsigned char *st = ring + static_cast<size_t>(s) * p.SB;
+        const float *sgs = reinterpret_cast<const float *>(st + 16 * rb_h);       // gate rows' scales
+        const float *sus = reinterpret_cast<const float *>(st + 16 * rb_h + sc1);  // up rows' scales
+        if (ok) {
+            for (int cc = 0; cc < cpw1; ++cc) {
+                const int c = wg * cpw1 + cc;                    // 64-byte chunk of the row
+                const uint4 qa = *reinterpret_cast<const uint4 *>(st + g8 * rb_h + 64 * c + 16 * tig);
+                const uint4 qb = *reinterpret_cast<const uint4 *>(st + (8 + g8) * rb_h + 64 * c + 16 * tig);
+                const unsigned char *xk = xb + static_cast<size_t>(c) * NCOL * colblk;
+                int Dc[NB][4], Dc1[NB][4];  // group-scaled container: this chunk's two groups
 #pragma unroll
-                    for (int u = 0; u < MPC / 2; ++u) {
-                        uint4 bv[NB];
+                for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-                        for (int nb = 0; nb < NB; ++nb) {
-                            const int col = nb * 8 + g8;
-                            bv[nb] = col < NCOL ? load_b2<FMT>(xk + col * colblk, col, tig, u) : make_uint4(0u, 0u, 0u, 0u);
-                        }
-                        int Du[NB][4];  // group-scaled container: this group's sums
+                    for (int i = 0; i < 4; ++i) { Dc[nb][i] = 0; Dc1[nb][i] = 0; }
+#pragma unroll
+                for (int u = 0; u < MPC / 2; ++u) {
+                    uint4 bv[NB];
+#pragma unroll
+                    for (int nb = 0; nb < NB; ++nb) {
+                        const int col = nb * 8 + g8;
+                        bv[nb] = col < NCOL ? load_b2<FMT>(xk + col * colblk, col, tig, u) : make_uint4(0u, 0u, 0u, 0u);
+                    }
+#pragma unroll
+                    for (int mm = 0; mm < 2; ++mm) {
+                        uint32_t a0, a2, a1, a3;
+                        F::unpack(qa, 2 * u + mm, a0, a2);
+                        F::unpack(qb, 2 * u + mm, a1, a3);
 #pragma unroll
                         for (int nb = 0; nb < NB; ++nb)
+                            mma_chunk(GS ? Dc[nb] : D[nb], Dc1[nb], a0, a1, a2, a3, mm ? bv[nb].z : bv[nb].x, mm ? bv[nb].w : bv[nb].y);
+                    }
+                }
+                if (GS) {  // groups 2c and 2c + 1 of rows g8 (gate) and g8 + 8 (up)
+                    const float ga0 = sgs[g8 * f.nsh + 2 * c], ga1 = sgs[g8 * f.nsh + 2 * c + 1];
+                    const float ua0 = sus[g8 * f.nsh + 2 * c], ua1 = sus[g8 * f.nsh + 2 * c + 1];
 #pragma unroll
-                            for (int i = 0; i < 4; ++i) Du[nb][i] = 0;
+                    for (int nb = 0; nb < NB; ++nb) {
 #pragma unroll
-                        for (int mm = 0; mm < 2; ++mm) {
-                            uint32_t a0, a2, a1, a3;
-                            F::unpack(qa, 2 * u + mm, a0, a2);
-                            F::unpack(qb, 2 * u + mm, a1, a3);
-#pragma unroll
-                            for (int nb = 0; nb < NB; ++nb)
-                                mma_s8(GS ? Du[nb] : D[nb], a0, a1, a2, a3, mm ? bv[nb].z : bv[nb].x, mm ? bv[nb].w : bv[nb].y);
-                        }
-                        if (GS) {  // group u of the chunk: rows g8 (gate) and g8 + 8 (up)
-                            const float *gsc = reinterpret_cast<const float *>(st + 16 * st1);
-                            const float sa = gsc[g8 * gps1 + 2 * c + u];
-                            const float sb = gsc[(g8 + 8) * gps1 + 2 * c + u];
-#pragma unroll
-                            for (int nb = 0; nb < NB; ++nb) {
-                                Dg[nb][0] = __fmaf_rn(static_cast<float>(Du[nb][0]), sa, Dg[nb][0]);
-                                Dg[nb][1] = __fmaf_rn(static_cast<float>(Du[nb][1]), sa, Dg[nb][1]);
-                                Dg[nb][2] = __fmaf_rn(static_cast<float>(Du[nb][2]), sb, Dg[nb][2]);
-                                Dg[nb][3] = __fmaf_rn(static_cast<float>(Du[nb][3]), sb, Dg[nb][3]);
-                            }
+                        for (int i = 0; i < 2; ++i) {
+                            Dg[nb][i] = __fmaf_rn(static_cast<float>(Dc1[nb][i]), ga1, __fmaf_rn(static_cast<float>(Dc[nb][i]), ga0, Dg[nb][i]));
+                            Dg[nb][2 + i] = __fmaf_rn(static_cast<float>(Dc1[nb][2 + i]), ua1, __fmaf_rn(static_cast<float>(Dc[nb][2 + i]), ua0, Dg[nb][2 + i]));
                         }
                     }
                 }
             }
-            __syncwarp();
-            // stage 0 of the tile holds the row scales until the epilogue has read them: it is
-            // released after the reduction (below), the other parts now
-            if (ok && part > 0 && lane == 0) mbar_arrive(empty_bar(s));
         }
         // group reduction of the partial sums, then one warp forms h
-        const int tile_seq0 = seq - nks1;
         if (my_tiles > 0 && wg != 0) named_sync(BAR_GFREE + grp, GW * 32);
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb)
@@ -793,56 +763,46 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
         if (wg == 0) {
             const int pr = lane & 7, t = lane >> 3;  // row pair, token
             const int slot = t < T ? rc.slot[we][t] : -1;
-            if (ok && slot >= 0 && GS) {
-                // group-scaled: the partials already carry the weights' scales
+            if (ok && slot >= 0) {
                 double gsum = 0.0, usum = 0.0;
 #pragma unroll
                 for (int sidx = 0; sidx < 3; ++sidx) {
                     const int col = 3 * t + sidx, nb = col >> 3, c8 = col & 7;
                     const int ln = pr * 4 + (c8 >> 1), ix = c8 & 1;
-                    float gs = 0.f, us = 0.f;
-                    for (int w2 = 0; w2 < GW; ++w2) {
-                        const float *v = reinterpret_cast<const float *>(&red1[((grp * GW + w2) * NB + nb) * 32 + ln]);
-                        gs = __fadd_rn(gs, v[ix]);
-                        us = __fadd_rn(us, v[2 + ix]);
-                    }
                     const double wsl = sidx == 0 ? 1.0 : (sidx == 1 ? 256.0 : 65536.0);
-                    gsum += wsl * gs;
-                    usum += wsl * us;
-                }
-                const double xs = static_cast<double>(rc.xscale[t]) / F::MUL;
-                const float gq = static_cast<float>(gsum * xs);
-                const float uq = static_cast<float>(usum * xs);
-                f.h[static_cast<size_t>(slot) * f.I + rb * 8 + pr] = __fmul_rn(__fdiv_rn(gq, __fadd_rn(1.0f, expf(-gq))), uq);
-            } else if (ok && slot >= 0) {
-                long long gsum = 0, usum = 0;
-#pragma unroll
-                for (int sidx = 0; sidx < 3; ++sidx) {
-                    const int col = 3 * t + sidx, nb = col >> 3, c8 = col & 7;
-                    const int ln = pr * 4 + (c8 >> 1), ix = c8 & 1;
-                    int gs = 0, us = 0;
-                    for (int w2 = 0; w2 < GW; ++w2) {
-                        const int *v = reinterpret_cast<const int *>(&red1[((grp * GW + w2) * NB + nb) * 32 + ln]);
-                        gs += v[ix];
-                        us += v[2 + ix];
+                    if (GS) {  // the partials already carry the weights' group scales
+                        float gs = 0.f, us = 0.f;
+                        for (int w2 = 0; w2 < GW; ++w2) {
+                            const float *v = reinterpret_cast<const float *>(&red1[((grp * GW + w2) * NB + nb) * 32 + ln]);
+                            gs = __fadd_rn(gs, v[ix]);
+                            us = __fadd_rn(us, v[2 + ix]);
+                        }
+                        gsum += wsl * gs;
+                        usum += wsl * us;
+                    } else {   // exact: int32 per slice, combined exactly in double (|sum| < 2^53)
+                        int gs = 0, us = 0;
+                        for (int w2 = 0; w2 < GW; ++w2) {
+                            const int *v = reinterpret_cast<const int *>(&red1[((grp * GW + w2) * NB + nb) * 32 + ln]);
+                            gs += v[ix];
+                            us += v[2 + ix];
+                        }
+                        gsum += wsl * gs;
+                        usum += wsl * us;
                     }
-                    const long long wsl = sidx == 0 ? 1LL : (sidx == 1 ? 256LL : 65536LL);
-                    gsum += wsl * gs;
-                    usum += wsl * us;
                 }
-                const float sgv = reinterpret_cast<const float *>(scal)[pr];
-                const float suv = reinterpret_cast<const float *>(scal + 32)[pr];
                 const double xs = static_cast<double>(rc.xscale[t]) / F::MUL;
-                const float gq = static_cast<float>(static_cast<double>(gsum) * xs * static_cast<double>(sgv));
-                const float uq = static_cast<float>(static_cast<double>(usum) * xs * static_cast<double>(suv));
+                const double gsc = GS ? 1.0 : static_cast<double>(sgs[pr]);
+                const double usc = GS ? 1.0 : static_cast<double>(sus[pr]);
+                const float gq = static_cast<float>(gsum * xs * gsc);
+                const float uq = static_cast<float>(usum * xs * usc);
                 f.h[static_cast<size_t>(slot) * f.I + rb * 8 + pr] = __fmul_rn(__fdiv_rn(gq, __fadd_rn(1.0f, expf(-gq))), uq);
             }
             __syncwarp();
             named_arrive(BAR_GFREE + grp, GW * 32);
         }
-        // stage 0 of the tile (it held the row scales) is released now
+        // the stage (rows and scales) is released once the epilogue has read the scales
         __syncwarp();
-        if (ok && lane == 0) mbar_arrive(empty_bar(tile_seq0 % S));
+        if (ok && lane == 0) mbar_arrive_cnt(empty_bar(s), NCW / GW);
         ++my_tiles;
     }
     if (my_tiles > 0 && wg != 0) named_sync(BAR_GFREE + grp, GW * 32);  // the last arrival
@@ -867,15 +827,15 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
     cons_sync();
 
     // ------------------------------------------------ phase 2: down + combine -------------
-    // warp cw owns chunk cw of the down rows (when the rows have that many 64-byte chunks)
+    // warp cw owns the 64-byte chunk cw of every down row of the CTA's block
     constexpr int CPL = CPC / 32;                     // h elements per lane of a chunk
     constexpr int RT2 = 3;                            // 16-row tiles of the CTA's output rows
     const int nch2 = rb_i / 64;
-    const int cpp2 = SK2 / 64;                        // chunks per phase-2 stage
+    const int nact = nch2 < NCW ? nch2 : NCW;         // warps with a chunk
     const bool active2 = cw < nch2;
-    const int part2 = cw / cpp2, cl2 = cw % cpp2;
     const int nwe = f.S + U;
     unsigned char *hb = sm + p.off_x + static_cast<size_t>(cw) * NCOL * colblk;  // this warp's h slices
+    const float *sdp0 = nullptr;
     float acc[RT2][NB][4];
 #pragma unroll
     for (int rt = 0; rt < RT2; ++rt)
@@ -897,13 +857,16 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
             }
         }
     };
+    (void)sdp0;
     if (nwe > 0) fetch_h(0);
     for (int we = 0; we < nwe; ++we) {
-        const int s = (seq + we * nks2 + part2) % S;
-        const uint32_t par = ((seq + we * nks2 + part2) / S) & 1;
+        const int s = (seq + we) % S;
+        const uint32_t par = ((seq + we) / S) & 1;
         // h of this expert's slots -> 24-bit fixed point per chunk, three byte slices
         float fcol[NB][2];
         if (active2) {
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) fcol[nb][0] = fcol[nb][1] = 0.f;
 #pragma unroll
             for (int t = 0; t < MAXT; ++t) {
                 if (t < T) {
@@ -929,18 +892,13 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
                         int s0, s1, s2;
                         slices3(__float2int_rn(hv[t][k] * up), s0, s1, s2);
                         int tg, m2, hf, by;
-                        PL::at(lane * CPL + k, tg, m2, hf, by);
+                        F::place(lane * CPL + k, tg, m2, hf, by);
                         hb[(3 * t + 0) * colblk + b_off<FMT>(3 * t + 0, tg, m2, hf, by)] = static_cast<unsigned char>(s0 & 0xff);
                         hb[(3 * t + 1) * colblk + b_off<FMT>(3 * t + 1, tg, m2, hf, by)] = static_cast<unsigned char>(s1 & 0xff);
                         hb[(3 * t + 2) * colblk + b_off<FMT>(3 * t + 2, tg, m2, hf, by)] = static_cast<unsigned char>(s2 & 0xff);
                     }
                 }
             }
-#pragma unroll
-            for (int nb = 0; nb < NB; ++nb)
-#pragma unroll
-                for (int i = 0; i < 2; ++i)
-                    if (nb * 8 + 2 * tig + i >= NCOL) fcol[nb][i] = 0.f;
         }
         __syncwarp();
         if (we + 1 < nwe) fetch_h(we + 1);
@@ -949,64 +907,67 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
         if (ok && active2) {
             const unsigned char *st = ring + static_cast<size_t>(s) * p.SB;
             const float *sdp = reinterpret_cast<const float *>(st + p.st_sd) + (j_lo - a0d);
-            const float *sdg = reinterpret_cast<const float *>(st + p.st_sd);  // [nrows][gps2]
-            uint32_t bf[MPC][NB][2];
+            const float *sdg = reinterpret_cast<const float *>(st + p.st_sd);  // [nrows][nsi]
+            uint32_t bfr[MPC][NB][2];
 #pragma unroll
             for (int u = 0; u < MPC / 2; ++u)
 #pragma unroll
                 for (int nb = 0; nb < NB; ++nb) {
                     const int col = nb * 8 + g8;
                     const uint4 v = col < NCOL ? load_b2<FMT>(hb + col * colblk, col, tig, u) : make_uint4(0u, 0u, 0u, 0u);
-                    bf[2 * u][nb][0] = v.x;
-                    bf[2 * u][nb][1] = v.y;
-                    bf[2 * u + 1][nb][0] = v.z;
-                    bf[2 * u + 1][nb][1] = v.w;
+                    bfr[2 * u][nb][0] = v.x;
+                    bfr[2 * u][nb][1] = v.y;
+                    bfr[2 * u + 1][nb][0] = v.z;
+                    bfr[2 * u + 1][nb][1] = v.w;
                 }
 #pragma unroll
             for (int rt = 0; rt < RT2; ++rt) {
                 const int ra = rt * 16 + g8, rbw = ra + 8;
                 if (rt * 16 < nrows) {
                     const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-                    const uint4 qa = ra < nrows ? PL::load_a(st + ra * st2 + 64 * cl2, tig) : z;
-                    const uint4 qb = rbw < nrows ? PL::load_a(st + rbw * st2 + 64 * cl2, tig) : z;
-                    // per-row scales: one sum over the chunk; group scales: one per group u
-                    constexpr int NU = GS ? MPC / 2 : 1;
+                    const uint4 qa = ra < nrows ? *reinterpret_cast<const uint4 *>(st + ra * rb_i + 64 * cw + 16 * tig) : z;
+                    const uint4 qb = rbw < nrows ? *reinterpret_cast<const uint4 *>(st + rbw * rb_i + 64 * cw + 16 * tig) : z;
+                    int D[NB][4], D1[NB][4];
 #pragma unroll
-                    for (int ug = 0; ug < NU; ++ug) {
-                        int D[NB][4];
+                    for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-                        for (int nb = 0; nb < NB; ++nb)
+                        for (int i = 0; i < 4; ++i) { D[nb][i] = 0; D1[nb][i] = 0; }
 #pragma unroll
-                            for (int i = 0; i < 4; ++i) D[nb][i] = 0;
+                    for (int m = 0; m < MPC; ++m) {
+                        uint32_t a0, a2, a1, a3;
+                        F::unpack(qa, m, a0, a2);
+                        F::unpack(qb, m, a1, a3);
 #pragma unroll
-                        for (int m = ug * (MPC / NU); m < (ug + 1) * (MPC / NU); ++m) {
-                            uint32_t a0, a2, a1, a3;
-                            F::unpack(qa, m, a0, a2);
-                            F::unpack(qb, m, a1, a3);
+                        for (int nb = 0; nb < NB; ++nb) mma_chunk(D[nb], D1[nb], a0, a1, a2, a3, bfr[m][nb][0], bfr[m][nb][1]);
+                    }
+                    float sda, sdb, sda1 = 0.f, sdb1 = 0.f;
+                    if (GS) {  // groups 2 cw and 2 cw + 1 of rows ra and rbw
+                        sda = ra < nrows ? sdg[ra * f.nsi + 2 * cw] : 0.f;
+                        sda1 = ra < nrows ? sdg[ra * f.nsi + 2 * cw + 1] : 0.f;
+                        sdb = rbw < nrows ? sdg[rbw * f.nsi + 2 * cw] : 0.f;
+                        sdb1 = rbw < nrows ? sdg[rbw * f.nsi + 2 * cw + 1] : 0.f;
+                    } else {
+                        sda = ra < nrows ? sdp[ra] : 0.f;
+                        sdb = rbw < nrows ? sdp[rbw] : 0.f;
+                    }
 #pragma unroll
-                            for (int nb = 0; nb < NB; ++nb) mma_s8(D[nb], a0, a1, a2, a3, bf[m][nb][0], bf[m][nb][1]);
-                        }
-                        float sda, sdb;
-                        if (GS) {  // group ug of this warp's chunk, rows ra and rbw
-                            sda = ra < nrows ? sdg[ra * gps2 + 2 * cl2 + ug] : 0.f;
-                            sdb = rbw < nrows ? sdg[rbw * gps2 + 2 * cl2 + ug] : 0.f;
-                        } else {
-                            sda = ra < nrows ? sdp[ra] : 0.f;
-                            sdb = rbw < nrows ? sdp[rbw] : 0.f;
-                        }
-#pragma unroll
-                        for (int nb = 0; nb < NB; ++nb) {
-                            acc[rt][nb][0] = __fmaf_rn(static_cast<float>(D[nb][0]), sda * fcol[nb][0], acc[rt][nb][0]);
-                            acc[rt][nb][1] = __fmaf_rn(static_cast<float>(D[nb][1]), sda * fcol[nb][1], acc[rt][nb][1]);
-                            acc[rt][nb][2] = __fmaf_rn(static_cast<float>(D[nb][2]), sdb * fcol[nb][0], acc[rt][nb][2]);
-                            acc[rt][nb][3] = __fmaf_rn(static_cast<float>(D[nb][3]), sdb * fcol[nb][1], acc[rt][nb][3]);
+                    for (int nb = 0; nb < NB; ++nb) {
+                        acc[rt][nb][0] = __fmaf_rn(static_cast<float>(D[nb][0]), sda * fcol[nb][0], acc[rt][nb][0]);
+                        acc[rt][nb][1] = __fmaf_rn(static_cast<float>(D[nb][1]), sda * fcol[nb][1], acc[rt][nb][1]);
+                        acc[rt][nb][2] = __fmaf_rn(static_cast<float>(D[nb][2]), sdb * fcol[nb][0], acc[rt][nb][2]);
+                        acc[rt][nb][3] = __fmaf_rn(static_cast<float>(D[nb][3]), sdb * fcol[nb][1], acc[rt][nb][3]);
+                        if (GS) {
+                            acc[rt][nb][0] = __fmaf_rn(static_cast<float>(D1[nb][0]), sda1 * fcol[nb][0], acc[rt][nb][0]);
+                            acc[rt][nb][1] = __fmaf_rn(static_cast<float>(D1[nb][1]), sda1 * fcol[nb][1], acc[rt][nb][1]);
+                            acc[rt][nb][2] = __fmaf_rn(static_cast<float>(D1[nb][2]), sdb1 * fcol[nb][0], acc[rt][nb][2]);
+                            acc[rt][nb][3] = __fmaf_rn(static_cast<float>(D1[nb][3]), sdb1 * fcol[nb][1], acc[rt][nb][3]);
                         }
                     }
                 }
             }
         }
         __syncwarp();
-        if (ok && active2 && lane == 0) mbar_arrive(empty_bar(s));
+        if (ok && active2 && lane == 0) mbar_arrive_cnt(empty_bar(s), NCW / nact);
     }
     if (!ok) atomicOr(f.err, COLI_DEVERR_TIMEOUT);
     // cross-warp reduction (the h slices are no longer needed: the region is reused)
@@ -1021,7 +982,6 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
                     make_float4(acc[rt][nb][0], acc[rt][nb][1], acc[rt][nb][2], acc[rt][nb][3]);
     }
     cons_sync();
-    const int nact = nch2 < NCW ? nch2 : NCW;
     for (int fi = ct; fi < nrows * T; fi += NC) {
         const int r = fi / T, t = fi % T;
         const int rt = r >> 4, rr = r & 15, gg = rr & 7, hi = rr >> 3;
@@ -1038,9 +998,9 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
     }
 }
 
-template <int FMT, int TT, int GI, int GS>
+template <int FMT, int TT, int GS>
 cudaError_t launch_k(const DecodeParams &p, size_t smem, cudaStream_t st) {
-    auto kern = ffn_decode_kernel<FMT, TT, GI, GS>;
+    auto kern = ffn_decode_kernel<FMT, TT, GS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     // cooperative: the grid barriers need every CTA resident at once; the launch waits for the
@@ -1058,20 +1018,18 @@ cudaError_t launch_k(const DecodeParams &p, size_t smem, cudaStream_t st) {
     return cudaLaunchKernelEx(&cfg, kern, p);
 }
 
-template <int FMT, int GI, int GS>
-cudaError_t launch_nb(const DecodeParams &p, size_t smem, cudaStream_t st) {
-    if (p.f.T <= 1) return launch_k<FMT, 1, GI, GS>(p, smem, st);
-    if (p.f.T <= 2) return launch_k<FMT, 2, GI, GS>(p, smem, st);
-    return launch_k<FMT, 4, GI, GS>(p, smem, st);
+template <int FMT, int GS>
+cudaError_t launch_t(const DecodeParams &p, size_t smem, cudaStream_t st) {
+    if (p.f.T <= 1) return launch_k<FMT, 1, GS>(p, smem, st);
+    if (p.f.T <= 2) return launch_k<FMT, 2, GS>(p, smem, st);
+    return launch_k<FMT, 4, GS>(p, smem, st);
 }
 
 static cudaError_t launch_any(const DecodeParams &p, size_t smem, cudaStream_t st) {
-    const int gi = p.f.H / 2048;
-    if (p.f.fmt == 4 && gi == 3 && p.f.group == 64) return launch_nb<4, 3, 64>(p, smem, st);
+    if (p.f.fmt == 4 && p.f.group == 64) return launch_t<4, 64>(p, smem, st);
     if (p.f.group) return cudaErrorInvalidValue;
-    if (p.f.fmt == 4 && gi == 3) return launch_nb<4, 3, 0>(p, smem, st);
-    if (p.f.fmt == 4 && gi == 1) return launch_nb<4, 1, 0>(p, smem, st);
-    if (p.f.fmt == 2 && gi == 3) return launch_nb<2, 3, 0>(p, smem, st);
+    if (p.f.fmt == 4) return launch_t<4, 0>(p, smem, st);
+    if (p.f.fmt == 2) return launch_t<2, 0>(p, smem, st);
     return cudaErrorInvalidValue;
 }
 
@@ -1082,51 +1040,38 @@ bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan) {
     if (T < 1 || T > MAXTOK) return false;
     if (c.act != COLI_ACT_BF16) return false;
     if (c.wfmt != COLI_W_INT4 && c.wfmt != COLI_W_INT2) return false;
-    const int gs = c.group_size;                      // 0 or 64 (int4 only)
-    if (gs && (c.wfmt != COLI_W_INT4 || gs != 64 || c.hidden != 6144)) return false;
+    const int gsz = c.group_size;                     // 0 or 64 (int4 only)
+    if (gsz && (c.wfmt != COLI_W_INT4 || gsz != 64)) return false;
     // router: blocks of 32 experts; groups are whole blocks; at most 32 candidates, K <= 8
     if (c.n_experts % 32 || c.n_experts > 32 * RMAX_BLOCKS || c.top_k > 8 || c.n_group > 32) return false;
     {
-        const int gsz = c.n_experts / c.n_group;
+        const int epg = c.n_experts / c.n_group;
         const bool grouped = c.n_group > 1 && c.topk_group < c.n_group;
-        if (grouped && gsz % 32) return false;
-        const int kept_blocks = grouped ? c.topk_group * gsz / 32 : c.n_experts / 32;
+        if (grouped && epg % 32) return false;
+        const int kept_blocks = grouped ? c.topk_group * epg / 32 : c.n_experts / 32;
         if (kept_blocks * c.top_k > 32) return false;
     }
     if (c.top_k * T > 32) return false;
-    // activations: 4 elements per consumer thread per 2048 (hidden 2048 or 6144)
-    if (c.hidden != 2048 && c.hidden != 6144) return false;
     const int bits = c.wfmt;
+    const int cpc = bits == 4 ? 128 : 256, eg = bits == 4 ? 8 : 16;
     const int rb_h = c.hidden * bits / 8, rb_i = c.inter * bits / 8;
-    const int cpc = bits == 4 ? 128 : 256;
-    if (c.hidden % cpc || c.inter % 8) return false;
-    // phase-1 stage: 16 rows x SK1 bytes, SK1 a multiple of 8 warps x 64 bytes, at most 1536
-    int nks1 = 1;
-    while (rb_h / nks1 > 1536 || rb_h % nks1) ++nks1;
-    const int SK1 = rb_h / nks1;
-    if (SK1 % (GW * 64)) return false;
-    // phase-2 stage: the CTA's rows x 512 bytes (8 chunks, one per warp of a half)
-    if (rb_i % 512) return false;
-    const int nch2 = rb_i / 64;
-    if (nch2 != 8 && nch2 != 16) return false;
-    const int SK2 = 512;
+    // phase 1: each of a group's 8 warps takes whole 64-byte chunks of a row
+    if (c.hidden % cpc || c.hidden % eg || rb_h % (GW * 64) || c.inter % 8) return false;
+    // phase 2: one 64-byte chunk of the down rows per warp, at most 16
+    if (rb_i % 64 || NCW % (rb_i / 64) || c.inter % cpc) return false;
     const int sms = device_sm_count();
     const int rows2 = (c.hidden + sms - 1) / sms;
-    if (rows2 > 48 || c.inter / 8 < 1) return false;
+    if (rows2 > 48) return false;
     if ((c.n_experts + sms - 1) / sms > 2) return false;  // at most two router rows per CTA
     const int NB = 3 * T <= 8 ? 1 : 2;
     const int mpc = bits == 4 ? 4 : 8;
     const size_t colblk = 4 * 8 * mpc;
     DecodePlan pl = {};
     pl.grid = sms;
-    pl.SK1 = SK1;
-    pl.SK2 = SK2;
-    const int pad = gs ? 16 : ROWPAD;
-    const int st1 = SK1 + pad, st2 = SK2 + pad;
-    const int gps1 = gs ? SK1 * 8 / bits / gs : 0, gps2 = gs ? SK2 * 8 / bits / gs : 0;
-    const int sb1 = 16 * st1 + (gs ? 16 * 4 * gps1 : 64);  // 16 rows + their scales
-    pl.st_sd = rows2 * st2;
-    const int sb2 = pl.st_sd + (gs ? rows2 * 4 * gps2 : ((rows2 + 8 + 3) / 4) * 16);
+    const int nsh = gsz ? c.hidden / gsz : 1, nsi = gsz ? c.inter / gsz : 1;
+    const int sb1 = 16 * rb_h + 2 * (gsz ? 8 * nsh * 4 : 32);          // tile rows + their scales
+    pl.st_sd = ((rows2 * rb_i) + 15) / 16 * 16;
+    const int sb2 = pl.st_sd + (gsz ? rows2 * nsi * 4 : ((rows2 + 6 + 3) / 4) * 16);
     pl.SB = ((sb1 > sb2 ? sb1 : sb2) + 127) / 128 * 128;
     size_t o = 1024;                                  // mbarriers (up to 60 stages)
     pl.off_route = o; o += (sizeof(RouteCache) + 127) / 128 * 128;
@@ -1145,7 +1090,7 @@ bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan) {
     o = (o + 1023) / 1024 * 1024;
     pl.off_ring = o;
     const size_t budget = device_smem_optin() - 1024;
-    if (o + 3 * static_cast<size_t>(pl.SB) > budget) return false;
+    if (o + 2 * static_cast<size_t>(pl.SB) > budget) return false;
     pl.S = static_cast<int>((budget - o) / pl.SB);
     if (pl.S > 60) pl.S = 60;
     pl.smem = o + static_cast<size_t>(pl.S) * pl.SB;
@@ -1154,7 +1099,7 @@ bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan) {
 }
 
 static void fill_plan(DecodeParams &p, const DecodePlan &pl) {
-    p.grid = pl.grid; p.SK1 = pl.SK1; p.SK2 = pl.SK2; p.S = pl.S; p.SB = pl.SB; p.st_sd = pl.st_sd;
+    p.grid = pl.grid; p.S = pl.S; p.SB = pl.SB; p.st_sd = pl.st_sd;
     p.off_route = pl.off_route; p.off_rtok = pl.off_rtok; p.off_gate = pl.off_gate;
     p.off_red1 = pl.off_red1; p.off_x = pl.off_x; p.off_ring = pl.off_ring;
 }

@@ -41,7 +41,7 @@ constexpr int WS_HEADER = 256;
 
 // Shared-memory plan of the fused decode kernel (decode.cu).
 struct DecodePlan {
-    int grid, S, SB, SK1, SK2, st_sd;                 // ring: S stages of SB bytes
+    int grid, S, SB, st_sd;                           // ring: S stages of SB bytes
     size_t off_route, off_rtok, off_gate, off_red1, off_x, off_ring, smem;
 };
 
@@ -61,7 +61,7 @@ struct DecodeParams {
     long long wait_cycles;  // bound of every device-side wait (0: the default, ~2 s)
     unsigned gate_extra;    // added to the grid-barrier targets (nonzero only to test the bound)
     // plan (copied from DecodePlan)
-    int grid, S, SB, SK1, SK2, st_sd;
+    int grid, S, SB, st_sd;
     size_t off_route, off_rtok, off_gate, off_red1, off_x, off_ring;
 };
 
