@@ -310,7 +310,7 @@ def measure(args, wl, T, n_layers, K, W, rank, world, dist, dev, label):
             "bound": "tensor", "kernel": tc_kernel, "achieved": round(tf_s, 1), "peak": peak_t,
             "unit": "TFLOP/s", "frac": round(tf_s / peak_t, 4), "traffic": traffic,
             "peak_source": f"{peak_kind} bf16_tflops{'_sustained' if bf16s else ''} (int8 with two "
-                           "activation slices runs algorithmic flops at the bf16 rate); frac of measured",
+                           f"activation slices runs algorithmic flops at the bf16 rate); frac of {peak_kind}",
             "launch_us": round(ffn_ms * 1e3, 2),
             "hbm_gbs_of_weights": round(ffn_bytes / (ffn_ms / 1e3) / 1e9, 1),
         }
@@ -322,7 +322,7 @@ def measure(args, wl, T, n_layers, K, W, rank, world, dist, dev, label):
                        tc_kernel if n_kern == 7 else "expert FFN (gate/up GEMV + down GEMV with fused combine)"),
             "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
             "frac": round(achieved / hbm, 4), "traffic": traffic,
-            "peak_source": f"{peak_kind} hbm_gbs (copy bandwidth); frac of measured",
+            "peak_source": f"{peak_kind} hbm_gbs (copy bandwidth); frac of {peak_kind}",
             "launch_us": round(ffn_ms * 1e3, 2),
         }
     # whole-layer roofline: max(bytes / HBM, flops / tensor peak) over the measured step time

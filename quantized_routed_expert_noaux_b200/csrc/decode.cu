@@ -451,103 +451,114 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
     auto bf = [](const uint32_t (&w)[EG / 2], int k) -> float {
         return __uint_as_float((k & 1) ? (w[k >> 1] & 0xffff0000u) : (w[k >> 1] << 16));
     };
+    constexpr int RQ = FMT == 4 ? 2 : 1;              // activation groups per thread (NQ <= RQ * NC)
     {
-        double acc[2][MAXT];
-        float mx[MAXT];
+        // every load is issued before any arithmetic: the activations of all tokens and this
+        // CTA's router rows, held in registers through the conversion below
+        uint32_t xw[MAXT][RQ][EG / 2];
+        float wv[2][RQ][EG];
 #pragma unroll
-        for (int t = 0; t < MAXT; ++t) { acc[0][t] = acc[1][t] = 0.0; mx[t] = 0.f; }
-        for (int q = ct; q < NQ; q += NC) {
-            float wv[2][EG];
+        for (int r = 0; r < RQ; ++r) {
+            const int q = ct + NC * r;
+            const bool in = q < NQ;
+#pragma unroll
+            for (int t = 0; t < MAXT; ++t) {
+                if (t < T && in) {
+                    load_x(t, q, xw[t][r]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < EG / 2; ++i) xw[t][r][i] = 0u;
+                }
+            }
 #pragma unroll
             for (int j = 0; j < 2; ++j)
 #pragma unroll
                 for (int i = 0; i < EG / 4; ++i) {
-                    const float4 v = j < ne ? __ldg(reinterpret_cast<const float4 *>(p.Wr + static_cast<size_t>(e0 + j) * f.H + q * EG) + i)
-                                            : make_float4(0.f, 0.f, 0.f, 0.f);
-                    wv[j][4 * i] = v.x; wv[j][4 * i + 1] = v.y; wv[j][4 * i + 2] = v.z; wv[j][4 * i + 3] = v.w;
+                    const float4 v = (j < ne && in) ? __ldg(reinterpret_cast<const float4 *>(p.Wr + static_cast<size_t>(e0 + j) * f.H + q * EG) + i)
+                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+                    wv[j][r][4 * i] = v.x; wv[j][r][4 * i + 1] = v.y; wv[j][r][4 * i + 2] = v.z; wv[j][r][4 * i + 3] = v.w;
                 }
-#pragma unroll
-            for (int t = 0; t < MAXT; ++t) {
-                if (t < T) {
-                    uint32_t w[EG / 2];
-                    load_x(t, q, w);
-#pragma unroll
-                    for (int k = 0; k < EG; ++k) {
-                        const float xv = bf(w, k);
-                        mx[t] = fmaxf(mx[t], fabsf(xv));
-                        acc[0][t] = fma(static_cast<double>(wv[0][k]), static_cast<double>(xv), acc[0][t]);
-                        acc[1][t] = fma(static_cast<double>(wv[1][k]), static_cast<double>(xv), acc[1][t]);
-                    }
-                }
-            }
         }
+        // gate partial dot products (exact double products, double sums) and row maxima
 #pragma unroll
         for (int t = 0; t < MAXT; ++t) {
+            double a0 = 0.0, a1 = 0.0;
+            float mx = 0.f;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                mx[t] = fmaxf(mx[t], __shfl_xor_sync(FULL, mx[t], o));
-                acc[0][t] += __shfl_xor_sync(FULL, acc[0][t], o);
-                acc[1][t] += __shfl_xor_sync(FULL, acc[1][t], o);
-            }
-            if (lane == 0) {
-                xmax[cw * MAXTOK + t] = mx[t];
-                gpart[cw * 2 * MAXTOK + t] = acc[0][t];
-                gpart[cw * 2 * MAXTOK + MAXTOK + t] = acc[1][t];
-            }
-        }
-    }
-    cons_sync();
-    if (ct < ne * T) {  // one logit per thread of warp 0: the 16 warps' partials in order
-        const int j = ct / T, t = ct % T;
-        double sum = 0.0;
-        for (int w2 = 0; w2 < NCW; ++w2) sum += gpart[w2 * 2 * MAXTOK + j * MAXTOK + t];
-        p.logits[static_cast<size_t>(t) * f.E + e0 + j] = static_cast<float>(sum);
-        __threadfence();
-    }
-    if (cw == 0 && p.route_here) {
-        __syncwarp();
-        if (lane == 0) atomicAdd(p.gbar, 1u);
-    }
-    // activation slices: X = rint(x * 2^(22 - e)), max|x| < 2^e, written as whole B words
-#pragma unroll
-    for (int t = 0; t < MAXT; ++t) {
-        if (t < T) {
-            float m = 0.f;
-            for (int w2 = 0; w2 < NCW; ++w2) m = fmaxf(m, xmax[w2 * MAXTOK + t]);
-            int ex = 0;
-            if (m > 0.f) frexpf(m, &ex);
-            const float up = ldexpf(1.0f, 22 - ex);
-            if (ct == 0) rc.xscale[t] = ldexpf(1.0f, ex - 22);
-            for (int q = ct; q < NQ; q += NC) {
-                uint32_t w[EG / 2];
-                load_x(t, q, w);
-                uint32_t sl[3][EG];  // slice bytes of the EG elements
+            for (int r = 0; r < RQ; ++r)
 #pragma unroll
                 for (int k = 0; k < EG; ++k) {
-                    int s0, s1, s2;
-                    slices3(__float2int_rn(bf(w, k) * up), s0, s1, s2);
-                    sl[0][k] = static_cast<uint32_t>(s0) & 0xffu;
-                    sl[1][k] = static_cast<uint32_t>(s1) & 0xffu;
-                    sl[2][k] = static_cast<uint32_t>(s2) & 0xffu;
+                    const float xv = bf(xw[t][r], k);
+                    mx = fmaxf(mx, fabsf(xv));
+                    a0 = fma(static_cast<double>(wv[0][r][k]), static_cast<double>(xv), a0);
+                    a1 = fma(static_cast<double>(wv[1][r][k]), static_cast<double>(xv), a1);
                 }
-                const int h0 = q * EG, kc = h0 / CPC, p0 = h0 % CPC;
 #pragma unroll
-                for (int s = 0; s < 3; ++s) {
-                    const int col = 3 * t + s;
-                    unsigned char *blk = xb + (static_cast<size_t>(kc) * NCOL + col) * colblk;
-                    if (FMT == 4) {  // elements p0 + 2j (+1) -> byte j of register half 0 (1)
-                        const int tg = p0 >> 5, m = (p0 >> 3) & 3;
+            for (int o = 16; o > 0; o >>= 1) {
+                mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
+                a0 += __shfl_xor_sync(FULL, a0, o);
+                a1 += __shfl_xor_sync(FULL, a1, o);
+            }
+            if (lane == 0) {
+                xmax[cw * MAXTOK + t] = mx;
+                gpart[cw * 2 * MAXTOK + t] = a0;
+                gpart[cw * 2 * MAXTOK + MAXTOK + t] = a1;
+            }
+        }
+        cons_sync();
+        if (ct < ne * T) {  // one logit per thread of warp 0: the 16 warps' partials in order
+            const int j = ct / T, t = ct % T;
+            double sum = 0.0;
+            for (int w2 = 0; w2 < NCW; ++w2) sum += gpart[w2 * 2 * MAXTOK + j * MAXTOK + t];
+            p.logits[static_cast<size_t>(t) * f.E + e0 + j] = static_cast<float>(sum);
+            __threadfence();
+        }
+        if (cw == 0 && p.route_here) {
+            __syncwarp();
+            if (lane == 0) atomicAdd(p.gbar, 1u);
+        }
+        // activation slices: X = rint(x * 2^(22 - e)), max|x| < 2^e, written as whole B words
 #pragma unroll
-                        for (int hf = 0; hf < 2; ++hf) {
-                            const uint32_t word = sl[s][hf] | (sl[s][2 + hf] << 8) | (sl[s][4 + hf] << 16) | (sl[s][6 + hf] << 24);
-                            *reinterpret_cast<uint32_t *>(blk + b_off<FMT>(col, tg, m, hf, 0)) = word;
-                        }
-                    } else {         // elements p0 + 4j + k -> byte j of field k's register
-                        const int tg = p0 >> 6, i4 = (p0 >> 4) & 3;
+        for (int t = 0; t < MAXT; ++t) {
+            if (t < T) {
+                float m = 0.f;
+                for (int w2 = 0; w2 < NCW; ++w2) m = fmaxf(m, xmax[w2 * MAXTOK + t]);
+                int ex = 0;
+                if (m > 0.f) frexpf(m, &ex);
+                const float up = ldexpf(1.0f, 22 - ex);
+                if (ct == 0) rc.xscale[t] = ldexpf(1.0f, ex - 22);
 #pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const uint32_t word = sl[s][k] | (sl[s][4 + k] << 8) | (sl[s][8 + k] << 16) | (sl[s][12 + k] << 24);
-                            *reinterpret_cast<uint32_t *>(blk + b_off<FMT>(col, tg, 2 * i4 + (k >> 1), k & 1, 0)) = word;
+                for (int r = 0; r < RQ; ++r) {
+                    const int q = ct + NC * r;
+                    if (q >= NQ) continue;
+                    uint32_t sl[3][EG];  // slice bytes of the EG elements
+#pragma unroll
+                    for (int k = 0; k < EG; ++k) {
+                        int s0, s1, s2;
+                        slices3(__float2int_rn(bf(xw[t][r], k) * up), s0, s1, s2);
+                        sl[0][k] = static_cast<uint32_t>(s0) & 0xffu;
+                        sl[1][k] = static_cast<uint32_t>(s1) & 0xffu;
+                        sl[2][k] = static_cast<uint32_t>(s2) & 0xffu;
+                    }
+                    const int h0 = q * EG, kc = h0 / CPC, p0 = h0 % CPC;
+#pragma unroll
+                    for (int s = 0; s < 3; ++s) {
+                        const int col = 3 * t + s;
+                        unsigned char *blk = xb + (static_cast<size_t>(kc) * NCOL + col) * colblk;
+                        if (FMT == 4) {  // elements p0 + 2j (+1) -> byte j of register half 0 (1)
+                            const int tg = p0 >> 5, m2 = (p0 >> 3) & 3;
+#pragma unroll
+                            for (int hf = 0; hf < 2; ++hf) {
+                                const uint32_t word = sl[s][hf] | (sl[s][2 + hf] << 8) | (sl[s][4 + hf] << 16) | (sl[s][6 + hf] << 24);
+                                *reinterpret_cast<uint32_t *>(blk + b_off<FMT>(col, tg, m2, hf, 0)) = word;
+                            }
+                        } else {         // elements p0 + 4j + k -> byte j of field k's register
+                            const int tg = p0 >> 6, i4 = (p0 >> 4) & 3;
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                const uint32_t word = sl[s][k] | (sl[s][4 + k] << 8) | (sl[s][8 + k] << 16) | (sl[s][12 + k] << 24);
+                                *reinterpret_cast<uint32_t *>(blk + b_off<FMT>(col, tg, 2 * i4 + (k >> 1), k & 1, 0)) = word;
+                            }
                         }
                     }
                 }
@@ -834,8 +845,9 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
     const int nact = nch2 < NCW ? nch2 : NCW;         // warps with a chunk
     const bool active2 = cw < nch2;
     const int nwe = f.S + U;
-    unsigned char *hb = sm + p.off_x + static_cast<size_t>(cw) * NCOL * colblk;  // this warp's h slices
-    const float *sdp0 = nullptr;
+    // this warp's two h-slice blocks (two experts in flight)
+    unsigned char *hbA = sm + p.off_x + static_cast<size_t>(cw) * (TT <= 2 ? 2 : 1) * NCOL * colblk;
+    unsigned char *hbB = hbA + NCOL * colblk;  // used when two experts are in flight (TT <= 2)
     float acc[RT2][NB][4];
 #pragma unroll
     for (int rt = 0; rt < RT2; ++rt)
@@ -843,8 +855,8 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
         for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
             for (int i = 0; i < 4; ++i) acc[rt][nb][i] = 0.f;
-    float hv[MAXT][CPL];
-    auto fetch_h = [&](int we) {
+    // This warp's chunk of each slot's h, fetched two experts ahead into two register buffers.
+    auto fetch_h = [&](int we, float (&hv)[MAXT][CPL]) {
 #pragma unroll
         for (int t = 0; t < MAXT; ++t) {
             const int slot = t < T ? rc.slot[we][t] : -1;
@@ -857,117 +869,191 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
             }
         }
     };
-    (void)sdp0;
-    if (nwe > 0) fetch_h(0);
-    for (int we = 0; we < nwe; ++we) {
-        const int s = (seq + we) % S;
-        const uint32_t par = ((seq + we) / S) & 1;
-        // h of this expert's slots -> 24-bit fixed point per chunk, three byte slices
-        float fcol[NB][2];
-        if (active2) {
+    // h -> 24-bit fixed point per chunk (three byte slices) in this warp's B block, and the
+    // column factors (combine weight x chunk scale x slice weight).  Lane l holds elements
+    // l * CPL + k; two neighbouring lanes fill each 32-bit B word, exchanged by one shuffle.
+    auto convert_h = [&](int we, const float (&hv)[MAXT][CPL], float (&fcol)[NB][2], unsigned char *hb) {
 #pragma unroll
-            for (int nb = 0; nb < NB; ++nb) fcol[nb][0] = fcol[nb][1] = 0.f;
+        for (int nb = 0; nb < NB; ++nb) fcol[nb][0] = fcol[nb][1] = 0.f;
+        const bool odd = lane & 1;
+        const int tg = lane >> 3;
 #pragma unroll
-            for (int t = 0; t < MAXT; ++t) {
-                if (t < T) {
-                    float m = 0.f;
+        for (int t = 0; t < MAXT; ++t) {
+            if (t >= T) continue;
+            float m = 0.f;
 #pragma unroll
-                    for (int k = 0; k < CPL; ++k) m = fmaxf(m, fabsf(hv[t][k]));
+            for (int k = 0; k < CPL; ++k) m = fmaxf(m, fabsf(hv[t][k]));
 #pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
-                    int ex = 0;
-                    if (m > 0.f) frexpf(m, &ex);
-                    const float up = ldexpf(1.0f, 22 - ex);
-                    // column factors of this token: combine weight x scale x slice weight
-                    const float base = rc.wgt[we][t] * ldexpf(1.0f, ex - 22) / F::MUL;
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
+            int ex = 0;
+            if (m > 0.f) frexpf(m, &ex);
+            const float up = ldexpf(1.0f, 22 - ex);
+            const float base = rc.wgt[we][t] * ldexpf(1.0f, ex - 22) / F::MUL;
 #pragma unroll
-                    for (int nb = 0; nb < NB; ++nb)
+            for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-                        for (int i = 0; i < 2; ++i) {
-                            const int col = nb * 8 + 2 * tig + i;
-                            if (col / 3 == t) fcol[nb][i] = base * (col % 3 == 0 ? 1.0f : (col % 3 == 1 ? 256.0f : 65536.0f));
-                        }
+                for (int i = 0; i < 2; ++i) {
+                    const int col = nb * 8 + 2 * tig + i;
+                    if (col / 3 == t) fcol[nb][i] = base * (col % 3 == 0 ? 1.0f : (col % 3 == 1 ? 256.0f : 65536.0f));
+                }
+            uint32_t by[3][CPL];  // slice bytes
 #pragma unroll
-                    for (int k = 0; k < CPL; ++k) {
-                        int s0, s1, s2;
-                        slices3(__float2int_rn(hv[t][k] * up), s0, s1, s2);
-                        int tg, m2, hf, by;
-                        F::place(lane * CPL + k, tg, m2, hf, by);
-                        hb[(3 * t + 0) * colblk + b_off<FMT>(3 * t + 0, tg, m2, hf, by)] = static_cast<unsigned char>(s0 & 0xff);
-                        hb[(3 * t + 1) * colblk + b_off<FMT>(3 * t + 1, tg, m2, hf, by)] = static_cast<unsigned char>(s1 & 0xff);
-                        hb[(3 * t + 2) * colblk + b_off<FMT>(3 * t + 2, tg, m2, hf, by)] = static_cast<unsigned char>(s2 & 0xff);
+            for (int k = 0; k < CPL; ++k) {
+                int s0, s1, s2;
+                slices3(__float2int_rn(hv[t][k] * up), s0, s1, s2);
+                by[0][k] = static_cast<uint32_t>(s0) & 0xffu;
+                by[1][k] = static_cast<uint32_t>(s1) & 0xffu;
+                by[2][k] = static_cast<uint32_t>(s2) & 0xffu;
+            }
+#pragma unroll
+            for (int sidx = 0; sidx < 3; ++sidx) {
+                const int col = 3 * t + sidx;
+                unsigned char *blk = hb + col * colblk;
+                if (FMT == 4) {
+                    // elements 4l + {0, 2} -> bytes 2(l&1) + {0, 1} of half 0; 4l + {1, 3} of half 1
+                    const uint32_t h0 = by[sidx][0] | (by[sidx][2] << 8), h1 = by[sidx][1] | (by[sidx][3] << 8);
+                    const uint32_t got = __shfl_xor_sync(FULL, odd ? h0 : h1, 1);
+                    const uint32_t word = odd ? (got | (h1 << 16)) : (h0 | (got << 16));
+                    const int m2 = (lane >> 1) & 3;
+                    *reinterpret_cast<uint32_t *>(blk + b_off<FMT>(col, tg, m2, odd ? 1 : 0, 0)) = word;
+                } else {
+                    // elements 8l + kk + {0, 4} -> bytes 2(l&1) + {0, 1} of field kk's register;
+                    // the even lane stores fields 0, 1 and the odd lane fields 2, 3
+                    const int i4 = (lane >> 1) & 3;
+                    uint32_t hw[4];
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) hw[kk] = by[sidx][kk] | (by[sidx][4 + kk] << 8);
+#pragma unroll
+                    for (int e2 = 0; e2 < 2; ++e2) {
+                        const uint32_t got = __shfl_xor_sync(FULL, odd ? hw[e2] : hw[2 + e2], 1);
+                        const int kk = odd ? 2 + e2 : e2;
+                        const uint32_t word = odd ? (got | (hw[kk] << 16)) : (hw[kk] | (got << 16));
+                        *reinterpret_cast<uint32_t *>(blk + b_off<FMT>(col, tg, 2 * i4 + (kk >> 1), kk & 1, 0)) = word;
                     }
                 }
             }
         }
         __syncwarp();
-        if (we + 1 < nwe) fetch_h(we + 1);
-        if (ok && active2 && !mbar_wait(full_bar(s), par, bound)) ok = false;
+    };
+    // The down projection of work experts we and we + 1 (when `two`) for this warp's chunk, once
+    // their stages have landed.  The two experts' instruction streams are independent, so their
+    // shared-memory loads and MMAs overlap; without a second expert the second stream repeats
+    // the first with zero column factors.
+    constexpr int NE = TT <= 2 ? 2 : 1;  // experts in flight (register budget)
+    auto down_pair = [&](int we, bool two, const float (&fA)[NB][2], const float (&fB)[NB][2]) {
+        const int sA = (seq + we) % S, sB = (seq + we + 1) % S;
+        const uint32_t pA = ((seq + we) / S) & 1, pB = ((seq + we + 1) / S) & 1;
+        if (ok && active2 && !mbar_wait(full_bar(sA), pA, bound)) ok = false;
+        if (ok && active2 && two && !mbar_wait(full_bar(sB), pB, bound)) ok = false;
         ok = __all_sync(FULL, ok);
         if (ok && active2) {
-            const unsigned char *st = ring + static_cast<size_t>(s) * p.SB;
-            const float *sdp = reinterpret_cast<const float *>(st + p.st_sd) + (j_lo - a0d);
-            const float *sdg = reinterpret_cast<const float *>(st + p.st_sd);  // [nrows][nsi]
-            uint32_t bfr[MPC][NB][2];
+            const unsigned char *st[2] = {ring + static_cast<size_t>(sA) * p.SB,
+                                          ring + static_cast<size_t>(two ? sB : sA) * p.SB};
+            const unsigned char *hbs[2] = {hbA, two ? hbB : hbA};
+            uint32_t bfr[NE][MPC][NB][2];
 #pragma unroll
-            for (int u = 0; u < MPC / 2; ++u)
+            for (int e = 0; e < NE; ++e)
 #pragma unroll
-                for (int nb = 0; nb < NB; ++nb) {
-                    const int col = nb * 8 + g8;
-                    const uint4 v = col < NCOL ? load_b2<FMT>(hb + col * colblk, col, tig, u) : make_uint4(0u, 0u, 0u, 0u);
-                    bfr[2 * u][nb][0] = v.x;
-                    bfr[2 * u][nb][1] = v.y;
-                    bfr[2 * u + 1][nb][0] = v.z;
-                    bfr[2 * u + 1][nb][1] = v.w;
-                }
+                for (int u = 0; u < MPC / 2; ++u)
+#pragma unroll
+                    for (int nb = 0; nb < NB; ++nb) {
+                        const int col = nb * 8 + g8;
+                        const uint4 v = col < NCOL ? load_b2<FMT>(hbs[e] + col * colblk, col, tig, u) : make_uint4(0u, 0u, 0u, 0u);
+                        bfr[e][2 * u][nb][0] = v.x;
+                        bfr[e][2 * u][nb][1] = v.y;
+                        bfr[e][2 * u + 1][nb][0] = v.z;
+                        bfr[e][2 * u + 1][nb][1] = v.w;
+                    }
 #pragma unroll
             for (int rt = 0; rt < RT2; ++rt) {
                 const int ra = rt * 16 + g8, rbw = ra + 8;
                 if (rt * 16 < nrows) {
-                    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-                    const uint4 qa = ra < nrows ? *reinterpret_cast<const uint4 *>(st + ra * rb_i + 64 * cw + 16 * tig) : z;
-                    const uint4 qb = rbw < nrows ? *reinterpret_cast<const uint4 *>(st + rbw * rb_i + 64 * cw + 16 * tig) : z;
-                    int D[NB][4], D1[NB][4];
 #pragma unroll
-                    for (int nb = 0; nb < NB; ++nb)
+                    for (int e = 0; e < NE; ++e) {
+                        const float (&fc)[NB][2] = e == 0 ? fA : fB;
+                        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+                        const uint4 qa = ra < nrows ? *reinterpret_cast<const uint4 *>(st[e] + ra * rb_i + 64 * cw + 16 * tig) : z;
+                        const uint4 qb = rbw < nrows ? *reinterpret_cast<const uint4 *>(st[e] + rbw * rb_i + 64 * cw + 16 * tig) : z;
+                        int D[NB][4], D1[NB][4];
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) { D[nb][i] = 0; D1[nb][i] = 0; }
+                        for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-                    for (int m = 0; m < MPC; ++m) {
-                        uint32_t a0, a2, a1, a3;
-                        F::unpack(qa, m, a0, a2);
-                        F::unpack(qb, m, a1, a3);
+                            for (int i = 0; i < 4; ++i) { D[nb][i] = 0; D1[nb][i] = 0; }
 #pragma unroll
-                        for (int nb = 0; nb < NB; ++nb) mma_chunk(D[nb], D1[nb], a0, a1, a2, a3, bfr[m][nb][0], bfr[m][nb][1]);
-                    }
-                    float sda, sdb, sda1 = 0.f, sdb1 = 0.f;
-                    if (GS) {  // groups 2 cw and 2 cw + 1 of rows ra and rbw
-                        sda = ra < nrows ? sdg[ra * f.nsi + 2 * cw] : 0.f;
-                        sda1 = ra < nrows ? sdg[ra * f.nsi + 2 * cw + 1] : 0.f;
-                        sdb = rbw < nrows ? sdg[rbw * f.nsi + 2 * cw] : 0.f;
-                        sdb1 = rbw < nrows ? sdg[rbw * f.nsi + 2 * cw + 1] : 0.f;
-                    } else {
-                        sda = ra < nrows ? sdp[ra] : 0.f;
-                        sdb = rbw < nrows ? sdp[rbw] : 0.f;
-                    }
+                        for (int m = 0; m < MPC; ++m) {
+                            uint32_t a0, a2, a1, a3;
+                            F::unpack(qa, m, a0, a2);
+                            F::unpack(qb, m, a1, a3);
 #pragma unroll
-                    for (int nb = 0; nb < NB; ++nb) {
-                        acc[rt][nb][0] = __fmaf_rn(static_cast<float>(D[nb][0]), sda * fcol[nb][0], acc[rt][nb][0]);
-                        acc[rt][nb][1] = __fmaf_rn(static_cast<float>(D[nb][1]), sda * fcol[nb][1], acc[rt][nb][1]);
-                        acc[rt][nb][2] = __fmaf_rn(static_cast<float>(D[nb][2]), sdb * fcol[nb][0], acc[rt][nb][2]);
-                        acc[rt][nb][3] = __fmaf_rn(static_cast<float>(D[nb][3]), sdb * fcol[nb][1], acc[rt][nb][3]);
-                        if (GS) {
-                            acc[rt][nb][0] = __fmaf_rn(static_cast<float>(D1[nb][0]), sda1 * fcol[nb][0], acc[rt][nb][0]);
-                            acc[rt][nb][1] = __fmaf_rn(static_cast<float>(D1[nb][1]), sda1 * fcol[nb][1], acc[rt][nb][1]);
-                            acc[rt][nb][2] = __fmaf_rn(static_cast<float>(D1[nb][2]), sdb1 * fcol[nb][0], acc[rt][nb][2]);
-                            acc[rt][nb][3] = __fmaf_rn(static_cast<float>(D1[nb][3]), sdb1 * fcol[nb][1], acc[rt][nb][3]);
+                            for (int nb = 0; nb < NB; ++nb) mma_chunk(D[nb], D1[nb], a0, a1, a2, a3, bfr[e][m][nb][0], bfr[e][m][nb][1]);
+                        }
+                        const float *sdp = reinterpret_cast<const float *>(st[e] + p.st_sd) + (j_lo - a0d);
+                        const float *sdg = reinterpret_cast<const float *>(st[e] + p.st_sd);  // [nrows][nsi]
+                        float sda, sdb, sda1 = 0.f, sdb1 = 0.f;
+                        if (GS) {  // groups 2 cw and 2 cw + 1 of rows ra and rbw
+                            sda = ra < nrows ? sdg[ra * f.nsi + 2 * cw] : 0.f;
+                            sda1 = ra < nrows ? sdg[ra * f.nsi + 2 * cw + 1] : 0.f;
+                            sdb = rbw < nrows ? sdg[rbw * f.nsi + 2 * cw] : 0.f;
+                            sdb1 = rbw < nrows ? sdg[rbw * f.nsi + 2 * cw + 1] : 0.f;
+                        } else {
+                            sda = ra < nrows ? sdp[ra] : 0.f;
+                            sdb = rbw < nrows ? sdp[rbw] : 0.f;
+                        }
+#pragma unroll
+                        for (int nb = 0; nb < NB; ++nb) {
+                            acc[rt][nb][0] = __fmaf_rn(static_cast<float>(D[nb][0]), sda * fc[nb][0], acc[rt][nb][0]);
+                            acc[rt][nb][1] = __fmaf_rn(static_cast<float>(D[nb][1]), sda * fc[nb][1], acc[rt][nb][1]);
+                            acc[rt][nb][2] = __fmaf_rn(static_cast<float>(D[nb][2]), sdb * fc[nb][0], acc[rt][nb][2]);
+                            acc[rt][nb][3] = __fmaf_rn(static_cast<float>(D[nb][3]), sdb * fc[nb][1], acc[rt][nb][3]);
+                            if (GS) {
+                                acc[rt][nb][0] = __fmaf_rn(static_cast<float>(D1[nb][0]), sda1 * fc[nb][0], acc[rt][nb][0]);
+                                acc[rt][nb][1] = __fmaf_rn(static_cast<float>(D1[nb][1]), sda1 * fc[nb][1], acc[rt][nb][1]);
+                                acc[rt][nb][2] = __fmaf_rn(static_cast<float>(D1[nb][2]), sdb1 * fc[nb][0], acc[rt][nb][2]);
+                                acc[rt][nb][3] = __fmaf_rn(static_cast<float>(D1[nb][3]), sdb1 * fc[nb][1], acc[rt][nb][3]);
+                            }
                         }
                     }
                 }
             }
         }
         __syncwarp();
-        if (ok && active2 && lane == 0) mbar_arrive_cnt(empty_bar(s), NCW / nact);
+        if (ok && active2 && lane == 0) {
+            mbar_arrive_cnt(empty_bar(sA), NCW / nact);
+            if (two) mbar_arrive_cnt(empty_bar(sB), NCW / nact);
+        }
+        __syncwarp();  // the B blocks are rewritten for the next pair only after every lane read them
+    };
+    float hvA[MAXT][CPL];
+    float fZ[NB][2];
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb) fZ[nb][0] = fZ[nb][1] = 0.f;
+    if (TT <= 2) {  // two experts at a time; h fetched one pair ahead
+        float hvB[MAXT][CPL];
+        if (nwe > 0) fetch_h(0, hvA);
+        if (nwe > 1) fetch_h(1, hvB);
+        for (int we = 0; we < nwe; we += 2) {
+            const bool two = we + 1 < nwe;
+            float fA[NB][2], fB[NB][2];
+            if (active2) {
+                convert_h(we, hvA, fA, hbA);
+                if (two) convert_h(we + 1, hvB, fB, hbB);
+            }
+            if (!two) {
+#pragma unroll
+                for (int nb = 0; nb < NB; ++nb) fB[nb][0] = fB[nb][1] = 0.f;
+            }
+            if (we + 2 < nwe) fetch_h(we + 2, hvA);
+            if (we + 3 < nwe) fetch_h(we + 3, hvB);
+            down_pair(we, two, fA, fB);
+        }
+    } else {        // one expert at a time (registers), h one expert ahead
+        if (nwe > 0) fetch_h(0, hvA);
+        for (int we = 0; we < nwe; ++we) {
+            float fA[NB][2];
+            if (active2) convert_h(we, hvA, fA, hbA);
+            if (we + 1 < nwe) fetch_h(we + 1, hvA);
+            down_pair(we, false, fA, fZ);
+        }
     }
     if (!ok) atomicOr(f.err, COLI_DEVERR_TIMEOUT);
     // cross-warp reduction (the h slices are no longer needed: the region is reused)
@@ -1059,6 +1145,8 @@ bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan) {
     if (c.hidden % cpc || c.hidden % eg || rb_h % (GW * 64) || c.inter % 8) return false;
     // phase 2: one 64-byte chunk of the down rows per warp, at most 16
     if (rb_i % 64 || NCW % (rb_i / 64) || c.inter % cpc) return false;
+    // activations: at most two groups of eg per consumer thread (int4), one (int2)
+    if (c.hidden / eg > (bits == 4 ? 2 : 1) * NC) return false;
     const int sms = device_sm_count();
     const int rows2 = (c.hidden + sms - 1) / sms;
     if (rows2 > 48) return false;
@@ -1082,7 +1170,8 @@ bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan) {
     o = (o + 127) / 128 * 128;
     // activation slices (phase 1) | per-warp h slices, then the final reduction (phase 2)
     const size_t xbytes = static_cast<size_t>(c.hidden / cpc) * 3 * T * colblk;
-    const size_t hbytes = static_cast<size_t>(NCW) * 3 * T * colblk;
+    // per warp one block of h slices per expert in flight: two for up to two tokens, else one
+    const size_t hbytes = static_cast<size_t>(NCW) * (T <= 2 ? 2 : 1) * 3 * T * colblk;
     const size_t rbytes = static_cast<size_t>(NCW) * 3 * NB * 32 * 16;
     size_t abytes = xbytes > hbytes ? xbytes : hbytes;
     abytes = abytes > rbytes ? abytes : rbytes;
