@@ -74,6 +74,7 @@ WsLayout ws_layout(const coli_moe_config &c, int T) {
     const size_t E = static_cast<size_t>(c.n_experts);
     size_t o = 0;
     L.err = o;      o = align256(o + WS_HEADER);
+    L.dsl = o;      o = align256(o + WS_DSL_BYTES);
     L.logits = o;   o = align256(o + static_cast<size_t>(T) * E * 4);
     L.ids = o;      o = align256(o + n * 4);
     L.w = o;        o = align256(o + n * 4);
@@ -295,6 +296,8 @@ static DecodeParams make_decode(const coli_moe_config *c, const FfnParams &f, ch
     d.TG = c->topk_group;
     d.gbar = reinterpret_cast<unsigned *>(base + WS_GBAR);
     d.gdep = reinterpret_cast<unsigned *>(base + WS_GDEP);
+    const WsLayout L = ws_layout(*c, f.T);
+    d.dsl = reinterpret_cast<uint4 *>(base + L.dsl);
     d.wait_cycles = g_wait_cycles;
     d.gate_extra = g_unreachable ? 1000000u : 0u;
     return d;

@@ -93,6 +93,13 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
                  ::"r"(dst), "l"(src), "r"(bytes), "r"(mbar), "l"(policy) : "memory");
 }
+// 16-byte asynchronous copy global -> shared (through L2), completed per thread by commit groups
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 __device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
@@ -304,6 +311,33 @@ __device__ void route_select(const DecodeParams &p, int t, int lane, RouteToken 
     }
 }
 
+// The order of a CTA's jobs once the batch is routed, walked identically by the producer and the
+// consumers.  Routed tile tau (tau = 0 .. U*NRB - 1; work expert S + tau / NRB, row block
+// tau % NRB) belongs to CTA tau mod G, so every CTA takes its tiles of expert 0 first, then of
+// expert 1, and so on, and at any moment the CTAs read neighbouring tiles (measured on B200:
+// contiguous ranges per CTA are 8% slower at one token and 40% at four).  The down projection of work expert S + u (job kind 2; u = -1 is the
+// shared expert) follows the CTA's tiles of every expert up to u + lag.
+struct JobIter {
+    int j = 0;   // next tile of this CTA
+    int u = 0;   // next down projection (-S: the shared expert's)
+};
+__device__ __forceinline__ int next_job(JobIter &it, int b, int G, int NRB, int U, int S, int lag,
+                                        int &we, int &rb) {
+    const unsigned tau = static_cast<unsigned>(b) + static_cast<unsigned>(G) * it.j;  // < 2^31
+    const bool more = tau < static_cast<unsigned>(U) * static_cast<unsigned>(NRB);
+    const int te = more ? static_cast<int>(tau / static_cast<unsigned>(NRB)) : 0x7fffffff;
+    if (it.u < U && te > it.u + lag) {
+        we = S + it.u;
+        ++it.u;
+        return 2;
+    }
+    if (!more) return 0;
+    we = S + te;
+    rb = static_cast<int>(tau - static_cast<unsigned>(te) * static_cast<unsigned>(NRB));
+    ++it.j;
+    return 1;
+}
+
 // ------------------------------------------------------------------------- the kernel ------
 // Shared-memory regions (byte offsets from the plan): barriers | routing cache | per-token
 // routing scratch | gate partials | group reduction buffers | activation slices (phase 1)
@@ -319,6 +353,7 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
     constexpr int MAXT = TT;                          // tokens of this instantiation (T <= TT)
     constexpr int NB = (3 * TT + 7) / 8;              // 8-column MMA blocks (3 slices per token)
     constexpr int EG = FMT == 4 ? 8 : 16;             // activations converted together (whole B words)
+    constexpr int DSTR = 3 * MAXTOK * 32 * MPC + 16;  // bytes per (work expert, chunk) of converted h
     extern __shared__ __align__(1024) unsigned char sm[];
     const FfnParams &f = p.f;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -392,25 +427,31 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
             bulk_prefetch_l2(f.shared + f.off_wd + static_cast<size_t>(j_lo) * rb_i, static_cast<uint32_t>(nrows) * rb_i);
         if (ok && !mbar_wait(route_bar, 0, bound)) ok = false;
         if (ok) U = rc.U;
-        const long nr = static_cast<long>(U) * NRB;
-        const int r_lo = static_cast<int>(nr * b / G), r_hi = static_cast<int>(nr * (b + 1) / G);
-        for (int tau = r_lo; tau < r_hi && ok; ++tau) stage1(record(f.S + tau / NRB), tau % NRB);
-        // phase 2: every work expert's block of down rows and their scales
+        // a down-projection stage: the CTA's block of one work expert's down rows and their scales
         const int a1 = (j_hi + 3) & ~3;
         const uint32_t sdb = GS ? static_cast<uint32_t>(nrows) * f.nsi * 4 : 4u * (a1 - a0d);
-        for (int we = 0; we < f.S + U && ok; ++we) {
+        auto stage2 = [&](int we) {
             const uint8_t *rec = record(we);
             const int s = seq % S;
             const uint32_t par = (seq / S) & 1;
-            if (!mbar_wait(empty_bar(s), par ^ 1, bound)) { ok = false; break; }
+            if (!mbar_wait(empty_bar(s), par ^ 1, bound)) { ok = false; return; }
             ++seq;
-            if (rec == nullptr) { mbar_arrive(full_bar(s)); continue; }
+            if (rec == nullptr) { mbar_arrive(full_bar(s)); return; }
             const uint32_t dst = smem_u32(ring + static_cast<size_t>(s) * p.SB);
             mbar_expect_tx(full_bar(s), static_cast<uint32_t>(nrows) * rb_i + sdb);
             const uint64_t pl = we < f.S ? keep : pol;
             bulk_g2s(dst, rec + f.off_wd + static_cast<size_t>(j_lo) * rb_i, static_cast<uint32_t>(nrows) * rb_i, full_bar(s), pl);
             bulk_g2s(dst + p.st_sd, rec + f.off_sd + (GS ? static_cast<size_t>(j_lo) * f.nsi * 4 : static_cast<size_t>(4 * a0d)),
                      sdb, full_bar(s), pl);
+        };
+        JobIter it;
+        it.u = -f.S;
+        while (ok) {
+            int we = 0, rb = 0;
+            const int kind = next_job(it, b, G, NRB, U, f.S, p.lag, we, rb);
+            if (kind == 0) break;
+            if (kind == 1) stage1(record(we), rb);
+            else stage2(we);
         }
         if (!ok) atomicOr(f.err, COLI_DEVERR_TIMEOUT);
         // Drain: the last fill of every ring slot has landed before this thread (and with it the
@@ -683,32 +724,114 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
         }
     };
 
-    // ------------------------------------------------ phase 1: gate/up, h = SiLU(g)*u -----
-    // After a timed-out wait a warp keeps walking the same loops and barriers (skipping later
-    // waits and MMAs), so that no consumer is ever left alone at a named barrier, and releases no
-    // more ring stages: the producer then runs out of its own bounded waits, and its drain makes
-    // sure no copy is still landing in shared memory when the CTA exits.
+    // ------------------------------------------------ jobs: gate/up tiles and down projections
+    // After a timed-out wait a warp keeps walking the same jobs and barriers (skipping later waits
+    // and MMAs), so that no consumer is ever left alone at a named barrier, and releases no more
+    // ring stages: the producer then runs out of its own bounded waits, and its drain makes sure
+    // no copy is still landing in shared memory when the CTA exits.
     const int grp = cw / GW, wg = cw % GW;
     const int cpw1 = rb_h / 64 / GW;                  // chunks of a row per warp
-    int seq = 0, U = 0, my_tiles = 0;
-    long r_lo = 0, r_hi = 0;
-    for (int lam = 0;; ++lam) {
-        if (lam == nsh) {
-            if (p.route_here) route_batch();
-            if (ct == 0) mbar_arrive(route_bar);
-            U = rc.U;
-            const long nr = static_cast<long>(U) * NRB;
-            r_lo = nr * b / G;
-            r_hi = nr * (b + 1) / G;
+    // down projection: warp cw owns the 64-byte chunk cw of every down row of the CTA's block
+    constexpr int CPL = CPC / 32;                     // h elements per lane of a chunk
+    constexpr int RT2 = 3;                            // 16-row tiles of the CTA's output rows
+    const int nch2 = rb_i / 64;
+    const int nact = nch2 < NCW ? nch2 : NCW;         // warps with a chunk
+    const bool active2 = cw < nch2;
+    unsigned char *hb = sm + p.off_hb + static_cast<size_t>(cw) * NCOL * colblk;  // this warp's h slices
+    float acc[RT2][NB][4];                            // down-projection sums (zeroed after the tiles)
+    int my_tiles = 0;
+
+    // Chunk c (CPC elements) of work expert we's h (all of h is written: after the grid barrier):
+    // per token 24-bit fixed point with one scale (three byte slices), laid out as this warp's
+    // MMA B fragments through its h-slice block in shared memory, then stored lane-major for the
+    // down projections of every CTA.  Lane l holds
+    // elements l * CPL + k; two neighbouring lanes fill each 32-bit B word (one shuffle).
+    auto convert_chunk = [&](int we, int c) {
+        float hv[MAXT][CPL];
+#pragma unroll
+        for (int t = 0; t < MAXT; ++t) {
+            const int slot = t < T ? rc.slot[we][t] : -1;
+#pragma unroll
+            for (int k = 0; k < CPL; k += 4) {
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (slot >= 0)
+                    v = __ldcg(reinterpret_cast<const float4 *>(f.h + static_cast<size_t>(slot) * f.I + c * CPC + lane * CPL + k));
+                hv[t][k] = v.x; hv[t][k + 1] = v.y; hv[t][k + 2] = v.z; hv[t][k + 3] = v.w;
+            }
         }
-        if (lam >= nsh && lam - nsh >= r_hi - r_lo) break;
-        int we, rb;
-        if (lam < nsh) { we = 0; rb = sh_lo + lam; }
-        else { const long tau = r_lo + (lam - nsh); we = f.S + static_cast<int>(tau / NRB); rb = static_cast<int>(tau % NRB); }
-        const int s = seq % S;
-        const uint32_t par = (seq / S) & 1;
-        ++seq;
-        if ((lam % NGRP) != grp) continue;
+        const bool odd = lane & 1;
+        const int tg = lane >> 3;
+        float scl[MAXT];
+#pragma unroll
+        for (int t = 0; t < MAXT; ++t) {
+            scl[t] = 0.f;
+            if (t >= T) continue;
+            float m = 0.f;
+#pragma unroll
+            for (int k = 0; k < CPL; ++k) m = fmaxf(m, fabsf(hv[t][k]));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
+            int ex = 0;
+            if (m > 0.f) frexpf(m, &ex);
+            const float up = ldexpf(1.0f, 22 - ex);
+            scl[t] = ldexpf(1.0f, ex - 22);
+            uint32_t by[3][CPL];  // slice bytes
+#pragma unroll
+            for (int k = 0; k < CPL; ++k) {
+                int s0, s1, s2;
+                slices3(__float2int_rn(hv[t][k] * up), s0, s1, s2);
+                by[0][k] = static_cast<uint32_t>(s0) & 0xffu;
+                by[1][k] = static_cast<uint32_t>(s1) & 0xffu;
+                by[2][k] = static_cast<uint32_t>(s2) & 0xffu;
+            }
+#pragma unroll
+            for (int sidx = 0; sidx < 3; ++sidx) {
+                const int col = 3 * t + sidx;
+                unsigned char *blk = hb + col * colblk;
+                if (FMT == 4) {
+                    // elements 4l + {0, 2} -> bytes 2(l&1) + {0, 1} of half 0; 4l + {1, 3} of half 1
+                    const uint32_t h0 = by[sidx][0] | (by[sidx][2] << 8), h1 = by[sidx][1] | (by[sidx][3] << 8);
+                    const uint32_t got = __shfl_xor_sync(FULL, odd ? h0 : h1, 1);
+                    const uint32_t word = odd ? (got | (h1 << 16)) : (h0 | (got << 16));
+                    const int m2 = (lane >> 1) & 3;
+                    *reinterpret_cast<uint32_t *>(blk + b_off<FMT>(col, tg, m2, odd ? 1 : 0, 0)) = word;
+                } else {
+                    // elements 8l + kk + {0, 4} -> bytes 2(l&1) + {0, 1} of field kk's register;
+                    // the even lane stores fields 0, 1 and the odd lane fields 2, 3
+                    const int i4 = (lane >> 1) & 3;
+                    uint32_t hw[4];
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) hw[kk] = by[sidx][kk] | (by[sidx][4 + kk] << 8);
+#pragma unroll
+                    for (int e2 = 0; e2 < 2; ++e2) {
+                        const uint32_t got = __shfl_xor_sync(FULL, odd ? hw[e2] : hw[2 + e2], 1);
+                        const int kk = odd ? 2 + e2 : e2;
+                        const uint32_t word = odd ? (got | (hw[kk] << 16)) : (hw[kk] | (got << 16));
+                        *reinterpret_cast<uint32_t *>(blk + b_off<FMT>(col, tg, 2 * i4 + (kk >> 1), kk & 1, 0)) = word;
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        // the block as it is in shared memory, then the tokens' scales (16 bytes)
+        uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<unsigned char *>(p.dsl) + static_cast<size_t>(we * DEC_CH + c) * DSTR);
+        const int n16 = NCOL * colblk / 16;
+        for (int i = lane; i < n16; i += 32) __stcg(dst + i, reinterpret_cast<const uint4 *>(hb)[i]);
+        if (lane == 0) {
+            float4 sv = make_float4(0.f, 0.f, 0.f, 0.f);
+            sv.x = scl[0];
+            if (MAXT > 1) sv.y = scl[MAXT > 1 ? 1 : 0];
+            if (MAXT > 2) sv.z = scl[MAXT > 2 ? 2 : 0];
+            if (MAXT > 3) sv.w = scl[MAXT > 3 ? 3 : 0];
+            __stcg(reinterpret_cast<float4 *>(dst + n16), sv);
+        }
+        __syncwarp();  // the h-slice block is reused only after every lane read it
+    };
+
+    // A gate/up tile (taken by one group of 8 warps): every warp multiplies its chunks of the 8
+    // gate and 8 up rows with all tokens' activation slices, the group reduces the partial sums,
+    // and its first warp forms and publishes h = SiLU(g)*u of the 8 rows.
+    auto gate_up_tile = [&](int we, int rb, int s, uint32_t par) {
         int D[NB][4];       // per-row scales: exact int32 sums over all of K
         float Dg[NB][4];    // group scales: float sums of (group sum x group scale)
 #pragma unroll
@@ -774,8 +897,8 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
         if (wg == 0) {
             const int pr = lane & 7, t = lane >> 3;  // row pair, token
             const int slot = t < T ? rc.slot[we][t] : -1;
+            double gsum = 0.0, usum = 0.0;
             if (ok && slot >= 0) {
-                double gsum = 0.0, usum = 0.0;
 #pragma unroll
                 for (int sidx = 0; sidx < 3; ++sidx) {
                     const int col = 3 * t + sidx, nb = col >> 3, c8 = col & 7;
@@ -801,6 +924,10 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
                         usum += wsl * us;
                     }
                 }
+            }
+            __syncwarp();
+            named_arrive(BAR_GFREE + grp, GW * 32);  // partials read: the group's next tile may go on
+            if (ok && slot >= 0) {
                 const double xs = static_cast<double>(rc.xscale[t]) / F::MUL;
                 const double gsc = GS ? 1.0 : static_cast<double>(sgs[pr]);
                 const double usc = GS ? 1.0 : static_cast<double>(sus[pr]);
@@ -808,255 +935,188 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
                 const float uq = static_cast<float>(usum * xs * usc);
                 f.h[static_cast<size_t>(slot) * f.I + rb * 8 + pr] = __fmul_rn(__fdiv_rn(gq, __fadd_rn(1.0f, expf(-gq))), uq);
             }
-            __syncwarp();
-            named_arrive(BAR_GFREE + grp, GW * 32);
         }
         // the stage (rows and scales) is released once the epilogue has read the scales
         __syncwarp();
         if (ok && lane == 0) mbar_arrive_cnt(empty_bar(s), NCW / GW);
         ++my_tiles;
-    }
+    };
+
+    // The down projection of work expert we for this warp's chunk (all warps): the warp's chunk
+    // of h as B fragments and scales (loaded one job ahead), and once the stage has landed the
+    // CTA's down rows multiplied with them into the per-row accumulators.
+    // Per-warp ring of fdepth fragment slots (the activation slices' region, free once the tiles
+    // are done): the warp's chunk of a work expert's converted h and its scales.
+    const int fslot = NCOL * colblk + 16, FD = p.fdepth;
+    unsigned char *fring = sm + p.off_x + static_cast<size_t>(cw) * FD * fslot;
+    auto issue_frag = [&](int we, int slot) {  // one commit group per call (empty if none)
+        if (active2) {
+            const unsigned char *g = reinterpret_cast<const unsigned char *>(p.dsl) + static_cast<size_t>(we * DEC_CH + cw) * DSTR;
+            unsigned char *d = fring + slot * fslot;
+            for (int i = lane; i < fslot / 16; i += 32) cp_async16(d + 16 * i, g + 16 * i);
+        }
+        cp_async_commit();
+    };
+    auto down_job = [&](int we, int s, uint32_t par, int slot) {
+        uint32_t bfr[MPC][NB][2];
+        float fcol[NB][2];
+        // this job's group (the FD - 1 later ones may still be in flight)
+        if (FD >= 3) cp_async_wait<2>();
+        else if (FD == 2) cp_async_wait<1>();
+        else cp_async_wait<0>();
+        __syncwarp();
+        if (active2) {
+            const unsigned char *fr = fring + slot * fslot;
+#pragma unroll
+            for (int u = 0; u < MPC / 2; ++u)
+#pragma unroll
+                for (int nb = 0; nb < NB; ++nb) {
+                    const int col = nb * 8 + g8;
+                    const uint4 v = col < NCOL ? load_b2<FMT>(fr + col * colblk, col, tig, u) : make_uint4(0u, 0u, 0u, 0u);
+                    bfr[2 * u][nb][0] = v.x;
+                    bfr[2 * u][nb][1] = v.y;
+                    bfr[2 * u + 1][nb][0] = v.z;
+                    bfr[2 * u + 1][nb][1] = v.w;
+                }
+            const float *scl = reinterpret_cast<const float *>(fr + NCOL * colblk);
+            // column factor: combine weight x chunk scale x slice weight (powers of two but the weight)
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int col = nb * 8 + 2 * tig + i, t = col / 3;
+                    const float base = t < T ? rc.wgt[we][t] * scl[t] / F::MUL : 0.f;
+                    fcol[nb][i] = base * (col % 3 == 0 ? 1.0f : (col % 3 == 1 ? 256.0f : 65536.0f));
+                }
+        }
+        if (ok && active2 && !mbar_wait(full_bar(s), par, bound)) ok = false;
+        ok = __all_sync(FULL, ok);
+        if (ok && active2) {
+            const unsigned char *st = ring + static_cast<size_t>(s) * p.SB;
+            const float *sdp = reinterpret_cast<const float *>(st + p.st_sd) + (j_lo - a0d);
+            const float *sdg = reinterpret_cast<const float *>(st + p.st_sd);  // [nrows][nsi]
+#pragma unroll
+            for (int rt = 0; rt < RT2; ++rt) {
+                const int ra = rt * 16 + g8, rbw = ra + 8;
+                if (rt * 16 < nrows) {
+                    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+                    const uint4 qa = ra < nrows ? *reinterpret_cast<const uint4 *>(st + ra * rb_i + 64 * cw + 16 * tig) : z;
+                    const uint4 qb = rbw < nrows ? *reinterpret_cast<const uint4 *>(st + rbw * rb_i + 64 * cw + 16 * tig) : z;
+                    int D[NB][4], D1[NB][4];
+#pragma unroll
+                    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) { D[nb][i] = 0; D1[nb][i] = 0; }
+#pragma unroll
+                    for (int m = 0; m < MPC; ++m) {
+                        uint32_t a0, a2, a1, a3;
+                        F::unpack(qa, m, a0, a2);
+                        F::unpack(qb, m, a1, a3);
+#pragma unroll
+                        for (int nb = 0; nb < NB; ++nb) mma_chunk(D[nb], D1[nb], a0, a1, a2, a3, bfr[m][nb][0], bfr[m][nb][1]);
+                    }
+                    float sda, sdb, sda1 = 0.f, sdb1 = 0.f;
+                    if (GS) {  // groups 2 cw and 2 cw + 1 of rows ra and rbw
+                        sda = ra < nrows ? sdg[ra * f.nsi + 2 * cw] : 0.f;
+                        sda1 = ra < nrows ? sdg[ra * f.nsi + 2 * cw + 1] : 0.f;
+                        sdb = rbw < nrows ? sdg[rbw * f.nsi + 2 * cw] : 0.f;
+                        sdb1 = rbw < nrows ? sdg[rbw * f.nsi + 2 * cw + 1] : 0.f;
+                    } else {
+                        sda = ra < nrows ? sdp[ra] : 0.f;
+                        sdb = rbw < nrows ? sdp[rbw] : 0.f;
+                    }
+#pragma unroll
+                    for (int nb = 0; nb < NB; ++nb) {
+                        acc[rt][nb][0] = __fmaf_rn(static_cast<float>(D[nb][0]), sda * fcol[nb][0], acc[rt][nb][0]);
+                        acc[rt][nb][1] = __fmaf_rn(static_cast<float>(D[nb][1]), sda * fcol[nb][1], acc[rt][nb][1]);
+                        acc[rt][nb][2] = __fmaf_rn(static_cast<float>(D[nb][2]), sdb * fcol[nb][0], acc[rt][nb][2]);
+                        acc[rt][nb][3] = __fmaf_rn(static_cast<float>(D[nb][3]), sdb * fcol[nb][1], acc[rt][nb][3]);
+                        if (GS) {
+                            acc[rt][nb][0] = __fmaf_rn(static_cast<float>(D1[nb][0]), sda1 * fcol[nb][0], acc[rt][nb][0]);
+                            acc[rt][nb][1] = __fmaf_rn(static_cast<float>(D1[nb][1]), sda1 * fcol[nb][1], acc[rt][nb][1]);
+                            acc[rt][nb][2] = __fmaf_rn(static_cast<float>(D1[nb][2]), sdb1 * fcol[nb][0], acc[rt][nb][2]);
+                            acc[rt][nb][3] = __fmaf_rn(static_cast<float>(D1[nb][3]), sdb1 * fcol[nb][1], acc[rt][nb][3]);
+                        }
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        if (ok && active2 && lane == 0) mbar_arrive_cnt(empty_bar(s), NCW / nact);
+    };
+
+    // Bounded grid barrier k (1, 2): the arrivals count on after the logits' (the counter is
+    // reset at departure).
+    auto grid_barrier = [&](unsigned k) {
+        cons_sync();
+        if (ct == 0) {
+            __threadfence();
+            atomicAdd(p.gbar, 1u);
+            const unsigned target = static_cast<unsigned>(G) * ((p.route_here ? 1u : 0u) + k) + p.gate_extra;
+            const long long t0 = clock64();
+            while (ld_acquire(p.gbar) < target) {
+                if (clock64() - t0 > bound) { atomicOr(f.err, COLI_DEVERR_TIMEOUT); break; }
+            }
+        }
+        cons_sync();
+    };
+
+    // The jobs, in the order next_job gives (the producer walks the same order): the shared
+    // expert's tiles of this CTA, the routing, the routed tiles (alternating between the two
+    // groups), then the down projections (every warp takes each).
+    int seq = 0, lam = 0, kind = 0, we = 0, rb = 0;
+    auto tile = [&](int we1, int rb1) {
+        const int s = seq % S;
+        const uint32_t par = (seq / S) & 1;
+        ++seq;
+        const bool mine = (lam % NGRP) == grp;
+        ++lam;
+        if (mine) gate_up_tile(we1, rb1, s, par);
+    };
+    for (int l = 0; l < nsh; ++l) tile(0, sh_lo + l);
+    if (p.route_here) route_batch();
+    if (ct == 0) mbar_arrive(route_bar);
+    JobIter it;
+    it.u = -f.S;
+    while ((kind = next_job(it, b, G, NRB, rc.U, f.S, p.lag, we, rb)) == 1) tile(we, rb);
     if (my_tiles > 0 && wg != 0) named_sync(BAR_GFREE + grp, GW * 32);  // the last arrival
 
-    // ------------------------------------------------ grid barrier ------------------------
-    cons_sync();
-    if (ct == 0) {
-        __threadfence();
-        atomicAdd(p.gbar, 1u);
-        const unsigned target = static_cast<unsigned>(G) * (p.route_here ? 2u : 1u) + p.gate_extra;
-        const long long t0 = clock64();
-        while (ld_acquire(p.gbar) < target) {
-            if (clock64() - t0 > bound) { atomicOr(f.err, COLI_DEVERR_TIMEOUT); break; }
-        }
-        // the last CTA to leave the barrier zeroes both counters for the next call
-        if (atomicAdd(p.gdep, 1u) == static_cast<unsigned>(G) - 1u) {
-            *p.gbar = 0u;
-            *p.gdep = 0u;
-            __threadfence();
-        }
+    // Down projections: once every CTA's h is written (grid barrier), each h chunk is converted
+    // once (chunk q by CTA q mod G, warp q / G), and once all are (second grid barrier) every CTA
+    // multiplies its block of down rows with them.
+    if (kind == 2) {
+        grid_barrier(1u);
+        const int nq = (f.S + rc.U) * nch2;
+        for (int q = b + G * cw; q < nq; q += G * NCW) convert_chunk(q / nch2, q % nch2);
+        grid_barrier(2u);
     }
-    cons_sync();
-
-    // ------------------------------------------------ phase 2: down + combine -------------
-    // warp cw owns the 64-byte chunk cw of every down row of the CTA's block
-    constexpr int CPL = CPC / 32;                     // h elements per lane of a chunk
-    constexpr int RT2 = 3;                            // 16-row tiles of the CTA's output rows
-    const int nch2 = rb_i / 64;
-    const int nact = nch2 < NCW ? nch2 : NCW;         // warps with a chunk
-    const bool active2 = cw < nch2;
-    const int nwe = f.S + U;
-    // this warp's two h-slice blocks (two experts in flight)
-    unsigned char *hbA = sm + p.off_x + static_cast<size_t>(cw) * (TT <= 2 ? 2 : 1) * NCOL * colblk;
-    unsigned char *hbB = hbA + NCOL * colblk;  // used when two experts are in flight (TT <= 2)
-    float acc[RT2][NB][4];
 #pragma unroll
     for (int rt = 0; rt < RT2; ++rt)
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
             for (int i = 0; i < 4; ++i) acc[rt][nb][i] = 0.f;
-    // This warp's chunk of each slot's h, fetched two experts ahead into two register buffers.
-    auto fetch_h = [&](int we, float (&hv)[MAXT][CPL]) {
-#pragma unroll
-        for (int t = 0; t < MAXT; ++t) {
-            const int slot = t < T ? rc.slot[we][t] : -1;
-#pragma unroll
-            for (int k = 0; k < CPL; k += 4) {
-                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (slot >= 0 && active2)
-                    v = __ldcg(reinterpret_cast<const float4 *>(f.h + static_cast<size_t>(slot) * f.I + cw * CPC + lane * CPL + k));
-                hv[t][k] = v.x; hv[t][k + 1] = v.y; hv[t][k + 2] = v.z; hv[t][k + 3] = v.w;
-            }
+    // The down jobs are the work experts in order (the shared one first); each one's fragments
+    // are fetched FD - 1 jobs ahead (they come from L2 behind the weight stream, over a
+    // microsecond).
+    if (kind == 2) {
+        const int nwe = f.S + rc.U;
+        int s = seq % S;
+        uint32_t par = (seq / S) & 1;
+        for (int j = 0; j + 1 < FD; ++j) {
+            if (j < nwe) issue_frag(j, j); else cp_async_commit();
         }
-    };
-    // h -> 24-bit fixed point per chunk (three byte slices) in this warp's B block, and the
-    // column factors (combine weight x chunk scale x slice weight).  Lane l holds elements
-    // l * CPL + k; two neighbouring lanes fill each 32-bit B word, exchanged by one shuffle.
-    auto convert_h = [&](int we, const float (&hv)[MAXT][CPL], float (&fcol)[NB][2], unsigned char *hb) {
-#pragma unroll
-        for (int nb = 0; nb < NB; ++nb) fcol[nb][0] = fcol[nb][1] = 0.f;
-        const bool odd = lane & 1;
-        const int tg = lane >> 3;
-#pragma unroll
-        for (int t = 0; t < MAXT; ++t) {
-            if (t >= T) continue;
-            float m = 0.f;
-#pragma unroll
-            for (int k = 0; k < CPL; ++k) m = fmaxf(m, fabsf(hv[t][k]));
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
-            int ex = 0;
-            if (m > 0.f) frexpf(m, &ex);
-            const float up = ldexpf(1.0f, 22 - ex);
-            const float base = rc.wgt[we][t] * ldexpf(1.0f, ex - 22) / F::MUL;
-#pragma unroll
-            for (int nb = 0; nb < NB; ++nb)
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const int col = nb * 8 + 2 * tig + i;
-                    if (col / 3 == t) fcol[nb][i] = base * (col % 3 == 0 ? 1.0f : (col % 3 == 1 ? 256.0f : 65536.0f));
-                }
-            uint32_t by[3][CPL];  // slice bytes
-#pragma unroll
-            for (int k = 0; k < CPL; ++k) {
-                int s0, s1, s2;
-                slices3(__float2int_rn(hv[t][k] * up), s0, s1, s2);
-                by[0][k] = static_cast<uint32_t>(s0) & 0xffu;
-                by[1][k] = static_cast<uint32_t>(s1) & 0xffu;
-                by[2][k] = static_cast<uint32_t>(s2) & 0xffu;
-            }
-#pragma unroll
-            for (int sidx = 0; sidx < 3; ++sidx) {
-                const int col = 3 * t + sidx;
-                unsigned char *blk = hb + col * colblk;
-                if (FMT == 4) {
-                    // elements 4l + {0, 2} -> bytes 2(l&1) + {0, 1} of half 0; 4l + {1, 3} of half 1
-                    const uint32_t h0 = by[sidx][0] | (by[sidx][2] << 8), h1 = by[sidx][1] | (by[sidx][3] << 8);
-                    const uint32_t got = __shfl_xor_sync(FULL, odd ? h0 : h1, 1);
-                    const uint32_t word = odd ? (got | (h1 << 16)) : (h0 | (got << 16));
-                    const int m2 = (lane >> 1) & 3;
-                    *reinterpret_cast<uint32_t *>(blk + b_off<FMT>(col, tg, m2, odd ? 1 : 0, 0)) = word;
-                } else {
-                    // elements 8l + kk + {0, 4} -> bytes 2(l&1) + {0, 1} of field kk's register;
-                    // the even lane stores fields 0, 1 and the odd lane fields 2, 3
-                    const int i4 = (lane >> 1) & 3;
-                    uint32_t hw[4];
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk) hw[kk] = by[sidx][kk] | (by[sidx][4 + kk] << 8);
-#pragma unroll
-                    for (int e2 = 0; e2 < 2; ++e2) {
-                        const uint32_t got = __shfl_xor_sync(FULL, odd ? hw[e2] : hw[2 + e2], 1);
-                        const int kk = odd ? 2 + e2 : e2;
-                        const uint32_t word = odd ? (got | (hw[kk] << 16)) : (hw[kk] | (got << 16));
-                        *reinterpret_cast<uint32_t *>(blk + b_off<FMT>(col, tg, 2 * i4 + (kk >> 1), kk & 1, 0)) = word;
-                    }
-                }
-            }
-        }
-        __syncwarp();
-    };
-    // The down projection of work experts we and we + 1 (when `two`) for this warp's chunk, once
-    // their stages have landed.  The two experts' instruction streams are independent, so their
-    // shared-memory loads and MMAs overlap; without a second expert the second stream repeats
-    // the first with zero column factors.
-    constexpr int NE = TT <= 2 ? 2 : 1;  // experts in flight (register budget)
-    auto down_pair = [&](int we, bool two, const float (&fA)[NB][2], const float (&fB)[NB][2]) {
-        const int sA = (seq + we) % S, sB = (seq + we + 1) % S;
-        const uint32_t pA = ((seq + we) / S) & 1, pB = ((seq + we + 1) / S) & 1;
-        if (ok && active2 && !mbar_wait(full_bar(sA), pA, bound)) ok = false;
-        if (ok && active2 && two && !mbar_wait(full_bar(sB), pB, bound)) ok = false;
-        ok = __all_sync(FULL, ok);
-        if (ok && active2) {
-            const unsigned char *st[2] = {ring + static_cast<size_t>(sA) * p.SB,
-                                          ring + static_cast<size_t>(two ? sB : sA) * p.SB};
-            const unsigned char *hbs[2] = {hbA, two ? hbB : hbA};
-            uint32_t bfr[NE][MPC][NB][2];
-#pragma unroll
-            for (int e = 0; e < NE; ++e)
-#pragma unroll
-                for (int u = 0; u < MPC / 2; ++u)
-#pragma unroll
-                    for (int nb = 0; nb < NB; ++nb) {
-                        const int col = nb * 8 + g8;
-                        const uint4 v = col < NCOL ? load_b2<FMT>(hbs[e] + col * colblk, col, tig, u) : make_uint4(0u, 0u, 0u, 0u);
-                        bfr[e][2 * u][nb][0] = v.x;
-                        bfr[e][2 * u][nb][1] = v.y;
-                        bfr[e][2 * u + 1][nb][0] = v.z;
-                        bfr[e][2 * u + 1][nb][1] = v.w;
-                    }
-#pragma unroll
-            for (int rt = 0; rt < RT2; ++rt) {
-                const int ra = rt * 16 + g8, rbw = ra + 8;
-                if (rt * 16 < nrows) {
-#pragma unroll
-                    for (int e = 0; e < NE; ++e) {
-                        const float (&fc)[NB][2] = e == 0 ? fA : fB;
-                        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-                        const uint4 qa = ra < nrows ? *reinterpret_cast<const uint4 *>(st[e] + ra * rb_i + 64 * cw + 16 * tig) : z;
-                        const uint4 qb = rbw < nrows ? *reinterpret_cast<const uint4 *>(st[e] + rbw * rb_i + 64 * cw + 16 * tig) : z;
-                        int D[NB][4], D1[NB][4];
-#pragma unroll
-                        for (int nb = 0; nb < NB; ++nb)
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) { D[nb][i] = 0; D1[nb][i] = 0; }
-#pragma unroll
-                        for (int m = 0; m < MPC; ++m) {
-                            uint32_t a0, a2, a1, a3;
-                            F::unpack(qa, m, a0, a2);
-                            F::unpack(qb, m, a1, a3);
-#pragma unroll
-                            for (int nb = 0; nb < NB; ++nb) mma_chunk(D[nb], D1[nb], a0, a1, a2, a3, bfr[e][m][nb][0], bfr[e][m][nb][1]);
-                        }
-                        const float *sdp = reinterpret_cast<const float *>(st[e] + p.st_sd) + (j_lo - a0d);
-                        const float *sdg = reinterpret_cast<const float *>(st[e] + p.st_sd);  // [nrows][nsi]
-                        float sda, sdb, sda1 = 0.f, sdb1 = 0.f;
-                        if (GS) {  // groups 2 cw and 2 cw + 1 of rows ra and rbw
-                            sda = ra < nrows ? sdg[ra * f.nsi + 2 * cw] : 0.f;
-                            sda1 = ra < nrows ? sdg[ra * f.nsi + 2 * cw + 1] : 0.f;
-                            sdb = rbw < nrows ? sdg[rbw * f.nsi + 2 * cw] : 0.f;
-                            sdb1 = rbw < nrows ? sdg[rbw * f.nsi + 2 * cw + 1] : 0.f;
-                        } else {
-                            sda = ra < nrows ? sdp[ra] : 0.f;
-                            sdb = rbw < nrows ? sdp[rbw] : 0.f;
-                        }
-#pragma unroll
-                        for (int nb = 0; nb < NB; ++nb) {
-                            acc[rt][nb][0] = __fmaf_rn(static_cast<float>(D[nb][0]), sda * fc[nb][0], acc[rt][nb][0]);
-                            acc[rt][nb][1] = __fmaf_rn(static_cast<float>(D[nb][1]), sda * fc[nb][1], acc[rt][nb][1]);
-                            acc[rt][nb][2] = __fmaf_rn(static_cast<float>(D[nb][2]), sdb * fc[nb][0], acc[rt][nb][2]);
-                            acc[rt][nb][3] = __fmaf_rn(static_cast<float>(D[nb][3]), sdb * fc[nb][1], acc[rt][nb][3]);
-                            if (GS) {
-                                acc[rt][nb][0] = __fmaf_rn(static_cast<float>(D1[nb][0]), sda1 * fc[nb][0], acc[rt][nb][0]);
-                                acc[rt][nb][1] = __fmaf_rn(static_cast<float>(D1[nb][1]), sda1 * fc[nb][1], acc[rt][nb][1]);
-                                acc[rt][nb][2] = __fmaf_rn(static_cast<float>(D1[nb][2]), sdb1 * fc[nb][0], acc[rt][nb][2]);
-                                acc[rt][nb][3] = __fmaf_rn(static_cast<float>(D1[nb][3]), sdb1 * fc[nb][1], acc[rt][nb][3]);
-                            }
-                        }
-                    }
-                }
-            }
-        }
-        __syncwarp();
-        if (ok && active2 && lane == 0) {
-            mbar_arrive_cnt(empty_bar(sA), NCW / nact);
-            if (two) mbar_arrive_cnt(empty_bar(sB), NCW / nact);
-        }
-        __syncwarp();  // the B blocks are rewritten for the next pair only after every lane read them
-    };
-    float hvA[MAXT][CPL];
-    float fZ[NB][2];
-#pragma unroll
-    for (int nb = 0; nb < NB; ++nb) fZ[nb][0] = fZ[nb][1] = 0.f;
-    if (TT <= 2) {  // two experts at a time; h fetched one pair ahead
-        float hvB[MAXT][CPL];
-        if (nwe > 0) fetch_h(0, hvA);
-        if (nwe > 1) fetch_h(1, hvB);
-        for (int we = 0; we < nwe; we += 2) {
-            const bool two = we + 1 < nwe;
-            float fA[NB][2], fB[NB][2];
-            if (active2) {
-                convert_h(we, hvA, fA, hbA);
-                if (two) convert_h(we + 1, hvB, fB, hbB);
-            }
-            if (!two) {
-#pragma unroll
-                for (int nb = 0; nb < NB; ++nb) fB[nb][0] = fB[nb][1] = 0.f;
-            }
-            if (we + 2 < nwe) fetch_h(we + 2, hvA);
-            if (we + 3 < nwe) fetch_h(we + 3, hvB);
-            down_pair(we, two, fA, fB);
-        }
-    } else {        // one expert at a time (registers), h one expert ahead
-        if (nwe > 0) fetch_h(0, hvA);
-        for (int we = 0; we < nwe; ++we) {
-            float fA[NB][2];
-            if (active2) convert_h(we, hvA, fA, hbA);
-            if (we + 1 < nwe) fetch_h(we + 1, hvA);
-            down_pair(we, false, fA, fZ);
+        for (int we2 = 0; we2 < nwe; ++we2) {
+            const int nx = we2 + FD - 1;
+            if (nx < nwe) issue_frag(nx, nx % FD); else cp_async_commit();
+            down_job(we2, s, par, we2 % FD);
+            if (++s == S) { s = 0; par ^= 1u; }
         }
     }
+    cp_async_wait<0>();
+
     if (!ok) atomicOr(f.err, COLI_DEVERR_TIMEOUT);
-    // cross-warp reduction (the h slices are no longer needed: the region is reused)
+    // cross-warp reduction (every job is done: the activation slices' region is reused)
     cons_sync();
     float *red2 = reinterpret_cast<float *>(sm + p.off_x);  // [warp][rt][nb][lane][4]
     if (active2) {
@@ -1082,6 +1142,16 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
         }
         f.out[static_cast<size_t>(t) * f.H + j_lo + r] = v;
     }
+    // Departure: every warp of this CTA is past its last wait on the counter; the last CTA to
+    // leave zeroes it for the next call on this workspace.
+    if (ct == 0) {
+        __threadfence();
+        if (atomicAdd(p.gdep, 1u) == static_cast<unsigned>(G) - 1u) {
+            *p.gbar = 0u;
+            *p.gdep = 0u;
+            __threadfence();
+        }
+    }
 }
 
 template <int FMT, int TT, int GS>
@@ -1089,8 +1159,9 @@ cudaError_t launch_k(const DecodeParams &p, size_t smem, cudaStream_t st) {
     auto kern = ffn_decode_kernel<FMT, TT, GS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    // cooperative: the grid barriers need every CTA resident at once; the launch waits for the
-    // whole grid to fit (or fails) instead of leaving CTAs spinning for SMs held elsewhere
+    // cooperative: the CTAs wait on one another's logits and h tiles, so every CTA must be
+    // resident at once; the launch waits for the whole grid to fit (or fails) instead of leaving
+    // CTAs spinning for SMs held elsewhere
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.grid);
     cfg.blockDim = dim3(NT);
@@ -1163,34 +1234,45 @@ bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan) {
     pl.SB = ((sb1 > sb2 ? sb1 : sb2) + 127) / 128 * 128;
     size_t o = 1024;                                  // mbarriers (up to 60 stages)
     pl.off_route = o; o += (sizeof(RouteCache) + 127) / 128 * 128;
-    pl.off_rtok = o; o += (static_cast<size_t>(T) * sizeof(RouteToken) + 127) / 128 * 128;
-    pl.off_gate = o; o += NCW * 2 * MAXTOK * 8 + NCW * MAXTOK * 4;
-    o = (o + 127) / 128 * 128;
     pl.off_red1 = o; o += static_cast<size_t>(NGRP) * GW * NB * 32 * 16;
     o = (o + 127) / 128 * 128;
-    // activation slices (phase 1) | per-warp h slices, then the final reduction (phase 2)
+    // activation slices (gate/up tiles), then the down jobs' fragment rings, then the final
+    // reduction
     const size_t xbytes = static_cast<size_t>(c.hidden / cpc) * 3 * T * colblk;
-    // per warp one block of h slices per expert in flight: two for up to two tokens, else one
-    const size_t hbytes = static_cast<size_t>(NCW) * (T <= 2 ? 2 : 1) * 3 * T * colblk;
     const size_t rbytes = static_cast<size_t>(NCW) * 3 * NB * 32 * 16;
-    size_t abytes = xbytes > hbytes ? xbytes : hbytes;
-    abytes = abytes > rbytes ? abytes : rbytes;
+    // fragment rings: as deep (3, 2, 1) as the region allows (up to 1 KB more)
+    size_t abytes = xbytes > rbytes ? xbytes : rbytes;
+    const size_t fper = static_cast<size_t>(NCW) * (3 * T * colblk + 16);
+    pl.fdepth = 3;
+    while (pl.fdepth > 1 && pl.fdepth * fper > abytes + 1024) --pl.fdepth;
+    abytes = abytes > pl.fdepth * fper ? abytes : pl.fdepth * fper;
     pl.off_x = o; o += (abytes + 127) / 128 * 128;
+    // per-warp h slices (down projections, only after the batch is routed), aliased with the
+    // per-token routing scratch and the gate partials (only until it is routed)
+    const size_t hbytes = static_cast<size_t>(NCW) * 3 * T * colblk;
+    const size_t tbytes = (static_cast<size_t>(T) * sizeof(RouteToken) + 127) / 128 * 128;
+    const size_t gbytes = NCW * 2 * MAXTOK * 8 + NCW * MAXTOK * 4;
+    pl.off_hb = o;
+    pl.off_rtok = o;
+    pl.off_gate = o + tbytes;
+    o += ((hbytes > tbytes + gbytes ? hbytes : tbytes + gbytes) + 127) / 128 * 128;
     o = (o + 1023) / 1024 * 1024;
     pl.off_ring = o;
     const size_t budget = device_smem_optin() - 1024;
     if (o + 2 * static_cast<size_t>(pl.SB) > budget) return false;
     pl.S = static_cast<int>((budget - o) / pl.SB);
     if (pl.S > 60) pl.S = 60;
+    // The down projections follow all the CTA's tiles (they need every CTA's h, converted once).
+    pl.lag = 1 << 20;
     pl.smem = o + static_cast<size_t>(pl.S) * pl.SB;
     *plan = pl;
     return true;
 }
 
 static void fill_plan(DecodeParams &p, const DecodePlan &pl) {
-    p.grid = pl.grid; p.S = pl.S; p.SB = pl.SB; p.st_sd = pl.st_sd;
+    p.grid = pl.grid; p.S = pl.S; p.SB = pl.SB; p.st_sd = pl.st_sd; p.lag = pl.lag; p.fdepth = pl.fdepth;
     p.off_route = pl.off_route; p.off_rtok = pl.off_rtok; p.off_gate = pl.off_gate;
-    p.off_red1 = pl.off_red1; p.off_x = pl.off_x; p.off_ring = pl.off_ring;
+    p.off_red1 = pl.off_red1; p.off_x = pl.off_x; p.off_hb = pl.off_hb; p.off_ring = pl.off_ring;
 }
 
 cudaError_t launch_ffn_decode(DecodeParams p, const DecodePlan &pl, cudaStream_t st) {

@@ -33,16 +33,24 @@ struct FfnParams {
     int *err;                          // device error word
 };
 
-// Workspace header (first 256 bytes): error word, then counters of the fused decode path.
-// All must be zero before the first call on a workspace (coli_moe_clear_error zeroes them);
-// the kernels leave them zero after every complete call.
+// Workspace header (first 256 bytes): error word, then counters of the fused decode path (the
+// arrival count of the logits and the grid barriers, the departure count).  All must be zero
+// before the first call on a workspace (coli_moe_clear_error zeroes them); the kernels leave
+// them zero after every complete call.
 constexpr int WS_ERR = 0, WS_GBAR = 64, WS_GDEP = 96;
 constexpr int WS_HEADER = 256;
+// Fused decode path: h of every (work expert, chunk of the down rows' K) converted once, as the
+// chunk's MMA B block (one column per token and slice, at most 12 columns of at most 256
+// bytes) followed by the tokens' 4 scales: [33 work experts][16 chunks] of 12 * 256 + 16 bytes.
+constexpr int DEC_WE = 33, DEC_CH = 16;
+constexpr size_t WS_DSL_BYTES = static_cast<size_t>(DEC_WE) * DEC_CH * (12 * 256 + 16);
 
 // Shared-memory plan of the fused decode kernel (decode.cu).
 struct DecodePlan {
     int grid, S, SB, st_sd;                           // ring: S stages of SB bytes
-    size_t off_route, off_rtok, off_gate, off_red1, off_x, off_ring, smem;
+    size_t off_route, off_rtok, off_gate, off_red1, off_x, off_hb, off_ring, smem;
+    int lag;                                          // down-projection lag (experts)
+    int fdepth;                                       // fragment ring depth per warp (1..3)
 };
 
 // Parameters of the fused decode kernel.
@@ -57,12 +65,13 @@ struct DecodeParams {
     double rsf;
     int G, TG;
     unsigned *gbar, *gdep;
+    uint4 *dsl;             // h chunks converted once (WS_DSL_BYTES)
     int route_here;         // 1: the kernel routes from its own logits; 0: routing arrays are inputs
     long long wait_cycles;  // bound of every device-side wait (0: the default, ~2 s)
-    unsigned gate_extra;    // added to the grid-barrier targets (nonzero only to test the bound)
+    unsigned gate_extra;    // added to the logits-arrival target (nonzero only to test the bound)
     // plan (copied from DecodePlan)
-    int grid, S, SB, st_sd;
-    size_t off_route, off_rtok, off_gate, off_red1, off_x, off_ring;
+    int grid, S, SB, st_sd, lag, fdepth;
+    size_t off_route, off_rtok, off_gate, off_red1, off_x, off_hb, off_ring;
 };
 
 bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan);
@@ -101,6 +110,7 @@ struct WsLayout {
     size_t perm;     // [T*K] i32
     size_t unique;   // [E] i32
     size_t nuniq;    // [1] i32
+    size_t dsl;      // fused decode path: h chunks converted once (WS_DSL_BYTES)
     size_t h;        // [(T*K+T*S)][I] f32 intermediate
     // tensor-core path only (zero size otherwise)
     size_t xq, hq, sx, sh, tok_of, w_of, chunks, n_chunks;
