@@ -51,6 +51,9 @@ constexpr int NT = NC + 32;          // + producer warp
 constexpr int GW = 8;                // warps of a phase-1 group
 constexpr int NGRP = NCW / GW;       // phase-1 groups
 constexpr int MAXTOK = 4;            // tokens of the fused path
+#ifndef DOWN_PIECES
+#define DOWN_PIECES 4
+#endif
 constexpr int MAXWE = 33;            // work experts: the shared one + up to 32 unique routed
 // named barriers: 0 __syncthreads, 1 all consumers, 2.. group full, 4.. group reduction free
 constexpr int BAR_CONS = 1, BAR_GFULL = 2, BAR_GFREE = 4;
@@ -71,6 +74,10 @@ __device__ __forceinline__ void mbar_arrive_cnt(uint32_t a, uint32_t count) {
 }
 __device__ __forceinline__ void mbar_expect_tx(uint32_t a, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(a), "r"(bytes) : "memory");
+}
+// more bytes expected in the current phase, without an arrival (the arrival comes later)
+__device__ __forceinline__ void mbar_add_tx(uint32_t a, uint32_t bytes) {
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(a), "r"(bytes) : "memory");
 }
 // try_wait with a suspend-time hint (ns): a waiting warp sleeps instead of spinning.
 __device__ __forceinline__ bool mbar_try(uint32_t a, uint32_t parity) {
@@ -93,13 +100,6 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
                  ::"r"(dst), "l"(src), "r"(bytes), "r"(mbar), "l"(policy) : "memory");
 }
-// 16-byte asynchronous copy global -> shared (through L2), completed per thread by commit groups
-__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 __device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
@@ -116,6 +116,11 @@ __device__ __forceinline__ uint64_t evict_last_policy() {
 __device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 __device__ __forceinline__ void named_arrive(int id, int n) { asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 __device__ __forceinline__ void cons_sync() { named_sync(BAR_CONS, NC); }
+// arrival on a grid counter that publishes every write made before it (by this thread, and by
+// the CTA's threads that met it at a barrier just before)
+__device__ __forceinline__ void red_release_add(unsigned *p, unsigned v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
 __device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
     unsigned v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -353,7 +358,6 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
     constexpr int MAXT = TT;                          // tokens of this instantiation (T <= TT)
     constexpr int NB = (3 * TT + 7) / 8;              // 8-column MMA blocks (3 slices per token)
     constexpr int EG = FMT == 4 ? 8 : 16;             // activations converted together (whole B words)
-    constexpr int DSTR = 3 * MAXTOK * 32 * MPC + 16;  // bytes per (work expert, chunk) of converted h
     extern __shared__ __align__(1024) unsigned char sm[];
     const FfnParams &f = p.f;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -383,6 +387,11 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
     const int sh_hi = f.S ? static_cast<int>(static_cast<long>(NRB) * (b + 1) / G) : 0;
     const int nsh = sh_hi - sh_lo;                     // shared-expert tiles of this CTA
     const int sc1 = GS ? 8 * f.nsh * 4 : 32;           // bytes of one matrix's scales in a tile stage
+    // converted h: per (work expert, chunk of K) the chunk's B block (3 T columns of 32 MPC bytes)
+    // and the tokens' 4 scales; a down job's fragments are its expert's nch chunks, contiguous
+    const int nch = rb_i / 64;
+    const int fch = 3 * T * 32 * MPC + 16;
+    unsigned char *frag = sm + p.off_frag;             // S slots of fslot bytes, one per ring stage
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S; ++s) {
@@ -430,19 +439,56 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
         // a down-projection stage: the CTA's block of one work expert's down rows and their scales
         const int a1 = (j_hi + 3) & ~3;
         const uint32_t sdb = GS ? static_cast<uint32_t>(nrows) * f.nsi * 4 : 4u * (a1 - a0d);
+        // A down stage carries the CTA's block of one work expert's down rows and their scales,
+        // and in a second part (its fragment slot) the expert's converted h.  Stages issued before
+        // the conversion is published (the second grid barrier) expect the rows' bytes only;
+        // their fragments and the arrival follow once this thread has seen that barrier.
+        const uint32_t fbytes = static_cast<uint32_t>(nch * fch);
+        auto frag_copy = [&](int we, int s) {
+            bulk_g2s(smem_u32(frag + static_cast<size_t>(s) * p.fslot),
+                     reinterpret_cast<const unsigned char *>(p.dsl) + static_cast<size_t>(we) * DEC_CH * fch, fbytes, full_bar(s), keep);
+        };
+        bool published = false;
+        int seq0 = -1, npend = 0;
+        auto publish = [&]() {  // wait for the second grid barrier, then complete the pending stages
+            const unsigned target = static_cast<unsigned>(G) * ((p.route_here ? 1u : 0u) + 2u) + p.gate_extra;
+            const long long t0 = clock64();
+            while (ld_acquire(p.gbar) < target) {
+                if (clock64() - t0 > bound) { ok = false; break; }
+            }
+            for (int j = 0; j < npend; ++j) {
+                const int s = (seq0 + j) % S;
+                if (ok) {
+                    mbar_expect_tx(full_bar(s), fbytes);
+                    frag_copy(j, s);
+                } else {
+                    mbar_arrive(full_bar(s));
+                }
+            }
+            npend = 0;
+            published = true;
+        };
         auto stage2 = [&](int we) {
             const uint8_t *rec = record(we);
+            if (seq0 < 0) seq0 = seq;
+            if (!published && seq - seq0 == S) publish();  // the ring is full of waiting stages
+            if (!ok) return;
             const int s = seq % S;
             const uint32_t par = (seq / S) & 1;
             if (!mbar_wait(empty_bar(s), par ^ 1, bound)) { ok = false; return; }
             ++seq;
-            if (rec == nullptr) { mbar_arrive(full_bar(s)); return; }
+            const uint32_t rows = rec ? static_cast<uint32_t>(nrows) * rb_i + sdb : 0u;
+            if (published) mbar_expect_tx(full_bar(s), rows + fbytes);
+            else mbar_add_tx(full_bar(s), rows);
             const uint32_t dst = smem_u32(ring + static_cast<size_t>(s) * p.SB);
-            mbar_expect_tx(full_bar(s), static_cast<uint32_t>(nrows) * rb_i + sdb);
             const uint64_t pl = we < f.S ? keep : pol;
-            bulk_g2s(dst, rec + f.off_wd + static_cast<size_t>(j_lo) * rb_i, static_cast<uint32_t>(nrows) * rb_i, full_bar(s), pl);
-            bulk_g2s(dst + p.st_sd, rec + f.off_sd + (GS ? static_cast<size_t>(j_lo) * f.nsi * 4 : static_cast<size_t>(4 * a0d)),
-                     sdb, full_bar(s), pl);
+            if (rec) {
+                bulk_g2s(dst, rec + f.off_wd + static_cast<size_t>(j_lo) * rb_i, static_cast<uint32_t>(nrows) * rb_i, full_bar(s), pl);
+                bulk_g2s(dst + p.st_sd, rec + f.off_sd + (GS ? static_cast<size_t>(j_lo) * f.nsi * 4 : static_cast<size_t>(4 * a0d)),
+                         sdb, full_bar(s), pl);
+            }
+            if (published) frag_copy(we, s);
+            else ++npend;
         };
         JobIter it;
         it.u = -f.S;
@@ -453,7 +499,11 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
             if (kind == 1) stage1(record(we), rb);
             else stage2(we);
         }
-        if (!ok) atomicOr(f.err, COLI_DEVERR_TIMEOUT);
+        if (ok && !published && npend > 0) publish();
+        if (!ok) {  // complete the stages still waiting for an arrival (their copies drain below)
+            for (int j = 0; j < npend; ++j) mbar_arrive(full_bar((seq0 + j) % S));
+            atomicOr(f.err, COLI_DEVERR_TIMEOUT);
+        }
         // Drain: the last fill of every ring slot has landed before this thread (and with it the
         // CTA) exits, also when a wait ran out and the consumers gave up on the stage.
         for (int s = 0; s < S && s < seq; ++s) {
@@ -814,7 +864,7 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
         }
         __syncwarp();
         // the block as it is in shared memory, then the tokens' scales (16 bytes)
-        uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<unsigned char *>(p.dsl) + static_cast<size_t>(we * DEC_CH + c) * DSTR);
+        uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<unsigned char *>(p.dsl) + static_cast<size_t>(we * DEC_CH + c) * fch);
         const int n16 = NCOL * colblk / 16;
         for (int i = lane; i < n16; i += 32) __stcg(dst + i, reinterpret_cast<const uint4 *>(hb)[i]);
         if (lane == 0) {
@@ -832,12 +882,12 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
     // gate and 8 up rows with all tokens' activation slices, the group reduces the partial sums,
     // and its first warp forms and publishes h = SiLU(g)*u of the 8 rows.
     auto gate_up_tile = [&](int we, int rb, int s, uint32_t par) {
-        int D[NB][4];       // per-row scales: exact int32 sums over all of K
-        float Dg[NB][4];    // group scales: float sums of (group sum x group scale)
+        int D[NB][4], D2[NB][4];  // per-row scales: exact int32 sums over all of K (two chains)
+        float Dg[NB][4];          // group scales: float sums of (group sum x group scale)
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) { D[nb][i] = 0; Dg[nb][i] = 0.f; }
+            for (int i = 0; i < 4; ++i) { D[nb][i] = 0; D2[nb][i] = 0; Dg[nb][i] = 0.f; }
         if (ok && !mbar_wait(full_bar(s), par, bound)) ok = false;
         ok = __all_sync(FULL, ok);  // warp-uniform: the MMAs below need every lane
         const unsigned char *st = ring + static_cast<size_t>(s) * p.SB;
@@ -868,8 +918,10 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
                         F::unpack(qa, 2 * u + mm, a0, a2);
                         F::unpack(qb, 2 * u + mm, a1, a3);
 #pragma unroll
-                        for (int nb = 0; nb < NB; ++nb)
-                            mma_chunk(GS ? Dc[nb] : D[nb], Dc1[nb], a0, a1, a2, a3, mm ? bv[nb].z : bv[nb].x, mm ? bv[nb].w : bv[nb].y);
+                        for (int nb = 0; nb < NB; ++nb) {
+                            if (GS) mma_chunk(Dc[nb], Dc1[nb], a0, a1, a2, a3, mm ? bv[nb].z : bv[nb].x, mm ? bv[nb].w : bv[nb].y);
+                            else mma_s8((NB == 1 && mm) ? D2[nb] : D[nb], a0, a1, a2, a3, mm ? bv[nb].z : bv[nb].x, mm ? bv[nb].w : bv[nb].y);
+                        }
                     }
                 }
                 if (GS) {  // groups 2c and 2c + 1 of rows g8 (gate) and g8 + 8 (up)
@@ -887,6 +939,10 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
             }
         }
         // group reduction of the partial sums, then one warp forms h
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) D[nb][i] += D2[nb][i];
         if (my_tiles > 0 && wg != 0) named_sync(BAR_GFREE + grp, GW * 32);
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb)
@@ -945,28 +1001,10 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
     // The down projection of work expert we for this warp's chunk (all warps): the warp's chunk
     // of h as B fragments and scales (loaded one job ahead), and once the stage has landed the
     // CTA's down rows multiplied with them into the per-row accumulators.
-    // Per-warp ring of fdepth fragment slots (the activation slices' region, free once the tiles
-    // are done): the warp's chunk of a work expert's converted h and its scales.
-    const int fslot = NCOL * colblk + 16, FD = p.fdepth;
-    unsigned char *fring = sm + p.off_x + static_cast<size_t>(cw) * FD * fslot;
-    auto issue_frag = [&](int we, int slot) {  // one commit group per call (empty if none)
+    // B fragments and column factors of job we from the fragment slot of its (landed) stage s
+    auto prep_frag = [&](int we, int s, uint32_t (&bfr)[MPC][NB][2], float (&fcol)[NB][2]) {
         if (active2) {
-            const unsigned char *g = reinterpret_cast<const unsigned char *>(p.dsl) + static_cast<size_t>(we * DEC_CH + cw) * DSTR;
-            unsigned char *d = fring + slot * fslot;
-            for (int i = lane; i < fslot / 16; i += 32) cp_async16(d + 16 * i, g + 16 * i);
-        }
-        cp_async_commit();
-    };
-    auto down_job = [&](int we, int s, uint32_t par, int slot) {
-        uint32_t bfr[MPC][NB][2];
-        float fcol[NB][2];
-        // this job's group (the FD - 1 later ones may still be in flight)
-        if (FD >= 3) cp_async_wait<2>();
-        else if (FD == 2) cp_async_wait<1>();
-        else cp_async_wait<0>();
-        __syncwarp();
-        if (active2) {
-            const unsigned char *fr = fring + slot * fslot;
+            const unsigned char *fr = frag + static_cast<size_t>(s) * p.fslot + cw * fch;
 #pragma unroll
             for (int u = 0; u < MPC / 2; ++u)
 #pragma unroll
@@ -989,54 +1027,77 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
                     fcol[nb][i] = base * (col % 3 == 0 ? 1.0f : (col % 3 == 1 ? 256.0f : 65536.0f));
                 }
         }
+    };
+    // The down projection of job we once its stage (rows, scales, fragments) has landed.
+    auto down_job = [&](int we, int s, uint32_t par) {
         if (ok && active2 && !mbar_wait(full_bar(s), par, bound)) ok = false;
         ok = __all_sync(FULL, ok);
         if (ok && active2) {
+            uint32_t bfr[MPC][NB][2];
+            float fcol[NB][2];
+            prep_frag(we, s, bfr, fcol);
             const unsigned char *st = ring + static_cast<size_t>(s) * p.SB;
             const float *sdp = reinterpret_cast<const float *>(st + p.st_sd) + (j_lo - a0d);
             const float *sdg = reinterpret_cast<const float *>(st + p.st_sd);  // [nrows][nsi]
+            // all row tiles' codes first, then independent MMA chains: per row tile the even and
+            // odd k-steps (per-row scales) or the two groups (group scales)
+            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+            uint4 qa[RT2], qb[RT2];
 #pragma unroll
             for (int rt = 0; rt < RT2; ++rt) {
                 const int ra = rt * 16 + g8, rbw = ra + 8;
-                if (rt * 16 < nrows) {
-                    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-                    const uint4 qa = ra < nrows ? *reinterpret_cast<const uint4 *>(st + ra * rb_i + 64 * cw + 16 * tig) : z;
-                    const uint4 qb = rbw < nrows ? *reinterpret_cast<const uint4 *>(st + rbw * rb_i + 64 * cw + 16 * tig) : z;
-                    int D[NB][4], D1[NB][4];
+                qa[rt] = ra < nrows ? *reinterpret_cast<const uint4 *>(st + ra * rb_i + 64 * cw + 16 * tig) : z;
+                qb[rt] = rbw < nrows ? *reinterpret_cast<const uint4 *>(st + rbw * rb_i + 64 * cw + 16 * tig) : z;
+            }
+            int D[RT2][NB][4], D1[RT2][NB][4];
 #pragma unroll
-                    for (int nb = 0; nb < NB; ++nb)
+            for (int rt = 0; rt < RT2; ++rt)
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) { D[nb][i] = 0; D1[nb][i] = 0; }
+                for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
-                    for (int m = 0; m < MPC; ++m) {
-                        uint32_t a0, a2, a1, a3;
-                        F::unpack(qa, m, a0, a2);
-                        F::unpack(qb, m, a1, a3);
+                    for (int i = 0; i < 4; ++i) { D[rt][nb][i] = 0; D1[rt][nb][i] = 0; }
 #pragma unroll
-                        for (int nb = 0; nb < NB; ++nb) mma_chunk(D[nb], D1[nb], a0, a1, a2, a3, bfr[m][nb][0], bfr[m][nb][1]);
-                    }
-                    float sda, sdb, sda1 = 0.f, sdb1 = 0.f;
-                    if (GS) {  // groups 2 cw and 2 cw + 1 of rows ra and rbw
-                        sda = ra < nrows ? sdg[ra * f.nsi + 2 * cw] : 0.f;
-                        sda1 = ra < nrows ? sdg[ra * f.nsi + 2 * cw + 1] : 0.f;
-                        sdb = rbw < nrows ? sdg[rbw * f.nsi + 2 * cw] : 0.f;
-                        sdb1 = rbw < nrows ? sdg[rbw * f.nsi + 2 * cw + 1] : 0.f;
-                    } else {
-                        sda = ra < nrows ? sdp[ra] : 0.f;
-                        sdb = rbw < nrows ? sdp[rbw] : 0.f;
-                    }
+            for (int m = 0; m < MPC; ++m)
+#pragma unroll
+                for (int rt = 0; rt < RT2; ++rt) {
+                    uint32_t a0, a2, a1, a3;
+                    F::unpack(qa[rt], m, a0, a2);
+                    F::unpack(qb[rt], m, a1, a3);
 #pragma unroll
                     for (int nb = 0; nb < NB; ++nb) {
-                        acc[rt][nb][0] = __fmaf_rn(static_cast<float>(D[nb][0]), sda * fcol[nb][0], acc[rt][nb][0]);
-                        acc[rt][nb][1] = __fmaf_rn(static_cast<float>(D[nb][1]), sda * fcol[nb][1], acc[rt][nb][1]);
-                        acc[rt][nb][2] = __fmaf_rn(static_cast<float>(D[nb][2]), sdb * fcol[nb][0], acc[rt][nb][2]);
-                        acc[rt][nb][3] = __fmaf_rn(static_cast<float>(D[nb][3]), sdb * fcol[nb][1], acc[rt][nb][3]);
-                        if (GS) {
-                            acc[rt][nb][0] = __fmaf_rn(static_cast<float>(D1[nb][0]), sda1 * fcol[nb][0], acc[rt][nb][0]);
-                            acc[rt][nb][1] = __fmaf_rn(static_cast<float>(D1[nb][1]), sda1 * fcol[nb][1], acc[rt][nb][1]);
-                            acc[rt][nb][2] = __fmaf_rn(static_cast<float>(D1[nb][2]), sdb1 * fcol[nb][0], acc[rt][nb][2]);
-                            acc[rt][nb][3] = __fmaf_rn(static_cast<float>(D1[nb][3]), sdb1 * fcol[nb][1], acc[rt][nb][3]);
-                        }
+                        if (GS) mma_chunk(D[rt][nb], D1[rt][nb], a0, a1, a2, a3, bfr[m][nb][0], bfr[m][nb][1]);
+                        else mma_s8((NB == 1 && (m & 1)) ? D1[rt][nb] : D[rt][nb], a0, a1, a2, a3, bfr[m][nb][0], bfr[m][nb][1]);
+                    }
+                }
+#pragma unroll
+            for (int rt = 0; rt < RT2; ++rt) {
+                const int ra = rt * 16 + g8, rbw = ra + 8;
+                float sda, sdb, sda1 = 0.f, sdb1 = 0.f;
+                if (GS) {  // groups 2 cw and 2 cw + 1 of rows ra and rbw
+                    sda = ra < nrows ? sdg[ra * f.nsi + 2 * cw] : 0.f;
+                    sda1 = ra < nrows ? sdg[ra * f.nsi + 2 * cw + 1] : 0.f;
+                    sdb = rbw < nrows ? sdg[rbw * f.nsi + 2 * cw] : 0.f;
+                    sdb1 = rbw < nrows ? sdg[rbw * f.nsi + 2 * cw + 1] : 0.f;
+                } else {
+                    sda = ra < nrows ? sdp[ra] : 0.f;
+                    sdb = rbw < nrows ? sdp[rbw] : 0.f;
+                }
+#pragma unroll
+                for (int nb = 0; nb < NB; ++nb) {
+                    if (GS) {
+                        acc[rt][nb][0] = __fmaf_rn(static_cast<float>(D[rt][nb][0]), sda * fcol[nb][0], acc[rt][nb][0]);
+                        acc[rt][nb][1] = __fmaf_rn(static_cast<float>(D[rt][nb][1]), sda * fcol[nb][1], acc[rt][nb][1]);
+                        acc[rt][nb][2] = __fmaf_rn(static_cast<float>(D[rt][nb][2]), sdb * fcol[nb][0], acc[rt][nb][2]);
+                        acc[rt][nb][3] = __fmaf_rn(static_cast<float>(D[rt][nb][3]), sdb * fcol[nb][1], acc[rt][nb][3]);
+                        acc[rt][nb][0] = __fmaf_rn(static_cast<float>(D1[rt][nb][0]), sda1 * fcol[nb][0], acc[rt][nb][0]);
+                        acc[rt][nb][1] = __fmaf_rn(static_cast<float>(D1[rt][nb][1]), sda1 * fcol[nb][1], acc[rt][nb][1]);
+                        acc[rt][nb][2] = __fmaf_rn(static_cast<float>(D1[rt][nb][2]), sdb1 * fcol[nb][0], acc[rt][nb][2]);
+                        acc[rt][nb][3] = __fmaf_rn(static_cast<float>(D1[rt][nb][3]), sdb1 * fcol[nb][1], acc[rt][nb][3]);
+                    } else {  // the two chains' int32 sums add exactly
+                        acc[rt][nb][0] = __fmaf_rn(static_cast<float>(D[rt][nb][0] + D1[rt][nb][0]), sda * fcol[nb][0], acc[rt][nb][0]);
+                        acc[rt][nb][1] = __fmaf_rn(static_cast<float>(D[rt][nb][1] + D1[rt][nb][1]), sda * fcol[nb][1], acc[rt][nb][1]);
+                        acc[rt][nb][2] = __fmaf_rn(static_cast<float>(D[rt][nb][2] + D1[rt][nb][2]), sdb * fcol[nb][0], acc[rt][nb][2]);
+                        acc[rt][nb][3] = __fmaf_rn(static_cast<float>(D[rt][nb][3] + D1[rt][nb][3]), sdb * fcol[nb][1], acc[rt][nb][3]);
                     }
                 }
             }
@@ -1050,8 +1111,7 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
     auto grid_barrier = [&](unsigned k) {
         cons_sync();
         if (ct == 0) {
-            __threadfence();
-            atomicAdd(p.gbar, 1u);
+            red_release_add(p.gbar, 1u);
             const unsigned target = static_cast<unsigned>(G) * ((p.route_here ? 1u : 0u) + k) + p.gate_extra;
             const long long t0 = clock64();
             while (ld_acquire(p.gbar) < target) {
@@ -1096,29 +1156,21 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
         for (int nb = 0; nb < NB; ++nb)
 #pragma unroll
             for (int i = 0; i < 4; ++i) acc[rt][nb][i] = 0.f;
-    // The down jobs are the work experts in order (the shared one first); each one's fragments
-    // are fetched FD - 1 jobs ahead (they come from L2 behind the weight stream, over a
-    // microsecond).
+    // The down jobs are the work experts in order (the shared one first).
     if (kind == 2) {
         const int nwe = f.S + rc.U;
         int s = seq % S;
         uint32_t par = (seq / S) & 1;
-        for (int j = 0; j + 1 < FD; ++j) {
-            if (j < nwe) issue_frag(j, j); else cp_async_commit();
-        }
         for (int we2 = 0; we2 < nwe; ++we2) {
-            const int nx = we2 + FD - 1;
-            if (nx < nwe) issue_frag(nx, nx % FD); else cp_async_commit();
-            down_job(we2, s, par, we2 % FD);
+            down_job(we2, s, par);
             if (++s == S) { s = 0; par ^= 1u; }
         }
     }
-    cp_async_wait<0>();
 
     if (!ok) atomicOr(f.err, COLI_DEVERR_TIMEOUT);
-    // cross-warp reduction (every job is done: the activation slices' region is reused)
+    // cross-warp reduction (every job is done: the ring is reused)
     cons_sync();
-    float *red2 = reinterpret_cast<float *>(sm + p.off_x);  // [warp][rt][nb][lane][4]
+    float *red2 = reinterpret_cast<float *>(ring);  // [warp][rt][nb][lane][4]
     if (active2) {
 #pragma unroll
         for (int rt = 0; rt < RT2; ++rt)
@@ -1234,34 +1286,41 @@ bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan) {
     pl.SB = ((sb1 > sb2 ? sb1 : sb2) + 127) / 128 * 128;
     size_t o = 1024;                                  // mbarriers (up to 60 stages)
     pl.off_route = o; o += (sizeof(RouteCache) + 127) / 128 * 128;
-    pl.off_red1 = o; o += static_cast<size_t>(NGRP) * GW * NB * 32 * 16;
-    o = (o + 127) / 128 * 128;
-    // activation slices (gate/up tiles), then the down jobs' fragment rings, then the final
-    // reduction
+    // One span for what lives in turn: the group reduction buffers and the activation slices
+    // (gate/up tiles), the converter's h slices (between the two grid barriers), the down
+    // stages' fragment slots (after them; one per ring stage).  Then the per-token routing
+    // scratch and the gate partials (until the batch is routed), then the ring; the final
+    // cross-warp reduction reuses the ring once every stage is consumed.
+    const size_t r1bytes = (static_cast<size_t>(NGRP) * GW * NB * 32 * 16 + 127) / 128 * 128;
     const size_t xbytes = static_cast<size_t>(c.hidden / cpc) * 3 * T * colblk;
-    const size_t rbytes = static_cast<size_t>(NCW) * 3 * NB * 32 * 16;
-    // fragment rings: as deep (3, 2, 1) as the region allows (up to 1 KB more)
-    size_t abytes = xbytes > rbytes ? xbytes : rbytes;
-    const size_t fper = static_cast<size_t>(NCW) * (3 * T * colblk + 16);
-    pl.fdepth = 3;
-    while (pl.fdepth > 1 && pl.fdepth * fper > abytes + 1024) --pl.fdepth;
-    abytes = abytes > pl.fdepth * fper ? abytes : pl.fdepth * fper;
-    pl.off_x = o; o += (abytes + 127) / 128 * 128;
-    // per-warp h slices (down projections, only after the batch is routed), aliased with the
-    // per-token routing scratch and the gate partials (only until it is routed)
     const size_t hbytes = static_cast<size_t>(NCW) * 3 * T * colblk;
+    const size_t abytes = ((xbytes > hbytes ? xbytes : hbytes) + 127) / 128 * 128;
+    pl.fslot = static_cast<int>((static_cast<size_t>(rb_i / 64) * (3 * T * colblk + 16) + 127) / 128 * 128);
     const size_t tbytes = (static_cast<size_t>(T) * sizeof(RouteToken) + 127) / 128 * 128;
-    const size_t gbytes = NCW * 2 * MAXTOK * 8 + NCW * MAXTOK * 4;
-    pl.off_hb = o;
-    pl.off_rtok = o;
-    pl.off_gate = o + tbytes;
-    o += ((hbytes > tbytes + gbytes ? hbytes : tbytes + gbytes) + 127) / 128 * 128;
-    o = (o + 1023) / 1024 * 1024;
-    pl.off_ring = o;
+    const size_t gbytes = (static_cast<size_t>(NCW) * 2 * MAXTOK * 8 + NCW * MAXTOK * 4 + 127) / 128 * 128;
     const size_t budget = device_smem_optin() - 1024;
-    if (o + 2 * static_cast<size_t>(pl.SB) > budget) return false;
-    pl.S = static_cast<int>((budget - o) / pl.SB);
-    if (pl.S > 60) pl.S = 60;
+    pl.off_red1 = o;
+    pl.off_frag = o;
+    pl.off_x = o + r1bytes;
+    pl.off_hb = pl.off_x;
+    pl.S = 0;
+    for (int S = 60; S >= 2; --S) {
+        size_t span = r1bytes + abytes;
+        const size_t fr = static_cast<size_t>(S) * pl.fslot;
+        span = span > fr ? span : fr;
+        const size_t ring = o + span + tbytes + gbytes;
+        if (ring + static_cast<size_t>(S) * pl.SB <= budget) {
+            pl.S = S;
+            pl.off_rtok = o + span;
+            pl.off_gate = pl.off_rtok + tbytes;
+            pl.off_ring = ring;
+            break;
+        }
+    }
+    if (pl.S < 2) return false;
+    o = pl.off_ring;
+    const size_t rbytes = static_cast<size_t>(NCW) * 3 * NB * 32 * 16;
+    if (rbytes > static_cast<size_t>(pl.S) * pl.SB) return false;
     // The down projections follow all the CTA's tiles (they need every CTA's h, converted once).
     pl.lag = 1 << 20;
     pl.smem = o + static_cast<size_t>(pl.S) * pl.SB;
@@ -1270,9 +1329,9 @@ bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan) {
 }
 
 static void fill_plan(DecodeParams &p, const DecodePlan &pl) {
-    p.grid = pl.grid; p.S = pl.S; p.SB = pl.SB; p.st_sd = pl.st_sd; p.lag = pl.lag; p.fdepth = pl.fdepth;
-    p.off_route = pl.off_route; p.off_rtok = pl.off_rtok; p.off_gate = pl.off_gate;
-    p.off_red1 = pl.off_red1; p.off_x = pl.off_x; p.off_hb = pl.off_hb; p.off_ring = pl.off_ring;
+    p.grid = pl.grid; p.S = pl.S; p.SB = pl.SB; p.st_sd = pl.st_sd; p.lag = pl.lag; p.fslot = pl.fslot;
+    p.off_route = pl.off_route; p.off_rtok = pl.off_rtok; p.off_gate = pl.off_gate; p.off_red1 = pl.off_red1;
+    p.off_x = pl.off_x; p.off_hb = pl.off_hb; p.off_frag = pl.off_frag; p.off_ring = pl.off_ring;
 }
 
 cudaError_t launch_ffn_decode(DecodeParams p, const DecodePlan &pl, cudaStream_t st) {

@@ -48,9 +48,9 @@ constexpr size_t WS_DSL_BYTES = static_cast<size_t>(DEC_WE) * DEC_CH * (12 * 256
 // Shared-memory plan of the fused decode kernel (decode.cu).
 struct DecodePlan {
     int grid, S, SB, st_sd;                           // ring: S stages of SB bytes
-    size_t off_route, off_rtok, off_gate, off_red1, off_x, off_hb, off_ring, smem;
+    size_t off_route, off_rtok, off_gate, off_red1, off_x, off_hb, off_frag, off_ring, smem;
     int lag;                                          // down-projection lag (experts)
-    int fdepth;                                       // fragment ring depth per warp (1..3)
+    int fslot;                                        // bytes of a down stage's fragment slot
 };
 
 // Parameters of the fused decode kernel.
@@ -70,8 +70,8 @@ struct DecodeParams {
     long long wait_cycles;  // bound of every device-side wait (0: the default, ~2 s)
     unsigned gate_extra;    // added to the logits-arrival target (nonzero only to test the bound)
     // plan (copied from DecodePlan)
-    int grid, S, SB, st_sd, lag, fdepth;
-    size_t off_route, off_rtok, off_gate, off_red1, off_x, off_hb, off_ring;
+    int grid, S, SB, st_sd, lag, fslot;
+    size_t off_route, off_rtok, off_gate, off_red1, off_x, off_hb, off_frag, off_ring;
 };
 
 bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan);
