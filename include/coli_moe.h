@@ -104,10 +104,10 @@ coli_status coli_moe_check_config(const coli_moe_config *cfg);
 
 /* Workspace bytes that coli_moe_layer / coli_moe_ffn / coli_moe_group need for up to
  * max_tokens tokens.  The workspace must be 256-byte aligned and is owned by the caller; calls
- * that share one workspace must be ordered on the GPU (same stream or events).  Its first 256
+ * that share one workspace must be ordered on the GPU (same stream or events).  Its first 512
  * bytes (error word and the counters of the fused decode path) must be zero before its first
  * use: call coli_moe_clear_error once after allocating it (and after a call that reported
- * COLI_DEVERR_TIMEOUT).  Complete calls leave the counters zero.  Host only. */
+ * COLI_DEVERR_TIMEOUT).  Complete calls leave the header ready for the next call.  Host only. */
 coli_status coli_moe_workspace_size(const coli_moe_config *cfg, int max_tokens, size_t *bytes);
 
 /* Number of kernels coli_moe_layer launches for T tokens with this configuration (1 on the fused

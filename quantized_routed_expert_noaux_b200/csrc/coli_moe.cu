@@ -294,8 +294,9 @@ static DecodeParams make_decode(const coli_moe_config *c, const FfnParams &f, ch
     d.rsf = c->routed_scaling;
     d.G = c->n_group;
     d.TG = c->topk_group;
+    d.phase = reinterpret_cast<unsigned *>(base + WS_PHASE);
     d.gbar = reinterpret_cast<unsigned *>(base + WS_GBAR);
-    d.gdep = reinterpret_cast<unsigned *>(base + WS_GDEP);
+    d.ready = reinterpret_cast<unsigned *>(base + WS_READY);
     const WsLayout L = ws_layout(*c, f.T);
     d.dsl = reinterpret_cast<uint4 *>(base + L.dsl);
     d.wait_cycles = g_wait_cycles;

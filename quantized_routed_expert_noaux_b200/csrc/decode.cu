@@ -51,9 +51,6 @@ constexpr int NT = NC + 32;          // + producer warp
 constexpr int GW = 8;                // warps of a phase-1 group
 constexpr int NGRP = NCW / GW;       // phase-1 groups
 constexpr int MAXTOK = 4;            // tokens of the fused path
-#ifndef DOWN_PIECES
-#define DOWN_PIECES 4
-#endif
 constexpr int MAXWE = 33;            // work experts: the shared one + up to 32 unique routed
 // named barriers: 0 __syncthreads, 1 all consumers, 2.. group full, 4.. group reduction free
 constexpr int BAR_CONS = 1, BAR_GFULL = 2, BAR_GFREE = 4;
@@ -364,6 +361,10 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
     const int G = gridDim.x, b = blockIdx.x;
     const int T = f.T, S = p.S;
     const long long bound = p.wait_cycles;
+    // This call's counter set (the previous call left it zero and flipped the phase to it)
+    const unsigned phase = __ldcg(p.phase) & 1u;
+    unsigned *const gbar = p.gbar + 8 * phase;         // logits and grid-barrier arrivals
+    unsigned *const ready = p.ready + 40 * phase;      // converted h chunks per work expert
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm);
     RouteCache &rc = *reinterpret_cast<RouteCache *>(sm + p.off_route);
     RouteToken *rtok = reinterpret_cast<RouteToken *>(sm + p.off_rtok);
@@ -441,24 +442,27 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
         const uint32_t sdb = GS ? static_cast<uint32_t>(nrows) * f.nsi * 4 : 4u * (a1 - a0d);
         // A down stage carries the CTA's block of one work expert's down rows and their scales,
         // and in a second part (its fragment slot) the expert's converted h.  Stages issued before
-        // the conversion is published (the second grid barrier) expect the rows' bytes only;
-        // their fragments and the arrival follow once this thread has seen that barrier.
+        // the expert's chunks are all converted (counted on its readiness counter) expect the
+        // rows' bytes only; their fragments and the arrival follow once this thread has seen the
+        // count complete.
         const uint32_t fbytes = static_cast<uint32_t>(nch * fch);
         auto frag_copy = [&](int we, int s) {
             bulk_g2s(smem_u32(frag + static_cast<size_t>(s) * p.fslot),
                      reinterpret_cast<const unsigned char *>(p.dsl) + static_cast<size_t>(we) * DEC_CH * fch, fbytes, full_bar(s), keep);
         };
-        bool published = false;
-        int seq0 = -1, npend = 0;
-        auto publish = [&]() {  // wait for the second grid barrier, then complete the pending stages
-            const unsigned target = static_cast<unsigned>(G) * ((p.route_here ? 1u : 0u) + 2u) + p.gate_extra;
+        auto converted = [&](int we) {  // bounded wait until every chunk of we is converted
             const long long t0 = clock64();
-            while (ld_acquire(p.gbar) < target) {
+            while (ld_acquire(ready + we) < static_cast<unsigned>(nch)) {
                 if (clock64() - t0 > bound) { ok = false; break; }
             }
+            return ok;
+        };
+        bool published = false;
+        int seq0 = -1, npend = 0;
+        auto publish = [&]() {  // complete the pending stages as their experts' h is converted
             for (int j = 0; j < npend; ++j) {
                 const int s = (seq0 + j) % S;
-                if (ok) {
+                if (ok && converted(j)) {
                     mbar_expect_tx(full_bar(s), fbytes);
                     frag_copy(j, s);
                 } else {
@@ -478,6 +482,7 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
             if (!mbar_wait(empty_bar(s), par ^ 1, bound)) { ok = false; return; }
             ++seq;
             const uint32_t rows = rec ? static_cast<uint32_t>(nrows) * rb_i + sdb : 0u;
+            if (published && !converted(we)) { mbar_arrive(full_bar(s)); return; }
             if (published) mbar_expect_tx(full_bar(s), rows + fbytes);
             else mbar_add_tx(full_bar(s), rows);
             const uint32_t dst = smem_u32(ring + static_cast<size_t>(s) * p.SB);
@@ -606,7 +611,7 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
         }
         if (cw == 0 && p.route_here) {
             __syncwarp();
-            if (lane == 0) atomicAdd(p.gbar, 1u);
+            if (lane == 0) atomicAdd(gbar, 1u);
         }
         // activation slices: X = rint(x * 2^(22 - e)), max|x| < 2^e, written as whole B words
 #pragma unroll
@@ -693,7 +698,7 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
         if (ct == 0) {  // every CTA's logits are written
             const long long t0 = clock64();
             const unsigned target = static_cast<unsigned>(G) + p.gate_extra;
-            while (ld_acquire(p.gbar) < target) {
+            while (ld_acquire(gbar) < target) {
                 if (clock64() - t0 > bound) { atomicOr(f.err, COLI_DEVERR_TIMEOUT); break; }
             }
         }
@@ -875,7 +880,8 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
             if (MAXT > 3) sv.w = scl[MAXT > 3 ? 3 : 0];
             __stcg(reinterpret_cast<float4 *>(dst + n16), sv);
         }
-        __syncwarp();  // the h-slice block is reused only after every lane read it
+        __syncwarp();  // every lane's stores precede lane 0's release; the block may be reused
+        if (lane == 0) red_release_add(ready + we, 1u);  // one more chunk of we converted
     };
 
     // A gate/up tile (taken by one group of 8 warps): every warp multiplies its chunks of the 8
@@ -1106,16 +1112,22 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
         if (ok && active2 && lane == 0) mbar_arrive_cnt(empty_bar(s), NCW / nact);
     };
 
-    // Bounded grid barrier k (1, 2): the arrivals count on after the logits' (the counter is
-    // reset at departure).
+    // Bounded grid barrier k: the arrivals count on after the logits'.
     auto grid_barrier = [&](unsigned k) {
         cons_sync();
         if (ct == 0) {
-            red_release_add(p.gbar, 1u);
+            red_release_add(gbar, 1u);
             const unsigned target = static_cast<unsigned>(G) * ((p.route_here ? 1u : 0u) + k) + p.gate_extra;
             const long long t0 = clock64();
-            while (ld_acquire(p.gbar) < target) {
+            while (ld_acquire(gbar) < target) {
                 if (clock64() - t0 > bound) { atomicOr(f.err, COLI_DEVERR_TIMEOUT); break; }
+            }
+            if (b == 0) {  // every CTA read the phase before arriving: hand the other set to the next call
+                unsigned *const ogbar = p.gbar + 8 * (phase ^ 1u);
+                unsigned *const oready = p.ready + 40 * (phase ^ 1u);
+                *ogbar = 0u;
+                for (int i = 0; i < MAXWE; ++i) oready[i] = 0u;
+                *p.phase = phase ^ 1u;
             }
         }
         cons_sync();
@@ -1142,13 +1154,13 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
     if (my_tiles > 0 && wg != 0) named_sync(BAR_GFREE + grp, GW * 32);  // the last arrival
 
     // Down projections: once every CTA's h is written (grid barrier), each h chunk is converted
-    // once (chunk q by CTA q mod G, warp q / G), and once all are (second grid barrier) every CTA
-    // multiplies its block of down rows with them.
+    // once (chunk q by CTA q mod G, warp q / G) and counted on its expert's readiness counter;
+    // the producer completes each down stage with the expert's converted h once the count is
+    // full, and every CTA multiplies its block of down rows with it.
     if (kind == 2) {
         grid_barrier(1u);
         const int nq = (f.S + rc.U) * nch2;
         for (int q = b + G * cw; q < nq; q += G * NCW) convert_chunk(q / nch2, q % nch2);
-        grid_barrier(2u);
     }
 #pragma unroll
     for (int rt = 0; rt < RT2; ++rt)
@@ -1183,26 +1195,22 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
     for (int fi = ct; fi < nrows * T; fi += NC) {
         const int r = fi / T, t = fi % T;
         const int rt = r >> 4, rr = r & 15, gg = rr & 7, hi = rr >> 3;
-        float v = 0.f;
-        for (int w2 = 0; w2 < nact; ++w2) {
+        float pv[NCW][3];  // every term first, then the sum in the fixed order
+#pragma unroll
+        for (int w2 = 0; w2 < NCW; ++w2)
 #pragma unroll
             for (int sidx = 0; sidx < 3; ++sidx) {
                 const int col = 3 * t + sidx, nb = col >> 3, c8 = col & 7;
                 const int ln = gg * 4 + (c8 >> 1), ix = 2 * hi + (c8 & 1);
-                v = __fadd_rn(v, red2[(((w2 * RT2 + rt) * NB + nb) * 32 + ln) * 4 + ix]);
+                pv[w2][sidx] = w2 < nact ? red2[(((w2 * RT2 + rt) * NB + nb) * 32 + ln) * 4 + ix] : 0.f;
             }
-        }
+        float v = 0.f;
+#pragma unroll
+        for (int w2 = 0; w2 < NCW; ++w2)
+#pragma unroll
+            for (int sidx = 0; sidx < 3; ++sidx)
+                if (w2 < nact) v = __fadd_rn(v, pv[w2][sidx]);
         f.out[static_cast<size_t>(t) * f.H + j_lo + r] = v;
-    }
-    // Departure: every warp of this CTA is past its last wait on the counter; the last CTA to
-    // leave zeroes it for the next call on this workspace.
-    if (ct == 0) {
-        __threadfence();
-        if (atomicAdd(p.gdep, 1u) == static_cast<unsigned>(G) - 1u) {
-            *p.gbar = 0u;
-            *p.gdep = 0u;
-            __threadfence();
-        }
     }
 }
 

@@ -33,12 +33,14 @@ struct FfnParams {
     int *err;                          // device error word
 };
 
-// Workspace header (first 256 bytes): error word, then counters of the fused decode path (the
-// arrival count of the logits and the grid barriers, the departure count).  All must be zero
-// before the first call on a workspace (coli_moe_clear_error zeroes them); the kernels leave
-// them zero after every complete call.
-constexpr int WS_ERR = 0, WS_GBAR = 64, WS_GDEP = 96;
-constexpr int WS_HEADER = 256;
+// Workspace header (first 512 bytes): error word; then the fused decode path's phase word and
+// two sets of counters (per set: the arrival count of the logits and the grid barrier at
+// WS_GBAR + 32 * set, the converted h chunks per work expert at WS_READY + 160 * set).  A call
+// uses the set the phase names; once every CTA has read the phase it zeroes the other set and
+// flips the phase.  All must be zero before the first call on a workspace
+// (coli_moe_clear_error zeroes them).
+constexpr int WS_ERR = 0, WS_PHASE = 32, WS_GBAR = 64, WS_READY = 128;
+constexpr int WS_HEADER = 512;
 // Fused decode path: h of every (work expert, chunk of the down rows' K) converted once, as the
 // chunk's MMA B block (one column per token and slice, at most 12 columns of at most 256
 // bytes) followed by the tokens' 4 scales: [33 work experts][16 chunks] of 12 * 256 + 16 bytes.
@@ -64,7 +66,9 @@ struct DecodeParams {
     int32_t *f_counts, *f_offsets, *f_perm, *f_unique, *f_nuniq;
     double rsf;
     int G, TG;
-    unsigned *gbar, *gdep;
+    unsigned *phase;        // which counter set this call uses
+    unsigned *gbar;         // [2 sets, 8 words apart]: logits and grid-barrier arrivals
+    unsigned *ready;        // [2 sets, 40 words apart][33]: converted h chunks per work expert
     uint4 *dsl;             // h chunks converted once (WS_DSL_BYTES)
     int route_here;         // 1: the kernel routes from its own logits; 0: routing arrays are inputs
     long long wait_cycles;  // bound of every device-side wait (0: the default, ~2 s)

@@ -178,7 +178,7 @@ def test_fused_kernel_waits_run_out_and_the_workspace_recovers():
     assert err & q.DEVERR_TIMEOUT, err
     assert elapsed < 5.0, elapsed
     q.coli_moe_clear_error(ws)
-    assert (ws[:256] == 0).all()
+    assert (ws[:512] == 0).all()  # the whole header: error word, phase and both counter sets
     q.coli_moe_layer(cfg, L.weights(), x, T, out, None, None, ws)
     assert q.coli_moe_error_word(ws) == 0
     ref, _, _, _ = oracle_layer_tokens(L, x.cpu(), range(T))

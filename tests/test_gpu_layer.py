@@ -308,8 +308,9 @@ def test_batch_union_equals_per_token_bitwise(name, T):
 
 @pytest.mark.parametrize("T", [1, 4])
 def test_layer_deterministic_and_repeatable(T):
-    """Repeated calls on one workspace give identical bits (the fused path's counters return to
-    zero after every call) and leave the error word clean."""
+    """Repeated calls on one workspace give identical bits and leave the error word clean; the
+    fused path leaves its header ready for the next call: the phase word names a counter set
+    that is all zero (the other set holds the last call's counts)."""
     L = layer_for("glm_decode")
     cfg = q.config_for(L.wl)
     ws = workspace(cfg, T)
@@ -321,8 +322,12 @@ def test_layer_deterministic_and_repeatable(T):
         q.coli_moe_layer(cfg, L.weights(), x, T, out, None, None, ws)
         outs.append(out.cpu().numpy())
     assert q.coli_moe_error_word(ws) == 0
-    hdr = ws[:256].view(torch.int32).cpu().numpy()
-    assert (hdr == 0).all(), hdr
+    hdr = ws[:512].view(torch.int32).cpu().numpy()  # header words: phase 8, arrivals 16 + 8 set,
+    phase = int(hdr[8])                              # converted chunks 32 + 40 set
+    assert phase in (0, 1), hdr
+    assert hdr[16 + 8 * phase] == 0, hdr
+    assert (hdr[32 + 40 * phase:32 + 40 * phase + 33] == 0).all(), hdr
+    assert (hdr[1:8] == 0).all(), hdr
     np.testing.assert_array_equal(outs[0], outs[1])
     np.testing.assert_array_equal(outs[0], outs[2])
 
