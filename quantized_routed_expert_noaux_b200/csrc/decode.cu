@@ -206,7 +206,7 @@ __device__ __forceinline__ void slices3(int X, int &s0, int &s1, int &s2) {
 
 // ------------------------------------------------------------------------- routing ---------
 __device__ __forceinline__ bool beats(double va, int ia, double vb, int ib) {
-    return va > vb || (va == vb && ia < ib);
+    return static_cast<bool>(static_cast<int>(va > vb) | (static_cast<int>(va == vb) & static_cast<int>(ia < ib)));
 }
 
 constexpr int RMAX_BLOCKS = 8;  // E <= 256 on the fused path: blocks of 32 experts
@@ -224,24 +224,31 @@ struct RouteCache {             // the routing of the call, shared memory
     int ids[MAXTOK][8];         // per token: selected ids, slot order
     float w[MAXTOK][8];         //            and weights
     int sorted[32];             // grouped order of the slots
+    int sid[32], stok[32];      // per grouped position: expert id and token of its slot
+    float sw[32];               //                       and its weight
     float xscale[MAXTOK];       // activation scale of each token row, 2^(e - 22)
     int err;
 };
 
 // Step A: the best max(K, 2) of one 32-expert block of token t (lane = expert in the block).
-__device__ void route_block(const DecodeParams &p, int t, int blk, int lane, RouteToken &r) {
+// Ranks within a warp come from broadcast reads of the warp's values in shared-memory scratch
+// (`scr`, 32 doubles) rather than shuffles.
+__device__ void route_block(const DecodeParams &p, int t, int blk, int lane, RouteToken &r, double *scr) {
     const int E = p.f.E, K = p.f.K;
     const int e = blk * 32 + lane;
     const float lf = __ldcg(p.logits + static_cast<size_t>(t) * E + e);
     const float bf = __ldg(p.bias + e);
     const double s = 1.0 / (1.0 + exp(-static_cast<double>(lf)));
     const double c = s + static_cast<double>(bf);
+    scr[lane] = c;
+    __syncwarp();
     int rank = 0;
 #pragma unroll
     for (int o = 0; o < 32; ++o) {
-        const double oc = __shfl_sync(FULL, c, o);
-        rank += (oc > c || (oc == c && o < lane)) ? 1 : 0;  // same block: id order = lane order
+        const double oc = scr[o];
+        rank += static_cast<int>(oc > c) | (static_cast<int>(oc == c) & static_cast<int>(o < lane));  // id order = lane order
     }
+    __syncwarp();  // the scratch is reused by the warp's next job only after every lane read it
     const int keep = K > 2 ? K : 2;
     if (rank < keep) {
         r.cval[blk][rank] = c;
@@ -254,7 +261,7 @@ __device__ void route_block(const DecodeParams &p, int t, int blk, int lane, Rou
 // weights are those of the per-token definition: largest biased score first, lower id on
 // ties; groups score the sum of their two largest biased scores, lower group on ties; weights
 // from the unbiased scores renormalised in slot order, times routed_scaling.
-__device__ void route_select(const DecodeParams &p, int t, int lane, RouteToken &r, RouteCache &rc) {
+__device__ void route_select(const DecodeParams &p, int t, int lane, RouteToken &r, RouteCache &rc, double *scr) {
     const int E = p.f.E, K = p.f.K, G = p.G, TG = p.TG;
     const int nb = E / 32;
     const bool grouped = G > 1 && TG < G;
@@ -277,7 +284,7 @@ __device__ void route_select(const DecodeParams &p, int t, int lane, RouteToken 
         int rk = 0;
         for (int o = 0; o < G; ++o) {
             const double og = __shfl_sync(FULL, gsc, o);
-            rk += (og > gsc || (og == gsc && o < lane)) ? 1 : 0;
+            rk += static_cast<int>(og > gsc) | (static_cast<int>(og == gsc) & static_cast<int>(o < lane));
         }
         const unsigned gmask = __ballot_sync(FULL, lane < G && rk < TG);
         kmask = __ballot_sync(FULL, lane < nb && ((gmask >> (lane / bpg)) & 1u));
@@ -296,13 +303,13 @@ __device__ void route_select(const DecodeParams &p, int t, int lane, RouteToken 
         s2 = r.cs[bk][k];
         id = r.cid[bk][k];
     }
+    int *scri = reinterpret_cast<int *>(scr + 32);
+    scr[lane] = c2;
+    scri[lane] = id;
+    __syncwarp();
     int rank2 = 0;
 #pragma unroll
-    for (int o = 0; o < 32; ++o) {
-        const double oc = __shfl_sync(FULL, c2, o);
-        const int oi = __shfl_sync(FULL, id, o);
-        rank2 += beats(oc, oi, c2, id) ? 1 : 0;
-    }
+    for (int o = 0; o < 32; ++o) rank2 += beats(scr[o], scri[o], c2, id) ? 1 : 0;
     if (rank2 < K) { r.sel_s[rank2] = s2; r.sel_id[rank2] = id; }
     __syncwarp();
     if (lane < K) {
@@ -704,29 +711,41 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
         }
         cons_sync();
         const int nb = f.E / 32;
-        for (int job = cw; job < T * nb; job += NCW) route_block(p, job / nb, job % nb, lane, rtok[job / nb]);
+        // the group reduction buffers are idle until the first tile: per-warp scratch of 48 doubles
+        double *scr = reinterpret_cast<double *>(red1) + cw * 48;
+        for (int job = cw; job < T * nb; job += NCW) route_block(p, job / nb, job % nb, lane, rtok[job / nb], scr);
         cons_sync();
-        if (cw < T) route_select(p, cw, lane, rtok[cw], rc);
+        if (cw < T) route_select(p, cw, lane, rtok[cw], rc, scr);
         cons_sync();
         if (cw == 0) {
-            // slot s = t K + k; stable sort of the slots by expert id
-            const int n = T * f.K;
-            const int t0 = lane < n ? lane / f.K : 0;
-            const int id = lane < n ? rc.ids[t0][lane - t0 * f.K] : 0x7fffffff;
-            const float w0 = lane < n ? rc.w[t0][lane - t0 * f.K] : 0.f;
+            // slot s = t K + k; stable sort of the slots by expert id (ranks from broadcast reads
+            // of the selected ids: no shuffles, whose cost here varies tenfold with code layout)
+            const int n = T * f.K, K = f.K;
+            const int t0 = lane < n ? lane / K : 0;
+            const int id = lane < n ? rc.ids[t0][lane - t0 * K] : 0x7fffffff;
+            const float w0 = lane < n ? rc.w[t0][lane - t0 * K] : 0.f;
             int rk = 0;
 #pragma unroll
-            for (int o = 0; o < 32; ++o) {
-                const int oid = __shfl_sync(FULL, id, o);
-                rk += ((oid < id) || (oid == id && o < lane)) ? 1 : 0;
+            for (int t2 = 0; t2 < MAXT; ++t2)
+#pragma unroll
+                for (int k2 = 0; k2 < 8; ++k2) {
+                    if (t2 < T && k2 < K) {
+                        const int oid = rc.ids[t2][k2], o = t2 * K + k2;
+                        rk += static_cast<int>(oid < id) | (static_cast<int>(oid == id) & static_cast<int>(o < lane));
+                    }
+                }
+            if (lane < n) {
+                rc.sorted[rk] = lane;
+                rc.sid[rk] = id;
+                rc.stok[rk] = t0;
+                rc.sw[rk] = w0;
             }
-            if (lane < n) rc.sorted[rk] = lane;
             __syncwarp();
             const int sl = lane < n ? rc.sorted[lane] : 0;  // position `lane` holds slot sl
-            const int idr = __shfl_sync(FULL, id, sl);
-            const int tr = __shfl_sync(FULL, t0, sl);
-            const float wr = __shfl_sync(FULL, w0, sl);
-            const int idp = __shfl_up_sync(FULL, idr, 1);
+            const int idr = lane < n ? rc.sid[lane] : 0x7fffffff;
+            const int tr = lane < n ? rc.stok[lane] : 0;
+            const float wr = lane < n ? rc.sw[lane] : 0.f;
+            const int idp = lane > 0 && lane < n ? rc.sid[lane - 1] : -1;
             const bool first = lane < n && (lane == 0 || idp != idr);
             const unsigned m = __ballot_sync(FULL, first);
             const int U = __popc(m);
@@ -1145,9 +1164,11 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
         ++lam;
         if (mine) gate_up_tile(we1, rb1, s, par);
     };
-    for (int l = 0; l < nsh; ++l) tile(0, sh_lo + l);
+    // the batch is routed first, so the routed tiles start streaming while the shared expert's
+    // (already in the ring) are multiplied (measured on B200: 45.5 against 48.0 us at one token)
     if (p.route_here) route_batch();
     if (ct == 0) mbar_arrive(route_bar);
+    for (int l = 0; l < nsh; ++l) tile(0, sh_lo + l);
     JobIter it;
     it.u = -f.S;
     while ((kind = next_job(it, b, G, NRB, rc.U, f.S, p.lag, we, rb)) == 1) tile(we, rb);
