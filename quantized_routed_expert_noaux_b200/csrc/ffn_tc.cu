@@ -54,9 +54,8 @@ constexpr int KB = 128;                       // k per ring stage
 // eight TMEM A stages instead of four, measured slower on the 2048-token Zipf layer: 2.45 against
 // 2.20 ms per step, the extra tiles costing more than the deeper A pipeline saves.)
 constexpr int MAXTOK = 96;
-constexpr int NA = 8;                         // A ring stages (packed int4 tiles)
+constexpr int NA_MAX = 8;                     // A ring stages (at most; per container below)
 constexpr int NB = 6;                         // B ring stages
-constexpr int A_RAW = 128 * (KB / 2);         // packed int4 A tile: 8 KB
 constexpr int B_MAX = 2 * MAXTOK * KB;        // B rows of one stage: 24 KB
 constexpr int NBOX = 4;                       // B box heights 16 << i rows
 constexpr int W_CONV = 4, W_EPI0 = 4, N_EPI = 8, W_PRODA = 12, W_MMA = 13, W_PRODB = 14;
@@ -69,7 +68,16 @@ static_assert(SPG >= 1, "no room for TMEM A stages");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr long long WAIT_CYCLES = 4000000000LL;  // ~2 s at 1.9 GHz: bound of every wait
 constexpr float QMAX = 32512.0f;              // |X| <= 32512 keeps Xh = (X + 128) >> 8 in [-127, 127]
-constexpr size_t TC_SMEM = static_cast<size_t>(NA) * A_RAW + static_cast<size_t>(NB) * B_MAX + 1024;
+// Weight containers: bytes of one row's k-block (RB), A ring stages, the code's multiplier (the
+// signed byte the MMA sees is MUL * q: int4 16q, int2 64q, int8 q).
+template <int FMT> struct TcFmt;
+template <> struct TcFmt<4> { static constexpr int RB = KB / 2, NA = 8; static constexpr float MUL = 16.0f; };
+template <> struct TcFmt<8> { static constexpr int RB = KB, NA = 4; static constexpr float MUL = 1.0f; };
+template <> struct TcFmt<2> { static constexpr int RB = KB / 4, NA = 8; static constexpr float MUL = 64.0f; };
+template <int FMT>
+constexpr size_t tc_smem() {
+    return static_cast<size_t>(TcFmt<FMT>::NA) * 128 * TcFmt<FMT>::RB + static_cast<size_t>(NB) * B_MAX + 1024;
+}
 constexpr int EPI_BAR = 1;                    // named barrier of the epilogue warps
 
 // kind::i8 instruction descriptor: D s32 (bits 4-5 = 2), A and B signed 8-bit (bits 7-9, 10-12
@@ -215,22 +223,28 @@ __device__ __forceinline__ bool elect_one() {
 }
 
 // ------------------------------------------------------------------ activation quantisation --
-// 8 consecutive values -> 8 hi bytes and 8 lo bytes of X = rint(v * inv), in the (0,2,4,6,1,3,5,7)
-// order of the unpacked weights.
-__device__ __forceinline__ void quant8(const float *v, float inv, uint2 &hi, uint2 &lo) {
-    constexpr int ORD[8] = {0, 2, 4, 6, 1, 3, 5, 7};
-    uint32_t h[2] = {0u, 0u}, l[2] = {0u, 0u};
+// Position p of every 16 consecutive k holds element ord<FMT>(p): the order in which the
+// converters lay out the unpacked weight codes (int4: a word's even codes, then its odd ones;
+// int2: codes 0, 4, 8, 12 of a word, then 1, 5, 9, 13, ...; int8: as stored).
+template <int FMT>
+__device__ __forceinline__ constexpr int ord16(int p) {
+    return FMT == 4 ? (p & 8) + 2 * (p & 3) + ((p >> 2) & 1) : (FMT == 2 ? 4 * (p & 3) + (p >> 2) : p);
+}
+// 16 consecutive values -> 16 hi bytes and 16 lo bytes of X = rint(v * inv), in that order.
+template <int FMT>
+__device__ __forceinline__ void quant16(const float *v, float inv, uint4 &hi, uint4 &lo) {
+    uint32_t h[4] = {0u, 0u, 0u, 0u}, l[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-    for (int p = 0; p < 8; ++p) {
-        int x = __float2int_rn(v[ORD[p]] * inv);
+    for (int p = 0; p < 16; ++p) {
+        int x = __float2int_rn(v[ord16<FMT>(p)] * inv);
         x = max(-32512, min(32512, x));
         const int xh = (x + 128) >> 8;
         const int xl = x - 256 * xh;
         h[p >> 2] |= (static_cast<uint32_t>(xh) & 0xFFu) << (8 * (p & 3));
         l[p >> 2] |= (static_cast<uint32_t>(xl) & 0xFFu) << (8 * (p & 3));
     }
-    hi = make_uint2(h[0], h[1]);
-    lo = make_uint2(l[0], l[1]);
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
 
 template <typename In>
@@ -258,7 +272,7 @@ struct QuantArgs {
     const int32_t *perm;     // x only: slot -> (token, k)
     const float *topk_w;     // x only
     int8_t *q;               // [2*slots][len]: hi row, lo row
-    float *scale;            // [slots]: max|v| / (32512 * 16)
+    float *scale;            // [slots]: max|v| / (32512 * MUL)
     int *tok_of;             // x only: [slots]
     float *w_of;             // x only: [slots]
     int *err;
@@ -266,7 +280,7 @@ struct QuantArgs {
 
 // One warp per slot.  GATHER: the row is x of the slot's token (grouped order of the batch
 // union), and the slot's token and combine weight are recorded for the down GEMM.
-template <typename In, bool GATHER>
+template <typename In, bool GATHER, int FMT>
 __device__ __forceinline__ void quant_slot(const QuantArgs &a, int pos, int lane) {
     const In *row;
     if (GATHER) {
@@ -305,14 +319,15 @@ __device__ __forceinline__ void quant_slot(const QuantArgs &a, int pos, int lane
 #pragma unroll
     for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     const float inv = amax > 0.f ? QMAX / amax : 0.f;
-    if (lane == 0) a.scale[pos] = amax / (QMAX * 16.0f);
-    uint2 *qh = reinterpret_cast<uint2 *>(a.q + static_cast<size_t>(2 * pos) * a.len);
-    uint2 *ql = reinterpret_cast<uint2 *>(a.q + static_cast<size_t>(2 * pos + 1) * a.len);
-    for (int j = lane; j < n8; j += 32) {
-        float v[8];
-        load8<In>(row, j, v);
-        uint2 hi, lo;
-        quant8(v, inv, hi, lo);
+    if (lane == 0) a.scale[pos] = amax / (QMAX * TcFmt<FMT>::MUL);
+    uint4 *qh = reinterpret_cast<uint4 *>(a.q + static_cast<size_t>(2 * pos) * a.len);
+    uint4 *ql = reinterpret_cast<uint4 *>(a.q + static_cast<size_t>(2 * pos + 1) * a.len);
+    for (int j = lane; j < n8 / 2; j += 32) {
+        float v[16];
+        load8<In>(row, 2 * j, v);
+        load8<In>(row, 2 * j + 1, v + 8);
+        uint4 hi, lo;
+        quant16<FMT>(v, inv, hi, lo);
         qh[j] = hi;
         ql[j] = lo;
     }
@@ -380,7 +395,7 @@ struct PrepArgs {
 };
 
 // x quantisation in grouped slot order + chunk table (last block) + zeroing of out.
-template <typename In>
+template <typename In, int FMT>
 __global__ void __launch_bounds__(256) tc_prep_kernel(const PrepArgs a) {
     const int slot_blocks = (a.qa.slots + 7) / 8;
     const size_t gt = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -391,12 +406,13 @@ __global__ void __launch_bounds__(256) tc_prep_kernel(const PrepArgs a) {
         return;
     }
     const int pos = blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (pos < a.qa.slots) quant_slot<In, true>(a.qa, pos, threadIdx.x & 31);
+    if (pos < a.qa.slots) quant_slot<In, true, FMT>(a.qa, pos, threadIdx.x & 31);
 }
 
+template <int FMT>
 __global__ void __launch_bounds__(256) tc_quant_h_kernel(const QuantArgs a) {
     const int pos = blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (pos < a.slots) quant_slot<float, false>(a, pos, threadIdx.x & 31);
+    if (pos < a.slots) quant_slot<float, false, FMT>(a, pos, threadIdx.x & 31);
 }
 
 struct GemmArgs {
@@ -421,13 +437,15 @@ struct TcMaps {
 //          gate rows 16q.., lanes 32q+16.. the matching up rows), B = quantised x; epilogue
 //          h = SiLU(g) * u into hbuf (float32).
 // PHASE 2: down.  A = 128 rows of Wd, B = quantised h; epilogue out[token] += w * y.
-template <int PHASE>
+template <int PHASE, int FMT>
 __global__ void __launch_bounds__(TC_THREADS, 1)
 tc_gemm_kernel(const __grid_constant__ TcMaps maps, const GemmArgs p) {
+    constexpr int NA = TcFmt<FMT>::NA, RB = TcFmt<FMT>::RB;
+    constexpr int A_RAW = 128 * RB;  // A tile of one k-block: 128 rows of RB bytes
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    __shared__ __align__(8) uint64_t bars[2 * NA + 2 * NB + 2 * NTS + 5];
+    __shared__ __align__(8) uint64_t bars[2 * NA_MAX + 2 * NB + 2 * NTS + 5];
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
     __shared__ float s_bs[2][MAXTOK], s_w[2][MAXTOK];
@@ -497,7 +515,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const GemmArgs p) {
                 if (lane == 0) mbar_expect_tx(fb, is_a ? A_RAW : n16 * 16 * KB);
                 __syncwarp();
                 if (is_a) {
-                    if (lane == 0) tma_load_4d(smem_u32(sa + s * A_RAW), ta, kb * (KB / 2), m * MROWS, 0, ez, fb);
+                    if (lane == 0) tma_load_4d(smem_u32(sa + s * A_RAW), ta, kb * RB, m * MROWS, 0, ez, fb);
                 } else if (lane < NBOX) {
                     const int bit = NBOX - 1 - lane;
                     if ((n16 >> bit) & 1) {
@@ -559,7 +577,8 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const GemmArgs p) {
         // ------------------------------------------------------------------ converters
         const int q = warp;
         const int rho = PHASE == 1 ? (lane < 16 ? 16 * q + lane : 64 + 16 * q + (lane - 16)) : 32 * q + lane;
-        const int swz = (rho >> 1) & 3;  // 64-byte swizzle: 16-byte chunk c of row r sits at c ^ ((r >> 1) & 3)
+        // RB-byte swizzle of the A tile: 16-byte chunk c of row r sits at c ^ ((r * RB >> 7) & (RB / 16 - 1))
+        const int swz = ((rho * RB) >> 7) & (RB / 16 - 1);
         const uint32_t ta = tbase + (static_cast<uint32_t>(32 * q) << 16);
         uint32_t it = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
@@ -567,19 +586,26 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const GemmArgs p) {
                 const int s = it % NA, ts = it % NTS;
                 if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&afull[s]), (it / NA) & 1, abort, f.err)))
                     goto conv_done;
-                const unsigned char *row = sa + s * A_RAW + rho * (KB / 2);
-                uint4 v[4];
+                const unsigned char *row = sa + s * A_RAW + rho * RB;
+                uint4 v[RB / 16];
 #pragma unroll
-                for (int cch = 0; cch < 4; ++cch) v[cch] = *reinterpret_cast<const uint4 *>(row + ((cch ^ swz) << 4));
+                for (int cch = 0; cch < RB / 16; ++cch) v[cch] = *reinterpret_cast<const uint4 *>(row + ((cch ^ swz) << 4));
                 mbar_arrive(smem_u32(&aempty[s]));
                 uint32_t o[32];
 #pragma unroll
-                for (int cch = 0; cch < 4; ++cch) {
+                for (int cch = 0; cch < RB / 16; ++cch) {
                     const uint32_t w4[4] = {v[cch].x, v[cch].y, v[cch].z, v[cch].w};
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        o[8 * cch + 2 * i] = (w4[i] << 4) & 0xF0F0F0F0u;  // codes 0,2,4,6 of the word
-                        o[8 * cch + 2 * i + 1] = w4[i] & 0xF0F0F0F0u;     // codes 1,3,5,7
+                        if (FMT == 8) {         // the codes as they are
+                            o[4 * cch + i] = w4[i];
+                        } else if (FMT == 4) {  // a word's codes 0,2,4,6 then 1,3,5,7, as 16q
+                            o[8 * cch + 2 * i] = (w4[i] << 4) & 0xF0F0F0F0u;
+                            o[8 * cch + 2 * i + 1] = w4[i] & 0xF0F0F0F0u;
+                        } else {                // codes 0,4,8,12, then 1,5,9,13, ..., as 64q
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) o[16 * cch + 4 * i + j] = (w4[i] << (6 - 2 * j)) & 0xC0C0C0C0u;
+                        }
                     }
                 }
                 if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&tempty[ts]), ((it / NTS) & 1) ^ 1, abort, f.err)))
@@ -701,11 +727,13 @@ bool encode_u8(CUtensorMap *m, const void *base, cuuint32_t rank, const cuuint64
 // Packed weight rows of a set of records as a 4-D byte tensor {row bytes, rows, matrices,
 // records}; the box takes `box_rows` rows of `box_mats` consecutive matrices.
 bool weight_map(CUtensorMap *m, const uint8_t *base, size_t row_bytes, size_t rows, size_t mats, size_t nrec,
-                size_t rec_stride, cuuint32_t box_rows, cuuint32_t box_mats) {
+                size_t rec_stride, cuuint32_t box_rows, cuuint32_t box_mats, int fmt) {
     const cuuint64_t dims[4] = {row_bytes, rows, mats, nrec};
     const cuuint64_t strides[3] = {row_bytes, rows * row_bytes, rec_stride};
-    const cuuint32_t box[4] = {KB / 2, box_rows, box_mats, 1};
-    return encode_u8(m, base, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B);
+    const cuuint32_t rb = static_cast<cuuint32_t>(KB * fmt / 8);  // one k-block of a row: 32/64/128 bytes
+    const cuuint32_t box[4] = {rb, box_rows, box_mats, 1};
+    const CUtensorMapSwizzle sw = rb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : (rb == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+    return encode_u8(m, base, 4, dims, strides, box, sw);
 }
 
 // Quantised B rows {len bytes, 2 * slots rows}, boxes of `box_rows` rows.
@@ -733,13 +761,16 @@ int tc_max_chunks(const coli_moe_config &c, int T) {
 
 bool tc_shape_ok(const coli_moe_config &c) {
     // m-blocks of 64 (gate/up) and 128 (down) rows, k-blocks of 128, int32 accumulators exact
-    // for K <= 65536 (|16q * X| <= 2^14 per product)
-    // per-row scales only: the int32 accumulation runs over all of K
-    return c.wfmt == COLI_W_INT4 && c.group_size == 0 && c.hidden % 128 == 0 && c.inter % 128 == 0 &&
-           c.hidden <= 65536 && c.inter <= 65536;
+    // for K <= 65536 (|MUL q * X| <= 128 * 128 = 2^14 per product: 16q for int4, 64q for int2,
+    // q for int8); per-row scales only: the int32 accumulation runs over all of K
+    return (c.wfmt == COLI_W_INT4 || c.wfmt == COLI_W_INT8 || c.wfmt == COLI_W_INT2) && c.group_size == 0 &&
+           c.hidden % 128 == 0 && c.inter % 128 == 0 && c.hidden <= 65536 && c.inter <= 65536;
 }
 
-cudaError_t launch_ffn_tc(const FfnParams &f, const TcBuffers &b, cudaStream_t st) {
+namespace {
+
+template <int FMT>
+cudaError_t launch_tc_fmt(const FfnParams &f, const TcBuffers &b, cudaStream_t st) {
     const int TK = f.T * f.K;
     const int slots = TK + f.T * f.S;
     cudaError_t e;
@@ -765,9 +796,9 @@ cudaError_t launch_ffn_tc(const FfnParams &f, const TcBuffers &b, cudaStream_t s
     pa.out_n4 = static_cast<size_t>(f.T) * f.H / 4;
     const int prep_blocks = (slots + 7) / 8 + 1;
     if (f.act == COLI_ACT_BF16)
-        tc_prep_kernel<uint16_t><<<prep_blocks, 256, 0, st>>>(pa);
+        tc_prep_kernel<uint16_t, FMT><<<prep_blocks, 256, 0, st>>>(pa);
     else
-        tc_prep_kernel<float><<<prep_blocks, 256, 0, st>>>(pa);
+        tc_prep_kernel<float, FMT><<<prep_blocks, 256, 0, st>>>(pa);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     // tensor maps (host-side encodings of the operands' shapes; no device work)
@@ -775,22 +806,23 @@ cudaError_t launch_ffn_tc(const FfnParams &f, const TcBuffers &b, cudaStream_t s
     const size_t rbh = f.rb_h, rbi = f.rb_i, I = f.I, H = f.H;
     const size_t rec_bytes = f.off_sd + H * 4;
     const size_t rec_pad = (rec_bytes + 255) & ~static_cast<size_t>(255);
-    bool ok = weight_map(&m1.a, f.experts, rbh, I, 2, f.E, f.stride, 64, 2) &&
-              weight_map(&m2.a, f.experts + f.off_wd, rbi, H, 1, f.E, f.stride, 128, 1) &&
+    bool ok = weight_map(&m1.a, f.experts, rbh, I, 2, f.E, f.stride, 64, 2, FMT) &&
+              weight_map(&m2.a, f.experts + f.off_wd, rbi, H, 1, f.E, f.stride, 128, 1, FMT) &&
               act_maps(&m1, b.xq, H, 2 * static_cast<size_t>(slots)) &&
               act_maps(&m2, b.hq, I, 2 * static_cast<size_t>(slots));
     if (ok && f.S) {
-        ok = weight_map(&m1.as, f.shared, rbh, I, 2, 1, rec_pad, 64, 2) &&
-             weight_map(&m2.as, f.shared + f.off_wd, rbi, H, 1, 1, rec_pad, 128, 1);
+        ok = weight_map(&m1.as, f.shared, rbh, I, 2, 1, rec_pad, 64, 2, FMT) &&
+             weight_map(&m2.as, f.shared + f.off_wd, rbi, H, 1, 1, rec_pad, 128, 1, FMT);
     } else {
         m1.as = m1.a;
         m2.as = m2.a;
     }
     if (!ok) return cudaErrorInvalidValue;
 
-    e = cudaFuncSetAttribute(tc_gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(TC_SMEM));
+    constexpr size_t TC_SMEM = tc_smem<FMT>();
+    e = cudaFuncSetAttribute(tc_gemm_kernel<1, FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(TC_SMEM));
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(tc_gemm_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(TC_SMEM));
+    e = cudaFuncSetAttribute(tc_gemm_kernel<2, FMT>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(TC_SMEM));
     if (e != cudaSuccess) return e;
 
     GemmArgs g;
@@ -805,7 +837,7 @@ cudaError_t launch_ffn_tc(const FfnParams &f, const TcBuffers &b, cudaStream_t s
 
     // 2. gate/up GEMM -> h (float32)
     g.bscale = b.sx;
-    tc_gemm_kernel<1><<<grid, TC_THREADS, TC_SMEM, st>>>(m1, g);
+    tc_gemm_kernel<1, FMT><<<grid, TC_THREADS, TC_SMEM, st>>>(m1, g);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     // 3. h quantisation
@@ -814,13 +846,21 @@ cudaError_t launch_ffn_tc(const FfnParams &f, const TcBuffers &b, cudaStream_t s
     qh.len = f.I;
     qh.q = b.hq;
     qh.scale = b.sh;
-    tc_quant_h_kernel<<<(slots + 7) / 8, 256, 0, st>>>(qh);
+    tc_quant_h_kernel<FMT><<<(slots + 7) / 8, 256, 0, st>>>(qh);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     // 4. down GEMM + weighted combine into out
     g.bscale = b.sh;
-    tc_gemm_kernel<2><<<grid, TC_THREADS, TC_SMEM, st>>>(m2, g);
+    tc_gemm_kernel<2, FMT><<<grid, TC_THREADS, TC_SMEM, st>>>(m2, g);
     return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_ffn_tc(const FfnParams &f, const TcBuffers &b, cudaStream_t st) {
+    if (f.fmt == 8) return launch_tc_fmt<8>(f, b, st);
+    if (f.fmt == 2) return launch_tc_fmt<2>(f, b, st);
+    return launch_tc_fmt<4>(f, b, st);
 }
 
 }  // namespace coli

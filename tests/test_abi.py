@@ -119,10 +119,12 @@ def test_dispatch_rule_on_the_host():
         assert q.coli_moe_layer_kernels(cfg, 0) == 0
         for T in (5, 8, 64, 65, 2048):
             assert q.coli_moe_layer_kernels(cfg, T) == 7, (name, T)
-    for name in ("glm_int8", "glm_int2"):
+    for name in ("glm_int8", "glm_int2"):  # int8 and int2 records take the tensor-core path too
         cfg = q.config_for(synth.WORKLOADS[name])
         for T in (5, 64, 256):
-            assert q.coli_moe_layer_kernels(cfg, T) == 5, (name, T)
+            assert q.coli_moe_layer_kernels(cfg, T) == 7, (name, T)
+    gs = q.config_for(synth.WORKLOADS["glm_gs64"])  # group scales: the GEMV path above 4 tokens
+    assert q.coli_moe_layer_kernels(gs, 64) == 5
     odd = q.config_for(synth.WORKLOADS["tiny"].replace(inter=64, shared_inter=64))
     assert q.coli_moe_layer_kernels(odd, 32) == 5  # inter not a multiple of 128
 

@@ -1,4 +1,5 @@
-"""GPU parity of the tensor-core grouped-GEMM path (batches above 4 tokens, int4 weights).
+"""GPU parity of the tensor-core grouped-GEMM path (batches above 4 tokens; int4, int8 and int2
+weights with per-row scales).
 
 x and h enter the int8 MMAs as 16-bit fixed point per row, so outputs are compared with the
 tensor-core tolerance (TOL_TC, normwise per token); routing and grouping stay bit-exact.  The
@@ -114,6 +115,35 @@ def test_tc_layer_olmoe_all_tokens():
     ref = oracle.ffn(ocfg, L.host_records(ids_ref), x.cpu(), T, ids_ref, w_ref)
     err = normwise_err(out.cpu().numpy(), ref)
     print(f"olmoe layer T={T}: normwise error {err:.2e}")
+    assert err <= TOL_TC, err
+
+
+@pytest.mark.parametrize("fmt", [8, 2])
+def test_tc_layer_int8_int2_all_tokens(fmt):
+    """Every token of a 48-token layer with int8 or int2 records on the tensor-core path: int8
+    codes enter the MMA as they are, int2 codes as 64q, each in the order the activations are
+    written in (tiny_wide's router and expert counts, 512 x 256 experts)."""
+    wl = _EXTRA["tiny_wide"].replace(name=f"tiny_wide_i{fmt}", fmt=fmt)
+    L = Layer(wl, "cuda", 0)
+    T = 48
+    cfg = q.config_for(wl)
+    assert q.coli_moe_layer_kernels(cfg, T) == TC_KERNELS
+    x = synth.make_activations(wl, T, device="cuda", step=9)
+    out = torch.empty(T, wl.hidden, dtype=torch.float32, device="cuda")
+    ids = torch.empty(T, wl.top_k, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, wl.top_k, dtype=torch.float32, device="cuda")
+    ws = torch.empty(q.coli_moe_workspace_size(cfg, T), dtype=torch.uint8, device="cuda")
+    q.coli_moe_clear_error(ws)
+    q.coli_moe_layer(cfg, L.weights(), x, T, out, ids, w, ws)
+    assert q.coli_moe_error_word(ws) == 0
+    ocfg = oracle.make_cfg(wl)
+    lg = oracle_gate(ocfg, L.Wr.cpu(), x.cpu(), T)
+    ids_ref, w_ref = oracle.route(ocfg, lg, L.bias.cpu(), T)
+    np.testing.assert_array_equal(ids.cpu().numpy(), ids_ref)
+    np.testing.assert_array_equal(w.cpu().numpy(), w_ref)
+    ref = oracle.ffn(ocfg, L.host_records(ids_ref), x.cpu(), T, ids_ref, w_ref)
+    err = normwise_err(out.cpu().numpy(), ref)
+    print(f"int{fmt} layer T={T}: normwise error {err:.2e}")
     assert err <= TOL_TC, err
 
 
