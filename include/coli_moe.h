@@ -179,6 +179,15 @@ coli_status coli_moe_layer(const coli_moe_config *cfg, const coli_moe_weights *w
 coli_status coli_moe_residual(const coli_moe_config *cfg, const void *x, const float *out, int T,
                               void *x_next, void *stream);
 
+/* a5' per-expert dispatch on the grouped tensor-core path (batches above 4 tokens): within a call,
+ * work experts with at most max_tokens routed tokens are computed by the CUDA-core GEMV kernels
+ * (streaming their codes once at HBM speed) and the others by the grouped GEMM; the GEMV kernels'
+ * down projection adds into out alongside the GEMM's combine.  0 puts every expert on the tensor
+ * cores.  Process-wide, read at each call; coli_moe_layer_kernels then reports 9 kernels on that
+ * path instead of 7.  Host only; COLI_ERR_INVALID_ARG outside [0, 65536]. */
+coli_status coli_moe_set_dispatch_threshold(int max_tokens);
+int coli_moe_dispatch_threshold(void);
+
 /* Testing aid for the bounded device-side waits of the fused decode kernel (the one-launch
  * path that coli_moe_layer_kernels reports as 1 kernel).  wait_cycles > 0 replaces the default
  * bound (about 2 s of SM clock) of every wait in that kernel's later launches made by the

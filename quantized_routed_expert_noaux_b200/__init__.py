@@ -19,6 +19,8 @@ __all__ = [
     "coli_moe_gate", "coli_moe_route", "coli_moe_group", "coli_moe_ffn", "coli_moe_layer",
     "coli_moe_layer_noalloc", "STATIC_SCRATCH_BYTES", "coli_moe_layer_kernels", "coli_moe_residual",
     "coli_moe_debug_set_wait",
+    "coli_moe_set_dispatch_threshold",
+    "coli_moe_dispatch_threshold",
     "config_for", "weights_for",
     "COLI_W_INT2", "COLI_W_INT4", "COLI_W_INT8", "COLI_ACT_F32", "COLI_ACT_BF16",
 ]
@@ -82,12 +84,15 @@ def _load():
     L.coli_moe_layer_kernels.argtypes = [cfgp, I, C.POINTER(I)]
     L.coli_moe_residual.argtypes = [cfgp, P, P, I, P, P]
     L.coli_moe_debug_set_wait.argtypes = [C.c_longlong, I]
+    L.coli_moe_set_dispatch_threshold.argtypes = [I]
+    L.coli_moe_dispatch_threshold.argtypes = []
+    L.coli_moe_dispatch_threshold.restype = I
     L.coli_moe_layer_kernels.restype = I
     L.coli_moe_layer_noalloc.restype = I
     for name in ("coli_moe_record_bytes", "coli_moe_check_config", "coli_moe_workspace_size",
                  "coli_moe_clear_error", "coli_moe_error_word", "coli_moe_gate",
                  "coli_moe_route", "coli_moe_group", "coli_moe_ffn", "coli_moe_layer",
-                 "coli_moe_residual", "coli_moe_debug_set_wait"):
+                 "coli_moe_residual", "coli_moe_debug_set_wait", "coli_moe_set_dispatch_threshold"):
         getattr(L, name).restype = I
     return L
 
@@ -216,6 +221,17 @@ def coli_moe_debug_set_wait(wait_cycles: int, unreachable: bool) -> None:
     """Testing aid: the fused decode kernel's wait bound (cycles, 0 = default) and whether its
     grid-barrier targets are out of reach (every wait then runs out and reports a timeout)."""
     _check("coli_moe_debug_set_wait", lib.coli_moe_debug_set_wait(wait_cycles, int(bool(unreachable))))
+
+
+def coli_moe_set_dispatch_threshold(max_tokens: int) -> None:
+    """a5' per-expert dispatch on the tensor-core path: work experts with at most max_tokens
+    routed tokens take the CUDA-core GEMV kernels, the rest the grouped GEMM (0: all GEMM)."""
+    _check("coli_moe_set_dispatch_threshold", lib.coli_moe_set_dispatch_threshold(int(max_tokens)))
+
+
+def coli_moe_dispatch_threshold() -> int:
+    """The current per-expert dispatch threshold."""
+    return int(lib.coli_moe_dispatch_threshold())
 
 
 def config_for(wl) -> MoEConfig:

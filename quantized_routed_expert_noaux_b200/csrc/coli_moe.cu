@@ -1,5 +1,6 @@
 // coli_moe.cu -- the C ABI of libcoli_moe.so: argument validation, workspace carve-up, and the
 // launch sequence of the layer.  No device memory is allocated here; no CPU fallback exists.
+#include <atomic>
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <stdio.h>
@@ -24,6 +25,9 @@ thread_local char g_last_cuda_error[256] = "";
 // makes its grid-barrier targets unreachable
 thread_local long long g_wait_cycles = 0;
 thread_local int g_unreachable = 0;
+// a5' per-expert dispatch on the grouped-GEMM path: work experts with at most this many tokens
+// take the GEMV kernels (coli_moe_set_dispatch_threshold; 0 = every expert on the tensor cores)
+std::atomic<int> g_dispatch{DISPATCH_DEFAULT};
 
 coli_status from_cuda(cudaError_t e) {
     if (e == cudaSuccess) return COLI_OK;
@@ -121,6 +125,14 @@ const char *coli_moe_status_str(coli_status s) {
 
 const char *coli_moe_last_cuda_error(void) { return g_last_cuda_error; }
 
+coli_status coli_moe_set_dispatch_threshold(int max_tokens) {
+    if (max_tokens < 0 || max_tokens > 65536) return COLI_ERR_INVALID_ARG;
+    g_dispatch.store(max_tokens);
+    return COLI_OK;
+}
+
+int coli_moe_dispatch_threshold(void) { return g_dispatch.load(); }
+
 coli_status coli_moe_debug_set_wait(long long wait_cycles, int unreachable) {
     if (wait_cycles < 0) return COLI_ERR_INVALID_ARG;
     g_wait_cycles = wait_cycles;
@@ -198,7 +210,7 @@ coli_status coli_moe_layer_kernels(const coli_moe_config *c, int T, int *n_kerne
     if (s != COLI_OK) return s;
     if (T < 0) return COLI_ERR_SHAPE;
     DecodePlan pl;
-    *n_kernels = T == 0 ? 0 : (decode_plan(*c, T, &pl) ? 1 : (use_tc(c, T) ? 7 : 5));
+    *n_kernels = T == 0 ? 0 : (decode_plan(*c, T, &pl) ? 1 : (use_tc(c, T) ? (g_dispatch.load() > 0 ? 9 : 7) : 5));
     return COLI_OK;
 }
 
@@ -285,6 +297,7 @@ static FfnParams make_params(const coli_moe_config *c, const coli_moe_weights *w
     p.off_sd = p.off_su + static_cast<size_t>(c->inter) * p.nsh * 4;
     p.x = x; p.topk_w = topk_w; p.offsets = offsets; p.perm = perm; p.unique = unique;
     p.n_unique = n_unique; p.h = h; p.out = out; p.err = err;
+    p.gemv_nmax = 0x7fffffff; p.tc_nmin = 0; p.gemv_atomic = 0;  // one path takes every expert
     return p;
 }
 
@@ -320,7 +333,12 @@ static coli_status run_ffn(const coli_moe_config *c, const FfnParams &p, char *b
         b.chunks = reinterpret_cast<int4 *>(base + L.chunks);
         b.n_chunks = reinterpret_cast<int *>(base + L.n_chunks);
         b.max_chunks = tc_max_chunks(*c, p.T);
-        return from_cuda(launch_ffn_tc(p, b, st));
+        FfnParams q = p;  // per-expert dispatch between the GEMV kernels and the grouped GEMM
+        const int n = g_dispatch.load();
+        q.gemv_nmax = n;
+        q.tc_nmin = n;
+        q.gemv_atomic = 1;
+        return from_cuda(launch_ffn_tc(q, b, st));
     }
     DecodePlan pl;
     if (decode_plan(*c, p.T, &pl)) return from_cuda(launch_ffn_decode(make_decode(c, p, base), pl, st));

@@ -210,6 +210,7 @@ __global__ void __launch_bounds__(GU_THREADS) gateup_kernel(FfnParams p, int L, 
                                               ? COLI_DEVERR_EXPERT_ID : COLI_DEVERR_GROUPING);
             continue;
         }
+        if (ex.count > p.gemv_nmax) continue;  // the grouped GEMM's expert
         const uint8_t *wg = ex.rec;
         const uint8_t *wu = ex.rec + p.off_wu;
         const float *sg = reinterpret_cast<const float *>(ex.rec + p.off_sg);
@@ -296,8 +297,9 @@ __global__ void __launch_bounds__(DN_THREADS) down_kernel(FfnParams p, int L, in
     extern __shared__ float dsm[];
     const int rpp = P * R;
     const int nwarp_row = L > 32 ? L / 32 : 1;
-    float *acc = dsm;                                   // [T][rpp]
-    float *red = dsm + static_cast<size_t>(p.T) * rpp;  // [P][R][L/32]
+    const int TA = p.gemv_atomic ? 0 : p.T;             // tokens with accumulators here
+    float *acc = dsm;                                   // [TA][rpp]
+    float *red = dsm + static_cast<size_t>(TA) * rpp;   // [P][R][L/32]
     const int tid = threadIdx.x;
     const int c = tid % L, slot = tid / L;
     const bool active = slot < P;
@@ -309,11 +311,11 @@ __global__ void __launch_bounds__(DN_THREADS) down_kernel(FfnParams p, int L, in
 
     for (int pass = beg; pass < end; ++pass) {
         const int j0 = pass * rpp;
-        for (int i = tid; i < p.T * rpp; i += blockDim.x) acc[i] = 0.f;
+        for (int i = tid; i < TA * rpp; i += blockDim.x) acc[i] = 0.f;
         __syncthreads();
         for (int we = 0; we < nwe; ++we) {
             const ExpertRef ex = expert_ref(p, we, U);
-            if (!ex.ok) continue;  // flagged by the gate/up kernel
+            if (!ex.ok || ex.count > p.gemv_nmax) continue;  // flagged by the gate/up kernel; or the GEMM's
             const uint8_t *wd = ex.rec + p.off_wd;
             const float *sd = reinterpret_cast<const float *>(ex.rec + p.off_sd);
             uint4 qd[R];
@@ -358,13 +360,16 @@ __global__ void __launch_bounds__(DN_THREADS) down_kernel(FfnParams p, int L, in
 #pragma unroll
                     for (int r = 0; r < R; ++r) {
                         const int j = j0 + slot * R + r;
-                        if (j < p.H) acc[tok * rpp + slot * R + r] += wt * ((p.group ? 1.0f : sd[j]) * a[r]);
+                        if (j >= p.H) continue;
+                        const float v = wt * ((p.group ? 1.0f : sd[j]) * a[r]);
+                        if (p.gemv_atomic) atomicAdd(p.out + static_cast<size_t>(tok) * p.H + j, v);
+                        else acc[tok * rpp + slot * R + r] += v;
                     }
                 }
             }
             __syncthreads();
         }
-        for (int i = tid; i < p.T * rpp; i += blockDim.x) {
+        for (int i = tid; i < TA * rpp; i += blockDim.x) {
             const int t = i / rpp, rr = i % rpp, j = j0 + rr;
             if (j < p.H) p.out[static_cast<size_t>(t) * p.H + j] = acc[i];
         }
@@ -373,11 +378,11 @@ __global__ void __launch_bounds__(DN_THREADS) down_kernel(FfnParams p, int L, in
 }
 
 template <int FMT, int ACT>
-cudaError_t launch_fmt(const FfnParams &p, cudaStream_t st) {
+cudaError_t launch_fmt(const FfnParams &p, cudaStream_t st, bool gateup, bool down) {
     constexpr int R_GU = 4, R_DN = 4;
     const int sms = device_sm_count();
     // gate/up
-    {
+    if (gateup) {
         const int L = static_cast<int>(p.rb_h / 16);
         const int P = GU_THREADS / L > 0 ? GU_THREADS / L : 1;
         const int threads = ((L * P + 31) / 32) * 32;
@@ -388,12 +393,12 @@ cudaError_t launch_fmt(const FfnParams &p, cudaStream_t st) {
         if (e != cudaSuccess) return e;
     }
     // down + combine
-    {
+    if (down) {
         const int L = static_cast<int>(p.rb_i / 16);
         const int P = DN_THREADS / L > 0 ? DN_THREADS / L : 1;
         const int threads = ((L * P + 31) / 32) * 32;
         const int rpp = P * R_DN;
-        const size_t smem = (static_cast<size_t>(p.T) * rpp +
+        const size_t smem = (static_cast<size_t>(p.gemv_atomic ? 0 : p.T) * rpp +
                              (L > 32 ? static_cast<size_t>(P) * R_DN * (L / 32) : 0)) * sizeof(float);
         if (smem > 48 * 1024) {
             cudaError_t e = cudaFuncSetAttribute(down_kernel<FMT, R_DN>,
@@ -425,17 +430,21 @@ int gemv_max_tokens(const coli_moe_config &) {
     return 256;
 }
 
-cudaError_t launch_ffn_gemv(const FfnParams &p, cudaStream_t st) {
+static cudaError_t launch_parts(const FfnParams &p, cudaStream_t st, bool gateup, bool down) {
     if (p.act == COLI_ACT_F32) {
-        if (p.fmt == 4) return launch_fmt<4, COLI_ACT_F32>(p, st);
-        if (p.fmt == 8) return launch_fmt<8, COLI_ACT_F32>(p, st);
-        if (p.fmt == 2) return launch_fmt<2, COLI_ACT_F32>(p, st);
+        if (p.fmt == 4) return launch_fmt<4, COLI_ACT_F32>(p, st, gateup, down);
+        if (p.fmt == 8) return launch_fmt<8, COLI_ACT_F32>(p, st, gateup, down);
+        if (p.fmt == 2) return launch_fmt<2, COLI_ACT_F32>(p, st, gateup, down);
     } else {
-        if (p.fmt == 4) return launch_fmt<4, COLI_ACT_BF16>(p, st);
-        if (p.fmt == 8) return launch_fmt<8, COLI_ACT_BF16>(p, st);
-        if (p.fmt == 2) return launch_fmt<2, COLI_ACT_BF16>(p, st);
+        if (p.fmt == 4) return launch_fmt<4, COLI_ACT_BF16>(p, st, gateup, down);
+        if (p.fmt == 8) return launch_fmt<8, COLI_ACT_BF16>(p, st, gateup, down);
+        if (p.fmt == 2) return launch_fmt<2, COLI_ACT_BF16>(p, st, gateup, down);
     }
     return cudaErrorInvalidValue;
 }
+
+cudaError_t launch_ffn_gemv(const FfnParams &p, cudaStream_t st) { return launch_parts(p, st, true, true); }
+cudaError_t launch_ffn_gemv_gateup(const FfnParams &p, cudaStream_t st) { return launch_parts(p, st, true, false); }
+cudaError_t launch_ffn_gemv_down(const FfnParams &p, cudaStream_t st) { return launch_parts(p, st, false, true); }
 
 }  // namespace coli

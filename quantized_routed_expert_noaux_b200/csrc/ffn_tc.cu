@@ -365,7 +365,8 @@ __device__ void build_chunks(const FfnParams &f, int4 *chunks, int *n_chunks, in
             pos0 = TK;
             cnt = f.T;
         }
-        const int nc = (cnt + MAXTOK - 1) / MAXTOK;
+        // per-expert dispatch: experts with at most tc_nmin tokens are the GEMV kernels'
+        const int nc = cnt > f.tc_nmin ? (cnt + MAXTOK - 1) / MAXTOK : 0;
         s_scan[tid] = nc;
         __syncthreads();
         for (int o = 1; o < 256; o <<= 1) {  // inclusive Hillis-Steele scan
@@ -835,10 +836,11 @@ cudaError_t launch_tc_fmt(const FfnParams &f, const TcBuffers &b, cudaStream_t s
     g.hbuf = b.hbuf;
     const int grid = device_sm_count();
 
-    // 2. gate/up GEMM -> h (float32)
+    // 2. gate/up GEMM -> h (float32); the small experts' h by the GEMV kernel
     g.bscale = b.sx;
     tc_gemm_kernel<1, FMT><<<grid, TC_THREADS, TC_SMEM, st>>>(m1, g);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (f.gemv_nmax > 0 && (e = launch_ffn_gemv_gateup(f, st)) != cudaSuccess) return e;
 
     // 3. h quantisation
     QuantArgs qh = pa.qa;
@@ -849,7 +851,9 @@ cudaError_t launch_tc_fmt(const FfnParams &f, const TcBuffers &b, cudaStream_t s
     tc_quant_h_kernel<FMT><<<(slots + 7) / 8, 256, 0, st>>>(qh);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
-    // 4. down GEMM + weighted combine into out
+    // 4. the small experts' down projections (atomic adds into out, zeroed by the prep kernel),
+    //    then the down GEMM + weighted combine into out
+    if (f.gemv_nmax > 0 && (e = launch_ffn_gemv_down(f, st)) != cudaSuccess) return e;
     g.bscale = b.sh;
     tc_gemm_kernel<2, FMT><<<grid, TC_THREADS, TC_SMEM, st>>>(m2, g);
     return cudaGetLastError();

@@ -31,6 +31,10 @@ struct FfnParams {
     float *h;                          // [(T*K + T*S)][I] f32 intermediate (GEMV path)
     float *out;                        // [T][H]
     int *err;                          // device error word
+    // per-expert dispatch (a5'): the GEMV kernels take the work experts with at most gemv_nmax
+    // tokens, the grouped GEMM those with more than tc_nmin; gemv_atomic: the GEMV down kernel
+    // adds into out (zeroed before) instead of writing it
+    int gemv_nmax, tc_nmin, gemv_atomic;
 };
 
 // Workspace header (first 512 bytes): error word; then the fused decode path's phase word and
@@ -79,6 +83,9 @@ struct DecodeParams {
 };
 
 bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan);
+// the GEMV kernels one at a time (the grouped-GEMM path runs them for its small experts)
+cudaError_t launch_ffn_gemv_gateup(const FfnParams &p, cudaStream_t st);
+cudaError_t launch_ffn_gemv_down(const FfnParams &p, cudaStream_t st);
 cudaError_t launch_ffn_decode(DecodeParams p, const DecodePlan &pl, cudaStream_t st);
 
 // Buffers of the tensor-core grouped-GEMM path (ffn_tc.cu), carved from the workspace.
@@ -102,6 +109,13 @@ cudaError_t launch_ffn_tc(const FfnParams &f, const TcBuffers &b, cudaStream_t s
 // on B200: from 8 tokens up it beats the CUDA-core GEMV path 3-13x on GLM- and OLMoE-shaped
 // layers; up to 4 tokens the fused decode kernel runs).
 constexpr int TC_MIN_TOKENS = 4;
+// Default of the per-expert dispatch threshold on that path (work experts with at most this many
+// tokens take the GEMV kernels), chosen by measurement on B200: on the 2048-token Zipf layer
+// (194 unique experts, 23 of them with one token) thresholds 0/1/2/4/8/16 took 2.06/2.51/2.80/
+// 3.46/4.67/8.80 ms; on the 512-token 64-expert Zipf layer 0.58/0.66/0.69/0.78/1.06/2.01 ms.
+// A one-token expert costs about as much on the tensor cores as streaming its codes through the
+// GEMV kernels, which also walk the whole expert list: every expert stays on the tensor cores.
+constexpr int DISPATCH_DEFAULT = 0;
 
 // Workspace carve-up (all offsets 256-B aligned).
 struct WsLayout {

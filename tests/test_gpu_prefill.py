@@ -72,7 +72,7 @@ def test_tc_ffn_matches_oracle(name, T, routing):
     L = layer(name)
     wl = L.wl
     cfg = q.config_for(wl)
-    assert q.coli_moe_layer_kernels(cfg, T) == TC_KERNELS
+    assert q.coli_moe_layer_kernels(cfg, T) == TC_KERNELS + (2 if q.coli_moe_dispatch_threshold() else 0)
     ocfg = oracle.make_cfg(wl)
     x = synth.make_activations(wl, T, device="cuda", step=30 + T)
     ids_np, w_np = _routing(L, ocfg, x, T, routing)
@@ -115,6 +115,42 @@ def test_tc_layer_olmoe_all_tokens():
     ref = oracle.ffn(ocfg, L.host_records(ids_ref), x.cpu(), T, ids_ref, w_ref)
     err = normwise_err(out.cpu().numpy(), ref)
     print(f"olmoe layer T={T}: normwise error {err:.2e}")
+    assert err <= TOL_TC, err
+
+
+@pytest.mark.parametrize("name,T,all_tokens", [("olmoe", 20, True), ("glm_decode", 40, False)])
+def test_tc_ffn_per_expert_dispatch(name, T, all_tokens):
+    """a5' per-expert dispatch: with the threshold at 3, the experts with 1..3 tokens take the
+    GEMV kernels and the rest (one expert on every token, the shared expert, the 4+-token ones)
+    the grouped GEMM, in one call; both add into the same out."""
+    L = layer(name)
+    wl = L.wl
+    cfg = q.config_for(wl)
+    ocfg = oracle.make_cfg(wl)
+    x = synth.make_activations(wl, T, device="cuda", step=50 + T)
+    ids_np, w_np = _routing(L, ocfg, x, T, "one_expert")
+    counts = np.bincount(ids_np.ravel(), minlength=wl.n_experts)
+    assert counts.max() == T and ((counts >= 1) & (counts <= 3)).sum() >= 10  # mixed sizes
+    old = q.coli_moe_dispatch_threshold()
+    q.coli_moe_set_dispatch_threshold(3)
+    try:
+        assert q.coli_moe_layer_kernels(cfg, T) == TC_KERNELS + 2
+        ws = torch.empty(q.coli_moe_workspace_size(cfg, T), dtype=torch.uint8, device="cuda")
+        q.coli_moe_clear_error(ws)
+        offsets, perm, uniq, nu = _group_gpu(cfg, torch.from_numpy(ids_np).cuda(), T, wl.n_experts, ws)
+        out = torch.full((T, wl.hidden), float("nan"), device="cuda")
+        q.coli_moe_ffn(cfg, L.weights(), x, T, torch.from_numpy(w_np).cuda(), offsets, perm, uniq,
+                       nu, out, ws)
+        assert q.coli_moe_error_word(ws) == 0
+    finally:
+        q.coli_moe_set_dispatch_threshold(old)
+    got = out.cpu().numpy()
+    assert np.isfinite(got).all()
+    toks = list(range(T)) if all_tokens else sorted(set([0, 1, T // 3, T // 2, T - 2, T - 1]))
+    ref = oracle.ffn(ocfg, L.host_records(ids_np[toks]), x.cpu()[toks], len(toks), ids_np[toks],
+                     w_np[toks])
+    err = normwise_err(got[toks], ref)
+    print(f"{name} T={T} mixed dispatch: normwise error {err:.2e}")
     assert err <= TOL_TC, err
 
 
