@@ -118,6 +118,10 @@ __device__ __forceinline__ void cons_sync() { named_sync(BAR_CONS, NC); }
 __device__ __forceinline__ void red_release_add(unsigned *p, unsigned v) {
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
+// orders this thread's generic-proxy global accesses with async-proxy ones (bulk copies)
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
 __device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
     unsigned v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -462,6 +466,7 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
             while (ld_acquire(ready + we) < static_cast<unsigned>(nch)) {
                 if (clock64() - t0 > bound) { ok = false; break; }
             }
+            fence_proxy_async_global();  // the converters' generic stores, before the bulk copy
             return ok;
         };
         bool published = false;
@@ -899,6 +904,7 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
             if (MAXT > 3) sv.w = scl[MAXT > 3 ? 3 : 0];
             __stcg(reinterpret_cast<float4 *>(dst + n16), sv);
         }
+        fence_proxy_async_global();  // the block is read by the producers' bulk copies
         __syncwarp();  // every lane's stores precede lane 0's release; the block may be reused
         if (lane == 0) red_release_add(ready + we, 1u);  // one more chunk of we converted
     };
