@@ -17,23 +17,26 @@
 // The approximations are the two 16-bit roundings (x, h; 2^-16 of the row maximum) and float32
 // epilogue arithmetic.
 //
-// One persistent CTA per SM, warp-specialised, tiles (chunk of <= 96 tokens of one expert x one
-// block of weight rows) taken round-robin:
-//   warp 12     A producer: per k-block of 128, the packed A tile (128 rows x 64 B, 64-byte
+// Two persistent CTAs per SM, warp-specialised, tiles (chunk of <= 96 tokens of one expert x one
+// block of weight rows) taken round-robin over all CTAs:
+//   warp 8      A producer: per k-block of 128, the packed A tile (128 rows x 64 B, 64-byte
 //               swizzle; one 4-D box holds the gate and the up rows) into the A ring, whose stages
 //               the converters release as soon as they have read them.
-//   warp 14     B producer: the k-block's B rows (boxes of 128/64/32/16 rows of 128 B, 128-byte
+//   warp 10     B producer: the k-block's B rows (boxes of 128/64/32/16 rows of 128 B, 128-byte
 //               swizzle) into the B ring, released by the MMAs' completion; one lane per box.
 //   warps 0-3   converters: one thread per weight row unpacks its 64 bytes into 128 signed bytes
 //               and stores them with tcgen05.st into a TMEM A stage; the MMA reads A from tensor
 //               memory, so unpacked weights never pass through shared memory.
-//   warp 13     MMA issuer (one elected lane, operands computed warp-uniformly): 4 x tcgen05.mma
-//               (K = 32, N <= 192) per k-block into one of two TMEM accumulators, so a tile's
-//               epilogue overlaps the next tile's main loop.
-//   warps 4-11  epilogue: tcgen05.ld of the accumulator and the output arithmetic; the tile's
+//   warp 9      MMA issuer (one elected lane, operands computed warp-uniformly): 4 x tcgen05.mma
+//               (K = 32, N <= 192) per k-block into the CTA's TMEM accumulator.
+//   warps 4-7   epilogue: tcgen05.ld of the accumulator and the output arithmetic; the tile's
 //               per-token scales, tokens and weights are staged in shared memory first.
-// TMEM (512 columns): accumulator b at columns [256b, 256b + 192); the four 32-column A stages
-// fill the gaps [192, 256) and [448, 512).
+// TMEM (256 columns per CTA, half of the SM's): the accumulator at columns [0, 192), two 32-column
+// A stages at [192, 256).  One accumulator per CTA: while a CTA's epilogue drains it, the SM's
+// other CTA keeps the tensor pipe busy (measured on B200 against one CTA per SM with two
+// accumulators, eight epilogue warps and deeper rings: 4% faster on the 2048-token Zipf layer
+// and on the full-chunk 32-expert layer; the per-k-block cost of one CTA is latency that rings,
+// MMA sizes and copy sizes did not move).
 // Inside every group of 8 k the order is permuted to (0,2,4,6,1,3,5,7) on both operands: the
 // unpacking yields the even and the odd codes of a word as separate words, and the activation
 // bytes are written in the same order, so every dot product is unchanged.
@@ -55,24 +58,24 @@ constexpr int KB = 128;                       // k per ring stage
 // 2.20 ms per step, the extra tiles costing more than the deeper A pipeline saves.)
 constexpr int MAXTOK = 96;
 constexpr int NA_MAX = 8;                     // A ring stages (at most; per container below)
-constexpr int NB = 6;                         // B ring stages
+constexpr int NB = 3;                         // B ring stages
 constexpr int B_MAX = 2 * MAXTOK * KB;        // B rows of one stage: 24 KB
 constexpr int NBOX = 4;                       // B box heights 16 << i rows
-constexpr int W_CONV = 4, W_EPI0 = 4, N_EPI = 8, W_PRODA = 12, W_MMA = 13, W_PRODB = 14;
-constexpr int TC_THREADS = 15 * 32;
-constexpr uint32_t D_STRIDE = 256;            // accumulator b at TMEM column 256 * b
+constexpr int W_CONV = 4, W_EPI0 = 4, N_EPI = 4, W_PRODA = 8, W_MMA = 9, W_PRODB = 10;
+constexpr int TC_THREADS = 11 * 32;
+constexpr int CTAS_PER_SM = 2;
+constexpr uint32_t TMEM_COLS = 256;           // per CTA
 constexpr uint32_t A_COL0 = 2 * MAXTOK;       // TMEM column of A stage 0
-constexpr int SPG = (256 - 2 * MAXTOK) / 32;  // 32-column A stages in the gap after each accumulator
-constexpr int NTS = 2 * SPG;                  // TMEM A stages
-static_assert(SPG >= 1, "no room for TMEM A stages");
-constexpr uint32_t TMEM_COLS = 512;
+constexpr int NTS = (TMEM_COLS - 2 * MAXTOK) / 32;  // 32-column TMEM A stages after the accumulator
+static_assert(NTS >= 2, "no room for TMEM A stages");
+static_assert(W_EPI0 % 4 == 0 && N_EPI == 4 && N_EPI * 32 >= MAXTOK, "epilogue warp q reaches TMEM lanes 32q..32q+31");
 constexpr long long WAIT_CYCLES = 4000000000LL;  // ~2 s at 1.9 GHz: bound of every wait
 constexpr float QMAX = 32512.0f;              // |X| <= 32512 keeps Xh = (X + 128) >> 8 in [-127, 127]
-// Weight containers: bytes of one row's k-block (RB), A ring stages, the code's multiplier (the
-// signed byte the MMA sees is MUL * q: int4 16q, int2 64q, int8 q).
+// Weight containers: bytes of one row's k-block (RB), A ring stages (32 KB of A per CTA), the
+// code's multiplier (the signed byte the MMA sees is MUL * q: int4 16q, int2 64q, int8 q).
 template <int FMT> struct TcFmt;
-template <> struct TcFmt<4> { static constexpr int RB = KB / 2, NA = 8; static constexpr float MUL = 16.0f; };
-template <> struct TcFmt<8> { static constexpr int RB = KB, NA = 4; static constexpr float MUL = 1.0f; };
+template <> struct TcFmt<4> { static constexpr int RB = KB / 2, NA = 4; static constexpr float MUL = 16.0f; };
+template <> struct TcFmt<8> { static constexpr int RB = KB, NA = 2; static constexpr float MUL = 1.0f; };
 template <> struct TcFmt<2> { static constexpr int RB = KB / 4, NA = 8; static constexpr float MUL = 64.0f; };
 template <int FMT>
 constexpr size_t tc_smem() {
@@ -213,9 +216,7 @@ __device__ __forceinline__ bool epi_sync_or(bool pred) {
 
 __device__ __forceinline__ int round16(int v) { return (v + 15) & ~15; }
 // TMEM column of A stage j: the gaps [2 * MAXTOK, 256) and [256 + 2 * MAXTOK, 512).
-__device__ __forceinline__ uint32_t a_col(int j) {
-    return static_cast<uint32_t>(j / SPG) * D_STRIDE + A_COL0 + 32u * static_cast<uint32_t>(j % SPG);
-}
+__device__ __forceinline__ uint32_t a_col(int j) { return A_COL0 + 32u * static_cast<uint32_t>(j); }
 __device__ __forceinline__ bool elect_one() {
     uint32_t pred = 0;
     asm volatile("{ .reg .pred P; elect.sync _|P, 0xffffffff; selp.b32 %0, 1, 0, P; }" : "=r"(pred));
@@ -439,21 +440,21 @@ struct TcMaps {
 //          h = SiLU(g) * u into hbuf (float32).
 // PHASE 2: down.  A = 128 rows of Wd, B = quantised h; epilogue out[token] += w * y.
 template <int PHASE, int FMT>
-__global__ void __launch_bounds__(TC_THREADS, 1)
+__global__ void __launch_bounds__(TC_THREADS, CTAS_PER_SM)
 tc_gemm_kernel(const __grid_constant__ TcMaps maps, const GemmArgs p) {
     constexpr int NA = TcFmt<FMT>::NA, RB = TcFmt<FMT>::RB;
     constexpr int A_RAW = 128 * RB;  // A tile of one k-block: 128 rows of RB bytes
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    __shared__ __align__(8) uint64_t bars[2 * NA_MAX + 2 * NB + 2 * NTS + 5];
+    __shared__ __align__(8) uint64_t bars[2 * NA_MAX + 2 * NB + 2 * NTS + 3];
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
     __shared__ float s_bs[2][MAXTOK], s_w[2][MAXTOK];
     __shared__ int s_tk[2][MAXTOK];
     uint64_t *afull = bars, *aempty = afull + NA, *bfull = aempty + NA, *bempty = bfull + NB;
     uint64_t *tfull = bempty + NB, *tempty = tfull + NTS;
-    uint64_t *dfull = tempty + NTS, *dempty = dfull + 2, *drain = dempty + 2;
+    uint64_t *dfull = tempty + NTS, *dempty = dfull + 1, *drain = dempty + 1;
     volatile int *abort = &s_abort;
 
     const FfnParams &f = p.f;
@@ -479,10 +480,8 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const GemmArgs p) {
             mbar_init(smem_u32(&tfull[i]), W_CONV * 32);
             mbar_init(smem_u32(&tempty[i]), 1);
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(smem_u32(&dfull[i]), 1);
-            mbar_init(smem_u32(&dempty[i]), N_EPI * 32);
-        }
+        mbar_init(smem_u32(dfull), 1);
+        mbar_init(smem_u32(dempty), N_EPI * 32);
         mbar_init(smem_u32(drain), 1);
         s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -543,11 +542,10 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const GemmArgs p) {
             const int4 c = p.chunks[t / MB];
             const int nrows = round16(2 * c.z);
             const uint32_t idesc = IDESC_I8 | (static_cast<uint32_t>(nrows >> 3) << 17);
-            const int db = tl & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&dempty[db]), ((tl >> 1) & 1) ^ 1, abort, f.err)))
+            if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(dempty), (tl & 1) ^ 1, abort, f.err)))
                 goto mma_done;
             tc_fence_after();
-            const uint32_t dt = tbase + db * D_STRIDE;
+            const uint32_t dt = tbase;
             for (int kb = 0; kb < KT; ++kb, ++it) {
                 const int s = it % NB, ts = it % NTS;
                 if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&bfull[s]), (it / NB) & 1, abort, f.err)))
@@ -566,7 +564,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const GemmArgs p) {
                 }
                 __syncwarp();
             }
-            if (elect_one()) mma_commit(smem_u32(&dfull[db]));
+            if (elect_one()) mma_commit(smem_u32(dfull));
             __syncwarp();
         }
     mma_done:
@@ -620,8 +618,8 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const GemmArgs p) {
     conv_done:;
     } else {
         // ------------------------------------------------------------------ epilogue
-        const int q = (warp - W_EPI0) & 3, half = (warp - W_EPI0) >> 2;
-        const int et = threadIdx.x - W_EPI0 * 32;  // 0 .. 255
+        const int q = warp - W_EPI0;  // TMEM lane quarter (warp % 4)
+        const int et = threadIdx.x - W_EPI0 * 32;  // 0 .. 127 (>= MAXTOK)
         uint32_t tl = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++tl) {
             const int4 c = p.chunks[t / MB];
@@ -629,7 +627,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const GemmArgs p) {
             const int n = c.z, pos0 = c.y;
             const int ngrp = (round16(2 * n) + 31) / 32;  // groups of 32 columns = 16 tokens
             const uint8_t *rec = c.x >= 0 ? f.experts + static_cast<size_t>(c.x) * f.stride : f.shared;
-            const int pb = tl & 1, db = tl & 1;
+            const int pb = tl & 1;
             // per-token data of the tile (double-buffered by tile parity; the barrier below also
             // orders every warp's reads of tile tl - 2 before these writes)
             if (et < n) {
@@ -641,15 +639,15 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const GemmArgs p) {
             }
             if (epi_sync_or(*abort != 0)) break;
             // warp-uniform: tcgen05.ld below is a warp-collective instruction
-            if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&dfull[db]), (tl >> 1) & 1, abort, f.err)))
+            if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(dfull), tl & 1, abort, f.err)))
                 continue;  // given up: every epilogue warp leaves at the next barrier
             tc_fence_after();
-            const uint32_t dt = tbase + (static_cast<uint32_t>(32 * q) << 16) + db * D_STRIDE;
+            const uint32_t dt = tbase + (static_cast<uint32_t>(32 * q) << 16);
             if (PHASE == 1) {
                 const bool gate = lane < 16;
                 const int irow = m * 64 + 16 * q + (lane & 15);
                 const float sc = reinterpret_cast<const float *>(rec + (gate ? f.off_sg : f.off_su))[irow];
-                for (int g = half; g < ngrp; g += 2) {
+                for (int g = 0; g < ngrp; ++g) {
                     int v[32];
                     tmem_ld32(dt + 32 * g, v);
                     float d[16];
@@ -673,7 +671,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const GemmArgs p) {
             } else {
                 const int r = m * 128 + 32 * q + lane;
                 const float sd = reinterpret_cast<const float *>(rec + f.off_sd)[r];
-                for (int g = half; g < ngrp; g += 2) {
+                for (int g = 0; g < ngrp; ++g) {
                     int v[32];
                     tmem_ld32(dt + 32 * g, v);
 #pragma unroll
@@ -688,7 +686,7 @@ tc_gemm_kernel(const __grid_constant__ TcMaps maps, const GemmArgs p) {
                 }
             }
             tc_fence_before();
-            mbar_arrive(smem_u32(&dempty[db]));
+            mbar_arrive(smem_u32(dempty));
         }
     }
 
@@ -834,7 +832,7 @@ cudaError_t launch_tc_fmt(const FfnParams &f, const TcBuffers &b, cudaStream_t s
     g.tok_of = b.tok_of;
     g.w_of = b.w_of;
     g.hbuf = b.hbuf;
-    const int grid = device_sm_count();
+    const int grid = CTAS_PER_SM * device_sm_count();
 
     // 2. gate/up GEMM -> h (float32); the small experts' h by the GEMV kernel
     g.bscale = b.sx;
