@@ -9,6 +9,10 @@
 //           The activations become 24-bit fixed point per token row (scale 2^(e-22) with
 //           max|x| < 2^e), exact for every bf16 element within 2^15 of the row's maximum, held
 //           as three signed byte slices in the layout of the tensor-core B operand.
+//  routing  every CTA waits for all logits and routes the batch itself (a2, noaux_tc,
+//           colibri-strix README "What's implemented") and groups it (a3, batch-union): the
+//           same code on the same inputs, so all CTAs agree bit for bit; CTA 0 writes the
+//           routing outputs of the call.  (For coli_moe_ffn the routing arrays are inputs.)
 //  phase 1  (a4, and a6 for the shared expert) gate/up rows stream through a shared-memory ring
 //           (bulk asynchronous copies by the producer warp, mbarrier completion).  A tile is 8
 //           gate rows and the same 8 up rows of one expert; two groups of 8 warps take tiles in
@@ -16,19 +20,24 @@
 //           int32 accumulation over all of K: exact) of the unpacked codes against every
 //           token's three slices.  A group's partial sums meet in shared memory; one warp
 //           forms g and u per (row, token) and writes h = SiLU(g) * u in float32.  The shared
-//           expert's tiles run first; then every CTA waits for all logits and routes the batch
-//           itself (a2, noaux_tc, colibri-strix README "What's implemented") and groups it (a3,
-//           batch-union): the same code on the same inputs, so all CTAs agree bit for bit; CTA
-//           0 writes the routing outputs of the call.  (For coli_moe_ffn the routing arrays
-//           are inputs.)  Routed tiles are dealt over the CTAs as one flat list.
+//           expert's tiles, issued at launch, are multiplied right after routing; the routed
+//           tiles are dealt over the CTAs as one flat list (tile tau to CTA tau mod G).
 //  barrier  bounded grid barrier (every h row complete).
-//  phase 2  (a5, a7) each CTA owns H/G output rows of every expert.  Warp w owns one 64-byte
-//           column chunk of the down rows: it turns its chunk of each slot's h into 24-bit
-//           fixed point per chunk (three byte slices, scale 2^(e-22)), multiplies with the
-//           tensor cores and accumulates w * sd * dot per (row, token) in float registers over
-//           the experts in a fixed order (shared expert first, then the unique ids ascending).
-//           One cross-warp reduction at the end, no atomics: deterministic, and batch-union
-//           output equals per-token output bit for bit.
+//  convert  each 128-element chunk of every work expert's h is converted once (chunk q by CTA
+//           q mod G) into 24-bit fixed point per (chunk, token), three byte slices in the MMA B
+//           layout, written to the workspace; a release-add counts it on the expert's
+//           readiness counter.
+//  phase 2  (a5, a7) each CTA owns H/G output rows of every expert.  A down stage carries the
+//           CTA's block of down rows and, once the producer has seen the expert's readiness
+//           count complete, the expert's converted h (two bulk copies).  Warp w multiplies its
+//           64-byte column chunk of the rows with the chunk's fragments on the tensor cores and
+//           accumulates w * sd * dot per (row, token) in float registers over the experts in a
+//           fixed order (shared expert first, then the unique ids ascending).  One cross-warp
+//           reduction at the end, no atomics: deterministic, and batch-union output equals
+//           per-token output bit for bit.
+//  counters the workspace header holds a phase word and two counter sets; a call uses the set
+//           the phase names, and CTA 0, past the grid barrier, zeroes the other set and flips
+//           the phase, so a completed call leaves the header ready for the next one.
 //
 // Dequantisation (dequant-on-use, same README section): the codes enter the MMA as signed
 // bytes scaled by a power of two (the int4 nibble in the high half of a byte is 16q, an int2
