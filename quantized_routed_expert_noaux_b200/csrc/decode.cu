@@ -825,16 +825,18 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
     const int nch2 = rb_i / 64;
     const int nact = nch2 < NCW ? nch2 : NCW;         // warps with a chunk
     const bool active2 = cw < nch2;
-    unsigned char *hb = sm + p.off_hb + static_cast<size_t>(cw) * NCOL * colblk;  // this warp's h slices
     float acc[RT2][NB][4];                            // down-projection sums (zeroed after the tiles)
     int my_tiles = 0;
 
     // Chunk c (CPC elements) of work expert we's h (all of h is written: after the grid barrier):
-    // per token 24-bit fixed point with one scale (three byte slices), laid out as this warp's
-    // MMA B fragments through its h-slice block in shared memory, then stored lane-major for the
-    // down projections of every CTA.  Lane l holds
-    // elements l * CPL + k; two neighbouring lanes fill each 32-bit B word (one shuffle).
+    // per token 24-bit fixed point with one scale (three byte slices), each 32-bit word stored
+    // straight into the chunk's block in the workspace at its place in the MMA B fragment layout
+    // (no shared-memory staging: the fragment slots, which the producer may fill with other
+    // experts' converted h at any time after the barrier, share the span that staging would
+    // use).  Lane l holds elements l * CPL + k; two neighbouring lanes fill each 32-bit B word
+    // (one shuffle).
     auto convert_chunk = [&](int we, int c) {
+        unsigned char *const gblk = reinterpret_cast<unsigned char *>(p.dsl) + static_cast<size_t>(we * DEC_CH + c) * fch;
         float hv[MAXT][CPL];
 #pragma unroll
         for (int t = 0; t < MAXT; ++t) {
@@ -875,14 +877,14 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
 #pragma unroll
             for (int sidx = 0; sidx < 3; ++sidx) {
                 const int col = 3 * t + sidx;
-                unsigned char *blk = hb + col * colblk;
+                unsigned char *blk = gblk + col * colblk;
                 if (FMT == 4) {
                     // elements 4l + {0, 2} -> bytes 2(l&1) + {0, 1} of half 0; 4l + {1, 3} of half 1
                     const uint32_t h0 = by[sidx][0] | (by[sidx][2] << 8), h1 = by[sidx][1] | (by[sidx][3] << 8);
                     const uint32_t got = __shfl_xor_sync(FULL, odd ? h0 : h1, 1);
                     const uint32_t word = odd ? (got | (h1 << 16)) : (h0 | (got << 16));
                     const int m2 = (lane >> 1) & 3;
-                    *reinterpret_cast<uint32_t *>(blk + b_off<FMT>(col, tg, m2, odd ? 1 : 0, 0)) = word;
+                    __stcg(reinterpret_cast<unsigned int *>(blk + b_off<FMT>(col, tg, m2, odd ? 1 : 0, 0)), word);
                 } else {
                     // elements 8l + kk + {0, 4} -> bytes 2(l&1) + {0, 1} of field kk's register;
                     // the even lane stores fields 0, 1 and the odd lane fields 2, 3
@@ -895,16 +897,14 @@ __global__ void __launch_bounds__(NT, 1) ffn_decode_kernel(DecodeParams p) {
                         const uint32_t got = __shfl_xor_sync(FULL, odd ? hw[e2] : hw[2 + e2], 1);
                         const int kk = odd ? 2 + e2 : e2;
                         const uint32_t word = odd ? (got | (hw[kk] << 16)) : (hw[kk] | (got << 16));
-                        *reinterpret_cast<uint32_t *>(blk + b_off<FMT>(col, tg, 2 * i4 + (kk >> 1), kk & 1, 0)) = word;
+                        __stcg(reinterpret_cast<unsigned int *>(blk + b_off<FMT>(col, tg, 2 * i4 + (kk >> 1), kk & 1, 0)), word);
                     }
                 }
             }
         }
-        __syncwarp();
-        // the block as it is in shared memory, then the tokens' scales (16 bytes)
-        uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<unsigned char *>(p.dsl) + static_cast<size_t>(we * DEC_CH + c) * fch);
+        // then the tokens' scales (16 bytes) after the block
+        uint4 *dst = reinterpret_cast<uint4 *>(gblk);
         const int n16 = NCOL * colblk / 16;
-        for (int i = lane; i < n16; i += 32) __stcg(dst + i, reinterpret_cast<const uint4 *>(hb)[i]);
         if (lane == 0) {
             float4 sv = make_float4(0.f, 0.f, 0.f, 0.f);
             sv.x = scl[0];
@@ -1331,14 +1331,12 @@ bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan) {
     size_t o = 1024;                                  // mbarriers (up to 60 stages)
     pl.off_route = o; o += (sizeof(RouteCache) + 127) / 128 * 128;
     // One span for what lives in turn: the group reduction buffers and the activation slices
-    // (gate/up tiles), the converter's h slices (between the two grid barriers), the down
-    // stages' fragment slots (after them; one per ring stage).  Then the per-token routing
+    // (gate/up tiles), then the down stages' fragment slots (one per ring stage).  Then the per-token routing
     // scratch and the gate partials (until the batch is routed), then the ring; the final
     // cross-warp reduction reuses the ring once every stage is consumed.
     const size_t r1bytes = (static_cast<size_t>(NGRP) * GW * NB * 32 * 16 + 127) / 128 * 128;
     const size_t xbytes = static_cast<size_t>(c.hidden / cpc) * 3 * T * colblk;
-    const size_t hbytes = static_cast<size_t>(NCW) * 3 * T * colblk;
-    const size_t abytes = ((xbytes > hbytes ? xbytes : hbytes) + 127) / 128 * 128;
+    const size_t abytes = (xbytes + 127) / 128 * 128;
     pl.fslot = static_cast<int>((static_cast<size_t>(rb_i / 64) * (3 * T * colblk + 16) + 127) / 128 * 128);
     const size_t tbytes = (static_cast<size_t>(T) * sizeof(RouteToken) + 127) / 128 * 128;
     const size_t gbytes = (static_cast<size_t>(NCW) * 2 * MAXTOK * 8 + NCW * MAXTOK * 4 + 127) / 128 * 128;
@@ -1346,7 +1344,6 @@ bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan) {
     pl.off_red1 = o;
     pl.off_frag = o;
     pl.off_x = o + r1bytes;
-    pl.off_hb = pl.off_x;
     pl.S = 0;
     for (int S = 60; S >= 2; --S) {
         size_t span = r1bytes + abytes;
@@ -1375,7 +1372,7 @@ bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan) {
 static void fill_plan(DecodeParams &p, const DecodePlan &pl) {
     p.grid = pl.grid; p.S = pl.S; p.SB = pl.SB; p.st_sd = pl.st_sd; p.lag = pl.lag; p.fslot = pl.fslot;
     p.off_route = pl.off_route; p.off_rtok = pl.off_rtok; p.off_gate = pl.off_gate; p.off_red1 = pl.off_red1;
-    p.off_x = pl.off_x; p.off_hb = pl.off_hb; p.off_frag = pl.off_frag; p.off_ring = pl.off_ring;
+    p.off_x = pl.off_x; p.off_frag = pl.off_frag; p.off_ring = pl.off_ring;
 }
 
 cudaError_t launch_ffn_decode(DecodeParams p, const DecodePlan &pl, cudaStream_t st) {

@@ -54,7 +54,7 @@ constexpr size_t WS_DSL_BYTES = static_cast<size_t>(DEC_WE) * DEC_CH * (12 * 256
 // Shared-memory plan of the fused decode kernel (decode.cu).
 struct DecodePlan {
     int grid, S, SB, st_sd;                           // ring: S stages of SB bytes
-    size_t off_route, off_rtok, off_gate, off_red1, off_x, off_hb, off_frag, off_ring, smem;
+    size_t off_route, off_rtok, off_gate, off_red1, off_x, off_frag, off_ring, smem;
     int lag;                                          // down-projection lag (experts)
     int fslot;                                        // bytes of a down stage's fragment slot
 };
@@ -79,7 +79,7 @@ struct DecodeParams {
     unsigned gate_extra;    // added to the logits-arrival target (nonzero only to test the bound)
     // plan (copied from DecodePlan)
     int grid, S, SB, st_sd, lag, fslot;
-    size_t off_route, off_rtok, off_gate, off_red1, off_x, off_hb, off_frag, off_ring;
+    size_t off_route, off_rtok, off_gate, off_red1, off_x, off_frag, off_ring;
 };
 
 bool decode_plan(const coli_moe_config &c, int T, DecodePlan *plan);
