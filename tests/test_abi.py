@@ -110,10 +110,11 @@ def test_residual_host_validation():
 
 
 def test_dispatch_rule_on_the_host():
-    """Batches above 4 tokens take the tensor-core path (7 launches) for int4 records whose
-    hidden and inter sizes are multiples of 128; int8 / int2 records take the GEMV path (5);
-    an empty batch launches nothing.  (Up to 4 tokens the fused decode kernel needs the device's
-    shared-memory size, so that choice is checked by the GPU tests.)"""
+    """Batches above 4 tokens take the tensor-core path (7 launches) for per-row int4, int8 and
+    int2 records whose hidden and inter sizes are multiples of 128; group-scaled records and
+    other sizes take the GEMV path (5); an empty batch launches nothing.  (Up to 4 tokens the
+    fused decode kernel needs the device's shared-memory size, so that choice is checked by the
+    GPU tests.)"""
     for name in ("tiny", "olmoe", "glm_decode", "glm_prefill"):
         cfg = q.config_for(synth.WORKLOADS[name])
         assert q.coli_moe_layer_kernels(cfg, 0) == 0
@@ -127,6 +128,25 @@ def test_dispatch_rule_on_the_host():
     assert q.coli_moe_layer_kernels(gs, 64) == 5
     odd = q.config_for(synth.WORKLOADS["tiny"].replace(inter=64, shared_inter=64))
     assert q.coli_moe_layer_kernels(odd, 32) == 5  # inter not a multiple of 128
+
+
+def test_per_expert_dispatch_threshold():
+    """The threshold is process-wide, defaults to 0 (every expert on the grouped GEMM), and a
+    positive value adds the two GEMV launches to the tensor-core path's count; negative values
+    are rejected."""
+    assert q.coli_moe_dispatch_threshold() == 0
+    cfg = q.config_for(synth.WORKLOADS["glm_prefill"])
+    try:
+        q.coli_moe_set_dispatch_threshold(4)
+        assert q.coli_moe_dispatch_threshold() == 4
+        assert q.coli_moe_layer_kernels(cfg, 2048) == 9
+        assert q.coli_moe_layer_kernels(cfg, 0) == 0
+        with pytest.raises(q.ColiError):
+            q.coli_moe_set_dispatch_threshold(-1)
+        assert q.coli_moe_dispatch_threshold() == 4
+    finally:
+        q.coli_moe_set_dispatch_threshold(0)
+    assert q.coli_moe_layer_kernels(cfg, 2048) == 7
 
 
 def test_group_scaled_container_is_int4_only():
