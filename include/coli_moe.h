@@ -161,7 +161,11 @@ coli_status coli_moe_ffn(const coli_moe_config *cfg, const coli_moe_weights *w, 
                          void *stream);
 
 /* The whole layer: gate, route, group, ffn (all of the above, in that order, on `stream`).
- * topk_ids_out / topk_w_out may be NULL; when given they receive the routing. */
+ * topk_ids_out / topk_w_out may be NULL; when given they receive the routing.
+ * The call issues no host-blocking operation and reads no device data on the host, so it may be
+ * captured into a CUDA graph and replayed: the fused decode kernel keeps its counters in the
+ * workspace header, and consecutive calls (or replays) on one workspace must be ordered on the
+ * GPU, as calls on one stream are.  Replays read the pointers captured with the call. */
 coli_status coli_moe_layer(const coli_moe_config *cfg, const coli_moe_weights *w,
                            const void *x, int T, float *out, int32_t *topk_ids_out,
                            float *topk_w_out, void *ws, size_t ws_bytes, void *stream);
