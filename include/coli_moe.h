@@ -218,11 +218,19 @@ coli_status coli_moe_debug_set_wait(long long wait_cycles, int unreachable);
  *   - All calls on a device share the one array and it keeps the last call's contents; each call
  *     clears the part that must start at zero.  Calls that overlap on the GPU (different streams
  *     without ordering between them) race on the array and give wrong results: order them.
- *   - The device error word lives inside the array and is not readable by the caller; device
- *     anomalies still never trap. */
+ *   - The device error word lives inside the array: coli_moe_noalloc_error_word reads it.
+ *     Device anomalies never trap. */
 coli_status coli_moe_layer_noalloc(const coli_moe_config *cfg, const coli_moe_weights *w,
                                    const void *x, int T, float *out, int32_t *topk_ids_out,
                                    float *topk_w_out, void *stream);
+
+/* Synchronises `stream` and returns in *code the device error word of the current device's
+ * static scratch array (the one coli_moe_layer_noalloc uses): 0 = clean, else COLI_DEVERR_*
+ * bits of the last coli_moe_layer_noalloc call on this device (each call clears it first).
+ * code NULL: COLI_ERR_INVALID_ARG; COLI_ERR_CUDA if the array cannot be reached.  Like the first
+ * coli_moe_layer_noalloc call, the first call on a device looks the array up (before any
+ * stream capture). */
+coli_status coli_moe_noalloc_error_word(void *stream, int *code);
 
 #ifdef __cplusplus
 }

@@ -17,7 +17,7 @@ __all__ = [
     "coli_moe_status_str", "coli_moe_last_cuda_error", "coli_moe_record_bytes", "coli_moe_check_config",
     "coli_moe_workspace_size", "coli_moe_clear_error", "coli_moe_error_word",
     "coli_moe_gate", "coli_moe_route", "coli_moe_group", "coli_moe_ffn", "coli_moe_layer",
-    "coli_moe_layer_noalloc", "STATIC_SCRATCH_BYTES", "coli_moe_layer_kernels", "coli_moe_residual",
+    "coli_moe_layer_noalloc", "coli_moe_noalloc_error_word", "STATIC_SCRATCH_BYTES", "coli_moe_layer_kernels", "coli_moe_residual",
     "coli_moe_debug_set_wait",
     "coli_moe_set_dispatch_threshold",
     "coli_moe_dispatch_threshold",
@@ -81,6 +81,7 @@ def _load():
     L.coli_moe_ffn.argtypes = [cfgp, wp, P, I, P, P, P, P, P, P, P, S, P]
     L.coli_moe_layer.argtypes = [cfgp, wp, P, I, P, P, P, P, S, P]
     L.coli_moe_layer_noalloc.argtypes = [cfgp, wp, P, I, P, P, P, P]
+    L.coli_moe_noalloc_error_word.argtypes = [P, C.POINTER(I)]
     L.coli_moe_layer_kernels.argtypes = [cfgp, I, C.POINTER(I)]
     L.coli_moe_residual.argtypes = [cfgp, P, P, I, P, P]
     L.coli_moe_debug_set_wait.argtypes = [C.c_longlong, I]
@@ -92,7 +93,8 @@ def _load():
     for name in ("coli_moe_record_bytes", "coli_moe_check_config", "coli_moe_workspace_size",
                  "coli_moe_clear_error", "coli_moe_error_word", "coli_moe_gate",
                  "coli_moe_route", "coli_moe_group", "coli_moe_ffn", "coli_moe_layer",
-                 "coli_moe_residual", "coli_moe_debug_set_wait", "coli_moe_set_dispatch_threshold"):
+                 "coli_moe_residual", "coli_moe_debug_set_wait", "coli_moe_set_dispatch_threshold",
+                 "coli_moe_noalloc_error_word"):
         getattr(L, name).restype = I
     return L
 
@@ -215,6 +217,14 @@ def coli_moe_layer_noalloc(cfg, weights: MoEWeights, x, T, out, topk_ids_out=Non
     _check("coli_moe_layer_noalloc", lib.coli_moe_layer_noalloc(
         C.byref(cfg), C.byref(weights), _p(x), T, _p(out), _p(topk_ids_out), _p(topk_w_out),
         _stream(stream)))
+
+
+def coli_moe_noalloc_error_word(stream=None) -> int:
+    """Device error word of the static scratch array behind coli_moe_layer_noalloc (synchronises
+    the stream): 0 when the last no-allocation call on this device ran clean."""
+    v = C.c_int()
+    _check("coli_moe_noalloc_error_word", lib.coli_moe_noalloc_error_word(_stream(stream), C.byref(v)))
+    return v.value
 
 
 def coli_moe_debug_set_wait(wait_cycles: int, unreachable: bool) -> None:

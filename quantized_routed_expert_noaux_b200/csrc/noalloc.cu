@@ -67,3 +67,11 @@ extern "C" coli_status coli_moe_layer_noalloc(const coli_moe_config *cfg, const 
     return coli_moe_layer(cfg, w, x, T, out, topk_ids_out, topk_w_out, ws,
                           static_cast<size_t>(COLI_MOE_STATIC_SCRATCH_BYTES), stream);
 }
+
+extern "C" coli_status coli_moe_noalloc_error_word(void *stream, int *code) {
+    if (!code) return COLI_ERR_INVALID_ARG;
+    void *ws = nullptr;
+    const coli_status s = static_scratch(&ws);
+    if (s != COLI_OK) return s;
+    return coli_moe_error_word(ws, stream, code);
+}

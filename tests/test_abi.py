@@ -149,6 +149,12 @@ def test_per_expert_dispatch_threshold():
     assert q.coli_moe_layer_kernels(cfg, 2048) == 7
 
 
+def test_noalloc_error_word_rejects_null_code():
+    """The static array's error-word accessor checks its output pointer before touching the
+    device (status 1, COLI_ERR_INVALID_ARG)."""
+    assert q.lib.coli_moe_noalloc_error_word(None, None) == 1
+
+
 def test_group_scaled_container_is_int4_only():
     wl = synth.WORKLOADS["glm_int8"].replace(group=64)
     with pytest.raises(q.ColiError) as ei:

@@ -45,6 +45,7 @@ def _both(cfg, weights, wl, T, step):
         w = torch.full((T, wl.top_k), float("nan"), dtype=torch.float32, device=dev)
         if noalloc:
             q.coli_moe_layer_noalloc(cfg, weights, x, T, out, ids, w)
+            assert q.coli_moe_noalloc_error_word() == 0  # the static array's error word reads clean
         else:
             q.coli_moe_clear_error(ws)
             q.coli_moe_layer(cfg, weights, x, T, out, ids, w, ws)
